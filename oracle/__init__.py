@@ -1,0 +1,25 @@
+"""CPU oracle of one FreeToken-style MoE layer forward pass with an expert cache.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  It shares
+no code with the CUDA library (``expert_offloaded_serving_b200``) and imports
+nothing from it; the two meet only through the seeded inputs of ``synth``.
+
+Plain, slow and fp64 throughout, written from the public write-ups of FreeToken
+(cited per function) plus the readings stated where those pages are silent:
+
+* ``fp4``      e2m1 / UE8M0 decoding, the scale-atom storage index, the OCP MX
+               quantiser and fp64 -> bf16 rounding.
+* ``routing``  fixed-order router logits, softmax top-k, stable permutation.
+* ``layer``    SwiGLU expert FFN and the weighted combine (decode bf16 mode and
+               MXFP4-activation mode).
+* ``lru``      the global LRU expert cache across layers, with resize.
+
+Pins (tests/test_oracle_*.py, all CPU): exhaustive code x scale tables against
+the closed form, hand-computed scale-atom offsets, quantiser ties and
+idempotence, brute-force top-k with injected ties, stable-sort permutation
+invariants, a hand-computed two-expert layer (tests/golden/), the partition
+invariant of the combine, and an LRU checked against a timestamp simulation.
+No function here is "parity unpinned".
+"""
+from . import fp4, routing, layer, lru  # noqa: F401

@@ -1,0 +1,79 @@
+"""SwiGLU expert FFN and the weighted combine of one MoE layer, in fp64.
+
+Test infrastructure only (see the package header).
+
+Pages: experts are computed on the GPU from weights fetched over PCIe or held
+in VRAM (jansverre.net page, section "Hvorfor er båndbredden viktigere enn
+antall kjerner?"), and the outputs of however the selected experts are split
+are summed at the end with no simplified expert, no changed router and no
+approximation (same section).  The expert type (SwiGLU: h = silu(Wg x) * (Wu x),
+y = Wd h) and the output rounding (one bf16 rounding of the fp64 sum) are the
+readings used here.
+
+Modes:
+* ``mxfp4=False`` (decode): x is the bf16 input as is; h stays unrounded.
+* ``mxfp4=True`` (prefill): x and h are quantised per 32 values along their
+  contraction axis by the OCP MX rule before each product.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import fp4, routing
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    return z / (1.0 + np.exp(-z))
+
+
+def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray, mxfp4: bool = False) -> np.ndarray:
+    """y [m, H] = Wd (silu(Wg x) * (Wu x)) for the rows of x [m, H] (fp64)."""
+    wg = fp4.dequant_matrix(blob, "wg", hidden, inter)
+    wu = fp4.dequant_matrix(blob, "wu", hidden, inter)
+    wd = fp4.dequant_matrix(blob, "wd", hidden, inter)
+    x = np.asarray(x, dtype=np.float64)
+    if mxfp4:
+        x = fp4.dequant_rows(*fp4.quantize_rows(x))
+    g = x @ wg.T
+    u = x @ wu.T
+    h = silu(g) * u
+    if mxfp4:
+        h = fp4.dequant_rows(*fp4.quantize_rows(h))
+    return h @ wd.T
+
+
+def moe_layer(x_bits: np.ndarray, blob_of, hidden: int, inter: int, n_experts: int, top_k: int,
+              logits: np.ndarray | None = None, router_w: np.ndarray | None = None,
+              renorm: bool = True, mxfp4: bool = False, shared_blob=None) -> dict:
+    """One MoE layer on T tokens.
+
+    x_bits   bf16 bits [T, H]
+    blob_of  callable expert id -> blob (uint8)
+    logits   fp32 [T, E] (used as given) or None to compute x . Wr^T
+    shared_blob  blob of an always-on shared expert (weight 1) or None
+
+    Returns dict with logits, ids, w (fp64), offs/perm/inv, out_f64 and
+    out_bits (bf16 of out_f64).
+    """
+    x = fp4.bf16_to_f64(x_bits)
+    T = x.shape[0]
+    if logits is None:
+        logits = routing.router_logits(x, router_w)
+    ids, bad = routing.topk(logits, top_k)
+    w = routing.softmax_weights(logits, ids, renorm)
+    offs, perm, inv = routing.permutation(ids, n_experts)
+    out = np.zeros((T, hidden), dtype=np.float64)
+    y = {}
+    for e in np.unique(ids):
+        rows = np.nonzero((ids == e).any(axis=1))[0]
+        y[int(e)] = (rows, expert_ffn(blob_of(int(e)), hidden, inter, x[rows], mxfp4))
+    for t in range(T):
+        acc = 0.0
+        for j in range(top_k):
+            rows, ye = y[int(ids[t, j])]
+            acc = acc + w[t, j] * ye[int(np.nonzero(rows == t)[0][0])]
+        if shared_blob is not None:
+            acc = acc + expert_ffn(shared_blob, hidden, inter, x[t:t + 1], mxfp4)[0]
+        out[t] = acc
+    return dict(logits=np.asarray(logits, dtype=np.float32), ids=ids, nonfinite=bad, w=w,
+                offs=offs, perm=perm, inv=inv, out_f64=out, out_bits=fp4.round_bf16(out))
