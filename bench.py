@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE-layer hot path on B200.
+
+Default workload: the 35B-A3B-class decode stack (hidden 2048, 256 routed
+experts top-8 plus 1 shared expert, intermediate 512, 40 layers, MXFP4 weights
+resident in HBM, batch 1), routed by seeded Zipf(1.1) traces with 0.6
+adjacent-token reuse.  One step = one token through all 40 MoE layers
+(route, permute, gate/up + SwiGLU GEMV, down GEMV + combine), replayed as one
+CUDA graph.  Each step reads ~600 MB of distinct expert weights, far more than
+the 126 MB L2, so no L2 flush is needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  Multi-GPU runs are independent replicas (the path does
+not shard): one process per GPU, timing = max over ranks, value = all tokens /
+that time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE decode tok/s + HBM GB/s vs roofline; prefill FP4 TFLOP/s; miss H2D GB/s"
+SEED = 1002
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 or 4)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks
+# ---------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, src="fallback")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every 10 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            pr = torch.cuda.get_device_properties(index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# ---------------------------------------------------------------------------
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# 35B-class decode stack
+# ---------------------------------------------------------------------------
+H, I, E, K_TOP, S_SHARED, L = 2048, 512, 256, 8, 1, 40
+TRACE_LEN = 512
+
+
+def decode_routing(T):
+    """Per token position p < TRACE_LEN: sets [L][T][k] of T independent sequences."""
+    import numpy as np
+    import synth
+    sets = np.empty((TRACE_LEN, L, T, K_TOP), np.int32)
+    for layer in range(L):
+        for t in range(T):
+            sets[:, layer, t] = synth.zipf_trace(SEED, layer, TRACE_LEN, E, K_TOP, 1.1, 0.6, stream=t)
+    return sets
+
+
+def decode_logits(sets):
+    import numpy as np
+    import synth
+    P, Lx, T, _ = sets.shape
+    out = np.empty((P, Lx, T, E), np.float32)
+    for p in range(P):
+        for layer in range(Lx):
+            out[p, layer] = synth.logits_for_sets(SEED, p * 1000 + layer, sets[p, layer], E)
+    return out
+
+
+def run_ours(args, world, rank):
+    import numpy as np
+    import torch
+
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+
+    T = args.tokens
+    lay = ft.ft_blob_layout(H, I)
+    used = lay["used"]
+    gu_bytes = lay["wd"] + (lay["wd_sf"] - lay["wg_sf"])          # Wg + Wu codes and scales
+    d_bytes = (lay["wd"] - lay["wu"]) + (lay["used"] - lay["wd_sf"])  # Wd codes and scales
+    pools = [synth.gpu.layer_pool(H, I, E + S_SHARED, SEED, layer) for layer in range(L)]
+    torch.cuda.synchronize()
+    ctx = ft.ft_create(ft.make_desc(H, I, E, K_TOP, L, S_SHARED, 0, T), None, pools)
+    sets = decode_routing(T)
+    logits_all = torch.from_numpy(decode_logits(sets)).cuda()        # [P][L][T][E]
+    logits_buf = torch.empty_like(logits_all[0])
+    xb = synth.activations_bf16(SEED, 7, T, H)
+    x0 = torch.from_numpy(xb.view(np.int16).copy()).cuda().view(torch.bfloat16)
+    bufs = [torch.empty_like(x0), torch.empty_like(x0)]
+    # algorithmic bytes per step position: distinct routed experts + shared, whole blobs
+    uniq = np.array([[len(np.unique(sets[p, layer])) for layer in range(L)] for p in range(TRACE_LEN)])
+    bytes_pos = (uniq + S_SHARED).sum(axis=1) * used                 # [P]
+    stream = torch.cuda.Stream()
+
+    def one_pass(src):
+        cur = src
+        for layer in range(L):
+            out = bufs[layer % 2]
+            ft.ft_moe_layer_forward(ctx, layer, cur, T, None, logits_buf[layer], out, ft.FT_ROUTE_RENORM,
+                                    stream.cuda_stream)
+            cur = out
+        return cur
+
+    with torch.cuda.stream(stream):
+        logits_buf.copy_(logits_all[0])
+        one_pass(x0)
+        stream.synchronize()
+        ft.ft_sync_status(ctx, stream.cuda_stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            final = one_pass(x0)
+    launches_per_step = L * 4
+
+    def step(p):
+        logits_buf.copy_(logits_all[p % TRACE_LEN], non_blocking=True)
+        g.replay()
+
+    with torch.cuda.stream(stream):
+        for w in range(args.warmup):
+            step(w)
+        stream.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            e0.record(stream)
+            for s in range(args.steps):
+                step(args.warmup + s)
+            e1.record(stream)
+            e1.synchronize()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = e0.elapsed_time(e1)
+    ft.ft_sync_status(ctx, stream.cuda_stream)
+    ms_max = max_over_ranks(ms, world)
+    positions = [(args.warmup + s) % TRACE_LEN for s in range(args.steps)]
+    step_bytes = float(np.mean(bytes_pos[positions]))
+    res = dict(ms=ms_max, tok_s=world * T * args.steps / (ms_max / 1e3), hbm_gbs=step_bytes * args.steps / (ms / 1e3) / 1e9,
+               step_bytes=step_bytes, launches=launches_per_step * args.steps, clocks=clk.summary())
+
+    # per-kernel device time over the same positions, eager launches bracketed by events
+    ft.ft_kernel_timing_enable(ctx, True)
+    nk = min(args.steps, 200)
+    with torch.cuda.stream(stream):
+        for s in range(nk):
+            logits_buf.copy_(logits_all[positions[s]], non_blocking=True)
+            one_pass(x0)
+    kt = ft.ft_kernel_timing_read(ctx)
+    ft.ft_kernel_timing_enable(ctx, False)
+    pos = positions[:nk]
+    gu_launch_bytes = float(np.mean([(uniq[p] + S_SHARED).mean() for p in pos])) * gu_bytes
+    dn_launch_bytes = float(np.mean([(uniq[p] + S_SHARED).mean() for p in pos])) * d_bytes
+    res["kernels"] = {k: {"ms_total": v[0], "launches": v[1], "us_avg": 1e3 * v[0] / v[1]} for k, v in kt.items() if v[1]}
+    res["gate_up_bytes"] = gu_launch_bytes
+    res["down_bytes"] = dn_launch_bytes
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs
+    # (x and the 40 layers' logits) from pinned memory, the pass, D2H of the output
+    host_x = x0.cpu().pin_memory()
+    host_lg = logits_all.cpu().pin_memory()
+    host_out = torch.empty_like(host_x).pin_memory()
+    xin = torch.empty_like(x0)
+    with torch.cuda.stream(stream):
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            final2 = one_pass(xin)
+        stream.synchronize()
+        barrier(world)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for s in range(args.steps):
+            p = positions[s]
+            xin.copy_(host_x, non_blocking=True)
+            logits_buf.copy_(host_lg[p], non_blocking=True)
+            g2.replay()
+            host_out.copy_(final2, non_blocking=True)
+        a1.record(stream)
+        a1.synchronize()
+        barrier(world)
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
+    res["e2e"] = {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tok/s",
+                  "h2d_bytes_per_step": int(host_x.numel() * 2 + host_lg[0].numel() * 4),
+                  "d2h_bytes_per_step": int(host_out.numel() * 2)}
+    del g, g2, final, final2
+    ft.ft_destroy(ctx)
+    return res
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_tok_s(T, n_layers, budget_s=12.0):
+    """Time the oracle on one token position through `n_layers` sampled layers
+    (stopping early past `budget_s`); returns (tok/s over all 40 layers, layers
+    timed, threads)."""
+    import numpy as np
+    import synth
+    from oracle import layer as olayer
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    sets = np.stack([synth.zipf_trace(SEED, 0, 4, E, K_TOP, 1.1, 0.6, stream=t)[-1] for t in range(T)])
+    xb = synth.activations_bf16(SEED, 7, T, H)
+    t0 = time.perf_counter()
+    done = 0
+    for layer in range(n_layers):
+        lg = synth.logits_for_sets(SEED, layer, sets, E)
+        cache = {}
+
+        def blob_of(e, layer=layer, cache=cache):
+            if e not in cache:
+                cache[e] = synth.expert_blob(SEED, layer, e, H, I)
+            return cache[e]
+        olayer.moe_layer(xb, blob_of, H, I, E, K_TOP, logits=lg, shared_blob=blob_of(E))
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    per_layer = dt / done
+    return T / (per_layer * L), done, threads
+
+
+def workload_config(T):
+    return {"workload": f"35B-A3B-class MoE decode stack: hidden {H}, {E} routed experts top-{K_TOP} + {S_SHARED} shared, "
+                        f"intermediate {I}, {L} layers, MXFP4 (e2m1 + UE8M0/32) weights resident in HBM, "
+                        f"batch {T}, Zipf(1.1) routing traces with 0.6 adjacent-token reuse",
+            "global_batch": T, "layers": L, "l2": "inputs larger than L2 (~600 MB of distinct expert weights per step)"}
+
+
+def main():
+    args = parse()
+    import torch
+    world, rank, local = dist_setup(args)
+    T = args.tokens
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per = []
+        for _ in range(args.warmup + args.steps):
+            v, done, threads = oracle_tok_s(T, 2, budget_s=30.0)
+            per.append(v)
+        v = statistics.median(per[args.warmup:]) if args.steps else per[-1]
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * T / v,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": workload_config(T),
+                "cpu_baseline": {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                                 "sample": f"each step: 1 token through {done} of {L} layers, extrapolated to {L}"},
+                "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+    res = run_ours(args, world, rank)
+    if rank != 0:
+        return
+    pk = peaks()
+    gu = res["kernels"].get("gate_up")
+    dn = res["kernels"].get("down_combine")
+    gu_gbs = res["gate_up_bytes"] / (gu["us_avg"] * 1e-6) / 1e9
+    line = {"metric": METRIC, "value": res["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(T),
+            "roofline": {"bound": "hbm", "kernel": "gate_up", "achieved": gu_gbs, "peak": pk["hbm"],
+                         "peak_source": pk["src"], "unit": "GB/s", "frac": gu_gbs / pk["hbm"], "traffic": None},
+            "hbm_gbs_step": res["hbm_gbs"], "hbm_frac_step": res["hbm_gbs"] / pk["hbm"],
+            "gpu_launches": res["launches"], "clocks": res["clocks"], "e2e": res["e2e"],
+            "kernels": res["kernels"]}
+    if dn:
+        line["down_combine_gbs"] = res["down_bytes"] / (dn["us_avg"] * 1e-6) / 1e9
+    if world == 1:
+        v, done, threads = oracle_tok_s(T, L, budget_s=12.0)
+        line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                                "sample": f"1 token through {done} of {L} layers, extrapolated to {L}"}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,974 @@
+// Host runtime and C ABI of libftmoe.so: context, scratch, global LRU expert
+// cache over a CUDA virtual-memory slot arena, pinned host pool, miss fetch,
+// prefill double-buffered prefetch, elastic resize, layer orchestration.
+//
+// Pages: experts that are not in VRAM are fetched over PCIe (jansverre.net,
+// "Hva er FreeToken?"); decoding uses one global LRU cache across the MoE
+// layers instead of pinning experts at start-up, and prefill streams the next
+// layer pack while the GPU works on the current one (jansverre.net, "Hvorfor
+// er båndbredden viktigere enn antall kjerner?"); the shared LRU exploits the
+// expert-path overlap of adjacent tokens (aipolix.com, paragraph on
+// semantic-aware caching); the GPU expert cache is resized without restarting
+// the engine or reloading the host-resident pool (aipolix.com, paragraph on
+// elastic memory management).
+#include <cuda.h>  // driver types only; entry points come from cudaGetDriverEntryPoint
+
+#include <algorithm>
+#include <chrono>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <list>
+#include <string>
+#include <thread>
+#include <unordered_map>
+#include <vector>
+
+#include "ft_common.cuh"
+#include "ft_kernels.h"
+#include "ft_runtime.h"
+
+using namespace ft;
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+static thread_local std::string g_err;
+
+static ft_status fail(ft_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+#define CUDA_TRY(expr)                                                                         \
+  do {                                                                                         \
+    cudaError_t e_ = (expr);                                                                   \
+    if (e_ != cudaSuccess) return fail(FT_ERR_CUDA, "%s: %s (%s:%d)", #expr, cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+#define CU_TRY(expr)                                                                           \
+  do {                                                                                         \
+    CUresult r_ = (expr);                                                                      \
+    if (r_ != CUDA_SUCCESS) return fail(FT_ERR_CUDA, "%s: CUresult %d (%s:%d)", #expr, (int)r_, __FILE__, __LINE__); \
+  } while (0)
+
+extern "C" const char* ft_last_error(void) { return g_err.c_str(); }
+
+// ---------------------------------------------------------------------------
+// driver API entry points (no link-time dependency on libcuda)
+// ---------------------------------------------------------------------------
+namespace {
+struct Drv {
+  CUresult (*memAddressReserve)(CUdeviceptr*, size_t, size_t, CUdeviceptr, unsigned long long) = nullptr;
+  CUresult (*memAddressFree)(CUdeviceptr, size_t) = nullptr;
+  CUresult (*memCreate)(CUmemGenericAllocationHandle*, size_t, const CUmemAllocationProp*, unsigned long long) = nullptr;
+  CUresult (*memRelease)(CUmemGenericAllocationHandle) = nullptr;
+  CUresult (*memMap)(CUdeviceptr, size_t, size_t, CUmemGenericAllocationHandle, unsigned long long) = nullptr;
+  CUresult (*memUnmap)(CUdeviceptr, size_t) = nullptr;
+  CUresult (*memSetAccess)(CUdeviceptr, size_t, const CUmemAccessDesc*, size_t) = nullptr;
+  CUresult (*memGetAllocationGranularity)(size_t*, const CUmemAllocationProp*, CUmemAllocationGranularity_flags) = nullptr;
+  bool ok = false;
+};
+
+ft_status load_driver(Drv& d) {
+  if (d.ok) return FT_OK;
+  struct Ent {
+    const char* name;
+    void** fn;
+  } ents[] = {{"cuMemAddressReserve", (void**)&d.memAddressReserve},
+              {"cuMemAddressFree", (void**)&d.memAddressFree},
+              {"cuMemCreate", (void**)&d.memCreate},
+              {"cuMemRelease", (void**)&d.memRelease},
+              {"cuMemMap", (void**)&d.memMap},
+              {"cuMemUnmap", (void**)&d.memUnmap},
+              {"cuMemSetAccess", (void**)&d.memSetAccess},
+              {"cuMemGetAllocationGranularity", (void**)&d.memGetAllocationGranularity}};
+  for (auto& e : ents) {
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t err = cudaGetDriverEntryPoint(e.name, e.fn, cudaEnableDefault, &q);
+    if (err != cudaSuccess || q != cudaDriverEntryPointSuccess || *e.fn == nullptr)
+      return fail(FT_ERR_CUDA, "driver entry point %s unavailable", e.name);
+  }
+  d.ok = true;
+  return FT_OK;
+}
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// global LRU over (layer, expert) keys
+// ---------------------------------------------------------------------------
+namespace {
+struct Lru {
+  // most recent at the back
+  std::list<int64_t> order;
+  std::unordered_map<int64_t, std::pair<int32_t, std::list<int64_t>::iterator>> map;  // key -> (slot, pos)
+  std::vector<char> slot_used;
+  int64_t capacity = 0;
+
+  int32_t lowest_free() const {
+    for (int64_t s = 0; s < capacity; s++)
+      if (!slot_used[s]) return (int32_t)s;
+    return -1;
+  }
+  void set_capacity(int64_t c) {
+    capacity = c;
+    if ((int64_t)slot_used.size() < c) slot_used.resize(c, 0);
+  }
+};
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// context
+// ---------------------------------------------------------------------------
+struct ft_ctx {
+  ft_model_desc d{};
+  BlobLayout lay{};
+  int64_t stride = 0;
+  int n_blobs = 0;  // E + n_shared per layer
+  int device = 0;
+  int max_tokens = 0;
+
+  std::vector<const uint8_t*> host_layers;
+  std::vector<void*> registered;  // host ranges we pinned with cudaHostRegister
+  std::vector<const uint8_t*> resident;
+
+  cudaStream_t copy_stream = nullptr;
+  cudaStream_t last_stream = nullptr;
+
+  // device scratch
+  int* d_status = nullptr;
+  float* d_logits = nullptr;
+  int32_t* d_ids = nullptr;
+  float* d_w = nullptr;
+  int32_t* d_offs = nullptr;
+  int32_t* d_perm = nullptr;
+  int32_t* d_inv = nullptr;
+  int32_t* d_active = nullptr;
+  int32_t* d_nact = nullptr;
+  int32_t* d_pad_offs = nullptr;
+  float* d_h = nullptr;
+  int decode_max_t = 0;
+
+  // pinned host scratch
+  int32_t* h_ids = nullptr;
+  int* h_status = nullptr;
+  cudaEvent_t ev_ids = nullptr;
+
+  // pointer tables
+  const uint8_t** d_eptr_res = nullptr;    // [L][n_blobs]
+  const uint8_t** h_eptr_cache = nullptr;  // pinned [L][n_blobs]
+  const uint8_t** d_eptr_cache = nullptr;  // [L][n_blobs]
+
+  // cache arena
+  Drv drv;
+  CUdeviceptr va = 0;
+  size_t va_size = 0;
+  size_t chunk = 0;
+  std::vector<CUmemGenericAllocationHandle> chunks;
+  Lru lru;
+  bool cache_on = false;
+  uint8_t* d_shared = nullptr;  // [L][n_shared] blobs for non-resident layers
+  std::vector<ft_cache_event> trace;
+  ft_cache_stats stats{};
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> copy_timing;  // pending (start, end)
+
+  // prefill staging
+  uint8_t* d_stage[2] = {nullptr, nullptr};
+  const uint8_t** d_eptr_stage[2] = {nullptr, nullptr};
+  int stage_layer[2] = {-1, -1};
+  cudaEvent_t ev_landed[2] = {nullptr, nullptr};
+  cudaEvent_t ev_done[2] = {nullptr, nullptr};
+  int64_t prefetch_bytes = 0;
+
+  // prefill scratch (allocated on first use)
+  PrefillScratch pf{};
+
+  // per-kernel timing
+  bool timing = false;
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> tmarks;  // (class, (start, stop))
+  double tms[FT_K_COUNT] = {0};
+  int64_t tlaunch[FT_K_COUNT] = {0};
+};
+
+// Bracket one launch with events when timing is on (and the stream is not capturing).
+struct KTimer {
+  ft_ctx* c;
+  int cls;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr, b = nullptr;
+  KTimer(ft_ctx* c_, int cls_, cudaStream_t s_) : c(c_), cls(cls_), s(s_) {
+    if (!c->timing) return;
+    cudaStreamCaptureStatus cs;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+    cudaEventCreate(&a);
+    cudaEventCreate(&b);
+    cudaEventRecord(a, s);
+  }
+  ~KTimer() {
+    if (!a) return;
+    cudaEventRecord(b, s);
+    c->tmarks.push_back({cls, {a, b}});
+  }
+};
+
+static ft_status check_desc(const ft_model_desc* d) {
+  if (!d) return fail(FT_ERR_INVALID, "desc is NULL");
+  if (d->hidden <= 0 || d->hidden % 128) return fail(FT_ERR_INVALID, "hidden %d not a positive multiple of 128", d->hidden);
+  if (d->inter <= 0 || d->inter % 128) return fail(FT_ERR_INVALID, "inter %d not a positive multiple of 128", d->inter);
+  if (d->n_experts <= 0 || d->n_experts > 1024) return fail(FT_ERR_INVALID, "n_experts %d not in [1, 1024]", d->n_experts);
+  if (d->top_k <= 0 || d->top_k > 16 || d->top_k > d->n_experts) return fail(FT_ERR_INVALID, "top_k %d invalid", d->top_k);
+  if (d->n_layers <= 0) return fail(FT_ERR_INVALID, "n_layers %d", d->n_layers);
+  if (d->n_shared < 0 || d->n_shared > 1) return fail(FT_ERR_INVALID, "n_shared %d not 0 or 1", d->n_shared);
+  if (d->cache_budget_bytes < 0) return fail(FT_ERR_INVALID, "negative cache budget");
+  if (d->max_tokens <= 0) return fail(FT_ERR_INVALID, "max_tokens %d", d->max_tokens);
+  return FT_OK;
+}
+
+extern "C" int64_t ft_blob_stride(int32_t hidden, int32_t inter) {
+  if (hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return -1;
+  return blob_layout(hidden, inter).stride;
+}
+
+extern "C" ft_status ft_blob_layout(int32_t hidden, int32_t inter, int64_t out[8]) {
+  if (!out || hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return fail(FT_ERR_INVALID, "bad shape");
+  BlobLayout b = blob_layout(hidden, inter);
+  int64_t v[8] = {b.wg, b.wu, b.wd, b.wg_sf, b.wu_sf, b.wd_sf, b.used, b.stride};
+  memcpy(out, v, sizeof v);
+  return FT_OK;
+}
+
+template <class T>
+static ft_status dev_alloc(T** p, size_t n) {
+  *p = nullptr;
+  if (n == 0) return FT_OK;
+  CUDA_TRY(cudaMalloc((void**)p, n * sizeof(T)));
+  return FT_OK;
+}
+
+#define FT_TRY(expr)            \
+  do {                          \
+    ft_status s_ = (expr);      \
+    if (s_ != FT_OK) return s_; \
+  } while (0)
+
+// physical memory under the arena so that `slots` slots are backed
+static ft_status arena_map(ft_ctx* c, int64_t slots) {
+  size_t need = (size_t)slots * (size_t)c->stride;
+  size_t nchunks = (need + c->chunk - 1) / c->chunk;
+  if (nchunks * c->chunk > c->va_size) return fail(FT_ERR_NO_SPACE, "cache budget exceeds the reserved arena");
+  while (c->chunks.size() > nchunks) {
+    size_t i = c->chunks.size() - 1;
+    CU_TRY(c->drv.memUnmap(c->va + i * c->chunk, c->chunk));
+    CU_TRY(c->drv.memRelease(c->chunks[i]));
+    c->chunks.pop_back();
+  }
+  while (c->chunks.size() < nchunks) {
+    size_t i = c->chunks.size();
+    CUmemAllocationProp prop{};
+    prop.type = CU_MEM_ALLOCATION_TYPE_PINNED;
+    prop.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
+    prop.location.id = c->device;
+    CUmemGenericAllocationHandle h;
+    CUresult r = c->drv.memCreate(&h, c->chunk, &prop, 0);
+    if (r != CUDA_SUCCESS) return fail(FT_ERR_CUDA, "cuMemCreate of %zu bytes failed (%d)", c->chunk, (int)r);
+    r = c->drv.memMap(c->va + i * c->chunk, c->chunk, 0, h, 0);
+    if (r != CUDA_SUCCESS) {
+      c->drv.memRelease(h);
+      return fail(FT_ERR_CUDA, "cuMemMap failed (%d)", (int)r);
+    }
+    CUmemAccessDesc acc{};
+    acc.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
+    acc.location.id = c->device;
+    acc.flags = CU_MEM_ACCESS_FLAGS_PROT_READWRITE;
+    CU_TRY(c->drv.memSetAccess(c->va + i * c->chunk, c->chunk, &acc, 1));
+    c->chunks.push_back(h);
+  }
+  c->stats.mapped_bytes = (int64_t)(c->chunks.size() * c->chunk);
+  return FT_OK;
+}
+
+static uint8_t* slot_ptr(ft_ctx* c, int32_t slot) { return (uint8_t*)(c->va + (size_t)slot * (size_t)c->stride); }
+
+extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* host_layers,
+                               const void* const* resident_layers, ft_ctx** out) {
+  FT_TRY(check_desc(desc));
+  if (!out) return fail(FT_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  ft_ctx* c = new ft_ctx();
+  c->d = *desc;
+  const int H = desc->hidden, I = desc->inter, E = desc->n_experts, k = desc->top_k, L = desc->n_layers;
+  c->lay = blob_layout(H, I);
+  c->stride = c->lay.stride;
+  c->n_blobs = E + desc->n_shared;
+  c->max_tokens = desc->max_tokens;
+  c->decode_max_t = std::min(desc->max_tokens, kDecodeMaxTokens);
+  auto bail = [&](ft_status st) {
+    std::string keep = g_err;
+    ft_destroy(c);
+    g_err = keep;
+    return st;
+  };
+  if (cudaGetDevice(&c->device) != cudaSuccess) return bail(fail(FT_ERR_CUDA, "no CUDA device"));
+  if (cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return bail(fail(FT_ERR_CUDA, "copy stream"));
+
+  c->host_layers.assign(L, nullptr);
+  c->resident.assign(L, nullptr);
+  for (int l = 0; l < L; l++) {
+    if (host_layers) c->host_layers[l] = (const uint8_t*)host_layers[l];
+    if (resident_layers) c->resident[l] = (const uint8_t*)resident_layers[l];
+  }
+  // pin pageable host pools
+  for (int l = 0; l < L; l++) {
+    const uint8_t* hp = c->host_layers[l];
+    if (!hp) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, hp) == cudaSuccess && at.type == cudaMemoryTypeHost) continue;
+    cudaGetLastError();
+    if (cudaHostRegister((void*)hp, (size_t)c->n_blobs * c->stride, cudaHostRegisterDefault) != cudaSuccess)
+      return bail(fail(FT_ERR_CUDA, "cudaHostRegister of layer %d pool failed", l));
+    c->registered.push_back((void*)hp);
+  }
+
+  const int T = desc->max_tokens;
+  ft_status st;
+  if ((st = dev_alloc(&c->d_status, 1)) || (st = dev_alloc(&c->d_logits, (size_t)T * E)) ||
+      (st = dev_alloc(&c->d_ids, (size_t)T * k)) || (st = dev_alloc(&c->d_w, (size_t)T * k)) ||
+      (st = dev_alloc(&c->d_offs, E + 1)) || (st = dev_alloc(&c->d_perm, (size_t)T * k)) ||
+      (st = dev_alloc(&c->d_inv, (size_t)T * k)) || (st = dev_alloc(&c->d_active, E)) ||
+      (st = dev_alloc(&c->d_nact, 1)) || (st = dev_alloc(&c->d_pad_offs, E + 1)) ||
+      (st = dev_alloc(&c->d_h, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * I)))
+    return bail(st);
+  if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return bail(fail(FT_ERR_CUDA, "memset"));
+  if (cudaMallocHost(&c->h_ids, (size_t)T * k * sizeof(int32_t)) != cudaSuccess ||
+      cudaMallocHost(&c->h_status, sizeof(int)) != cudaSuccess)
+    return bail(fail(FT_ERR_CUDA, "pinned scratch"));
+  if (cudaEventCreateWithFlags(&c->ev_ids, cudaEventDisableTiming) != cudaSuccess)
+    return bail(fail(FT_ERR_CUDA, "event"));
+  for (int b = 0; b < 2; b++) {
+    if (cudaEventCreateWithFlags(&c->ev_landed[b], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_done[b], cudaEventDisableTiming) != cudaSuccess)
+      return bail(fail(FT_ERR_CUDA, "event"));
+  }
+
+  // resident pointer table
+  bool any_resident = false, any_host_only = false;
+  std::vector<const uint8_t*> tab((size_t)L * c->n_blobs, nullptr);
+  for (int l = 0; l < L; l++) {
+    if (c->resident[l]) {
+      any_resident = true;
+      for (int e = 0; e < c->n_blobs; e++) tab[(size_t)l * c->n_blobs + e] = c->resident[l] + (size_t)e * c->stride;
+    } else if (c->host_layers[l]) {
+      any_host_only = true;
+    }
+  }
+  if (any_resident) {
+    if ((st = dev_alloc(&c->d_eptr_res, tab.size()))) return bail(st);
+    if (cudaMemcpy(c->d_eptr_res, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(fail(FT_ERR_CUDA, "resident table"));
+  }
+
+  // expert cache over a reserved virtual range
+  if (desc->cache_budget_bytes > 0 && any_host_only) {
+    if ((st = load_driver(c->drv))) return bail(st);
+    CUmemAllocationProp prop{};
+    prop.type = CU_MEM_ALLOCATION_TYPE_PINNED;
+    prop.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
+    prop.location.id = c->device;
+    size_t gran = 0;
+    if (c->drv.memGetAllocationGranularity(&gran, &prop, CU_MEM_ALLOC_GRANULARITY_RECOMMENDED) != CUDA_SUCCESS)
+      return bail(fail(FT_ERR_CUDA, "granularity"));
+    c->chunk = pad_up(kArenaChunkBytes, gran);
+    size_t total = 0, freeb = 0;
+    cudaMemGetInfo(&freeb, &total);
+    size_t pool = (size_t)L * c->n_blobs * c->stride;
+    c->va_size = pad_up(std::min(pool, total) + c->chunk, c->chunk);
+    if (c->drv.memAddressReserve(&c->va, c->va_size, c->chunk, 0, 0) != CUDA_SUCCESS)
+      return bail(fail(FT_ERR_CUDA, "cuMemAddressReserve of %zu bytes failed", c->va_size));
+    c->cache_on = true;
+    int64_t cap = desc->cache_budget_bytes / c->stride;
+    c->lru.set_capacity(cap);
+    if ((st = arena_map(c, cap))) return bail(st);
+    c->stats.capacity_slots = cap;
+    if (cudaMallocHost(&c->h_eptr_cache, (size_t)L * c->n_blobs * sizeof(void*)) != cudaSuccess)
+      return bail(fail(FT_ERR_CUDA, "pinned table"));
+    memset(c->h_eptr_cache, 0, (size_t)L * c->n_blobs * sizeof(void*));
+    if ((st = dev_alloc(&c->d_eptr_cache, (size_t)L * c->n_blobs))) return bail(st);
+    // shared experts stay resident outside the LRU
+    if (desc->n_shared > 0) {
+      if ((st = dev_alloc(&c->d_shared, (size_t)L * desc->n_shared * c->stride))) return bail(st);
+      for (int l = 0; l < L; l++) {
+        if (!c->host_layers[l]) continue;
+        for (int s = 0; s < desc->n_shared; s++) {
+          uint8_t* dst = c->d_shared + ((size_t)l * desc->n_shared + s) * c->stride;
+          if (cudaMemcpy(dst, c->host_layers[l] + (size_t)(E + s) * c->stride, c->stride, cudaMemcpyHostToDevice) !=
+              cudaSuccess)
+            return bail(fail(FT_ERR_CUDA, "shared expert copy"));
+          c->h_eptr_cache[(size_t)l * c->n_blobs + E + s] = dst;
+        }
+      }
+    }
+    if (cudaMemcpy(c->d_eptr_cache, c->h_eptr_cache, (size_t)L * c->n_blobs * sizeof(void*), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+      return bail(fail(FT_ERR_CUDA, "cache table"));
+  }
+  for (int b = 0; b < 2; b++) cudaEventRecord(c->ev_done[b], c->copy_stream);
+  if (cudaDeviceSynchronize() != cudaSuccess) return bail(fail(FT_ERR_CUDA, "create sync"));
+  *out = c;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_destroy(ft_ctx* c) {
+  if (!c) return FT_OK;
+  cudaDeviceSynchronize();
+  for (auto& m : c->tmarks) {
+    cudaEventDestroy(m.second.first);
+    cudaEventDestroy(m.second.second);
+  }
+  for (auto& pr : c->copy_timing) {
+    cudaEventDestroy(pr.first);
+    cudaEventDestroy(pr.second);
+  }
+  free_prefill_scratch(c->pf);
+  cudaFree(c->d_status);
+  cudaFree(c->d_logits);
+  cudaFree(c->d_ids);
+  cudaFree(c->d_w);
+  cudaFree(c->d_offs);
+  cudaFree(c->d_perm);
+  cudaFree(c->d_inv);
+  cudaFree(c->d_active);
+  cudaFree(c->d_nact);
+  cudaFree(c->d_pad_offs);
+  cudaFree(c->d_h);
+  cudaFree(c->d_eptr_res);
+  cudaFree(c->d_eptr_cache);
+  cudaFree(c->d_shared);
+  for (int b = 0; b < 2; b++) {
+    cudaFree(c->d_stage[b]);
+    cudaFree(c->d_eptr_stage[b]);
+    if (c->ev_landed[b]) cudaEventDestroy(c->ev_landed[b]);
+    if (c->ev_done[b]) cudaEventDestroy(c->ev_done[b]);
+  }
+  if (c->h_eptr_cache) cudaFreeHost(c->h_eptr_cache);
+  if (c->h_ids) cudaFreeHost(c->h_ids);
+  if (c->h_status) cudaFreeHost(c->h_status);
+  if (c->ev_ids) cudaEventDestroy(c->ev_ids);
+  if (c->va) {
+    for (size_t i = 0; i < c->chunks.size(); i++) {
+      c->drv.memUnmap(c->va + i * c->chunk, c->chunk);
+      c->drv.memRelease(c->chunks[i]);
+    }
+    c->drv.memAddressFree(c->va, c->va_size);
+  }
+  for (void* p : c->registered) cudaHostUnregister(p);
+  if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
+  delete c;
+  cudaGetLastError();
+  return FT_OK;
+}
+
+// bounded host wait on an event: polls, gives up after kHostWaitSeconds
+static ft_status wait_event(cudaEvent_t ev, const char* what) {
+  auto t0 = std::chrono::steady_clock::now();
+  int spins = 0;
+  while (true) {
+    cudaError_t q = cudaEventQuery(ev);
+    if (q == cudaSuccess) return FT_OK;
+    if (q != cudaErrorNotReady) return fail(FT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(q));
+    if (++spins > 64) std::this_thread::sleep_for(std::chrono::microseconds(20));
+    double s = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+    if (s > kHostWaitSeconds) return fail(FT_ERR_TIMEOUT, "%s: gave up after %.1f s", what, s);
+  }
+}
+
+static ft_status status_to_ft(int st) {
+  if (st & kStNonfinite) return fail(FT_ERR_NONFINITE, "NaN or +inf router logit (or no finite logit in a row)");
+  if (st & kStBadId) return fail(FT_ERR_INVALID, "expert id out of range");
+  if (st & kStMissing) return fail(FT_ERR_NOT_FOUND, "an expert blob pointer was NULL at kernel time");
+  if (st & kStTimeout) return fail(FT_ERR_TIMEOUT, "a device wait gave up");
+  return FT_OK;
+}
+
+extern "C" ft_status ft_sync_status(ft_ctx* c, void* stream) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  CUDA_TRY(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  return status_to_ft(*c->h_status);
+}
+
+// ---------------------------------------------------------------------------
+// single steps
+// ---------------------------------------------------------------------------
+extern "C" ft_status ft_router_logits(ft_ctx* c, const void* x, int64_t T, int32_t H, const float* wr, int32_t E,
+                                      float* logits, void* stream) {
+  if (!c || (!x && T > 0) || !wr || !logits) return fail(FT_ERR_INVALID, "NULL argument");
+  if (T < 0 || H <= 0 || H % 128 || E <= 0) return fail(FT_ERR_INVALID, "bad shape T=%lld H=%d E=%d", (long long)T, H, E);
+  CUDA_TRY(launch_router_logits((const uint16_t*)x, wr, (int)T, H, E, logits, (cudaStream_t)stream));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_moe_route(ft_ctx* c, const float* logits, int64_t T, int32_t E, int32_t k, uint32_t flags,
+                                  int32_t* ids, float* w, void* stream) {
+  if (!c || !logits || !ids || !w) return fail(FT_ERR_INVALID, "NULL argument");
+  if (T < 0 || E <= 0 || E > 1024 || k <= 0 || k > 16 || k > E) return fail(FT_ERR_INVALID, "bad shape E=%d k=%d", E, k);
+  CUDA_TRY(launch_topk(logits, (int)T, E, k, (flags & FT_ROUTE_RENORM) ? 1 : 0, ids, w, c->d_status,
+                       (cudaStream_t)stream));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_moe_permute(ft_ctx* c, const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t* offs,
+                                    int32_t* perm, int32_t* inv, void* stream) {
+  if (!c || !ids || !offs || !perm || !inv) return fail(FT_ERR_INVALID, "NULL argument");
+  if (T < 0 || E <= 0 || E > 1024 || k <= 0) return fail(FT_ERR_INVALID, "bad shape");
+  if (E > c->d.n_experts) {
+    return fail(FT_ERR_INVALID, "E=%d larger than the context's n_experts %d (scratch)", E, c->d.n_experts);
+  }
+  CUDA_TRY(launch_permute(ids, (int)(T * k), E, offs, perm, inv, c->d_active, c->d_nact, nullptr, c->d_status,
+                          (cudaStream_t)stream));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_quantize_mxfp4(ft_ctx* c, const float* x, int64_t R, int32_t K, uint8_t* codes,
+                                       uint8_t* scales, void* stream) {
+  if (!c || (!x && R > 0) || !codes || !scales) return fail(FT_ERR_INVALID, "NULL argument");
+  if (R < 0 || K <= 0 || K % 128) return fail(FT_ERR_INVALID, "K=%d not a positive multiple of 128", K);
+  CUDA_TRY(launch_quantize_rows(x, R, K, codes, scales, (cudaStream_t)stream));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_debug_dequant(ft_ctx* c, const void* blob, int32_t mat, float* out, void* stream) {
+  if (!c || !blob || !out || mat < 0 || mat > 2) return fail(FT_ERR_INVALID, "bad argument");
+  int rows = mat < 2 ? c->d.inter : c->d.hidden;
+  int K = mat < 2 ? c->d.hidden : c->d.inter;
+  CUDA_TRY(launch_dequant((const uint8_t*)blob, c->lay, mat, rows, K, out, (cudaStream_t)stream));
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// expert cache
+// ---------------------------------------------------------------------------
+static void record(ft_ctx* c, int kind, int layer, int expert, int slot, int from) {
+  c->trace.push_back(ft_cache_event{kind, layer, expert, slot, from});
+}
+
+static int64_t key_of(ft_ctx* c, int layer, int expert) { return (int64_t)layer * c->d.n_experts + expert; }
+
+// Evict the least recent key not in `keep` (may be empty); returns its slot
+// (-1 if none) and the evicted key in *victim.
+static int32_t evict_one(ft_ctx* c, const std::vector<int64_t>& keep, int64_t* victim = nullptr) {
+  for (auto it = c->lru.order.begin(); it != c->lru.order.end(); ++it) {
+    int64_t key = *it;
+    if (std::find(keep.begin(), keep.end(), key) != keep.end()) continue;
+    auto m = c->lru.map.find(key);
+    int32_t slot = m->second.first;
+    c->lru.order.erase(it);
+    c->lru.map.erase(m);
+    c->lru.slot_used[slot] = 0;
+    int layer = (int)(key / c->d.n_experts), e = (int)(key % c->d.n_experts);
+    c->h_eptr_cache[(size_t)layer * c->n_blobs + e] = nullptr;
+    record(c, FT_EV_EVICT, layer, e, slot, -1);
+    c->stats.evictions++;
+    if (victim) *victim = key;
+    return slot;
+  }
+  return -1;
+}
+
+// Issue the H2D copy of (layer, e) into `slot` on the copy stream.
+static ft_status fetch(ft_ctx* c, int layer, int e, int32_t slot) {
+  const uint8_t* src = c->host_layers[layer] + (size_t)e * c->stride;
+  CUDA_TRY(cudaMemcpyAsync(slot_ptr(c, slot), src, (size_t)c->lay.used, cudaMemcpyHostToDevice, c->copy_stream));
+  c->stats.h2d_bytes += c->lay.used;
+  return FT_OK;
+}
+
+// One decode step of the cache for `layer` over the distinct experts S (ascending).
+static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, bool& any_miss, std::vector<int>& dirty) {
+  any_miss = false;
+  if ((int64_t)S.size() > c->lru.capacity)
+    return fail(FT_ERR_NO_SPACE, "%zu experts in one step exceed the cache capacity of %lld slots", S.size(),
+                (long long)c->lru.capacity);
+  std::vector<int64_t> keep;
+  keep.reserve(S.size());
+  for (int e : S) keep.push_back(key_of(c, layer, e));
+  cudaEvent_t t0 = nullptr, t1 = nullptr;
+  for (int e : S) {
+    int64_t key = key_of(c, layer, e);
+    auto m = c->lru.map.find(key);
+    if (m != c->lru.map.end()) {
+      c->lru.order.splice(c->lru.order.end(), c->lru.order, m->second.second);
+      record(c, FT_EV_HIT, layer, e, m->second.first, -1);
+      c->stats.hits++;
+      continue;
+    }
+    int32_t slot;
+    if ((int64_t)c->lru.map.size() >= c->lru.capacity) {
+      int64_t victim = -1;
+      slot = evict_one(c, keep, &victim);
+      if (slot < 0) return fail(FT_ERR_NO_SPACE, "no evictable key");
+      dirty.push_back((int)(victim / c->d.n_experts));
+    } else {
+      slot = c->lru.lowest_free();
+    }
+    if (!any_miss) {
+      cudaEventCreate(&t0);
+      cudaEventCreate(&t1);
+      cudaEventRecord(t0, c->copy_stream);
+    }
+    any_miss = true;
+    c->lru.order.push_back(key);
+    c->lru.map[key] = {slot, std::prev(c->lru.order.end())};
+    c->lru.slot_used[slot] = 1;
+    c->h_eptr_cache[(size_t)layer * c->n_blobs + e] = slot_ptr(c, slot);
+    record(c, FT_EV_MISS, layer, e, slot, -1);
+    c->stats.misses++;
+    FT_TRY(fetch(c, layer, e, slot));
+  }
+  if (any_miss) {
+    cudaEventRecord(t1, c->copy_stream);
+    c->copy_timing.push_back({t0, t1});
+  }
+  c->stats.used_slots = (int64_t)c->lru.map.size();
+  return FT_OK;
+}
+
+static ft_status push_table_rows(ft_ctx* c, const std::vector<int>& rows, cudaStream_t s) {
+  std::vector<int> r = rows;
+  std::sort(r.begin(), r.end());
+  r.erase(std::unique(r.begin(), r.end()), r.end());
+  for (int l : r)
+    CUDA_TRY(cudaMemcpyAsync(c->d_eptr_cache + (size_t)l * c->n_blobs, c->h_eptr_cache + (size_t)l * c->n_blobs,
+                             c->n_blobs * sizeof(void*), cudaMemcpyHostToDevice, s));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_expert_cache_lookup(ft_ctx* c, int32_t layer, int32_t expert, int32_t* slot) {
+  if (!c || !slot) return fail(FT_ERR_INVALID, "NULL argument");
+  if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
+  if (layer < 0 || layer >= c->d.n_layers || expert < 0 || expert >= c->d.n_experts)
+    return fail(FT_ERR_INVALID, "bad key (%d, %d)", layer, expert);
+  auto m = c->lru.map.find(key_of(c, layer, expert));
+  if (m == c->lru.map.end()) {
+    *slot = -1;
+    return FT_OK;
+  }
+  c->lru.order.splice(c->lru.order.end(), c->lru.order, m->second.second);
+  *slot = m->second.first;
+  record(c, FT_EV_HIT, layer, expert, *slot, -1);
+  c->stats.hits++;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_expert_cache_insert(ft_ctx* c, int32_t layer, int32_t expert, int32_t* slot,
+                                            int64_t* evicted_key, void* stream) {
+  if (!c || !slot) return fail(FT_ERR_INVALID, "NULL argument");
+  if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
+  if (layer < 0 || layer >= c->d.n_layers || expert < 0 || expert >= c->d.n_experts)
+    return fail(FT_ERR_INVALID, "bad key (%d, %d)", layer, expert);
+  if (!c->host_layers[layer]) return fail(FT_ERR_NOT_FOUND, "layer %d has no host pool", layer);
+  if (evicted_key) *evicted_key = -1;
+  if (c->lru.capacity <= 0) return fail(FT_ERR_NO_SPACE, "cache capacity is 0");
+  cudaStream_t s = (cudaStream_t)stream;
+  // table rows may still be read by queued work: order after it
+  if (c->last_stream) CUDA_TRY(cudaStreamSynchronize(c->last_stream));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  std::vector<int> S{expert};
+  std::vector<int> dirty{layer};
+  int64_t before_evict = c->stats.evictions;
+  int64_t victim = -1;
+  if (c->lru.map.find(key_of(c, layer, expert)) == c->lru.map.end() && (int64_t)c->lru.map.size() >= c->lru.capacity)
+    victim = c->lru.order.front();
+  bool any_miss;
+  FT_TRY(cache_step(c, layer, S, any_miss, dirty));
+  if (evicted_key && c->stats.evictions > before_evict) *evicted_key = victim;
+  *slot = c->lru.map[key_of(c, layer, expert)].first;
+  if (any_miss) {
+    cudaEvent_t done = c->copy_timing.back().second;
+    CUDA_TRY(cudaStreamWaitEvent(s, done, 0));
+  }
+  FT_TRY(push_table_rows(c, dirty, s));
+  c->last_stream = s;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_expert_cache_resize(ft_ctx* c, int64_t new_budget) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (new_budget < 0) return fail(FT_ERR_INVALID, "negative budget");
+  if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
+  CUDA_TRY(cudaDeviceSynchronize());
+  int64_t cap = new_budget / c->stride;
+  if ((size_t)cap * c->stride > c->va_size) return fail(FT_ERR_NO_SPACE, "budget larger than the reserved arena");
+  if (cap < c->lru.capacity) {
+    while ((int64_t)c->lru.map.size() > cap) evict_one(c, {});
+    // survivors in slots >= cap move down to the lowest free slots, ascending
+    std::vector<std::pair<int32_t, int64_t>> movers;
+    for (auto& kv : c->lru.map)
+      if (kv.second.first >= cap) movers.push_back({kv.second.first, kv.first});
+    std::sort(movers.begin(), movers.end());
+    for (auto& mv : movers) {
+      int32_t from = mv.first;
+      int32_t to = -1;
+      for (int64_t s2 = 0; s2 < cap; s2++)
+        if (!c->lru.slot_used[s2]) {
+          to = (int32_t)s2;
+          break;
+        }
+      CUDA_TRY(cudaMemcpyAsync(slot_ptr(c, to), slot_ptr(c, from), (size_t)c->lay.used, cudaMemcpyDeviceToDevice,
+                               c->copy_stream));
+      c->lru.slot_used[from] = 0;
+      c->lru.slot_used[to] = 1;
+      c->lru.map[mv.second].first = to;
+      int layer = (int)(mv.second / c->d.n_experts), e = (int)(mv.second % c->d.n_experts);
+      c->h_eptr_cache[(size_t)layer * c->n_blobs + e] = slot_ptr(c, to);
+      record(c, FT_EV_MOVE, layer, e, to, from);
+      c->stats.moves++;
+    }
+    CUDA_TRY(cudaStreamSynchronize(c->copy_stream));
+  }
+  c->lru.set_capacity(cap);
+  for (int64_t s2 = cap; s2 < (int64_t)c->lru.slot_used.size(); s2++) c->lru.slot_used[s2] = 0;
+  FT_TRY(arena_map(c, cap));
+  c->stats.capacity_slots = cap;
+  c->stats.used_slots = (int64_t)c->lru.map.size();
+  CUDA_TRY(cudaMemcpy(c->d_eptr_cache, c->h_eptr_cache, (size_t)c->d.n_layers * c->n_blobs * sizeof(void*),
+                      cudaMemcpyHostToDevice));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_cache_trace(ft_ctx* c, ft_cache_event* buf, int64_t cap, int64_t* n) {
+  if (!c || !n || (cap > 0 && !buf)) return fail(FT_ERR_INVALID, "NULL argument");
+  int64_t m = std::min<int64_t>(cap, (int64_t)c->trace.size());
+  if (m > 0) memcpy(buf, c->trace.data(), (size_t)m * sizeof(ft_cache_event));
+  *n = m;
+  bool over = (int64_t)c->trace.size() > cap;
+  c->trace.clear();
+  if (over) return fail(FT_ERR_NO_SPACE, "trace had more events than cap");
+  return FT_OK;
+}
+
+extern "C" ft_status ft_cache_stats_get(ft_ctx* c, ft_cache_stats* out, int32_t reset) {
+  if (!c || !out) return fail(FT_ERR_INVALID, "NULL argument");
+  if (!c->copy_timing.empty()) {
+    CUDA_TRY(cudaStreamSynchronize(c->copy_stream));
+    for (auto& pr : c->copy_timing) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess) c->stats.h2d_ms += ms;
+      cudaEventDestroy(pr.first);
+      cudaEventDestroy(pr.second);
+    }
+    c->copy_timing.clear();
+  }
+  *out = c->stats;
+  if (reset) {
+    int64_t cap = c->stats.capacity_slots, used = c->stats.used_slots, mapped = c->stats.mapped_bytes;
+    c->stats = ft_cache_stats{};
+    c->stats.capacity_slots = cap;
+    c->stats.used_slots = used;
+    c->stats.mapped_bytes = mapped;
+  }
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// prefetch
+// ---------------------------------------------------------------------------
+extern "C" ft_status ft_prefetch_layer(ft_ctx* c, int32_t layer, void* compute_stream) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (layer < 0 || layer >= c->d.n_layers) return fail(FT_ERR_INVALID, "layer %d out of range", layer);
+  if (!c->host_layers[layer]) return fail(FT_ERR_NOT_FOUND, "layer %d has no host pool", layer);
+  (void)compute_stream;
+  const int b = layer & 1;
+  const size_t bytes = (size_t)c->n_blobs * c->stride;
+  if (!c->d_stage[b]) {
+    CUDA_TRY(cudaMalloc((void**)&c->d_stage[b], bytes));
+    std::vector<const uint8_t*> tab(c->n_blobs);
+    for (int e = 0; e < c->n_blobs; e++) tab[e] = c->d_stage[b] + (size_t)e * c->stride;
+    CUDA_TRY(cudaMalloc((void**)&c->d_eptr_stage[b], c->n_blobs * sizeof(void*)));
+    CUDA_TRY(cudaMemcpy(c->d_eptr_stage[b], tab.data(), c->n_blobs * sizeof(void*), cudaMemcpyHostToDevice));
+  }
+  // reuse only after the last forward that read this buffer is done
+  CUDA_TRY(cudaStreamWaitEvent(c->copy_stream, c->ev_done[b], 0));
+  CUDA_TRY(cudaMemcpyAsync(c->d_stage[b], c->host_layers[layer], bytes, cudaMemcpyHostToDevice, c->copy_stream));
+  CUDA_TRY(cudaEventRecord(c->ev_landed[b], c->copy_stream));
+  c->stage_layer[b] = layer;
+  c->prefetch_bytes += (int64_t)bytes;
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// layer forward
+// ---------------------------------------------------------------------------
+extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* x, int64_t T,
+                                          const float* router_w, const float* logits_override, void* out,
+                                          uint32_t flags, void* stream) {
+  if (!c || !out || (!x && T > 0)) return fail(FT_ERR_INVALID, "NULL argument");
+  if (layer < 0 || layer >= c->d.n_layers) return fail(FT_ERR_INVALID, "layer %d out of range", layer);
+  if (T < 0 || T > c->max_tokens) return fail(FT_ERR_INVALID, "T=%lld outside [0, max_tokens=%d]", (long long)T, c->max_tokens);
+  if (!logits_override && !router_w) return fail(FT_ERR_INVALID, "need router_w or logits_override");
+  if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
+  const bool mx = (flags & FT_ACT_MXFP4) != 0;
+  if (!mx && T > c->decode_max_t)
+    return fail(FT_ERR_INVALID, "decode GEMV path takes T <= %d (use FT_ACT_MXFP4 for prefill)", c->decode_max_t);
+  if (T == 0) return FT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int H = c->d.hidden, E = c->d.n_experts, k = c->d.top_k, Ti = (int)T;
+
+  // 1-3: logits, top-k, permutation
+  const float* logits = logits_override;
+  if (!logits) {
+    KTimer kt(c, FT_K_ROUTER_LOGITS, s);
+    CUDA_TRY(launch_router_logits((const uint16_t*)x, router_w, Ti, H, E, c->d_logits, s));
+    logits = c->d_logits;
+  }
+  {
+    KTimer kt(c, FT_K_TOPK, s);
+    CUDA_TRY(launch_topk(logits, Ti, E, k, (flags & FT_ROUTE_RENORM) ? 1 : 0, c->d_ids, c->d_w, c->d_status, s));
+  }
+  {
+    KTimer kt(c, FT_K_PERMUTE, s);
+    CUDA_TRY(launch_permute(c->d_ids, Ti * k, E, c->d_offs, c->d_perm, c->d_inv, c->d_active, c->d_nact,
+                            mx ? c->d_pad_offs : nullptr, c->d_status, s));
+  }
+
+  // 4: weight source.  Prefill (MXFP4) reads resident or staged layers and
+  // never touches the cache; decode reads resident layers or the cache.
+  const uint8_t* const* eptr = nullptr;
+  int stage_buf = -1;
+  if (c->resident[layer]) {
+    eptr = c->d_eptr_res + (size_t)layer * c->n_blobs;
+  } else if (mx) {
+    if (c->stage_layer[layer & 1] != layer)
+      return fail(FT_ERR_NOT_FOUND, "prefill of layer %d: not resident and not prefetched", layer);
+    stage_buf = layer & 1;
+    CUDA_TRY(cudaStreamWaitEvent(s, c->ev_landed[stage_buf], 0));
+    eptr = c->d_eptr_stage[stage_buf];
+  } else if (c->cache_on && c->host_layers[layer]) {
+    CUDA_TRY(cudaMemcpyAsync(c->h_ids, c->d_ids, (size_t)Ti * k * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaEventRecord(c->ev_ids, s));
+    FT_TRY(wait_event(c->ev_ids, "routing ids"));
+    if (*c->h_status) {
+      int st = *c->h_status;
+      CUDA_TRY(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
+      return status_to_ft(st);
+    }
+    std::vector<int> S(c->h_ids, c->h_ids + (size_t)Ti * k);
+    for (int e : S)
+      if (e < 0 || e >= E) return fail(FT_ERR_INVALID, "expert id %d out of range", e);
+    std::sort(S.begin(), S.end());
+    S.erase(std::unique(S.begin(), S.end()), S.end());
+    std::vector<int> dirty{layer};
+    bool any_miss = false;
+    FT_TRY(cache_step(c, layer, S, any_miss, dirty));
+    if (any_miss) CUDA_TRY(cudaStreamWaitEvent(s, c->copy_timing.back().second, 0));
+    FT_TRY(push_table_rows(c, dirty, s));
+    eptr = c->d_eptr_cache + (size_t)layer * c->n_blobs;
+  } else {
+    return fail(FT_ERR_NOT_FOUND, "layer %d is neither resident nor cached", layer);
+  }
+
+  // 5: experts and combine
+  if (!mx) {
+    GemvParams p{};
+    p.x = (const uint16_t*)x;
+    p.T = Ti;
+    p.H = H;
+    p.I = c->d.inter;
+    p.E = E;
+    p.k = k;
+    p.n_shared = c->d.n_shared;
+    p.max_active = std::min(E, Ti * k);
+    p.offs = c->d_offs;
+    p.perm = c->d_perm;
+    p.inv = c->d_inv;
+    p.w = c->d_w;
+    p.active = c->d_active;
+    p.n_active = c->d_nact;
+    p.eptr = eptr;
+    p.lay = c->lay;
+    p.h = c->d_h;
+    p.out = (uint16_t*)out;
+    p.status = c->d_status;
+    {
+      KTimer kt(c, FT_K_GATE_UP, s);
+      CUDA_TRY(launch_gate_up(p, s));
+    }
+    {
+      KTimer kt(c, FT_K_DOWN_COMBINE, s);
+      CUDA_TRY(launch_down_combine(p, s));
+    }
+  } else {
+    FT_TRY(ensure_prefill_scratch(c->pf, c->d, c->max_tokens));
+    PrefillArgs a{};
+    a.x = (const uint16_t*)x;
+    a.T = Ti;
+    a.H = H;
+    a.I = c->d.inter;
+    a.E = E;
+    a.k = k;
+    a.n_shared = c->d.n_shared;
+    a.ids = c->d_ids;
+    a.w = c->d_w;
+    a.offs = c->d_offs;
+    a.perm = c->d_perm;
+    a.inv = c->d_inv;
+    a.pad_offs = c->d_pad_offs;
+    a.eptr = eptr;
+    a.lay = c->lay;
+    a.out = (uint16_t*)out;
+    a.status = c->d_status;
+    cudaError_t e = run_prefill(c->pf, a, s);
+    if (e != cudaSuccess) return fail(FT_ERR_CUDA, "prefill: %s", cudaGetErrorString(e));
+  }
+  if (stage_buf >= 0) CUDA_TRY(cudaEventRecord(c->ev_done[stage_buf], s));
+  c->last_stream = s;
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// per-kernel timing
+// ---------------------------------------------------------------------------
+static void drop_marks(ft_ctx* c) {
+  for (auto& m : c->tmarks) {
+    cudaEventDestroy(m.second.first);
+    cudaEventDestroy(m.second.second);
+  }
+  c->tmarks.clear();
+}
+
+extern "C" ft_status ft_kernel_timing_enable(ft_ctx* c, int32_t on) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  CUDA_TRY(cudaDeviceSynchronize());
+  drop_marks(c);
+  for (int i = 0; i < FT_K_COUNT; i++) {
+    c->tms[i] = 0;
+    c->tlaunch[i] = 0;
+  }
+  c->timing = on != 0;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_kernel_timing_read(ft_ctx* c, double* ms, int64_t* launches, int32_t n) {
+  if (!c || !ms || !launches || n < 0) return fail(FT_ERR_INVALID, "bad argument");
+  CUDA_TRY(cudaDeviceSynchronize());
+  for (auto& m : c->tmarks) {
+    float t = 0.f;
+    CUDA_TRY(cudaEventElapsedTime(&t, m.second.first, m.second.second));
+    c->tms[m.first] += t;
+    c->tlaunch[m.first] += 1;
+  }
+  drop_marks(c);
+  for (int i = 0; i < n && i < FT_K_COUNT; i++) {
+    ms[i] = c->tms[i];
+    launches[i] = c->tlaunch[i];
+  }
+  return FT_OK;
+}

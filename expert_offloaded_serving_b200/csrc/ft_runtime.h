@@ -1,0 +1,46 @@
+// Runtime-internal declarations shared by the runtime and the prefill path.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ft_common.cuh"
+
+namespace ft {
+
+constexpr int kDecodeMaxTokens = 16;               // largest T of the decode GEMV path
+constexpr size_t kArenaChunkBytes = 256ull << 20;  // physical chunk under the slot arena
+constexpr double kHostWaitSeconds = 30.0;          // bounded host waits
+
+struct PrefillArgs {
+  const uint16_t* x;  // bf16 [T][H]
+  int T, H, I, E, k, n_shared;
+  const int32_t* ids;       // [T*k]
+  const float* w;           // [T*k]
+  const int32_t* offs;      // [E+1]
+  const int32_t* perm;      // [T*k]
+  const int32_t* inv;       // [T*k]
+  const int32_t* pad_offs;  // [E+1] 128-padded segment starts
+  const uint8_t* const* eptr;
+  BlobLayout lay;
+  uint16_t* out;  // bf16 [T][H]
+  int* status;
+};
+
+struct PrefillScratch {
+  int64_t max_rows = 0;     // padded activation rows
+  int64_t max_pairs = 0;    // rows of y
+  int H = 0, I = 0;
+  uint8_t* xq = nullptr;    // [max_rows][H/2]
+  uint8_t* xq_sf = nullptr; // atoms over [max_rows][H/32]
+  uint8_t* hq = nullptr;    // [max_rows][I/2]
+  uint8_t* hq_sf = nullptr; // atoms over [max_rows][I/32]
+  float* y = nullptr;       // [max_pairs][H]
+  int* work = nullptr;      // tile list scratch
+};
+
+ft_status ensure_prefill_scratch(PrefillScratch& s, const ft_model_desc& d, int max_tokens);
+void free_prefill_scratch(PrefillScratch& s);
+cudaError_t run_prefill(PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
+
+}  // namespace ft

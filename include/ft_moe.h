@@ -1,0 +1,304 @@
+/*
+ * ft_moe.h — C ABI of libftmoe.so: one MoE layer forward pass with a GPU
+ * expert cache over a pinned host expert pool, for NVIDIA B200 (sm_100a).
+ *
+ * Method: the FreeToken serving engine as described in its public write-ups.
+ * Citations name the page and its section (or paragraph topic):
+ *   [hu]  aiforradalom.hu, "Egyetlen munkaállomás-GPU-n futtatja a 753
+ *         milliárdos GLM-5.2 modellt a FreeToken", section "A Mixture-of-Experts
+ *         (MoE) kihívásai és a FreeToken megoldásai"
+ *   [no]  jansverre.net, "FreeToken GLM-5.2 en GPU", sections "Hva er
+ *         FreeToken?" and "Hvorfor er båndbredden viktigere enn antall kjerner?"
+ *   [fa]  aipolix.com, "FreeToken مدلهای عظیم MoE را روی GPUهای مصرفی اجرا
+ *         میکند", paragraphs on bandwidth-adaptive execution, on
+ *         semantic-aware caching and on elastic memory management
+ *
+ * Conventions
+ *   - Every call returns ft_status; nothing throws across the ABI.  On error
+ *     ft_last_error() gives a message (thread-local, valid until the next call
+ *     from the same thread).
+ *   - "dev" pointers are CUDA device pointers owned by the caller; "host"
+ *     pointers are host memory owned by the caller.  Streams are cudaStream_t
+ *     values passed as void* (NULL = the legacy default stream).
+ *   - Kernels run asynchronously on the given stream.  Errors that only the
+ *     device can see (a NaN or +inf logit, an expert id out of range, a bounded
+ *     device wait that gave up) set a status word in the context; they are
+ *     returned by ft_sync_status() and by the next call that synchronises
+ *     with the host (the cache path of ft_moe_layer_forward does).
+ *   - Sizes are int64_t, ids int32_t.  Calls on one context are not
+ *     thread-safe and must be ordered by the caller (one compute stream).
+ *
+ * Expert weight format (one "blob" per expert, stride ft_blob_stride()):
+ *   codes, row-major, K contiguous, two e2m1 codes per byte (element 2i in the
+ *   low nibble): Wg [I][H], Wu [I][H], Wd [H][I]; then UE8M0 block scales (one
+ *   byte per 32 elements along K) of Wg, Wu, Wd, each region tiled in 512-byte
+ *   atoms of 128 rows x 4 blocks (row r at byte (r%32)*16 + ((r%128)/32)*4 +
+ *   block%4; atoms along K first); zero padding to a multiple of 256 bytes.
+ *   A layer holds n_experts routed blobs followed by n_shared shared blobs.
+ *   MXFP4 = e2m1 elements with per-32 UE8M0 scales ([no] "MXFP4";
+ *   [hu] FP4 expert pool).
+ */
+#ifndef FT_MOE_H
+#define FT_MOE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FT_API __attribute__((visibility("default")))
+#else
+#define FT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FT_OK = 0,
+  FT_ERR_INVALID = 1,    /* bad argument or shape */
+  FT_ERR_CUDA = 2,       /* a CUDA runtime / driver call failed */
+  FT_ERR_NO_SPACE = 3,   /* cache capacity below the experts one step needs */
+  FT_ERR_TIMEOUT = 4,    /* a bounded host or device wait gave up */
+  FT_ERR_NOT_FOUND = 5,  /* key not resident / layer not staged */
+  FT_ERR_NONFINITE = 6,  /* NaN or +inf router logit, or a row with no finite logit */
+  FT_ERR_STATE = 7       /* call not valid in the context's current state */
+} ft_status;
+
+typedef struct ft_ctx ft_ctx;
+
+typedef struct {
+  int32_t hidden;             /* H, multiple of 128 */
+  int32_t inter;              /* I, expert intermediate size, multiple of 128 */
+  int32_t n_experts;          /* E routed experts per layer, <= 1024 */
+  int32_t top_k;              /* k experts per token, <= 16 and <= E */
+  int32_t n_layers;           /* L */
+  int32_t n_shared;           /* always-on shared experts per layer (weight 1), 0 or 1 */
+  int64_t cache_budget_bytes; /* GPU expert-cache budget (0 = no cache) */
+  int32_t max_tokens;         /* largest T any forward call passes; sizes scratch */
+  int32_t reserved;
+} ft_model_desc;
+
+/* forward / route flags */
+#define FT_ROUTE_RENORM 1u    /* renormalise the k softmax weights to sum 1 (default on) */
+#define FT_ACT_BF16     0u    /* decode: bf16 activations, fp32 h, split-K FP4 GEMV */
+#define FT_ACT_MXFP4    2u    /* prefill: x and h quantised to MXFP4, tcgen05 grouped GEMM */
+
+/* cache trace events */
+#define FT_EV_HIT   0
+#define FT_EV_MISS  1
+#define FT_EV_EVICT 2
+#define FT_EV_MOVE  3
+typedef struct {
+  int32_t kind;      /* FT_EV_* */
+  int32_t layer;
+  int32_t expert;
+  int32_t slot;      /* slot after the event (the freed slot for EVICT) */
+  int32_t from_slot; /* old slot for MOVE, -1 otherwise */
+} ft_cache_event;
+
+typedef struct {
+  int64_t hits, misses, evictions, moves;
+  int64_t h2d_bytes;          /* bytes fetched from the host pool by misses */
+  double  h2d_ms;             /* copy-stream time of those fetches (CUDA events) */
+  int64_t capacity_slots, used_slots;
+  int64_t mapped_bytes;       /* physical memory mapped under the slot arena */
+} ft_cache_stats;
+
+/* ---------------------------------------------------------------------- */
+/* format                                                                  */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes per expert blob for hidden H and intermediate I (>= 0; -1 on bad shape).
+ * Equals 3*H*I*17/32 when the scale regions fill whole atoms. */
+FT_API int64_t ft_blob_stride(int32_t hidden, int32_t inter);
+
+/* Byte offsets of the regions of a blob: out[0..7] = Wg, Wu, Wd codes,
+ * Wg, Wu, Wd scales, used bytes, stride.  FT_ERR_INVALID on a bad shape. */
+FT_API ft_status ft_blob_layout(int32_t hidden, int32_t inter, int64_t out[8]);
+
+/* Message of the last error on this thread ("" if none). */
+FT_API const char* ft_last_error(void);
+
+/* ---------------------------------------------------------------------- */
+/* context                                                                 */
+/* ---------------------------------------------------------------------- */
+
+/* Create a context on the current CUDA device.
+ *   host_layers     host [L] pointers (or NULL): layer l's pool of
+ *                   (E + n_shared) blobs at ft_blob_stride() each, in host
+ *                   memory that must outlive the context.  Page-locked memory
+ *                   is used as is; pageable memory is registered (pinned) here
+ *                   and unregistered by ft_destroy.  Resize never reloads it
+ *                   ([fa] elastic memory management).
+ *   resident_layers host [L] pointers (or NULL): per-layer device copies of
+ *                   the same pools; a layer with a non-NULL entry is served
+ *                   from it and never touches the cache.
+ *   The library allocates the cache slot arena (CUDA virtual memory, sized by
+ *   desc->cache_budget_bytes), device scratch for desc->max_tokens tokens,
+ *   a copy stream and events.  Prefill staging buffers (2 layer pools) are
+ *   allocated on the first ft_prefetch_layer().
+ * Errors: FT_ERR_INVALID (shape limits above, NULL desc/out), FT_ERR_CUDA. */
+FT_API ft_status ft_create(const ft_model_desc* desc, const void* const* host_layers,
+                    const void* const* resident_layers, ft_ctx** out);
+
+/* Wait for the context's streams, free everything it allocated. */
+FT_API ft_status ft_destroy(ft_ctx* ctx);
+
+/* Copy the device status word to the host (synchronising `stream`), clear it,
+ * and map it: NaN/+inf logit -> FT_ERR_NONFINITE, bad id -> FT_ERR_INVALID,
+ * device wait gave up -> FT_ERR_TIMEOUT; else FT_OK. */
+FT_API ft_status ft_sync_status(ft_ctx* ctx, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* hot-path steps (also used by ft_moe_layer_forward)                      */
+/* ---------------------------------------------------------------------- */
+
+/* Router logits = x . Wr^T ([hu]: a gate picks 6 of 256 experts per layer).
+ *   x dev bf16 [T][H], wr dev fp32 [E][H], logits dev fp32 [T][E].
+ * Each bf16*fp32 product is exact in fp64; the sum runs in fp64 in a fixed
+ * order (element k joins partial sum (k/4) mod 32 in ascending k; the 32
+ * partials meet in an xor butterfly 16,8,4,2,1) and is rounded once to fp32,
+ * so results are reproducible bit for bit.  H % 128 == 0. */
+FT_API ft_status ft_router_logits(ft_ctx* ctx, const void* x, int64_t T, int32_t H,
+                           const float* wr, int32_t E, float* logits, void* stream);
+
+/* Softmax top-k routing ([hu], [no] "Hva er FreeToken?": the router picks a
+ * few experts per token).  logits dev fp32 [T][E]; ids dev int32 [T][k] in
+ * rank order (logit descending, ties to the lower id, -0 == +0, NaN below
+ * -inf); w dev fp32 [T][k]: softmax over all E at the chosen ids, divided by
+ * their sum when flags has FT_ROUTE_RENORM.  NaN/+inf logits or a row with no
+ * finite logit set the NONFINITE status (ids are still written).  E <= 1024,
+ * k <= 16. */
+FT_API ft_status ft_moe_route(ft_ctx* ctx, const float* logits, int64_t T, int32_t E, int32_t k,
+                       uint32_t flags, int32_t* ids, float* w, void* stream);
+
+/* Permutation of the T*k (token, rank) pairs by expert: histogram, scan and
+ * stable scatter.  ids dev int32 [T*k]; offs dev int32 [E+1] (pairs of expert
+ * e at positions offs[e]..offs[e+1]-1, ascending token); perm dev int32 [T*k]
+ * (perm[pos] = t*k + j); inv dev int32 [T*k] (inv[t*k+j] = pos).  Ids outside
+ * [0, E) set the INVALID status and are left out. */
+FT_API ft_status ft_moe_permute(ft_ctx* ctx, const int32_t* ids, int64_t T, int32_t k, int32_t E,
+                         int32_t* offs, int32_t* perm, int32_t* inv, void* stream);
+
+/* OCP MX quantisation of rows (prefill activations): x dev fp32 [R][K] ->
+ * codes dev uint8 [R][K/2] (two e2m1 per byte, element 2i low) and scales dev
+ * uint8 laid out in 128x4 atoms over [pad128(R)][K/32] (the blob scale
+ * layout).  Block scale = clamp(floor(log2 amax) - 2 + 127, 0, 254), elements
+ * rounded to nearest-even onto the e2m1 grid with saturation at 6, sign kept
+ * (a negative value that rounds to zero gives code 8).  K % 128 == 0. */
+FT_API ft_status ft_quantize_mxfp4(ft_ctx* ctx, const float* x, int64_t R, int32_t K,
+                            uint8_t* codes, uint8_t* scales, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* layer forward                                                           */
+/* ---------------------------------------------------------------------- */
+
+/* One MoE layer on T tokens ([no]: experts fetched to the GPU over PCIe or
+ * already cached are computed there, and the partial results are summed
+ * exactly):
+ *   out[t] = sum_j w[t][j] * FFN_{ids[t][j]}(x[t])  (+ shared FFN(x[t])),
+ *   FFN(x) = Wd (silu(Wg x) * (Wu x)), summed over j ascending in fp32,
+ *   rounded once to bf16.
+ *   x dev bf16 [T][H]; out dev bf16 [T][H] (must not alias x).
+ *   router_w dev fp32 [E][H], used when logits_override is NULL.
+ *   logits_override dev fp32 [T][E] or NULL.
+ *   flags: FT_ACT_BF16 (decode GEMV; T <= 64) or FT_ACT_MXFP4 (prefill
+ *   grouped GEMM; any T <= max_tokens), | FT_ROUTE_RENORM.
+ * Weights come from, in this order: the layer's resident device pool; the
+ * prefill staging buffer if ft_prefetch_layer(layer) was issued (the compute
+ * stream waits for that copy, [fa] double-buffered prefill); otherwise the
+ * expert cache: the selected ids are copied to the host (a stream
+ * synchronisation), the global LRU ([no] one LRU across MoE layers; [fa]
+ * shared LRU) is updated in ascending expert id, misses are copied from the
+ * host pool into their slots on the copy stream, and the experts run once
+ * their copies landed.
+ * Errors: FT_ERR_INVALID, FT_ERR_NO_SPACE (more distinct experts than
+ * slots), FT_ERR_NONFINITE / FT_ERR_TIMEOUT (cache path: checked at its
+ * synchronisation), FT_ERR_NOT_FOUND (no pool holds the layer), FT_ERR_CUDA. */
+FT_API ft_status ft_moe_layer_forward(ft_ctx* ctx, int32_t layer, const void* x, int64_t T,
+                               const float* router_w, const float* logits_override,
+                               void* out, uint32_t flags, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* expert cache ([no] global LRU; [fa] elastic resize)                     */
+/* ---------------------------------------------------------------------- */
+
+/* Slot of (layer, expert), touching it as most recent; *slot = -1 on a miss
+ * (no other change).  FT_ERR_INVALID on bad ids or no cache. */
+FT_API ft_status ft_expert_cache_lookup(ft_ctx* ctx, int32_t layer, int32_t expert, int32_t* slot);
+
+/* Make (layer, expert) resident: a hit only touches it; a miss evicts the
+ * least-recent key when full, then copies the blob from the host pool into
+ * its slot on the copy stream (`stream` waits for that copy).  *slot gets the
+ * slot, *evicted_key the evicted layer*E+expert or -1.  FT_ERR_NO_SPACE if
+ * the capacity is 0. */
+FT_API ft_status ft_expert_cache_insert(ft_ctx* ctx, int32_t layer, int32_t expert, int32_t* slot,
+                                 int64_t* evicted_key, void* stream);
+
+/* Change the cache budget ([fa]: resize without restart or pool reload).
+ * Waits for the context's streams.  Shrink: evict least-recent keys until the
+ * survivors fit, move survivors from slots >= the new capacity to the lowest
+ * free slots below it (device-to-device copies), then unmap the physical
+ * memory past the new size.  Grow: map more physical memory.  The host pool is
+ * not touched.  FT_ERR_INVALID for a negative budget; FT_ERR_CUDA if physical
+ * memory cannot be mapped. */
+FT_API ft_status ft_expert_cache_resize(ft_ctx* ctx, int64_t new_budget_bytes);
+
+/* Copy out the cache events recorded since the last call (HIT, MISS, EVICT,
+ * MOVE in order) and clear them.  *n = events written (<= cap); if more were
+ * recorded than cap the rest are dropped and FT_ERR_NO_SPACE is returned. */
+FT_API ft_status ft_cache_trace(ft_ctx* ctx, ft_cache_event* buf, int64_t cap, int64_t* n);
+
+/* Counters since creation (or the last reset). */
+FT_API ft_status ft_cache_stats_get(ft_ctx* ctx, ft_cache_stats* out, int32_t reset);
+
+/* ---------------------------------------------------------------------- */
+/* prefill prefetch ([fa]: next layer's experts cross PCIe while the GPU  */
+/* computes the current one; [no]: streams the next layer pack)            */
+/* ---------------------------------------------------------------------- */
+
+/* Start copying layer `layer`'s whole pool from host into staging buffer
+ * (layer & 1) on the copy stream.  The copy first waits until the last
+ * forward that read that buffer (recorded on its compute stream) finished.
+ * Returns at once.  FT_ERR_NOT_FOUND without a host pool; FT_ERR_CUDA. */
+FT_API ft_status ft_prefetch_layer(ft_ctx* ctx, int32_t layer, void* compute_stream);
+
+/* ---------------------------------------------------------------------- */
+/* parity export                                                           */
+/* ---------------------------------------------------------------------- */
+
+/* Dequantise matrix `mat` (0 = Wg, 1 = Wu, 2 = Wd) of a blob at dev pointer
+ * `blob` to fp32 out dev [rows][K] (exact).  Decodes with the same device
+ * routine the GEMV uses. */
+FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, float* out, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* measurement                                                             */
+/* ---------------------------------------------------------------------- */
+
+/* Kernel classes of the per-kernel timers. */
+#define FT_K_ROUTER_LOGITS 0
+#define FT_K_TOPK          1
+#define FT_K_PERMUTE       2
+#define FT_K_GATE_UP       3   /* decode gate/up + SwiGLU GEMV */
+#define FT_K_DOWN_COMBINE  4   /* decode down GEMV + combine */
+#define FT_K_QUANT_X       5   /* prefill activation quantiser */
+#define FT_K_GEMM_GATE_UP  6   /* prefill grouped GEMM, gate/up + SwiGLU + quantise h */
+#define FT_K_GEMM_DOWN     7   /* prefill grouped GEMM, down */
+#define FT_K_COMBINE       8   /* prefill combine */
+#define FT_K_COUNT         9
+
+/* Turn per-kernel CUDA-event timing on (1) or off (0).  While on, every
+ * kernel launch of the forward path is bracketed by events on its stream;
+ * launches inside stream capture are not timed.  Turning it on resets the
+ * counters. */
+FT_API ft_status ft_kernel_timing_enable(ft_ctx* ctx, int32_t on);
+
+/* Synchronise, then fill ms[i] (total device time) and launches[i] for the
+ * first n kernel classes (FT_K_*) since timing was enabled. */
+FT_API ft_status ft_kernel_timing_read(ft_ctx* ctx, double* ms, int64_t* launches, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FT_MOE_H */

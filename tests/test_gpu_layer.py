@@ -1,0 +1,102 @@
+"""GPU parity of ft_moe_layer_forward (decode path) against the oracle, on the
+shapes of the tiny layer and the 35B-class, DeepSeek-V4-Flash-class and
+GLM-class layers, with resident expert pools."""
+import numpy as np
+import pytest
+import torch
+
+import expert_offloaded_serving_b200 as ft
+import synth
+import synth.gpu
+from oracle import layer as olayer
+
+from _gpu import Ctx, assert_close, bf16_bits, x_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_layer(H, I, E, k, S, T, seed, use_router, renorm=True, trace=True, max_tokens=16):
+    pool = synth.gpu.layer_pool(H, I, E + S, seed, 0)
+    xb = synth.activations_bf16(seed, 1, T, H)
+    wr = synth.router_weights(seed, 0, E, H) if use_router else None
+    if use_router:
+        lg = None
+    elif trace:
+        sets = np.stack([synth.zipf_trace(seed, 0, 3, E, k, 1.1, 0.6, stream=t)[-1] for t in range(T)])
+        lg = synth.logits_for_sets(seed, 2, sets, E)
+    else:
+        lg = np.random.default_rng(seed).standard_normal((T, E)).astype(np.float32)
+    desc = ft.make_desc(H, I, E, k, 1, S, 0, max_tokens)
+    with Ctx(desc, None, [pool]) as c:
+        x = x_dev(xb)
+        out = torch.empty_like(x)
+        ft.ft_moe_layer_forward(c.h, 0, x, T, torch.from_numpy(wr).cuda() if use_router else None,
+                                torch.from_numpy(lg).cuda() if lg is not None else None, out,
+                                (ft.FT_ROUTE_RENORM if renorm else 0) | ft.FT_ACT_BF16)
+        ft.ft_sync_status(c.h)
+        got = bf16_bits(out)
+    want_ids_needed = None
+    blobs = {}
+
+    def blob_of(e):
+        if e not in blobs:
+            blobs[e] = synth.expert_blob(seed, 0, e, H, I)
+        return blobs[e]
+    r = olayer.moe_layer(xb, blob_of, H, I, E, k, logits=lg, router_w=wr, renorm=renorm,
+                         shared_blob=blob_of(E) if S else None)
+    return got, r
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 8])
+@pytest.mark.parametrize("use_router", [True, False])
+def test_tiny_layer(T, use_router):
+    got, r = run_layer(256, 128, 16, 2, 0, T, 1001, use_router, trace=False)
+    assert_close(got, r["out_f64"])
+
+
+def test_tiny_layer_no_renorm():
+    got, r = run_layer(256, 128, 16, 2, 0, 8, 1001, True, renorm=False)
+    assert_close(got, r["out_f64"])
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_35b_class_layer(T):
+    got, r = run_layer(2048, 512, 256, 8, 1, T, 1002, False)
+    assert_close(got, r["out_f64"])
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_dsv4_class_layer(T):
+    got, r = run_layer(4096, 2048, 256, 6, 0, T, 1003, False)
+    assert_close(got, r["out_f64"])
+
+
+def test_dsv4_class_layer_router_gemv():
+    got, r = run_layer(4096, 2048, 256, 6, 0, 2, 1003, True)
+    assert_close(got, r["out_f64"])
+
+
+def test_glm_class_layer():
+    got, r = run_layer(6144, 2048, 256, 8, 0, 1, 1005, False)
+    assert_close(got, r["out_f64"])
+
+
+def test_deterministic_repeat():
+    a, _ = run_layer(2048, 512, 256, 8, 1, 4, 1002, False)
+    b, _ = run_layer(2048, 512, 256, 8, 1, 4, 1002, False)
+    assert (a == b).all()
+
+
+def test_zero_tokens_and_limits():
+    pool = synth.gpu.layer_pool(256, 128, 16, 1, 0)
+    with Ctx(ft.make_desc(256, 128, 16, 2, 1, 0, 0, 4), None, [pool]) as c:
+        x = torch.zeros((4, 256), dtype=torch.bfloat16, device="cuda")
+        out = torch.zeros_like(x)
+        lg = torch.zeros((4, 16), dtype=torch.float32, device="cuda")
+        ft.ft_moe_layer_forward(c.h, 0, x, 0, None, lg, out, 1)     # T = 0 is a no-op
+        with pytest.raises(ft.FtError):
+            ft.ft_moe_layer_forward(c.h, 0, x, 5, None, lg, out, 1)  # above max_tokens
+        with pytest.raises(ft.FtError):
+            ft.ft_moe_layer_forward(c.h, 1, x, 1, None, lg, out, 1)  # no such layer
+        with pytest.raises(ft.FtError):
+            ft.ft_moe_layer_forward(c.h, 0, x, 1, None, lg, x, 1)    # out aliases x
