@@ -28,7 +28,8 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_router_logits", "ft_moe_route", "ft_moe_permute", "ft_quantize_mxfp4", "ft_moe_layer_forward",
            "ft_expert_cache_lookup", "ft_expert_cache_insert", "ft_expert_cache_resize", "ft_cache_trace",
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
-           "ft_kernel_timing_read")
+           "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc")
+FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine")
 
@@ -94,6 +95,7 @@ def lib() -> C.CDLL:
         "ft_debug_dequant": (ST, [P, P, I32, P, P]),
         "ft_kernel_timing_enable": (ST, [P, I32]),
         "ft_kernel_timing_read": (ST, [P, C.POINTER(C.c_double), C.POINTER(I64), I32]),
+        "ft_moe_layer_forward_noalloc": (ST, [I32, I32, I32, I32, I32, P, P, I64, P, P, P, U32, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -235,6 +237,15 @@ def ft_kernel_timing_read(ctx) -> dict:
     cnt = (I64 * n)()
     _check(lib().ft_kernel_timing_read(ctx, ms, cnt, n))
     return {KERNELS[i]: (ms[i], cnt[i]) for i in range(n)}
+
+
+def ft_moe_layer_forward_noalloc(hidden, inter, n_experts, top_k, n_shared, layer_pool, x, T, router_w,
+                                 logits_override, out, flags, status=None, stream=None) -> None:
+    """Decode forward that allocates no device memory (scratch in a static
+    device array shared by all calls; see ft_moe.h)."""
+    _check(lib().ft_moe_layer_forward_noalloc(hidden, inter, n_experts, top_k, n_shared, _ptr(layer_pool), _ptr(x),
+                                              T, _ptr(router_w), _ptr(logits_override), _ptr(out), flags,
+                                              _ptr(status), _stream(stream)))
 
 
 def make_desc(hidden, inter, n_experts, top_k, n_layers=1, n_shared=0, cache_budget_bytes=0,

@@ -59,6 +59,8 @@ static ft_status fail(ft_status st, const char* fmt, ...) {
 
 extern "C" const char* ft_last_error(void) { return g_err.c_str(); }
 
+void ft::set_last_error(const char* msg) { g_err = msg; }
+
 // ---------------------------------------------------------------------------
 // driver API entry points (no link-time dependency on libcuda)
 // ---------------------------------------------------------------------------

@@ -39,6 +39,9 @@ struct PrefillScratch {
   int* work = nullptr;      // tile list scratch
 };
 
+// Set the message ft_last_error() returns on this thread.
+void set_last_error(const char* msg);
+
 ft_status ensure_prefill_scratch(PrefillScratch& s, const ft_model_desc& d, int max_tokens);
 void free_prefill_scratch(PrefillScratch& s);
 cudaError_t run_prefill(PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);

@@ -298,6 +298,45 @@ FT_API ft_status ft_kernel_timing_enable(ft_ctx* ctx, int32_t on);
  * first n kernel classes (FT_K_*) since timing was enabled. */
 FT_API ft_status ft_kernel_timing_read(ft_ctx* ctx, double* ms, int64_t* launches, int32_t n);
 
+/* ---------------------------------------------------------------------- */
+/* forward without allocation                                              */
+/* ---------------------------------------------------------------------- */
+
+/* Largest scratch one ft_moe_layer_forward_noalloc call may use (bytes). */
+#define FT_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* The decode forward of ft_moe_layer_forward for callers that cannot
+ * allocate device memory: processes whose device memory belongs entirely to
+ * another allocator, and latency-critical paths that cannot afford the device
+ * synchronisation cudaMalloc / cudaFree may bring.  The write-ups describe no
+ * counterpart; this is a library convenience.
+ *
+ * Needs no context and allocates nothing: its scratch is one static device
+ * array of FT_NOALLOC_SCRATCH_BYTES that every GPU loading the library keeps
+ * until the process exits.  The first call on a device looks up that array's
+ * device address (cudaGetSymbolAddress) with the device current; make that
+ * first call before any stream capture on the device.  All calls share the
+ * array and it keeps the last call's contents: calls whose work overlaps on
+ * the GPU (other streams, other host threads) race and corrupt each other, so
+ * order them on one stream.
+ *   shape       hidden, inter (multiples of 128), n_experts (<= 1024), top_k
+ *               (<= 16), n_shared (0 or 1), as in ft_model_desc
+ *   layer_pool  dev: the layer's (n_experts + n_shared) blobs at
+ *               ft_blob_stride(hidden, inter) each, resident on the device
+ *   x, out      dev bf16 [T][hidden], T in [0, 16]; out must not alias x
+ *   router_w / logits_override, flags   as in ft_moe_layer_forward
+ *               (FT_ACT_MXFP4 is rejected: decode path only)
+ *   status      dev int32 or NULL: device-detected errors (bits: 1 NaN/+inf
+ *               logit, 2 bad id) are OR-ed into it; the caller clears it.
+ *               With NULL they are dropped.
+ * Errors: FT_ERR_INVALID for bad arguments or when the call's scratch
+ * (routing arrays plus (T*top_k + n_shared*T) * inter * 4 bytes of
+ * activations) exceeds FT_NOALLOC_SCRATCH_BYTES; FT_ERR_CUDA. */
+FT_API ft_status ft_moe_layer_forward_noalloc(int32_t hidden, int32_t inter, int32_t n_experts, int32_t top_k,
+                                              int32_t n_shared, const void* layer_pool, const void* x, int64_t T,
+                                              const float* router_w, const float* logits_override, void* out,
+                                              uint32_t flags, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
