@@ -196,15 +196,11 @@ def run_ours(args, world, rank):
     uniq = np.array([[len(np.unique(sets[p, layer])) for layer in range(L)] for p in range(TRACE_LEN)])
     bytes_pos = (uniq + S_SHARED).sum(axis=1) * used                 # [P]
     stream = torch.cuda.Stream()
+    out_buf = torch.empty_like(x0)
 
     def one_pass(src):
-        cur = src
-        for layer in range(L):
-            out = bufs[layer % 2]
-            ft.ft_moe_layer_forward(ctx, layer, cur, T, None, logits_buf[layer], out, ft.FT_ROUTE_RENORM,
-                                    stream.cuda_stream)
-            cur = out
-        return cur
+        ft.ft_moe_stack_forward(ctx, 0, L, src, T, logits_buf, out_buf, ft.FT_ROUTE_RENORM, stream.cuda_stream)
+        return out_buf
 
     with torch.cuda.stream(stream):
         logits_buf.copy_(logits_all[0])
@@ -214,7 +210,7 @@ def run_ours(args, world, rank):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             final = one_pass(x0)
-    launches_per_step = L * 4
+    launches_per_step = L * 2
 
     def step(p):
         logits_buf.copy_(logits_all[p % TRACE_LEN], non_blocking=True)
@@ -243,14 +239,20 @@ def run_ours(args, world, rank):
     res = dict(ms=ms_max, tok_s=world * T * args.steps / (ms_max / 1e3), hbm_gbs=step_bytes * args.steps / (ms / 1e3) / 1e9,
                step_bytes=step_bytes, launches=launches_per_step * args.steps, clocks=clk.summary())
 
-    # per-kernel device time over the same positions, eager launches bracketed by events
+    # per-kernel device time over the same positions: a graph of the same pass
+    # with every kernel bracketed by events, replayed and read step by step
     ft.ft_kernel_timing_enable(ctx, True)
     nk = min(args.steps, 200)
     with torch.cuda.stream(stream):
+        gt = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gt, stream=stream):
+            one_pass(x0)
+        stream.synchronize()
         for s in range(nk):
             logits_buf.copy_(logits_all[positions[s]], non_blocking=True)
-            one_pass(x0)
-    kt = ft.ft_kernel_timing_read(ctx)
+            gt.replay()
+            kt = ft.ft_kernel_timing_read(ctx)
+    del gt
     ft.ft_kernel_timing_enable(ctx, False)
     pos = positions[:nk]
     gu_launch_bytes = float(np.mean([(uniq[p] + S_SHARED).mean() for p in pos])) * gu_bytes

@@ -28,7 +28,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_router_logits", "ft_moe_route", "ft_moe_permute", "ft_quantize_mxfp4", "ft_moe_layer_forward",
            "ft_expert_cache_lookup", "ft_expert_cache_insert", "ft_expert_cache_resize", "ft_cache_trace",
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
-           "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc")
+           "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine")
@@ -96,6 +96,8 @@ def lib() -> C.CDLL:
         "ft_kernel_timing_enable": (ST, [P, I32]),
         "ft_kernel_timing_read": (ST, [P, C.POINTER(C.c_double), C.POINTER(I64), I32]),
         "ft_moe_layer_forward_noalloc": (ST, [I32, I32, I32, I32, I32, P, P, I64, P, P, P, U32, P, P]),
+        "ft_moe_stack_forward": (ST, [P, I32, I32, P, I64, P, P, U32, P]),
+        "ft_last_routing": (ST, [P, P, P, I64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -188,6 +190,15 @@ def ft_quantize_mxfp4(ctx, x, R, K, codes, scales, stream=None) -> None:
 def ft_moe_layer_forward(ctx, layer, x, T, router_w, logits_override, out, flags, stream=None) -> None:
     _check(lib().ft_moe_layer_forward(ctx, layer, _ptr(x), T, _ptr(router_w), _ptr(logits_override), _ptr(out),
                                       flags, _stream(stream)))
+
+
+def ft_moe_stack_forward(ctx, first_layer, n_layers, x, T, logits, out, flags, stream=None) -> None:
+    _check(lib().ft_moe_stack_forward(ctx, first_layer, n_layers, _ptr(x), T, _ptr(logits), _ptr(out), flags,
+                                      _stream(stream)))
+
+
+def ft_last_routing(ctx, ids, w, n, stream=None) -> None:
+    _check(lib().ft_last_routing(ctx, _ptr(ids), _ptr(w), n, _stream(stream)))
 
 
 def ft_expert_cache_lookup(ctx, layer, expert) -> int:

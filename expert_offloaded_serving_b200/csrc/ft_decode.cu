@@ -1,0 +1,623 @@
+// Decode path for small batches (T <= 16): fused routing + split-K FP4 GEMV.
+//
+//   k_dec_gate_up   every CTA routes the T tokens itself (softmax top-k +
+//                   permutation, a few hundred pairs at most), takes one unit
+//                   (a distinct selected expert, or the shared expert), one
+//                   128-row block of Wg/Wu and one K-slice, stages that tile in
+//                   shared memory with bulk async copies (cp.async.bulk + an
+//                   mbarrier), dequantises e2m1 codes with their UE8M0 scales in
+//                   registers, and reduces the K-slices of a row block across
+//                   the CTAs of a thread-block cluster through distributed
+//                   shared memory; the owner CTA applies SwiGLU and writes fp32 h.
+//   k_dec_down      same routing; one unit, one 128-row block of Wd, one
+//                   K-slice of I; launched as a programmatic dependent of the
+//                   gate/up kernel so its weight tile streams in while gate/up
+//                   still runs; after griddepcontrol.wait it reads h, reduces
+//                   its K-slices in the cluster and writes y.  The last CTA to
+//                   finish a row block (an atomic counter per row block) sums
+//                   w[t][j] * y over j ascending plus the shared expert and
+//                   rounds once to bf16.
+//
+// Pages: decode fetches or reuses the selected experts and sums their partial
+// results exactly (jansverre.net, "Hvorfor er båndbredden viktigere enn antall
+// kjerner?"); a gate picks a few experts per token (aiforradalom.hu, "A
+// Mixture-of-Experts (MoE) kihívásai és a FreeToken megoldásai").
+#include "ft_common.cuh"
+#include "ft_decode.h"
+
+namespace ft {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRows = 128;        // rows per CTA tile (one scale-atom row block)
+constexpr int kMaxPairs = 256;    // T * k
+constexpr int kMaxUnits = 257;
+constexpr uint32_t kSpinLimit = 1u << 26;
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+  asm volatile("fence.mbarrier_init.release.cluster;" ::);
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Bounded wait on phase `parity`; returns false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t addr = smem_u32(bar);
+  for (uint32_t it = 0; it < kSpinLimit; it++) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(const float* local_addr, uint32_t rank, float v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local_addr)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// routing inside a CTA
+// ---------------------------------------------------------------------------
+struct Route {
+  int32_t ids[kMaxPairs];    // [t*k + j], rank order
+  float w[kMaxPairs];
+  int32_t pos[kMaxPairs];    // permuted position of pair f (= inv)
+  int32_t perm[kMaxPairs];   // pair at permuted position
+  int32_t unit_e[kMaxUnits];
+  int32_t unit_p0[kMaxUnits];
+  int32_t unit_m[kMaxUnits];
+  uint8_t first[kMaxPairs];  // pair is its expert's lowest-token pair
+  int32_t n_active;
+  int32_t bad;
+};
+
+// Order key of a logit: larger key = ranks first.  NaN -> 1 (below -inf),
+// -0 -> +0, absent -> 0.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  uint32_t b = __float_as_uint(v);
+  if (isnan(v)) return 1u;
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Warp w routes tokens w, w+8, ...; then every thread finds the permuted
+// position of its pair; finally units (distinct experts, ascending) are listed.
+__device__ void route_in_cta(const float* __restrict__ logits, int T, int E, int k, int renorm, Route& r,
+                             int* status) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) r.bad = 0;
+  __syncthreads();
+  const int per = (E + 31) >> 5;
+  for (int t = warp; t < T; t += kThreads / 32) {
+    const float* row = logits + (size_t)t * E;
+    uint32_t key[32];
+    bool bad = false;
+    float vmax = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 32; q++) {
+      key[q] = 0u;
+      if (q < per) {
+        int e = lane + 32 * q;
+        if (e < E) {
+          float v = __ldg(row + e);
+          key[q] = order_key(v);
+          if (isnan(v) || v == INFINITY) bad = true;
+          if (!isnan(v)) vmax = fmaxf(vmax, v);
+        }
+      }
+    }
+    for (int d = 16; d >= 1; d >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, d));
+    if (vmax == -INFINITY) bad = true;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) r.bad = 1;
+    float my_v = 0.f;
+    int my_id = -1;
+    for (int j = 0; j < k; j++) {
+      // lane-local best: largest key, lowest id (ids ascend with q)
+      uint32_t bk = 0u;
+      int bq = -1;
+#pragma unroll
+      for (int q = 0; q < 32; q++)
+        if (key[q] > bk) {
+          bk = key[q];
+          bq = q;
+        }
+      uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+      uint32_t cand = (bk == kmax && bq >= 0) ? (uint32_t)(lane + 32 * bq) : 0xffffffffu;
+      uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+      if ((int)(win & 31) == lane) {
+#pragma unroll
+        for (int q = 0; q < 32; q++)
+          if (q == (int)(win >> 5)) key[q] = 0u;
+      }
+      if (lane == j) {
+        my_id = (int)win;
+        my_v = win < (uint32_t)E ? __ldg(row + win) : -INFINITY;
+      }
+    }
+    // weights: softmax at the chosen ids (renormalised over k, or over all E)
+    float m = __shfl_sync(0xffffffffu, my_v, 0);
+    float ex = (lane < k) ? expf(my_v - m) : 0.f;
+    float denom;
+    if (renorm) {
+      denom = ex;
+      for (int d = 16; d >= 1; d >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, d);
+    } else {
+      float part = 0.f;
+      for (int q = 0; q < per; q++) {
+        int e = lane + 32 * q;
+        if (e < E) part += expf(__ldg(row + e) - m);
+      }
+      for (int d = 16; d >= 1; d >>= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
+      denom = part;
+    }
+    if (lane < k) {
+      r.ids[t * k + lane] = my_id;
+      r.w[t * k + lane] = ex / denom;
+    }
+  }
+  __syncthreads();
+  const int P = T * k;
+  // permuted position of pair f: pairs of lower experts, then same expert at
+  // lower tokens; `first` marks the lowest-token pair of each expert
+  for (int f = threadIdx.x; f < P; f += kThreads) {
+    int e = r.ids[f], t = f / k;
+    int pos = 0;
+    bool first = true;
+    for (int f2 = 0; f2 < P; f2++) {
+      int e2 = r.ids[f2], t2 = f2 / k;
+      pos += (e2 < e) || (e2 == e && t2 < t);
+      if (e2 == e && t2 < t) first = false;
+    }
+    r.pos[f] = pos;
+    r.perm[pos] = f;
+    r.first[f] = first ? 1 : 0;
+  }
+  __syncthreads();
+  // units = distinct experts in ascending order
+  for (int f = threadIdx.x; f < P; f += kThreads) {
+    if (!r.first[f]) continue;
+    int e = r.ids[f];
+    int unit = 0, cnt = 0;
+    for (int f2 = 0; f2 < P; f2++) {
+      int e2 = r.ids[f2];
+      unit += (r.first[f2] && e2 < e);
+      cnt += (e2 == e);
+    }
+    r.unit_e[unit] = e;
+    r.unit_p0[unit] = r.pos[f];
+    r.unit_m[unit] = cnt;
+  }
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int f = 0; f < P; f++) n += r.first[f];
+    r.n_active = n;
+    if (r.bad) set_status(status, kStNonfinite);
+  }
+  __syncthreads();
+}
+
+struct UnitInfo {
+  int e, m, hbase;
+  bool shared;
+};
+
+__device__ __forceinline__ bool resolve_unit(const DecodeArgs& a, const Route& r, int u, UnitInfo& ui) {
+  if (u < a.max_units) {
+    if (u >= r.n_active) return false;
+    ui.e = r.unit_e[u];
+    ui.m = r.unit_m[u];
+    ui.hbase = r.unit_p0[u];
+    ui.shared = false;
+  } else {
+    int s = u - a.max_units;
+    ui.e = a.E + s;
+    ui.m = a.T;
+    ui.hbase = a.T * a.k + s * a.T;
+    ui.shared = true;
+  }
+  return true;
+}
+
+__device__ __forceinline__ int unit_token(const DecodeArgs& a, const Route& r, const UnitInfo& ui, int i) {
+  return ui.shared ? i : r.perm[ui.hbase + i] / a.k;
+}
+
+// Dot of 32 e2m1 codes (16 bytes) with 32 activations (16 float pairs).
+__device__ __forceinline__ float chunk_dot(uint4 q, const float2* xv) {
+  float2 acc = make_float2(0.f, 0.f);
+  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int wv = 0; wv < 4; wv++)
+#pragma unroll
+    for (int b = 0; b < 4; b++) acc = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> (8 * b))), xv[wv * 4 + b], acc);
+  return acc.x + acc.y;
+}
+
+// Scale byte of row r (0..127), block b of a staged scale tile (atoms along K).
+__device__ __forceinline__ uint32_t tile_scale(const uint8_t* sc, int r, int b) {
+  return sc[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)];
+}
+
+// Issue the bulk copies of one 128-row tile: codes rows [row0, row0+128),
+// bytes [kbyte0, kbyte0 + kbytes) of each row (row pitch `pitch`), and the
+// scale atoms of that row block for blocks [kblk0, kblk0 + kbytes/16).
+// Called by warp 0; returns the bytes issued.
+__device__ __forceinline__ uint32_t issue_tile(uint8_t* codes_s, uint8_t* sc_s, const uint8_t* codes_g,
+                                               const uint8_t* sc_g, int row0, int pitch, int kbyte0, int kbytes,
+                                               int atoms_k, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  for (int r = lane; r < kRows; r += 32)
+    bulk_g2s(codes_s + r * kbytes, codes_g + (size_t)(row0 + r) * pitch + kbyte0, (uint32_t)kbytes, bar);
+  const int atoms = kbytes / 64;                // 128 elements (64 bytes) per atom column
+  const int atom0 = kbyte0 / 64;
+  if (lane == 0)
+    bulk_g2s(sc_s, sc_g + ((size_t)(row0 >> 7) * atoms_k + atom0) * 512, (uint32_t)(atoms * 512), bar);
+  return (uint32_t)(kRows * kbytes + atoms * 512);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory plan of a CTA (dynamic smem)
+// ---------------------------------------------------------------------------
+struct Plan {
+  int ks, lpr, cpl;   // K-slice (elements), lanes per row, chunks per lane
+  int nmat;           // 2 (gate/up) or 1 (down)
+  size_t codes, scales, act, part, recv, total;
+};
+
+__host__ __device__ inline Plan make_plan(int ks, int nmat, int T) {
+  Plan p;
+  p.ks = ks;
+  int chunks = ks / 32;
+  p.lpr = 16;
+  while (p.lpr > 1 && chunks % p.lpr) p.lpr >>= 1;
+  p.cpl = chunks / p.lpr;
+  p.nmat = nmat;
+  size_t off = sizeof(Route) + 64;
+  off = (off + 127) / 128 * 128;
+  p.codes = off;
+  off += (size_t)nmat * kRows * ks / 2;
+  p.scales = off;
+  off += (size_t)nmat * kRows * ks / 32;
+  p.act = off;
+  off += (size_t)T * ks * sizeof(float);
+  p.part = off;
+  off += (size_t)kRows * nmat * T * sizeof(float);
+  p.recv = off;
+  off += (size_t)kRows * nmat * T * sizeof(float);
+  p.total = off;
+  return p;
+}
+
+// Partial dot products of the staged tile rows with the staged activations:
+// part[row][mat][tok] (unreduced over K-slices).
+__device__ void tile_dots(const Plan& pl, const uint8_t* codes_s, const uint8_t* sc_s, const float* act, int m, int T,
+                          float* part) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lpr = pl.lpr, cpl = pl.cpl, rows_per_pass = (kThreads / 32) * (32 / lpr);
+  const int g = lane / lpr, sl = lane % lpr;
+  const int kbytes = pl.ks / 2;
+  constexpr int MT = 2;
+  for (int t0 = 0; t0 < m; t0 += MT) {
+    for (int c = 0; c < cpl; c++) {
+      const int chunk = sl + lpr * c;
+      float2 xv[MT][16];
+#pragma unroll
+      for (int mm = 0; mm < MT; mm++) {
+        const float4* src = reinterpret_cast<const float4*>(act + (size_t)(t0 + mm < m ? t0 + mm : t0) * pl.ks + chunk * 32);
+#pragma unroll
+        for (int v = 0; v < 8; v++) {
+          float4 f = src[v];
+          xv[mm][2 * v] = make_float2(f.x, f.y);
+          xv[mm][2 * v + 1] = make_float2(f.z, f.w);
+        }
+      }
+      for (int mat = 0; mat < pl.nmat; mat++) {
+        const uint8_t* cs = codes_s + (size_t)mat * kRows * kbytes;
+        const uint8_t* ss = sc_s + (size_t)mat * kRows * (pl.ks / 32);
+        for (int r = warp * (32 / lpr) + g; r < kRows; r += rows_per_pass) {
+          uint4 q = *reinterpret_cast<const uint4*>(cs + (size_t)r * kbytes + chunk * 16);
+          float sc = ue8m0_to_f32(tile_scale(ss, r, chunk));
+          float d0 = chunk_dot(q, xv[0]) * sc;
+          float d1 = (t0 + 1 < m) ? chunk_dot(q, xv[1]) * sc : 0.f;
+          for (int dd = lpr >> 1; dd >= 1; dd >>= 1) {
+            d0 += __shfl_xor_sync(0xffffffffu, d0, dd);
+            d1 += __shfl_xor_sync(0xffffffffu, d1, dd);
+          }
+          if (sl == 0) {
+            float* pr = part + ((size_t)r * pl.nmat + mat) * T;
+            if (c == 0) {
+              pr[t0] = d0;
+              if (t0 + 1 < m) pr[t0 + 1] = d1;
+            } else {
+              pr[t0] += d0;
+              if (t0 + 1 < m) pr[t0 + 1] += d1;
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+// Send this CTA's partials of the rows owned by cluster rank `o` to rank o's
+// receive buffer [slice][row_in_owner][mat][tok], then cluster barrier.
+__device__ void cluster_exchange(const Plan& pl, const float* part, float* recv, int S, int slice, int m, int T) {
+  const int rows_per_owner = kRows / S;
+  const int n = kRows * pl.nmat * m;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    int tok = i % m;
+    int mat = (i / m) % pl.nmat;
+    int r = i / (m * pl.nmat);
+    int owner = r / rows_per_owner;
+    int rl = r % rows_per_owner;
+    float v = part[((size_t)r * pl.nmat + mat) * T + tok];
+    const float* dst = recv + (((size_t)slice * rows_per_owner + rl) * pl.nmat + mat) * T + tok;
+    if (S == 1)
+      *const_cast<float*>(dst) = v;
+    else
+      st_cluster_f32(dst, (uint32_t)owner, v);
+  }
+  if (S > 1)
+    cluster_sync();
+  else
+    __syncthreads();
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// gate/up + SwiGLU
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  Route& r = *reinterpret_cast<Route*>(smem);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + sizeof(Route));
+  const int S = a.s_gu;
+  const Plan pl = make_plan(a.H / S, 2, a.T);
+  uint8_t* codes_s = smem + pl.codes;
+  uint8_t* sc_s = smem + pl.scales;
+  float* act = reinterpret_cast<float*>(smem + pl.act);
+  float* part = reinterpret_cast<float*>(smem + pl.part);
+  float* recv = reinterpret_cast<float*>(smem + pl.recv);
+
+  const int RB = a.I / kRows;
+  const int slice = blockIdx.x % S;
+  const int rb = (blockIdx.x / S) % RB;
+  const int u = blockIdx.x / (S * RB);
+
+  route_in_cta(a.logits, a.T, a.E, a.k, a.renorm, r, a.status);
+  if (blockIdx.x == 0 && a.ids_out) {
+    for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
+      a.ids_out[f] = r.ids[f];
+      a.w_out[f] = r.w[f];
+    }
+  }
+  UnitInfo ui;
+  if (!resolve_unit(a, r, u, ui)) {
+    pdl_trigger();
+    return;  // the whole cluster (same unit) leaves together
+  }
+  const uint8_t* blob = a.eptr[ui.e];
+  if (blob == nullptr) {
+    if (threadIdx.x == 0) set_status(a.status, kStMissing);
+    pdl_trigger();
+    return;
+  }
+  const int kbytes = pl.ks / 2, pitch = a.H / 2;
+  const int atoms_k = (int)(pad_up(a.H / 32, 4) / 4);
+  if (threadIdx.x == 0) mbar_init(bar, 1);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t bytes = 0;
+    if (threadIdx.x == 0) mbar_expect_tx(bar, 2u * (kRows * kbytes + (kbytes / 64) * 512));
+    __syncwarp();
+    bytes += issue_tile(codes_s, sc_s, blob + a.lay.wg, blob + a.lay.wg_sf, rb * kRows, pitch, slice * kbytes, kbytes,
+                        atoms_k, bar);
+    bytes += issue_tile(codes_s + kRows * kbytes, sc_s + kRows * (pl.ks / 32), blob + a.lay.wu, blob + a.lay.wu_sf,
+                        rb * kRows, pitch, slice * kbytes, kbytes, atoms_k, bar);
+    (void)bytes;
+  }
+  pdl_trigger();
+  pdl_wait();  // activations come from the previous kernel when launched as a dependent
+  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
+    int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
+    int t = unit_token(a, r, ui, mm);
+    uint2 xv = *reinterpret_cast<const uint2*>(a.x + (size_t)t * a.H + slice * pl.ks + k4 * 4);
+    reinterpret_cast<float4*>(act)[i] = make_float4(bf16_bits_to_f32(xv.x & 0xffff), bf16_bits_to_f32(xv.x >> 16),
+                                                    bf16_bits_to_f32(xv.y & 0xffff), bf16_bits_to_f32(xv.y >> 16));
+  }
+  __syncthreads();
+  if (!mbar_wait(bar, 0)) {
+    if (threadIdx.x == 0) set_status(a.status, kStTimeout);
+    mbar_wait(bar, 0);
+  }
+  tile_dots(pl, codes_s, sc_s, act, ui.m, a.T, part);
+  __syncthreads();
+  cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
+  // owner rows: sum slices in order, SwiGLU, write h
+  const int rows_per_owner = kRows / S;
+  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kThreads) {
+    int rl = i / ui.m, tok = i % ui.m;
+    float gs = 0.f, us = 0.f;
+    for (int s = 0; s < S; s++) {
+      gs += recv[(((size_t)s * rows_per_owner + rl) * 2 + 0) * a.T + tok];
+      us += recv[(((size_t)s * rows_per_owner + rl) * 2 + 1) * a.T + tok];
+    }
+    int row = rb * kRows + slice * rows_per_owner + rl;
+    a.h[(size_t)(ui.hbase + tok) * a.I + row] = silu(gs) * us;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// down + combine
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  Route& r = *reinterpret_cast<Route*>(smem);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + sizeof(Route));
+  __shared__ int last;
+  const int S = a.s_dn;
+  const Plan pl = make_plan(a.I / S, 1, a.T);
+  uint8_t* codes_s = smem + pl.codes;
+  uint8_t* sc_s = smem + pl.scales;
+  float* act = reinterpret_cast<float*>(smem + pl.act);
+  float* part = reinterpret_cast<float*>(smem + pl.part);
+  float* recv = reinterpret_cast<float*>(smem + pl.recv);
+
+  const int RB = a.H / kRows;
+  const int slice = blockIdx.x % S;
+  const int rb = (blockIdx.x / S) % RB;
+  const int u = blockIdx.x / (S * RB);
+
+  route_in_cta(a.logits, a.T, a.E, a.k, a.renorm, r, nullptr);
+  UnitInfo ui;
+  if (!resolve_unit(a, r, u, ui)) {
+    pdl_trigger();
+    return;
+  }
+  const uint8_t* blob = a.eptr[ui.e];
+  if (blob == nullptr) {
+    pdl_trigger();
+    return;  // already reported by the gate/up kernel
+  }
+  const int kbytes = pl.ks / 2, pitch = a.I / 2;
+  const int atoms_k = (int)(pad_up(a.I / 32, 4) / 4);
+  if (threadIdx.x == 0) mbar_init(bar, 1);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    if (threadIdx.x == 0) mbar_expect_tx(bar, (uint32_t)(kRows * kbytes + (kbytes / 64) * 512));
+    __syncwarp();
+    issue_tile(codes_s, sc_s, blob + a.lay.wd, blob + a.lay.wd_sf, rb * kRows, pitch, slice * kbytes, kbytes, atoms_k,
+               bar);
+  }
+  pdl_trigger();
+  pdl_wait();  // h is written by the gate/up kernel
+  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
+    int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
+    reinterpret_cast<float4*>(act)[i] =
+        *reinterpret_cast<const float4*>(a.h + (size_t)(ui.hbase + mm) * a.I + slice * pl.ks + k4 * 4);
+  }
+  __syncthreads();
+  if (!mbar_wait(bar, 0)) {
+    if (threadIdx.x == 0) set_status(a.status, kStTimeout);
+    mbar_wait(bar, 0);
+  }
+  tile_dots(pl, codes_s, sc_s, act, ui.m, a.T, part);
+  __syncthreads();
+  cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
+  const int rows_per_owner = kRows / S;
+  const int row0 = rb * kRows + slice * rows_per_owner;
+  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kThreads) {
+    int rl = i / ui.m, tok = i % ui.m;
+    float ys = 0.f;
+    for (int s = 0; s < S; s++) ys += recv[((size_t)s * rows_per_owner + rl) * a.T + tok];
+    a.y[(size_t)(ui.hbase + tok) * a.H + row0 + rl] = ys;
+  }
+  // last CTA of this row group combines
+  __threadfence();
+  __syncthreads();
+  const int units = r.n_active + a.n_shared;
+  if (threadIdx.x == 0) {
+    int* ctr = a.counters + rb * S + slice;
+    int old = atomicAdd(ctr, 1);
+    last = (old == units - 1);
+    if (last) *ctr = 0;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < a.T * rows_per_owner; i += kThreads) {
+    int t = i / rows_per_owner, rl = i % rows_per_owner;
+    int n = row0 + rl;
+    float acc = 0.f;
+    for (int j = 0; j < a.k; j++) {
+      int f = t * a.k + j;
+      acc = fmaf(r.w[f], __ldcg(a.y + (size_t)r.pos[f] * a.H + n), acc);
+    }
+    for (int s = 0; s < a.n_shared; s++) acc += __ldcg(a.y + (size_t)(a.T * a.k + s * a.T + t) * a.H + n);
+    __nv_bfloat16 b = __float2bfloat16_rn(acc);
+    a.out[(size_t)t * a.H + n] = *reinterpret_cast<uint16_t*>(&b);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+int choose_slices(int K) {
+  // largest S <= 8 with K/S a multiple of 128 and K/S >= 256 (or S = 1)
+  for (int s = 8; s >= 2; s--)
+    if (K % (s * 128) == 0 && K / s >= 256 && K / s <= 1024) return s;
+  return 1;
+}
+
+size_t decode_smem_bytes(int K, int S, int nmat, int T) { return make_plan(K / S, nmat, T).total; }
+
+static void set_attrs() {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_dec_gate_up, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+    cudaFuncSetAttribute(k_dec_down, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+    attr = true;
+  }
+}
+
+static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, int grid, int cluster, size_t smem,
+                              bool pdl, cudaStream_t s) {
+  set_attrs();
+  cudaLaunchAttribute at[2];
+  cudaLaunchConfig_t cfg{};
+  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = dim3(grid);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cluster;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
+  const int U = a.max_units + a.n_shared;
+  return launch_one(k_dec_gate_up, a, U * (a.I / kRows) * a.s_gu, a.s_gu, decode_smem_bytes(a.H, a.s_gu, 2, a.T), pdl,
+                    s);
+}
+
+cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
+  const int U = a.max_units + a.n_shared;
+  return launch_one(k_dec_down, a, U * (a.H / kRows) * a.s_dn, a.s_dn, decode_smem_bytes(a.I, a.s_dn, 1, a.T), pdl,
+                    s);
+}
+
+}  // namespace ft

@@ -25,6 +25,7 @@
 #include <vector>
 
 #include "ft_common.cuh"
+#include "ft_decode.h"
 #include "ft_kernels.h"
 #include "ft_runtime.h"
 
@@ -154,7 +155,11 @@ struct ft_ctx {
   int32_t* d_nact = nullptr;
   int32_t* d_pad_offs = nullptr;
   float* d_h = nullptr;
+  float* d_y = nullptr;        // decode y [(T*k + S*T)][H]
+  int* d_counters = nullptr;   // decode combine counters [(H/128) * 8]
+  uint16_t* d_xbuf[2] = {nullptr, nullptr};  // stack forward ping-pong [T][H]
   int decode_max_t = 0;
+  int s_gu = 1, s_dn = 1;
 
   // pinned host scratch
   int32_t* h_ids = nullptr;
@@ -192,7 +197,8 @@ struct ft_ctx {
 
   // per-kernel timing
   bool timing = false;
-  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> tmarks;  // (class, (start, stop))
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> tmarks;  // eager (class, (start, stop))
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> gmarks;  // recorded inside stream capture
   double tms[FT_K_COUNT] = {0};
   int64_t tlaunch[FT_K_COUNT] = {0};
 };
@@ -203,10 +209,12 @@ struct KTimer {
   int cls;
   cudaStream_t s;
   cudaEvent_t a = nullptr, b = nullptr;
+  bool captured = false;
   KTimer(ft_ctx* c_, int cls_, cudaStream_t s_) : c(c_), cls(cls_), s(s_) {
     if (!c->timing) return;
     cudaStreamCaptureStatus cs;
-    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return;
+    captured = cs != cudaStreamCaptureStatusNone;
     cudaEventCreate(&a);
     cudaEventCreate(&b);
     cudaEventRecord(a, s);
@@ -214,7 +222,7 @@ struct KTimer {
   ~KTimer() {
     if (!a) return;
     cudaEventRecord(b, s);
-    c->tmarks.push_back({cls, {a, b}});
+    (captured ? c->gmarks : c->tmarks).push_back({cls, {a, b}});
   }
 };
 
@@ -344,8 +352,16 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
       (st = dev_alloc(&c->d_offs, E + 1)) || (st = dev_alloc(&c->d_perm, (size_t)T * k)) ||
       (st = dev_alloc(&c->d_inv, (size_t)T * k)) || (st = dev_alloc(&c->d_active, E)) ||
       (st = dev_alloc(&c->d_nact, 1)) || (st = dev_alloc(&c->d_pad_offs, E + 1)) ||
-      (st = dev_alloc(&c->d_h, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * I)))
+      (st = dev_alloc(&c->d_h, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * I)) ||
+      (st = dev_alloc(&c->d_y, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * H)) ||
+      (st = dev_alloc(&c->d_counters, (size_t)(H / 128) * 8)) ||
+      (st = dev_alloc(&c->d_xbuf[0], (size_t)c->decode_max_t * H)) ||
+      (st = dev_alloc(&c->d_xbuf[1], (size_t)c->decode_max_t * H)))
     return bail(st);
+  if (cudaMemset(c->d_counters, 0, (size_t)(H / 128) * 8 * sizeof(int)) != cudaSuccess)
+    return bail(fail(FT_ERR_CUDA, "memset"));
+  c->s_gu = choose_slices(H);
+  c->s_dn = choose_slices(I);
   if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return bail(fail(FT_ERR_CUDA, "memset"));
   if (cudaMallocHost(&c->h_ids, (size_t)T * k * sizeof(int32_t)) != cudaSuccess ||
       cudaMallocHost(&c->h_status, sizeof(int)) != cudaSuccess)
@@ -428,10 +444,11 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
 extern "C" ft_status ft_destroy(ft_ctx* c) {
   if (!c) return FT_OK;
   cudaDeviceSynchronize();
-  for (auto& m : c->tmarks) {
-    cudaEventDestroy(m.second.first);
-    cudaEventDestroy(m.second.second);
-  }
+  for (auto* v : {&c->tmarks, &c->gmarks})
+    for (auto& m : *v) {
+      cudaEventDestroy(m.second.first);
+      cudaEventDestroy(m.second.second);
+    }
   for (auto& pr : c->copy_timing) {
     cudaEventDestroy(pr.first);
     cudaEventDestroy(pr.second);
@@ -448,6 +465,10 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   cudaFree(c->d_nact);
   cudaFree(c->d_pad_offs);
   cudaFree(c->d_h);
+  cudaFree(c->d_y);
+  cudaFree(c->d_counters);
+  cudaFree(c->d_xbuf[0]);
+  cudaFree(c->d_xbuf[1]);
   cudaFree(c->d_eptr_res);
   cudaFree(c->d_eptr_cache);
   cudaFree(c->d_shared);
@@ -808,6 +829,32 @@ extern "C" ft_status ft_prefetch_layer(ft_ctx* c, int32_t layer, void* compute_s
 // ---------------------------------------------------------------------------
 // layer forward
 // ---------------------------------------------------------------------------
+static DecodeArgs decode_args(ft_ctx* c, const uint16_t* x, const float* logits, int T, uint32_t flags,
+                              const uint8_t* const* eptr, uint16_t* out) {
+  DecodeArgs a{};
+  a.x = x;
+  a.logits = logits;
+  a.T = T;
+  a.H = c->d.hidden;
+  a.I = c->d.inter;
+  a.E = c->d.n_experts;
+  a.k = c->d.top_k;
+  a.n_shared = c->d.n_shared;
+  a.renorm = (flags & FT_ROUTE_RENORM) ? 1 : 0;
+  a.max_units = std::min(a.E, T * a.k);
+  a.s_gu = c->s_gu;
+  a.s_dn = c->s_dn;
+  a.eptr = eptr;
+  a.lay = c->lay;
+  a.h = c->d_h;
+  a.y = c->d_y;
+  a.out = out;
+  a.ids_out = c->d_ids;
+  a.w_out = c->d_w;
+  a.counters = c->d_counters;
+  a.status = c->d_status;
+  return a;
+}
 extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* x, int64_t T,
                                           const float* router_w, const float* logits_override, void* out,
                                           uint32_t flags, void* stream) {
@@ -823,21 +870,24 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   cudaStream_t s = (cudaStream_t)stream;
   const int H = c->d.hidden, E = c->d.n_experts, k = c->d.top_k, Ti = (int)T;
 
-  // 1-3: logits, top-k, permutation
+  // 1-3: logits, then routing.  The decode kernels route inside every CTA;
+  // the separate top-k / permutation kernels run for prefill, and top-k alone
+  // for the cache path, whose host LRU needs the ids first.
   const float* logits = logits_override;
   if (!logits) {
     KTimer kt(c, FT_K_ROUTER_LOGITS, s);
     CUDA_TRY(launch_router_logits((const uint16_t*)x, router_w, Ti, H, E, c->d_logits, s));
     logits = c->d_logits;
   }
-  {
+  const bool cache_path = !mx && !c->resident[layer];
+  if (mx || cache_path) {
     KTimer kt(c, FT_K_TOPK, s);
     CUDA_TRY(launch_topk(logits, Ti, E, k, (flags & FT_ROUTE_RENORM) ? 1 : 0, c->d_ids, c->d_w, c->d_status, s));
   }
-  {
+  if (mx) {
     KTimer kt(c, FT_K_PERMUTE, s);
     CUDA_TRY(launch_permute(c->d_ids, Ti * k, E, c->d_offs, c->d_perm, c->d_inv, c->d_active, c->d_nact,
-                            mx ? c->d_pad_offs : nullptr, c->d_status, s));
+                            c->d_pad_offs, c->d_status, s));
   }
 
   // 4: weight source.  Prefill (MXFP4) reads resident or staged layers and
@@ -879,33 +929,14 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
 
   // 5: experts and combine
   if (!mx) {
-    GemvParams p{};
-    p.x = (const uint16_t*)x;
-    p.T = Ti;
-    p.H = H;
-    p.I = c->d.inter;
-    p.E = E;
-    p.k = k;
-    p.n_shared = c->d.n_shared;
-    p.max_active = std::min(E, Ti * k);
-    p.offs = c->d_offs;
-    p.perm = c->d_perm;
-    p.inv = c->d_inv;
-    p.w = c->d_w;
-    p.active = c->d_active;
-    p.n_active = c->d_nact;
-    p.eptr = eptr;
-    p.lay = c->lay;
-    p.h = c->d_h;
-    p.out = (uint16_t*)out;
-    p.status = c->d_status;
+    DecodeArgs a = decode_args(c, (const uint16_t*)x, logits, Ti, flags, eptr, (uint16_t*)out);
     {
       KTimer kt(c, FT_K_GATE_UP, s);
-      CUDA_TRY(launch_gate_up(p, s));
+      CUDA_TRY(launch_dec_gate_up(a, false, s));
     }
     {
       KTimer kt(c, FT_K_DOWN_COMBINE, s);
-      CUDA_TRY(launch_down_combine(p, s));
+      CUDA_TRY(launch_dec_down(a, true, s));
     }
   } else {
     FT_TRY(ensure_prefill_scratch(c->pf, c->d, c->max_tokens));
@@ -938,18 +969,24 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
 // ---------------------------------------------------------------------------
 // per-kernel timing
 // ---------------------------------------------------------------------------
-static void drop_marks(ft_ctx* c) {
+static void drop_marks(ft_ctx* c, bool graph_too) {
   for (auto& m : c->tmarks) {
     cudaEventDestroy(m.second.first);
     cudaEventDestroy(m.second.second);
   }
   c->tmarks.clear();
+  if (!graph_too) return;
+  for (auto& m : c->gmarks) {
+    cudaEventDestroy(m.second.first);
+    cudaEventDestroy(m.second.second);
+  }
+  c->gmarks.clear();
 }
 
 extern "C" ft_status ft_kernel_timing_enable(ft_ctx* c, int32_t on) {
   if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
   CUDA_TRY(cudaDeviceSynchronize());
-  drop_marks(c);
+  drop_marks(c, true);
   for (int i = 0; i < FT_K_COUNT; i++) {
     c->tms[i] = 0;
     c->tlaunch[i] = 0;
@@ -961,16 +998,67 @@ extern "C" ft_status ft_kernel_timing_enable(ft_ctx* c, int32_t on) {
 extern "C" ft_status ft_kernel_timing_read(ft_ctx* c, double* ms, int64_t* launches, int32_t n) {
   if (!c || !ms || !launches || n < 0) return fail(FT_ERR_INVALID, "bad argument");
   CUDA_TRY(cudaDeviceSynchronize());
-  for (auto& m : c->tmarks) {
-    float t = 0.f;
-    CUDA_TRY(cudaEventElapsedTime(&t, m.second.first, m.second.second));
-    c->tms[m.first] += t;
-    c->tlaunch[m.first] += 1;
-  }
-  drop_marks(c);
+  for (auto* v : {&c->tmarks, &c->gmarks})
+    for (auto& m : *v) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, m.second.first, m.second.second) != cudaSuccess) {
+        cudaGetLastError();  // a captured mark whose graph has not run yet
+        continue;
+      }
+      c->tms[m.first] += t;
+      c->tlaunch[m.first] += 1;
+    }
+  drop_marks(c, false);
   for (int i = 0; i < n && i < FT_K_COUNT; i++) {
     ms[i] = c->tms[i];
     launches[i] = c->tlaunch[i];
   }
+  return FT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// stacked decode over consecutive resident layers
+// ---------------------------------------------------------------------------
+extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_t n_layers, const void* x, int64_t T,
+                                          const float* logits, void* out, uint32_t flags, void* stream) {
+  if (!c || !x || !out || !logits) return fail(FT_ERR_INVALID, "NULL argument");
+  if (n_layers <= 0 || first_layer < 0 || first_layer + n_layers > c->d.n_layers)
+    return fail(FT_ERR_INVALID, "layers [%d, %d) outside [0, %d)", first_layer, first_layer + n_layers, c->d.n_layers);
+  if (T < 0 || T > c->decode_max_t) return fail(FT_ERR_INVALID, "T=%lld outside [0, %d]", (long long)T, c->decode_max_t);
+  if (flags & FT_ACT_MXFP4) return fail(FT_ERR_INVALID, "the stacked forward is the decode path (FT_ACT_BF16)");
+  if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
+  for (int l = first_layer; l < first_layer + n_layers; l++)
+    if (!c->resident[l]) return fail(FT_ERR_STATE, "layer %d is not resident", l);
+  if (T == 0) return FT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int Ti = (int)T, E = c->d.n_experts;
+  const uint16_t* cur = (const uint16_t*)x;
+  for (int i = 0; i < n_layers; i++) {
+    const int l = first_layer + i;
+    uint16_t* dst = (i == n_layers - 1) ? (uint16_t*)out : c->d_xbuf[i & 1];
+    DecodeArgs a = decode_args(c, cur, logits + (size_t)i * Ti * E, Ti, flags, c->d_eptr_res + (size_t)l * c->n_blobs,
+                               dst);
+    // layers after the first start their routing and weight streaming while
+    // the previous layer finishes: their logits and pointer tables are inputs
+    // of this call, complete before its first kernel
+    {
+      KTimer kt(c, FT_K_GATE_UP, s);
+      CUDA_TRY(launch_dec_gate_up(a, i > 0 && !c->timing, s));
+    }
+    {
+      KTimer kt(c, FT_K_DOWN_COMBINE, s);
+      CUDA_TRY(launch_dec_down(a, true, s));
+    }
+    cur = dst;
+  }
+  c->last_stream = s;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_last_routing(ft_ctx* c, int32_t* ids, float* w, int64_t n, void* stream) {
+  if (!c || !ids || !w) return fail(FT_ERR_INVALID, "NULL argument");
+  if (n < 0 || n > (int64_t)c->max_tokens * c->d.top_k) return fail(FT_ERR_INVALID, "n out of range");
+  CUDA_TRY(cudaMemcpyAsync(ids, c->d_ids, (size_t)n * sizeof(int32_t), cudaMemcpyDefault, (cudaStream_t)stream));
+  CUDA_TRY(cudaMemcpyAsync(w, c->d_w, (size_t)n * sizeof(float), cudaMemcpyDefault, (cudaStream_t)stream));
   return FT_OK;
 }

@@ -219,6 +219,24 @@ FT_API ft_status ft_moe_layer_forward(ft_ctx* ctx, int32_t layer, const void* x,
                                const float* router_w, const float* logits_override,
                                void* out, uint32_t flags, void* stream);
 
+/* Decode of T tokens (T <= 16) through n_layers consecutive layers, all with
+ * resident pools: layer i's output is layer i+1's input.
+ *   x dev bf16 [T][H] (input of first_layer), out dev bf16 [T][H] (output of
+ *   the last layer; must not alias x); logits dev fp32 [n_layers][T][E]
+ *   (router logits of each layer, all ready before the call).
+ * Each layer is the ft_moe_layer_forward decode path.  Because every layer's
+ * routing input is known up front, a layer's kernels are launched as
+ * programmatic dependents of the previous layer's, so its routing and weight
+ * streaming overlap the previous layer's tail; intermediate activations live
+ * in context scratch.  flags: FT_ROUTE_RENORM.
+ * Errors: FT_ERR_INVALID, FT_ERR_STATE (a layer is not resident), FT_ERR_CUDA. */
+FT_API ft_status ft_moe_stack_forward(ft_ctx* ctx, int32_t first_layer, int32_t n_layers, const void* x, int64_t T,
+                                      const float* logits, void* out, uint32_t flags, void* stream);
+
+/* Copy the ids [T][k] and weights [T][k] of the last decode or prefill
+ * routing (n = T*k entries) to ids / w (device or host memory), on `stream`. */
+FT_API ft_status ft_last_routing(ft_ctx* ctx, int32_t* ids, float* w, int64_t n, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* expert cache ([no] global LRU; [fa] elastic resize)                     */
 /* ---------------------------------------------------------------------- */
@@ -289,13 +307,15 @@ FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, fl
 #define FT_K_COUNT         9
 
 /* Turn per-kernel CUDA-event timing on (1) or off (0).  While on, every
- * kernel launch of the forward path is bracketed by events on its stream;
- * launches inside stream capture are not timed.  Turning it on resets the
- * counters. */
+ * kernel launch of the forward path is bracketed by events on its stream (and
+ * consecutive layers are not overlapped).  Launches made under stream capture
+ * record their events into the graph: each ft_kernel_timing_read after a
+ * replay adds that replay's times.  Enabling or disabling resets the counters
+ * and releases the events, so destroy graphs that hold them first. */
 FT_API ft_status ft_kernel_timing_enable(ft_ctx* ctx, int32_t on);
 
 /* Synchronise, then fill ms[i] (total device time) and launches[i] for the
- * first n kernel classes (FT_K_*) since timing was enabled. */
+ * first n kernel classes (FT_K_*) accumulated since timing was enabled. */
 FT_API ft_status ft_kernel_timing_read(ft_ctx* ctx, double* ms, int64_t* launches, int32_t n);
 
 /* ---------------------------------------------------------------------- */

@@ -35,7 +35,11 @@ def run_layer(H, I, E, k, S, T, seed, use_router, renorm=True, trace=True, max_t
                                 (ft.FT_ROUTE_RENORM if renorm else 0) | ft.FT_ACT_BF16)
         ft.ft_sync_status(c.h)
         got = bf16_bits(out)
-    want_ids_needed = None
+        ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T * k, dtype=torch.float32, device="cuda")
+        ft.ft_last_routing(c.h, ids, w, T * k)
+        torch.cuda.synchronize()
+        got_ids, got_w = ids.cpu().numpy().reshape(T, k), w.cpu().numpy().reshape(T, k)
     blobs = {}
 
     def blob_of(e):
@@ -44,6 +48,8 @@ def run_layer(H, I, E, k, S, T, seed, use_router, renorm=True, trace=True, max_t
         return blobs[e]
     r = olayer.moe_layer(xb, blob_of, H, I, E, k, logits=lg, router_w=wr, renorm=renorm,
                          shared_blob=blob_of(E) if S else None)
+    assert (got_ids == r["ids"]).all()
+    assert np.allclose(got_w, r["w"], rtol=2e-6, atol=1e-9)
     return got, r
 
 
@@ -100,3 +106,62 @@ def test_zero_tokens_and_limits():
             ft.ft_moe_layer_forward(c.h, 1, x, 1, None, lg, out, 1)  # no such layer
         with pytest.raises(ft.FtError):
             ft.ft_moe_layer_forward(c.h, 0, x, 1, None, lg, x, 1)    # out aliases x
+
+
+def test_fused_routing_ties_and_no_renorm():
+    """Exact ties in the logits resolve to the lower id inside the fused kernels."""
+    H, I, E, k, T, seed = 2048, 512, 256, 8, 4, 77
+    pool = synth.gpu.layer_pool(H, I, E, seed, 0)
+    lg = np.random.default_rng(1).standard_normal((T, E)).astype(np.float32)
+    lg[:, 10:30] = 2.5                  # 20 tied experts above the rest
+    lg[1, :] = 0.0                      # a fully tied row
+    lg[2, 7] = -0.0
+    xb = synth.activations_bf16(seed, 1, T, H)
+    with Ctx(ft.make_desc(H, I, E, k, 1, 0, 0, 16), None, [pool]) as c:
+        x = x_dev(xb)
+        out = torch.empty_like(x)
+        for renorm in (1, 0):
+            ft.ft_moe_layer_forward(c.h, 0, x, T, None, torch.from_numpy(lg).cuda(), out, renorm)
+            ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
+            w = torch.empty(T * k, dtype=torch.float32, device="cuda")
+            ft.ft_last_routing(c.h, ids, w, T * k)
+            torch.cuda.synchronize()
+            want, _ = olayer.routing.topk(lg, k)
+            assert (ids.cpu().numpy().reshape(T, k) == want).all()
+            ww = olayer.routing.softmax_weights(lg, want, bool(renorm))
+            assert np.allclose(w.cpu().numpy().reshape(T, k), ww, rtol=2e-6, atol=1e-9)
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_stack_forward_matches_layer_by_layer(T):
+    H, I, E, k, S, L, seed = 2048, 512, 256, 8, 1, 3, 1002
+    pools = [synth.gpu.layer_pool(H, I, E + S, seed, l) for l in range(L)]
+    lgs = []
+    for l in range(L):
+        sets = np.stack([synth.zipf_trace(seed, l, 3, E, k, 1.1, 0.6, stream=t)[-1] for t in range(T)])
+        lgs.append(synth.logits_for_sets(seed, 10 + l, sets, E))
+    lg_all = torch.from_numpy(np.stack(lgs)).cuda()
+    xb = synth.activations_bf16(seed, 1, T, H)
+    with Ctx(ft.make_desc(H, I, E, k, L, S, 0, 16), None, pools) as c:
+        x = x_dev(xb)
+        out = torch.empty_like(x)
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, out, 1)
+        ft.ft_sync_status(c.h)
+        cur = x
+        inputs = []
+        for l in range(L):
+            inputs.append(bf16_bits(cur))
+            nxt = torch.empty_like(x)
+            ft.ft_moe_layer_forward(c.h, l, cur, T, None, lg_all[l], nxt, 1)
+            cur = nxt
+        torch.cuda.synchronize()
+        assert (bf16_bits(out) == bf16_bits(cur)).all()
+    # layer-local parity of the last layer against the oracle
+    blobs = {}
+
+    def blob_of(e):
+        if e not in blobs:
+            blobs[e] = synth.expert_blob(seed, L - 1, e, H, I)
+        return blobs[e]
+    r = olayer.moe_layer(inputs[-1], blob_of, H, I, E, k, logits=lgs[-1], shared_blob=blob_of(E))
+    assert_close(bf16_bits(out), r["out_f64"])
