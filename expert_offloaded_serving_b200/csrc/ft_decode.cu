@@ -85,7 +85,7 @@ __device__ __forceinline__ void st_cluster_f32(const float* local_addr, uint32_t
 // ---------------------------------------------------------------------------
 // routing inside a CTA
 // ---------------------------------------------------------------------------
-struct Route {
+struct alignas(16) Route {
   int32_t ids[kMaxPairs];    // [t*k + j], rank order
   float w[kMaxPairs];
   int32_t pos[kMaxPairs];    // permuted position of pair f (= inv)
@@ -96,7 +96,12 @@ struct Route {
   uint8_t first[kMaxPairs];  // pair is its expert's lowest-token pair
   int32_t n_active;
   int32_t bad;
+  int32_t last;              // this CTA finished its row group last
 };
+static_assert(sizeof(Route) % 16 == 0, "Route must keep the mbarrier behind it 16-byte aligned");
+// shared-memory offsets: Route, then the mbarrier (8-byte aligned object), then tiles
+constexpr size_t kBarOff = sizeof(Route);
+constexpr size_t kTileOff = (kBarOff + 16 + 127) / 128 * 128;
 
 // Order key of a logit: larger key = ranks first.  NaN -> 1 (below -inf),
 // -0 -> +0, absent -> 0.
@@ -299,8 +304,7 @@ __host__ __device__ inline Plan make_plan(int ks, int nmat, int T) {
   while (p.lpr > 1 && chunks % p.lpr) p.lpr >>= 1;
   p.cpl = chunks / p.lpr;
   p.nmat = nmat;
-  size_t off = sizeof(Route) + 64;
-  off = (off + 127) / 128 * 128;
+  size_t off = kTileOff;
   p.codes = off;
   off += (size_t)nmat * kRows * ks / 2;
   p.scales = off;
@@ -398,7 +402,7 @@ __device__ void cluster_exchange(const Plan& pl, const float* part, float* recv,
 __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Route& r = *reinterpret_cast<Route*>(smem);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + sizeof(Route));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   const int S = a.s_gu;
   const Plan pl = make_plan(a.H / S, 2, a.T);
   uint8_t* codes_s = smem + pl.codes;
@@ -481,8 +485,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
 __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Route& r = *reinterpret_cast<Route*>(smem);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + sizeof(Route));
-  __shared__ int last;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   const int S = a.s_dn;
   const Plan pl = make_plan(a.I / S, 1, a.T);
   uint8_t* codes_s = smem + pl.codes;
@@ -547,11 +550,11 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   if (threadIdx.x == 0) {
     int* ctr = a.counters + rb * S + slice;
     int old = atomicAdd(ctr, 1);
-    last = (old == units - 1);
-    if (last) *ctr = 0;
+    r.last = (old == units - 1);
+    if (r.last) *ctr = 0;
   }
   __syncthreads();
-  if (!last) return;
+  if (!r.last) return;
   __threadfence();
   for (int i = threadIdx.x; i < a.T * rows_per_owner; i += kThreads) {
     int t = i / rows_per_owner, rl = i % rows_per_owner;
