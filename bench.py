@@ -364,7 +364,8 @@ def main():
     pk = peaks()
     gu = res["kernels"].get("gate_up")
     dn = res["kernels"].get("down_combine")
-    gu_gbs = res["gate_up_bytes"] / (gu["us_avg"] * 1e-6) / 1e9
+    print(f"# tok/s {res['tok_s']:.1f}  step HBM {res['hbm_gbs']:.0f} GB/s  kernels {res['kernels']}", file=sys.stderr)
+    gu_gbs = res["gate_up_bytes"] / (gu["us_avg"] * 1e-6) / 1e9 if gu else float("nan")
     line = {"metric": METRIC, "value": res["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",

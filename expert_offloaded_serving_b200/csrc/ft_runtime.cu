@@ -217,11 +217,12 @@ struct KTimer {
     captured = cs != cudaStreamCaptureStatusNone;
     cudaEventCreate(&a);
     cudaEventCreate(&b);
-    cudaEventRecord(a, s);
+    // under capture only an external record becomes a graph node that records
+    cudaEventRecordWithFlags(a, s, captured ? cudaEventRecordExternal : cudaEventRecordDefault);
   }
   ~KTimer() {
     if (!a) return;
-    cudaEventRecord(b, s);
+    cudaEventRecordWithFlags(b, s, captured ? cudaEventRecordExternal : cudaEventRecordDefault);
     (captured ? c->gmarks : c->tmarks).push_back({cls, {a, b}});
   }
 };
