@@ -114,52 +114,53 @@ __device__ __forceinline__ uint32_t order_key(float v) {
 
 // Warp w routes tokens w, w+8, ...; then every thread finds the permuted
 // position of its pair; finally units (distinct experts, ascending) are listed.
+// PER = logits per lane (E <= 32 * PER), a compile-time bound so that the keys
+// stay in registers.
+template <int PER>
 __device__ void route_in_cta(const float* __restrict__ logits, int T, int E, int k, int renorm, Route& r,
                              int* status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) r.bad = 0;
   __syncthreads();
-  const int per = (E + 31) >> 5;
   for (int t = warp; t < T; t += kThreads / 32) {
     const float* row = logits + (size_t)t * E;
-    uint32_t key[32];
+    uint32_t key[PER];
     bool bad = false;
     float vmax = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < 32; q++) {
-      key[q] = 0u;
-      if (q < per) {
-        int e = lane + 32 * q;
-        if (e < E) {
-          float v = __ldg(row + e);
-          key[q] = order_key(v);
-          if (isnan(v) || v == INFINITY) bad = true;
-          if (!isnan(v)) vmax = fmaxf(vmax, v);
-        }
-      }
+    for (int q = 0; q < PER; q++) {
+      int e = lane + 32 * q;
+      float v = e < E ? __ldg(row + e) : -INFINITY;
+      key[q] = e < E ? order_key(v) : 0u;
+      if (e < E && (isnan(v) || v == INFINITY)) bad = true;
+      if (e < E && !isnan(v)) vmax = fmaxf(vmax, v);
     }
-    for (int d = 16; d >= 1; d >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, d));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 1));
     if (vmax == -INFINITY) bad = true;
     if (__any_sync(0xffffffffu, bad) && lane == 0) r.bad = 1;
     float my_v = 0.f;
     int my_id = -1;
     for (int j = 0; j < k; j++) {
       // lane-local best: largest key, lowest id (ids ascend with q)
-      uint32_t bk = 0u;
-      int bq = -1;
+      uint32_t bk = key[0];
+      int bq = 0;
 #pragma unroll
-      for (int q = 0; q < 32; q++)
+      for (int q = 1; q < PER; q++)
         if (key[q] > bk) {
           bk = key[q];
           bq = q;
         }
-      uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
-      uint32_t cand = (bk == kmax && bq >= 0) ? (uint32_t)(lane + 32 * bq) : 0xffffffffu;
-      uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t cand = (bk == kmax && bk != 0u) ? (uint32_t)(lane + 32 * bq) : 0xffffffffu;
+      const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
       if ((int)(win & 31) == lane) {
 #pragma unroll
-        for (int q = 0; q < 32; q++)
-          if (q == (int)(win >> 5)) key[q] = 0u;
+        for (int q = 0; q < PER; q++)
+          if (q == bq) key[q] = 0u;
       }
       if (lane == j) {
         my_id = (int)win;
@@ -175,7 +176,8 @@ __device__ void route_in_cta(const float* __restrict__ logits, int T, int E, int
       for (int d = 16; d >= 1; d >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, d);
     } else {
       float part = 0.f;
-      for (int q = 0; q < per; q++) {
+#pragma unroll
+      for (int q = 0; q < PER; q++) {
         int e = lane + 32 * q;
         if (e < E) part += expf(__ldg(row + e) - m);
       }
@@ -399,6 +401,7 @@ __device__ void cluster_exchange(const Plan& pl, const float* part, float* recv,
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU
 // ---------------------------------------------------------------------------
+template <int PER>
 __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Route& r = *reinterpret_cast<Route*>(smem);
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   const int rb = (blockIdx.x / S) % RB;
   const int u = blockIdx.x / (S * RB);
 
-  route_in_cta(a.logits, a.T, a.E, a.k, a.renorm, r, a.status);
+  route_in_cta<PER>(a.logits, a.T, a.E, a.k, a.renorm, r, a.status);
   if (blockIdx.x == 0 && a.ids_out) {
     for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
       a.ids_out[f] = r.ids[f];
@@ -482,6 +485,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
 // ---------------------------------------------------------------------------
 // down + combine
 // ---------------------------------------------------------------------------
+template <int PER>
 __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Route& r = *reinterpret_cast<Route*>(smem);
@@ -499,7 +503,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   const int rb = (blockIdx.x / S) % RB;
   const int u = blockIdx.x / (S * RB);
 
-  route_in_cta(a.logits, a.T, a.E, a.k, a.renorm, r, nullptr);
+  route_in_cta<PER>(a.logits, a.T, a.E, a.k, a.renorm, r, nullptr);
   UnitInfo ui;
   if (!resolve_unit(a, r, u, ui)) {
     pdl_trigger();
@@ -582,18 +586,10 @@ int choose_slices(int K) {
 
 size_t decode_smem_bytes(int K, int S, int nmat, int T) { return make_plan(K / S, nmat, T).total; }
 
-static void set_attrs() {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_dec_gate_up, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    cudaFuncSetAttribute(k_dec_down, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    attr = true;
-  }
-}
-
 static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, int grid, int cluster, size_t smem,
                               bool pdl, cudaStream_t s) {
-  set_attrs();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   cudaLaunchAttribute at[2];
   cudaLaunchConfig_t cfg{};
   cfg.blockDim = dim3(kThreads);
@@ -611,16 +607,34 @@ static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, int
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+using KernFn = void (*)(DecodeArgs);
+static KernFn pick_gate_up(int E) {
+  if (E <= 32) return k_dec_gate_up<1>;
+  if (E <= 64) return k_dec_gate_up<2>;
+  if (E <= 128) return k_dec_gate_up<4>;
+  if (E <= 256) return k_dec_gate_up<8>;
+  if (E <= 512) return k_dec_gate_up<16>;
+  return k_dec_gate_up<32>;
+}
+static KernFn pick_down(int E) {
+  if (E <= 32) return k_dec_down<1>;
+  if (E <= 64) return k_dec_down<2>;
+  if (E <= 128) return k_dec_down<4>;
+  if (E <= 256) return k_dec_down<8>;
+  if (E <= 512) return k_dec_down<16>;
+  return k_dec_down<32>;
+}
+
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const int U = a.max_units + a.n_shared;
-  return launch_one(k_dec_gate_up, a, U * (a.I / kRows) * a.s_gu, a.s_gu, decode_smem_bytes(a.H, a.s_gu, 2, a.T), pdl,
-                    s);
+  return launch_one(pick_gate_up(a.E), a, U * (a.I / kRows) * a.s_gu, a.s_gu,
+                    decode_smem_bytes(a.H, a.s_gu, 2, a.T), pdl, s);
 }
 
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const int U = a.max_units + a.n_shared;
-  return launch_one(k_dec_down, a, U * (a.H / kRows) * a.s_dn, a.s_dn, decode_smem_bytes(a.I, a.s_dn, 1, a.T), pdl,
-                    s);
+  return launch_one(pick_down(a.E), a, U * (a.H / kRows) * a.s_dn, a.s_dn, decode_smem_bytes(a.I, a.s_dn, 1, a.T),
+                    pdl, s);
 }
 
 }  // namespace ft
