@@ -4,8 +4,8 @@
 //                   permutation, a few hundred pairs at most), takes one unit
 //                   (a distinct selected expert, or the shared expert), one
 //                   128-row block of Wg/Wu and one K-slice, stages that tile in
-//                   shared memory with bulk async copies (cp.async.bulk + an
-//                   mbarrier), dequantises e2m1 codes with their UE8M0 scales in
+//                   shared memory with coalesced 16-byte cp.async copies from
+//                   all threads, dequantises e2m1 codes with their UE8M0 scales in
 //                   registers, and reduces the K-slices of a row block across
 //                   the CTAs of a thread-block cluster through distributed
 //                   shared memory; the owner CTA applies SwiGLU and writes fp32 h.
@@ -32,43 +32,11 @@ constexpr int kThreads = 256;
 constexpr int kRows = 128;        // rows per CTA tile (one scale-atom row block)
 constexpr int kMaxPairs = 256;    // T * k
 constexpr int kMaxUnits = 257;
-constexpr uint32_t kSpinLimit = 1u << 26;
 
 // ---------------------------------------------------------------------------
 // PTX helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-  asm volatile("fence.mbarrier_init.release.cluster;" ::);
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
-// Bounded wait on phase `parity`; returns false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t addr = smem_u32(bar);
-  for (uint32_t it = 0; it < kSpinLimit; it++) {
-    uint32_t done;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
-}
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
@@ -98,10 +66,9 @@ struct alignas(16) Route {
   int32_t bad;
   int32_t last;              // this CTA finished its row group last
 };
-static_assert(sizeof(Route) % 16 == 0, "Route must keep the mbarrier behind it 16-byte aligned");
-// shared-memory offsets: Route, then the mbarrier (8-byte aligned object), then tiles
-constexpr size_t kBarOff = sizeof(Route);
-constexpr size_t kTileOff = (kBarOff + 16 + 127) / 128 * 128;
+static_assert(sizeof(Route) % 16 == 0, "tiles behind Route must stay 16-byte aligned");
+// shared-memory offsets: Route, then the tiles
+constexpr size_t kTileOff = (sizeof(Route) + 127) / 128 * 128;
 
 // Order key of a logit: larger key = ranks first.  NaN -> 1 (below -inf),
 // -0 -> +0, absent -> 0.
@@ -272,21 +239,28 @@ __device__ __forceinline__ uint32_t tile_scale(const uint8_t* sc, int r, int b) 
   return sc[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)];
 }
 
-// Issue the bulk copies of one 128-row tile: codes rows [row0, row0+128),
-// bytes [kbyte0, kbyte0 + kbytes) of each row (row pitch `pitch`), and the
-// scale atoms of that row block for blocks [kblk0, kblk0 + kbytes/16).
-// Called by warp 0; returns the bytes issued.
-__device__ __forceinline__ uint32_t issue_tile(uint8_t* codes_s, uint8_t* sc_s, const uint8_t* codes_g,
-                                               const uint8_t* sc_g, int row0, int pitch, int kbyte0, int kbytes,
-                                               int atoms_k, uint64_t* bar) {
-  const int lane = threadIdx.x & 31;
-  for (int r = lane; r < kRows; r += 32)
-    bulk_g2s(codes_s + r * kbytes, codes_g + (size_t)(row0 + r) * pitch + kbyte0, (uint32_t)kbytes, bar);
-  const int atoms = kbytes / 64;                // 128 elements (64 bytes) per atom column
-  const int atom0 = kbyte0 / 64;
-  if (lane == 0)
-    bulk_g2s(sc_s, sc_g + ((size_t)(row0 >> 7) * atoms_k + atom0) * 512, (uint32_t)(atoms * 512), bar);
-  return (uint32_t)(kRows * kbytes + atoms * 512);
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Stage one 128-row tile with 16-byte asynchronous copies issued by all
+// threads: code rows [row0, row0+128), bytes [kbyte0, kbyte0 + kbytes) of each
+// row (row pitch `pitch`), and the scale atoms of that row block covering
+// those blocks (contiguous).  Consecutive threads take consecutive 16-byte
+// pieces of a row, so each warp load is coalesced.
+__device__ __forceinline__ void stage_tile(uint8_t* codes_s, uint8_t* sc_s, const uint8_t* codes_g,
+                                           const uint8_t* sc_g, int row0, int pitch, int kbyte0, int kbytes,
+                                           int atoms_k) {
+  const int pieces = kbytes / 16;
+  for (int i = threadIdx.x; i < kRows * pieces; i += kThreads) {
+    int r = i / pieces, p = i % pieces;
+    cp_async16(codes_s + r * kbytes + p * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
+  }
+  const int sc_bytes = (kbytes / 64) * 512;
+  const uint8_t* sg = sc_g + ((size_t)(row0 >> 7) * atoms_k + kbyte0 / 64) * 512;
+  for (int i = threadIdx.x; i < sc_bytes / 16; i += kThreads) cp_async16(sc_s + i * 16, sg + i * 16);
 }
 
 // ---------------------------------------------------------------------------
@@ -405,7 +379,6 @@ template <int PER>
 __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Route& r = *reinterpret_cast<Route*>(smem);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   const int S = a.s_gu;
   const Plan pl = make_plan(a.H / S, 2, a.T);
   uint8_t* codes_s = smem + pl.codes;
@@ -439,18 +412,10 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   }
   const int kbytes = pl.ks / 2, pitch = a.H / 2;
   const int atoms_k = (int)(pad_up(a.H / 32, 4) / 4);
-  if (threadIdx.x == 0) mbar_init(bar, 1);
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    uint32_t bytes = 0;
-    if (threadIdx.x == 0) mbar_expect_tx(bar, 2u * (kRows * kbytes + (kbytes / 64) * 512));
-    __syncwarp();
-    bytes += issue_tile(codes_s, sc_s, blob + a.lay.wg, blob + a.lay.wg_sf, rb * kRows, pitch, slice * kbytes, kbytes,
-                        atoms_k, bar);
-    bytes += issue_tile(codes_s + kRows * kbytes, sc_s + kRows * (pl.ks / 32), blob + a.lay.wu, blob + a.lay.wu_sf,
-                        rb * kRows, pitch, slice * kbytes, kbytes, atoms_k, bar);
-    (void)bytes;
-  }
+  stage_tile(codes_s, sc_s, blob + a.lay.wg, blob + a.lay.wg_sf, rb * kRows, pitch, slice * kbytes, kbytes, atoms_k);
+  stage_tile(codes_s + kRows * kbytes, sc_s + kRows * (pl.ks / 32), blob + a.lay.wu, blob + a.lay.wu_sf, rb * kRows,
+             pitch, slice * kbytes, kbytes, atoms_k);
+  cp_async_commit();
   pdl_trigger();
   pdl_wait();  // activations come from the previous kernel when launched as a dependent
   for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
@@ -460,11 +425,8 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
     reinterpret_cast<float4*>(act)[i] = make_float4(bf16_bits_to_f32(xv.x & 0xffff), bf16_bits_to_f32(xv.x >> 16),
                                                     bf16_bits_to_f32(xv.y & 0xffff), bf16_bits_to_f32(xv.y >> 16));
   }
+  cp_async_wait_all();
   __syncthreads();
-  if (!mbar_wait(bar, 0)) {
-    if (threadIdx.x == 0) set_status(a.status, kStTimeout);
-    mbar_wait(bar, 0);
-  }
   tile_dots(pl, codes_s, sc_s, act, ui.m, a.T, part);
   __syncthreads();
   cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
@@ -489,7 +451,6 @@ template <int PER>
 __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   Route& r = *reinterpret_cast<Route*>(smem);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   const int S = a.s_dn;
   const Plan pl = make_plan(a.I / S, 1, a.T);
   uint8_t* codes_s = smem + pl.codes;
@@ -516,14 +477,8 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   }
   const int kbytes = pl.ks / 2, pitch = a.I / 2;
   const int atoms_k = (int)(pad_up(a.I / 32, 4) / 4);
-  if (threadIdx.x == 0) mbar_init(bar, 1);
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    if (threadIdx.x == 0) mbar_expect_tx(bar, (uint32_t)(kRows * kbytes + (kbytes / 64) * 512));
-    __syncwarp();
-    issue_tile(codes_s, sc_s, blob + a.lay.wd, blob + a.lay.wd_sf, rb * kRows, pitch, slice * kbytes, kbytes, atoms_k,
-               bar);
-  }
+  stage_tile(codes_s, sc_s, blob + a.lay.wd, blob + a.lay.wd_sf, rb * kRows, pitch, slice * kbytes, kbytes, atoms_k);
+  cp_async_commit();
   pdl_trigger();
   pdl_wait();  // h is written by the gate/up kernel
   for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
@@ -531,11 +486,8 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
     reinterpret_cast<float4*>(act)[i] =
         *reinterpret_cast<const float4*>(a.h + (size_t)(ui.hbase + mm) * a.I + slice * pl.ks + k4 * 4);
   }
+  cp_async_wait_all();
   __syncthreads();
-  if (!mbar_wait(bar, 0)) {
-    if (threadIdx.x == 0) set_status(a.status, kStTimeout);
-    mbar_wait(bar, 0);
-  }
   tile_dots(pl, codes_s, sc_s, act, ui.m, a.T, part);
   __syncthreads();
   cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
@@ -578,9 +530,9 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
 // host side
 // ---------------------------------------------------------------------------
 int choose_slices(int K) {
-  // largest S <= 8 with K/S a multiple of 128 and K/S >= 256 (or S = 1)
+  // largest S <= 8 with K/S a multiple of 128 in [512, 1024] (else S = 1)
   for (int s = 8; s >= 2; s--)
-    if (K % (s * 128) == 0 && K / s >= 256 && K / s <= 1024) return s;
+    if (K % (s * 128) == 0 && K / s >= 512 && K / s <= 1024) return s;
   return 1;
 }
 
