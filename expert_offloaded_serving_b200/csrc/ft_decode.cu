@@ -239,6 +239,13 @@ __device__ __forceinline__ uint32_t tile_scale(const uint8_t* sc, int r, int b) 
   return sc[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)];
 }
 
+// Shared-memory position of 16-byte chunk c of tile row r (row of `pieces`
+// chunks, a multiple of 4): chunks are XOR-ed with the row's low bits so that
+// consecutive rows reading the same logical chunk hit different 16-byte bank
+// groups.  The XOR only touches bits inside an aligned group of 8 (or 4)
+// chunks, so the result stays inside the row.
+__device__ __forceinline__ int swz(int c, int r, int pieces) { return c ^ (r & ((pieces & 7) ? 3 : 7)); }
+
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
@@ -256,7 +263,7 @@ __device__ __forceinline__ void stage_tile(uint8_t* codes_s, uint8_t* sc_s, cons
   const int pieces = kbytes / 16;
   for (int i = threadIdx.x; i < kRows * pieces; i += kThreads) {
     int r = i / pieces, p = i % pieces;
-    cp_async16(codes_s + r * kbytes + p * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
+    cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
   }
   const int sc_bytes = (kbytes / 64) * 512;
   const uint8_t* sg = sc_g + ((size_t)(row0 >> 7) * atoms_k + kbyte0 / 64) * 512;
@@ -296,52 +303,73 @@ __host__ __device__ inline Plan make_plan(int ks, int nmat, int T) {
 }
 
 // Partial dot products of the staged tile rows with the staged activations:
-// part[row][mat][tok] (unreduced over K-slices).
+// part[row][mat][tok] (unreduced over K-slices).  Each thread owns one row of
+// one matrix (or a contiguous share of its chunks when a row has more threads),
+// so a row needs no cross-lane reduction; activations are broadcast reads.
 __device__ void tile_dots(const Plan& pl, const uint8_t* codes_s, const uint8_t* sc_s, const float* act, int m, int T,
                           float* part) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lpr = pl.lpr, cpl = pl.cpl, rows_per_pass = (kThreads / 32) * (32 / lpr);
-  const int g = lane / lpr, sl = lane % lpr;
+  const int rows_total = kRows * pl.nmat;
+  const int tpr = kThreads / rows_total;        // threads per row: 1 (gate/up) or 2 (down)
+  const int chunks = pl.ks / 32, cpt = chunks / tpr;
   const int kbytes = pl.ks / 2;
-  constexpr int MT = 2;
-  for (int t0 = 0; t0 < m; t0 += MT) {
-    for (int c = 0; c < cpl; c++) {
-      const int chunk = sl + lpr * c;
-      float2 xv[MT][16];
+  const int rr = threadIdx.x % rows_total;      // consecutive lanes -> consecutive rows
+  const int sub = threadIdx.x / rows_total;
+  const int mat = rr / kRows, r = rr % kRows;
+  const uint8_t* cs = codes_s + (size_t)mat * kRows * kbytes + (size_t)r * kbytes;
+  const uint8_t* ss = sc_s + (size_t)mat * kRows * (pl.ks / 32);
+  for (int t0 = 0; t0 < m; t0 += 2) {
+    const bool two = t0 + 1 < m;
+    const float* a0 = act + (size_t)t0 * pl.ks;
+    const float* a1 = act + (size_t)(two ? t0 + 1 : t0) * pl.ks;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+    for (int cc = 0; cc < cpt; cc++) {
+      const int c = sub * cpt + cc;
+      const uint4 q = *reinterpret_cast<const uint4*>(cs + swz(c, r, chunks) * 16);
+      const float sc = ue8m0_to_f32(tile_scale(ss, r, c));
+      const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+      float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
+      float2 p2 = make_float2(0.f, 0.f), p3 = make_float2(0.f, 0.f);
+      const float4* x0 = reinterpret_cast<const float4*>(a0 + c * 32);
+      const float4* x1 = reinterpret_cast<const float4*>(a1 + c * 32);
 #pragma unroll
-      for (int mm = 0; mm < MT; mm++) {
-        const float4* src = reinterpret_cast<const float4*>(act + (size_t)(t0 + mm < m ? t0 + mm : t0) * pl.ks + chunk * 32);
-#pragma unroll
-        for (int v = 0; v < 8; v++) {
-          float4 f = src[v];
-          xv[mm][2 * v] = make_float2(f.x, f.y);
-          xv[mm][2 * v + 1] = make_float2(f.z, f.w);
+      for (int wv = 0; wv < 4; wv++) {
+        const float4 xa = x0[2 * wv], xb = x0[2 * wv + 1];
+        const float2 w0 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv]));
+        const float2 w1 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 8));
+        const float2 w2 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 16));
+        const float2 w3 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 24));
+        p0 = ffma2(w0, make_float2(xa.x, xa.y), p0);
+        p1 = ffma2(w1, make_float2(xa.z, xa.w), p1);
+        p0 = ffma2(w2, make_float2(xb.x, xb.y), p0);
+        p1 = ffma2(w3, make_float2(xb.z, xb.w), p1);
+        if (two) {
+          const float4 ya = x1[2 * wv], yb = x1[2 * wv + 1];
+          p2 = ffma2(w0, make_float2(ya.x, ya.y), p2);
+          p3 = ffma2(w1, make_float2(ya.z, ya.w), p3);
+          p2 = ffma2(w2, make_float2(yb.x, yb.y), p2);
+          p3 = ffma2(w3, make_float2(yb.z, yb.w), p3);
         }
       }
-      for (int mat = 0; mat < pl.nmat; mat++) {
-        const uint8_t* cs = codes_s + (size_t)mat * kRows * kbytes;
-        const uint8_t* ss = sc_s + (size_t)mat * kRows * (pl.ks / 32);
-        for (int r = warp * (32 / lpr) + g; r < kRows; r += rows_per_pass) {
-          uint4 q = *reinterpret_cast<const uint4*>(cs + (size_t)r * kbytes + chunk * 16);
-          float sc = ue8m0_to_f32(tile_scale(ss, r, chunk));
-          float d0 = chunk_dot(q, xv[0]) * sc;
-          float d1 = (t0 + 1 < m) ? chunk_dot(q, xv[1]) * sc : 0.f;
-          for (int dd = lpr >> 1; dd >= 1; dd >>= 1) {
-            d0 += __shfl_xor_sync(0xffffffffu, d0, dd);
-            d1 += __shfl_xor_sync(0xffffffffu, d1, dd);
-          }
-          if (sl == 0) {
-            float* pr = part + ((size_t)r * pl.nmat + mat) * T;
-            if (c == 0) {
-              pr[t0] = d0;
-              if (t0 + 1 < m) pr[t0 + 1] = d1;
-            } else {
-              pr[t0] += d0;
-              if (t0 + 1 < m) pr[t0 + 1] += d1;
-            }
-          }
-        }
+      s0 = fmaf((p0.x + p0.y) + (p1.x + p1.y), sc, s0);
+      s1 = fmaf((p2.x + p2.y) + (p3.x + p3.y), sc, s1);
+    }
+    float* pr = part + ((size_t)r * pl.nmat + mat) * T;
+    if (tpr == 1) {
+      pr[t0] = s0;
+      if (two) pr[t0 + 1] = s1;
+    } else {
+      // two threads per row (down): the second adds after the first wrote
+      if (sub == 0) {
+        pr[t0] = s0;
+        if (two) pr[t0 + 1] = s1;
       }
+      __syncthreads();
+      if (sub == 1) {
+        pr[t0] += s0;
+        if (two) pr[t0 + 1] += s1;
+      }
+      __syncthreads();
     }
   }
 }
