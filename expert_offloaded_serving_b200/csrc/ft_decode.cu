@@ -30,8 +30,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kRows = 128;        // rows per CTA tile (one scale-atom row block)
-constexpr int kMaxPairs = 256;    // T * k
-constexpr int kMaxUnits = 257;
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -53,22 +51,13 @@ __device__ __forceinline__ void st_cluster_f32(const float* local_addr, uint32_t
 // ---------------------------------------------------------------------------
 // routing inside a CTA
 // ---------------------------------------------------------------------------
-struct alignas(16) Route {
-  int32_t ids[kMaxPairs];    // [t*k + j], rank order
-  float w[kMaxPairs];
-  int32_t pos[kMaxPairs];    // permuted position of pair f (= inv)
-  int32_t perm[kMaxPairs];   // pair at permuted position
-  int32_t unit_e[kMaxUnits];
-  int32_t unit_p0[kMaxUnits];
-  int32_t unit_m[kMaxUnits];
-  uint8_t first[kMaxPairs];  // pair is its expert's lowest-token pair
-  int32_t n_active;
-  int32_t bad;
-  int32_t last;              // this CTA finished its row group last
+// Per-CTA shared header of the GEMV kernels, then the tiles.
+struct CtaHdr {
+  int32_t tok[16];
+  int32_t last;
+  int32_t pad[3];
 };
-static_assert(sizeof(Route) % 16 == 0, "tiles behind Route must stay 16-byte aligned");
-// shared-memory offsets: Route, then the tiles
-constexpr size_t kTileOff = (sizeof(Route) + 127) / 128 * 128;
+constexpr size_t kTileOff = 128;
 
 // Order key of a logit: larger key = ranks first.  NaN -> 1 (below -inf),
 // -0 -> +0, absent -> 0.
@@ -202,12 +191,15 @@ struct UnitInfo {
   bool shared;
 };
 
-__device__ __forceinline__ bool resolve_unit(const DecodeArgs& a, const Route& r, int u, UnitInfo& ui) {
+// Unit u of the layer's routing record: a distinct selected expert (ascending
+// id) or, past max_units, a shared expert.  Token ids of the unit go to tok[].
+__device__ __forceinline__ bool resolve_unit(const DecodeArgs& a, const Route* __restrict__ rec, int u, UnitInfo& ui,
+                                             int* tok) {
   if (u < a.max_units) {
-    if (u >= r.n_active) return false;
-    ui.e = r.unit_e[u];
-    ui.m = r.unit_m[u];
-    ui.hbase = r.unit_p0[u];
+    if (u >= rec->n_active) return false;
+    ui.e = rec->unit_e[u];
+    ui.m = rec->unit_m[u];
+    ui.hbase = rec->unit_p0[u];
     ui.shared = false;
   } else {
     int s = u - a.max_units;
@@ -216,11 +208,8 @@ __device__ __forceinline__ bool resolve_unit(const DecodeArgs& a, const Route& r
     ui.hbase = a.T * a.k + s * a.T;
     ui.shared = true;
   }
+  if (threadIdx.x < ui.m) tok[threadIdx.x] = ui.shared ? threadIdx.x : rec->perm[ui.hbase + threadIdx.x] / a.k;
   return true;
-}
-
-__device__ __forceinline__ int unit_token(const DecodeArgs& a, const Route& r, const UnitInfo& ui, int i) {
-  return ui.shared ? i : r.perm[ui.hbase + i] / a.k;
 }
 
 // Dot of 32 e2m1 codes (16 bytes) with 32 activations (16 float pairs).
@@ -261,9 +250,16 @@ __device__ __forceinline__ void stage_tile(uint8_t* codes_s, uint8_t* sc_s, cons
                                            const uint8_t* sc_g, int row0, int pitch, int kbyte0, int kbytes,
                                            int atoms_k) {
   const int pieces = kbytes / 16;
-  for (int i = threadIdx.x; i < kRows * pieces; i += kThreads) {
-    int r = i / pieces, p = i % pieces;
-    cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
+  if (kThreads % pieces == 0) {
+    const int p = threadIdx.x % pieces, rstep = kThreads / pieces;
+    const uint8_t* src = codes_g + (size_t)row0 * pitch + kbyte0 + p * 16;
+    for (int r = threadIdx.x / pieces; r < kRows; r += rstep)
+      cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, src + (size_t)r * pitch);
+  } else {
+    for (int i = threadIdx.x; i < kRows * pieces; i += kThreads) {
+      int r = i / pieces, p = i % pieces;
+      cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
+    }
   }
   const int sc_bytes = (kbytes / 64) * 512;
   const uint8_t* sg = sc_g + ((size_t)(row0 >> 7) * atoms_k + kbyte0 / 64) * 512;
@@ -403,10 +399,9 @@ __device__ void cluster_exchange(const Plan& pl, const float* part, float* recv,
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU
 // ---------------------------------------------------------------------------
-template <int PER>
 __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  Route& r = *reinterpret_cast<Route*>(smem);
+  CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
   const int S = a.s_gu;
   const Plan pl = make_plan(a.H / S, 2, a.T);
   uint8_t* codes_s = smem + pl.codes;
@@ -420,15 +415,8 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   const int rb = (blockIdx.x / S) % RB;
   const int u = blockIdx.x / (S * RB);
 
-  route_in_cta<PER>(a.logits, a.T, a.E, a.k, a.renorm, r, a.status);
-  if (blockIdx.x == 0 && a.ids_out) {
-    for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
-      a.ids_out[f] = r.ids[f];
-      a.w_out[f] = r.w[f];
-    }
-  }
   UnitInfo ui;
-  if (!resolve_unit(a, r, u, ui)) {
+  if (!resolve_unit(a, a.rec, u, ui, hd.tok)) {
     pdl_trigger();
     return;  // the whole cluster (same unit) leaves together
   }
@@ -448,7 +436,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   pdl_wait();  // activations come from the previous kernel when launched as a dependent
   for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
     int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
-    int t = unit_token(a, r, ui, mm);
+    int t = hd.tok[mm];
     uint2 xv = *reinterpret_cast<const uint2*>(a.x + (size_t)t * a.H + slice * pl.ks + k4 * 4);
     reinterpret_cast<float4*>(act)[i] = make_float4(bf16_bits_to_f32(xv.x & 0xffff), bf16_bits_to_f32(xv.x >> 16),
                                                     bf16_bits_to_f32(xv.y & 0xffff), bf16_bits_to_f32(xv.y >> 16));
@@ -475,10 +463,9 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
 // ---------------------------------------------------------------------------
 // down + combine
 // ---------------------------------------------------------------------------
-template <int PER>
 __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  Route& r = *reinterpret_cast<Route*>(smem);
+  CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
   const int S = a.s_dn;
   const Plan pl = make_plan(a.I / S, 1, a.T);
   uint8_t* codes_s = smem + pl.codes;
@@ -492,9 +479,8 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   const int rb = (blockIdx.x / S) % RB;
   const int u = blockIdx.x / (S * RB);
 
-  route_in_cta<PER>(a.logits, a.T, a.E, a.k, a.renorm, r, nullptr);
   UnitInfo ui;
-  if (!resolve_unit(a, r, u, ui)) {
+  if (!resolve_unit(a, a.rec, u, ui, hd.tok)) {
     pdl_trigger();
     return;
   }
@@ -530,15 +516,15 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   // last CTA of this row group combines
   __threadfence();
   __syncthreads();
-  const int units = r.n_active + a.n_shared;
+  const int units = a.rec->n_active + a.n_shared;
   if (threadIdx.x == 0) {
     int* ctr = a.counters + rb * S + slice;
     int old = atomicAdd(ctr, 1);
-    r.last = (old == units - 1);
-    if (r.last) *ctr = 0;
+    hd.last = (old == units - 1);
+    if (hd.last) *ctr = 0;
   }
   __syncthreads();
-  if (!r.last) return;
+  if (!hd.last) return;
   __threadfence();
   for (int i = threadIdx.x; i < a.T * rows_per_owner; i += kThreads) {
     int t = i / rows_per_owner, rl = i % rows_per_owner;
@@ -546,11 +532,30 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
     float acc = 0.f;
     for (int j = 0; j < a.k; j++) {
       int f = t * a.k + j;
-      acc = fmaf(r.w[f], __ldcg(a.y + (size_t)r.pos[f] * a.H + n), acc);
+      acc = fmaf(a.rec->w[f], __ldcg(a.y + (size_t)a.rec->pos[f] * a.H + n), acc);
     }
     for (int s = 0; s < a.n_shared; s++) acc += __ldcg(a.y + (size_t)(a.T * a.k + s * a.T + t) * a.H + n);
     __nv_bfloat16 b = __float2bfloat16_rn(acc);
     a.out[(size_t)t * a.H + n] = *reinterpret_cast<uint16_t*>(&b);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// routing kernel: CTA l routes layer l and stores its record
+// ---------------------------------------------------------------------------
+template <int PER>
+__global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
+  __shared__ Route r;
+  const int l = blockIdx.x;
+  route_in_cta<PER>(a.logits + (size_t)l * a.T * a.E, a.T, a.E, a.k, a.renorm, r, a.status);
+  const int4* src = reinterpret_cast<const int4*>(&r);
+  int4* dst = reinterpret_cast<int4*>(a.rec + l);
+  for (int i = threadIdx.x; i < (int)(sizeof(Route) / 16); i += kThreads) dst[i] = src[i];
+  if (l == a.n_layers - 1 && a.ids_out) {
+    for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
+      a.ids_out[f] = r.ids[f];
+      a.w_out[f] = r.w[f];
+    }
   }
 }
 
@@ -587,33 +592,27 @@ static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, int
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-using KernFn = void (*)(DecodeArgs);
-static KernFn pick_gate_up(int E) {
-  if (E <= 32) return k_dec_gate_up<1>;
-  if (E <= 64) return k_dec_gate_up<2>;
-  if (E <= 128) return k_dec_gate_up<4>;
-  if (E <= 256) return k_dec_gate_up<8>;
-  if (E <= 512) return k_dec_gate_up<16>;
-  return k_dec_gate_up<32>;
-}
-static KernFn pick_down(int E) {
-  if (E <= 32) return k_dec_down<1>;
-  if (E <= 64) return k_dec_down<2>;
-  if (E <= 128) return k_dec_down<4>;
-  if (E <= 256) return k_dec_down<8>;
-  if (E <= 512) return k_dec_down<16>;
-  return k_dec_down<32>;
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
+  void (*k)(RouteArgs);
+  if (a.E <= 32) k = k_route<1>;
+  else if (a.E <= 64) k = k_route<2>;
+  else if (a.E <= 128) k = k_route<4>;
+  else if (a.E <= 256) k = k_route<8>;
+  else if (a.E <= 512) k = k_route<16>;
+  else k = k_route<32>;
+  k<<<a.n_layers, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const int U = a.max_units + a.n_shared;
-  return launch_one(pick_gate_up(a.E), a, U * (a.I / kRows) * a.s_gu, a.s_gu,
+  return launch_one(k_dec_gate_up, a, U * (a.I / kRows) * a.s_gu, a.s_gu,
                     decode_smem_bytes(a.H, a.s_gu, 2, a.T), pdl, s);
 }
 
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const int U = a.max_units + a.n_shared;
-  return launch_one(pick_down(a.E), a, U * (a.H / kRows) * a.s_dn, a.s_dn, decode_smem_bytes(a.I, a.s_dn, 1, a.T),
+  return launch_one(k_dec_down, a, U * (a.H / kRows) * a.s_dn, a.s_dn, decode_smem_bytes(a.I, a.s_dn, 1, a.T),
                     pdl, s);
 }
 

@@ -1,5 +1,7 @@
-// Small-batch decode kernels (fused routing, bulk-staged FP4 GEMV, cluster
-// split-K reduction, programmatic dependent launch).
+// Small-batch decode kernels: a routing kernel that writes one compact routing
+// record per layer, then per layer a gate/up + SwiGLU GEMV and a down GEMV with
+// the combine (cp.async-staged FP4 tiles, cluster split-K reduction,
+// programmatic dependent launch).
 #pragma once
 
 #include <cstdint>
@@ -9,10 +11,37 @@
 
 namespace ft {
 
+constexpr int kMaxPairs = 256;  // T * k
+constexpr int kMaxUnits = 257;  // distinct experts + shared
+
+// Routing of one layer for T <= 16 tokens (device memory, written by k_route).
+struct alignas(16) Route {
+  int32_t ids[kMaxPairs];    // [t*k + j], rank order
+  float w[kMaxPairs];        // combine weights
+  int32_t pos[kMaxPairs];    // permuted position of pair f (= inv)
+  int32_t perm[kMaxPairs];   // pair at permuted position
+  int32_t unit_e[kMaxUnits]; // distinct experts, ascending
+  int32_t unit_p0[kMaxUnits];
+  int32_t unit_m[kMaxUnits];
+  uint8_t first[kMaxPairs];  // pair is its expert's lowest-token pair
+  int32_t n_active;
+  int32_t bad;
+  int32_t pad[2];
+};
+
+struct RouteArgs {
+  const float* logits;  // fp32 [n_layers][T][E]
+  int T, E, k, renorm, n_layers;
+  Route* rec;           // [n_layers]
+  int32_t* ids_out;     // [T*k] of the last layer, or NULL
+  float* w_out;
+  int* status;
+};
+
 struct DecodeArgs {
   const uint16_t* x;       // bf16 [T][H]
-  const float* logits;     // fp32 [T][E]
-  int T, H, I, E, k, n_shared, renorm;
+  const Route* rec;        // this layer's routing record
+  int T, H, I, E, k, n_shared;
   int max_units;           // routed unit slots: min(E, T*k)
   int s_gu, s_dn;          // cluster sizes (K-slices) of gate/up and down
   const uint8_t* const* eptr;  // [E + n_shared] blob pointers
@@ -20,19 +49,18 @@ struct DecodeArgs {
   float* h;                // [T*k + n_shared*T][I]
   float* y;                // [T*k + n_shared*T][H]
   uint16_t* out;           // bf16 [T][H]
-  int32_t* ids_out;        // [T*k] or NULL (written by one CTA)
-  float* w_out;            // [T*k] or NULL
   int* counters;           // [(H/128) * s_dn], zero before the first launch
   int* status;
 };
 
 int choose_slices(int K);
 size_t decode_smem_bytes(int K, int S, int nmat, int T);
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // pdl: launch as a programmatic dependent of the previous kernel in the
-// stream.  The gate/up kernel reads its routing inputs (logits, pointer table)
-// before griddepcontrol.wait, so it may only be launched that way when those
-// inputs were complete before the previous kernel started; the down kernel
-// reads nothing produced by gate/up before its wait.
+// stream.  The gate/up kernel reads its routing record and pointer table
+// before griddepcontrol.wait, so it may only be launched that way when both
+// were complete before the previous kernel started; the down kernel reads
+// nothing produced by gate/up before its wait.
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s);
 

@@ -156,6 +156,7 @@ struct ft_ctx {
   int32_t* d_pad_offs = nullptr;
   float* d_h = nullptr;
   float* d_y = nullptr;        // decode y [(T*k + S*T)][H]
+  Route* d_routes = nullptr;   // decode routing records [L]
   int* d_counters = nullptr;   // decode combine counters [(H/128) * 8]
   uint16_t* d_xbuf[2] = {nullptr, nullptr};  // stack forward ping-pong [T][H]
   int decode_max_t = 0;
@@ -356,6 +357,7 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
       (st = dev_alloc(&c->d_h, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * I)) ||
       (st = dev_alloc(&c->d_y, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * H)) ||
       (st = dev_alloc(&c->d_counters, (size_t)(H / 128) * 8)) ||
+      (st = dev_alloc(&c->d_routes, (size_t)L)) ||
       (st = dev_alloc(&c->d_xbuf[0], (size_t)c->decode_max_t * H)) ||
       (st = dev_alloc(&c->d_xbuf[1], (size_t)c->decode_max_t * H)))
     return bail(st);
@@ -468,6 +470,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   cudaFree(c->d_h);
   cudaFree(c->d_y);
   cudaFree(c->d_counters);
+  cudaFree(c->d_routes);
   cudaFree(c->d_xbuf[0]);
   cudaFree(c->d_xbuf[1]);
   cudaFree(c->d_eptr_res);
@@ -830,18 +833,17 @@ extern "C" ft_status ft_prefetch_layer(ft_ctx* c, int32_t layer, void* compute_s
 // ---------------------------------------------------------------------------
 // layer forward
 // ---------------------------------------------------------------------------
-static DecodeArgs decode_args(ft_ctx* c, const uint16_t* x, const float* logits, int T, uint32_t flags,
-                              const uint8_t* const* eptr, uint16_t* out) {
+static DecodeArgs decode_args(ft_ctx* c, const uint16_t* x, const Route* rec, int T, const uint8_t* const* eptr,
+                              uint16_t* out) {
   DecodeArgs a{};
   a.x = x;
-  a.logits = logits;
+  a.rec = rec;
   a.T = T;
   a.H = c->d.hidden;
   a.I = c->d.inter;
   a.E = c->d.n_experts;
   a.k = c->d.top_k;
   a.n_shared = c->d.n_shared;
-  a.renorm = (flags & FT_ROUTE_RENORM) ? 1 : 0;
   a.max_units = std::min(a.E, T * a.k);
   a.s_gu = c->s_gu;
   a.s_dn = c->s_dn;
@@ -850,12 +852,26 @@ static DecodeArgs decode_args(ft_ctx* c, const uint16_t* x, const float* logits,
   a.h = c->d_h;
   a.y = c->d_y;
   a.out = out;
-  a.ids_out = c->d_ids;
-  a.w_out = c->d_w;
   a.counters = c->d_counters;
   a.status = c->d_status;
   return a;
 }
+
+static RouteArgs route_args(ft_ctx* c, const float* logits, int T, int n_layers, uint32_t flags, Route* rec) {
+  RouteArgs r{};
+  r.logits = logits;
+  r.T = T;
+  r.E = c->d.n_experts;
+  r.k = c->d.top_k;
+  r.renorm = (flags & FT_ROUTE_RENORM) ? 1 : 0;
+  r.n_layers = n_layers;
+  r.rec = rec;
+  r.ids_out = c->d_ids;
+  r.w_out = c->d_w;
+  r.status = c->d_status;
+  return r;
+}
+
 extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* x, int64_t T,
                                           const float* router_w, const float* logits_override, void* out,
                                           uint32_t flags, void* stream) {
@@ -880,10 +896,13 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     CUDA_TRY(launch_router_logits((const uint16_t*)x, router_w, Ti, H, E, c->d_logits, s));
     logits = c->d_logits;
   }
-  const bool cache_path = !mx && !c->resident[layer];
-  if (mx || cache_path) {
+  Route* rec = c->d_routes + layer;
+  if (mx) {
     KTimer kt(c, FT_K_TOPK, s);
     CUDA_TRY(launch_topk(logits, Ti, E, k, (flags & FT_ROUTE_RENORM) ? 1 : 0, c->d_ids, c->d_w, c->d_status, s));
+  } else {
+    KTimer kt(c, FT_K_TOPK, s);
+    CUDA_TRY(launch_route(route_args(c, logits, Ti, 1, flags, rec), s));
   }
   if (mx) {
     KTimer kt(c, FT_K_PERMUTE, s);
@@ -930,7 +949,7 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
 
   // 5: experts and combine
   if (!mx) {
-    DecodeArgs a = decode_args(c, (const uint16_t*)x, logits, Ti, flags, eptr, (uint16_t*)out);
+    DecodeArgs a = decode_args(c, (const uint16_t*)x, rec, Ti, eptr, (uint16_t*)out);
     {
       KTimer kt(c, FT_K_GATE_UP, s);
       CUDA_TRY(launch_dec_gate_up(a, false, s));
@@ -1032,16 +1051,20 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     if (!c->resident[l]) return fail(FT_ERR_STATE, "layer %d is not resident", l);
   if (T == 0) return FT_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  const int Ti = (int)T, E = c->d.n_experts;
+  const int Ti = (int)T;
+  // all layers' routing records in one launch (their logits are inputs)
+  {
+    KTimer kt(c, FT_K_TOPK, s);
+    CUDA_TRY(launch_route(route_args(c, logits, Ti, n_layers, flags, c->d_routes + first_layer), s));
+  }
   const uint16_t* cur = (const uint16_t*)x;
   for (int i = 0; i < n_layers; i++) {
     const int l = first_layer + i;
     uint16_t* dst = (i == n_layers - 1) ? (uint16_t*)out : c->d_xbuf[i & 1];
-    DecodeArgs a = decode_args(c, cur, logits + (size_t)i * Ti * E, Ti, flags, c->d_eptr_res + (size_t)l * c->n_blobs,
-                               dst);
-    // layers after the first start their routing and weight streaming while
-    // the previous layer finishes: their logits and pointer tables are inputs
-    // of this call, complete before its first kernel
+    DecodeArgs a = decode_args(c, cur, c->d_routes + l, Ti, c->d_eptr_res + (size_t)l * c->n_blobs, dst);
+    // after the first layer, a layer's gate/up starts staging its weights
+    // while the previous layer finishes: its routing record and pointer
+    // table were complete before the first layer's gate/up started
     {
       KTimer kt(c, FT_K_GATE_UP, s);
       CUDA_TRY(launch_dec_gate_up(a, i > 0 && !c->timing, s));
