@@ -28,7 +28,8 @@
 namespace ft {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;       // routing kernel
+constexpr int kGemvThreads = 512;   // GEMV kernels
 constexpr int kRows = 128;        // rows per CTA tile (one scale-atom row block)
 
 // ---------------------------------------------------------------------------
@@ -250,20 +251,20 @@ __device__ __forceinline__ void stage_tile(uint8_t* codes_s, uint8_t* sc_s, cons
                                            const uint8_t* sc_g, int row0, int pitch, int kbyte0, int kbytes,
                                            int atoms_k) {
   const int pieces = kbytes / 16;
-  if (kThreads % pieces == 0) {
-    const int p = threadIdx.x % pieces, rstep = kThreads / pieces;
+  if (kGemvThreads % pieces == 0) {
+    const int p = threadIdx.x % pieces, rstep = kGemvThreads / pieces;
     const uint8_t* src = codes_g + (size_t)row0 * pitch + kbyte0 + p * 16;
     for (int r = threadIdx.x / pieces; r < kRows; r += rstep)
       cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, src + (size_t)r * pitch);
   } else {
-    for (int i = threadIdx.x; i < kRows * pieces; i += kThreads) {
+    for (int i = threadIdx.x; i < kRows * pieces; i += kGemvThreads) {
       int r = i / pieces, p = i % pieces;
       cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
     }
   }
   const int sc_bytes = (kbytes / 64) * 512;
   const uint8_t* sg = sc_g + ((size_t)(row0 >> 7) * atoms_k + kbyte0 / 64) * 512;
-  for (int i = threadIdx.x; i < sc_bytes / 16; i += kThreads) cp_async16(sc_s + i * 16, sg + i * 16);
+  for (int i = threadIdx.x; i < sc_bytes / 16; i += kGemvThreads) cp_async16(sc_s + i * 16, sg + i * 16);
 }
 
 // ---------------------------------------------------------------------------
@@ -290,8 +291,8 @@ __host__ __device__ inline Plan make_plan(int ks, int nmat, int T) {
   off += (size_t)nmat * kRows * ks / 32;
   p.act = off;
   off += (size_t)T * ks * sizeof(float);
-  p.part = off;
-  off += (size_t)kRows * nmat * T * sizeof(float);
+  p.part = off;  // [tpr][row][mat][tok] unreduced partials of the threads sharing a row
+  off += (size_t)(kGemvThreads / (kRows * nmat)) * kRows * nmat * T * sizeof(float);
   p.recv = off;
   off += (size_t)kRows * nmat * T * sizeof(float);
   p.total = off;
@@ -305,7 +306,7 @@ __host__ __device__ inline Plan make_plan(int ks, int nmat, int T) {
 __device__ void tile_dots(const Plan& pl, const uint8_t* codes_s, const uint8_t* sc_s, const float* act, int m, int T,
                           float* part) {
   const int rows_total = kRows * pl.nmat;
-  const int tpr = kThreads / rows_total;        // threads per row: 1 (gate/up) or 2 (down)
+  const int tpr = kGemvThreads / rows_total;    // threads per row: 2 (gate/up) or 4 (down)
   const int chunks = pl.ks / 32, cpt = chunks / tpr;
   const int kbytes = pl.ks / 2;
   const int rr = threadIdx.x % rows_total;      // consecutive lanes -> consecutive rows
@@ -350,23 +351,9 @@ __device__ void tile_dots(const Plan& pl, const uint8_t* codes_s, const uint8_t*
       s0 = fmaf((p0.x + p0.y) + (p1.x + p1.y), sc, s0);
       s1 = fmaf((p2.x + p2.y) + (p3.x + p3.y), sc, s1);
     }
-    float* pr = part + ((size_t)r * pl.nmat + mat) * T;
-    if (tpr == 1) {
-      pr[t0] = s0;
-      if (two) pr[t0 + 1] = s1;
-    } else {
-      // two threads per row (down): the second adds after the first wrote
-      if (sub == 0) {
-        pr[t0] = s0;
-        if (two) pr[t0 + 1] = s1;
-      }
-      __syncthreads();
-      if (sub == 1) {
-        pr[t0] += s0;
-        if (two) pr[t0 + 1] += s1;
-      }
-      __syncthreads();
-    }
+    float* pr = part + (((size_t)sub * kRows + r) * pl.nmat + mat) * T;
+    pr[t0] = s0;
+    if (two) pr[t0 + 1] = s1;
   }
 }
 
@@ -375,13 +362,15 @@ __device__ void tile_dots(const Plan& pl, const uint8_t* codes_s, const uint8_t*
 __device__ void cluster_exchange(const Plan& pl, const float* part, float* recv, int S, int slice, int m, int T) {
   const int rows_per_owner = kRows / S;
   const int n = kRows * pl.nmat * m;
-  for (int i = threadIdx.x; i < n; i += kThreads) {
+  const int tpr = kGemvThreads / (kRows * pl.nmat);
+  for (int i = threadIdx.x; i < n; i += kGemvThreads) {
     int tok = i % m;
     int mat = (i / m) % pl.nmat;
     int r = i / (m * pl.nmat);
     int owner = r / rows_per_owner;
     int rl = r % rows_per_owner;
-    float v = part[((size_t)r * pl.nmat + mat) * T + tok];
+    float v = 0.f;
+    for (int sb = 0; sb < tpr; sb++) v += part[(((size_t)sb * kRows + r) * pl.nmat + mat) * T + tok];
     const float* dst = recv + (((size_t)slice * rows_per_owner + rl) * pl.nmat + mat) * T + tok;
     if (S == 1)
       *const_cast<float*>(dst) = v;
@@ -399,7 +388,7 @@ __device__ void cluster_exchange(const Plan& pl, const float* part, float* recv,
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
+__global__ void __launch_bounds__(kGemvThreads) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
   const int S = a.s_gu;
@@ -434,7 +423,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   cp_async_commit();
   pdl_trigger();
   pdl_wait();  // activations come from the previous kernel when launched as a dependent
-  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
+  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kGemvThreads) {
     int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
     int t = hd.tok[mm];
     uint2 xv = *reinterpret_cast<const uint2*>(a.x + (size_t)t * a.H + slice * pl.ks + k4 * 4);
@@ -448,7 +437,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
   cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
   // owner rows: sum slices in order, SwiGLU, write h
   const int rows_per_owner = kRows / S;
-  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kThreads) {
+  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kGemvThreads) {
     int rl = i / ui.m, tok = i % ui.m;
     float gs = 0.f, us = 0.f;
     for (int s = 0; s < S; s++) {
@@ -463,7 +452,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_gate_up(DecodeArgs a) {
 // ---------------------------------------------------------------------------
 // down + combine
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
+__global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
   const int S = a.s_dn;
@@ -495,7 +484,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   cp_async_commit();
   pdl_trigger();
   pdl_wait();  // h is written by the gate/up kernel
-  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kThreads) {
+  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kGemvThreads) {
     int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
     reinterpret_cast<float4*>(act)[i] =
         *reinterpret_cast<const float4*>(a.h + (size_t)(ui.hbase + mm) * a.I + slice * pl.ks + k4 * 4);
@@ -507,7 +496,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
   const int rows_per_owner = kRows / S;
   const int row0 = rb * kRows + slice * rows_per_owner;
-  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kThreads) {
+  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kGemvThreads) {
     int rl = i / ui.m, tok = i % ui.m;
     float ys = 0.f;
     for (int s = 0; s < S; s++) ys += recv[((size_t)s * rows_per_owner + rl) * a.T + tok];
@@ -526,7 +515,7 @@ __global__ void __launch_bounds__(kThreads) k_dec_down(DecodeArgs a) {
   __syncthreads();
   if (!hd.last) return;
   __threadfence();
-  for (int i = threadIdx.x; i < a.T * rows_per_owner; i += kThreads) {
+  for (int i = threadIdx.x; i < a.T * rows_per_owner; i += kGemvThreads) {
     int t = i / rows_per_owner, rl = i % rows_per_owner;
     int n = row0 + rl;
     float acc = 0.f;
@@ -577,7 +566,7 @@ static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, int
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute at[2];
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kGemvThreads);
   cfg.gridDim = dim3(grid);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
