@@ -1,25 +1,110 @@
-// Prefill path (MXFP4 activations): scratch management and the driver of the
-// quantise -> grouped GEMM (gate/up + SwiGLU + quantise h) -> grouped GEMM
-// (down) -> combine sequence.
+// Prefill path (MXFP4 activations): scratch, the activation quantiser into
+// 128-padded per-expert segments, and the weighted combine.  The grouped GEMMs
+// are in ft_gemm.cu; the runtime sequences the steps.
+//
+//   rows:  every expert e owns padded rows [pad_offs[e], pad_offs[e+1]) of the
+//          activation matrices, a multiple of 128 so that a token tile of the
+//          GEMM and a scale atom never straddle two experts; its first
+//          offs[e+1]-offs[e] rows hold its tokens in ascending order, the rest
+//          are zero.  A shared expert owns one more segment holding all tokens.
 #include "ft_common.cuh"
+#include "ft_gemm.h"
 #include "ft_kernels.h"
+#include "ft_mx.cuh"
 #include "ft_runtime.h"
 
 namespace ft {
+namespace {
+
+__device__ __forceinline__ int segment_of(const int32_t* pad_offs, int nseg, int row) {
+  int lo = 0, hi = nseg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pad_offs[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void k_shared_segments(int32_t* pad_offs, int E, int T, int n_shared) {
+  if (threadIdx.x == 0)
+    for (int s = 0; s < n_shared; s++) pad_offs[E + 1 + s] = pad_offs[E + s] + (int32_t)pad_up(T, 128);
+}
+
+// Warp per padded row: quantise the row's token (or zeros) per 32 values.
+__global__ void __launch_bounds__(256) k_quant_x(const uint16_t* __restrict__ x, int T, int H, int E, int k,
+                                                 int n_seg, const int32_t* __restrict__ pad_offs,
+                                                 const int32_t* __restrict__ offs, const int32_t* __restrict__ perm,
+                                                 int rows_bound, uint8_t* __restrict__ xq, uint8_t* __restrict__ xq_sf) {
+  const int lane = threadIdx.x & 31;
+  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (p >= rows_bound || p >= pad_offs[n_seg]) return;
+  const int e = segment_of(pad_offs, n_seg, p);
+  const int r = p - pad_offs[e];
+  const bool shared = e >= E;
+  const int count = shared ? T : offs[e + 1] - offs[e];
+  const int token = r < count ? (shared ? r : perm[offs[e] + r] / k) : -1;
+  const int nb = H / 32, atoms_k = H / 128;
+  for (int b = lane; b < nb; b += 32) {
+    uint4 q = make_uint4(0, 0, 0, 0);
+    uint32_t sc = 0;
+    if (token >= 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)token * H + b * 32);
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const uint4 w = __ldg(src + i);
+        v[2 * i] = make_float4(bf16_bits_to_f32(w.x & 0xffff), bf16_bits_to_f32(w.x >> 16),
+                               bf16_bits_to_f32(w.y & 0xffff), bf16_bits_to_f32(w.y >> 16));
+        v[2 * i + 1] = make_float4(bf16_bits_to_f32(w.z & 0xffff), bf16_bits_to_f32(w.z >> 16),
+                                   bf16_bits_to_f32(w.w & 0xffff), bf16_bits_to_f32(w.w >> 16));
+      }
+      sc = mx_quant_block(v, q);
+    }
+    *reinterpret_cast<uint4*>(xq + (size_t)p * (H / 2) + b * 16) = q;
+    xq_sf[sf_word(p, b >> 2, atoms_k) + (b & 3)] = (uint8_t)sc;
+  }
+}
+
+// out[t][n] = bf16( sum_j w[t][j] * y[inv[t*k+j]][n]  +  sum_s y[T*k + s*T + t][n] )
+__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y, const float* __restrict__ w,
+                                                 const int32_t* __restrict__ inv, int T, int H, int k, int n_shared,
+                                                 uint16_t* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)T * H) return;
+  const int t = (int)(i / H), n = (int)(i % H);
+  float acc = 0.f;
+  for (int j = 0; j < k; j++) {
+    const int f = t * k + j;
+    acc = fmaf(w[f], y[(size_t)inv[f] * H + n], acc);
+  }
+  for (int s = 0; s < n_shared; s++) acc += y[(size_t)(T * k + s * T + t) * H + n];
+  __nv_bfloat16 b = __float2bfloat16_rn(acc);
+  out[i] = *reinterpret_cast<uint16_t*>(&b);
+}
+
+}  // namespace
+
+int64_t prefill_rows_bound(int T, int E, int k, int n_shared) {
+  return pad_up((int64_t)T * k + 127ll * E + (int64_t)n_shared * pad_up(T, 128), 128);
+}
 
 ft_status ensure_prefill_scratch(PrefillScratch& s, const ft_model_desc& d, int max_tokens) {
   if (s.y) return FT_OK;
-  const int64_t T = max_tokens, E = d.n_experts, k = d.top_k, S = d.n_shared;
+  const int64_t T = max_tokens, k = d.top_k, S = d.n_shared;
   s.H = d.hidden;
   s.I = d.inter;
   s.max_pairs = T * k + S * T;
-  s.max_rows = pad_up(T * k + 127 * E + S * pad_up(T, 128), 128);
+  s.max_rows = prefill_rows_bound(max_tokens, d.n_experts, d.top_k, d.n_shared);
   if (cudaMalloc(&s.xq, (size_t)s.max_rows * s.H / 2) != cudaSuccess ||
       cudaMalloc(&s.xq_sf, (size_t)s.max_rows * s.H / 32) != cudaSuccess ||
       cudaMalloc(&s.hq, (size_t)s.max_rows * s.I / 2) != cudaSuccess ||
       cudaMalloc(&s.hq_sf, (size_t)s.max_rows * s.I / 32) != cudaSuccess ||
-      cudaMalloc(&s.y, (size_t)s.max_pairs * s.H * sizeof(float)) != cudaSuccess ||
-      cudaMalloc(&s.work, (size_t)(4 * (E + S) + 16) * sizeof(int)) != cudaSuccess) {
+      cudaMalloc(&s.y, (size_t)s.max_pairs * s.H * sizeof(float)) != cudaSuccess) {
+    free_prefill_scratch(s);
+    return FT_ERR_CUDA;
+  }
+  if (encode_tmap_2d(&s.map_xq, s.xq, s.H / 2, s.max_rows, s.H / 2) != FT_OK ||
+      encode_tmap_2d(&s.map_hq, s.hq, s.I / 2, s.max_rows, s.I / 2) != FT_OK) {
     free_prefill_scratch(s);
     return FT_ERR_CUDA;
   }
@@ -32,15 +117,68 @@ void free_prefill_scratch(PrefillScratch& s) {
   cudaFree(s.hq);
   cudaFree(s.hq_sf);
   cudaFree(s.y);
-  cudaFree(s.work);
   s = PrefillScratch{};
 }
 
-cudaError_t run_prefill(PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
-  (void)s;
-  (void)a;
-  (void)st;
-  return cudaErrorNotSupported;
+cudaError_t launch_shared_segments(int32_t* pad_offs, int E, int T, int n_shared, cudaStream_t st) {
+  if (n_shared <= 0) return cudaSuccess;
+  k_shared_segments<<<1, 32, 0, st>>>(pad_offs, E, T, n_shared);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_x(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
+  const int64_t rows = prefill_rows_bound(a.T, a.E, a.k, a.n_shared);
+  k_quant_x<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a.x, a.T, a.H, a.E, a.k, a.E + a.n_shared, a.pad_offs, a.offs,
+                                                       a.perm, (int)rows, s.xq, s.xq_sf);
+  return cudaGetLastError();
+}
+
+static GemmArgs gemm_args(const PrefillScratch& s, const PrefillArgs& a, int mode) {
+  GemmArgs g{};
+  g.K = mode == 0 ? a.H : a.I;
+  g.M = mode == 0 ? a.I : a.H;
+  g.n_tiles_max = (int)(prefill_rows_bound(a.T, a.E, a.k, a.n_shared) / kGemmBN);
+  g.n_segments = a.E + a.n_shared;
+  g.pad_offs = a.pad_offs;
+  g.offs = a.offs;
+  g.T = a.T;
+  g.k = a.k;
+  g.E = a.E;
+  g.blob_stride = a.lay.stride;
+  g.sfa_off[0] = mode == 0 ? a.lay.wg_sf : a.lay.wd_sf;
+  g.sfa_off[1] = mode == 0 ? a.lay.wu_sf : a.lay.wd_sf;
+  g.pool = a.pool;
+  g.sfb = mode == 0 ? s.xq_sf : s.hq_sf;
+  g.mode = mode;
+  g.hq = s.hq;
+  g.hq_sf = s.hq_sf;
+  g.y = s.y;
+  g.status = a.status;
+  return g;
+}
+
+cudaError_t launch_prefill_gemm(const PrefillScratch& s, const PrefillArgs& a, int mode, cudaStream_t st) {
+  GemmMaps m{};
+  const int n_blobs = a.E + a.n_shared;
+  const uint64_t stride = (uint64_t)a.lay.stride;
+  if (mode == 0) {
+    if (encode_tmap_3d(&m.a[0], a.pool + a.lay.wg, a.H / 2, a.I, n_blobs, a.H / 2, stride) != FT_OK ||
+        encode_tmap_3d(&m.a[1], a.pool + a.lay.wu, a.H / 2, a.I, n_blobs, a.H / 2, stride) != FT_OK)
+      return cudaErrorInvalidValue;
+    m.b = s.map_xq;
+  } else {
+    if (encode_tmap_3d(&m.a[0], a.pool + a.lay.wd, a.I / 2, a.H, n_blobs, a.I / 2, stride) != FT_OK)
+      return cudaErrorInvalidValue;
+    m.a[1] = m.a[0];
+    m.b = s.map_hq;
+  }
+  return launch_gemm(gemm_args(s, a, mode), m, st);
+}
+
+cudaError_t launch_prefill_combine(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
+  const int64_t n = (int64_t)a.T * a.H;
+  k_combine<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(s.y, a.w, a.inv, a.T, a.H, a.k, a.n_shared, a.out);
+  return cudaGetLastError();
 }
 
 }  // namespace ft

@@ -10,43 +10,9 @@
 // (jansverre.net, "Hvor raskt kjører modellene?").
 #include "ft_common.cuh"
 #include "ft_kernels.h"
+#include "ft_mx.cuh"
 
 namespace ft {
-
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t r;
-  asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u32.u8 %0, b; }" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// 2^(127 - e) for e in [0, 254]
-__device__ __forceinline__ float inv_scale(int e) {
-  return e <= 253 ? __uint_as_float((uint32_t)(254 - e) << 23) : __uint_as_float(0x00400000u);
-}
-
-// Quantise one 32-element block held as 8 float4; returns the scale byte and
-// writes 16 bytes of codes.
-__device__ __forceinline__ uint32_t quant_block(const float4* v, uint4& q) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; i++)
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
-  int be = (int)((__float_as_uint(amax) >> 23) & 0xff);
-  int e = amax == 0.f ? 0 : min(max(be - 2, 0), 254);
-  float s = inv_scale(e);
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-    float4 a = v[2 * i], b = v[2 * i + 1];
-    uint32_t b0 = cvt_e2m1x2(a.x * s, a.y * s);
-    uint32_t b1 = cvt_e2m1x2(a.z * s, a.w * s);
-    uint32_t b2 = cvt_e2m1x2(b.x * s, b.y * s);
-    uint32_t b3 = cvt_e2m1x2(b.z * s, b.w * s);
-    w[i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-  }
-  q = make_uint4(w[0], w[1], w[2], w[3]);
-  return (uint32_t)e;
-}
 
 __global__ void __launch_bounds__(256) k_quant_rows(const float* __restrict__ x, int64_t R, int K,
                                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
@@ -61,7 +27,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const float* __restrict__ x,
 #pragma unroll
     for (int i = 0; i < 8; i++) v[i] = __ldg(src + i);
     uint4 q;
-    uint32_t e = quant_block(v, q);
+    uint32_t e = mx_quant_block(v, q);
     *reinterpret_cast<uint4*>(codes + row * (K / 2) + b * 16) = q;
     scales[sf_word((int)row, b >> 2, atoms_k) + (b & 3)] = (uint8_t)e;
   }

@@ -353,7 +353,7 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
       (st = dev_alloc(&c->d_ids, (size_t)T * k)) || (st = dev_alloc(&c->d_w, (size_t)T * k)) ||
       (st = dev_alloc(&c->d_offs, E + 1)) || (st = dev_alloc(&c->d_perm, (size_t)T * k)) ||
       (st = dev_alloc(&c->d_inv, (size_t)T * k)) || (st = dev_alloc(&c->d_active, E)) ||
-      (st = dev_alloc(&c->d_nact, 1)) || (st = dev_alloc(&c->d_pad_offs, E + 1)) ||
+      (st = dev_alloc(&c->d_nact, 1)) || (st = dev_alloc(&c->d_pad_offs, E + 2)) ||
       (st = dev_alloc(&c->d_h, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * I)) ||
       (st = dev_alloc(&c->d_y, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * H)) ||
       (st = dev_alloc(&c->d_counters, (size_t)(H / 128) * 8)) ||
@@ -881,6 +881,8 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   if (!logits_override && !router_w) return fail(FT_ERR_INVALID, "need router_w or logits_override");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
   const bool mx = (flags & FT_ACT_MXFP4) != 0;
+  if (mx && (c->d.hidden % 256 || c->d.inter % 256))
+    return fail(FT_ERR_INVALID, "the MXFP4 prefill path needs hidden and inter to be multiples of 256");
   if (!mx && T > c->decode_max_t)
     return fail(FT_ERR_INVALID, "decode GEMV path takes T <= %d (use FT_ACT_MXFP4 for prefill)", c->decode_max_t);
   if (T == 0) return FT_OK;
@@ -913,15 +915,18 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   // 4: weight source.  Prefill (MXFP4) reads resident or staged layers and
   // never touches the cache; decode reads resident layers or the cache.
   const uint8_t* const* eptr = nullptr;
+  const uint8_t* pool = nullptr;
   int stage_buf = -1;
   if (c->resident[layer]) {
     eptr = c->d_eptr_res + (size_t)layer * c->n_blobs;
+    pool = c->resident[layer];
   } else if (mx) {
     if (c->stage_layer[layer & 1] != layer)
       return fail(FT_ERR_NOT_FOUND, "prefill of layer %d: not resident and not prefetched", layer);
     stage_buf = layer & 1;
     CUDA_TRY(cudaStreamWaitEvent(s, c->ev_landed[stage_buf], 0));
     eptr = c->d_eptr_stage[stage_buf];
+    pool = c->d_stage[stage_buf];
   } else if (c->cache_on && c->host_layers[layer]) {
     CUDA_TRY(cudaMemcpyAsync(c->h_ids, c->d_ids, (size_t)Ti * k * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
@@ -959,7 +964,8 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
       CUDA_TRY(launch_dec_down(a, true, s));
     }
   } else {
-    FT_TRY(ensure_prefill_scratch(c->pf, c->d, c->max_tokens));
+    if (ensure_prefill_scratch(c->pf, c->d, c->max_tokens) != FT_OK)
+      return fail(FT_ERR_CUDA, "prefill scratch allocation failed");
     PrefillArgs a{};
     a.x = (const uint16_t*)x;
     a.T = Ti;
@@ -975,11 +981,27 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     a.inv = c->d_inv;
     a.pad_offs = c->d_pad_offs;
     a.eptr = eptr;
+    a.pool = pool;
     a.lay = c->lay;
     a.out = (uint16_t*)out;
     a.status = c->d_status;
-    cudaError_t e = run_prefill(c->pf, a, s);
-    if (e != cudaSuccess) return fail(FT_ERR_CUDA, "prefill: %s", cudaGetErrorString(e));
+    CUDA_TRY(launch_shared_segments(c->d_pad_offs, E, Ti, c->d.n_shared, s));
+    {
+      KTimer kt(c, FT_K_QUANT_X, s);
+      CUDA_TRY(launch_quant_x(c->pf, a, s));
+    }
+    {
+      KTimer kt(c, FT_K_GEMM_GATE_UP, s);
+      CUDA_TRY(launch_prefill_gemm(c->pf, a, 0, s));
+    }
+    {
+      KTimer kt(c, FT_K_GEMM_DOWN, s);
+      CUDA_TRY(launch_prefill_gemm(c->pf, a, 1, s));
+    }
+    {
+      KTimer kt(c, FT_K_COMBINE, s);
+      CUDA_TRY(launch_prefill_combine(c->pf, a, s));
+    }
   }
   if (stage_buf >= 0) CUDA_TRY(cudaEventRecord(c->ev_done[stage_buf], s));
   c->last_stream = s;

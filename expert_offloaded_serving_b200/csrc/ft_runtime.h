@@ -1,6 +1,7 @@
 // Runtime-internal declarations shared by the runtime and the prefill path.
 #pragma once
 
+#include <cuda.h>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -22,6 +23,7 @@ struct PrefillArgs {
   const int32_t* inv;       // [T*k]
   const int32_t* pad_offs;  // [E+1] 128-padded segment starts
   const uint8_t* const* eptr;
+  const uint8_t* pool;      // blob 0 of the layer pool (blobs contiguous at lay.stride)
   BlobLayout lay;
   uint16_t* out;  // bf16 [T][H]
   int* status;
@@ -36,14 +38,20 @@ struct PrefillScratch {
   uint8_t* hq = nullptr;    // [max_rows][I/2]
   uint8_t* hq_sf = nullptr; // atoms over [max_rows][I/32]
   float* y = nullptr;       // [max_pairs][H]
-  int* work = nullptr;      // tile list scratch
+  CUtensorMap map_xq;       // TMA maps of xq and hq (token side of the GEMMs)
+  CUtensorMap map_hq;
 };
 
 // Set the message ft_last_error() returns on this thread.
 void set_last_error(const char* msg);
 
+int64_t prefill_rows_bound(int T, int E, int k, int n_shared);
 ft_status ensure_prefill_scratch(PrefillScratch& s, const ft_model_desc& d, int max_tokens);
 void free_prefill_scratch(PrefillScratch& s);
-cudaError_t run_prefill(PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
+cudaError_t launch_shared_segments(int32_t* pad_offs, int E, int T, int n_shared, cudaStream_t st);
+cudaError_t launch_quant_x(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
+// mode 0: gate/up GEMM + SwiGLU + MXFP4 h;  mode 1: down GEMM -> y
+cudaError_t launch_prefill_gemm(const PrefillScratch& s, const PrefillArgs& a, int mode, cudaStream_t st);
+cudaError_t launch_prefill_combine(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace ft
