@@ -329,6 +329,162 @@ def oracle_tok_s(T, n_layers, budget_s=12.0):
     return T / (per_layer * L), done, threads
 
 
+# ---------------------------------------------------------------------------
+# secondary measurements: prefill FP4 GEMM throughput with double-buffered
+# prefetch, expert-cache miss fetch bandwidth
+# ---------------------------------------------------------------------------
+def pinned_h2d_gbs(nbytes=1 << 30, reps=10):
+    """Best-of-reps pinned host -> device copy bandwidth (GB/s)."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    best = 1e9
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        d.copy_(h, non_blocking=True)
+        b.record()
+        b.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del h, d
+    return nbytes / (best / 1e3) / 1e9
+
+
+def host_layer_pools(H, I, n_blobs, seed, layers):
+    """Pinned host pools of `layers` layers, filled on the GPU and copied down."""
+    import torch
+    import synth.gpu
+    stride = synth.blob_stride(H, I)
+    pools = []
+    for layer in range(layers):
+        h = torch.empty(n_blobs * stride, dtype=torch.uint8).pin_memory()
+        d = synth.gpu.layer_pool(H, I, n_blobs, seed, layer)
+        h.copy_(d)
+        del d
+        pools.append(h)
+    torch.cuda.synchronize()
+    return pools
+
+
+def measure_prefill(reps=3, layers=3):
+    """DeepSeek-V4-Flash-class prefill: hidden 4096, 256 experts top-6,
+    intermediate 2048, one 4096-token chunk, near-uniform routing through the
+    router GEMV.  (a) GEMM throughput on a resident layer (kernel timers);
+    (b) layers served from pinned host pools with double-buffered prefetch."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+    H2, I2, E2, k2, T2, seed = 4096, 2048, 256, 6, 4096, 1004
+    flops = 2.0 * T2 * k2 * 3 * H2 * I2
+    pool = synth.gpu.layer_pool(H2, I2, E2, seed, 0)
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, 1, 0, 0, T2), None, [pool])
+    x = torch.from_numpy(synth.activations_bf16(seed, 1, T2, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    wr = torch.from_numpy(synth.router_weights(seed, 0, E2, H2)).cuda()
+    out = torch.empty_like(x)
+    flags = ft.FT_ACT_MXFP4 | ft.FT_ROUTE_RENORM
+    for _ in range(2):
+        ft.ft_moe_layer_forward(ctx, 0, x, T2, wr, None, out, flags)
+    torch.cuda.synchronize()
+    ft.ft_kernel_timing_enable(ctx, True)
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, x, T2, wr, None, out, flags)
+    kt = ft.ft_kernel_timing_read(ctx)
+    ft.ft_kernel_timing_enable(ctx, False)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, x, T2, wr, None, out, flags)
+    b.record()
+    b.synchronize()
+    layer_ms = a.elapsed_time(b) / reps
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    del pool
+    torch.cuda.empty_cache()
+    gemm_ms = (kt["gemm_gate_up"][0] + kt["gemm_down"][0]) / reps
+    res = {"workload": "DSV4-class prefill layer: hidden 4096, 256 experts top-6, intermediate 2048, 4096 tokens",
+           "flop_per_layer": flops, "gemm_ms": gemm_ms, "gemm_tflops": flops / (gemm_ms * 1e-3) / 1e12,
+           "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps,
+           "layer_ms_resident": layer_ms,
+           "kernels_ms": {k: v[0] / reps for k, v in kt.items() if v[1]}}
+    res["gemm_weight_gbs"] = E2 * ft.ft_blob_layout(H2, I2)["used"] / (gemm_ms * 1e-3) / 1e9
+    # (b) pinned host pools, double-buffered prefetch
+    hp = host_layer_pools(H2, I2, E2, seed, layers)
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, layers, 0, 0, T2), hp, None)
+    torch.cuda.synchronize()
+    a.record()
+    ft.ft_prefetch_layer(ctx, 0)
+    cur = x
+    for l in range(layers):
+        if l + 1 < layers:
+            ft.ft_prefetch_layer(ctx, l + 1)
+        ft.ft_moe_layer_forward(ctx, l, x, T2, wr, None, out, flags)
+    b.record()
+    b.synchronize()
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    pack = E2 * ft.ft_blob_stride(H2, I2)
+    res["prefetch_layers"] = layers
+    res["layer_ms_prefetched"] = a.elapsed_time(b) / layers
+    res["prefetch_h2d_gbs"] = pack * layers / (a.elapsed_time(b) * 1e-3) / 1e9
+    del hp
+    return res
+
+
+def measure_misses(tokens=64, layers=8):
+    """DeepSeek-V4-Flash-class decode over a GPU LRU expert cache: hidden 4096,
+    256 experts top-6, intermediate 2048; `layers` of the 43 layers with their
+    full pools in pinned host memory and the cache budget scaled from 32 GB of
+    the 147 GB pool; batch 1; Zipf(1.0) traces with 0.5 adjacent reuse;
+    budget shrunk to half and restored mid-trace."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    H3, I3, E3, k3, seed = 4096, 2048, 256, 6, 1003
+    stride = ft.ft_blob_stride(H3, I3)
+    budget = int(32e9 * layers / 43) // stride * stride
+    hp = host_layer_pools(H3, I3, E3, seed, layers)
+    h2d_peak = pinned_h2d_gbs()
+    ctx = ft.ft_create(ft.make_desc(H3, I3, E3, k3, layers, 0, budget, 1), hp, None)
+    sets = np.stack([synth.zipf_trace(seed, l, tokens, E3, k3, 1.0, 0.5) for l in range(layers)], axis=1)
+    lg = torch.from_numpy(np.stack([[synth.logits_for_sets(seed, p * 100 + l, sets[p, l][None], E3)[0]
+                                     for l in range(layers)] for p in range(tokens)])).cuda()
+    x = torch.from_numpy(synth.activations_bf16(seed, 1, 1, H3).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    bufs = [torch.empty_like(x), torch.empty_like(x)]
+    ft.ft_cache_stats_get(ctx, reset=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    cur = x
+    for p in range(tokens):
+        if p == tokens // 3:
+            ft.ft_expert_cache_resize(ctx, budget // 2)
+        if p == 2 * tokens // 3:
+            ft.ft_expert_cache_resize(ctx, budget)
+        for l in range(layers):
+            nxt = bufs[(p * layers + l) % 2]
+            ft.ft_moe_layer_forward(ctx, l, cur, 1, None, lg[p, l], nxt, ft.FT_ROUTE_RENORM)
+            cur = nxt
+    b.record()
+    b.synchronize()
+    st = ft.ft_cache_stats_get(ctx)
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    del hp
+    lookups = st["hits"] + st["misses"]
+    miss_gbs = st["h2d_bytes"] / (st["h2d_ms"] * 1e-3) / 1e9 if st["h2d_ms"] > 0 else None
+    return {"workload": f"DSV4-class decode with expert cache: {layers} of 43 layers, pools in pinned host memory, "
+                        f"budget {budget / 1e9:.1f} GB (32 GB x {layers}/43), batch 1, {tokens} tokens, "
+                        "resize to half and back",
+            "tok_s": tokens / (a.elapsed_time(b) * 1e-3) * layers / 43,
+            "miss_rate": st["misses"] / max(lookups, 1), "hits": st["hits"], "misses": st["misses"],
+            "evictions": st["evictions"], "moves": st["moves"], "miss_h2d_gbs": miss_gbs,
+            "pinned_h2d_gbs": h2d_peak, "miss_h2d_frac": (miss_gbs / h2d_peak) if miss_gbs else None}
+
+
+
 def workload_config(T):
     return {"workload": f"35B-A3B-class MoE decode stack: hidden {H}, {E} routed experts top-{K_TOP} + {S_SHARED} shared, "
                         f"intermediate {I}, {L} layers, MXFP4 (e2m1 + UE8M0/32) weights resident in HBM, "
@@ -377,6 +533,15 @@ def main():
             "kernels": res["kernels"]}
     if dn:
         line["down_combine_gbs"] = res["down_bytes"] / (dn["us_avg"] * 1e-6) / 1e9
+    if not args.no_extra and world == 1:
+        try:
+            line["prefill"] = measure_prefill()
+        except Exception as ex:  # report, do not hide the main line
+            line["prefill"] = {"error": repr(ex)}
+        try:
+            line["miss"] = measure_misses()
+        except Exception as ex:
+            line["miss"] = {"error": repr(ex)}
     if world == 1:
         v, done, threads = oracle_tok_s(T, L, budget_s=12.0)
         line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",
