@@ -40,6 +40,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 or 4)")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
+    ap.add_argument("--case", default="decode", choices=["decode", "prefill", "miss"],
+                    help="decode: the 35B-class decode stack (default line); prefill / miss: only that measurement")
+    ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     return ap.parse_args()
 
 
@@ -493,10 +496,17 @@ def workload_config(T):
 
 
 def main():
+    global L
     args = parse()
     import torch
     world, rank, local = dist_setup(args)
     T = args.tokens
+    L = args.layers
+    if args.case != "decode":
+        if rank == 0:
+            r = measure_prefill(reps=max(args.steps, 1)) if args.case == "prefill" else measure_misses()
+            print(json.dumps({"case": args.case, **r}))
+        return
     if args.impl == "reference":
         if rank != 0:
             return
