@@ -1,22 +1,21 @@
-// Decode path for small batches (T <= 16): fused routing + split-K FP4 GEMV.
+// Decode path for small batches (T <= 16).
 //
-//   k_dec_gate_up   every CTA routes the T tokens itself (softmax top-k +
-//                   permutation, a few hundred pairs at most), takes one unit
-//                   (a distinct selected expert, or the shared expert), one
-//                   128-row block of Wg/Wu and one K-slice, stages that tile in
-//                   shared memory with coalesced 16-byte cp.async copies from
-//                   all threads, dequantises e2m1 codes with their UE8M0 scales in
-//                   registers, and reduces the K-slices of a row block across
-//                   the CTAs of a thread-block cluster through distributed
-//                   shared memory; the owner CTA applies SwiGLU and writes fp32 h.
-//   k_dec_down      same routing; one unit, one 128-row block of Wd, one
-//                   K-slice of I; launched as a programmatic dependent of the
-//                   gate/up kernel so its weight tile streams in while gate/up
-//                   still runs; after griddepcontrol.wait it reads h, reduces
-//                   its K-slices in the cluster and writes y.  The last CTA to
-//                   finish a row block (an atomic counter per row block) sums
-//                   w[t][j] * y over j ascending plus the shared expert and
-//                   rounds once to bf16.
+//   k_route         one CTA per layer: softmax top-k of the T tokens and the
+//                   permutation of their (token, rank) pairs by expert, stored
+//                   as a compact routing record (distinct experts = units).
+//   k_dec_gate_up   CTA = (unit, block of R rows of Wg and Wu) over the full K:
+//                   the tile is staged in shared memory with coalesced 16-byte
+//                   cp.async copies; tpr threads share a row, each dequantising
+//                   its scale-atom columns of e2m1 codes with their UE8M0 scales
+//                   in registers (split-K inside the row group, reduced by
+//                   shuffles); gate and up share the activation reads; SwiGLU
+//                   gives fp32 h.
+//   k_dec_down      CTA = (unit, block of R rows of Wd) over K = I; launched as a
+//                   programmatic dependent of gate/up, so its tile streams in
+//                   while gate/up runs; after griddepcontrol.wait it reads h and
+//                   writes y.  The last CTA to finish a row block (an atomic
+//                   counter per block) sums w[t][j] * y over j ascending plus
+//                   the shared expert and rounds once to bf16.
 //
 // Pages: decode fetches or reuses the selected experts and sums their partial
 // results exactly (jansverre.net, "Hvorfor er båndbredden viktigere enn antall
@@ -40,14 +39,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)_
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(const float* local_addr, uint32_t rank, float v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local_addr)), "r"(rank));
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
-}
 
 // ---------------------------------------------------------------------------
 // routing inside a CTA
@@ -213,201 +204,159 @@ __device__ __forceinline__ bool resolve_unit(const DecodeArgs& a, const Route* _
   return true;
 }
 
-// Dot of 32 e2m1 codes (16 bytes) with 32 activations (16 float pairs).
-__device__ __forceinline__ float chunk_dot(uint4 q, const float2* xv) {
-  float2 acc = make_float2(0.f, 0.f);
-  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int wv = 0; wv < 4; wv++)
-#pragma unroll
-    for (int b = 0; b < 4; b++) acc = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> (8 * b))), xv[wv * 4 + b], acc);
-  return acc.x + acc.y;
-}
-
-// Scale byte of row r (0..127), block b of a staged scale tile (atoms along K).
-__device__ __forceinline__ uint32_t tile_scale(const uint8_t* sc, int r, int b) {
-  return sc[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)];
-}
-
-// Shared-memory position of 16-byte chunk c of tile row r (row of `pieces`
-// chunks, a multiple of 4): chunks are XOR-ed with the row's low bits so that
-// consecutive rows reading the same logical chunk hit different 16-byte bank
-// groups.  The XOR only touches bits inside an aligned group of 8 (or 4)
-// chunks, so the result stays inside the row.
-__device__ __forceinline__ int swz(int c, int r, int pieces) { return c ^ (r & ((pieces & 7) ? 3 : 7)); }
-
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Stage one 128-row tile with 16-byte asynchronous copies issued by all
-// threads: code rows [row0, row0+128), bytes [kbyte0, kbyte0 + kbytes) of each
-// row (row pitch `pitch`), and the scale atoms of that row block covering
-// those blocks (contiguous).  Consecutive threads take consecutive 16-byte
-// pieces of a row, so each warp load is coalesced.
-__device__ __forceinline__ void stage_tile(uint8_t* codes_s, uint8_t* sc_s, const uint8_t* codes_g,
-                                           const uint8_t* sc_g, int row0, int pitch, int kbyte0, int kbytes,
-                                           int atoms_k) {
-  const int pieces = kbytes / 16;
-  if (kGemvThreads % pieces == 0) {
-    const int p = threadIdx.x % pieces, rstep = kGemvThreads / pieces;
-    const uint8_t* src = codes_g + (size_t)row0 * pitch + kbyte0 + p * 16;
-    for (int r = threadIdx.x / pieces; r < kRows; r += rstep)
-      cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, src + (size_t)r * pitch);
-  } else {
-    for (int i = threadIdx.x; i < kRows * pieces; i += kGemvThreads) {
-      int r = i / pieces, p = i % pieces;
-      cp_async16(codes_s + r * kbytes + swz(p, r, pieces) * 16, codes_g + (size_t)(row0 + r) * pitch + kbyte0 + p * 16);
-    }
+// Dot of 32 e2m1 codes (16 bytes) with 32 activations read as 8 float4 from
+// shared memory at `x` with a stride of `xs` float4 between consecutive ones.
+__device__ __forceinline__ float chunk_dot(uint4 q, const float4* x, int xs) {
+  float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
+  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int wv = 0; wv < 4; wv++) {
+    const float4 xa = x[(2 * wv) * xs], xb = x[(2 * wv + 1) * xs];
+    p0 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv])), make_float2(xa.x, xa.y), p0);
+    p1 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 8)), make_float2(xa.z, xa.w), p1);
+    p0 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 16)), make_float2(xb.x, xb.y), p0);
+    p1 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 24)), make_float2(xb.z, xb.w), p1);
   }
-  const int sc_bytes = (kbytes / 64) * 512;
-  const uint8_t* sg = sc_g + ((size_t)(row0 >> 7) * atoms_k + kbyte0 / 64) * 512;
-  for (int i = threadIdx.x; i < sc_bytes / 16; i += kGemvThreads) cp_async16(sc_s + i * 16, sg + i * 16);
+  return (p0.x + p0.y) + (p1.x + p1.y);
 }
 
 // ---------------------------------------------------------------------------
-// shared-memory plan of a CTA (dynamic smem)
+// CTA geometry (host and device).  A CTA takes R consecutive weight rows over
+// the full K of one unit.  tpr threads share a row: thread `sub` owns apr
+// scale-atom columns (128 elements each) sub*apr .. sub*apr+apr-1.  Shared
+// memory holds the R rows' codes, their scale words and the activations of
+// MT tokens, each laid out so that the tpr threads of a row read consecutive
+// 16-byte words (no bank conflicts):
+//   codes: row r, logical chunk c = 4*atom + j, atom = sub*apr + al  ->
+//          16-byte slot r*chunks + (al*4 + j)*tpr + sub
+//   acts:  token t, float4 f = atom*32 + j*8 + v  ->  t*K/4 + ((al*4 + j)*8 + v)*tpr + sub
+//   scales: row r, atom -> word r*atoms + atom (4 blocks' bytes)
 // ---------------------------------------------------------------------------
-struct Plan {
-  int ks, lpr, cpl;   // K-slice (elements), lanes per row, chunks per lane
-  int nmat;           // 2 (gate/up) or 1 (down)
-  size_t codes, scales, act, part, recv, total;
+constexpr int kMT = 2;            // tokens per pass over the tile
+constexpr size_t kSmemLimit = 220 * 1024;
+
+struct Geo {
+  int K, atoms, tpr, apr, R, threads, nmat;
+  size_t codes, scales, act, total;
 };
 
-__host__ __device__ inline Plan make_plan(int ks, int nmat, int T) {
-  Plan p;
-  p.ks = ks;
-  int chunks = ks / 32;
-  p.lpr = 16;
-  while (p.lpr > 1 && chunks % p.lpr) p.lpr >>= 1;
-  p.cpl = chunks / p.lpr;
-  p.nmat = nmat;
-  size_t off = kTileOff;
-  p.codes = off;
-  off += (size_t)nmat * kRows * ks / 2;
-  p.scales = off;
-  off += (size_t)nmat * kRows * ks / 32;
-  p.act = off;
-  off += (size_t)T * ks * sizeof(float);
-  p.part = off;  // [tpr][row][mat][tok] unreduced partials of the threads sharing a row
-  off += (size_t)(kGemvThreads / (kRows * nmat)) * kRows * nmat * T * sizeof(float);
-  p.recv = off;
-  off += (size_t)kRows * nmat * T * sizeof(float);
-  p.total = off;
-  return p;
+__host__ __device__ inline Geo make_geo(int K, int rows, int nmat) {
+  Geo g;
+  g.K = K;
+  g.nmat = nmat;
+  g.atoms = K / 128;
+  g.tpr = 16;
+  while (g.tpr > 1 && g.atoms % g.tpr) g.tpr >>= 1;
+  g.apr = g.atoms / g.tpr;
+  g.R = kGemvThreads / g.tpr;
+  if (g.R > 128) g.R = 128;
+  if (g.R > rows) g.R = rows;
+  for (;;) {
+    g.codes = kTileOff;
+    g.scales = g.codes + (size_t)nmat * g.R * K / 2;
+    g.act = g.scales + (size_t)nmat * g.R * g.atoms * 4;
+    g.total = g.act + (size_t)kMT * K * 4;
+    if (g.total <= kSmemLimit || g.R <= 8) break;
+    g.R >>= 1;
+  }
+  g.threads = g.R * g.tpr;
+  return g;
 }
 
-// Partial dot products of the staged tile rows with the staged activations:
-// part[row][mat][tok] (unreduced over K-slices).  Each thread owns one row of
-// one matrix (or a contiguous share of its chunks when a row has more threads),
-// so a row needs no cross-lane reduction; activations are broadcast reads.
-__device__ void tile_dots(const Plan& pl, const uint8_t* codes_s, const uint8_t* sc_s, const float* act, int m, int T,
-                          float* part) {
-  const int rows_total = kRows * pl.nmat;
-  const int tpr = kGemvThreads / rows_total;    // threads per row: 2 (gate/up) or 4 (down)
-  const int chunks = pl.ks / 32, cpt = chunks / tpr;
-  const int kbytes = pl.ks / 2;
-  const int rr = threadIdx.x % rows_total;      // consecutive lanes -> consecutive rows
-  const int sub = threadIdx.x / rows_total;
-  const int mat = rr / kRows, r = rr % kRows;
-  const uint8_t* cs = codes_s + (size_t)mat * kRows * kbytes + (size_t)r * kbytes;
-  const uint8_t* ss = sc_s + (size_t)mat * kRows * (pl.ks / 32);
-  for (int t0 = 0; t0 < m; t0 += 2) {
-    const bool two = t0 + 1 < m;
-    const float* a0 = act + (size_t)t0 * pl.ks;
-    const float* a1 = act + (size_t)(two ? t0 + 1 : t0) * pl.ks;
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll 4
-    for (int cc = 0; cc < cpt; cc++) {
-      const int c = sub * cpt + cc;
-      const uint4 q = *reinterpret_cast<const uint4*>(cs + swz(c, r, chunks) * 16);
-      const float sc = ue8m0_to_f32(tile_scale(ss, r, c));
-      const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
-      float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
-      float2 p2 = make_float2(0.f, 0.f), p3 = make_float2(0.f, 0.f);
-      const float4* x0 = reinterpret_cast<const float4*>(a0 + c * 32);
-      const float4* x1 = reinterpret_cast<const float4*>(a1 + c * 32);
-#pragma unroll
-      for (int wv = 0; wv < 4; wv++) {
-        const float4 xa = x0[2 * wv], xb = x0[2 * wv + 1];
-        const float2 w0 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv]));
-        const float2 w1 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 8));
-        const float2 w2 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 16));
-        const float2 w3 = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 24));
-        p0 = ffma2(w0, make_float2(xa.x, xa.y), p0);
-        p1 = ffma2(w1, make_float2(xa.z, xa.w), p1);
-        p0 = ffma2(w2, make_float2(xb.x, xb.y), p0);
-        p1 = ffma2(w3, make_float2(xb.z, xb.w), p1);
-        if (two) {
-          const float4 ya = x1[2 * wv], yb = x1[2 * wv + 1];
-          p2 = ffma2(w0, make_float2(ya.x, ya.y), p2);
-          p3 = ffma2(w1, make_float2(ya.z, ya.w), p3);
-          p2 = ffma2(w2, make_float2(yb.x, yb.y), p2);
-          p3 = ffma2(w3, make_float2(yb.z, yb.w), p3);
-        }
+// Stage rows [row0, row0 + R) of one matrix (codes at `codes_g`, row pitch
+// K/2; scale region `sc_g`) with cp.async.
+__device__ __forceinline__ void stage_rows(const Geo& g, uint8_t* codes_s, uint32_t* sc_s, const uint8_t* codes_g,
+                                           const uint8_t* sc_g, int row0) {
+  const int chunks = g.K / 32;
+  const uint8_t* src = codes_g + (size_t)row0 * (g.K / 2);
+  for (int i = threadIdx.x; i < g.R * chunks; i += g.threads) {
+    const int r = i / chunks, c = i - r * chunks;
+    const int atom = c >> 2, j = c & 3, sub = atom / g.apr, al = atom - sub * g.apr;
+    cp_async16(codes_s + ((size_t)r * chunks + (al * 4 + j) * g.tpr + sub) * 16, src + (size_t)i * 16);
+  }
+  for (int i = threadIdx.x; i < g.R * g.atoms; i += g.threads) {
+    const int r = i / g.atoms, atom = i - r * g.atoms;
+    cp_async4(sc_s + i, sc_g + sf_word(row0 + r, atom, g.atoms));
+  }
+}
+
+// Stage tokens tok[t0 .. t0+n) of x (bf16 [.][K]) or of h (fp32 rows) as fp32
+// in the swizzled activation layout.
+template <bool BF16>
+__device__ __forceinline__ void stage_act(const Geo& g, float* act, const void* src, const int* rowidx, int n) {
+  const int f4 = g.K / 4;
+  for (int i = threadIdx.x; i < kMT * f4; i += g.threads) {
+    const int t = i / f4, f = i - t * f4;
+    const int atom = f >> 5, jv = f & 31, sub = atom / g.apr, al = atom - sub * g.apr;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < n) {
+      if (BF16) {
+        const uint2 w = *reinterpret_cast<const uint2*>((const uint16_t*)src + (size_t)rowidx[t] * g.K + f * 4);
+        v = make_float4(bf16_bits_to_f32(w.x & 0xffff), bf16_bits_to_f32(w.x >> 16), bf16_bits_to_f32(w.y & 0xffff),
+                        bf16_bits_to_f32(w.y >> 16));
+      } else {
+        v = *reinterpret_cast<const float4*>((const float*)src + (size_t)rowidx[t] * g.K + f * 4);
       }
-      s0 = fmaf((p0.x + p0.y) + (p1.x + p1.y), sc, s0);
-      s1 = fmaf((p2.x + p2.y) + (p3.x + p3.y), sc, s1);
     }
-    float* pr = part + (((size_t)sub * kRows + r) * pl.nmat + mat) * T;
-    pr[t0] = s0;
-    if (two) pr[t0 + 1] = s1;
+    reinterpret_cast<float4*>(act)[(size_t)t * f4 + ((al * 32 + jv) * g.tpr + sub)] = v;
   }
 }
 
-// Send this CTA's partials of the rows owned by cluster rank `o` to rank o's
-// receive buffer [slice][row_in_owner][mat][tok], then cluster barrier.
-__device__ void cluster_exchange(const Plan& pl, const float* part, float* recv, int S, int slice, int m, int T) {
-  const int rows_per_owner = kRows / S;
-  const int n = kRows * pl.nmat * m;
-  const int tpr = kGemvThreads / (kRows * pl.nmat);
-  for (int i = threadIdx.x; i < n; i += kGemvThreads) {
-    int tok = i % m;
-    int mat = (i / m) % pl.nmat;
-    int r = i / (m * pl.nmat);
-    int owner = r / rows_per_owner;
-    int rl = r % rows_per_owner;
-    float v = 0.f;
-    for (int sb = 0; sb < tpr; sb++) v += part[(((size_t)sb * kRows + r) * pl.nmat + mat) * T + tok];
-    const float* dst = recv + (((size_t)slice * rows_per_owner + rl) * pl.nmat + mat) * T + tok;
-    if (S == 1)
-      *const_cast<float*>(dst) = v;
-    else
-      st_cluster_f32(dst, (uint32_t)owner, v);
+// Row-partial dots of this thread's atoms for matrix `mat` and the (up to)
+// kMT staged tokens; reduced over the tpr threads of the row.
+__device__ __forceinline__ void row_dots(const Geo& g, const uint8_t* codes_s, const uint32_t* sc_s, const float* act,
+                                         int mat, int r, int sub, int n, float* out) {
+  const int chunks = g.K / 32;
+  const int f4 = g.K / 4;
+  const uint8_t* cs = codes_s + (size_t)mat * g.R * g.K / 2 + (size_t)r * chunks * 16;
+  const uint32_t* ss = sc_s + (size_t)mat * g.R * g.atoms + (size_t)r * g.atoms;
+  float s0 = 0.f, s1 = 0.f;
+  for (int al = 0; al < g.apr; al++) {
+    const uint32_t sw = ss[sub * g.apr + al];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const uint4 q = *reinterpret_cast<const uint4*>(cs + ((al * 4 + j) * g.tpr + sub) * 16);
+      const float sc = ue8m0_to_f32((sw >> (8 * j)) & 0xff);
+      const float4* x0 = reinterpret_cast<const float4*>(act) + ((al * 4 + j) * 8) * g.tpr + sub;
+      s0 = fmaf(chunk_dot(q, x0, g.tpr), sc, s0);
+      if (n > 1) s1 = fmaf(chunk_dot(q, x0 + f4, g.tpr), sc, s1);
+    }
   }
-  if (S > 1)
-    cluster_sync();
-  else
-    __syncthreads();
+  for (int d = g.tpr >> 1; d >= 1; d >>= 1) {
+    s0 += __shfl_xor_sync(0xffffffffu, s0, d);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, d);
+  }
+  out[0] = s0;
+  out[1] = s1;
 }
 
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// gate/up + SwiGLU
+// gate/up + SwiGLU: CTA = (unit, block of R rows of Wg and Wu), full K = H
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kGemvThreads) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
-  const int S = a.s_gu;
-  const Plan pl = make_plan(a.H / S, 2, a.T);
-  uint8_t* codes_s = smem + pl.codes;
-  uint8_t* sc_s = smem + pl.scales;
-  float* act = reinterpret_cast<float*>(smem + pl.act);
-  float* part = reinterpret_cast<float*>(smem + pl.part);
-  float* recv = reinterpret_cast<float*>(smem + pl.recv);
-
-  const int RB = a.I / kRows;
-  const int slice = blockIdx.x % S;
-  const int rb = (blockIdx.x / S) % RB;
-  const int u = blockIdx.x / (S * RB);
-
+  const Geo g = make_geo(a.H, a.I, 2);
+  uint8_t* codes_s = smem + g.codes;
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + g.scales);
+  float* act = reinterpret_cast<float*>(smem + g.act);
+  const int nrb = a.I / g.R;
+  const int rb = blockIdx.x % nrb, u = blockIdx.x / nrb;
   UnitInfo ui;
   if (!resolve_unit(a, a.rec, u, ui, hd.tok)) {
     pdl_trigger();
-    return;  // the whole cluster (same unit) leaves together
+    return;
   }
   const uint8_t* blob = a.eptr[ui.e];
   if (blob == nullptr) {
@@ -415,59 +364,43 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_gate_up(DecodeArgs a) {
     pdl_trigger();
     return;
   }
-  const int kbytes = pl.ks / 2, pitch = a.H / 2;
-  const int atoms_k = (int)(pad_up(a.H / 32, 4) / 4);
-  stage_tile(codes_s, sc_s, blob + a.lay.wg, blob + a.lay.wg_sf, rb * kRows, pitch, slice * kbytes, kbytes, atoms_k);
-  stage_tile(codes_s + kRows * kbytes, sc_s + kRows * (pl.ks / 32), blob + a.lay.wu, blob + a.lay.wu_sf, rb * kRows,
-             pitch, slice * kbytes, kbytes, atoms_k);
+  const int row0 = rb * g.R;
+  stage_rows(g, codes_s, sc_s, blob + a.lay.wg, blob + a.lay.wg_sf, row0);
+  stage_rows(g, codes_s + (size_t)g.R * a.H / 2, sc_s + (size_t)g.R * g.atoms, blob + a.lay.wu, blob + a.lay.wu_sf,
+             row0);
   cp_async_commit();
   pdl_trigger();
-  pdl_wait();  // activations come from the previous kernel when launched as a dependent
-  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kGemvThreads) {
-    int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
-    int t = hd.tok[mm];
-    uint2 xv = *reinterpret_cast<const uint2*>(a.x + (size_t)t * a.H + slice * pl.ks + k4 * 4);
-    reinterpret_cast<float4*>(act)[i] = make_float4(bf16_bits_to_f32(xv.x & 0xffff), bf16_bits_to_f32(xv.x >> 16),
-                                                    bf16_bits_to_f32(xv.y & 0xffff), bf16_bits_to_f32(xv.y >> 16));
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  tile_dots(pl, codes_s, sc_s, act, ui.m, a.T, part);
-  __syncthreads();
-  cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
-  // owner rows: sum slices in order, SwiGLU, write h
-  const int rows_per_owner = kRows / S;
-  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kGemvThreads) {
-    int rl = i / ui.m, tok = i % ui.m;
-    float gs = 0.f, us = 0.f;
-    for (int s = 0; s < S; s++) {
-      gs += recv[(((size_t)s * rows_per_owner + rl) * 2 + 0) * a.T + tok];
-      us += recv[(((size_t)s * rows_per_owner + rl) * 2 + 1) * a.T + tok];
+  pdl_wait();  // x is the previous kernel's output when launched as a dependent
+  const int r = threadIdx.x / g.tpr, sub = threadIdx.x % g.tpr;
+  for (int t0 = 0; t0 < ui.m; t0 += kMT) {
+    const int n = min(kMT, ui.m - t0);
+    __syncthreads();
+    stage_act<true>(g, act, a.x, hd.tok + t0, n);
+    cp_async_wait_all();
+    __syncthreads();
+    float gs[2], us[2];
+    row_dots(g, codes_s, sc_s, act, 0, r, sub, n, gs);
+    row_dots(g, codes_s, sc_s, act, 1, r, sub, n, us);
+    if (sub == 0) {
+      a.h[(size_t)(ui.hbase + t0) * a.I + row0 + r] = silu(gs[0]) * us[0];
+      if (n > 1) a.h[(size_t)(ui.hbase + t0 + 1) * a.I + row0 + r] = silu(gs[1]) * us[1];
     }
-    int row = rb * kRows + slice * rows_per_owner + rl;
-    a.h[(size_t)(ui.hbase + tok) * a.I + row] = silu(gs) * us;
   }
 }
 
 // ---------------------------------------------------------------------------
-// down + combine
+// down + combine: CTA = (unit, block of R rows of Wd), full K = I.  The last
+// CTA to finish a row block (one counter per block) does the weighted combine.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
-  const int S = a.s_dn;
-  const Plan pl = make_plan(a.I / S, 1, a.T);
-  uint8_t* codes_s = smem + pl.codes;
-  uint8_t* sc_s = smem + pl.scales;
-  float* act = reinterpret_cast<float*>(smem + pl.act);
-  float* part = reinterpret_cast<float*>(smem + pl.part);
-  float* recv = reinterpret_cast<float*>(smem + pl.recv);
-
-  const int RB = a.H / kRows;
-  const int slice = blockIdx.x % S;
-  const int rb = (blockIdx.x / S) % RB;
-  const int u = blockIdx.x / (S * RB);
-
+  const Geo g = make_geo(a.I, a.H, 1);
+  uint8_t* codes_s = smem + g.codes;
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + g.scales);
+  float* act = reinterpret_cast<float*>(smem + g.act);
+  const int nrb = a.H / g.R;
+  const int rb = blockIdx.x % nrb, u = blockIdx.x / nrb;
   UnitInfo ui;
   if (!resolve_unit(a, a.rec, u, ui, hd.tok)) {
     pdl_trigger();
@@ -478,49 +411,44 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
     pdl_trigger();
     return;  // already reported by the gate/up kernel
   }
-  const int kbytes = pl.ks / 2, pitch = a.I / 2;
-  const int atoms_k = (int)(pad_up(a.I / 32, 4) / 4);
-  stage_tile(codes_s, sc_s, blob + a.lay.wd, blob + a.lay.wd_sf, rb * kRows, pitch, slice * kbytes, kbytes, atoms_k);
+  const int row0 = rb * g.R;
+  stage_rows(g, codes_s, sc_s, blob + a.lay.wd, blob + a.lay.wd_sf, row0);
   cp_async_commit();
   pdl_trigger();
   pdl_wait();  // h is written by the gate/up kernel
-  for (int i = threadIdx.x; i < ui.m * (pl.ks / 4); i += kGemvThreads) {
-    int mm = i / (pl.ks / 4), k4 = i % (pl.ks / 4);
-    reinterpret_cast<float4*>(act)[i] =
-        *reinterpret_cast<const float4*>(a.h + (size_t)(ui.hbase + mm) * a.I + slice * pl.ks + k4 * 4);
+  if (threadIdx.x < 16) hd.tok[threadIdx.x] = ui.hbase + threadIdx.x;  // h rows of the unit's tokens
+  const int r = threadIdx.x / g.tpr, sub = threadIdx.x % g.tpr;
+  for (int t0 = 0; t0 < ui.m; t0 += kMT) {
+    const int n = min(kMT, ui.m - t0);
+    __syncthreads();
+    stage_act<false>(g, act, a.h, hd.tok + t0, n);
+    cp_async_wait_all();
+    __syncthreads();
+    float ys[2];
+    row_dots(g, codes_s, sc_s, act, 0, r, sub, n, ys);
+    if (sub == 0) {
+      a.y[(size_t)(ui.hbase + t0) * a.H + row0 + r] = ys[0];
+      if (n > 1) a.y[(size_t)(ui.hbase + t0 + 1) * a.H + row0 + r] = ys[1];
+    }
   }
-  cp_async_wait_all();
-  __syncthreads();
-  tile_dots(pl, codes_s, sc_s, act, ui.m, a.T, part);
-  __syncthreads();
-  cluster_exchange(pl, part, recv, S, slice, ui.m, a.T);
-  const int rows_per_owner = kRows / S;
-  const int row0 = rb * kRows + slice * rows_per_owner;
-  for (int i = threadIdx.x; i < rows_per_owner * ui.m; i += kGemvThreads) {
-    int rl = i / ui.m, tok = i % ui.m;
-    float ys = 0.f;
-    for (int s = 0; s < S; s++) ys += recv[((size_t)s * rows_per_owner + rl) * a.T + tok];
-    a.y[(size_t)(ui.hbase + tok) * a.H + row0 + rl] = ys;
-  }
-  // last CTA of this row group combines
+  // last CTA of this row block combines
   __threadfence();
   __syncthreads();
   const int units = a.rec->n_active + a.n_shared;
   if (threadIdx.x == 0) {
-    int* ctr = a.counters + rb * S + slice;
-    int old = atomicAdd(ctr, 1);
+    int* ctr = a.counters + rb;
+    const int old = atomicAdd(ctr, 1);
     hd.last = (old == units - 1);
     if (hd.last) *ctr = 0;
   }
   __syncthreads();
   if (!hd.last) return;
   __threadfence();
-  for (int i = threadIdx.x; i < a.T * rows_per_owner; i += kGemvThreads) {
-    int t = i / rows_per_owner, rl = i % rows_per_owner;
-    int n = row0 + rl;
+  for (int i = threadIdx.x; i < a.T * g.R; i += g.threads) {
+    const int t = i / g.R, n = row0 + (i - t * g.R);
     float acc = 0.f;
     for (int j = 0; j < a.k; j++) {
-      int f = t * a.k + j;
+      const int f = t * a.k + j;
       acc = fmaf(a.rec->w[f], __ldcg(a.y + (size_t)a.rec->pos[f] * a.H + n), acc);
     }
     for (int s = 0; s < a.n_shared; s++) acc += __ldcg(a.y + (size_t)(a.T * a.k + s * a.T + t) * a.H + n);
@@ -551,33 +479,22 @@ __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-int choose_slices(int K) {
-  // largest S <= 8 with K/S a multiple of 128 in [512, 1024] (else S = 1)
-  for (int s = 8; s >= 2; s--)
-    if (K % (s * 128) == 0 && K / s >= 512 && K / s <= 1024) return s;
-  return 1;
-}
+size_t decode_smem_bytes(int K, int rows, int nmat) { return make_geo(K, rows, nmat).total; }
 
-size_t decode_smem_bytes(int K, int S, int nmat, int T) { return make_plan(K / S, nmat, T).total; }
-
-static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, int grid, int cluster, size_t smem,
-                              bool pdl, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, const Geo& g, int grid, bool pdl,
+                              cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.total);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute at[2];
+  cudaLaunchAttribute at[1];
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(kGemvThreads);
+  cfg.blockDim = dim3(g.threads);
   cfg.gridDim = dim3(grid);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = g.total;
   cfg.stream = s;
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = cluster;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = at;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
@@ -594,15 +511,13 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
-  const int U = a.max_units + a.n_shared;
-  return launch_one(k_dec_gate_up, a, U * (a.I / kRows) * a.s_gu, a.s_gu,
-                    decode_smem_bytes(a.H, a.s_gu, 2, a.T), pdl, s);
+  const Geo g = make_geo(a.H, a.I, 2);
+  return launch_one(k_dec_gate_up, a, g, (a.max_units + a.n_shared) * (a.I / g.R), pdl, s);
 }
 
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
-  const int U = a.max_units + a.n_shared;
-  return launch_one(k_dec_down, a, U * (a.H / kRows) * a.s_dn, a.s_dn, decode_smem_bytes(a.I, a.s_dn, 1, a.T),
-                    pdl, s);
+  const Geo g = make_geo(a.I, a.H, 1);
+  return launch_one(k_dec_down, a, g, (a.max_units + a.n_shared) * (a.H / g.R), pdl, s);
 }
 
 }  // namespace ft

@@ -1,6 +1,6 @@
 // Small-batch decode kernels: a routing kernel that writes one compact routing
 // record per layer, then per layer a gate/up + SwiGLU GEMV and a down GEMV with
-// the combine (cp.async-staged FP4 tiles, cluster split-K reduction,
+// the combine (cp.async-staged FP4 tiles, split-K inside a row's thread group,
 // programmatic dependent launch).
 #pragma once
 
@@ -43,18 +43,16 @@ struct DecodeArgs {
   const Route* rec;        // this layer's routing record
   int T, H, I, E, k, n_shared;
   int max_units;           // routed unit slots: min(E, T*k)
-  int s_gu, s_dn;          // cluster sizes (K-slices) of gate/up and down
   const uint8_t* const* eptr;  // [E + n_shared] blob pointers
   BlobLayout lay;
   float* h;                // [T*k + n_shared*T][I]
   float* y;                // [T*k + n_shared*T][H]
   uint16_t* out;           // bf16 [T][H]
-  int* counters;           // [(H/128) * s_dn], zero before the first launch
+  int* counters;           // [H/8] combine counters, zero before the first launch
   int* status;
 };
 
-int choose_slices(int K);
-size_t decode_smem_bytes(int K, int S, int nmat, int T);
+size_t decode_smem_bytes(int K, int rows, int nmat);
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // pdl: launch as a programmatic dependent of the previous kernel in the
 // stream.  The gate/up kernel reads its routing record and pointer table

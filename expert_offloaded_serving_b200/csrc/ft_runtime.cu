@@ -160,7 +160,6 @@ struct ft_ctx {
   int* d_counters = nullptr;   // decode combine counters [(H/128) * 8]
   uint16_t* d_xbuf[2] = {nullptr, nullptr};  // stack forward ping-pong [T][H]
   int decode_max_t = 0;
-  int s_gu = 1, s_dn = 1;
 
   // pinned host scratch
   int32_t* h_ids = nullptr;
@@ -356,15 +355,13 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
       (st = dev_alloc(&c->d_nact, 1)) || (st = dev_alloc(&c->d_pad_offs, E + 2)) ||
       (st = dev_alloc(&c->d_h, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * I)) ||
       (st = dev_alloc(&c->d_y, (size_t)(c->decode_max_t * k + desc->n_shared * c->decode_max_t) * H)) ||
-      (st = dev_alloc(&c->d_counters, (size_t)(H / 128) * 8)) ||
+      (st = dev_alloc(&c->d_counters, (size_t)H / 8)) ||
       (st = dev_alloc(&c->d_routes, (size_t)L)) ||
       (st = dev_alloc(&c->d_xbuf[0], (size_t)c->decode_max_t * H)) ||
       (st = dev_alloc(&c->d_xbuf[1], (size_t)c->decode_max_t * H)))
     return bail(st);
-  if (cudaMemset(c->d_counters, 0, (size_t)(H / 128) * 8 * sizeof(int)) != cudaSuccess)
+  if (cudaMemset(c->d_counters, 0, (size_t)H / 8 * sizeof(int)) != cudaSuccess)
     return bail(fail(FT_ERR_CUDA, "memset"));
-  c->s_gu = choose_slices(H);
-  c->s_dn = choose_slices(I);
   if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return bail(fail(FT_ERR_CUDA, "memset"));
   if (cudaMallocHost(&c->h_ids, (size_t)T * k * sizeof(int32_t)) != cudaSuccess ||
       cudaMallocHost(&c->h_status, sizeof(int)) != cudaSuccess)
@@ -845,8 +842,6 @@ static DecodeArgs decode_args(ft_ctx* c, const uint16_t* x, const Route* rec, in
   a.k = c->d.top_k;
   a.n_shared = c->d.n_shared;
   a.max_units = std::min(a.E, T * a.k);
-  a.s_gu = c->s_gu;
-  a.s_dn = c->s_dn;
   a.eptr = eptr;
   a.lay = c->lay;
   a.h = c->d_h;
