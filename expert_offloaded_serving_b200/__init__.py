@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "FT_OK", 1: "FT_ERR_INVALID", 2: "FT_ERR_CUDA", 3: "FT_ERR_NO
 FT_ROUTE_RENORM = 1
 FT_ACT_BF16 = 0
 FT_ACT_MXFP4 = 2
+FT_STACK_LAYERWISE = 4
 FT_EV_HIT, FT_EV_MISS, FT_EV_EVICT, FT_EV_MOVE = range(4)
 
 EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft_destroy", "ft_sync_status",
@@ -31,7 +32,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
-           "combine")
+           "combine", "dec_stack")
 
 
 class FtError(RuntimeError):

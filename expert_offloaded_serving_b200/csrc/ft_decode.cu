@@ -17,10 +17,18 @@
 //                   counter per block) sums w[t][j] * y over j ascending plus
 //                   the shared expert and rounds once to bf16.
 //
+//   k_dec_stack     persistent and cooperative: one launch runs a stack of
+//                   layers; each CTA takes the gate/up and the down tiles with
+//                   its index modulo the grid, layer after layer, and the layers
+//                   hand over through counters in global memory instead of
+//                   kernel boundaries (same arithmetic as the two kernels above).
+//
 // Pages: decode fetches or reuses the selected experts and sums their partial
 // results exactly (jansverre.net, "Hvorfor er båndbredden viktigere enn antall
 // kjerner?"); a gate picks a few experts per token (aiforradalom.hu, "A
 // Mixture-of-Experts (MoE) kihívásai és a FreeToken megoldásai").
+#include <algorithm>
+
 #include "ft_common.cuh"
 #include "ft_decode.h"
 
@@ -29,7 +37,6 @@ namespace {
 
 constexpr int kThreads = 256;       // routing kernel
 constexpr int kGemvThreads = 512;   // GEMV kernels
-constexpr int kRows = 128;        // rows per CTA tile (one scale-atom row block)
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -213,130 +220,330 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Dot of 32 e2m1 codes (16 bytes) with 32 activations read as 8 float4 from
-// shared memory at `x` with a stride of `xs` float4 between consecutive ones.
-__device__ __forceinline__ float chunk_dot(uint4 q, const float4* x, int xs) {
-  float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
-  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int wv = 0; wv < 4; wv++) {
-    const float4 xa = x[(2 * wv) * xs], xb = x[(2 * wv + 1) * xs];
-    p0 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv])), make_float2(xa.x, xa.y), p0);
-    p1 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 8)), make_float2(xa.z, xa.w), p1);
-    p0 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 16)), make_float2(xb.x, xb.y), p0);
-    p1 = ffma2(f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> 24)), make_float2(xb.z, xb.w), p1);
-  }
-  return (p0.x + p0.y) + (p1.x + p1.y);
-}
-
 // ---------------------------------------------------------------------------
-// CTA geometry (host and device).  A CTA takes R consecutive weight rows over
-// the full K of one unit.  tpr threads share a row: thread `sub` owns apr
-// scale-atom columns (128 elements each) sub*apr .. sub*apr+apr-1.  Shared
-// memory holds the R rows' codes, their scale words and the activations of
-// MT tokens, each laid out so that the tpr threads of a row read consecutive
-// 16-byte words (no bank conflicts):
-//   codes: row r, logical chunk c = 4*atom + j, atom = sub*apr + al  ->
-//          16-byte slot r*chunks + (al*4 + j)*tpr + sub
-//   acts:  token t, float4 f = atom*32 + j*8 + v  ->  t*K/4 + ((al*4 + j)*8 + v)*tpr + sub
-//   scales: row r, atom -> word r*atoms + atom (4 blocks' bytes)
+// GEMV tile (host and device).  A CTA of kGemvThreads threads takes R
+// consecutive weight rows of nmat matrices over the full K of one unit.  K is
+// cut into chunks of 32 codes (16 bytes under one UE8M0 scale).  A lane owns
+// one chunk: it holds that chunk's activations of up to kMT tokens in
+// registers and takes the chunk in every row given to its lane group.  A lane
+// group is lpr lanes (a power of two) on lpr consecutive chunks; rpw = 32/lpr
+// groups share a warp; when K has more than 32 chunks, `parts` groups side by
+// side cover it (warp w takes part w % parts).
+//
+// Arithmetic.  The activations of a pass are first re-encoded in shared
+// memory as f16 with one power-of-two factor per 32-element block, chosen so
+// that the block's largest magnitude lands in [2^14, 2^15): a bf16 x is
+// re-encoded exactly (down to 2^-28 of its block's largest element), an fp32 h
+// is rounded to 11 significant bits.  A weight code becomes f16 exactly
+// (cvt.rn.f16x2.e2m1x2), each product w*x is exact in fp32, and the 32 terms
+// of a chunk are summed by fp32 fused multiply-adds (fma.rn.f32.f16) in a fixed
+// order into two accumulators; the chunk's value is that sum times (weight
+// scale x inverse activation factor).  A row's value is the sum of its
+// chunks' values: the lanes of a group add theirs with xor shuffles, then the
+// parts are added in ascending order through shared memory.
+//
+// Shared memory, from the tile's base:
+//   codes  [nmat][R][K/2]        as in global memory (16-byte cp.async copies)
+//   scales [nmat][R][K/128]      words of four blocks' UE8M0 bytes
+//   xh     [kMT][K]              activations, f16
+//   xinv   [kMT][K/32]           inverse block factors
+//   red    [parts][nmat][R][kMT] partial sums
 // ---------------------------------------------------------------------------
-constexpr int kMT = 2;            // tokens per pass over the tile
+constexpr int kMT = 2;                      // tokens per pass over the tile
+constexpr int kWarps = kGemvThreads / 32;
 constexpr size_t kSmemLimit = 220 * 1024;
+constexpr size_t kTileBytes = 64 * 1024;    // weight codes per tile, about
 
-struct Geo {
-  int K, atoms, tpr, apr, R, threads, nmat;
-  size_t codes, scales, act, total;
+struct Gv {
+  int K, chunks, atoms;
+  int lpr, rpw, parts, rsets, groups;
+  int R, nmat;
+  size_t codes, scales, xh, xinv, red, total;
 };
 
-__host__ __device__ inline Geo make_geo(int K, int rows, int nmat) {
-  Geo g;
+__host__ __device__ inline Gv make_gv(int K, int rows, int nmat) {
+  Gv g;
   g.K = K;
   g.nmat = nmat;
+  g.chunks = K / 32;
   g.atoms = K / 128;
-  g.tpr = 16;
-  while (g.tpr > 1 && g.atoms % g.tpr) g.tpr >>= 1;
-  g.apr = g.atoms / g.tpr;
-  g.R = kGemvThreads / g.tpr;
-  if (g.R > 128) g.R = 128;
-  if (g.R > rows) g.R = rows;
+  g.lpr = 1;
+  while (g.lpr < 32 && g.lpr < g.chunks) g.lpr <<= 1;
+  g.rpw = 32 / g.lpr;
+  g.parts = (g.chunks + g.lpr - 1) / g.lpr;
+  g.rsets = kWarps / g.parts;  // 0 for K > 16384: not supported
+  g.groups = g.rsets * g.rpw;
+  int R = 128;
+  while (R > 8 && (size_t)R * nmat * K / 2 > kTileBytes) R >>= 1;
+  if (R > rows) R = rows;
   for (;;) {
-    g.codes = kTileOff;
-    g.scales = g.codes + (size_t)nmat * g.R * K / 2;
-    g.act = g.scales + (size_t)nmat * g.R * g.atoms * 4;
-    g.total = g.act + (size_t)kMT * K * 4;
-    if (g.total <= kSmemLimit || g.R <= 8) break;
-    g.R >>= 1;
+    g.codes = 0;
+    g.scales = (size_t)nmat * R * K / 2;
+    g.xh = g.scales + (size_t)nmat * R * g.atoms * 4;
+    g.xinv = g.xh + (size_t)kMT * K * 2;
+    g.red = g.xinv + (((size_t)kMT * g.chunks * 4 + 15) & ~(size_t)15);
+    g.total = g.red + (size_t)g.parts * nmat * R * kMT * 4;
+    if (g.total <= kSmemLimit || R <= 8) break;
+    R >>= 1;
   }
-  g.threads = g.R * g.tpr;
+  g.R = R;
   return g;
 }
 
-// Stage rows [row0, row0 + R) of one matrix (codes at `codes_g`, row pitch
-// K/2; scale region `sc_g`) with cp.async.
-__device__ __forceinline__ void stage_rows(const Geo& g, uint8_t* codes_s, uint32_t* sc_s, const uint8_t* codes_g,
-                                           const uint8_t* sc_g, int row0) {
-  const int chunks = g.K / 32;
+// Shapes the decode kernels take: K and rows multiples of 128, K <= 16384.
+__host__ __device__ inline bool gv_ok(const Gv& g, int rows) {
+  return g.rsets > 0 && g.total <= kSmemLimit && rows % g.R == 0;
+}
+
+// This thread's place in the tile.
+struct LaneMap {
+  int c;      // chunk (>= chunks: the lane holds no chunk and adds zeros)
+  int grp;    // lane group: rows grp, grp + groups, ...
+  int part;   // K part
+  bool on;    // the warp has a row set
+  bool lead;  // first lane of its group
+};
+
+__device__ __forceinline__ LaneMap lane_map(const Gv& g) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  LaneMap m;
+  m.part = w % g.parts;
+  const int rs = w / g.parts;
+  m.on = rs < g.rsets;
+  m.c = m.part * g.lpr + (lane & (g.lpr - 1));
+  m.grp = rs * g.rpw + lane / g.lpr;
+  m.lead = (lane & (g.lpr - 1)) == 0;
+  return m;
+}
+
+// Stage rows [row0, row0 + R) of matrix `mat` (codes at codes_g, row pitch
+// K/2; scale region sc_g) into the tile with cp.async.
+__device__ __forceinline__ void stage_mat(const Gv& g, uint8_t* base, int mat, const uint8_t* codes_g,
+                                          const uint8_t* sc_g, int row0) {
+  uint8_t* dst = base + g.codes + (size_t)mat * g.R * (g.K / 2);
   const uint8_t* src = codes_g + (size_t)row0 * (g.K / 2);
-  for (int i = threadIdx.x; i < g.R * chunks; i += g.threads) {
-    const int r = i / chunks, c = i - r * chunks;
-    const int atom = c >> 2, j = c & 3, sub = atom / g.apr, al = atom - sub * g.apr;
-    cp_async16(codes_s + ((size_t)r * chunks + (al * 4 + j) * g.tpr + sub) * 16, src + (size_t)i * 16);
-  }
-  for (int i = threadIdx.x; i < g.R * g.atoms; i += g.threads) {
-    const int r = i / g.atoms, atom = i - r * g.atoms;
-    cp_async4(sc_s + i, sc_g + sf_word(row0 + r, atom, g.atoms));
+  const int n16 = g.R * g.chunks;
+  for (int i = threadIdx.x; i < n16; i += kGemvThreads) cp_async16(dst + (size_t)i * 16, src + (size_t)i * 16);
+  uint32_t* sd = reinterpret_cast<uint32_t*>(base + g.scales) + (size_t)mat * g.R * g.atoms;
+  for (int i = threadIdx.x; i < g.R * g.atoms; i += kGemvThreads) {
+    const int r = i / g.atoms, at = i - r * g.atoms;
+    cp_async4(sd + i, sc_g + sf_word(row0 + r, at, g.atoms));
   }
 }
 
-// Stage tokens tok[t0 .. t0+n) of x (bf16 [.][K]) or of h (fp32 rows) as fp32
-// in the swizzled activation layout.
+// Re-encode tokens rows[0 .. n) of a bf16 (x) or fp32 (h) matrix with row
+// length K into the tile's f16 activations (read from L2).  Thread i takes 8
+// consecutive elements; the 4 threads of a 32-element block agree on its
+// factor by shuffles.  Tokens n .. kMT-1 are zero.
 template <bool BF16>
-__device__ __forceinline__ void stage_act(const Geo& g, float* act, const void* src, const int* rowidx, int n) {
-  const int f4 = g.K / 4;
-  for (int i = threadIdx.x; i < kMT * f4; i += g.threads) {
-    const int t = i / f4, f = i - t * f4;
-    const int atom = f >> 5, jv = f & 31, sub = atom / g.apr, al = atom - sub * g.apr;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+__device__ __forceinline__ void stage_x(const Gv& g, uint8_t* base, const void* src, const int* rows, int n) {
+  uint4* xh = reinterpret_cast<uint4*>(base + g.xh);
+  float* xinv = reinterpret_cast<float*>(base + g.xinv);
+  const int per = g.K / 8;
+  // kMT * per is a multiple of 32: a warp is wholly inside or outside
+  for (int i = threadIdx.x; i < kMT * per; i += kGemvThreads) {
+    const int t = i / per, q = i - t * per;
+    float v[8];
     if (t < n) {
       if (BF16) {
-        const uint2 w = *reinterpret_cast<const uint2*>((const uint16_t*)src + (size_t)rowidx[t] * g.K + f * 4);
-        v = make_float4(bf16_bits_to_f32(w.x & 0xffff), bf16_bits_to_f32(w.x >> 16), bf16_bits_to_f32(w.y & 0xffff),
-                        bf16_bits_to_f32(w.y >> 16));
+        const uint4 w = __ldcg(reinterpret_cast<const uint4*>((const uint16_t*)src + (size_t)rows[t] * g.K) + q);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          v[2 * j] = __uint_as_float(ws[j] << 16);
+          v[2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+        }
       } else {
-        v = *reinterpret_cast<const float4*>((const float*)src + (size_t)rowidx[t] * g.K + f * 4);
+        const float4* p = reinterpret_cast<const float4*>((const float*)src + (size_t)rows[t] * g.K) + 2 * q;
+        const float4 a = __ldcg(p), b = __ldcg(p + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; j++) v[j] = 0.f;
     }
-    reinterpret_cast<float4*>(act)[(size_t)t * f4 + ((al * 32 + jv) * g.tpr + sub)] = v;
+    uint32_t e = 0;
+#pragma unroll
+    for (int j = 0; j < 8; j++) e = max(e, __float_as_uint(v[j]) & 0x7f800000u);
+    e = max(e, __shfl_xor_sync(0xffffffffu, e, 1));
+    e = max(e, __shfl_xor_sync(0xffffffffu, e, 2));
+    // largest biased exponent of the block, at least 15 so that both factors
+    // are normal floats: 2^(141-eb) maps the block's maximum into [2^14, 2^15)
+    const int eb = max((int)(e >> 23), 15);
+    const float f = __uint_as_float((uint32_t)(268 - eb) << 23);
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      __half2 hh = __float22half2_rn(make_float2(v[2 * j] * f, v[2 * j + 1] * f));
+      h[j] = *reinterpret_cast<uint32_t*>(&hh);
+    }
+    xh[(size_t)t * per + q] = make_uint4(h[0], h[1], h[2], h[3]);
+    if ((q & 3) == 0) xinv[t * g.chunks + (q >> 2)] = __uint_as_float((uint32_t)(eb - 14) << 23);
   }
 }
 
-// Row-partial dots of this thread's atoms for matrix `mat` and the (up to)
-// kMT staged tokens; reduced over the tpr threads of the row.
-__device__ __forceinline__ void row_dots(const Geo& g, const uint8_t* codes_s, const uint32_t* sc_s, const float* act,
-                                         int mat, int r, int sub, int n, float* out) {
-  const int chunks = g.K / 32;
-  const int f4 = g.K / 4;
-  const uint8_t* cs = codes_s + (size_t)mat * g.R * g.K / 2 + (size_t)r * chunks * 16;
-  const uint32_t* ss = sc_s + (size_t)mat * g.R * g.atoms + (size_t)r * g.atoms;
-  float s0 = 0.f, s1 = 0.f;
-  for (int al = 0; al < g.apr; al++) {
-    const uint32_t sw = ss[sub * g.apr + al];
+// Two e2m1 codes per byte of w -> four f16 pairs (byte b: elements 2b, 2b+1).
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t (&h)[4]) {
+  asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;"
+      " cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;"
+      " cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
+}
+
+// acc += w.lo * x.lo, then acc += w.hi * x.hi (f16 operands, fp32 fused).
+__device__ __forceinline__ float fma_f16x2(uint32_t w, uint32_t x, float acc) {
+  asm("{ .reg .f16 wl, wh, xl, xh; mov.b32 {wl, wh}, %1; mov.b32 {xl, xh}, %2;"
+      " fma.rn.f32.f16 %0, wl, xl, %0; fma.rn.f32.f16 %0, wh, xh, %0; }"
+      : "+f"(acc) : "r"(w), "r"(x));
+  return acc;
+}
+
+// Dot of one chunk of 32 e2m1 codes with NT tokens' f16 activations x[t][i]
+// (elements 2i, 2i+1); even code bytes feed one accumulator, odd ones the
+// other.
+template <int NT>
+__device__ __forceinline__ void chunk_dot(uint4 q, const uint32_t (&x)[kMT][16], float* d) {
+  float acc[NT][2];
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const uint4 q = *reinterpret_cast<const uint4*>(cs + ((al * 4 + j) * g.tpr + sub) * 16);
-      const float sc = ue8m0_to_f32((sw >> (8 * j)) & 0xff);
-      const float4* x0 = reinterpret_cast<const float4*>(act) + ((al * 4 + j) * 8) * g.tpr + sub;
-      s0 = fmaf(chunk_dot(q, x0, g.tpr), sc, s0);
-      if (n > 1) s1 = fmaf(chunk_dot(q, x0 + f4, g.tpr), sc, s1);
+  for (int t = 0; t < NT; t++) acc[t][0] = acc[t][1] = 0.f;
+  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int wv = 0; wv < 4; wv++) {
+    uint32_t h[4];
+    e2m1x8_to_f16x8(qs[wv], h);
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+#pragma unroll
+      for (int t = 0; t < NT; t++) acc[t][j & 1] = fma_f16x2(h[j], x[t][4 * wv + j], acc[t][j & 1]);
+  }
+#pragma unroll
+  for (int t = 0; t < NT; t++) d[t] = acc[t][0] + acc[t][1];
+}
+
+// Sum over the lpr lanes of a group of RU rows' partial sums v[u][t] (RU = 1,
+// 2 or 4, RU <= lpr).  The first one or two xor steps exchange halves of the
+// rows (each lane keeps the half its lane bit selects) and the remaining
+// steps add; afterwards row u's sum is on the lanes whose two group-lane bits
+// (lpr/2, lpr/4) spell u and whose lower bits are zero.  Returns that row.
+template <int RU, int NT>
+__device__ __forceinline__ int group_reduce(float (&v)[4][kMT], int lpr) {
+  const int lane = threadIdx.x & 31;
+  int row = 0, d = lpr >> 1;
+  if (RU == 4) {
+    const bool hi = lane & d;
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const float s0 = hi ? v[0][t] : v[2][t], s1 = hi ? v[1][t] : v[3][t];
+      const float k0 = hi ? v[2][t] : v[0][t], k1 = hi ? v[3][t] : v[1][t];
+      v[0][t] = k0 + __shfl_xor_sync(0xffffffffu, s0, d);
+      v[1][t] = k1 + __shfl_xor_sync(0xffffffffu, s1, d);
+    }
+    row = hi ? 2 : 0;
+    d >>= 1;
+  }
+  if (RU >= 2) {
+    const bool hi = lane & d;
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const float sd = hi ? v[0][t] : v[1][t], kp = hi ? v[1][t] : v[0][t];
+      v[0][t] = kp + __shfl_xor_sync(0xffffffffu, sd, d);
+    }
+    row += hi ? 1 : 0;
+    d >>= 1;
+  }
+  for (; d >= 1; d >>= 1)
+#pragma unroll
+    for (int t = 0; t < NT; t++) v[0][t] += __shfl_xor_sync(0xffffffffu, v[0][t], d);
+  return row;
+}
+
+// Partial sums of the staged tile's rows for NT tokens into red.  Lane group
+// grp takes rows grp + j*groups, RU of them at a time.
+template <int RU, int NT>
+__device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8_t* base,
+                                            const uint32_t (&x)[kMT][16], const float (&xi)[kMT]) {
+  const uint8_t* codes = base + g.codes;
+  const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
+  float* red = reinterpret_cast<float*>(base + g.red);
+  const bool cv = m.c < g.chunks;
+  const int lmask = RU == 4 ? (g.lpr >> 2) - 1 : RU == 2 ? (g.lpr >> 1) - 1 : g.lpr - 1;
+  for (int mat = 0; mat < g.nmat; mat++) {
+    // the trip count is the same for every lane of a warp, so the shuffles
+    // see the whole warp
+    for (int j0 = 0; m.grp + j0 * g.groups < g.R; j0 += RU) {
+      float v[4][kMT];
+#pragma unroll
+      for (int u = 0; u < RU; u++) {
+        v[u][0] = v[u][1] = 0.f;
+        if (cv) {
+          const int row = mat * g.R + m.grp + (j0 + u) * g.groups;
+          const uint4 q = *reinterpret_cast<const uint4*>(codes + (size_t)row * (g.K / 2) + m.c * 16);
+          const uint32_t sw = sc[(size_t)row * g.atoms + (m.c >> 2)];
+          const float s = ue8m0_to_f32((sw >> (8 * (m.c & 3))) & 0xffu);
+          float d[NT];
+          chunk_dot<NT>(q, x, d);
+#pragma unroll
+          for (int t = 0; t < NT; t++) v[u][t] = d[t] * (s * xi[t]);
+        }
+      }
+      const int u = group_reduce<RU, NT>(v, g.lpr);
+      if (((threadIdx.x & 31) & lmask) == 0) {
+        const int r = m.grp + (j0 + u) * g.groups;
+        float* o = red + ((size_t)(m.part * g.nmat + mat) * g.R + r) * kMT;
+#pragma unroll
+        for (int t = 0; t < NT; t++) o[t] = v[0][t];
+      }
     }
   }
-  for (int d = g.tpr >> 1; d >= 1; d >>= 1) {
-    s0 += __shfl_xor_sync(0xffffffffu, s0, d);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, d);
+}
+
+// Partial sums of every row of the staged tile for n (<= kMT) tokens into red.
+__device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t* base, int n) {
+  if (!m.on) return;
+  uint32_t x[kMT][16];
+  float xi[kMT] = {0.f, 0.f};
+  if (m.c < g.chunks) {
+    const uint4* xh = reinterpret_cast<const uint4*>(base + g.xh);
+    const float* xinv = reinterpret_cast<const float*>(base + g.xinv);
+#pragma unroll
+    for (int t = 0; t < kMT; t++) {
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const uint4 u = xh[((size_t)t * g.K + m.c * 32) / 8 + i];
+        x[t][4 * i] = u.x;
+        x[t][4 * i + 1] = u.y;
+        x[t][4 * i + 2] = u.z;
+        x[t][4 * i + 3] = u.w;
+      }
+      xi[t] = xinv[t * g.chunks + m.c];
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < kMT; t++)
+#pragma unroll
+      for (int i = 0; i < 16; i++) x[t][i] = 0u;
   }
-  out[0] = s0;
-  out[1] = s1;
+  // rows per lane group and matrix; groups of 4 or 2 when they divide it
+  const int per = g.R % g.groups == 0 ? g.R / g.groups : 0;
+  const int ru = (per % 4 == 0 && per > 0 && g.lpr >= 4) ? 4 : (per % 2 == 0 && per > 0 && g.lpr >= 2) ? 2 : 1;
+  if (n > 1) {
+    if (ru == 4) tile_dots_t<4, 2>(g, m, base, x, xi);
+    else if (ru == 2) tile_dots_t<2, 2>(g, m, base, x, xi);
+    else tile_dots_t<1, 2>(g, m, base, x, xi);
+  } else {
+    if (ru == 4) tile_dots_t<4, 1>(g, m, base, x, xi);
+    else if (ru == 2) tile_dots_t<2, 1>(g, m, base, x, xi);
+    else tile_dots_t<1, 1>(g, m, base, x, xi);
+  }
+}
+
+// Row r of matrix mat for token t: the parts' partial sums in ascending order.
+__device__ __forceinline__ float row_value(const Gv& g, const uint8_t* base, int mat, int r, int t) {
+  const float* red = reinterpret_cast<const float*>(base + g.red);
+  float s = red[((size_t)mat * g.R + r) * kMT + t];
+  for (int p = 1; p < g.parts; p++) s += red[((size_t)(p * g.nmat + mat) * g.R + r) * kMT + t];
+  return s;
 }
 
 }  // namespace
@@ -344,13 +551,11 @@ __device__ __forceinline__ void row_dots(const Geo& g, const uint8_t* codes_s, c
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU: CTA = (unit, block of R rows of Wg and Wu), full K = H
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kGemvThreads) k_dec_gate_up(DecodeArgs a) {
+__global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
-  const Geo g = make_geo(a.H, a.I, 2);
-  uint8_t* codes_s = smem + g.codes;
-  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + g.scales);
-  float* act = reinterpret_cast<float*>(smem + g.act);
+  uint8_t* base = smem + kTileOff;
+  const Gv g = make_gv(a.H, a.I, 2);
   const int nrb = a.I / g.R;
   const int rb = blockIdx.x % nrb, u = blockIdx.x / nrb;
   UnitInfo ui;
@@ -365,25 +570,24 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_gate_up(DecodeArgs a) {
     return;
   }
   const int row0 = rb * g.R;
-  stage_rows(g, codes_s, sc_s, blob + a.lay.wg, blob + a.lay.wg_sf, row0);
-  stage_rows(g, codes_s + (size_t)g.R * a.H / 2, sc_s + (size_t)g.R * g.atoms, blob + a.lay.wu, blob + a.lay.wu_sf,
-             row0);
+  stage_mat(g, base, 0, blob + a.lay.wg, blob + a.lay.wg_sf, row0);
+  stage_mat(g, base, 1, blob + a.lay.wu, blob + a.lay.wu_sf, row0);
   cp_async_commit();
   pdl_trigger();
   pdl_wait();  // x is the previous kernel's output when launched as a dependent
-  const int r = threadIdx.x / g.tpr, sub = threadIdx.x % g.tpr;
+  const LaneMap m = lane_map(g);
   for (int t0 = 0; t0 < ui.m; t0 += kMT) {
     const int n = min(kMT, ui.m - t0);
     __syncthreads();
-    stage_act<true>(g, act, a.x, hd.tok + t0, n);
+    stage_x<true>(g, base, a.x, hd.tok + t0, n);
     cp_async_wait_all();
     __syncthreads();
-    float gs[2], us[2];
-    row_dots(g, codes_s, sc_s, act, 0, r, sub, n, gs);
-    row_dots(g, codes_s, sc_s, act, 1, r, sub, n, us);
-    if (sub == 0) {
-      a.h[(size_t)(ui.hbase + t0) * a.I + row0 + r] = silu(gs[0]) * us[0];
-      if (n > 1) a.h[(size_t)(ui.hbase + t0 + 1) * a.I + row0 + r] = silu(gs[1]) * us[1];
+    tile_dots(g, m, base, n);
+    __syncthreads();
+    if (threadIdx.x < g.R * n) {
+      const int t = threadIdx.x / g.R, r = threadIdx.x - t * g.R;
+      a.h[(size_t)(ui.hbase + t0 + t) * a.I + row0 + r] =
+          silu(row_value(g, base, 0, r, t)) * row_value(g, base, 1, r, t);
     }
   }
 }
@@ -392,13 +596,11 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_gate_up(DecodeArgs a) {
 // down + combine: CTA = (unit, block of R rows of Wd), full K = I.  The last
 // CTA to finish a row block (one counter per block) does the weighted combine.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
+__global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
-  const Geo g = make_geo(a.I, a.H, 1);
-  uint8_t* codes_s = smem + g.codes;
-  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + g.scales);
-  float* act = reinterpret_cast<float*>(smem + g.act);
+  uint8_t* base = smem + kTileOff;
+  const Gv g = make_gv(a.I, a.H, 1);
   const int nrb = a.H / g.R;
   const int rb = blockIdx.x % nrb, u = blockIdx.x / nrb;
   UnitInfo ui;
@@ -412,23 +614,23 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
     return;  // already reported by the gate/up kernel
   }
   const int row0 = rb * g.R;
-  stage_rows(g, codes_s, sc_s, blob + a.lay.wd, blob + a.lay.wd_sf, row0);
+  stage_mat(g, base, 0, blob + a.lay.wd, blob + a.lay.wd_sf, row0);
   cp_async_commit();
   pdl_trigger();
   pdl_wait();  // h is written by the gate/up kernel
   if (threadIdx.x < 16) hd.tok[threadIdx.x] = ui.hbase + threadIdx.x;  // h rows of the unit's tokens
-  const int r = threadIdx.x / g.tpr, sub = threadIdx.x % g.tpr;
+  const LaneMap m = lane_map(g);
   for (int t0 = 0; t0 < ui.m; t0 += kMT) {
     const int n = min(kMT, ui.m - t0);
     __syncthreads();
-    stage_act<false>(g, act, a.h, hd.tok + t0, n);
+    stage_x<false>(g, base, a.h, hd.tok + t0, n);
     cp_async_wait_all();
     __syncthreads();
-    float ys[2];
-    row_dots(g, codes_s, sc_s, act, 0, r, sub, n, ys);
-    if (sub == 0) {
-      a.y[(size_t)(ui.hbase + t0) * a.H + row0 + r] = ys[0];
-      if (n > 1) a.y[(size_t)(ui.hbase + t0 + 1) * a.H + row0 + r] = ys[1];
+    tile_dots(g, m, base, n);
+    __syncthreads();
+    if (threadIdx.x < g.R * n) {
+      const int t = threadIdx.x / g.R, r = threadIdx.x - t * g.R;
+      a.y[(size_t)(ui.hbase + t0 + t) * a.H + row0 + r] = row_value(g, base, 0, r, t);
     }
   }
   // last CTA of this row block combines
@@ -444,7 +646,7 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
   __syncthreads();
   if (!hd.last) return;
   __threadfence();
-  for (int i = threadIdx.x; i < a.T * g.R; i += g.threads) {
+  for (int i = threadIdx.x; i < a.T * g.R; i += kGemvThreads) {
     const int t = i / g.R, n = row0 + (i - t * g.R);
     float acc = 0.f;
     for (int j = 0; j < a.k; j++) {
@@ -458,6 +660,296 @@ __global__ void __launch_bounds__(kGemvThreads) k_dec_down(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// persistent stacked decode: one cooperative launch for n_layers layers
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr uint64_t kSpinNs = 2000ull * 1000 * 1000;  // a dependency wait gives up after 2 s
+
+// One tile of a layer as resolved from the routing record: resolving takes a
+// chain of dependent global loads (record -> unit -> pointer table ->
+// permutation), so it is done when the tile's weights are issued, ahead of
+// the wait that precedes its compute.
+struct TileMeta {
+  const uint8_t* blob;  // NULL: the expert is missing
+  int32_t m;            // tokens of the unit
+  int32_t hbase;        // first h / y row of the unit
+  int32_t row0;         // first weight row of the tile
+  int32_t pad;
+  int32_t tok[16];      // gate/up: token ids; down: h rows
+};
+
+// Shared header of the persistent kernel, followed in shared memory by
+// TileMeta first[n_layers][2] (this CTA's first gate/up and first down tile
+// of every layer, resolved before the first layer) and int32 units[n_layers].
+struct StackHdr {
+  TileMeta mx;          // a later tile of the current phase
+  int32_t last;
+  int32_t abort;
+  int32_t pad[2];
+  float cw[kMaxPairs];  // combine weights of the layer, pair order
+  int32_t cpos[kMaxPairs];  // y row of each pair
+};
+
+__host__ __device__ inline size_t stack_hdr_bytes(int n_layers) {
+  return sizeof(StackHdr) + (size_t)n_layers * (2 * sizeof(TileMeta) + sizeof(int32_t));
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t gclock() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void red_add(int* p, int v) {
+  asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int atom_add(int* p, int v) {
+  int old;
+  asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Thread 0 waits (acquire, bounded) until *p >= target, then the CTA
+// synchronises; false (and the timeout status bit) when the wait gave up.
+__device__ bool cta_wait_geq(const int* p, int target, StackHdr& hd, int* status) {
+  if (threadIdx.x == 0 && ld_acquire(p) < target) {
+    const uint64_t t0 = gclock();
+    while (ld_acquire(p) < target) {
+      if (gclock() - t0 > kSpinNs) {
+        set_status(status, kStTimeout);
+        hd.abort = 1;
+        break;
+      }
+      __nanosleep(20);
+    }
+  }
+  __syncthreads();
+  return hd.abort == 0;
+}
+
+// The CTA's global writes so far, then one arrival at *p (release by thread 0
+// after the barrier; the fence is cumulative over the barrier).
+__device__ __forceinline__ void cta_arrive(int* p) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    fence_acq_rel();
+    red_add(p, 1);
+  }
+}
+
+// One warp resolves tile i of a phase (nrb row blocks of R rows per unit) of
+// layer `rec` into m; the caller synchronises before the CTA reads it.
+__device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* rec, const uint8_t* const* eptr, int i,
+                                             int nrb, int R, bool gate_up, TileMeta& m) {
+  const int u = i / nrb, n_act = rec->n_active;
+  int e, cnt, hbase;
+  bool shared;
+  if (u < n_act) {
+    e = rec->unit_e[u];
+    cnt = rec->unit_m[u];
+    hbase = rec->unit_p0[u];
+    shared = false;
+  } else {
+    e = a.E + (u - n_act);
+    cnt = a.T;
+    hbase = a.T * a.k + (u - n_act) * a.T;
+    shared = true;
+  }
+  const int t = threadIdx.x & 31;
+  if (t < cnt) m.tok[t] = !gate_up ? hbase + t : shared ? t : rec->perm[hbase + t] / a.k;
+  if (t == 0) {
+    const uint8_t* blob = eptr[e];
+    m.blob = blob;
+    m.m = cnt;
+    m.hbase = hbase;
+    m.row0 = (i % nrb) * R;
+    if (!blob) set_status(a.status, kStMissing);
+  }
+}
+
+}  // namespace
+
+// Each CTA walks, layer after layer, its gate/up tiles (unit x R rows of Wg and
+// Wu) and then its down tiles (unit x R rows of Wd); tile i of a phase goes to
+// CTA i mod gridDim.  Dependencies between CTAs go through counters in global
+// memory, per layer: gate/up tiles done (down waits for all of them); down
+// tiles done per row block (the last one combines that row block into the
+// layer's output); row blocks combined (the next layer's gate/up waits for all
+// of them).  A CTA streams its next tiles' weights while it waits: the next
+// layer's gate/up tile during the down phase, the next layer's down tile
+// during the gate/up phase.  Activations written by other CTAs are read from
+// L2 only.
+__global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Gv gA = make_gv(a.H, a.I, 2), gB = make_gv(a.I, a.H, 1);
+  uint8_t* baseA = smem;
+  uint8_t* baseB = smem + gA.total;
+  StackHdr& hd = *reinterpret_cast<StackHdr*>(smem + gA.total + gB.total);
+  TileMeta* first = reinterpret_cast<TileMeta*>(&hd + 1);
+  int32_t* units_of = reinterpret_cast<int32_t*>(first + 2 * a.n_layers);
+  const LaneMap lmA = lane_map(gA), lmB = lane_map(gB);
+  const int G = gridDim.x, b = blockIdx.x;
+  const int nrbA = a.I / gA.R, nrbB = a.H / gB.R;
+
+  auto issue_A = [&](const TileMeta& m) {
+    if (m.blob) {
+      stage_mat(gA, baseA, 0, m.blob + a.lay.wg, m.blob + a.lay.wg_sf, m.row0);
+      stage_mat(gA, baseA, 1, m.blob + a.lay.wu, m.blob + a.lay.wu_sf, m.row0);
+    }
+    cp_async_commit();
+  };
+  auto issue_B = [&](const TileMeta& m) {
+    if (m.blob) stage_mat(gB, baseB, 0, m.blob + a.lay.wd, m.blob + a.lay.wd_sf, m.row0);
+    cp_async_commit();
+  };
+
+  // Before the first layer, warp w resolves layers w, w + 16, ...: their
+  // units and this CTA's first tile of each phase.  Every routing record is
+  // complete before the launch.
+  if (threadIdx.x == 0) hd.abort = 0;
+  for (int l = threadIdx.x >> 5; l < a.n_layers; l += kWarps) {
+    const Route* rec = a.rec + l;
+    const uint8_t* const* eptr = a.eptr + (size_t)l * a.n_blobs;
+    const int un = rec->n_active + a.n_shared;
+    if ((threadIdx.x & 31) == 0) units_of[l] = un;
+    if (b < un * nrbA) resolve_tile(a, rec, eptr, b, nrbA, gA.R, true, first[2 * l]);
+    if (b < un * nrbB) resolve_tile(a, rec, eptr, b, nrbB, gB.R, false, first[2 * l + 1]);
+  }
+  __syncthreads();
+  int units = units_of[0];
+  bool preB = b < units * nrbB;
+  if (b < units * nrbA) issue_A(first[0]);
+  if (preB) issue_B(first[1]);
+
+  for (int l = 0; l < a.n_layers; l++) {
+    const Route* rec = a.rec + l;
+    const uint8_t* const* eptr = a.eptr + (size_t)l * a.n_blobs;
+    const int tilesA = units * nrbA, tilesB = units * nrbB;
+    const uint16_t* xin = l == 0 ? a.x0 : a.xbuf[(l - 1) & 1];
+    uint16_t* xout = l == a.n_layers - 1 ? a.out : a.xbuf[l & 1];
+    int* sy = a.sync + (size_t)l * a.sync_stride;
+    // ---------------- gate/up + SwiGLU ----------------
+    for (int i = b; i < tilesA; i += G) {
+      if (i == b) {
+        // the first tile was issued ahead: wait for the previous layer's output
+        if (l > 0 && !cta_wait_geq(a.sync + (size_t)(l - 1) * a.sync_stride + 1, nrbB, hd, a.status)) {
+          cp_async_wait_all();
+          return;
+        }
+      } else {
+        if (threadIdx.x < 32) resolve_tile(a, rec, eptr, i, nrbA, gA.R, true, hd.mx);
+        __syncthreads();
+        issue_A(hd.mx);
+      }
+      const TileMeta& m = i == b ? first[2 * l] : hd.mx;
+      for (int t0 = 0; t0 < m.m; t0 += kMT) {
+        const int n = min(kMT, m.m - t0);
+        if (t0 > 0) __syncthreads();
+        stage_x<true>(gA, baseA, xin, m.tok + t0, n);
+        // the first tile's down weights were issued after it: leave them in flight
+        if (i == b && preB) cp_async_wait_1(); else cp_async_wait_all();
+        __syncthreads();
+        tile_dots(gA, lmA, baseA, n);
+        __syncthreads();
+        if (threadIdx.x < gA.R * n && m.blob) {
+          const int t = threadIdx.x / gA.R, r = threadIdx.x - t * gA.R;
+          a.h[(size_t)(m.hbase + t0 + t) * a.I + m.row0 + r] =
+              silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t);
+        }
+      }
+      cta_arrive(&sy[0]);
+    }
+    // buffer A is free: issue the next layer's first gate/up tile
+    bool nextA = false, nextB = false;
+    int units_n = 0;
+    if (l + 1 < a.n_layers) {
+      units_n = units_of[l + 1];
+      nextA = b < units_n * nrbA;
+      nextB = b < units_n * nrbB;
+      if (nextA) {
+        __syncthreads();
+        issue_A(first[2 * (l + 1)]);
+      }
+    }
+    // ---------------- down + combine ----------------
+    if (b < tilesB) {
+      for (int f = threadIdx.x; f < a.T * a.k; f += kGemvThreads) {
+        hd.cw[f] = rec->w[f];
+        hd.cpos[f] = rec->pos[f];
+      }
+      // every gate/up tile of this layer is done
+      if (!cta_wait_geq(&sy[0], tilesA, hd, a.status)) {
+        cp_async_wait_all();
+        return;
+      }
+      for (int i = b; i < tilesB; i += G) {
+        if (i != b) {
+          __syncthreads();
+          if (threadIdx.x < 32) resolve_tile(a, rec, eptr, i, nrbB, gB.R, false, hd.mx);
+          __syncthreads();
+          issue_B(hd.mx);
+        }
+        const TileMeta& mb = i == b ? first[2 * l + 1] : hd.mx;
+        const int rb = i % nrbB;
+        for (int t0 = 0; t0 < mb.m; t0 += kMT) {
+          const int n = min(kMT, mb.m - t0);
+          if (t0 > 0) __syncthreads();
+          stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
+          // the next layer's gate/up weights were issued after this tile's
+          if (i == b && nextA) cp_async_wait_1(); else cp_async_wait_all();
+          __syncthreads();
+          tile_dots(gB, lmB, baseB, n);
+          __syncthreads();
+          if (threadIdx.x < gB.R * n) {
+            const int t = threadIdx.x / gB.R, r = threadIdx.x - t * gB.R;
+            a.y[(size_t)(mb.hbase + t0 + t) * a.H + mb.row0 + r] = mb.blob ? row_value(gB, baseB, 0, r, t) : 0.f;
+          }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          fence_acq_rel();
+          const int old = atom_add(&sy[2 + rb], 1);
+          hd.last = old == units - 1;
+          if (hd.last) fence_acq_rel();  // acquire the other tiles' y of this row block
+        }
+        __syncthreads();
+        if (hd.last) {
+          const int row0 = mb.row0;
+          for (int q = threadIdx.x; q < a.T * gB.R; q += kGemvThreads) {
+            const int t = q / gB.R, nn = row0 + (q - t * gB.R);
+            float acc = 0.f;
+            for (int j = 0; j < a.k; j++) {
+              const int f = t * a.k + j;
+              acc = fmaf(hd.cw[f], __ldcg(a.y + (size_t)hd.cpos[f] * a.H + nn), acc);
+            }
+            for (int s2 = 0; s2 < a.n_shared; s2++)
+              acc += __ldcg(a.y + (size_t)(a.T * a.k + s2 * a.T + t) * a.H + nn);
+            __nv_bfloat16 bb = __float2bfloat16_rn(acc);
+            xout[(size_t)t * a.H + nn] = *reinterpret_cast<uint16_t*>(&bb);
+          }
+          cta_arrive(&sy[1]);
+        }
+      }
+    }
+    // buffer B is free: issue the next layer's first down tile
+    if (nextB) {
+      __syncthreads();
+      issue_B(first[2 * (l + 1) + 1]);
+    }
+    preB = nextB;
+    units = units_n;
+  }
+  cp_async_wait_all();
+}
+
+// ---------------------------------------------------------------------------
 // routing kernel: CTA l routes layer l and stores its record
 // ---------------------------------------------------------------------------
 template <int PER>
@@ -468,6 +960,8 @@ __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
   const int4* src = reinterpret_cast<const int4*>(&r);
   int4* dst = reinterpret_cast<int4*>(a.rec + l);
   for (int i = threadIdx.x; i < (int)(sizeof(Route) / 16); i += kThreads) dst[i] = src[i];
+  if (a.sync)
+    for (int i = threadIdx.x; i < a.sync_stride; i += kThreads) a.sync[(size_t)l * a.sync_stride + i] = 0;
   if (l == a.n_layers - 1 && a.ids_out) {
     for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
       a.ids_out[f] = r.ids[f];
@@ -479,17 +973,17 @@ __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t decode_smem_bytes(int K, int rows, int nmat) { return make_geo(K, rows, nmat).total; }
-
-static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, const Geo& g, int grid, bool pdl,
-                              cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.total);
+static cudaError_t launch_one(void (*kern)(DecodeArgs), const DecodeArgs& a, const Gv& g, int rows, int grid,
+                              bool pdl, cudaStream_t s) {
+  if (!gv_ok(g, rows)) return cudaErrorInvalidValue;
+  const size_t smem = kTileOff + g.total;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute at[1];
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(g.threads);
+  cfg.blockDim = dim3(kGemvThreads);
   cfg.gridDim = dim3(grid);
-  cfg.dynamicSmemBytes = g.total;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
@@ -511,13 +1005,54 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
-  const Geo g = make_geo(a.H, a.I, 2);
-  return launch_one(k_dec_gate_up, a, g, (a.max_units + a.n_shared) * (a.I / g.R), pdl, s);
+  const Gv g = make_gv(a.H, a.I, 2);
+  return launch_one(k_dec_gate_up, a, g, a.I, (a.max_units + a.n_shared) * (a.I / g.R), pdl, s);
 }
 
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
-  const Geo g = make_geo(a.I, a.H, 1);
-  return launch_one(k_dec_down, a, g, (a.max_units + a.n_shared) * (a.H / g.R), pdl, s);
+  const Gv g = make_gv(a.I, a.H, 1);
+  return launch_one(k_dec_down, a, g, a.H, (a.max_units + a.n_shared) * (a.H / g.R), pdl, s);
+}
+
+bool decode_supported(int H, int I) { return gv_ok(make_gv(H, I, 2), I) && gv_ok(make_gv(I, H, 1), H); }
+
+constexpr size_t kStackSmemMax = 227 * 1024;  // opt-in dynamic shared memory per CTA
+
+bool stack_supported(int H, int I, int n_layers) {
+  const Gv gA = make_gv(H, I, 2), gB = make_gv(I, H, 1);
+  return gv_ok(gA, I) && gv_ok(gB, H) && gA.total + gB.total + stack_hdr_bytes(n_layers) <= kStackSmemMax;
+}
+
+int stack_sync_stride(int H, int I) { return 2 + H / make_gv(I, H, 1).R; }
+
+cudaError_t launch_dec_stack(const StackArgs& a, cudaStream_t s) {
+  if (!stack_supported(a.H, a.I, a.n_layers) || a.sync_stride < stack_sync_stride(a.H, a.I))
+    return cudaErrorInvalidValue;
+  const Gv gA = make_gv(a.H, a.I, 2), gB = make_gv(a.I, a.H, 1);
+  const size_t smem = gA.total + gB.total + stack_hdr_bytes(a.n_layers);
+  cudaError_t e = cudaFuncSetAttribute(k_dec_stack, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 0, occ = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+      (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_dec_stack, kGemvThreads, smem)) != cudaSuccess)
+    return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  // no layer has more tiles than (distinct experts + shared) x row blocks
+  const int units_max = std::min(a.E, a.T * a.k) + a.n_shared;
+  const int tiles_max = units_max * std::max(a.I / gA.R, a.H / gB.R);
+  const int grid = std::min(nsm * occ, tiles_max);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.gridDim = dim3(grid);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_dec_stack, a);
 }
 
 }  // namespace ft

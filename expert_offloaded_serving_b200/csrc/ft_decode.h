@@ -1,7 +1,7 @@
 // Small-batch decode kernels: a routing kernel that writes one compact routing
-// record per layer, then per layer a gate/up + SwiGLU GEMV and a down GEMV with
-// the combine (cp.async-staged FP4 tiles, split-K inside a row's thread group,
-// programmatic dependent launch).
+// record per layer, then either one persistent kernel for a stack of layers or,
+// per layer, a gate/up + SwiGLU GEMV and a down GEMV with the combine
+// (cp.async-staged FP4 tiles, split-K inside a row's thread group).
 #pragma once
 
 #include <cstdint>
@@ -36,6 +36,8 @@ struct RouteArgs {
   int32_t* ids_out;     // [T*k] of the last layer, or NULL
   float* w_out;
   int* status;
+  int* sync;            // [n_layers][sync_stride] zeroed by CTA l for layer l, or NULL
+  int sync_stride;
 };
 
 struct DecodeArgs {
@@ -52,7 +54,9 @@ struct DecodeArgs {
   int* status;
 };
 
-size_t decode_smem_bytes(int K, int rows, int nmat);
+// True when the decode kernels take this shape (hidden and inter multiples of
+// 128, both at most 16384).
+bool decode_supported(int H, int I);
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // pdl: launch as a programmatic dependent of the previous kernel in the
 // stream.  The gate/up kernel reads its routing record and pointer table
@@ -61,5 +65,28 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // nothing produced by gate/up before its wait.
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s);
+
+// Persistent decode over n_layers consecutive layers in one cooperative launch.
+struct StackArgs {
+  const uint16_t* x0;      // bf16 [T][H] input of the first layer
+  uint16_t* out;           // bf16 [T][H] output of the last layer
+  uint16_t* xbuf[2];       // bf16 [T][H] ping-pong between layers
+  const Route* rec;        // [n_layers] routing records
+  const uint8_t* const* eptr;  // [n_layers][n_blobs] blob pointers
+  int n_layers, n_blobs;
+  int T, H, I, E, k, n_shared;
+  BlobLayout lay;
+  float* h;                // [T*k + n_shared*T][I]
+  float* y;                // [T*k + n_shared*T][H]
+  int* sync;               // [n_layers][sync_stride], zero at launch
+  int sync_stride;         // >= stack_sync_stride(H, I)
+  int* status;
+};
+
+// True when the persistent kernel takes this shape and stack depth (both
+// tiles of a layer and the per-layer tile table fit in shared memory).
+bool stack_supported(int H, int I, int n_layers);
+int stack_sync_stride(int H, int I);
+cudaError_t launch_dec_stack(const StackArgs& a, cudaStream_t s);
 
 }  // namespace ft

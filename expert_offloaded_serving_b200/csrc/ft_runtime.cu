@@ -159,6 +159,8 @@ struct ft_ctx {
   Route* d_routes = nullptr;   // decode routing records [L]
   int* d_counters = nullptr;   // decode combine counters [(H/128) * 8]
   uint16_t* d_xbuf[2] = {nullptr, nullptr};  // stack forward ping-pong [T][H]
+  int* d_sync = nullptr;       // persistent stack kernel counters [L][sync_stride]
+  int sync_stride = 0;
   int decode_max_t = 0;
 
   // pinned host scratch
@@ -360,6 +362,10 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
       (st = dev_alloc(&c->d_xbuf[0], (size_t)c->decode_max_t * H)) ||
       (st = dev_alloc(&c->d_xbuf[1], (size_t)c->decode_max_t * H)))
     return bail(st);
+  if (stack_supported(H, I, 1)) {
+    c->sync_stride = stack_sync_stride(H, I);
+    if ((st = dev_alloc(&c->d_sync, (size_t)L * c->sync_stride))) return bail(st);
+  }
   if (cudaMemset(c->d_counters, 0, (size_t)H / 8 * sizeof(int)) != cudaSuccess)
     return bail(fail(FT_ERR_CUDA, "memset"));
   if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return bail(fail(FT_ERR_CUDA, "memset"));
@@ -470,6 +476,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   cudaFree(c->d_routes);
   cudaFree(c->d_xbuf[0]);
   cudaFree(c->d_xbuf[1]);
+  cudaFree(c->d_sync);
   cudaFree(c->d_eptr_res);
   cudaFree(c->d_eptr_cache);
   cudaFree(c->d_shared);
@@ -1069,10 +1076,45 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   if (T == 0) return FT_OK;
   cudaStream_t s = (cudaStream_t)stream;
   const int Ti = (int)T;
-  // all layers' routing records in one launch (their logits are inputs)
+  const bool persistent =
+      !(flags & FT_STACK_LAYERWISE) && c->d_sync != nullptr && stack_supported(c->d.hidden, c->d.inter, n_layers);
+  // all layers' routing records in one launch (their logits are inputs); it
+  // also zeroes the persistent kernel's counters of those layers
   {
     KTimer kt(c, FT_K_TOPK, s);
-    CUDA_TRY(launch_route(route_args(c, logits, Ti, n_layers, flags, c->d_routes + first_layer), s));
+    RouteArgs ra = route_args(c, logits, Ti, n_layers, flags, c->d_routes + first_layer);
+    if (persistent) {
+      ra.sync = c->d_sync;
+      ra.sync_stride = c->sync_stride;
+    }
+    CUDA_TRY(launch_route(ra, s));
+  }
+  if (persistent) {
+    StackArgs a{};
+    a.x0 = (const uint16_t*)x;
+    a.out = (uint16_t*)out;
+    a.xbuf[0] = c->d_xbuf[0];
+    a.xbuf[1] = c->d_xbuf[1];
+    a.rec = c->d_routes + first_layer;
+    a.eptr = c->d_eptr_res + (size_t)first_layer * c->n_blobs;
+    a.n_layers = n_layers;
+    a.n_blobs = c->n_blobs;
+    a.T = Ti;
+    a.H = c->d.hidden;
+    a.I = c->d.inter;
+    a.E = c->d.n_experts;
+    a.k = c->d.top_k;
+    a.n_shared = c->d.n_shared;
+    a.lay = c->lay;
+    a.h = c->d_h;
+    a.y = c->d_y;
+    a.sync = c->d_sync;
+    a.sync_stride = c->sync_stride;
+    a.status = c->d_status;
+    KTimer kt(c, FT_K_DEC_STACK, s);
+    CUDA_TRY(launch_dec_stack(a, s));
+    c->last_stream = s;
+    return FT_OK;
   }
   const uint16_t* cur = (const uint16_t*)x;
   for (int i = 0; i < n_layers; i++) {

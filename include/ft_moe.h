@@ -82,6 +82,7 @@ typedef struct {
 #define FT_ROUTE_RENORM 1u    /* renormalise the k softmax weights to sum 1 (default on) */
 #define FT_ACT_BF16     0u    /* decode: bf16 activations, fp32 h, split-K FP4 GEMV */
 #define FT_ACT_MXFP4    2u    /* prefill: x and h quantised to MXFP4, tcgen05 grouped GEMM */
+#define FT_STACK_LAYERWISE 4u /* ft_moe_stack_forward: two kernels per layer, not the persistent kernel */
 
 /* cache trace events */
 #define FT_EV_HIT   0
@@ -224,11 +225,18 @@ FT_API ft_status ft_moe_layer_forward(ft_ctx* ctx, int32_t layer, const void* x,
  *   x dev bf16 [T][H] (input of first_layer), out dev bf16 [T][H] (output of
  *   the last layer; must not alias x); logits dev fp32 [n_layers][T][E]
  *   (router logits of each layer, all ready before the call).
- * Each layer is the ft_moe_layer_forward decode path.  Because every layer's
- * routing input is known up front, a layer's kernels are launched as
- * programmatic dependents of the previous layer's, so its routing and weight
- * streaming overlap the previous layer's tail; intermediate activations live
- * in context scratch.  flags: FT_ROUTE_RENORM.
+ * Each layer computes what the ft_moe_layer_forward decode path computes, bit
+ * for bit.  Because every layer's routing input is known up front, one
+ * kernel routes all layers first.  Then, by default, one persistent
+ * cooperative kernel runs every layer: each CTA takes its gate/up tile and its
+ * down tile of a layer in turn, streams its next tiles' weights while it waits
+ * for the layer's other CTAs, and layers hand over through counters in global
+ * memory (waits bounded at 2 s; a timeout sets FT_ERR_TIMEOUT's status bit).
+ * With FT_STACK_LAYERWISE, or for shapes whose two tiles do not fit one CTA's
+ * shared memory, each layer runs as a gate/up and a down kernel instead, the
+ * next layer's launched as programmatic dependents of the previous layer's.
+ * Intermediate activations live in context scratch; calls on different
+ * streams must not overlap.  flags: FT_ROUTE_RENORM | FT_STACK_LAYERWISE.
  * Errors: FT_ERR_INVALID, FT_ERR_STATE (a layer is not resident), FT_ERR_CUDA. */
 FT_API ft_status ft_moe_stack_forward(ft_ctx* ctx, int32_t first_layer, int32_t n_layers, const void* x, int64_t T,
                                       const float* logits, void* out, uint32_t flags, void* stream);
@@ -304,7 +312,8 @@ FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, fl
 #define FT_K_GEMM_GATE_UP  6   /* prefill grouped GEMM, gate/up + SwiGLU + quantise h */
 #define FT_K_GEMM_DOWN     7   /* prefill grouped GEMM, down */
 #define FT_K_COMBINE       8   /* prefill combine */
-#define FT_K_COUNT         9
+#define FT_K_DEC_STACK     9   /* persistent decode kernel over a stack of layers */
+#define FT_K_COUNT         10
 
 /* Turn per-kernel CUDA-event timing on (1) or off (0).  While on, every
  * kernel launch of the forward path is bracketed by events on its stream (and

@@ -132,20 +132,37 @@ def test_fused_routing_ties_and_no_renorm():
             assert np.allclose(w.cpu().numpy().reshape(T, k), ww, rtol=2e-6, atol=1e-9)
 
 
-@pytest.mark.parametrize("T", [1, 4])
-def test_stack_forward_matches_layer_by_layer(T):
-    H, I, E, k, S, L, seed = 2048, 512, 256, 8, 1, 3, 1002
+STACK_SHAPES = {
+    # name: H, I, E, k, S, seed
+    "35b": (2048, 512, 256, 8, 1, 1002),
+    "no_shared": (1024, 512, 64, 4, 0, 1004),
+    "narrow_down": (1024, 768, 64, 4, 1, 1005),   # down tile of 256 threads
+    "dsv4": (4096, 2048, 256, 6, 0, 1003),
+}
+
+
+def stack_case(name, T, L):
+    H, I, E, k, S, seed = STACK_SHAPES[name]
     pools = [synth.gpu.layer_pool(H, I, E + S, seed, l) for l in range(L)]
     lgs = []
     for l in range(L):
         sets = np.stack([synth.zipf_trace(seed, l, 3, E, k, 1.1, 0.6, stream=t)[-1] for t in range(T)])
         lgs.append(synth.logits_for_sets(seed, 10 + l, sets, E))
+    return (H, I, E, k, S, seed), pools, lgs
+
+
+@pytest.mark.parametrize("name,T", [("35b", 1), ("35b", 4), ("35b", 16), ("no_shared", 1), ("no_shared", 16),
+                                    ("narrow_down", 3), ("dsv4", 2)])
+@pytest.mark.parametrize("flags", [1, 1 | ft.FT_STACK_LAYERWISE], ids=["persistent", "layerwise"])
+def test_stack_forward_matches_layer_by_layer(name, T, flags):
+    L = 3
+    (H, I, E, k, S, seed), pools, lgs = stack_case(name, T, L)
     lg_all = torch.from_numpy(np.stack(lgs)).cuda()
     xb = synth.activations_bf16(seed, 1, T, H)
     with Ctx(ft.make_desc(H, I, E, k, L, S, 0, 16), None, pools) as c:
         x = x_dev(xb)
         out = torch.empty_like(x)
-        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, out, 1)
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, out, flags)
         ft.ft_sync_status(c.h)
         cur = x
         inputs = []
@@ -156,6 +173,14 @@ def test_stack_forward_matches_layer_by_layer(T):
             cur = nxt
         torch.cuda.synchronize()
         assert (bf16_bits(out) == bf16_bits(cur)).all()
+        # the routing the stack leaves behind is the last layer's
+        ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T * k, dtype=torch.float32, device="cuda")
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, out, flags)
+        ft.ft_last_routing(c.h, ids, w, T * k)
+        torch.cuda.synchronize()
+        want, _ = olayer.routing.topk(lgs[-1], k)
+        assert (ids.cpu().numpy().reshape(T, k) == want).all()
     # layer-local parity of the last layer against the oracle
     blobs = {}
 
@@ -163,5 +188,34 @@ def test_stack_forward_matches_layer_by_layer(T):
         if e not in blobs:
             blobs[e] = synth.expert_blob(seed, L - 1, e, H, I)
         return blobs[e]
-    r = olayer.moe_layer(inputs[-1], blob_of, H, I, E, k, logits=lgs[-1], shared_blob=blob_of(E))
+    r = olayer.moe_layer(inputs[-1], blob_of, H, I, E, k, logits=lgs[-1], shared_blob=blob_of(E) if S else None)
     assert_close(bf16_bits(out), r["out_f64"])
+
+
+def test_stack_forward_repeated_and_sub_stacks():
+    """Back-to-back persistent launches reuse the counters (zeroed by the
+    routing kernel): 40 layers at once equal the same layers run as two
+    sub-stacks, and a second identical call gives identical bits."""
+    L, T = 40, 2
+    (H, I, E, k, S, seed), pools, lgs = stack_case("35b", T, L)
+    lg_all = torch.from_numpy(np.stack(lgs)).cuda()
+    xb = synth.activations_bf16(seed, 1, T, H)
+    with Ctx(ft.make_desc(H, I, E, k, L, S, 0, 16), None, pools) as c:
+        x = x_dev(xb)
+        a = torch.empty_like(x)
+        b = torch.empty_like(x)
+        mid = torch.empty_like(x)
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, a, 1)
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, b, 1)
+        ft.ft_sync_status(c.h)
+        torch.cuda.synchronize()
+        assert (bf16_bits(a) == bf16_bits(b)).all()
+        ft.ft_moe_stack_forward(c.h, 0, 17, x, T, lg_all[:17].contiguous(), mid, 1)
+        ft.ft_moe_stack_forward(c.h, 17, L - 17, mid, T, lg_all[17:].contiguous(), b, 1)
+        ft.ft_sync_status(c.h)
+        torch.cuda.synchronize()
+        assert (bf16_bits(a) == bf16_bits(b)).all()
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, b, 1 | ft.FT_STACK_LAYERWISE)
+        ft.ft_sync_status(c.h)
+        torch.cuda.synchronize()
+        assert (bf16_bits(a) == bf16_bits(b)).all()
