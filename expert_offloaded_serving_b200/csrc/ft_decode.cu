@@ -245,7 +245,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Shared memory, from the tile's base:
 //   codes  [nmat][R][K/2]        as in global memory (16-byte cp.async copies)
 //   scales [nmat][R][K/128]      words of four blocks' UE8M0 bytes
-//   xh     [kMT][K]              activations, f16
+//   xh     [kMT][4][K/32] x 16 B  activations, f16: quad i of chunk c at [t][i][c]
 //   xinv   [kMT][K/32]           inverse block factors
 //   red    [parts][nmat][R][kMT] partial sums
 // ---------------------------------------------------------------------------
@@ -316,6 +316,16 @@ __device__ __forceinline__ LaneMap lane_map(const Gv& g) {
   return m;
 }
 
+// Scale words of rows [row0, row0 + R) of matrix `mat` (scale region sc_g),
+// one 4-byte cp.async each.
+__device__ __forceinline__ void stage_scales(const Gv& g, uint8_t* base, int mat, const uint8_t* sc_g, int row0) {
+  uint32_t* sd = reinterpret_cast<uint32_t*>(base + g.scales) + (size_t)mat * g.R * g.atoms;
+  for (int i = threadIdx.x; i < g.R * g.atoms; i += kGemvThreads) {
+    const int r = i / g.atoms, at = i - r * g.atoms;
+    cp_async4(sd + i, sc_g + sf_word(row0 + r, at, g.atoms));
+  }
+}
+
 // Stage rows [row0, row0 + R) of matrix `mat` (codes at codes_g, row pitch
 // K/2; scale region sc_g) into the tile with cp.async.
 __device__ __forceinline__ void stage_mat(const Gv& g, uint8_t* base, int mat, const uint8_t* codes_g,
@@ -324,62 +334,61 @@ __device__ __forceinline__ void stage_mat(const Gv& g, uint8_t* base, int mat, c
   const uint8_t* src = codes_g + (size_t)row0 * (g.K / 2);
   const int n16 = g.R * g.chunks;
   for (int i = threadIdx.x; i < n16; i += kGemvThreads) cp_async16(dst + (size_t)i * 16, src + (size_t)i * 16);
-  uint32_t* sd = reinterpret_cast<uint32_t*>(base + g.scales) + (size_t)mat * g.R * g.atoms;
-  for (int i = threadIdx.x; i < g.R * g.atoms; i += kGemvThreads) {
-    const int r = i / g.atoms, at = i - r * g.atoms;
-    cp_async4(sd + i, sc_g + sf_word(row0 + r, at, g.atoms));
-  }
+  stage_scales(g, base, mat, sc_g, row0);
+}
+
+// Encode 4 consecutive activations v (group q of token t) into the tile's f16
+// activations; the 8 lanes of a 32-element block agree on its factor by
+// shuffles, so all 32 lanes of the warp must call this together.
+__device__ __forceinline__ void encode4(const Gv& g, uint8_t* base, int t, int q, const float (&v)[4]) {
+  uint2* xh = reinterpret_cast<uint2*>(base + g.xh);
+  float* xinv = reinterpret_cast<float*>(base + g.xinv);
+  uint32_t e = 0;
+#pragma unroll
+  for (int j = 0; j < 4; j++) e = max(e, __float_as_uint(v[j]) & 0x7f800000u);
+  e = max(e, __shfl_xor_sync(0xffffffffu, e, 1));
+  e = max(e, __shfl_xor_sync(0xffffffffu, e, 2));
+  e = max(e, __shfl_xor_sync(0xffffffffu, e, 4));
+  // largest biased exponent of the block, at least 15 so that both factors
+  // are normal floats: 2^(141-eb) maps the block's maximum into [2^14, 2^15)
+  const int eb = max((int)(e >> 23), 15);
+  const float f = __uint_as_float((uint32_t)(268 - eb) << 23);
+  __half2 h0 = __float22half2_rn(make_float2(v[0] * f, v[1] * f));
+  __half2 h1 = __float22half2_rn(make_float2(v[2] * f, v[3] * f));
+  // quad i (16 bytes) of chunk c sits at [t][i][c], so that the lanes of a
+  // warp, one chunk each, read consecutive 16-byte words
+  const int c = q >> 3, i = (q & 7) >> 1;
+  xh[(size_t)t * (g.K / 4) + 2 * ((size_t)i * g.chunks + c) + (q & 1)] =
+      make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+  if ((q & 7) == 0) xinv[t * g.chunks + c] = __uint_as_float((uint32_t)(eb - 14) << 23);
 }
 
 // Re-encode tokens rows[0 .. n) of a bf16 (x) or fp32 (h) matrix with row
-// length K into the tile's f16 activations (read from L2).  Thread i takes 8
-// consecutive elements; the 4 threads of a 32-element block agree on its
-// factor by shuffles.  Tokens n .. kMT-1 are zero.
+// length K into the tile's f16 activations (read from L2).  Thread i takes 4
+// consecutive elements.  Tokens n .. kMT-1 are zero.
 template <bool BF16>
 __device__ __forceinline__ void stage_x(const Gv& g, uint8_t* base, const void* src, const int* rows, int n) {
-  uint4* xh = reinterpret_cast<uint4*>(base + g.xh);
-  float* xinv = reinterpret_cast<float*>(base + g.xinv);
-  const int per = g.K / 8;
+  const int per = g.K / 4;
   // kMT * per is a multiple of 32: a warp is wholly inside or outside
   for (int i = threadIdx.x; i < kMT * per; i += kGemvThreads) {
     const int t = i / per, q = i - t * per;
-    float v[8];
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (t < n) {
       if (BF16) {
-        const uint4 w = __ldcg(reinterpret_cast<const uint4*>((const uint16_t*)src + (size_t)rows[t] * g.K) + q);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-          v[2 * j] = __uint_as_float(ws[j] << 16);
-          v[2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
-        }
+        const uint2 w = __ldcg(reinterpret_cast<const uint2*>((const uint16_t*)src + (size_t)rows[t] * g.K) + q);
+        v[0] = __uint_as_float(w.x << 16);
+        v[1] = __uint_as_float(w.x & 0xffff0000u);
+        v[2] = __uint_as_float(w.y << 16);
+        v[3] = __uint_as_float(w.y & 0xffff0000u);
       } else {
-        const float4* p = reinterpret_cast<const float4*>((const float*)src + (size_t)rows[t] * g.K) + 2 * q;
-        const float4 a = __ldcg(p), b = __ldcg(p + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        const float4 u = __ldcg(reinterpret_cast<const float4*>((const float*)src + (size_t)rows[t] * g.K) + q);
+        v[0] = u.x;
+        v[1] = u.y;
+        v[2] = u.z;
+        v[3] = u.w;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; j++) v[j] = 0.f;
     }
-    uint32_t e = 0;
-#pragma unroll
-    for (int j = 0; j < 8; j++) e = max(e, __float_as_uint(v[j]) & 0x7f800000u);
-    e = max(e, __shfl_xor_sync(0xffffffffu, e, 1));
-    e = max(e, __shfl_xor_sync(0xffffffffu, e, 2));
-    // largest biased exponent of the block, at least 15 so that both factors
-    // are normal floats: 2^(141-eb) maps the block's maximum into [2^14, 2^15)
-    const int eb = max((int)(e >> 23), 15);
-    const float f = __uint_as_float((uint32_t)(268 - eb) << 23);
-    uint32_t h[4];
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      __half2 hh = __float22half2_rn(make_float2(v[2 * j] * f, v[2 * j + 1] * f));
-      h[j] = *reinterpret_cast<uint32_t*>(&hh);
-    }
-    xh[(size_t)t * per + q] = make_uint4(h[0], h[1], h[2], h[3]);
-    if ((q & 3) == 0) xinv[t * g.chunks + (q >> 2)] = __uint_as_float((uint32_t)(eb - 14) << 23);
+    encode4(g, base, t, q, v);
   }
 }
 
@@ -508,15 +517,20 @@ __device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t
     const float* xinv = reinterpret_cast<const float*>(base + g.xinv);
 #pragma unroll
     for (int t = 0; t < kMT; t++) {
+      if (t < n) {
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const uint4 u = xh[((size_t)t * g.K + m.c * 32) / 8 + i];
-        x[t][4 * i] = u.x;
-        x[t][4 * i + 1] = u.y;
-        x[t][4 * i + 2] = u.z;
-        x[t][4 * i + 3] = u.w;
+        for (int i = 0; i < 4; i++) {
+          const uint4 u = xh[(size_t)t * (g.K / 8) + (size_t)i * g.chunks + m.c];
+          x[t][4 * i] = u.x;
+          x[t][4 * i + 1] = u.y;
+          x[t][4 * i + 2] = u.z;
+          x[t][4 * i + 3] = u.w;
+        }
+        xi[t] = xinv[t * g.chunks + m.c];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) x[t][i] = 0u;
       }
-      xi[t] = xinv[t * g.chunks + m.c];
     }
   } else {
 #pragma unroll
@@ -683,6 +697,7 @@ struct TileMeta {
 // TileMeta first[n_layers][2] (this CTA's first gate/up and first down tile
 // of every layer, resolved before the first layer) and int32 units[n_layers].
 struct StackHdr {
+  uint64_t bar[2];      // completion of the bulk weight copies into buffers A and B
   TileMeta mx;          // a later tile of the current phase
   int32_t last;
   int32_t abort;
@@ -716,6 +731,39 @@ __device__ __forceinline__ int atom_add(int* p, int v) {
 }
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
+__device__ __forceinline__ void mbar_init(uint64_t* bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase with this parity; false (and the timeout status
+// bit) when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = gclock();
+  while (!mbar_try(bar, parity)) {
+    if (gclock() - t0 > kSpinNs) {
+      set_status(status, kStTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+// One contiguous global -> shared copy by the bulk-copy engine, completing on bar.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // Thread 0 waits (acquire, bounded) until *p >= target, then the CTA
 // synchronises; false (and the timeout status bit) when the wait gave up.
 __device__ bool cta_wait_geq(const int* p, int target, StackHdr& hd, int* status) {
@@ -734,13 +782,80 @@ __device__ bool cta_wait_geq(const int* p, int target, StackHdr& hd, int* status
   return hd.abort == 0;
 }
 
-// The CTA's global writes so far, then one arrival at *p (release by thread 0
-// after the barrier; the fence is cumulative over the barrier).
+// Lane 0 of the last warp publishes arrivals, so that thread 0, which polls,
+// goes on to its next wait without waiting for the fence.
+constexpr int kArriver = kGemvThreads - 32;
+// Lane 0 of warp 1 issues the bulk weight copies.
+constexpr int kIssuer = 32;
+
+// The CTA's global writes so far, then one arrival at *p (after the barrier,
+// a fence by the arriving thread is cumulative over the CTA's writes).  The
+// arriver's warp issues nothing more until the fence is done, so that the
+// fence does not also wait for the warp's next loads; the other warps go on.
 __device__ __forceinline__ void cta_arrive(int* p) {
   __syncthreads();
-  if (threadIdx.x == 0) {
-    fence_acq_rel();
-    red_add(p, 1);
+  if ((threadIdx.x >> 5) == (kArriver >> 5)) {
+    if (threadIdx.x == kArriver) {
+      fence_acq_rel();
+      red_add(p, 1);
+    }
+    __syncwarp();
+  }
+}
+
+// out[t][n] = bf16( sum_j w[t][j] * y[pos[t][j]][n]  (j ascending, fused)
+//                   + sum_s y[T*k + s*T + t][n] ) for 4 consecutive n (group q)
+// of row length H; the same arithmetic as the combine of the per-layer kernels.
+__device__ __forceinline__ void combine4(const float* y, const float* cw, const int* cpos, int tok, int q, int H, int T,
+                                         int k, int S, float (&v)[4]) {
+  constexpr int kBatch = 8;  // rows in flight at once
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // the shared expert's row is loaded with the first batch and added last
+  float4 sh = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (S > 0) sh = __ldcg(reinterpret_cast<const float4*>(y + (size_t)(T * k + tok) * H) + q);
+  for (int j0 = 0; j0 < k; j0 += kBatch) {
+    float4 u[kBatch];
+    float w[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; j++) {
+      if (j0 + j < k) {
+        const int f = tok * k + j0 + j;
+        w[j] = cw[f];
+        u[j] = __ldcg(reinterpret_cast<const float4*>(y + (size_t)cpos[f] * H) + q);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; j++) {
+      if (j0 + j < k) {
+        acc[0] = fmaf(w[j], u[j].x, acc[0]);
+        acc[1] = fmaf(w[j], u[j].y, acc[1]);
+        acc[2] = fmaf(w[j], u[j].z, acc[2]);
+        acc[3] = fmaf(w[j], u[j].w, acc[3]);
+      }
+    }
+  }
+  for (int s2 = 0; s2 < S; s2++) {
+    const float4 u = s2 == 0 ? sh : __ldcg(reinterpret_cast<const float4*>(y + (size_t)(T * k + s2 * T + tok) * H) + q);
+    acc[0] += u.x;
+    acc[1] += u.y;
+    acc[2] += u.z;
+    acc[3] += u.w;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; e++) v[e] = __bfloat162float(__float2bfloat16_rn(acc[e]));
+}
+
+// The gate/up activations of tokens toks[0 .. n) rebuilt from the previous
+// layer's y (the layer input is that layer's combined output), re-encoded like
+// stage_x.
+__device__ __forceinline__ void stage_comb(const Gv& g, uint8_t* base, const StackArgs& a, const float* cw,
+                                           const int* cpos, const int* toks, int n) {
+  const int per = g.K / 4;
+  for (int i = threadIdx.x; i < kMT * per; i += kGemvThreads) {
+    const int t = i / per, q = i - t * per;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (t < n) combine4(a.y, cw, cpos, toks[t], q, a.H, a.T, a.k, a.n_shared, v);
+    encode4(g, base, t, q, v);
   }
 }
 
@@ -779,13 +894,16 @@ __device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* re
 // Each CTA walks, layer after layer, its gate/up tiles (unit x R rows of Wg and
 // Wu) and then its down tiles (unit x R rows of Wd); tile i of a phase goes to
 // CTA i mod gridDim.  Dependencies between CTAs go through counters in global
-// memory, per layer: gate/up tiles done (down waits for all of them); down
-// tiles done per row block (the last one combines that row block into the
-// layer's output); row blocks combined (the next layer's gate/up waits for all
-// of them).  A CTA streams its next tiles' weights while it waits: the next
-// layer's gate/up tile during the down phase, the next layer's down tile
-// during the gate/up phase.  Activations written by other CTAs are read from
-// L2 only.
+// memory.  Per layer: [0] gate/up tiles done (down waits for all of them);
+// [1] down tiles done (fused combine) or row blocks combined; [2 + rb] down
+// tiles done in row block rb.  With the fused combine (a.fused, few tokens)
+// the next layer's gate/up tiles rebuild their input from y themselves, so a
+// layer hands over after its last down tile; otherwise the last down tile of
+// a row block combines that block into the layer output and the next layer
+// waits for every row block.  A CTA streams its next tiles' weights while it
+// waits: the next layer's gate/up tile during the down phase, the next
+// layer's down tile during the gate/up phase.  Activations written by other
+// CTAs are read from L2 only.
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Gv gA = make_gv(a.H, a.I, 2), gB = make_gv(a.I, a.H, 1);
@@ -797,23 +915,64 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   const LaneMap lmA = lane_map(gA), lmB = lane_map(gB);
   const int G = gridDim.x, b = blockIdx.x;
   const int nrbA = a.I / gA.R, nrbB = a.H / gB.R;
+  const bool fused = a.fused != 0;
 
+  // A tile's codes (R contiguous rows per matrix) arrive by bulk copies that
+  // one thread issues and that complete on the buffer's mbarrier; its scale
+  // words by 4-byte cp.async from every thread (one commit group per tile).
+  uint32_t phase[2] = {0u, 0u};     // parity of each buffer's next phase
+  bool pending[2] = {false, false};  // a tile issued into the buffer and not waited for
+  auto issue_codes = [&](int buf, const Gv& g, uint8_t* base, const uint8_t* m0, const uint8_t* m1, int row0) {
+    if (threadIdx.x == kIssuer) {
+      const uint32_t bytes = (uint32_t)g.R * (uint32_t)(g.K / 2);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(&hd.bar[buf], m0 ? bytes * (m1 ? 2u : 1u) : 0u);
+      if (m0) bulk_g2s(base + g.codes, m0 + (size_t)row0 * (g.K / 2), bytes, &hd.bar[buf]);
+      if (m0 && m1) bulk_g2s(base + g.codes + bytes, m1 + (size_t)row0 * (g.K / 2), bytes, &hd.bar[buf]);
+    }
+    pending[buf] = true;
+  };
   auto issue_A = [&](const TileMeta& m) {
+    issue_codes(0, gA, baseA, m.blob ? m.blob + a.lay.wg : nullptr, m.blob ? m.blob + a.lay.wu : nullptr, m.row0);
     if (m.blob) {
-      stage_mat(gA, baseA, 0, m.blob + a.lay.wg, m.blob + a.lay.wg_sf, m.row0);
-      stage_mat(gA, baseA, 1, m.blob + a.lay.wu, m.blob + a.lay.wu_sf, m.row0);
+      stage_scales(gA, baseA, 0, m.blob + a.lay.wg_sf, m.row0);
+      stage_scales(gA, baseA, 1, m.blob + a.lay.wu_sf, m.row0);
     }
     cp_async_commit();
   };
   auto issue_B = [&](const TileMeta& m) {
-    if (m.blob) stage_mat(gB, baseB, 0, m.blob + a.lay.wd, m.blob + a.lay.wd_sf, m.row0);
+    issue_codes(1, gB, baseB, m.blob ? m.blob + a.lay.wd : nullptr, nullptr, m.row0);
+    if (m.blob) stage_scales(gB, baseB, 0, m.blob + a.lay.wd_sf, m.row0);
     cp_async_commit();
+  };
+  // every thread waits for buffer buf's codes; a timeout marks the CTA aborted
+  auto wait_codes = [&](int buf) {
+    if (!mbar_wait(&hd.bar[buf], phase[buf], a.status)) hd.abort = 1;
+    phase[buf] ^= 1u;
+    pending[buf] = false;
+  };
+  // before an early return: let the copies in flight land (bounded)
+  auto drain = [&]() {
+    for (int buf = 0; buf < 2; buf++)
+      if (pending[buf]) mbar_wait(&hd.bar[buf], phase[buf], a.status);
+    cp_async_wait_all();
+  };
+  auto load_combine = [&](const Route* rec) {  // combine weights and y rows of a layer
+    for (int f = threadIdx.x; f < a.T * a.k; f += kGemvThreads) {
+      hd.cw[f] = rec->w[f];
+      hd.cpos[f] = rec->pos[f];
+    }
   };
 
   // Before the first layer, warp w resolves layers w, w + 16, ...: their
   // units and this CTA's first tile of each phase.  Every routing record is
   // complete before the launch.
-  if (threadIdx.x == 0) hd.abort = 0;
+  if (threadIdx.x == 0) {
+    hd.abort = 0;
+    mbar_init(&hd.bar[0]);
+    mbar_init(&hd.bar[1]);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   for (int l = threadIdx.x >> 5; l < a.n_layers; l += kWarps) {
     const Route* rec = a.rec + l;
     const uint8_t* const* eptr = a.eptr + (size_t)l * a.n_blobs;
@@ -828,20 +987,42 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   if (b < units * nrbA) issue_A(first[0]);
   if (preB) issue_B(first[1]);
 
+  // Prefetch order: a layer's first down tile is issued once its gate/up wait
+  // returns, the next layer's first gate/up tile once the down wait returns,
+  // so each streams in during a compute phase and no arrival's fence runs
+  // while weight copies of this CTA are in flight.
+  bool issuedB = preB;  // layer 0's down tile went out at the start
   for (int l = 0; l < a.n_layers; l++) {
     const Route* rec = a.rec + l;
     const uint8_t* const* eptr = a.eptr + (size_t)l * a.n_blobs;
     const int tilesA = units * nrbA, tilesB = units * nrbB;
+    const bool haveA = b < tilesA, haveB = b < tilesB;
     const uint16_t* xin = l == 0 ? a.x0 : a.xbuf[(l - 1) & 1];
     uint16_t* xout = l == a.n_layers - 1 ? a.out : a.xbuf[l & 1];
     int* sy = a.sync + (size_t)l * a.sync_stride;
+    const int units_n = l + 1 < a.n_layers ? units_of[l + 1] : 0;
+    const bool nextA = b < units_n * nrbA;
+    // the combine weights this layer uses: the previous layer's for the fused
+    // gate/up input, else this layer's for its row-block combines
+    if (fused ? l > 0 : haveB) load_combine(fused ? rec - 1 : rec);
+    if (haveB && !haveA && !issuedB) {
+      issue_B(first[2 * l + 1]);
+      issuedB = true;
+    }
     // ---------------- gate/up + SwiGLU ----------------
     for (int i = b; i < tilesA; i += G) {
       if (i == b) {
-        // the first tile was issued ahead: wait for the previous layer's output
-        if (l > 0 && !cta_wait_geq(a.sync + (size_t)(l - 1) * a.sync_stride + 1, nrbB, hd, a.status)) {
-          cp_async_wait_all();
-          return;
+        // the first tile was issued ahead: wait for the previous layer
+        if (l > 0) {
+          const int* prev = a.sync + (size_t)(l - 1) * a.sync_stride + 1;
+          if (!cta_wait_geq(prev, fused ? units_of[l - 1] * nrbB : nrbB, hd, a.status)) {
+            drain();
+            return;
+          }
+        }
+        if (haveB && !issuedB) {
+          issue_B(first[2 * l + 1]);
+          issuedB = true;
         }
       } else {
         if (threadIdx.x < 32) resolve_tile(a, rec, eptr, i, nrbA, gA.R, true, hd.mx);
@@ -851,11 +1032,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
       const TileMeta& m = i == b ? first[2 * l] : hd.mx;
       for (int t0 = 0; t0 < m.m; t0 += kMT) {
         const int n = min(kMT, m.m - t0);
-        if (t0 > 0) __syncthreads();
-        stage_x<true>(gA, baseA, xin, m.tok + t0, n);
-        // the first tile's down weights were issued after it: leave them in flight
-        if (i == b && preB) cp_async_wait_1(); else cp_async_wait_all();
         __syncthreads();
+        if (fused && l > 0) stage_comb(gA, baseA, a, hd.cw, hd.cpos, m.tok + t0, n);
+        else stage_x<true>(gA, baseA, xin, m.tok + t0, n);
+        // the first tile's down weights were issued after it: leave them in flight
+        if (i == b && haveB) cp_async_wait_1(); else cp_async_wait_all();
+        if (t0 == 0) wait_codes(0);
+        __syncthreads();
+        if (hd.abort) {
+          drain();
+          return;
+        }
         tile_dots(gA, lmA, baseA, n);
         __syncthreads();
         if (threadIdx.x < gA.R * n && m.blob) {
@@ -866,29 +1053,20 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
       }
       cta_arrive(&sy[0]);
     }
-    // buffer A is free: issue the next layer's first gate/up tile
-    bool nextA = false, nextB = false;
-    int units_n = 0;
-    if (l + 1 < a.n_layers) {
-      units_n = units_of[l + 1];
-      nextA = b < units_n * nrbA;
-      nextB = b < units_n * nrbB;
-      if (nextA) {
-        __syncthreads();
-        issue_A(first[2 * (l + 1)]);
-      }
+    // without a down phase, the next layer's first gate/up tile goes out now
+    if (!haveB && nextA) {
+      __syncthreads();
+      issue_A(first[2 * (l + 1)]);
     }
-    // ---------------- down + combine ----------------
-    if (b < tilesB) {
-      for (int f = threadIdx.x; f < a.T * a.k; f += kGemvThreads) {
-        hd.cw[f] = rec->w[f];
-        hd.cpos[f] = rec->pos[f];
-      }
+    // ---------------- down (+ row-block combine) ----------------
+    if (haveB) {
       // every gate/up tile of this layer is done
       if (!cta_wait_geq(&sy[0], tilesA, hd, a.status)) {
-        cp_async_wait_all();
+        drain();
         return;
       }
+      // buffer A is free since the gate/up phase
+      if (nextA) issue_A(first[2 * (l + 1)]);
       for (int i = b; i < tilesB; i += G) {
         if (i != b) {
           __syncthreads();
@@ -904,7 +1082,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
           stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
           // the next layer's gate/up weights were issued after this tile's
           if (i == b && nextA) cp_async_wait_1(); else cp_async_wait_all();
+          if (t0 == 0) wait_codes(1);
           __syncthreads();
+          if (hd.abort) {
+            drain();
+            return;
+          }
           tile_dots(gB, lmB, baseB, n);
           __syncthreads();
           if (threadIdx.x < gB.R * n) {
@@ -912,8 +1095,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
             a.y[(size_t)(mb.hbase + t0 + t) * a.H + mb.row0 + r] = mb.blob ? row_value(gB, baseB, 0, r, t) : 0.f;
           }
         }
+        if (fused) {
+          cta_arrive(&sy[1]);
+          continue;
+        }
         __syncthreads();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == kArriver) {
           fence_acq_rel();
           const int old = atom_add(&sy[2 + rb], 1);
           hd.last = old == units - 1;
@@ -938,15 +1125,26 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         }
       }
     }
-    // buffer B is free: issue the next layer's first down tile
-    if (nextB) {
-      __syncthreads();
-      issue_B(first[2 * (l + 1) + 1]);
-    }
-    preB = nextB;
+    issuedB = false;
     units = units_n;
   }
   cp_async_wait_all();
+  // fused combine: CTA 0 writes the last layer's output once its down tiles are done
+  if (fused && b == 0) {
+    const int L = a.n_layers;
+    __syncthreads();
+    load_combine(a.rec + L - 1);
+    if (!cta_wait_geq(a.sync + (size_t)(L - 1) * a.sync_stride + 1, units_of[L - 1] * nrbB, hd, a.status)) return;
+    const int per = a.H / 4;
+    for (int i = threadIdx.x; i < a.T * per; i += kGemvThreads) {
+      const int t = i / per, q = i - t * per;
+      float v[4];
+      combine4(a.y, hd.cw, hd.cpos, t, q, a.H, a.T, a.k, a.n_shared, v);
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
+      reinterpret_cast<uint2*>(a.out + (size_t)t * a.H)[q] =
+          make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

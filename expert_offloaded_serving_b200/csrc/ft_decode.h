@@ -80,6 +80,7 @@ struct StackArgs {
   float* y;                // [T*k + n_shared*T][H]
   int* sync;               // [n_layers][sync_stride], zero at launch
   int sync_stride;         // >= stack_sync_stride(H, I)
+  int fused;               // 1: each gate/up tile rebuilds its input from the previous layer's y (T <= 2)
   int* status;
 };
 

@@ -1110,6 +1110,7 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     a.y = c->d_y;
     a.sync = c->d_sync;
     a.sync_stride = c->sync_stride;
+    a.fused = Ti <= 2 ? 1 : 0;  // beyond that the per-tile recombination costs more L2 reads than a hand-over
     a.status = c->d_status;
     KTimer kt(c, FT_K_DEC_STACK, s);
     CUDA_TRY(launch_dec_stack(a, s));
