@@ -257,7 +257,7 @@ constexpr size_t kTileBytes = 64 * 1024;    // weight codes per tile, about
 struct Gv {
   int K, chunks, atoms;
   int lpr, rpw, parts, rsets, groups;
-  int R, nmat;
+  int R, rlog, nmat;  // rows per tile, a power of two (R = 1 << rlog)
   size_t codes, scales, xh, xinv, red, total;
 };
 
@@ -287,6 +287,8 @@ __host__ __device__ inline Gv make_gv(int K, int rows, int nmat) {
     R >>= 1;
   }
   g.R = R;
+  g.rlog = 0;
+  while ((1 << g.rlog) < R) g.rlog++;
   return g;
 }
 
@@ -599,7 +601,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
     tile_dots(g, m, base, n);
     __syncthreads();
     if (threadIdx.x < g.R * n) {
-      const int t = threadIdx.x / g.R, r = threadIdx.x - t * g.R;
+      const int t = threadIdx.x >> g.rlog, r = threadIdx.x & (g.R - 1);
       a.h[(size_t)(ui.hbase + t0 + t) * a.I + row0 + r] =
           silu(row_value(g, base, 0, r, t)) * row_value(g, base, 1, r, t);
     }
@@ -643,7 +645,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
     tile_dots(g, m, base, n);
     __syncthreads();
     if (threadIdx.x < g.R * n) {
-      const int t = threadIdx.x / g.R, r = threadIdx.x - t * g.R;
+      const int t = threadIdx.x >> g.rlog, r = threadIdx.x & (g.R - 1);
       a.y[(size_t)(ui.hbase + t0 + t) * a.H + row0 + r] = row_value(g, base, 0, r, t);
     }
   }
@@ -848,13 +850,13 @@ __device__ __forceinline__ void combine4(const float* y, const float* cw, const 
 // The gate/up activations of tokens toks[0 .. n) rebuilt from the previous
 // layer's y (the layer input is that layer's combined output), re-encoded like
 // stage_x.
-__device__ __forceinline__ void stage_comb(const Gv& g, uint8_t* base, const StackArgs& a, const float* cw,
+__device__ __forceinline__ void stage_comb(const Gv& g, uint8_t* base, const StackArgs& a, int H, const float* cw,
                                            const int* cpos, const int* toks, int n) {
   const int per = g.K / 4;
   for (int i = threadIdx.x; i < kMT * per; i += kGemvThreads) {
     const int t = i / per, q = i - t * per;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (t < n) combine4(a.y, cw, cpos, toks[t], q, a.H, a.T, a.k, a.n_shared, v);
+    if (t < n) combine4(a.y, cw, cpos, toks[t], q, H, a.T, a.k, a.n_shared, v);
     encode4(g, base, t, q, v);
   }
 }
@@ -904,9 +906,13 @@ __device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* re
 // waits: the next layer's gate/up tile during the down phase, the next
 // layer's down tile during the gate/up phase.  Activations written by other
 // CTAs are read from L2 only.
+// HS, IS: hidden and intermediate size fixed at compile time (the tile
+// geometry then folds to constants), or 0, 0 for any supported shape.
+template <int HS, int IS>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const Gv gA = make_gv(a.H, a.I, 2), gB = make_gv(a.I, a.H, 1);
+  const int H = HS ? HS : a.H, I = IS ? IS : a.I;
+  const Gv gA = make_gv(H, I, 2), gB = make_gv(I, H, 1);
   uint8_t* baseA = smem;
   uint8_t* baseB = smem + gA.total;
   StackHdr& hd = *reinterpret_cast<StackHdr*>(smem + gA.total + gB.total);
@@ -914,7 +920,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   int32_t* units_of = reinterpret_cast<int32_t*>(first + 2 * a.n_layers);
   const LaneMap lmA = lane_map(gA), lmB = lane_map(gB);
   const int G = gridDim.x, b = blockIdx.x;
-  const int nrbA = a.I / gA.R, nrbB = a.H / gB.R;
+  const int nrbA = I / gA.R, nrbB = H / gB.R;
   const bool fused = a.fused != 0;
 
   // A tile's codes (R contiguous rows per matrix) arrive by bulk copies that
@@ -987,10 +993,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   if (b < units * nrbA) issue_A(first[0]);
   if (preB) issue_B(first[1]);
 
-  // Prefetch order: a layer's first down tile is issued once its gate/up wait
-  // returns, the next layer's first gate/up tile once the down wait returns,
-  // so each streams in during a compute phase and no arrival's fence runs
-  // while weight copies of this CTA are in flight.
+  // Prefetch order: a layer's first down tile is issued once its gate/up
+  // activations are staged, the next layer's first gate/up tile once the down
+  // activations are staged, so each streams in during a compute phase, behind
+  // the staging loads, and no arrival's fence runs while weight copies of
+  // this CTA are in flight.
   bool issuedB = preB;  // layer 0's down tile went out at the start
   for (int l = 0; l < a.n_layers; l++) {
     const Route* rec = a.rec + l;
@@ -1020,10 +1027,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
             return;
           }
         }
-        if (haveB && !issuedB) {
-          issue_B(first[2 * l + 1]);
-          issuedB = true;
-        }
       } else {
         if (threadIdx.x < 32) resolve_tile(a, rec, eptr, i, nrbA, gA.R, true, hd.mx);
         __syncthreads();
@@ -1032,9 +1035,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
       const TileMeta& m = i == b ? first[2 * l] : hd.mx;
       for (int t0 = 0; t0 < m.m; t0 += kMT) {
         const int n = min(kMT, m.m - t0);
-        __syncthreads();
-        if (fused && l > 0) stage_comb(gA, baseA, a, hd.cw, hd.cpos, m.tok + t0, n);
+        if (t0 > 0) __syncthreads();
+        if (fused && l > 0) stage_comb(gA, baseA, a, H, hd.cw, hd.cpos, m.tok + t0, n);
         else stage_x<true>(gA, baseA, xin, m.tok + t0, n);
+        // the layer's first down tile streams in during the gate/up compute;
+        // issued after the staging loads so as not to queue ahead of them
+        if (i == b && t0 == 0 && haveB && !issuedB) {
+          issue_B(first[2 * l + 1]);
+          issuedB = true;
+        }
         // the first tile's down weights were issued after it: leave them in flight
         if (i == b && haveB) cp_async_wait_1(); else cp_async_wait_all();
         if (t0 == 0) wait_codes(0);
@@ -1046,8 +1055,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         tile_dots(gA, lmA, baseA, n);
         __syncthreads();
         if (threadIdx.x < gA.R * n && m.blob) {
-          const int t = threadIdx.x / gA.R, r = threadIdx.x - t * gA.R;
-          a.h[(size_t)(m.hbase + t0 + t) * a.I + m.row0 + r] =
+          const int t = threadIdx.x >> gA.rlog, r = threadIdx.x & (gA.R - 1);
+          a.h[(size_t)(m.hbase + t0 + t) * I + m.row0 + r] =
               silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t);
         }
       }
@@ -1065,8 +1074,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         drain();
         return;
       }
-      // buffer A is free since the gate/up phase
-      if (nextA) issue_A(first[2 * (l + 1)]);
       for (int i = b; i < tilesB; i += G) {
         if (i != b) {
           __syncthreads();
@@ -1080,6 +1087,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
           const int n = min(kMT, mb.m - t0);
           if (t0 > 0) __syncthreads();
           stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
+          // buffer A is free since the gate/up phase: the next layer's first
+          // gate/up tile streams in during the down compute
+          if (i == b && t0 == 0 && nextA) issue_A(first[2 * (l + 1)]);
           // the next layer's gate/up weights were issued after this tile's
           if (i == b && nextA) cp_async_wait_1(); else cp_async_wait_all();
           if (t0 == 0) wait_codes(1);
@@ -1091,8 +1101,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
           tile_dots(gB, lmB, baseB, n);
           __syncthreads();
           if (threadIdx.x < gB.R * n) {
-            const int t = threadIdx.x / gB.R, r = threadIdx.x - t * gB.R;
-            a.y[(size_t)(mb.hbase + t0 + t) * a.H + mb.row0 + r] = mb.blob ? row_value(gB, baseB, 0, r, t) : 0.f;
+            const int t = threadIdx.x >> gB.rlog, r = threadIdx.x & (gB.R - 1);
+            a.y[(size_t)(mb.hbase + t0 + t) * H + mb.row0 + r] = mb.blob ? row_value(gB, baseB, 0, r, t) : 0.f;
           }
         }
         if (fused) {
@@ -1114,12 +1124,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
             float acc = 0.f;
             for (int j = 0; j < a.k; j++) {
               const int f = t * a.k + j;
-              acc = fmaf(hd.cw[f], __ldcg(a.y + (size_t)hd.cpos[f] * a.H + nn), acc);
+              acc = fmaf(hd.cw[f], __ldcg(a.y + (size_t)hd.cpos[f] * H + nn), acc);
             }
             for (int s2 = 0; s2 < a.n_shared; s2++)
-              acc += __ldcg(a.y + (size_t)(a.T * a.k + s2 * a.T + t) * a.H + nn);
+              acc += __ldcg(a.y + (size_t)(a.T * a.k + s2 * a.T + t) * H + nn);
             __nv_bfloat16 bb = __float2bfloat16_rn(acc);
-            xout[(size_t)t * a.H + nn] = *reinterpret_cast<uint16_t*>(&bb);
+            xout[(size_t)t * H + nn] = *reinterpret_cast<uint16_t*>(&bb);
           }
           cta_arrive(&sy[1]);
         }
@@ -1135,13 +1145,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     __syncthreads();
     load_combine(a.rec + L - 1);
     if (!cta_wait_geq(a.sync + (size_t)(L - 1) * a.sync_stride + 1, units_of[L - 1] * nrbB, hd, a.status)) return;
-    const int per = a.H / 4;
+    const int per = H / 4;
     for (int i = threadIdx.x; i < a.T * per; i += kGemvThreads) {
       const int t = i / per, q = i - t * per;
       float v[4];
-      combine4(a.y, hd.cw, hd.cpos, t, q, a.H, a.T, a.k, a.n_shared, v);
+      combine4(a.y, hd.cw, hd.cpos, t, q, H, a.T, a.k, a.n_shared, v);
       __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-      reinterpret_cast<uint2*>(a.out + (size_t)t * a.H)[q] =
+      reinterpret_cast<uint2*>(a.out + (size_t)t * H)[q] =
           make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
     }
   }
@@ -1228,12 +1238,14 @@ cudaError_t launch_dec_stack(const StackArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   const Gv gA = make_gv(a.H, a.I, 2), gB = make_gv(a.I, a.H, 1);
   const size_t smem = gA.total + gB.total + stack_hdr_bytes(a.n_layers);
-  cudaError_t e = cudaFuncSetAttribute(k_dec_stack, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the 35B-class shape (hidden 2048, intermediate 512) has its own build
+  void (*kern)(StackArgs) = (a.H == 2048 && a.I == 512) ? k_dec_stack<2048, 512> : k_dec_stack<0, 0>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 0, occ = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-      (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_dec_stack, kGemvThreads, smem)) != cudaSuccess)
+      (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem)) != cudaSuccess)
     return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   // no layer has more tiles than (distinct experts + shared) x row blocks
@@ -1250,7 +1262,7 @@ cudaError_t launch_dec_stack(const StackArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_dec_stack, a);
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace ft
