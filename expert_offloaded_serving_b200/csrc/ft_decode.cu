@@ -367,12 +367,14 @@ __device__ __forceinline__ void encode4(const Gv& g, uint8_t* base, int t, int q
 
 // Re-encode tokens rows[0 .. n) of a bf16 (x) or fp32 (h) matrix with row
 // length K into the tile's f16 activations (read from L2).  Thread i takes 4
-// consecutive elements.  Tokens n .. kMT-1 are zero.
+// consecutive elements.  With n > 1, tokens n .. kMT-1 are zero.
 template <bool BF16>
 __device__ __forceinline__ void stage_x(const Gv& g, uint8_t* base, const void* src, const int* rows, int n) {
   const int per = g.K / 4;
-  // kMT * per is a multiple of 32: a warp is wholly inside or outside
-  for (int i = threadIdx.x; i < kMT * per; i += kGemvThreads) {
+  // tokens n .. kMT-1 are staged only when a pass reads them (n > 1); the
+  // bound is a multiple of 32, so a warp is wholly inside or outside
+  const int items = (n > 1 ? kMT : 1) * per;
+  for (int i = threadIdx.x; i < items; i += kGemvThreads) {
     const int t = i / per, q = i - t * per;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (t < n) {
@@ -853,7 +855,8 @@ __device__ __forceinline__ void combine4(const float* y, const float* cw, const 
 __device__ __forceinline__ void stage_comb(const Gv& g, uint8_t* base, const StackArgs& a, int H, const float* cw,
                                            const int* cpos, const int* toks, int n) {
   const int per = g.K / 4;
-  for (int i = threadIdx.x; i < kMT * per; i += kGemvThreads) {
+  const int items = (n > 1 ? kMT : 1) * per;
+  for (int i = threadIdx.x; i < items; i += kGemvThreads) {
     const int t = i / per, q = i - t * per;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (t < n) combine4(a.y, cw, cpos, toks[t], q, H, a.T, a.k, a.n_shared, v);
