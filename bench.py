@@ -151,6 +151,12 @@ def max_over_ranks(v, world):
 # ---------------------------------------------------------------------------
 H, I, E, K_TOP, S_SHARED, L = 2048, 512, 256, 8, 1, 40
 TRACE_LEN = 512
+# DRAM bytes (read + write) of k_dec_stack per algorithmic byte, from an ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of a 4-layer launch of
+# this workload: 60,253,440 B read + 998,144 B written against 60,162,048 B.
+# The full 40-layer launch is too large to capture; its traffic grows with the
+# layers.
+STACK_TRAFFIC_PER_BYTE = (60253440 + 998144) / 60162048
 
 
 def decode_routing(T):
@@ -541,15 +547,17 @@ def main():
     print(f"# tok/s {res['tok_s']:.1f}  step HBM {res['hbm_gbs']:.0f} GB/s  kernels {res['kernels']}", file=sys.stderr)
     if st:  # the persistent kernel reads every layer's weights in one launch
         rk, rk_bytes, rk_us = "dec_stack", res["stack_bytes"], st["us_avg"]
+        rk_traffic = STACK_TRAFFIC_PER_BYTE * rk_bytes if H == 2048 and I == 512 else None
     else:
         rk, rk_bytes, rk_us = "gate_up", res["gate_up_bytes"], gu["us_avg"] if gu else float("nan")
+        rk_traffic = None
     rk_gbs = rk_bytes / (rk_us * 1e-6) / 1e9
     line = {"metric": METRIC, "value": res["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(T, args.layerwise),
             "roofline": {"bound": "hbm", "kernel": rk, "achieved": rk_gbs, "peak": pk["hbm"],
-                         "peak_source": pk["src"], "unit": "GB/s", "frac": rk_gbs / pk["hbm"], "traffic": None,
+                         "peak_source": pk["src"], "unit": "GB/s", "frac": rk_gbs / pk["hbm"], "traffic": rk_traffic,
                          "algorithmic_bytes_per_launch": rk_bytes},
             "hbm_gbs_step": res["hbm_gbs"], "hbm_frac_step": res["hbm_gbs"] / pk["hbm"],
             "gpu_launches": res["launches"], "clocks": res["clocks"], "e2e": res["e2e"],
