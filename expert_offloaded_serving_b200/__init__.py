@@ -29,7 +29,8 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_router_logits", "ft_moe_route", "ft_moe_permute", "ft_quantize_mxfp4", "ft_moe_layer_forward",
            "ft_expert_cache_lookup", "ft_expert_cache_insert", "ft_expert_cache_resize", "ft_cache_trace",
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
-           "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing")
+           "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
+           "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -99,6 +100,9 @@ def lib() -> C.CDLL:
         "ft_moe_layer_forward_noalloc": (ST, [I32, I32, I32, I32, I32, P, P, I64, P, P, P, U32, P, P]),
         "ft_moe_stack_forward": (ST, [P, I32, I32, P, I64, P, P, U32, P]),
         "ft_last_routing": (ST, [P, P, P, I64, P]),
+        "ft_debug_device_wait": (ST, [P, I64, P]),
+        "ft_debug_host_wait_limit": (ST, [P, C.c_double]),
+        "ft_debug_fail_copy": (ST, [P, I64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -237,6 +241,18 @@ def ft_prefetch_layer(ctx, layer, compute_stream=None) -> None:
 
 def ft_debug_dequant(ctx, blob, mat, out, stream=None) -> None:
     _check(lib().ft_debug_dequant(ctx, _ptr(blob), mat, _ptr(out), _stream(stream)))
+
+
+def ft_debug_device_wait(ctx, timeout_us: int, stream=None) -> None:
+    _check(lib().ft_debug_device_wait(ctx, timeout_us, _stream(stream)))
+
+
+def ft_debug_host_wait_limit(ctx, seconds: float) -> None:
+    _check(lib().ft_debug_host_wait_limit(ctx, seconds))
+
+
+def ft_debug_fail_copy(ctx, n: int) -> None:
+    _check(lib().ft_debug_fail_copy(ctx, n))
 
 
 def ft_kernel_timing_enable(ctx, on: bool) -> None:

@@ -768,22 +768,23 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                : "memory");
 }
 
-// Thread 0 waits (acquire, bounded) until *p >= target, then the CTA
-// synchronises; false (and the timeout status bit) when the wait gave up.
-__device__ bool cta_wait_geq(const int* p, int target, StackHdr& hd, int* status) {
+// Thread 0 waits (acquire, bounded by limit_ns) until *p >= target, then the
+// CTA synchronises; false (and the timeout status bit) when the wait gave up.
+// `abort` is a shared flag, zero until a wait of this CTA gives up.
+__device__ bool cta_wait_geq(const int* p, int target, int& abort, int* status, uint64_t limit_ns = kSpinNs) {
   if (threadIdx.x == 0 && ld_acquire(p) < target) {
     const uint64_t t0 = gclock();
     while (ld_acquire(p) < target) {
-      if (gclock() - t0 > kSpinNs) {
+      if (gclock() - t0 > limit_ns) {
         set_status(status, kStTimeout);
-        hd.abort = 1;
+        abort = 1;
         break;
       }
       __nanosleep(20);
     }
   }
   __syncthreads();
-  return hd.abort == 0;
+  return abort == 0;
 }
 
 // Lane 0 of the last warp publishes arrivals, so that thread 0, which polls,
@@ -1025,7 +1026,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         // the first tile was issued ahead: wait for the previous layer
         if (l > 0) {
           const int* prev = a.sync + (size_t)(l - 1) * a.sync_stride + 1;
-          if (!cta_wait_geq(prev, fused ? units_of[l - 1] * nrbB : nrbB, hd, a.status)) {
+          if (!cta_wait_geq(prev, fused ? units_of[l - 1] * nrbB : nrbB, hd.abort, a.status)) {
             drain();
             return;
           }
@@ -1073,7 +1074,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     // ---------------- down (+ row-block combine) ----------------
     if (haveB) {
       // every gate/up tile of this layer is done
-      if (!cta_wait_geq(&sy[0], tilesA, hd, a.status)) {
+      if (!cta_wait_geq(&sy[0], tilesA, hd.abort, a.status)) {
         drain();
         return;
       }
@@ -1147,7 +1148,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     const int L = a.n_layers;
     __syncthreads();
     load_combine(a.rec + L - 1);
-    if (!cta_wait_geq(a.sync + (size_t)(L - 1) * a.sync_stride + 1, units_of[L - 1] * nrbB, hd, a.status)) return;
+    if (!cta_wait_geq(a.sync + (size_t)(L - 1) * a.sync_stride + 1, units_of[L - 1] * nrbB, hd.abort, a.status)) return;
     const int per = H / 4;
     for (int i = threadIdx.x; i < a.T * per; i += kGemvThreads) {
       const int t = i / per, q = i - t * per;
@@ -1158,6 +1159,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
           make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// failure injection: the persistent kernel's bounded wait on a flag nothing sets
+// ---------------------------------------------------------------------------
+__global__ void k_debug_wait(const int* flag, int* status, uint64_t limit_ns) {
+  __shared__ int abort;
+  if (threadIdx.x == 0) abort = 0;
+  __syncthreads();
+  cta_wait_geq(flag, 1, abort, status, limit_ns);
 }
 
 // ---------------------------------------------------------------------------
@@ -1232,6 +1243,11 @@ constexpr size_t kStackSmemMax = 227 * 1024;  // opt-in dynamic shared memory pe
 bool stack_supported(int H, int I, int n_layers) {
   const Gv gA = make_gv(H, I, 2), gB = make_gv(I, H, 1);
   return gv_ok(gA, I) && gv_ok(gB, H) && gA.total + gB.total + stack_hdr_bytes(n_layers) <= kStackSmemMax;
+}
+
+cudaError_t launch_debug_wait(const int* flag, int* status, uint64_t limit_ns, cudaStream_t s) {
+  k_debug_wait<<<1, 32, 0, s>>>(flag, status, limit_ns);
+  return cudaGetLastError();
 }
 
 int stack_sync_stride(int H, int I) { return 2 + H / make_gv(I, H, 1).R; }

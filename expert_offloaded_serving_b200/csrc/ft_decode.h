@@ -90,4 +90,8 @@ bool stack_supported(int H, int I, int n_layers);
 int stack_sync_stride(int H, int I);
 cudaError_t launch_dec_stack(const StackArgs& a, cudaStream_t s);
 
+// One CTA waiting, with the persistent kernel's bounded wait, for *flag >= 1;
+// sets the timeout bit of *status after limit_ns.
+cudaError_t launch_debug_wait(const int* flag, int* status, uint64_t limit_ns, cudaStream_t s);
+
 }  // namespace ft

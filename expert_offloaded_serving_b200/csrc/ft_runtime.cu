@@ -161,6 +161,11 @@ struct ft_ctx {
   uint16_t* d_xbuf[2] = {nullptr, nullptr};  // stack forward ping-pong [T][H]
   int* d_sync = nullptr;       // persistent stack kernel counters [L][sync_stride]
   int sync_stride = 0;
+  int* d_flag = nullptr;       // a device flag nothing sets (failure injection)
+
+  // failure injection
+  double host_wait_s = kHostWaitSeconds;  // limit of the bounded host waits
+  int64_t fail_copy_in = 0;               // the n-th next expert copy fails (0: off)
   int decode_max_t = 0;
 
   // pinned host scratch
@@ -350,7 +355,8 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
 
   const int T = desc->max_tokens;
   ft_status st;
-  if ((st = dev_alloc(&c->d_status, 1)) || (st = dev_alloc(&c->d_logits, (size_t)T * E)) ||
+  if ((st = dev_alloc(&c->d_status, 1)) || (st = dev_alloc(&c->d_flag, 1)) ||
+      (st = dev_alloc(&c->d_logits, (size_t)T * E)) ||
       (st = dev_alloc(&c->d_ids, (size_t)T * k)) || (st = dev_alloc(&c->d_w, (size_t)T * k)) ||
       (st = dev_alloc(&c->d_offs, E + 1)) || (st = dev_alloc(&c->d_perm, (size_t)T * k)) ||
       (st = dev_alloc(&c->d_inv, (size_t)T * k)) || (st = dev_alloc(&c->d_active, E)) ||
@@ -368,7 +374,8 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
   }
   if (cudaMemset(c->d_counters, 0, (size_t)H / 8 * sizeof(int)) != cudaSuccess)
     return bail(fail(FT_ERR_CUDA, "memset"));
-  if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return bail(fail(FT_ERR_CUDA, "memset"));
+  if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess || cudaMemset(c->d_flag, 0, sizeof(int)) != cudaSuccess)
+    return bail(fail(FT_ERR_CUDA, "memset"));
   if (cudaMallocHost(&c->h_ids, (size_t)T * k * sizeof(int32_t)) != cudaSuccess ||
       cudaMallocHost(&c->h_status, sizeof(int)) != cudaSuccess)
     return bail(fail(FT_ERR_CUDA, "pinned scratch"));
@@ -461,6 +468,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   }
   free_prefill_scratch(c->pf);
   cudaFree(c->d_status);
+  cudaFree(c->d_flag);
   cudaFree(c->d_logits);
   cudaFree(c->d_ids);
   cudaFree(c->d_w);
@@ -504,8 +512,8 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   return FT_OK;
 }
 
-// bounded host wait on an event: polls, gives up after kHostWaitSeconds
-static ft_status wait_event(cudaEvent_t ev, const char* what) {
+// bounded host wait on an event: polls, gives up after `limit` seconds
+static ft_status wait_event(cudaEvent_t ev, const char* what, double limit) {
   auto t0 = std::chrono::steady_clock::now();
   int spins = 0;
   while (true) {
@@ -514,7 +522,7 @@ static ft_status wait_event(cudaEvent_t ev, const char* what) {
     if (q != cudaErrorNotReady) return fail(FT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(q));
     if (++spins > 64) std::this_thread::sleep_for(std::chrono::microseconds(20));
     double s = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
-    if (s > kHostWaitSeconds) return fail(FT_ERR_TIMEOUT, "%s: gave up after %.1f s", what, s);
+    if (s > limit) return fail(FT_ERR_TIMEOUT, "%s: gave up after %.3f s", what, s);
   }
 }
 
@@ -583,6 +591,28 @@ extern "C" ft_status ft_debug_dequant(ft_ctx* c, const void* blob, int32_t mat, 
   return FT_OK;
 }
 
+extern "C" ft_status ft_debug_device_wait(ft_ctx* c, int64_t timeout_us, void* stream) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (timeout_us < 1 || timeout_us > 2000000) return fail(FT_ERR_INVALID, "timeout_us %lld outside [1, 2e6]", (long long)timeout_us);
+  CUDA_TRY(launch_debug_wait(c->d_flag, c->d_status, (uint64_t)timeout_us * 1000u, (cudaStream_t)stream));
+  c->last_stream = (cudaStream_t)stream;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_debug_host_wait_limit(ft_ctx* c, double seconds) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (!(seconds > 0.0)) return fail(FT_ERR_INVALID, "limit must be positive");
+  c->host_wait_s = seconds;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_debug_fail_copy(ft_ctx* c, int64_t n) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (n < 0) return fail(FT_ERR_INVALID, "n must be >= 0");
+  c->fail_copy_in = n;
+  return FT_OK;
+}
+
 // ---------------------------------------------------------------------------
 // expert cache
 // ---------------------------------------------------------------------------
@@ -615,6 +645,8 @@ static int32_t evict_one(ft_ctx* c, const std::vector<int64_t>& keep, int64_t* v
 
 // Issue the H2D copy of (layer, e) into `slot` on the copy stream.
 static ft_status fetch(ft_ctx* c, int layer, int e, int32_t slot) {
+  if (c->fail_copy_in > 0 && --c->fail_copy_in == 0)
+    return fail(FT_ERR_CUDA, "injected failure of the host-to-device copy of expert (%d, %d)", layer, e);
   const uint8_t* src = c->host_layers[layer] + (size_t)e * c->stride;
   CUDA_TRY(cudaMemcpyAsync(slot_ptr(c, slot), src, (size_t)c->lay.used, cudaMemcpyHostToDevice, c->copy_stream));
   c->stats.h2d_bytes += c->lay.used;
@@ -661,7 +693,24 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
     c->h_eptr_cache[(size_t)layer * c->n_blobs + e] = slot_ptr(c, slot);
     record(c, FT_EV_MISS, layer, e, slot, -1);
     c->stats.misses++;
-    FT_TRY(fetch(c, layer, e, slot));
+    const ft_status fs = fetch(c, layer, e, slot);
+    if (fs != FT_OK) {
+      // the key never became resident: drop it again; keys fetched earlier
+      // in this step stay (their copies are queued on the copy stream)
+      c->lru.order.pop_back();
+      c->lru.map.erase(key);
+      c->lru.slot_used[slot] = 0;
+      c->h_eptr_cache[(size_t)layer * c->n_blobs + e] = nullptr;
+      record(c, FT_EV_EVICT, layer, e, slot, -1);
+      c->stats.evictions++;
+      c->stats.used_slots = (int64_t)c->lru.map.size();
+      cudaEventRecord(t1, c->copy_stream);
+      c->copy_timing.push_back({t0, t1});
+      // a later step counts the earlier keys as hits and does not wait for
+      // their copies: let them land now
+      cudaStreamSynchronize(c->copy_stream);
+      return fs;
+    }
   }
   if (any_miss) {
     cudaEventRecord(t1, c->copy_stream);
@@ -933,7 +982,7 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     CUDA_TRY(cudaMemcpyAsync(c->h_ids, c->d_ids, (size_t)Ti * k * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaEventRecord(c->ev_ids, s));
-    FT_TRY(wait_event(c->ev_ids, "routing ids"));
+    FT_TRY(wait_event(c->ev_ids, "routing ids", c->host_wait_s));
     if (*c->h_status) {
       int st = *c->h_status;
       CUDA_TRY(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));

@@ -298,6 +298,32 @@ FT_API ft_status ft_prefetch_layer(ft_ctx* ctx, int32_t layer, void* compute_str
  * routine the GEMV uses. */
 FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, float* out, void* stream);
 
+/* Failure injection for tests: none of these fault or hang a GPU.
+ *
+ * ft_debug_device_wait: launch, on `stream`, one CTA that waits for a device
+ * flag nothing ever sets, with the bounded wait the persistent decode kernel
+ * uses between layers, limited to timeout_us microseconds (1 .. 2,000,000);
+ * when the limit runs out the CTA sets the timeout bit of the context's
+ * status word and returns, so the next ft_sync_status reports
+ * FT_ERR_TIMEOUT and the context stays usable.  Errors: FT_ERR_INVALID,
+ * FT_ERR_CUDA.
+ *
+ * ft_debug_host_wait_limit: the limit (seconds, > 0) of the context's bounded
+ * host waits on device events (the cache path's wait for the routed ids
+ * before its LRU step); the default is 30 s.  A wait that runs out returns
+ * FT_ERR_TIMEOUT with the cache unchanged; the work already queued stays
+ * queued.
+ *
+ * ft_debug_fail_copy: the n-th host-to-device expert copy the cache issues
+ * from now on (n >= 1; 0 turns injection off) fails instead of being issued:
+ * the call returns FT_ERR_CUDA, the key whose copy failed is dropped from the
+ * cache again (a MISS then an EVICT event in the trace), keys fetched earlier
+ * in the same step stay resident, and a retry of the step fetches the dropped
+ * key. */
+FT_API ft_status ft_debug_device_wait(ft_ctx* ctx, int64_t timeout_us, void* stream);
+FT_API ft_status ft_debug_host_wait_limit(ft_ctx* ctx, double seconds);
+FT_API ft_status ft_debug_fail_copy(ft_ctx* ctx, int64_t n);
+
 /* ---------------------------------------------------------------------- */
 /* measurement                                                             */
 /* ---------------------------------------------------------------------- */
