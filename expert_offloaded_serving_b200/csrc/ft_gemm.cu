@@ -12,8 +12,10 @@
 //   warp 1, one thread   tcgen05.cp of the scale atoms into tensor memory and
 //                        tcgen05.mma (K = 64 per instruction); tcgen05.commit
 //                        frees a stage and finally signals the accumulators
-//   warps 0..3           epilogue from tensor memory (tcgen05.ld): SwiGLU and
-//                        MXFP4 quantisation of h (gate/up), or fp32 y (down)
+//   warps 0..15          epilogue from tensor memory (tcgen05.ld): warp w reads
+//                        TMEM lanes 32(w%4).. (its weight rows) and every
+//                        fourth 16-column group of tokens from 16(w/4): SwiGLU
+//                        and MXFP4 quantisation of h (gate/up), or fp32 y (down)
 // All mbarrier waits are bounded; on a timeout the CTA records the TIMEOUT
 // status, stops issuing, frees its tensor memory and returns.
 //
@@ -29,7 +31,8 @@
 namespace ft {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 512;    // 16 warps: warps w, w+4, w+8, w+12 share TMEM lanes 32(w%4).. in the epilogue
+constexpr int kEpiGroups = kThreads / 128;  // column groups of the epilogue
 constexpr int kStagesGU = 3;     // gate/up: 2 weight tiles + 1 token tile per stage
 constexpr int kStagesDn = 4;     // down: 1 + 1
 constexpr int kTileBytes = kGemmBM * kGemmBK / 2;   // 16 KB of e2m1 codes
@@ -50,6 +53,36 @@ __device__ __forceinline__ uint64_t gtime() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// One lane of the warp waits for phase `parity` with a sleep between polls
+// (the warps that only wait for the accumulators do not compete for issue
+// slots with the producer and MMA threads), then the warp reconverges; false
+// after kWaitNs of wall time.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity) {
+  uint32_t ok = 0;
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t a = s_u32(b);
+    const uint64_t t0 = gtime();
+    for (;;) {
+      asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                   : "=r"(ok)
+                   : "r"(a), "r"(parity)
+                   : "memory");
+      if (ok || gtime() - t0 > kWaitNs) break;
+      __nanosleep(256);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) {  // every lane observes the completed phase (acquire) before reading its results
+    uint32_t again;
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(again)
+                 : "r"(s_u32(b)), "r"(parity)
+                 : "memory");
+    (void)again;
+  }
+  return ok != 0;
+}
+
 // wait for phase `parity`, giving up after kWaitNs of wall time
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
   const uint32_t a = s_u32(b);
@@ -242,17 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
   }
   __syncwarp();
 
-  // ---- epilogue: warp w owns TMEM lanes 32w..32w+31 = weight rows ----
-  const bool have = mbar_wait(accb, 0);
+  // ---- epilogue: warp w owns TMEM lanes 32(w%4).. = weight rows and the
+  // token columns 16 * (w/4 + kEpiGroups * j) ----
+  const bool have = mbar_wait_warp(accb, 0);
   if (!have && threadIdx.x == 0) set_status(a.status, kStTimeout);
+  const int quad = warp & 3, cg = warp >> 2;
   if (have) {
     tc_fence_after();
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     if (MODE == 0) {
       const int I = a.M;
-      const int irow = mt * kGemmBM + warp * 32 + lane;
+      const int irow = mt * kGemmBM + quad * 32 + lane;
       const int atoms_i = I / 128;
-      for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+      for (int c0 = 16 * cg; c0 < kGemmBN; c0 += 16 * kEpiGroups) {
         float g[16], u[16];
         tmem_ld16(d0 + lane_off + c0, g);
         tmem_ld16(d1 + lane_off + c0, u);
@@ -267,17 +302,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
           const float v = hv * mx_inv_scale(e8);
           const float nb = __shfl_xor_sync(0xffffffffu, v, 1);
           if ((lane & 1) == 0) a.hq[(size_t)p * (I / 2) + (irow >> 1)] = (uint8_t)cvt_e2m1x2(v, nb);
-          if (lane == 0) a.hq_sf[sf_word(p, mt, atoms_i) + warp] = (uint8_t)e8;
+          if (lane == 0) a.hq_sf[sf_word(p, mt, atoms_i) + quad] = (uint8_t)e8;
         }
       }
     } else {
       const int H = a.M;
-      const int hrow = mt * kGemmBM + warp * 32 + lane;
+      const int hrow = mt * kGemmBM + quad * 32 + lane;
       const bool shared = e >= a.E;
       const int valid = shared ? a.T : a.offs[e + 1] - a.offs[e];
       const int base_pos = shared ? a.T * a.k + (e - a.E) * a.T : a.offs[e];
       const int r0 = row0 - a.pad_offs[e];
-      for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+      for (int c0 = 16 * cg; c0 < kGemmBN; c0 += 16 * kEpiGroups) {
         float v[16];
         tmem_ld16(d0 + lane_off + c0, v);
 #pragma unroll
