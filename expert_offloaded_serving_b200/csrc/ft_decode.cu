@@ -865,6 +865,57 @@ __device__ __forceinline__ void stage_comb(const Gv& g, uint8_t* base, const Sta
   }
 }
 
+// h of the fused mode travels as 64-bit words (tag << 32 | fp32 bits), each
+// stored and loaded whole (single-copy atomic), so a reader that sees this
+// layer's tag sees the value that came with it.
+__device__ __forceinline__ void st_tagged(uint64_t* p, float v, uint32_t tag) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(((uint64_t)tag << 32) | __float_as_uint(v))
+               : "memory");
+}
+__device__ __forceinline__ void ld_tagged4(const uint64_t* p, uint64_t (&w)[4]) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w[0]), "=l"(w[1]) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w[2]), "=l"(w[3]) : "l"(p + 2) : "memory");
+}
+
+// The down tile's activations from the tagged h: a word whose tag is not
+// this layer's has not arrived yet and is read again, for at most 2 s (then
+// the timeout bit and the CTA's abort flag are set).  Re-encoded like
+// stage_x.
+__device__ __forceinline__ void stage_h_tagged(const Gv& g, uint8_t* base, const uint64_t* ht, const int* rows, int n,
+                                               uint32_t tag, int& abort, int* status) {
+  const int per = g.K / 4;
+  const int items = (n > 1 ? kMT : 1) * per;
+  for (int i = threadIdx.x; i < items; i += kGemvThreads) {
+    const int t = i / per, q = i - t * per;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (t < n) {
+      const uint64_t* p = ht + (size_t)rows[t] * g.K + 4 * q;
+      uint64_t w[4];
+      ld_tagged4(p, w);
+      auto ready = [&]() {
+        return (uint32_t)(w[0] >> 32) == tag && (uint32_t)(w[1] >> 32) == tag && (uint32_t)(w[2] >> 32) == tag &&
+               (uint32_t)(w[3] >> 32) == tag;
+      };
+      if (!ready()) {
+        const uint64_t t0 = gclock();
+        for (;;) {
+          __nanosleep(20);
+          ld_tagged4(p, w);
+          if (ready()) break;
+          if (gclock() - t0 > kSpinNs) {
+            set_status(status, kStTimeout);
+            abort = 1;
+            break;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; j++) v[j] = __uint_as_float((uint32_t)w[j]);
+    }
+    encode4(g, base, t, q, v);
+  }
+}
+
 // One warp resolves tile i of a phase (nrb row blocks of R rows per unit) of
 // layer `rec` into m; the caller synchronises before the CTA reads it.
 __device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* rec, const uint8_t* const* eptr, int i,
@@ -926,6 +977,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   const int G = gridDim.x, b = blockIdx.x;
   const int nrbA = I / gA.R, nrbB = H / gB.R;
   const bool fused = a.fused != 0;
+  const uint32_t epoch = fused ? *a.epoch : 0u;  // tag of layer l: epoch << 7 | l
 
   // A tile's codes (R contiguous rows per matrix) arrive by bulk copies that
   // one thread issues and that complete on the buffer's mbarrier; its scale
@@ -1058,13 +1110,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         }
         tile_dots(gA, lmA, baseA, n);
         __syncthreads();
-        if (threadIdx.x < gA.R * n && m.blob) {
+        if (threadIdx.x < gA.R * n) {
           const int t = threadIdx.x >> gA.rlog, r = threadIdx.x & (gA.R - 1);
-          a.h[(size_t)(m.hbase + t0 + t) * I + m.row0 + r] =
-              silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t);
+          const size_t at = (size_t)(m.hbase + t0 + t) * I + m.row0 + r;
+          if (fused)  // a missing expert still delivers (zeros), so no reader waits for it
+            st_tagged(a.h_tagged + at,
+                      m.blob ? silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t) : 0.f,
+                      (epoch << 7) | (uint32_t)l);
+          else if (m.blob)
+            a.h[at] = silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t);
         }
       }
-      cta_arrive(&sy[0]);
+      // the fused mode's h carries its own tag: no counter to publish
+      if (fused) __syncthreads(); else cta_arrive(&sy[0]);
     }
     // without a down phase, the next layer's first gate/up tile goes out now
     if (!haveB && nextA) {
@@ -1073,8 +1131,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     }
     // ---------------- down (+ row-block combine) ----------------
     if (haveB) {
-      // every gate/up tile of this layer is done
-      if (!cta_wait_geq(&sy[0], tilesA, hd.abort, a.status)) {
+      // every gate/up tile of this layer is done (the fused mode polls its
+      // tagged h instead)
+      if (!fused && !cta_wait_geq(&sy[0], tilesA, hd.abort, a.status)) {
         drain();
         return;
       }
@@ -1090,7 +1149,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         for (int t0 = 0; t0 < mb.m; t0 += kMT) {
           const int n = min(kMT, mb.m - t0);
           if (t0 > 0) __syncthreads();
-          stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
+          if (fused) stage_h_tagged(gB, baseB, a.h_tagged, mb.tok + t0, n, (epoch << 7) | (uint32_t)l, hd.abort, a.status);
+          else stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
           // buffer A is free since the gate/up phase: the next layer's first
           // gate/up tile streams in during the down compute
           if (i == b && t0 == 0 && nextA) issue_A(first[2 * (l + 1)]);
@@ -1184,6 +1244,11 @@ __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
   for (int i = threadIdx.x; i < (int)(sizeof(Route) / 16); i += kThreads) dst[i] = src[i];
   if (a.sync)
     for (int i = threadIdx.x; i < a.sync_stride; i += kThreads) a.sync[(size_t)l * a.sync_stride + i] = 0;
+  if (a.epoch && l == 0 && threadIdx.x == 0) {
+    uint32_t e = *a.epoch + 1u;
+    if ((e << 7) == 0u) e += 1u;  // tags (e << 7 | layer) never equal the zeroed buffer's
+    *a.epoch = e;
+  }
   if (l == a.n_layers - 1 && a.ids_out) {
     for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
       a.ids_out[f] = r.ids[f];

@@ -38,6 +38,7 @@ struct RouteArgs {
   int* status;
   int* sync;            // [n_layers][sync_stride] zeroed by CTA l for layer l, or NULL
   int sync_stride;
+  uint32_t* epoch;      // launch counter the persistent kernel tags its h with; CTA 0 adds 1, or NULL
 };
 
 struct DecodeArgs {
@@ -81,6 +82,10 @@ struct StackArgs {
   int* sync;               // [n_layers][sync_stride], zero at launch
   int sync_stride;         // >= stack_sync_stride(H, I)
   int fused;               // 1: each gate/up tile rebuilds its input from the previous layer's y (T <= 2)
+  // With fused: h travels tagged, [T*k + n_shared*T][I] words (tag << 32 | fp32 bits), and
+  // the down tiles poll it instead of a counter; the tag is (*epoch << 7) | layer.
+  uint64_t* h_tagged;
+  const uint32_t* epoch;   // advanced by the routing kernel before this launch
   int* status;
 };
 

@@ -162,6 +162,8 @@ struct ft_ctx {
   int* d_sync = nullptr;       // persistent stack kernel counters [L][sync_stride]
   int sync_stride = 0;
   int* d_flag = nullptr;       // a device flag nothing sets (failure injection)
+  uint64_t* d_h_tagged = nullptr;  // persistent kernel, T <= 2: tagged h [T*k + S*T][I]
+  uint32_t* d_epoch = nullptr;     // launch counter for those tags
 
   // failure injection
   double host_wait_s = kHostWaitSeconds;  // limit of the bounded host waits
@@ -370,7 +372,13 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
     return bail(st);
   if (stack_supported(H, I, 1)) {
     c->sync_stride = stack_sync_stride(H, I);
-    if ((st = dev_alloc(&c->d_sync, (size_t)L * c->sync_stride))) return bail(st);
+    const size_t hrows = (size_t)(std::min(c->decode_max_t, 2) * k + desc->n_shared * std::min(c->decode_max_t, 2));
+    if ((st = dev_alloc(&c->d_sync, (size_t)L * c->sync_stride)) || (st = dev_alloc(&c->d_h_tagged, hrows * I)) ||
+        (st = dev_alloc(&c->d_epoch, 1)))
+      return bail(st);
+    if (cudaMemset(c->d_h_tagged, 0, hrows * I * sizeof(uint64_t)) != cudaSuccess ||
+        cudaMemset(c->d_epoch, 0, sizeof(uint32_t)) != cudaSuccess)
+      return bail(fail(FT_ERR_CUDA, "memset"));
   }
   if (cudaMemset(c->d_counters, 0, (size_t)H / 8 * sizeof(int)) != cudaSuccess)
     return bail(fail(FT_ERR_CUDA, "memset"));
@@ -485,6 +493,8 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   cudaFree(c->d_xbuf[0]);
   cudaFree(c->d_xbuf[1]);
   cudaFree(c->d_sync);
+  cudaFree(c->d_h_tagged);
+  cudaFree(c->d_epoch);
   cudaFree(c->d_eptr_res);
   cudaFree(c->d_eptr_cache);
   cudaFree(c->d_shared);
@@ -1127,6 +1137,9 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   const int Ti = (int)T;
   const bool persistent =
       !(flags & FT_STACK_LAYERWISE) && c->d_sync != nullptr && stack_supported(c->d.hidden, c->d.inter, n_layers);
+  // with one or two tokens the persistent kernel folds the combine into the
+  // next layer and hands h over tagged (the tag holds the layer in 7 bits)
+  const bool fused = persistent && Ti <= 2 && n_layers <= 128;
   // all layers' routing records in one launch (their logits are inputs); it
   // also zeroes the persistent kernel's counters of those layers
   {
@@ -1135,6 +1148,7 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     if (persistent) {
       ra.sync = c->d_sync;
       ra.sync_stride = c->sync_stride;
+      if (fused) ra.epoch = c->d_epoch;
     }
     CUDA_TRY(launch_route(ra, s));
   }
@@ -1159,7 +1173,9 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     a.y = c->d_y;
     a.sync = c->d_sync;
     a.sync_stride = c->sync_stride;
-    a.fused = Ti <= 2 ? 1 : 0;  // beyond that the per-tile recombination costs more L2 reads than a hand-over
+    a.fused = fused ? 1 : 0;  // beyond two tokens the per-tile recombination costs more L2 reads than a hand-over
+    a.h_tagged = c->d_h_tagged;
+    a.epoch = c->d_epoch;
     a.status = c->d_status;
     KTimer kt(c, FT_K_DEC_STACK, s);
     CUDA_TRY(launch_dec_stack(a, s));
