@@ -3,12 +3,9 @@
 //   k_route         one CTA per layer: softmax top-k of the T tokens and the
 //                   permutation of their (token, rank) pairs by expert, stored
 //                   as a compact routing record (distinct experts = units).
-//   k_dec_gate_up   CTA = (unit, block of R rows of Wg and Wu) over the full K:
-//                   the tile is staged in shared memory with coalesced 16-byte
-//                   cp.async copies; tpr threads share a row, each dequantising
-//                   its scale-atom columns of e2m1 codes with their UE8M0 scales
-//                   in registers (split-K inside the row group, reduced by
-//                   shuffles); gate and up share the activation reads; SwiGLU
+//   k_dec_gate_up   CTA = (unit, block of R rows of Wg and Wu) over the full K,
+//                   staged in shared memory by 16-byte cp.async copies; the
+//                   GEMV tile below computes both matrices' rows and SwiGLU
 //                   gives fp32 h.
 //   k_dec_down      CTA = (unit, block of R rows of Wd) over K = I; launched as a
 //                   programmatic dependent of gate/up, so its tile streams in
@@ -16,12 +13,17 @@
 //                   writes y.  The last CTA to finish a row block (an atomic
 //                   counter per block) sums w[t][j] * y over j ascending plus
 //                   the shared expert and rounds once to bf16.
-//
 //   k_dec_stack     persistent and cooperative: one launch runs a stack of
 //                   layers; each CTA takes the gate/up and the down tiles with
-//                   its index modulo the grid, layer after layer, and the layers
-//                   hand over through counters in global memory instead of
-//                   kernel boundaries (same arithmetic as the two kernels above).
+//                   its index modulo the grid, layer after layer; layers hand
+//                   over through bounded counters in global memory (and, for
+//                   one or two tokens, h through tagged words) instead of
+//                   kernel boundaries; same arithmetic as the two kernels above.
+//
+// All three share the GEMV tile: lanes own 32-code chunks of K and hold their
+// chunk's activations (re-encoded per 32-element block as f16) in registers,
+// dots by fma.rn.f32.f16 on exact products, four rows per lane group reduced by
+// a transposing shuffle tree.
 //
 // Pages: decode fetches or reuses the selected experts and sums their partial
 // results exactly (jansverre.net, "Hvorfor er båndbredden viktigere enn antall

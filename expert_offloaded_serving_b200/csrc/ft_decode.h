@@ -1,7 +1,7 @@
 // Small-batch decode kernels: a routing kernel that writes one compact routing
 // record per layer, then either one persistent kernel for a stack of layers or,
-// per layer, a gate/up + SwiGLU GEMV and a down GEMV with the combine
-// (cp.async-staged FP4 tiles, split-K inside a row's thread group).
+// per layer, a gate/up + SwiGLU GEMV and a down GEMV with the combine (FP4
+// tiles staged in shared memory; each lane owns a 32-code chunk of K).
 #pragma once
 
 #include <cstdint>

@@ -1,5 +1,7 @@
-// Decode path: split-K FP4 GEMV of the selected experts, dequantising e2m1
-// codes with their UE8M0 block scales in registers.
+// Decode GEMV of the allocation-free forward (ft_moe_layer_forward_noalloc)
+// and the dequantiser behind ft_debug_dequant: split-K FP4 GEMV of the
+// selected experts, dequantising e2m1 codes with their UE8M0 block scales in
+// registers.  (The context's decode path is ft_decode.cu.)
 //
 //   k_gate_up        h[pair][i] = silu(Wg[i] . x) * (Wu[i] . x)      (fp32 h)
 //   k_down_combine   y[pair][n] = Wd[n] . h[pair];

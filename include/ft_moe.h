@@ -80,7 +80,7 @@ typedef struct {
 
 /* forward / route flags */
 #define FT_ROUTE_RENORM 1u    /* renormalise the k softmax weights to sum 1 (default on) */
-#define FT_ACT_BF16     0u    /* decode: bf16 activations, fp32 h, split-K FP4 GEMV */
+#define FT_ACT_BF16     0u    /* decode: bf16 activations, fp32 h, FP4 GEMV on CUDA cores */
 #define FT_ACT_MXFP4    2u    /* prefill: x and h quantised to MXFP4, tcgen05 grouped GEMM */
 #define FT_STACK_LAYERWISE 4u /* ft_moe_stack_forward: two kernels per layer, not the persistent kernel */
 
