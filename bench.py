@@ -5,8 +5,8 @@ Default workload: the 35B-A3B-class decode stack (hidden 2048, 256 routed
 experts top-8 plus 1 shared expert, intermediate 512, 40 layers, MXFP4 weights
 resident in HBM, batch 1), routed by seeded Zipf(1.1) traces with 0.6
 adjacent-token reuse.  One step = one token through all 40 MoE layers
-(route, permute, gate/up + SwiGLU GEMV, down GEMV + combine), replayed as one
-CUDA graph.  Each step reads ~600 MB of distinct expert weights, far more than
+(the routing kernel and the persistent decode kernel: gate/up + SwiGLU,
+down, combine for every layer), replayed as one CUDA graph.  Each step reads ~600 MB of distinct expert weights, far more than
 the 126 MB L2, so no L2 flush is needed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -137,13 +137,22 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of the ranks' values (a device time): the job ends when the
+    slowest replica does."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank_step, steps, ms_max, world):
+    """Whole-job throughput of `world` independent replicas: every rank's
+    units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -250,7 +259,7 @@ def run_ours(args, world, rank):
     ms_max = max_over_ranks(ms, world)
     positions = [(args.warmup + s) % TRACE_LEN for s in range(args.steps)]
     step_bytes = float(np.mean(bytes_pos[positions]))
-    res = dict(ms=ms_max, tok_s=world * T * args.steps / (ms_max / 1e3), hbm_gbs=step_bytes * args.steps / (ms / 1e3) / 1e9,
+    res = dict(ms=ms_max, tok_s=replica_throughput(T, args.steps, ms_max, world), hbm_gbs=step_bytes * args.steps / (ms / 1e3) / 1e9,
                step_bytes=step_bytes, launches=launches_per_step * args.steps, clocks=clk.summary())
 
     # per-kernel device time over the same positions: a graph of the same pass
@@ -300,7 +309,7 @@ def run_ours(args, world, rank):
         a1.synchronize()
         barrier(world)
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
-    res["e2e"] = {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tok/s",
+    res["e2e"] = {"value": replica_throughput(T, args.steps, e2e_ms, world), "unit": "tok/s",
                   "h2d_bytes_per_step": int(host_x.numel() * 2 + host_lg[0].numel() * 4),
                   "d2h_bytes_per_step": int(host_out.numel() * 2)}
     del g, g2, final, final2
