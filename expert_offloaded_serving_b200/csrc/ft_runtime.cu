@@ -946,6 +946,8 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     return fail(FT_ERR_INVALID, "the MXFP4 prefill path needs hidden and inter to be multiples of 256");
   if (!mx && T > c->decode_max_t)
     return fail(FT_ERR_INVALID, "decode GEMV path takes T <= %d (use FT_ACT_MXFP4 for prefill)", c->decode_max_t);
+  if (!mx && !decode_supported(c->d.hidden, c->d.inter))
+    return fail(FT_ERR_INVALID, "decode GEMV path takes hidden and inter up to 16384 (use FT_ACT_MXFP4)");
   if (T == 0) return FT_OK;
   cudaStream_t s = (cudaStream_t)stream;
   const int H = c->d.hidden, E = c->d.n_experts, k = c->d.top_k, Ti = (int)T;
@@ -1128,6 +1130,8 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   if (n_layers <= 0 || first_layer < 0 || first_layer + n_layers > c->d.n_layers)
     return fail(FT_ERR_INVALID, "layers [%d, %d) outside [0, %d)", first_layer, first_layer + n_layers, c->d.n_layers);
   if (T < 0 || T > c->decode_max_t) return fail(FT_ERR_INVALID, "T=%lld outside [0, %d]", (long long)T, c->decode_max_t);
+  if (!decode_supported(c->d.hidden, c->d.inter))
+    return fail(FT_ERR_INVALID, "decode kernels take hidden and inter up to 16384");
   if (flags & FT_ACT_MXFP4) return fail(FT_ERR_INVALID, "the stacked forward is the decode path (FT_ACT_BF16)");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
   for (int l = first_layer; l < first_layer + n_layers; l++)
