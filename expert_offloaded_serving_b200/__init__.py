@@ -30,7 +30,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_expert_cache_lookup", "ft_expert_cache_insert", "ft_expert_cache_resize", "ft_cache_trace",
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
-           "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy")
+           "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -103,6 +103,7 @@ def lib() -> C.CDLL:
         "ft_debug_device_wait": (ST, [P, I64, P]),
         "ft_debug_host_wait_limit": (ST, [P, C.c_double]),
         "ft_debug_fail_copy": (ST, [P, I64]),
+        "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -253,6 +254,17 @@ def ft_debug_host_wait_limit(ctx, seconds: float) -> None:
 
 def ft_debug_fail_copy(ctx, n: int) -> None:
     _check(lib().ft_debug_fail_copy(ctx, n))
+
+
+GEOMETRY_FIELDS = ("K", "chunks", "lpr", "rpw", "parts", "rsets", "groups", "R", "smem", "taken")
+
+
+def ft_decode_geometry(hidden: int, inter: int, n_layers: int = 1) -> dict:
+    out = (I64 * 24)()
+    _check(lib().ft_decode_geometry(hidden, inter, n_layers, out))
+    tile = lambda o: {k: int(out[o + i]) for i, k in enumerate(GEOMETRY_FIELDS)}
+    return {"gate_up": tile(0), "down": tile(10), "threads": int(out[20]), "smem_limit": int(out[21]),
+            "stack": bool(out[22]), "sync_stride": int(out[23])}
 
 
 def ft_kernel_timing_enable(ctx, on: bool) -> None:

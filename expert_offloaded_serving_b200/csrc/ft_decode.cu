@@ -1305,6 +1305,27 @@ cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
 
 bool decode_supported(int H, int I) { return gv_ok(make_gv(H, I, 2), I) && gv_ok(make_gv(I, H, 1), H); }
 
+void decode_geometry(int H, int I, int64_t* out) {
+  const Gv gs[2] = {make_gv(H, I, 2), make_gv(I, H, 1)};
+  const int rows[2] = {I, H};
+  for (int p = 0; p < 2; p++) {
+    const Gv& g = gs[p];
+    int64_t* o = out + 10 * p;
+    o[0] = g.K;
+    o[1] = g.chunks;
+    o[2] = g.lpr;
+    o[3] = g.rpw;
+    o[4] = g.parts;
+    o[5] = g.rsets;
+    o[6] = g.groups;
+    o[7] = g.R;
+    o[8] = (int64_t)(kTileOff + g.total);
+    o[9] = gv_ok(g, rows[p]) ? 1 : 0;
+  }
+  out[20] = kGemvThreads;
+  out[21] = (int64_t)kSmemLimit;
+}
+
 constexpr size_t kStackSmemMax = 227 * 1024;  // opt-in dynamic shared memory per CTA
 
 bool stack_supported(int H, int I, int n_layers) {

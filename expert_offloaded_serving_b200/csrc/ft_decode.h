@@ -58,6 +58,11 @@ struct DecodeArgs {
 // True when the decode kernels take this shape (hidden and inter multiples of
 // 128, both at most 16384).
 bool decode_supported(int H, int I);
+// Tile geometry of the decode kernels for hidden H and intermediate I:
+// out[0..9] gate/up tile, out[10..19] down tile, each K, chunks, lpr, rpw,
+// parts, rsets, groups, R, shared bytes of a per-layer CTA, taken (0/1);
+// out[20] threads per CTA, out[21] the shared-memory limit of a tile.
+void decode_geometry(int H, int I, int64_t* out);
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // pdl: launch as a programmatic dependent of the previous kernel in the
 // stream.  The gate/up kernel reads its routing record and pointer table

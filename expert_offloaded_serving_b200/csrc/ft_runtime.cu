@@ -601,6 +601,17 @@ extern "C" ft_status ft_debug_dequant(ft_ctx* c, const void* blob, int32_t mat, 
   return FT_OK;
 }
 
+extern "C" ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_layers, int64_t out[24]) {
+  if (!out) return fail(FT_ERR_INVALID, "out is NULL");
+  if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128 || n_layers <= 0)
+    return fail(FT_ERR_INVALID, "hidden %d / inter %d not positive multiples of 128, or n_layers %d", hidden, inter,
+                n_layers);
+  decode_geometry(hidden, inter, out);
+  out[22] = stack_supported(hidden, inter, n_layers) ? 1 : 0;
+  out[23] = out[22] ? stack_sync_stride(hidden, inter) : 0;
+  return FT_OK;
+}
+
 extern "C" ft_status ft_debug_device_wait(ft_ctx* c, int64_t timeout_us, void* stream) {
   if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
   if (timeout_us < 1 || timeout_us > 2000000) return fail(FT_ERR_INVALID, "timeout_us %lld outside [1, 2e6]", (long long)timeout_us);

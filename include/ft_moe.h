@@ -298,6 +298,16 @@ FT_API ft_status ft_prefetch_layer(ft_ctx* ctx, int32_t layer, void* compute_str
  * routine the GEMV uses. */
 FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, float* out, void* stream);
 
+/* Tile geometry the decode kernels use for hidden H and intermediate I
+ * (host only, no device needed).  out[0..9] describe the gate/up tile and
+ * out[10..19] the down tile, each: K, 32-code chunks of K, lanes per row group
+ * (lpr), row groups per warp (rpw), K parts, row sets, lane groups per CTA, R
+ * rows per tile, shared-memory bytes of a per-layer CTA, 1 if the tile is
+ * taken; out[20] threads per CTA, out[21] the shared-memory limit of a tile,
+ * out[22] 1 if the persistent kernel takes a stack of n_layers layers of this
+ * shape, out[23] its counter words per layer.  FT_ERR_INVALID on a bad shape. */
+FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_layers, int64_t out[24]);
+
 /* Failure injection for tests: none of these fault or hang a GPU.
  *
  * ft_debug_device_wait: launch, on `stream`, one CTA that waits for a device

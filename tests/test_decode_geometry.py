@@ -1,0 +1,63 @@
+"""Tile geometry of the decode GEMV kernels (host logic, no GPU): for every
+shape the kernels take, the tile fits shared memory, covers K and the rows
+exactly, and keeps the row loop's trip count equal for all lanes of a warp
+(the xor-shuffle reductions need the whole warp); shapes past the limits are
+refused."""
+import pytest
+
+import expert_offloaded_serving_b200 as ft
+
+SIZES = [128, 256, 384, 512, 640, 768, 1024, 1536, 2048, 2560, 3072, 4096, 5120, 6144, 7168, 8192, 12288, 16384]
+OPT_IN_SMEM = 227 * 1024
+
+
+def is_pow2(v):
+    return v > 0 and (v & (v - 1)) == 0
+
+
+def check_tile(t, K, rows, threads, limit):
+    warps = threads // 32
+    assert t["K"] == K and t["chunks"] == K // 32
+    assert is_pow2(t["lpr"]) and t["lpr"] <= 32 and t["lpr"] * t["rpw"] == 32
+    assert t["lpr"] >= min(t["chunks"], 32)            # a lane group spans all chunks it can
+    assert t["parts"] * t["lpr"] >= t["chunks"] > (t["parts"] - 1) * t["lpr"]
+    assert 1 <= t["rsets"] and t["rsets"] * t["parts"] <= warps
+    assert t["groups"] == t["rsets"] * t["rpw"]
+    assert is_pow2(t["R"]) and 8 <= t["R"] <= 128 and rows % t["R"] == 0
+    assert t["smem"] <= 128 + limit <= OPT_IN_SMEM
+    # several lane groups share a warp only with one K part, and then R is a
+    # multiple of the groups per warp: every lane of a warp runs the same rows loop
+    if t["rpw"] > 1:
+        assert t["parts"] == 1 and t["R"] % t["rpw"] == 0
+
+
+@pytest.mark.parametrize("H", SIZES)
+@pytest.mark.parametrize("I", [128, 512, 768, 1536, 2048, 4096])
+def test_tiles_of_every_supported_shape(H, I):
+    g = ft.ft_decode_geometry(H, I, 40)
+    assert g["threads"] == 512
+    assert g["gate_up"]["taken"] and g["down"]["taken"]
+    check_tile(g["gate_up"], H, I, g["threads"], g["smem_limit"])
+    check_tile(g["down"], I, H, g["threads"], g["smem_limit"])
+    if g["stack"]:
+        assert g["sync_stride"] == 2 + H // g["down"]["R"]
+
+
+def test_35b_class_tiles_and_stack():
+    g = ft.ft_decode_geometry(2048, 512, 40)
+    assert (g["gate_up"]["R"], g["gate_up"]["lpr"], g["gate_up"]["parts"]) == (32, 32, 2)
+    assert (g["down"]["R"], g["down"]["lpr"], g["down"]["rpw"]) == (128, 16, 2)
+    # 9 units (8 routed + shared) x I/R = 144 gate/up tiles and x H/R = 144 down
+    # tiles: one of each per CTA on 148 SMs
+    assert 9 * 512 // g["gate_up"]["R"] == 144 and 9 * 2048 // g["down"]["R"] == 144
+    assert g["stack"] and g["sync_stride"] == 18
+
+
+def test_limits_are_refused():
+    g = ft.ft_decode_geometry(16384 + 128, 512, 1)        # K past 16384 chunks-per-warp coverage
+    assert not g["gate_up"]["taken"]
+    g = ft.ft_decode_geometry(2048, 512, 100000)           # the per-layer tile table outgrows shared memory
+    assert not g["stack"] and g["sync_stride"] == 0
+    with pytest.raises(ft.FtError) as e:
+        ft.ft_decode_geometry(2000, 512, 1)
+    assert e.value.status == ft.FT_ERR_INVALID
