@@ -305,7 +305,12 @@ static ft_status arena_map(ft_ctx* c, int64_t slots) {
     acc.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
     acc.location.id = c->device;
     acc.flags = CU_MEM_ACCESS_FLAGS_PROT_READWRITE;
-    CU_TRY(c->drv.memSetAccess(c->va + i * c->chunk, c->chunk, &acc, 1));
+    r = c->drv.memSetAccess(c->va + i * c->chunk, c->chunk, &acc, 1);
+    if (r != CUDA_SUCCESS) {  // undo this chunk's mapping; the chunks before it stay recorded
+      c->drv.memUnmap(c->va + i * c->chunk, c->chunk);
+      c->drv.memRelease(h);
+      return fail(FT_ERR_CUDA, "cuMemSetAccess failed (%d)", (int)r);
+    }
     c->chunks.push_back(h);
   }
   c->stats.mapped_bytes = (int64_t)(c->chunks.size() * c->chunk);
@@ -889,11 +894,25 @@ extern "C" ft_status ft_prefetch_layer(ft_ctx* c, int32_t layer, void* compute_s
   const int b = layer & 1;
   const size_t bytes = (size_t)c->n_blobs * c->stride;
   if (!c->d_stage[b]) {
-    CUDA_TRY(cudaMalloc((void**)&c->d_stage[b], bytes));
+    // both allocations, or neither: a later call must not find a buffer
+    // without its pointer table
+    uint8_t* stage = nullptr;
+    const uint8_t** table = nullptr;
     std::vector<const uint8_t*> tab(c->n_blobs);
-    for (int e = 0; e < c->n_blobs; e++) tab[e] = c->d_stage[b] + (size_t)e * c->stride;
-    CUDA_TRY(cudaMalloc((void**)&c->d_eptr_stage[b], c->n_blobs * sizeof(void*)));
-    CUDA_TRY(cudaMemcpy(c->d_eptr_stage[b], tab.data(), c->n_blobs * sizeof(void*), cudaMemcpyHostToDevice));
+    if (cudaMalloc((void**)&stage, bytes) != cudaSuccess ||
+        cudaMalloc((void**)&table, c->n_blobs * sizeof(void*)) != cudaSuccess) {
+      cudaFree(stage);
+      cudaGetLastError();
+      return fail(FT_ERR_CUDA, "staging buffer of %zu bytes", bytes);
+    }
+    for (int e = 0; e < c->n_blobs; e++) tab[e] = stage + (size_t)e * c->stride;
+    if (cudaMemcpy(table, tab.data(), c->n_blobs * sizeof(void*), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(stage);
+      cudaFree(table);
+      return fail(FT_ERR_CUDA, "staging pointer table");
+    }
+    c->d_stage[b] = stage;
+    c->d_eptr_stage[b] = table;
   }
   // reuse only after the last forward that read this buffer is done
   CUDA_TRY(cudaStreamWaitEvent(c->copy_stream, c->ev_done[b], 0));
