@@ -1,0 +1,72 @@
+"""Argument checks of the C ABI that run before any CUDA call, so they are
+tested without a GPU: every refusal of ft_create's descriptor check and of the
+allocation-free forward (fake, never dereferenced pointers stand in for
+device buffers)."""
+import pytest
+
+import expert_offloaded_serving_b200 as ft
+
+# stand-ins for device pointers: the calls refuse before touching them
+POOL, X, OUT, LG, WR = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000
+
+
+@pytest.mark.parametrize("desc,what", [
+    (dict(hidden=100), "hidden"),
+    (dict(hidden=0), "hidden"),
+    (dict(inter=96), "inter"),
+    (dict(n_experts=0), "n_experts"),
+    (dict(n_experts=1025), "n_experts"),
+    (dict(top_k=0), "top_k"),
+    (dict(top_k=17), "top_k"),
+    (dict(n_experts=4, top_k=5), "top_k"),
+    (dict(n_layers=0), "n_layers"),
+    (dict(n_shared=2), "n_shared"),
+    (dict(cache_budget_bytes=-1), "budget"),
+    (dict(max_tokens=0), "max_tokens"),
+])
+def test_create_refuses_each_bad_descriptor_field(desc, what):
+    base = dict(hidden=256, inter=128, n_experts=16, top_k=2, n_layers=1, n_shared=0, cache_budget_bytes=0,
+                max_tokens=16)
+    base.update(desc)
+    with pytest.raises(ft.FtError) as e:
+        ft.ft_create(ft.make_desc(**base))
+    assert e.value.status == ft.FT_ERR_INVALID
+    assert what in str(e.value)
+
+
+def noalloc(**kw):
+    a = dict(hidden=256, inter=128, n_experts=16, top_k=2, n_shared=0, layer_pool=POOL, x=X, T=1, router_w=None,
+             logits_override=LG, out=OUT, flags=ft.FT_ROUTE_RENORM)
+    a.update(kw)
+    ft.ft_moe_layer_forward_noalloc(a["hidden"], a["inter"], a["n_experts"], a["top_k"], a["n_shared"],
+                                    a["layer_pool"], a["x"], a["T"], a["router_w"], a["logits_override"], a["out"],
+                                    a["flags"], None, 0)  # stream 0: never used, the call refuses first
+
+
+@pytest.mark.parametrize("kw,what", [
+    (dict(layer_pool=None), "NULL"),
+    (dict(out=None), "NULL"),
+    (dict(x=None), "NULL"),
+    (dict(hidden=200), "multiples of 128"),
+    (dict(inter=0), "multiples of 128"),
+    (dict(n_experts=2000), "expert counts"),
+    (dict(top_k=17), "expert counts"),
+    (dict(n_shared=2), "expert counts"),
+    (dict(T=17), "T outside"),
+    (dict(T=-1), "T outside"),
+    (dict(flags=ft.FT_ACT_MXFP4), "decode"),
+    (dict(logits_override=None, router_w=None), "router_w or logits_override"),
+    (dict(out=X), "alias"),
+    # (16*8 + 16) rows of h at inter 16384 in fp32: 9.4 MB > 8 MiB of scratch
+    (dict(hidden=1024, inter=16384, top_k=8, n_shared=1, T=16), "maximum"),
+])
+def test_noalloc_refuses_before_touching_the_device(kw, what):
+    with pytest.raises(ft.FtError) as e:
+        noalloc(**kw)
+    assert e.value.status == ft.FT_ERR_INVALID
+    assert what in str(e.value)
+
+
+def test_noalloc_with_no_tokens_is_a_no_op():
+    noalloc(T=0)
+    noalloc(T=0, x=None)
