@@ -954,15 +954,16 @@ __device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* re
 // Wu) and then its down tiles (unit x R rows of Wd); tile i of a phase goes to
 // CTA i mod gridDim.  Dependencies between CTAs go through counters in global
 // memory.  Per layer: [0] gate/up tiles done (down waits for all of them);
-// [1] down tiles done (fused combine) or row blocks combined; [2 + rb] down
-// tiles done in row block rb.  With the fused combine (a.fused, few tokens)
+// [1] down tiles done (fused mode) or row blocks combined; [2 + rb] down
+// tiles done in row block rb.  In the fused mode (a.fused, one or two tokens)
 // the next layer's gate/up tiles rebuild their input from y themselves, so a
-// layer hands over after its last down tile; otherwise the last down tile of
-// a row block combines that block into the layer output and the next layer
-// waits for every row block.  A CTA streams its next tiles' weights while it
-// waits: the next layer's gate/up tile during the down phase, the next
-// layer's down tile during the gate/up phase.  Activations written by other
-// CTAs are read from L2 only.
+// layer hands over after its last down tile, and h goes from gate/up to down
+// as tagged words that the down tiles poll, without counter [0]; otherwise
+// the last down tile of a row block combines that block into the layer output
+// and the next layer waits for every row block.  A CTA streams its next
+// tiles' weights during a compute phase: the layer's first down tile during
+// gate/up, the next layer's first gate/up tile during down.  Activations
+// written by other CTAs are read from L2 only.
 // HS, IS: hidden and intermediate size fixed at compile time (the tile
 // geometry then folds to constants), or 0, 0 for any supported shape.
 template <int HS, int IS>
