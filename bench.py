@@ -363,6 +363,48 @@ def oracle_tok_s(T, budget_s=12.0, max_layers=12):
 # secondary measurements: prefill FP4 GEMM throughput with double-buffered
 # prefetch, expert-cache miss fetch bandwidth
 # ---------------------------------------------------------------------------
+FP4_DENSE_TFLOPS_NOMINAL = 9000.0   # B200 dense FP4 tensor peak, spec figure (not measured on this machine)
+EV_HIT, EV_MISS = 0, 1               # cache event kinds of the C ABI
+
+
+def miss_phases(events, per_token, phases):
+    """Miss rate of each named token range [a, b) of a decode run, from the
+    cache's event trace: the HIT/MISS lookups in order, per_token of them per
+    token (batch 1: one per selected expert and layer).  Returns None when the
+    trace does not hold exactly that many lookups."""
+    look = [e[0] for e in events if e[0] in (EV_HIT, EV_MISS)]
+    n_tok = max((b for _, (a, b) in phases), default=0)
+    if len(look) != n_tok * per_token:
+        return None
+    out = {}
+    for name, (a, b) in phases:
+        seg = look[a * per_token:b * per_token]
+        out[name] = sum(1 for k in seg if k == EV_MISS) / len(seg) if seg else None
+    return out
+
+
+def prefill_roofline(flops, weight_bytes, hbm_gbs, tflops):
+    """The prefill GEMM against its own roofline: min(FP4 dense peak, HBM
+    bandwidth x arithmetic intensity over the weight bytes it must read)."""
+    ai = flops / weight_bytes
+    roof = min(FP4_DENSE_TFLOPS_NOMINAL, hbm_gbs * ai / 1e3)
+    return {"flop_per_weight_byte": ai, "roofline_tflops": roof, "frac_of_roofline": tflops / roof,
+            "frac_of_fp4_nominal": tflops / FP4_DENSE_TFLOPS_NOMINAL,
+            "bound": "hbm" if roof < FP4_DENSE_TFLOPS_NOMINAL else "tensor"}
+
+
+def overlap_fraction(copy_ms, compute_ms, total_ms, hideable_ms):
+    """Share of the hideable compute time that ran under the copies, when
+    copies totalling copy_ms and computes totalling compute_ms took total_ms
+    together (1: all hideable compute hidden, 0: serialised), clamped to
+    [0, 1].  In a double-buffered run over n layers the first copy and the
+    last layer's compute have nothing to overlap with, so hideable_ms is the
+    compute of n - 1 layers."""
+    if hideable_ms <= 0:
+        return None
+    return max(0.0, min(1.0, (copy_ms + compute_ms - total_ms) / hideable_ms))
+
+
 def pinned_h2d_gbs(nbytes=1 << 30, reps=10):
     """Best-of-reps pinned host -> device copy bandwidth (GB/s)."""
     import torch
@@ -439,7 +481,12 @@ def measure_prefill(reps=3, layers=3):
            "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps,
            "layer_ms_resident": layer_ms,
            "kernels_ms": {k: v[0] / reps for k, v in kt.items() if v[1]}}
-    res["gemm_weight_gbs"] = E2 * ft.ft_blob_layout(H2, I2)["used"] / (gemm_ms * 1e-3) / 1e9
+    wbytes = E2 * ft.ft_blob_layout(H2, I2)["used"]
+    res["gemm_weight_gbs"] = wbytes / (gemm_ms * 1e-3) / 1e9
+    pk = peaks()
+    res["gemm_roofline"] = {**prefill_roofline(flops, wbytes, pk["hbm"], res["gemm_tflops"]),
+                            "hbm_peak_gbs": pk["hbm"], "hbm_peak_source": pk["src"],
+                            "fp4_peak_tflops": FP4_DENSE_TFLOPS_NOMINAL, "fp4_peak_source": "nominal"}
     # (b) pinned host pools, double-buffered prefetch
     hp = host_layer_pools(H2, I2, E2, seed, layers)
     ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, layers, 0, 0, T2), hp, None)
@@ -460,6 +507,14 @@ def measure_prefill(reps=3, layers=3):
     res["layer_ms_prefetched"] = a.elapsed_time(b) / layers
     res["prefetch_h2d_gbs"] = pack * layers / (a.elapsed_time(b) * 1e-3) / 1e9
     del hp
+    # overlap: each layer's copy alone at the measured pinned H2D rate and the
+    # resident layer's compute, against the prefetched run's time
+    h2d = pinned_h2d_gbs()
+    copy_ms = pack / (h2d * 1e9) * 1e3
+    res["pinned_h2d_gbs"] = h2d
+    res["copy_ms_per_layer_at_pinned"] = copy_ms
+    res["compute_hidden_frac"] = overlap_fraction(layers * copy_ms, layers * layer_ms, a.elapsed_time(b),
+                                                  (layers - 1) * layer_ms)
     return res
 
 
@@ -500,16 +555,23 @@ def measure_misses(tokens=64, layers=8):
     b.record()
     b.synchronize()
     st = ft.ft_cache_stats_get(ctx)
+    ev = ft.ft_cache_trace(ctx, cap=1 << 16)
     ft.ft_sync_status(ctx)
     ft.ft_destroy(ctx)
     del hp
+    total_ms = a.elapsed_time(b)
     lookups = st["hits"] + st["misses"]
     miss_gbs = st["h2d_bytes"] / (st["h2d_ms"] * 1e-3) / 1e9 if st["h2d_ms"] > 0 else None
+    t3 = tokens // 3
+    phases = miss_phases(ev, layers * k3, [("cold_first_token", (0, 1)), ("warm_full_budget", (1, t3)),
+                                          ("half_budget", (t3, 2 * t3)), ("restored_budget", (2 * t3, tokens))])
     return {"workload": f"DSV4-class decode with expert cache: {layers} of 43 layers, pools in pinned host memory, "
                         f"budget {budget / 1e9:.1f} GB (32 GB x {layers}/43), batch 1, {tokens} tokens, "
                         "resize to half and back",
-            "tok_s": tokens / (a.elapsed_time(b) * 1e-3) * layers / 43,
-            "miss_rate": st["misses"] / max(lookups, 1), "hits": st["hits"], "misses": st["misses"],
+            "tok_s": tokens / (total_ms * 1e-3) * layers / 43,
+            "miss_rate": st["misses"] / max(lookups, 1), "miss_rate_by_phase": phases,
+            "copy_busy_share": st["h2d_ms"] / total_ms if total_ms > 0 else None,
+            "hits": st["hits"], "misses": st["misses"],
             "evictions": st["evictions"], "moves": st["moves"], "miss_h2d_gbs": miss_gbs,
             "pinned_h2d_gbs": h2d_peak, "miss_h2d_frac": (miss_gbs / h2d_peak) if miss_gbs else None}
 
