@@ -128,6 +128,22 @@ def test_quantise_vectorised_matches_scalar():
             assert (c == codes[r, 32 * b:32 * b + 32]).all()
 
 
+def test_quantiser_keeps_the_sign_of_values_that_round_to_zero():
+    """A negative value whose scaled magnitude rounds to zero is stored as
+    code 8 (-0), a positive one as code 0, in both quantiser forms: the
+    element's sign bit is its input's sign bit (OCP MX: sign, then the
+    rounded magnitude)."""
+    v = np.zeros(32)
+    v[0] = 6.0                            # amax 6: scale 2^0, the grid itself
+    v[1], v[2], v[3], v[4] = -0.2, 0.2, -0.25, -0.0
+    c, e = fp4.quantize_block(v)
+    assert e == 127
+    assert (int(c[1]), int(c[2]), int(c[3]), int(c[4])) == (8, 0, 8, 8)
+    assert int(c[0]) == 7 and (c[5:] == 0).all()
+    rc, rs = fp4.quantize_rows(v[None, :])
+    assert (rc[0] == c).all() and int(rs[0, 0]) == 127
+
+
 def test_quantise_idempotent_on_representable_blocks():
     rng = np.random.default_rng(7)
     codes = rng.integers(0, 16, (64, 96)).astype(np.uint8)

@@ -64,6 +64,23 @@ def test_worked_example_mxfp4():
     assert (fp4.bf16_to_f64(r["out_bits"]) == 0.46875).all()
 
 
+def test_mxfp4_mode_sees_x_only_through_its_quantisation():
+    """In MXFP4-activation mode the expert reads x only as quantise(x):
+    feeding the dequantised codes instead gives the same output bit for bit
+    (quantisation is idempotent on representable blocks), while x itself is
+    not representable, so an expert that skipped the quantisation of x would
+    give a different output."""
+    H, I, seed = 256, 128, 1001
+    blob = synth.expert_blob(seed, 0, 3, H, I)
+    x = fp4.bf16_to_f64(synth.activations_bf16(seed, 2, 4, H))
+    xq = fp4.dequant_rows(*fp4.quantize_rows(x))
+    assert (xq != x).mean() > 0.5
+    y = layer.expert_ffn(blob, H, I, x, mxfp4=True)
+    assert (layer.expert_ffn(blob, H, I, xq, mxfp4=True) == y).all()
+    assert not np.allclose(layer.expert_ffn(blob, H, I, x, mxfp4=False),
+                           layer.expert_ffn(blob, H, I, xq, mxfp4=False), rtol=1e-3, atol=0)
+
+
 def test_partition_invariant_tiny_config():
     """Splitting a token's selected experts into any two groups, computing each
     group's weighted sum separately and adding the two gives the full output
