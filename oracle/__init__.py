@@ -14,6 +14,7 @@ Plain, slow and fp64 throughout, written from the public write-ups of FreeToken
 * ``layer``    SwiGLU expert FFN and the weighted combine (decode bf16 mode and
                MXFP4-activation mode).
 * ``lru``      the global LRU expert cache across layers, with resize.
+* ``formats``  BF16 and NVFP4 expert blobs (decode only), decoded to fp64.
 
 Pins (tests/test_oracle_*.py, all CPU): exhaustive code x scale tables against
 the closed form, hand-computed scale-atom offsets, quantiser ties and
@@ -21,10 +22,10 @@ idempotence, brute-force top-k with injected ties, stable-sort permutation
 invariants, a hand-computed two-expert layer (tests/golden/), the partition
 invariant of the combine, an LRU checked against a timestamp simulation, and
 sign, idempotence and quantised-input invariants of the quantiser and of the
-MXFP4 expert.  tests/test_oracle_mutants.py plants 33 plausible mistakes in
+MXFP4 expert.  tests/test_oracle_mutants.py plants 40 plausible mistakes in
 this package one at a time (wrong table entries, nibble and byte orders,
 rounding and tie rules, summation orders, swapped operands, dropped terms,
 recency rules); each makes at least one of those pins fail.
 No function here is "parity unpinned".
 """
-from . import fp4, routing, layer, lru  # noqa: F401
+from . import fp4, formats, routing, layer, lru  # noqa: F401

@@ -14,23 +14,29 @@ Modes:
 * ``mxfp4=False`` (decode): x is the bf16 input as is; h stays unrounded.
 * ``mxfp4=True`` (prefill): x and h are quantised per 32 values along their
   contraction axis by the OCP MX rule before each product.
+
+Weight formats (``weights``): "mxfp4" (the default), or "nvfp4" / "bf16"
+(``formats``), which are decode mode only.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from . import fp4, routing
+from . import formats, fp4, routing
 
 
 def silu(z: np.ndarray) -> np.ndarray:
     return z / (1.0 + np.exp(-z))
 
 
-def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray, mxfp4: bool = False) -> np.ndarray:
+def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray, mxfp4: bool = False,
+               weights: str = "mxfp4") -> np.ndarray:
     """y [m, H] = Wd (silu(Wg x) * (Wu x)) for the rows of x [m, H] (fp64)."""
-    wg = fp4.dequant_matrix(blob, "wg", hidden, inter)
-    wu = fp4.dequant_matrix(blob, "wu", hidden, inter)
-    wd = fp4.dequant_matrix(blob, "wd", hidden, inter)
+    if mxfp4 and weights != "mxfp4":
+        raise ValueError("MXFP4 activations are defined for MXFP4 weights only")
+    wg = formats.weight_matrix(blob, "wg", hidden, inter, weights)
+    wu = formats.weight_matrix(blob, "wu", hidden, inter, weights)
+    wd = formats.weight_matrix(blob, "wd", hidden, inter, weights)
     x = np.asarray(x, dtype=np.float64)
     if mxfp4:
         x = fp4.dequant_rows(*fp4.quantize_rows(x))
@@ -44,13 +50,14 @@ def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray, mxfp4: 
 
 def moe_layer(x_bits: np.ndarray, blob_of, hidden: int, inter: int, n_experts: int, top_k: int,
               logits: np.ndarray | None = None, router_w: np.ndarray | None = None,
-              renorm: bool = True, mxfp4: bool = False, shared_blob=None) -> dict:
+              renorm: bool = True, mxfp4: bool = False, shared_blob=None, weights: str = "mxfp4") -> dict:
     """One MoE layer on T tokens.
 
     x_bits   bf16 bits [T, H]
     blob_of  callable expert id -> blob (uint8)
     logits   fp32 [T, E] (used as given) or None to compute x . Wr^T
     shared_blob  blob of an always-on shared expert (weight 1) or None
+    weights  format of every blob ("mxfp4", "nvfp4", "bf16")
 
     Returns dict with logits, ids, w (fp64), offs/perm/inv, out_f64 and
     out_bits (bf16 of out_f64).
@@ -66,14 +73,14 @@ def moe_layer(x_bits: np.ndarray, blob_of, hidden: int, inter: int, n_experts: i
     y = {}
     for e in np.unique(ids):
         rows = np.nonzero((ids == e).any(axis=1))[0]
-        y[int(e)] = (rows, expert_ffn(blob_of(int(e)), hidden, inter, x[rows], mxfp4))
+        y[int(e)] = (rows, expert_ffn(blob_of(int(e)), hidden, inter, x[rows], mxfp4, weights))
     for t in range(T):
         acc = 0.0
         for j in range(top_k):
             rows, ye = y[int(ids[t, j])]
             acc = acc + w[t, j] * ye[int(np.nonzero(rows == t)[0][0])]
         if shared_blob is not None:
-            acc = acc + expert_ffn(shared_blob, hidden, inter, x[t:t + 1], mxfp4)[0]
+            acc = acc + expert_ffn(shared_blob, hidden, inter, x[t:t + 1], mxfp4, weights)[0]
         out[t] = acc
     return dict(logits=np.asarray(logits, dtype=np.float32), ids=ids, nonfinite=bad, w=w,
                 offs=offs, perm=perm, inv=inv, out_f64=out, out_bits=fp4.round_bf16(out))

@@ -137,6 +137,77 @@ def expert_blob(seed: int, layer: int, expert: int, hidden: int, inter: int) -> 
 
 
 # ---------------------------------------------------------------------------
+# BF16 and NVFP4 expert blobs
+# ---------------------------------------------------------------------------
+# BF16 blob: Wg [I][H], Wu [I][H], Wd [H][I] as little-endian bf16, zero padded
+# to a multiple of 256 bytes.  Each weight takes 16 random bits: 7 fraction
+# bits, a sign bit and an 8-bit draw of its binade [2^e, 2^(e+1)) from
+# BF16_BINADE_COUNTS (e = -14 .. -4, out of 256: the binade probabilities of
+# N(0, 0.02); the lowest binade also takes the mass below it), so that the
+# bytes are integer functions of the counter and a GPU filler can match them.
+BF16_BINADE_COUNTS = (1, 1, 2, 5, 10, 20, 38, 67, 81, 30, 1)
+BF16_BINADE_CUM = np.cumsum(BF16_BINADE_COUNTS).astype(np.uint64)
+BF16_EXP_LOW = 127 - 14                      # biased exponent of the lowest binade
+# NVFP4 blob: the MXFP4 code region (same code histogram), E4M3 block scales
+# (one per 16 elements) drawn uniformly from NVFP4_SCALE_BYTES, then the three
+# fp32 matrix scales NVFP4_TENSOR_SCALES (Wg, Wu, Wd) and 4 zero bytes.
+NVFP4_SCALE_BYTES = (0x72, 0x73, 0x74, 0x75)  # 160, 176, 192, 208
+NVFP4_TENSOR_SCALES = (0.875 * 2.0 ** -14, 1.125 * 2.0 ** -14, 1.375 * 2.0 ** -14)
+
+REGION_BF16 = 2
+REGION_E4M3 = 3
+
+
+def bf16_blob_regions(hidden: int, inter: int) -> dict:
+    H, I = hidden, inter
+    used = 6 * I * H
+    return dict(wg=0, wu=2 * I * H, wd=4 * I * H, used=used, stride=pad_up(used, 256))
+
+
+def nvfp4_blob_regions(hidden: int, inter: int) -> dict:
+    H, I = hidden, inter
+    codes_end = I * H + H * I // 2
+    sf_gu = pad_up(I, 128) * pad_up(H // 16, 4)
+    sf_d = pad_up(H, 128) * pad_up(I // 16, 4)
+    ts = codes_end + 2 * sf_gu + sf_d
+    return dict(wg=0, wu=I * H // 2, wd=I * H, codes_end=codes_end, wg_sf=codes_end, wu_sf=codes_end + sf_gu,
+                wd_sf=codes_end + 2 * sf_gu, tensor_scales=ts, used=ts + 16, stride=pad_up(ts + 16, 256))
+
+
+def bf16_weight_bits(seed: int, layer: int, expert: int, n: int) -> np.ndarray:
+    """``n`` bf16 bit patterns (uint16) of one expert's weights, in blob order."""
+    w = words(seed, blob_stream(layer, expert, REGION_BF16), 0, (n + 3) // 4)
+    f = np.stack([(w >> np.uint64(16 * q)) & np.uint64(0xFFFF) for q in range(4)], axis=1).reshape(-1)[:n]
+    binade = np.searchsorted(BF16_BINADE_CUM, f & np.uint64(0xFF), side="right").astype(np.uint64)
+    frac = (f >> np.uint64(8)) & np.uint64(0x7F)
+    sign = (f >> np.uint64(15)) & np.uint64(1)
+    return ((sign << np.uint64(15)) | ((binade + np.uint64(BF16_EXP_LOW)) << np.uint64(7)) | frac).astype(np.uint16)
+
+
+def expert_blob_bf16(seed: int, layer: int, expert: int, hidden: int, inter: int) -> np.ndarray:
+    r = bf16_blob_regions(hidden, inter)
+    blob = np.zeros(r["stride"], dtype=np.uint8)
+    blob[: r["used"]] = bf16_weight_bits(seed, layer, expert, r["used"] // 2).astype("<u2").view(np.uint8)
+    return blob
+
+
+def e4m3_scale_bytes(seed: int, layer: int, expert: int, nbytes: int) -> np.ndarray:
+    w = words(seed, blob_stream(layer, expert, REGION_E4M3), 0, (nbytes + 7) // 8)
+    b = np.stack([(w >> np.uint64(8 * q)) & np.uint64(0xFF) for q in range(8)], axis=1).reshape(-1)[:nbytes]
+    return np.asarray(NVFP4_SCALE_BYTES, dtype=np.uint8)[(b & np.uint64(3)).astype(np.int64)]
+
+
+def expert_blob_nvfp4(seed: int, layer: int, expert: int, hidden: int, inter: int) -> np.ndarray:
+    r = nvfp4_blob_regions(hidden, inter)
+    blob = np.zeros(r["stride"], dtype=np.uint8)
+    blob[: r["codes_end"]] = code_bytes(seed, layer, expert, r["codes_end"])
+    blob[r["codes_end"]: r["tensor_scales"]] = e4m3_scale_bytes(seed, layer, expert,
+                                                                  r["tensor_scales"] - r["codes_end"])
+    blob[r["tensor_scales"]: r["tensor_scales"] + 12] = np.asarray(NVFP4_TENSOR_SCALES, dtype="<f4").view(np.uint8)
+    return blob
+
+
+# ---------------------------------------------------------------------------
 # activations, router weights, traces, logits
 # ---------------------------------------------------------------------------
 

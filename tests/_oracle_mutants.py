@@ -11,7 +11,7 @@ import math
 
 import numpy as np
 
-from oracle import fp4, layer, lru, routing
+from oracle import formats, fp4, layer, lru, routing
 
 
 # ---------------------------------------------------------------------------
@@ -112,7 +112,7 @@ def quant_sign_of_zero():
     _rows_via_blocks()
 
 
-def _bf16(mode):
+def _bf16_rounding(mode):
     def bits(v):
         v = np.asarray(v, dtype=np.float64)
         if mode == "via_fp32":
@@ -139,15 +139,15 @@ def _bf16(mode):
 
 
 def bf16_ties_away():
-    _bf16("away")
+    _bf16_rounding("away")
 
 
 def bf16_truncate():
-    _bf16("truncate")
+    _bf16_rounding("truncate")
 
 
 def bf16_via_fp32():
-    _bf16("via_fp32")
+    _bf16_rounding("via_fp32")
 
 
 # ---------------------------------------------------------------------------
@@ -251,10 +251,10 @@ def silu_sign():
 
 
 def _ffn(swap=False, quant_x=True, quant_h=True):
-    def f(blob, hidden, inter, x, mxfp4=False):
-        wg = fp4.dequant_matrix(blob, "wg", hidden, inter)
-        wu = fp4.dequant_matrix(blob, "wu", hidden, inter)
-        wd = fp4.dequant_matrix(blob, "wd", hidden, inter)
+    def f(blob, hidden, inter, x, mxfp4=False, weights="mxfp4"):
+        wg = formats.weight_matrix(blob, "wg", hidden, inter, weights)
+        wu = formats.weight_matrix(blob, "wu", hidden, inter, weights)
+        wd = formats.weight_matrix(blob, "wd", hidden, inter, weights)
         x = np.asarray(x, dtype=np.float64)
         if mxfp4 and quant_x:
             x = fp4.dequant_rows(*fp4.quantize_rows(x))
@@ -285,6 +285,74 @@ def shared_expert_dropped():
         kw["shared_blob"] = None
         return orig(*a, **kw)
     layer.moe_layer = f
+
+
+# ---------------------------------------------------------------------------
+# BF16 and NVFP4 expert formats
+# ---------------------------------------------------------------------------
+
+def e4m3_bias():
+    formats.E4M3_TABLE[:] = [math.nan if (b & 0x7F) == 0x7F else
+                             (-1.0 if b & 0x80 else 1.0) * (math.ldexp((b & 7) / 8.0, -5) if (b >> 3) & 15 == 0
+                                                           else math.ldexp(1.0 + (b & 7) / 8.0, ((b >> 3) & 15) - 6))
+                             for b in range(256)]
+
+
+def e4m3_subnormal_as_normal():
+    for b in range(256):
+        if (b >> 3) & 15 == 0:
+            formats.E4M3_TABLE[b] = (-1.0 if b & 0x80 else 1.0) * math.ldexp(1.0 + (b & 7) / 8.0, -7)
+
+
+def _nvfp4(block=16, use_ts=True, ts_order=("wg", "wu", "wd")):
+    def f(blob, which, hidden, inter):
+        off = formats.nvfp4_layout(hidden, inter)
+        rows, K = (inter, hidden) if which in ("wg", "wu") else (hidden, inter)
+        blob = np.asarray(blob, dtype=np.uint8)
+        codes = blob[off[which]: off[which] + rows * K // 2].reshape(rows, K // 2)
+        elem = np.empty((rows, K), dtype=np.uint8)
+        elem[:, 0::2] = codes & 0x0F
+        elem[:, 1::2] = codes >> 4
+        nb = K // block
+        r = np.arange(rows, dtype=np.int64)[:, None]
+        b = np.arange(nb, dtype=np.int64)[None, :]
+        sc = formats.E4M3_TABLE[blob[off[which + "_sf"] + fp4.scale_index(r, b, nb)]]
+        t = blob[off["tensor_scales"]: off["tensor_scales"] + 12].copy().view("<f4").astype(np.float64)
+        ts = float(t[ts_order.index(which)]) if use_ts else 1.0
+        return fp4.E2M1_TABLE[elem] * np.repeat(sc, block, axis=1) * ts
+    formats.nvfp4_matrix = f
+
+
+def nvfp4_blocks_of_32():
+    _nvfp4(block=32)
+
+
+def nvfp4_matrix_scale_dropped():
+    _nvfp4(use_ts=False)
+
+
+def nvfp4_matrix_scales_rotated():
+    _nvfp4(ts_order=("wu", "wd", "wg"))
+
+
+def _bf16_matrix(big_endian=False, transposed=False):
+    def f(blob, which, hidden, inter):
+        off = formats.bf16_layout(hidden, inter)
+        rows, K = (inter, hidden) if which in ("wg", "wu") else (hidden, inter)
+        raw = np.asarray(blob, dtype=np.uint8)[off[which]: off[which] + 2 * rows * K].reshape(rows * K, 2)
+        hi, lo = (raw[:, 0], raw[:, 1]) if big_endian else (raw[:, 1], raw[:, 0])
+        bits = lo.astype(np.uint32) | (hi.astype(np.uint32) << 8)
+        v = (bits << np.uint32(16)).view(np.float32).astype(np.float64)
+        return v.reshape(K, rows).T.copy() if transposed else v.reshape(rows, K)
+    formats.bf16_matrix = f
+
+
+def bf16_big_endian():
+    _bf16_matrix(big_endian=True)
+
+
+def bf16_matrix_transposed():
+    _bf16_matrix(transposed=True)
 
 
 # ---------------------------------------------------------------------------
@@ -379,6 +447,8 @@ MUTANTS = {f.__name__: f for f in (
     topk_ties_to_higher_id, topk_nan_on_top, weights_not_renormalised, weights_reversed, logits_lane_of_element,
     logits_fp32_partials, logits_left_to_right, permutation_unstable, offsets_inclusive,
     silu_sign, gate_up_swapped, mxfp4_x_not_quantised, mxfp4_h_not_quantised, shared_expert_dropped,
+    e4m3_bias, e4m3_subnormal_as_normal, nvfp4_blocks_of_32, nvfp4_matrix_scale_dropped,
+    nvfp4_matrix_scales_rotated, bf16_big_endian, bf16_matrix_transposed,
     lru_evicts_most_recent, lru_may_evict_a_key_of_the_step, lru_takes_highest_free_slot, lru_hit_does_not_touch,
     resize_evicts_most_recent, resize_moves_descending, resize_moves_to_highest_free)}
 

@@ -12,7 +12,7 @@ import _oracle_mutants
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join("tests", f) for f in ("test_oracle_fp4.py", "test_oracle_routing.py", "test_oracle_layer.py",
-                                           "test_oracle_lru.py")]
+                                           "test_oracle_lru.py", "test_oracle_formats.py")]
 
 
 def run_pins(mutant):
@@ -31,6 +31,15 @@ def test_every_planted_mistake_fails_a_pin():
     broken = {n: out for n, (rc, failed, out) in res.items() if rc != 0 and (rc != 1 or not failed)}
     assert not broken, broken
     assert not survivors, f"pins do not catch: {survivors}"
+
+
+def test_mutant_helpers_are_not_shadowed():
+    """A second top-level definition with the same name would silently replace
+    the first and plant a different mistake than the one named."""
+    import ast
+    with open(_oracle_mutants.__file__) as f:
+        names = [n.name for n in ast.parse(f.read()).body if isinstance(n, ast.FunctionDef)]
+    assert len(names) == len(set(names)), sorted(n for n in set(names) if names.count(n) > 1)
 
 
 def test_an_unknown_mutant_is_refused():

@@ -34,3 +34,30 @@ def test_trace_overlap_and_distinct():
     lg = synth.logits_for_sets(1, 0, tr[:10], 256)
     top = np.argsort(-lg, axis=1, kind="stable")[:, :8]
     assert (top == tr[:10]).all()
+
+
+def test_bf16_blob_deterministic_keyed_and_shaped():
+    a = synth.expert_blob_bf16(7, 3, 5, 2048, 512)
+    assert (a == synth.expert_blob_bf16(7, 3, 5, 2048, 512)).all()
+    assert not (a == synth.expert_blob_bf16(7, 3, 6, 2048, 512)).all()
+    bits = a[:synth.bf16_blob_regions(2048, 512)["used"]].view("<u2")
+    binade = ((bits >> 7) & 0xFF).astype(np.int64) - synth.BF16_EXP_LOW
+    assert binade.min() >= 0 and binade.max() < len(synth.BF16_BINADE_COUNTS)
+    assert np.allclose(np.bincount(binade, minlength=11) / bits.size, np.array(synth.BF16_BINADE_COUNTS) / 256,
+                       atol=0.002)
+    assert abs((bits >> 15).mean() - 0.5) < 0.005
+    v = (bits.astype(np.uint32) << 16).view(np.float32)
+    assert 0.018 < v.std() < 0.026          # about N(0, 0.02)
+
+
+def test_nvfp4_blob_regions_and_bytes():
+    r = synth.nvfp4_blob_regions(2048, 512)
+    a = synth.expert_blob_nvfp4(7, 3, 5, 2048, 512)
+    assert (a == synth.expert_blob_nvfp4(7, 3, 5, 2048, 512)).all()
+    # the code region is the MXFP4 generator's, byte for byte
+    assert (a[:r["codes_end"]] == synth.code_bytes(7, 3, 5, r["codes_end"])).all()
+    sc = a[r["codes_end"]:r["tensor_scales"]]
+    assert set(np.unique(sc)) == set(synth.NVFP4_SCALE_BYTES)
+    ts = a[r["tensor_scales"]:r["tensor_scales"] + 12].view("<f4")
+    assert list(ts) == list(np.float32(synth.NVFP4_TENSOR_SCALES))
+    assert (a[r["tensor_scales"] + 12:] == 0).all()
