@@ -211,7 +211,6 @@ def run_ours(args, world, rank):
     logits_buf = torch.empty_like(logits_all[0])
     xb = synth.activations_bf16(SEED, 7, T, H)
     x0 = torch.from_numpy(xb.view(np.int16).copy()).cuda().view(torch.bfloat16)
-    bufs = [torch.empty_like(x0), torch.empty_like(x0)]
     # algorithmic bytes per step position: distinct routed experts + shared, whole blobs
     uniq = np.array([[len(np.unique(sets[p, layer])) for layer in range(L)] for p in range(TRACE_LEN)])
     bytes_pos = (uniq + S_SHARED).sum(axis=1) * used                 # [P]
@@ -493,7 +492,6 @@ def measure_prefill(reps=3, layers=3):
     torch.cuda.synchronize()
     a.record()
     ft.ft_prefetch_layer(ctx, 0)
-    cur = x
     for l in range(layers):
         if l + 1 < layers:
             ft.ft_prefetch_layer(ctx, l + 1)

@@ -3,7 +3,6 @@ whose output has a closed form, and the partition invariant of the combine."""
 import math
 
 import numpy as np
-import pytest
 
 from oracle import fp4, layer
 import synth
