@@ -17,7 +17,8 @@
 //                        fourth 16-column group of tokens from 16(w/4): SwiGLU
 //                        and MXFP4 quantisation of h (gate/up), or fp32 y (down)
 // All mbarrier waits are bounded; on a timeout the CTA records the TIMEOUT
-// status, stops issuing, frees its tensor memory and returns.
+// status, stops issuing, waits (bounded) for its copies still in flight, frees
+// its tensor memory and returns.
 //
 // Pages: prefill computes a whole layer's experts over many tokens while the
 // next layer's experts cross PCIe (aipolix.com, paragraph on bandwidth-
@@ -225,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
     // ---- producer ----
     const uint8_t* blob = a.pool + (int64_t)e * a.blob_stride;
     const uint32_t bytes = (NA + 1) * (kTileBytes + kSfBytes);
+    int issued = 0;  // K stages whose copies went out
     for (int kt = 0; kt < KT; kt++) {
       const int s = kt % S;
       if (kt >= S && !mbar_wait(&empty[s], ((kt / S) - 1) & 1)) {
@@ -240,7 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
       }
       tma_2d(tileB + s * kTileBytes, &maps.b, kt * (kGemmBK / 2), row0, &full[s]);
       bulk_g2s(sfB + s * kSfBytes, a.sfb + ((int64_t)jt * atoms_k + 2 * kt) * 512, kSfBytes, &full[s]);
+      issued = kt + 1;
     }
+    // No copy may still be writing this CTA's shared memory when it exits,
+    // also after a timeout of either role.  A stage is reissued only after
+    // the MMA consumed its previous round, so only the last S issued stages
+    // can be in flight; without a timeout the MMA thread has waited for the
+    // same phases, so these waits succeed at once.
+    for (int kt = issued > S ? issued - S : 0; kt < issued; kt++) mbar_wait(&full[kt % S], (kt / S) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issuer ----
     for (int kt = 0; kt < KT; kt++) {
