@@ -246,6 +246,7 @@ static ft_status check_desc(const ft_model_desc* d) {
   if (d->n_shared < 0 || d->n_shared > 1) return fail(FT_ERR_INVALID, "n_shared %d not 0 or 1", d->n_shared);
   if (d->cache_budget_bytes < 0) return fail(FT_ERR_INVALID, "negative cache budget");
   if (d->max_tokens <= 0) return fail(FT_ERR_INVALID, "max_tokens %d", d->max_tokens);
+  if (d->reserved != 0) return fail(FT_ERR_INVALID, "reserved field %d is not 0", d->reserved);
   return FT_OK;
 }
 

@@ -75,7 +75,7 @@ typedef struct {
   int32_t n_shared;           /* always-on shared experts per layer (weight 1), 0 or 1 */
   int64_t cache_budget_bytes; /* GPU expert-cache budget (0 = no cache) */
   int32_t max_tokens;         /* largest T any forward call passes; sizes scratch */
-  int32_t reserved;
+  int32_t reserved;           /* must be 0 */
 } ft_model_desc;
 
 /* forward / route flags */
@@ -203,8 +203,8 @@ FT_API ft_status ft_quantize_mxfp4(ft_ctx* ctx, const float* x, int64_t R, int32
  *   x dev bf16 [T][H]; out dev bf16 [T][H] (must not alias x).
  *   router_w dev fp32 [E][H], used when logits_override is NULL.
  *   logits_override dev fp32 [T][E] or NULL.
- *   flags: FT_ACT_BF16 (decode GEMV; T <= 64) or FT_ACT_MXFP4 (prefill
- *   grouped GEMM; any T <= max_tokens), | FT_ROUTE_RENORM.
+ *   flags: FT_ACT_BF16 (decode GEMV; T <= 16 and <= max_tokens) or
+ *   FT_ACT_MXFP4 (prefill grouped GEMM; any T <= max_tokens), | FT_ROUTE_RENORM.
  * Weights come from, in this order: the layer's resident device pool; the
  * prefill staging buffer if ft_prefetch_layer(layer) was issued (the compute
  * stream waits for that copy, [fa] double-buffered prefill); otherwise the
