@@ -66,3 +66,53 @@ def test_overlap_fraction_limits():
     assert bench.overlap_fraction(n * copy, n * comp, pipelined + comp / 2, (n - 1) * comp) == pytest.approx(0.75)
     assert bench.overlap_fraction(n * copy, n * comp, 1.0, (n - 1) * comp) == 1.0      # clamped
     assert bench.overlap_fraction(copy, comp, copy + comp, 0.0) is None
+
+
+def test_clock_reason_bits_match_nvml():
+    import pynvml
+    names = {"gpu_idle": "GpuIdle", "applications_clocks_setting": "ApplicationsClocksSetting",
+             "sw_power_cap": "SwPowerCap", "hw_slowdown": "HwSlowdown", "sw_thermal_slowdown": "SwThermalSlowdown",
+             "hw_thermal_slowdown": "HwThermalSlowdown", "hw_power_brake_slowdown": "HwPowerBrakeSlowdown",
+             "display_clock_setting": "DisplayClockSetting"}
+    for bit, name in bench.ClockSampler.REASONS.items():
+        assert getattr(pynvml, "nvmlClocksEventReason" + names[name]) == bit
+
+
+class FakeNvml:
+    """Stands in for pynvml during a timed region: SM clocks and the
+    clock-event reason bits it reports, one sample per poll."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, clocks, reasons):
+        self.clocks, self.reasons, self.i = clocks, reasons, 0
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        return self.clocks[min(self.i, len(self.clocks) - 1)]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        v = self.reasons[min(self.i, len(self.reasons) - 1)]
+        self.i += 1
+        return v
+
+
+def test_clock_sampler_reports_median_and_every_reason_seen():
+    import time
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples, s.reasons, s.max_mhz, s.h = [], 0, 1965, None
+    s._stop = bench.threading.Event()
+    s.nv = FakeNvml([1965, 1950, 1965, 1300, 1965], [0x1, 0x4, 0x0, 0x0, 0x20])
+    with s:
+        time.sleep(0.2)
+    out = s.summary()
+    assert out["sm_max_mhz"] == 1965 and out["samples"] == len(s.samples) >= 5
+    assert out["sm_mhz"] == 1965                                  # median, not the dip
+    assert out["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]   # idle is not a throttle reason
+
+
+def test_clock_sampler_without_nvml_says_so():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples, s.reasons, s.max_mhz, s.nv = [], 0, None, None
+    s._stop = bench.threading.Event()
+    with s:
+        pass
+    assert s.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
