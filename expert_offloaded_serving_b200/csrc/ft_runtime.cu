@@ -529,16 +529,19 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
 }
 
 // bounded host wait on an event: polls, gives up after `limit` seconds
+// Bounded host wait on an event: polls without sleeping for the first
+// kHostSpinSeconds (a decode layer's wait for its routed ids is tens of
+// microseconds, and a short sleep lasts tens of microseconds more than asked
+// on a stock kernel timer), then sleeps between polls until `limit`.
 static ft_status wait_event(cudaEvent_t ev, const char* what, double limit) {
-  auto t0 = std::chrono::steady_clock::now();
-  int spins = 0;
+  const auto t0 = std::chrono::steady_clock::now();
   while (true) {
     cudaError_t q = cudaEventQuery(ev);
     if (q == cudaSuccess) return FT_OK;
     if (q != cudaErrorNotReady) return fail(FT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(q));
-    if (++spins > 64) std::this_thread::sleep_for(std::chrono::microseconds(20));
-    double s = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+    const double s = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
     if (s > limit) return fail(FT_ERR_TIMEOUT, "%s: gave up after %.3f s", what, s);
+    if (s > kHostSpinSeconds) std::this_thread::sleep_for(std::chrono::microseconds(20));
   }
 }
 

@@ -12,6 +12,7 @@ namespace ft {
 constexpr int kDecodeMaxTokens = 16;               // largest T of the decode GEMV path
 constexpr size_t kArenaChunkBytes = 256ull << 20;  // physical chunk under the slot arena
 constexpr double kHostWaitSeconds = 30.0;          // bounded host waits
+constexpr double kHostSpinSeconds = 2e-3;          // ... polled without sleeping for this long first
 
 struct PrefillArgs {
   const uint16_t* x;  // bf16 [T][H]
