@@ -191,7 +191,8 @@ struct ft_ctx {
   uint8_t* d_shared = nullptr;  // [L][n_shared] blobs for non-resident layers
   std::vector<ft_cache_event> trace;
   ft_cache_stats stats{};
-  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> copy_timing;  // pending (start, end)
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> copy_timing;  // (start, end) of miss copies in flight
+  std::vector<cudaEvent_t> spare_events;                          // finished timing events, reused
 
   // prefill staging
   uint8_t* d_stage[2] = {nullptr, nullptr};
@@ -480,6 +481,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
     cudaEventDestroy(pr.first);
     cudaEventDestroy(pr.second);
   }
+  for (cudaEvent_t e : c->spare_events) cudaEventDestroy(e);
   free_prefill_scratch(c->pf);
   cudaFree(c->d_status);
   cudaFree(c->d_flag);
@@ -673,6 +675,34 @@ static int32_t evict_one(ft_ctx* c, const std::vector<int64_t>& keep, int64_t* v
   return -1;
 }
 
+// Timing of the miss copies: each cache step with a miss records a (start,
+// end) event pair around its copies on the copy stream.  Pairs finish in
+// issue order; finished ones are folded into stats.h2d_ms and their events
+// reused, so a long run holds only the pairs still in flight.
+static void fold_copy_timing(ft_ctx* c) {
+  size_t n = 0;
+  for (; n < c->copy_timing.size(); n++) {
+    const auto& pr = c->copy_timing[n];
+    if (cudaEventQuery(pr.second) != cudaSuccess) break;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess) c->stats.h2d_ms += ms;
+    c->spare_events.push_back(pr.first);
+    c->spare_events.push_back(pr.second);
+  }
+  c->copy_timing.erase(c->copy_timing.begin(), c->copy_timing.begin() + (std::ptrdiff_t)n);
+}
+
+static cudaEvent_t copy_event(ft_ctx* c) {
+  if (!c->spare_events.empty()) {
+    cudaEvent_t e = c->spare_events.back();
+    c->spare_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
 // Issue the H2D copy of (layer, e) into `slot` on the copy stream.
 static ft_status fetch(ft_ctx* c, int layer, int e, int32_t slot) {
   if (c->fail_copy_in > 0 && --c->fail_copy_in == 0)
@@ -689,6 +719,7 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
   if ((int64_t)S.size() > c->lru.capacity)
     return fail(FT_ERR_NO_SPACE, "%zu experts in one step exceed the cache capacity of %lld slots", S.size(),
                 (long long)c->lru.capacity);
+  fold_copy_timing(c);
   std::vector<int64_t> keep;
   keep.reserve(S.size());
   for (int e : S) keep.push_back(key_of(c, layer, e));
@@ -712,8 +743,8 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
       slot = c->lru.lowest_free();
     }
     if (!any_miss) {
-      cudaEventCreate(&t0);
-      cudaEventCreate(&t1);
+      t0 = copy_event(c);
+      t1 = copy_event(c);
       cudaEventRecord(t0, c->copy_stream);
     }
     any_miss = true;
@@ -868,13 +899,7 @@ extern "C" ft_status ft_cache_stats_get(ft_ctx* c, ft_cache_stats* out, int32_t 
   if (!c || !out) return fail(FT_ERR_INVALID, "NULL argument");
   if (!c->copy_timing.empty()) {
     CUDA_TRY(cudaStreamSynchronize(c->copy_stream));
-    for (auto& pr : c->copy_timing) {
-      float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess) c->stats.h2d_ms += ms;
-      cudaEventDestroy(pr.first);
-      cudaEventDestroy(pr.second);
-    }
-    c->copy_timing.clear();
+    fold_copy_timing(c);
   }
   *out = c->stats;
   if (reset) {
