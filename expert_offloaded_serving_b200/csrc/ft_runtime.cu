@@ -190,6 +190,7 @@ struct ft_ctx {
   bool cache_on = false;
   uint8_t* d_shared = nullptr;  // [L][n_shared] blobs for non-resident layers
   std::vector<ft_cache_event> trace;
+  int64_t trace_dropped = 0;  // events not recorded because the trace was full
   ft_cache_stats stats{};
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> copy_timing;  // (start, end) of miss copies in flight
   std::vector<cudaEvent_t> spare_events;                          // finished timing events, reused
@@ -648,7 +649,13 @@ extern "C" ft_status ft_debug_fail_copy(ft_ctx* c, int64_t n) {
 // ---------------------------------------------------------------------------
 // expert cache
 // ---------------------------------------------------------------------------
+// Between two reads the trace keeps at most kTraceMaxEvents events; later
+// ones are counted and dropped, so a run that never reads it stays bounded.
 static void record(ft_ctx* c, int kind, int layer, int expert, int slot, int from) {
+  if ((int64_t)c->trace.size() >= kTraceMaxEvents) {
+    c->trace_dropped++;
+    return;
+  }
   c->trace.push_back(ft_cache_event{kind, layer, expert, slot, from});
 }
 
@@ -889,8 +896,13 @@ extern "C" ft_status ft_cache_trace(ft_ctx* c, ft_cache_event* buf, int64_t cap,
   int64_t m = std::min<int64_t>(cap, (int64_t)c->trace.size());
   if (m > 0) memcpy(buf, c->trace.data(), (size_t)m * sizeof(ft_cache_event));
   *n = m;
-  bool over = (int64_t)c->trace.size() > cap;
+  const bool over = (int64_t)c->trace.size() > cap;
+  const int64_t dropped = c->trace_dropped;
   c->trace.clear();
+  c->trace_dropped = 0;
+  if (dropped > 0)
+    return fail(FT_ERR_NO_SPACE, "%lld events were dropped: the trace holds at most %lld between reads",
+                (long long)dropped, (long long)kTraceMaxEvents);
   if (over) return fail(FT_ERR_NO_SPACE, "trace had more events than cap");
   return FT_OK;
 }

@@ -13,6 +13,7 @@ constexpr int kDecodeMaxTokens = 16;               // largest T of the decode GE
 constexpr size_t kArenaChunkBytes = 256ull << 20;  // physical chunk under the slot arena
 constexpr double kHostWaitSeconds = 30.0;          // bounded host waits
 constexpr double kHostSpinSeconds = 2e-3;          // ... polled without sleeping for this long first
+constexpr int64_t kTraceMaxEvents = 1ll << 22;     // cache events kept between two trace reads
 
 struct PrefillArgs {
   const uint16_t* x;  // bf16 [T][H]

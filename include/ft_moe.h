@@ -272,7 +272,10 @@ FT_API ft_status ft_expert_cache_resize(ft_ctx* ctx, int64_t new_budget_bytes);
 
 /* Copy out the cache events recorded since the last call (HIT, MISS, EVICT,
  * MOVE in order) and clear them.  *n = events written (<= cap); if more were
- * recorded than cap the rest are dropped and FT_ERR_NO_SPACE is returned. */
+ * recorded than cap the rest are dropped and FT_ERR_NO_SPACE is returned.
+ * Between two calls the context keeps at most 4,194,304 events (80 MiB); the
+ * events after that are not recorded, and the next call copies out the ones
+ * kept and returns FT_ERR_NO_SPACE. */
 FT_API ft_status ft_cache_trace(ft_ctx* ctx, ft_cache_event* buf, int64_t cap, int64_t* n);
 
 /* Counters since creation (or the last reset). */
