@@ -854,7 +854,11 @@ extern "C" ft_status ft_expert_cache_resize(ft_ctx* c, int64_t new_budget) {
   CUDA_TRY(cudaDeviceSynchronize());
   int64_t cap = new_budget / c->stride;
   if ((size_t)cap * c->stride > c->va_size) return fail(FT_ERR_NO_SPACE, "budget larger than the reserved arena");
-  if (cap < c->lru.capacity) {
+  const int64_t old_cap = c->lru.capacity;
+  // grow: map the physical memory first, so that the capacity only ever
+  // covers mapped slots (a failed map leaves the old capacity in force)
+  if (cap > old_cap) FT_TRY(arena_map(c, cap));
+  if (cap < old_cap) {
     while ((int64_t)c->lru.map.size() > cap) evict_one(c, {});
     // survivors in slots >= cap move down to the lowest free slots, ascending
     std::vector<std::pair<int32_t, int64_t>> movers;
@@ -883,9 +887,10 @@ extern "C" ft_status ft_expert_cache_resize(ft_ctx* c, int64_t new_budget) {
   }
   c->lru.set_capacity(cap);
   for (int64_t s2 = cap; s2 < (int64_t)c->lru.slot_used.size(); s2++) c->lru.slot_used[s2] = 0;
-  FT_TRY(arena_map(c, cap));
   c->stats.capacity_slots = cap;
   c->stats.used_slots = (int64_t)c->lru.map.size();
+  // shrink: unmap only after the survivors moved below the new capacity
+  if (cap < old_cap) FT_TRY(arena_map(c, cap));
   CUDA_TRY(cudaMemcpy(c->d_eptr_cache, c->h_eptr_cache, (size_t)c->d.n_layers * c->n_blobs * sizeof(void*),
                       cudaMemcpyHostToDevice));
   return FT_OK;
