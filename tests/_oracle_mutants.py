@@ -429,6 +429,12 @@ def lru_hit_does_not_touch():
     _step(hit_touches=False)
 
 
+def lru_lookup_does_not_touch():
+    def lookup(self, lay, expert):
+        return self.slot.get((lay, int(expert)), -1)
+    lru.LRUCache.lookup = lookup
+
+
 def resize_evicts_most_recent():
     _resize(evict_mru=True)
 
@@ -450,6 +456,7 @@ MUTANTS = {f.__name__: f for f in (
     e4m3_bias, e4m3_subnormal_as_normal, nvfp4_blocks_of_32, nvfp4_matrix_scale_dropped,
     nvfp4_matrix_scales_rotated, bf16_big_endian, bf16_matrix_transposed,
     lru_evicts_most_recent, lru_may_evict_a_key_of_the_step, lru_takes_highest_free_slot, lru_hit_does_not_touch,
+    lru_lookup_does_not_touch,
     resize_evicts_most_recent, resize_moves_descending, resize_moves_to_highest_free)}
 
 

@@ -108,3 +108,19 @@ def test_lru_all_hits_when_everything_fits():
             else:
                 assert kind == lru.MISS
             seen.add((l, e))
+
+
+def test_lookup_touches_a_hit_and_leaves_a_miss_alone():
+    """A lookup hit makes the key most recent, which changes the next victim;
+    a lookup miss returns -1 and changes nothing."""
+    c = lru.LRUCache(2)
+    c.step(0, [1])
+    c.step(0, [2])                                   # recency: (0,1) then (0,2)
+    assert c.lookup(0, 1) == 0                       # (0,1) becomes most recent
+    assert c.lookup(0, 7) == -1
+    ev = c.step(0, [3])
+    assert ev == [(lru.EVICT, 0, 2, 1, -1), (lru.MISS, 0, 3, 1, -1)]
+    d = lru.LRUCache(2)
+    d.step(0, [1])
+    d.step(0, [2])
+    assert d.step(0, [3]) == [(lru.EVICT, 0, 1, 0, -1), (lru.MISS, 0, 3, 0, -1)]   # without the lookup
