@@ -22,7 +22,7 @@ idempotence, brute-force top-k with injected ties, stable-sort permutation
 invariants, a hand-computed two-expert layer (tests/golden/), the partition
 invariant of the combine, an LRU checked against a timestamp simulation, and
 sign, idempotence and quantised-input invariants of the quantiser and of the
-MXFP4 expert.  tests/test_oracle_mutants.py plants 41 plausible mistakes in
+MXFP4 expert.  tests/test_oracle_mutants.py plants 44 plausible mistakes in
 this package one at a time (wrong table entries, nibble and byte orders,
 rounding and tie rules, summation orders, swapped operands, dropped terms,
 recency rules); each makes at least one of those pins fail.

@@ -157,13 +157,3 @@ def weight_matrix(blob: np.ndarray, which: str, hidden: int, inter: int, weights
     if weights == "bf16":
         return bf16_matrix(blob, which, hidden, inter)
     raise ValueError(f"unknown weight format {weights!r}")
-
-
-def blob_stride(hidden: int, inter: int, weights: str = "mxfp4") -> int:
-    if weights == "mxfp4":
-        return fp4.layout(hidden, inter)["stride"]
-    if weights == "nvfp4":
-        return nvfp4_layout(hidden, inter)["stride"]
-    if weights == "bf16":
-        return bf16_layout(hidden, inter)["stride"]
-    raise ValueError(f"unknown weight format {weights!r}")

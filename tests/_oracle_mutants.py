@@ -43,6 +43,20 @@ def nibble_order():
     fp4.dequant_matrix = f
 
 
+def pack_high_nibble_first():
+    fp4.pack_codes = lambda codes: ((codes[:, 0::2] << 4) | codes[:, 1::2]).astype(np.uint8)
+
+
+def dequant_rows_scales_tiled():
+    # np.tile where np.repeat belongs: element k takes block k mod (K/32)'s scale
+    fp4.dequant_rows = lambda codes, scales: fp4.E2M1_TABLE[codes] * np.tile(fp4.UE8M0_TABLE[scales], (1, 32))
+
+
+def bf16_decode_low_half():
+    fp4.bf16_to_f64 = lambda bits: (np.asarray(bits, dtype=np.uint16).astype(np.uint32)).view(np.float32).astype(
+        np.float64)
+
+
 def _scale_index(word_of, byte_of):
     def f(row, kblock, n_kblocks):
         atoms_k = -(-int(n_kblocks) // 4)
@@ -449,6 +463,7 @@ def resize_moves_to_highest_free():
 
 MUTANTS = {f.__name__: f for f in (
     e2m1_magnitude, e2m1_negative_zero, ue8m0_bias, nibble_order, scale_atom_row_major, scale_word_byte_swapped,
+    pack_high_nibble_first, dequant_rows_scales_tiled, bf16_decode_low_half,
     quant_emax_one, quant_ties_away, quant_sign_of_zero, bf16_ties_away, bf16_truncate, bf16_via_fp32,
     topk_ties_to_higher_id, topk_nan_on_top, weights_not_renormalised, weights_reversed, logits_lane_of_element,
     logits_fp32_partials, logits_left_to_right, permutation_unstable, offsets_inclusive,
