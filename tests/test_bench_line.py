@@ -62,3 +62,27 @@ def test_derived_figures(line):
     assert line["value"] == pytest.approx(1e3 / 0.3238)
     assert line["gpu_launches"] == 20
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 16
+
+
+def test_layerwise_line_reports_the_gate_up_kernel(monkeypatch, capsys):
+    gu_bytes = 9 * 1_114_112.0                      # Wg + Wu codes and scales of 9 units
+
+    def fake(args, world, rank):
+        r = fake_decode(args, world, rank)
+        r["kernels"] = {"gate_up": {"ms_total": 0.0136 * 40 * args.steps, "launches": 40 * args.steps, "us_avg": 13.6},
+                        "down_combine": {"ms_total": 0.0136 * 40 * args.steps, "launches": 40 * args.steps,
+                                         "us_avg": 13.6}}
+        r["gate_up_bytes"], r["down_bytes"] = gu_bytes, gu_bytes / 2
+        return r
+    monkeypatch.setattr(bench, "dist_setup", lambda args: (1, 0, 0))
+    monkeypatch.setattr(bench, "run_ours", fake)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "4", "--warmup", "3", "--layerwise", "--no-extra"])
+    monkeypatch.setattr(bench, "oracle_tok_s", lambda T: (0.22, 12, 16))
+    bench.main()
+    line = json.loads([ln for ln in capsys.readouterr().out.splitlines() if ln.strip()][0])
+    r = line["roofline"]
+    assert r["kernel"] == "gate_up" and r["traffic"] is None
+    assert r["achieved"] == pytest.approx(gu_bytes / 13.6e-6 / 1e9)
+    assert line["gate_up_gbs"] == pytest.approx(r["achieved"])
+    assert "prefill" not in line and "miss" not in line
+    assert line["config"]["decode_kernels"] == "two per layer"
