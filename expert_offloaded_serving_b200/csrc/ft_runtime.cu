@@ -12,6 +12,7 @@
 // the engine or reloading the host-resident pool (aipolix.com, paragraph on
 // elastic memory management).
 #include <cuda.h>  // driver types only; entry points come from cudaGetDriverEntryPoint
+#include <nvtx3/nvToolsExt.h>  // header-only; inert unless a profiler attaches
 
 #include <algorithm>
 #include <chrono>
@@ -30,6 +31,19 @@
 #include "ft_runtime.h"
 
 using namespace ft;
+
+// ---------------------------------------------------------------------------
+// host-side ranges for NVTX-aware profilers (ncu --nvtx, nsys); without one
+// attached the calls return at once
+// ---------------------------------------------------------------------------
+namespace {
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace
 
 // ---------------------------------------------------------------------------
 // errors
@@ -817,6 +831,7 @@ extern "C" ft_status ft_expert_cache_lookup(ft_ctx* c, int32_t layer, int32_t ex
 
 extern "C" ft_status ft_expert_cache_insert(ft_ctx* c, int32_t layer, int32_t expert, int32_t* slot,
                                             int64_t* evicted_key, void* stream) {
+  NvtxRange nvtx_range("ft_expert_cache_insert");
   if (!c || !slot) return fail(FT_ERR_INVALID, "NULL argument");
   if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
   if (layer < 0 || layer >= c->d.n_layers || expert < 0 || expert >= c->d.n_experts)
@@ -848,6 +863,7 @@ extern "C" ft_status ft_expert_cache_insert(ft_ctx* c, int32_t layer, int32_t ex
 }
 
 extern "C" ft_status ft_expert_cache_resize(ft_ctx* c, int64_t new_budget) {
+  NvtxRange nvtx_range("ft_expert_cache_resize");
   if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
   if (new_budget < 0) return fail(FT_ERR_INVALID, "negative budget");
   if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
@@ -933,6 +949,7 @@ extern "C" ft_status ft_cache_stats_get(ft_ctx* c, ft_cache_stats* out, int32_t 
 // prefetch
 // ---------------------------------------------------------------------------
 extern "C" ft_status ft_prefetch_layer(ft_ctx* c, int32_t layer, void* compute_stream) {
+  NvtxRange nvtx_range("ft_prefetch_layer");
   if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
   if (layer < 0 || layer >= c->d.n_layers) return fail(FT_ERR_INVALID, "layer %d out of range", layer);
   if (!c->host_layers[layer]) return fail(FT_ERR_NOT_FOUND, "layer %d has no host pool", layer);
@@ -1012,6 +1029,7 @@ static RouteArgs route_args(ft_ctx* c, const float* logits, int T, int n_layers,
 extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* x, int64_t T,
                                           const float* router_w, const float* logits_override, void* out,
                                           uint32_t flags, void* stream) {
+  NvtxRange nvtx_range("ft_moe_layer_forward");
   if (!c || !out || (!x && T > 0)) return fail(FT_ERR_INVALID, "NULL argument");
   if (layer < 0 || layer >= c->d.n_layers) return fail(FT_ERR_INVALID, "layer %d out of range", layer);
   if (T < 0 || T > c->max_tokens) return fail(FT_ERR_INVALID, "T=%lld outside [0, max_tokens=%d]", (long long)T, c->max_tokens);
@@ -1083,7 +1101,10 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     S.erase(std::unique(S.begin(), S.end()), S.end());
     std::vector<int> dirty{layer};
     bool any_miss = false;
-    FT_TRY(cache_step(c, layer, S, any_miss, dirty));
+    {
+      NvtxRange step_range("cache_step");
+      FT_TRY(cache_step(c, layer, S, any_miss, dirty));
+    }
     if (any_miss) CUDA_TRY(cudaStreamWaitEvent(s, c->copy_timing.back().second, 0));
     FT_TRY(push_table_rows(c, dirty, s));
     eptr = c->d_eptr_cache + (size_t)layer * c->n_blobs;
@@ -1202,6 +1223,7 @@ extern "C" ft_status ft_kernel_timing_read(ft_ctx* c, double* ms, int64_t* launc
 // ---------------------------------------------------------------------------
 extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_t n_layers, const void* x, int64_t T,
                                           const float* logits, void* out, uint32_t flags, void* stream) {
+  NvtxRange nvtx_range("ft_moe_stack_forward");
   if (!c || !x || !out || !logits) return fail(FT_ERR_INVALID, "NULL argument");
   if (n_layers <= 0 || first_layer < 0 || first_layer + n_layers > c->d.n_layers)
     return fail(FT_ERR_INVALID, "layers [%d, %d) outside [0, %d)", first_layer, first_layer + n_layers, c->d.n_layers);
