@@ -114,11 +114,16 @@ def lib() -> C.CDLL:
 
 
 def _ptr(t) -> int | None:
-    """Device/host pointer of a torch tensor, an int, or None."""
+    """Device/host pointer of a torch tensor, an int, or None.  The ABI takes
+    dense row-major buffers, so a strided view is refused rather than read
+    with the wrong layout."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_contiguous():
+        raise ValueError(f"tensor of shape {tuple(t.shape)} and strides {t.stride()} is not contiguous; "
+                         "the C ABI takes dense row-major buffers")
     return t.data_ptr()
 
 

@@ -75,3 +75,15 @@ def test_noalloc_refuses_before_touching_the_device(kw, what):
 def test_noalloc_with_no_tokens_is_a_no_op():
     noalloc(T=0)
     noalloc(T=0, x=None)
+
+
+def test_binding_refuses_strided_views():
+    """The binding passes data pointers: a transposed or sliced-with-step view
+    would be read as if dense, so it is refused before the library is called."""
+    import torch
+    x = torch.zeros(8, 4, dtype=torch.bfloat16).t()
+    with pytest.raises(ValueError, match="not contiguous"):
+        ft.ft_moe_layer_forward(0, 0, x, 4, None, torch.zeros(4, 16), torch.zeros(4, 8), 1, 0)
+    with pytest.raises(ValueError, match="not contiguous"):
+        ft.ft_moe_route(0, torch.zeros(4, 32)[:, ::2], 4, 16, 2, 1, torch.zeros(4, 2, dtype=torch.int32),
+                        torch.zeros(4, 2), 0)
