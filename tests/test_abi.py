@@ -48,3 +48,18 @@ def test_create_rejects_bad_desc_without_touching_the_gpu():
     assert e.value.status == ft.FT_ERR_INVALID
     with pytest.raises(ft.FtError):
         ft.ft_create(ft.make_desc(256, 128, 16, 17))
+
+
+def test_every_declaration_is_documented():
+    """Each entry point of the header has its own comment above it, or is
+    named in an earlier comment block that documents it with its neighbours
+    (meaning of the arguments, layouts, ownership, errors live there)."""
+    src = open(os.path.join(ROOT, "include", "ft_moe.h")).read()
+    comments = [m for m in re.finditer(r"/\*.*?\*/", src, flags=re.S)]
+    prev = 0
+    for m in re.finditer(r"^FT_API\s+[\w\s\*]*?\b(ft_\w+)\s*\(", src, flags=re.M):
+        name = m.group(1)
+        own = [c for c in comments if prev <= c.start() and c.end() <= m.start() and len(c.group(0)) > 40]
+        named = [c for c in comments if c.end() <= m.start() and name in c.group(0)]
+        assert own or named, name
+        prev = src.index(";", m.end()) + 1
