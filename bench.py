@@ -575,6 +575,25 @@ def measure_misses(tokens=64, layers=8):
 
 
 
+def measure_decode_batch(args, T, pk):
+    """The same 35B-class decode stack at batch T (the workload's other batch
+    size): tokens/s, ms per step, end-to-end tokens/s and the persistent
+    kernel's bandwidth on its algorithmic bytes (the union of the batch's
+    experts and the shared one per layer)."""
+    import copy
+    a = copy.copy(args)
+    a.tokens = T
+    res = run_ours(a, 1, 0)
+    out = {"workload": workload_config(T)["workload"], "tok_s": res["tok_s"], "ms_per_step": res["ms"] / a.steps,
+           "e2e_tok_s": res["e2e"]["value"], "algorithmic_bytes_per_step": res["stack_bytes"],
+           "clocks": res["clocks"]}
+    st = res["kernels"].get("dec_stack")
+    if st:
+        gbs = res["stack_bytes"] / (st["us_avg"] * 1e-6) / 1e9
+        out.update(kernel_us=st["us_avg"], kernel_gbs=gbs, kernel_frac=gbs / pk["hbm"])
+    return out
+
+
 def workload_config(T, layerwise=False):
     return {"decode_kernels": "two per layer" if layerwise else "persistent stack kernel",
             "workload": f"35B-A3B-class MoE decode stack: hidden {H}, {E} routed experts top-{K_TOP} + {S_SHARED} shared, "
@@ -655,6 +674,11 @@ def main():
             line["miss"] = measure_misses()
         except Exception as ex:
             line["miss"] = {"error": repr(ex)}
+        if T == 1 and not args.layerwise:
+            try:
+                line["decode_batch4"] = measure_decode_batch(args, 4, pk)
+            except Exception as ex:
+                line["decode_batch4"] = {"error": repr(ex)}
     if world == 1:
         v, done, threads = oracle_tok_s(T)
         line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",

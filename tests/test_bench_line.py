@@ -14,6 +14,7 @@ STACK_BYTES = 601_620_480.0          # 40 layers x 9 units x 1,671,168 B at batc
 
 
 def fake_decode(args, world, rank):
+    assert world == 1 and args.tokens in (1, 4)
     us = 316.0
     return dict(ms=args.steps * 0.3238, tok_s=1e3 / 0.3238, hbm_gbs=1858.0, step_bytes=STACK_BYTES,
                 launches=2 * args.steps, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 40},
@@ -50,6 +51,8 @@ def test_contract_keys(line):
     assert set(line["e2e"]) == {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
     assert set(line["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
     assert line["prefill"] == {"workload": "prefill"} and line["miss"] == {"workload": "miss"}
+    b4 = line["decode_batch4"]
+    assert "batch 4" in b4["workload"] and b4["tok_s"] > 0 and 0 < b4["kernel_frac"] < 1.5
 
 
 def test_derived_figures(line):
