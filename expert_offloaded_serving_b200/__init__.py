@@ -113,10 +113,12 @@ def lib() -> C.CDLL:
     return L
 
 
-def _ptr(t) -> int | None:
+def _ptr(t, size: int | None = None) -> int | None:
     """Device/host pointer of a torch tensor, an int, or None.  The ABI takes
     dense row-major buffers, so a strided view is refused rather than read
-    with the wrong layout."""
+    with the wrong layout; `size` is the element size in bytes the argument
+    holds (2 for bf16 activations, 4 for fp32 / int32, 1 for codes), checked
+    on tensors."""
     if t is None:
         return None
     if isinstance(t, int):
@@ -124,6 +126,9 @@ def _ptr(t) -> int | None:
     if not t.is_contiguous():
         raise ValueError(f"tensor of shape {tuple(t.shape)} and strides {t.stride()} is not contiguous; "
                          "the C ABI takes dense row-major buffers")
+    if size is not None and t.element_size() != size:
+        raise ValueError(f"tensor of dtype {t.dtype} has {t.element_size()}-byte elements where the C ABI "
+                         f"takes {size}-byte ones")
     return t.data_ptr()
 
 
@@ -183,33 +188,34 @@ def ft_sync_status(ctx: int, stream=None) -> None:
 
 
 def ft_router_logits(ctx, x, T, H, wr, E, logits, stream=None) -> None:
-    _check(lib().ft_router_logits(ctx, _ptr(x), T, H, _ptr(wr), E, _ptr(logits), _stream(stream)))
+    _check(lib().ft_router_logits(ctx, _ptr(x, 2), T, H, _ptr(wr, 4), E, _ptr(logits, 4), _stream(stream)))
 
 
 def ft_moe_route(ctx, logits, T, E, k, flags, ids, w, stream=None) -> None:
-    _check(lib().ft_moe_route(ctx, _ptr(logits), T, E, k, flags, _ptr(ids), _ptr(w), _stream(stream)))
+    _check(lib().ft_moe_route(ctx, _ptr(logits, 4), T, E, k, flags, _ptr(ids, 4), _ptr(w, 4), _stream(stream)))
 
 
 def ft_moe_permute(ctx, ids, T, k, E, offs, perm, inv, stream=None) -> None:
-    _check(lib().ft_moe_permute(ctx, _ptr(ids), T, k, E, _ptr(offs), _ptr(perm), _ptr(inv), _stream(stream)))
+    _check(lib().ft_moe_permute(ctx, _ptr(ids, 4), T, k, E, _ptr(offs, 4), _ptr(perm, 4), _ptr(inv, 4),
+                                _stream(stream)))
 
 
 def ft_quantize_mxfp4(ctx, x, R, K, codes, scales, stream=None) -> None:
-    _check(lib().ft_quantize_mxfp4(ctx, _ptr(x), R, K, _ptr(codes), _ptr(scales), _stream(stream)))
+    _check(lib().ft_quantize_mxfp4(ctx, _ptr(x, 4), R, K, _ptr(codes, 1), _ptr(scales, 1), _stream(stream)))
 
 
 def ft_moe_layer_forward(ctx, layer, x, T, router_w, logits_override, out, flags, stream=None) -> None:
-    _check(lib().ft_moe_layer_forward(ctx, layer, _ptr(x), T, _ptr(router_w), _ptr(logits_override), _ptr(out),
-                                      flags, _stream(stream)))
+    _check(lib().ft_moe_layer_forward(ctx, layer, _ptr(x, 2), T, _ptr(router_w, 4), _ptr(logits_override, 4),
+                                      _ptr(out, 2), flags, _stream(stream)))
 
 
 def ft_moe_stack_forward(ctx, first_layer, n_layers, x, T, logits, out, flags, stream=None) -> None:
-    _check(lib().ft_moe_stack_forward(ctx, first_layer, n_layers, _ptr(x), T, _ptr(logits), _ptr(out), flags,
-                                      _stream(stream)))
+    _check(lib().ft_moe_stack_forward(ctx, first_layer, n_layers, _ptr(x, 2), T, _ptr(logits, 4), _ptr(out, 2),
+                                      flags, _stream(stream)))
 
 
 def ft_last_routing(ctx, ids, w, n, stream=None) -> None:
-    _check(lib().ft_last_routing(ctx, _ptr(ids), _ptr(w), n, _stream(stream)))
+    _check(lib().ft_last_routing(ctx, _ptr(ids, 4), _ptr(w, 4), n, _stream(stream)))
 
 
 def ft_expert_cache_lookup(ctx, layer, expert) -> int:
@@ -288,9 +294,9 @@ def ft_moe_layer_forward_noalloc(hidden, inter, n_experts, top_k, n_shared, laye
                                  logits_override, out, flags, status=None, stream=None) -> None:
     """Decode forward that allocates no device memory (scratch in a static
     device array shared by all calls; see ft_moe.h)."""
-    _check(lib().ft_moe_layer_forward_noalloc(hidden, inter, n_experts, top_k, n_shared, _ptr(layer_pool), _ptr(x),
-                                              T, _ptr(router_w), _ptr(logits_override), _ptr(out), flags,
-                                              _ptr(status), _stream(stream)))
+    _check(lib().ft_moe_layer_forward_noalloc(hidden, inter, n_experts, top_k, n_shared, _ptr(layer_pool),
+                                              _ptr(x, 2), T, _ptr(router_w, 4), _ptr(logits_override, 4),
+                                              _ptr(out, 2), flags, _ptr(status, 4), _stream(stream)))
 
 
 def make_desc(hidden, inter, n_experts, top_k, n_layers=1, n_shared=0, cache_budget_bytes=0,

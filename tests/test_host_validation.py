@@ -87,3 +87,13 @@ def test_binding_refuses_strided_views():
     with pytest.raises(ValueError, match="not contiguous"):
         ft.ft_moe_route(0, torch.zeros(4, 32)[:, ::2], 4, 16, 2, 1, torch.zeros(4, 2, dtype=torch.int32),
                         torch.zeros(4, 2), 0)
+
+
+def test_binding_refuses_wrong_element_sizes():
+    """fp32 where bf16 activations go, or int64 ids, would be misread: refused."""
+    import torch
+    with pytest.raises(ValueError, match="2-byte"):
+        ft.ft_moe_layer_forward(0, 0, torch.zeros(4, 8), 4, None, torch.zeros(4, 16), torch.zeros(4, 8), 1, 0)
+    with pytest.raises(ValueError, match="4-byte"):
+        ft.ft_moe_route(0, torch.zeros(4, 16), 4, 16, 2, 1, torch.zeros(4, 2, dtype=torch.int64), torch.zeros(4, 2),
+                        0)
