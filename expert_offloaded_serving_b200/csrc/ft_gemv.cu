@@ -273,17 +273,30 @@ static int dn_rows_per_cta(int I, int RW) {
   return 4 * (32 / lpr) * RW;
 }
 
+// A K of c = K/32 chunks is split over lpr = min(32, c) lanes: the xor
+// butterfly of group_sum needs lpr to be a power of two, and the chunk loop
+// (J = c / lpr chunks per lane) needs c to be a multiple of lpr.  So c is 4, 8,
+// 16 or a multiple of 32 (K = 128, 256, 512 or a multiple of 1024).  The
+// gate/up kernel stages up to 4 tokens of x as fp32 in shared memory (16 * H
+// bytes), which bounds H by the 227 KB a CTA may use.
+static bool gemv_k_ok(int K) {
+  if (K <= 0 || K % 128) return false;
+  const int c = K / 32;
+  return c < 32 ? (c & (c - 1)) == 0 : c % 32 == 0;
+}
+
+bool gemv_shape_ok(int H, int I) { return gemv_k_ok(H) && gemv_k_ok(I) && (size_t)16 * H <= 227 * 1024; }
+
 template <int MT>
 static cudaError_t launch_gu_mt(const GemvParams& p, cudaStream_t s) {
   constexpr int RW = 4;
   int rows = gu_rows_per_cta(p.H, RW);
   dim3 grid((p.I + rows - 1) / rows, p.max_active + p.n_shared);
   size_t smem = (size_t)MT * p.H * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_gate_up<MT, RW>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr = true;
-  }
+  // the attribute is per device: set it on every launch (cheap, and correct
+  // when several devices or host threads use the library)
+  cudaError_t e = cudaFuncSetAttribute(k_gate_up<MT, RW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   k_gate_up<MT, RW><<<grid, 256, smem, s>>>(p);
   return cudaGetLastError();
 }
@@ -299,11 +312,8 @@ cudaError_t launch_down_combine(const GemvParams& p, cudaStream_t s) {
   int rows = dn_rows_per_cta(p.I, RW);
   int n_pairs = p.T * p.k + p.n_shared * p.T;
   size_t smem = (size_t)n_pairs * rows * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_down_combine<RW>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr = true;
-  }
+  cudaError_t e = cudaFuncSetAttribute(k_down_combine<RW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   k_down_combine<RW><<<(p.H + rows - 1) / rows, 128, smem, s>>>(p);
   return cudaGetLastError();
 }

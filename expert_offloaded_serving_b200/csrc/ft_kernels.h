@@ -32,6 +32,10 @@ cudaError_t launch_topk(const float* logits, int T, int E, int k, int renorm, in
 size_t permute_smem_bytes(int E);
 cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* offs, int32_t* perm, int32_t* inv,
                            int32_t* active, int32_t* n_active, int32_t* pad_offs, int* status, cudaStream_t s);
+// True when the context-free GEMV kernels below take hidden H and
+// intermediate I: each K (H or I) is 128, 256, 512 or a multiple of 1024,
+// and H <= 14336 (four tokens of fp32 x fit one CTA's shared memory).
+bool gemv_shape_ok(int H, int I);
 cudaError_t launch_gate_up(const GemvParams& p, cudaStream_t s);
 cudaError_t launch_down_combine(const GemvParams& p, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int rows, int K, float* out,

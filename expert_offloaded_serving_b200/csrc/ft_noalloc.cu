@@ -9,8 +9,14 @@
 // nothing: its scratch (routing ids and weights, the permutation, the blob
 // pointer table and the fp32 SwiGLU activations) lives in one file-scope
 // __device__ array of kNoAllocScratchBytes, which every GPU that loads the
-// library holds until the process exits.  It runs the same kernels as
-// ft_moe_layer_forward on a resident layer pool.
+// library holds until the process exits.  It computes what the decode path of
+// ft_moe_layer_forward computes on a resident layer pool, with the
+// context-free kernels: the router GEMV, top-k and permutation of
+// ft_route.cu, then the split-K GEMVs of ft_gemv.cu (launch_gate_up,
+// launch_down_combine).  Those GEMVs take fewer shapes than the context's
+// decode kernels (see gemv_shape_ok) and round differently (fp32 x and h, no
+// f16 re-encoding), so the two paths agree within the output tolerance, not
+// bit for bit.
 #include <cstdio>
 #include <mutex>
 
@@ -72,6 +78,8 @@ extern "C" ft_status ft_moe_layer_forward_noalloc(int32_t hidden, int32_t inter,
   const int H = hidden, I = inter, E = n_experts, k = top_k, S = n_shared;
   if (!layer_pool || !out || (!x && T > 0)) return bad("NULL argument");
   if (H <= 0 || H % 128 || I <= 0 || I % 128) return bad("hidden and inter must be positive multiples of 128");
+  if (!ft::gemv_shape_ok(H, I))
+    return bad("hidden and inter must each be 128, 256, 512 or a multiple of 1024, and hidden at most 14336");
   if (E <= 0 || E > 1024 || k <= 0 || k > 16 || k > E || S < 0 || S > 1) return bad("bad expert counts");
   if (T < 0 || T > ft::kDecodeMaxTokens) return bad("T outside [0, 16] (decode path only)");
   if (flags & FT_ACT_MXFP4) return bad("only the decode (bf16-activation) path has a no-alloc form");

@@ -54,6 +54,14 @@ def noalloc(**kw):
     (dict(x=None), "NULL"),
     (dict(hidden=200), "multiples of 128"),
     (dict(inter=0), "multiples of 128"),
+    # the split-K GEMV spreads a row over min(32, K/32) lanes: that count must
+    # be a power of two and divide K/32 (K = 384 gives 12 lanes, K = 1152 gives
+    # 36 chunks over 32 lanes)
+    (dict(hidden=384), "multiple of 1024"),
+    (dict(hidden=1152), "multiple of 1024"),
+    (dict(inter=384), "multiple of 1024"),
+    (dict(inter=1152), "multiple of 1024"),
+    (dict(hidden=15360), "at most 14336"),
     (dict(n_experts=2000), "expert counts"),
     (dict(top_k=17), "expert counts"),
     (dict(n_shared=2), "expert counts"),
