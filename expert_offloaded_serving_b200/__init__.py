@@ -30,7 +30,8 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_expert_cache_lookup", "ft_expert_cache_insert", "ft_expert_cache_resize", "ft_cache_trace",
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
-           "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry")
+           "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry",
+           "ft_debug_stack_epoch")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -103,6 +104,7 @@ def lib() -> C.CDLL:
         "ft_debug_device_wait": (ST, [P, I64, P]),
         "ft_debug_host_wait_limit": (ST, [P, C.c_double]),
         "ft_debug_fail_copy": (ST, [P, I64]),
+        "ft_debug_stack_epoch": (ST, [P, U32, I32]),
         "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
     for name, (res, args) in sig.items():
@@ -265,6 +267,10 @@ def ft_debug_host_wait_limit(ctx, seconds: float) -> None:
 
 def ft_debug_fail_copy(ctx, n: int) -> None:
     _check(lib().ft_debug_fail_copy(ctx, n))
+
+
+def ft_debug_stack_epoch(ctx, epoch: int, poison_layer: int = -1) -> None:
+    _check(lib().ft_debug_stack_epoch(ctx, epoch & 0xFFFFFFFF, poison_layer))
 
 
 GEOMETRY_FIELDS = ("K", "chunks", "lpr", "rpw", "parts", "rsets", "groups", "R", "smem", "taken")

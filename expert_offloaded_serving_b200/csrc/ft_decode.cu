@@ -414,6 +414,15 @@ __device__ __forceinline__ float fma_f16x2(uint32_t w, uint32_t x, float acc) {
   return acc;
 }
 
+// Codes (16 bytes, 32 e2m1 values) and decoded UE8M0 scale of chunk c of
+// staged row `row` (rows of all matrices of the tile counted in order).
+__device__ __forceinline__ void tile_chunk(const Gv& g, const uint8_t* codes, const uint32_t* sc, int row, int c,
+                                           uint4& q, float& s) {
+  q = *reinterpret_cast<const uint4*>(codes + (size_t)row * (g.K / 2) + c * 16);
+  const uint32_t sw = sc[(size_t)row * g.atoms + (c >> 2)];
+  s = ue8m0_to_f32((sw >> (8 * (c & 3))) & 0xffu);
+}
+
 // Dot of one chunk of 32 e2m1 codes with NT tokens' f16 activations x[t][i]
 // (elements 2i, 2i+1); even code bytes feed one accumulator, odd ones the
 // other.
@@ -493,9 +502,9 @@ __device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8
         v[u][0] = v[u][1] = 0.f;
         if (cv) {
           const int row = mat * g.R + m.grp + (j0 + u) * g.groups;
-          const uint4 q = *reinterpret_cast<const uint4*>(codes + (size_t)row * (g.K / 2) + m.c * 16);
-          const uint32_t sw = sc[(size_t)row * g.atoms + (m.c >> 2)];
-          const float s = ue8m0_to_f32((sw >> (8 * (m.c & 3))) & 0xffu);
+          uint4 q;
+          float s;
+          tile_chunk(g, codes, sc, row, m.c, q, s);
           float d[NT];
           chunk_dot<NT>(q, x, d);
 #pragma unroll
@@ -676,6 +685,49 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
     for (int s = 0; s < a.n_shared; s++) acc += __ldcg(a.y + (size_t)(a.T * a.k + s * a.T + t) * a.H + n);
     __nv_bfloat16 b = __float2bfloat16_rn(acc);
     a.out[(size_t)t * a.H + n] = *reinterpret_cast<uint16_t*>(&b);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// parity export: matrix `mat` of a blob dequantised through the GEMV tile.
+// CTA = R rows staged exactly as the GEMV kernels stage them (stage_mat),
+// then each (row, chunk) is read back with tile_chunk and its codes decoded by
+// e2m1x8_to_f16x8, the conversion the dot products use; out = f16 value x
+// UE8M0 scale (exact in fp32 unless it overflows).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kGemvThreads, 1) k_dec_dequant(const uint8_t* blob, BlobLayout lay, int mat, int H,
+                                                                 int I, float* out) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* base = smem + kTileOff;
+  const int K = mat < 2 ? H : I, rows = mat < 2 ? I : H;
+  const Gv g = make_gv(K, rows, 1);
+  const int row0 = blockIdx.x * g.R;
+  const int64_t co = mat == 0 ? lay.wg : mat == 1 ? lay.wu : lay.wd;
+  const int64_t so = mat == 0 ? lay.wg_sf : mat == 1 ? lay.wu_sf : lay.wd_sf;
+  stage_mat(g, base, 0, blob + co, blob + so, row0);
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+  const uint8_t* codes = base + g.codes;
+  const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
+  for (int i = threadIdx.x; i < g.R * g.chunks; i += kGemvThreads) {
+    const int r = i / g.chunks, c = i - r * g.chunks;
+    uint4 q;
+    float s;
+    tile_chunk(g, codes, sc, r, c, q, s);
+    const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+    float* o = out + (size_t)(row0 + r) * K + c * 32;
+#pragma unroll
+    for (int wv = 0; wv < 4; wv++) {
+      uint32_t hv[4];
+      e2m1x8_to_f16x8(qs[wv], hv);
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const float2 f = f16x2_to_f32x2(hv[j]);
+        o[8 * wv + 2 * j] = f.x * s;
+        o[8 * wv + 2 * j + 1] = f.y * s;
+      }
+    }
   }
 }
 
@@ -1247,10 +1299,19 @@ __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
   for (int i = threadIdx.x; i < (int)(sizeof(Route) / 16); i += kThreads) dst[i] = src[i];
   if (a.sync)
     for (int i = threadIdx.x; i < a.sync_stride; i += kThreads) a.sync[(size_t)l * a.sync_stride + i] = 0;
-  if (a.epoch && l == 0 && threadIdx.x == 0) {
-    uint32_t e = *a.epoch + 1u;
-    if ((e << 7) == 0u) e += 1u;  // tags (e << 7 | layer) never equal the zeroed buffer's
-    *a.epoch = e;
+  if (a.epoch && l == 0) {
+    // tags (e << 7 | layer) never equal a zeroed word's; when they wrap (every
+    // 2^25 launches) the tagged words are zeroed, so that no word left from
+    // 2^25 launches ago can carry a tag of this launch
+    __shared__ int wrapped;
+    if (threadIdx.x == 0) {
+      bool w;
+      *a.epoch = next_epoch(*a.epoch, &w);
+      wrapped = w;
+    }
+    __syncthreads();
+    if (wrapped)
+      for (int64_t i = threadIdx.x; i < a.tagged_words; i += kThreads) a.tagged[i] = 0ull;
   }
   if (l == a.n_layers - 1 && a.ids_out) {
     for (int f = threadIdx.x; f < a.T * a.k; f += kThreads) {
@@ -1302,6 +1363,18 @@ cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const Gv g = make_gv(a.I, a.H, 1);
   return launch_one(k_dec_down, a, g, a.H, (a.max_units + a.n_shared) * (a.H / g.R), pdl, s);
+}
+
+cudaError_t launch_dec_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int H, int I, float* out,
+                               cudaStream_t s) {
+  const int K = mat < 2 ? H : I, rows = mat < 2 ? I : H;
+  const Gv g = make_gv(K, rows, 1);
+  if (!gv_ok(g, rows)) return cudaErrorInvalidValue;
+  const size_t smem = kTileOff + g.total;
+  cudaError_t e = cudaFuncSetAttribute(k_dec_dequant, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_dec_dequant<<<rows / g.R, kGemvThreads, smem, s>>>(blob, lay, mat, H, I, out);
+  return cudaGetLastError();
 }
 
 bool decode_supported(int H, int I) { return gv_ok(make_gv(H, I, 2), I) && gv_ok(make_gv(I, H, 1), H); }

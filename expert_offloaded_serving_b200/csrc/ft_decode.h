@@ -39,7 +39,20 @@ struct RouteArgs {
   int* sync;            // [n_layers][sync_stride] zeroed by CTA l for layer l, or NULL
   int sync_stride;
   uint32_t* epoch;      // launch counter the persistent kernel tags its h with; CTA 0 adds 1, or NULL
+  uint64_t* tagged;     // the persistent kernel's tagged words: CTA 0 zeroes them when the counter wraps
+  int64_t tagged_words;
 };
+
+// Launch counter after `e`: e + 1, skipping values whose tags (e << 7 | layer,
+// 32 bits) could equal a zeroed word's.  *wrapped is set when it skipped, i.e.
+// when the tags start repeating those of 2^25 launches before.
+__host__ __device__ inline uint32_t next_epoch(uint32_t e, bool* wrapped) {
+  uint32_t n = e + 1u;
+  const bool w = (n << 7) == 0u;
+  if (w) n += 1u;
+  if (wrapped) *wrapped = w;
+  return n;
+}
 
 struct DecodeArgs {
   const uint16_t* x;       // bf16 [T][H]
@@ -64,6 +77,11 @@ bool decode_supported(int H, int I);
 // out[20] threads per CTA, out[21] the shared-memory limit of a tile.
 void decode_geometry(int H, int I, int64_t* out);
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+// Matrix mat (0 Wg, 1 Wu, 2 Wd) of one blob dequantised to fp32 [rows][K]
+// through the GEMV tile's staging and code decoder (shape must satisfy
+// decode_supported).
+cudaError_t launch_dec_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int H, int I, float* out,
+                               cudaStream_t s);
 // pdl: launch as a programmatic dependent of the previous kernel in the
 // stream.  The gate/up kernel reads its routing record and pointer table
 // before griddepcontrol.wait, so it may only be launched that way when both

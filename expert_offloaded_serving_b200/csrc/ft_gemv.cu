@@ -1,7 +1,7 @@
-// Decode GEMV of the allocation-free forward (ft_moe_layer_forward_noalloc)
-// and the dequantiser behind ft_debug_dequant: split-K FP4 GEMV of the
-// selected experts, dequantising e2m1 codes with their UE8M0 block scales in
-// registers.  (The context's decode path is ft_decode.cu.)
+// Decode GEMV of the allocation-free forward (ft_moe_layer_forward_noalloc):
+// split-K FP4 GEMV of the selected experts, dequantising e2m1 codes with their
+// UE8M0 block scales in registers.  (The context's decode path is
+// ft_decode.cu.)
 //
 //   k_gate_up        h[pair][i] = silu(Wg[i] . x) * (Wu[i] . x)      (fp32 h)
 //   k_down_combine   y[pair][n] = Wd[n] . h[pair];
@@ -315,39 +315,6 @@ cudaError_t launch_down_combine(const GemvParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k_down_combine<RW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_down_combine<RW><<<(p.H + rows - 1) / rows, 128, smem, s>>>(p);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// parity export: dequantise one matrix of a blob with the same chunk decoder
-// ---------------------------------------------------------------------------
-__global__ void k_dequant(const uint8_t* __restrict__ blob, BlobLayout lay, int mat, int rows, int K,
-                          float* __restrict__ out) {
-  int chunks = K / 32;
-  int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows * chunks) return;
-  int row = idx / chunks, c = idx % chunks;
-  int64_t off = mat == 0 ? lay.wg : (mat == 1 ? lay.wu : lay.wd);
-  int64_t sfo = mat == 0 ? lay.wg_sf : (mat == 1 ? lay.wu_sf : lay.wd_sf);
-  int atoms_k = (int)(pad_up(K / 32, 4) / 4);
-  uint4 q = *(reinterpret_cast<const uint4*>(blob + off + (size_t)row * (K / 2)) + c);
-  float sc = ue8m0_to_f32(blob[sfo + sf_word(row, c >> 2, atoms_k) + (c & 3)]);
-  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
-  float* o = out + (size_t)row * K + c * 32;
-#pragma unroll
-  for (int wv = 0; wv < 4; wv++)
-#pragma unroll
-    for (int b = 0; b < 4; b++) {
-      float2 f = f16x2_to_f32x2(e2m1x2_to_f16x2(qs[wv] >> (8 * b)));
-      o[(wv * 4 + b) * 2] = f.x * sc;
-      o[(wv * 4 + b) * 2 + 1] = f.y * sc;
-    }
-}
-
-cudaError_t launch_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int rows, int K, float* out,
-                           cudaStream_t s) {
-  int n = rows * (K / 32);
-  k_dequant<<<(n + 255) / 256, 256, 0, s>>>(blob, lay, mat, rows, K, out);
   return cudaGetLastError();
 }
 

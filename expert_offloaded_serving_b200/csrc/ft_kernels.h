@@ -38,8 +38,6 @@ cudaError_t launch_permute(const int32_t* ids, int P, int E, int32_t* offs, int3
 bool gemv_shape_ok(int H, int I);
 cudaError_t launch_gate_up(const GemvParams& p, cudaStream_t s);
 cudaError_t launch_down_combine(const GemvParams& p, cudaStream_t s);
-cudaError_t launch_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int rows, int K, float* out,
-                           cudaStream_t s);
 cudaError_t launch_quantize_rows(const float* x, int64_t R, int K, uint8_t* codes, uint8_t* scales, cudaStream_t s);
 
 }  // namespace ft

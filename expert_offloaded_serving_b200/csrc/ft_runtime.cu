@@ -177,6 +177,7 @@ struct ft_ctx {
   int sync_stride = 0;
   int* d_flag = nullptr;       // a device flag nothing sets (failure injection)
   uint64_t* d_h_tagged = nullptr;  // persistent kernel, T <= 2: tagged h [T*k + S*T][I]
+  int64_t tagged_words = 0;
   uint32_t* d_epoch = nullptr;     // launch counter for those tags
 
   // failure injection
@@ -398,6 +399,7 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
     if ((st = dev_alloc(&c->d_sync, (size_t)L * c->sync_stride)) || (st = dev_alloc(&c->d_h_tagged, hrows * I)) ||
         (st = dev_alloc(&c->d_epoch, 1)))
       return bail(st);
+    c->tagged_words = (int64_t)(hrows * I);
     if (cudaMemset(c->d_h_tagged, 0, hrows * I * sizeof(uint64_t)) != cudaSuccess ||
         cudaMemset(c->d_epoch, 0, sizeof(uint32_t)) != cudaSuccess)
       return bail(fail(FT_ERR_CUDA, "memset"));
@@ -621,9 +623,9 @@ extern "C" ft_status ft_quantize_mxfp4(ft_ctx* c, const float* x, int64_t R, int
 
 extern "C" ft_status ft_debug_dequant(ft_ctx* c, const void* blob, int32_t mat, float* out, void* stream) {
   if (!c || !blob || !out || mat < 0 || mat > 2) return fail(FT_ERR_INVALID, "bad argument");
-  int rows = mat < 2 ? c->d.inter : c->d.hidden;
-  int K = mat < 2 ? c->d.hidden : c->d.inter;
-  CUDA_TRY(launch_dequant((const uint8_t*)blob, c->lay, mat, rows, K, out, (cudaStream_t)stream));
+  if (!decode_supported(c->d.hidden, c->d.inter))
+    return fail(FT_ERR_INVALID, "the decode tile does not take hidden %d / inter %d", c->d.hidden, c->d.inter);
+  CUDA_TRY(launch_dec_dequant((const uint8_t*)blob, c->lay, mat, c->d.hidden, c->d.inter, out, (cudaStream_t)stream));
   return FT_OK;
 }
 
@@ -643,6 +645,21 @@ extern "C" ft_status ft_debug_device_wait(ft_ctx* c, int64_t timeout_us, void* s
   if (timeout_us < 1 || timeout_us > 2000000) return fail(FT_ERR_INVALID, "timeout_us %lld outside [1, 2e6]", (long long)timeout_us);
   CUDA_TRY(launch_debug_wait(c->d_flag, c->d_status, (uint64_t)timeout_us * 1000u, (cudaStream_t)stream));
   c->last_stream = (cudaStream_t)stream;
+  return FT_OK;
+}
+
+extern "C" ft_status ft_debug_stack_epoch(ft_ctx* c, uint32_t epoch, int32_t poison_layer) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (!c->d_epoch) return fail(FT_ERR_STATE, "this context has no persistent decode kernel");
+  if (poison_layer > 127) return fail(FT_ERR_INVALID, "poison_layer %d above 127", poison_layer);
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(c->d_epoch, &epoch, sizeof(epoch), cudaMemcpyHostToDevice));
+  if (poison_layer >= 0) {
+    const uint32_t tag = (next_epoch(epoch, nullptr) << 7) | (uint32_t)poison_layer;
+    const uint64_t word = ((uint64_t)tag << 32) | 0x7fc00000ull;  // a NaN under the next launch's tag
+    std::vector<uint64_t> w((size_t)c->tagged_words, word);
+    CUDA_TRY(cudaMemcpy(c->d_h_tagged, w.data(), w.size() * sizeof(uint64_t), cudaMemcpyHostToDevice));
+  }
   return FT_OK;
 }
 
@@ -1250,7 +1267,11 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     if (persistent) {
       ra.sync = c->d_sync;
       ra.sync_stride = c->sync_stride;
-      if (fused) ra.epoch = c->d_epoch;
+      if (fused) {
+        ra.epoch = c->d_epoch;
+        ra.tagged = c->d_h_tagged;
+        ra.tagged_words = c->tagged_words;
+      }
     }
     CUDA_TRY(launch_route(ra, s));
   }

@@ -297,8 +297,12 @@ FT_API ft_status ft_prefetch_layer(ft_ctx* ctx, int32_t layer, void* compute_str
 /* ---------------------------------------------------------------------- */
 
 /* Dequantise matrix `mat` (0 = Wg, 1 = Wu, 2 = Wd) of a blob at dev pointer
- * `blob` to fp32 out dev [rows][K] (exact).  Decodes with the same device
- * routine the GEMV uses. */
+ * `blob` to fp32 out dev [rows][K]: code value x UE8M0 scale, exact in fp32
+ * unless the product overflows (then +-inf) ([no] "MXFP4": e2m1 values with
+ * per-32 power-of-two scales).  The rows pass through the decode kernels' own
+ * tile: staged into shared memory as the decode GEMVs stage them, read back
+ * chunk by chunk and converted by the same e2m1 -> f16 decoder their dot
+ * products use.  FT_ERR_INVALID for a shape the decode kernels do not take. */
 FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, float* out, void* stream);
 
 /* Tile geometry the decode kernels use for hidden H and intermediate I
@@ -334,6 +338,18 @@ FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_lay
  * in the same step stay resident, and a retry of the step fetches the dropped
  * key. */
 FT_API ft_status ft_debug_device_wait(ft_ctx* ctx, int64_t timeout_us, void* stream);
+
+/* Test hook for the persistent decode kernel's tagged hand-over words.  Each
+ * such word carries a 32-bit tag (launch counter << 7 | layer) that repeats
+ * every 2^25 launches; the routing kernel zeroes all tagged words when the
+ * counter wraps, so that a word left from 2^25 launches earlier cannot pass
+ * for one of the current launch.  This call waits for the device, sets the
+ * launch counter to `epoch` and, when poison_layer is in [0, 127], fills every
+ * tagged word with a NaN carrying the tag the next launch gives layer
+ * poison_layer (a stale word of exactly the kind the zeroing removes).
+ * Errors: FT_ERR_INVALID, FT_ERR_STATE (no persistent kernel in this
+ * context), FT_ERR_CUDA. */
+FT_API ft_status ft_debug_stack_epoch(ft_ctx* ctx, uint32_t epoch, int32_t poison_layer);
 FT_API ft_status ft_debug_host_wait_limit(ft_ctx* ctx, double seconds);
 FT_API ft_status ft_debug_fail_copy(ft_ctx* ctx, int64_t n);
 

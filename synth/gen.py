@@ -208,6 +208,42 @@ def expert_blob_nvfp4(seed: int, layer: int, expert: int, hidden: int, inter: in
 
 
 # ---------------------------------------------------------------------------
+# wide-range MXFP4 blobs (parity tests of the extremes of the format)
+# ---------------------------------------------------------------------------
+# The matrices named in ``wide`` get codes uniform over all 16 e2m1 codes and
+# UE8M0 scale bytes uniform over 0 .. 254 (every finite scale, 2^-127 ..
+# 2^127); the other matrices keep the usual code histogram with their scale
+# bytes moved from SCALE_BASE +- 1 to ``narrow_base`` +- 1.  Pure byte draws
+# from the same counter-based generator (stream region REGION_WIDE).
+REGION_WIDE = 4
+
+
+def expert_blob_wide(seed: int, layer: int, expert: int, hidden: int, inter: int,
+                     wide=("wg", "wu"), narrow_base: int = SCALE_BASE) -> np.ndarray:
+    r = blob_regions(hidden, inter)
+    blob = expert_blob(seed, layer, expert, hidden, inter)
+    code_rng = {"wg": (r["wg"], r["wu"]), "wu": (r["wu"], r["wd"]), "wd": (r["wd"], r["codes_end"])}
+    sc_rng = {"wg": (r["wg_sf"], r["wu_sf"]), "wu": (r["wu_sf"], r["wd_sf"]), "wd": (r["wd_sf"], r["used"])}
+    shift = int(narrow_base) - SCALE_BASE
+    for name in ("wg", "wu", "wd"):
+        a, b = sc_rng[name]
+        if name not in wide and shift:
+            blob[a:b] = (blob[a:b].astype(np.int64) + shift).astype(np.uint8)
+    n_draw = 0
+    for name in wide:
+        for a, b in (code_rng[name], sc_rng[name]):
+            n = b - a
+            w = words(seed, blob_stream(layer, expert, REGION_WIDE), n_draw, (n + 3) // 4)
+            n_draw += (n + 3) // 4
+            f = np.stack([(w >> np.uint64(16 * q)) & np.uint64(0xFFFF) for q in range(4)], axis=1).reshape(-1)[:n]
+            if (a, b) == code_rng[name]:
+                blob[a:b] = (f & np.uint64(0xFF)).astype(np.uint8)       # two uniform 4-bit codes
+            else:
+                blob[a:b] = (f % np.uint64(255)).astype(np.uint8)        # 0 .. 254
+    return blob
+
+
+# ---------------------------------------------------------------------------
 # activations, router weights, traces, logits
 # ---------------------------------------------------------------------------
 

@@ -31,6 +31,23 @@ def assert_close(got_bits: np.ndarray, want: np.ndarray):
     return err.max(), rel
 
 
+def assert_close_scaled(got_bits: np.ndarray, want: np.ndarray):
+    """The layer tolerance on outputs divided by their largest magnitude, for
+    inputs whose outputs span many binades (wide-range block scales): max
+    |got - want| <= MAX_ABS * max |want| and relative L2 <= REL_L2.  Every
+    output must be finite."""
+    g = bits_to_f64(got_bits)
+    want = np.asarray(want, np.float64)
+    assert np.isfinite(g).all() and np.isfinite(want).all()
+    scale = np.abs(want).max()
+    assert scale > 0
+    err = np.abs(g - want) / scale
+    rel = np.linalg.norm(g - want) / np.linalg.norm(want)
+    assert err.max() <= MAX_ABS, f"max abs / max |want| {err.max():.3e}"
+    assert rel <= REL_L2, f"rel L2 {rel:.3e}"
+    return err.max(), rel
+
+
 class Ctx:
     def __init__(self, desc, host_layers=None, resident_layers=None):
         self.desc = desc

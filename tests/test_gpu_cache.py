@@ -124,3 +124,57 @@ def test_cache_nonfinite_logit_is_reported():
         ft.ft_sync_status(c.h)
     finally:
         c.close()
+
+
+def test_cache_trace_dsv4_shape_matches_oracle():
+    """The DeepSeek-V4-Flash-class cache path (hidden 4096, 256 experts top-6,
+    intermediate 2048; 13.4 MB blobs from pinned host pools) on 4 layers with
+    the 32 GiB budget scaled to 4 of the 43 layers (239 slots), 48 tokens of a
+    Zipf(1.0) / 0.5-overlap trace, the budget halved at token 16 and restored
+    at token 32: every step's HIT/MISS/EVICT/MOVE sequence equals the oracle
+    LRU's, and every output equals the resident path's bit for bit."""
+    H3, I3, E3, k3, L3, seed, n_tok = 4096, 2048, 256, 6, 4, 1003, 48
+    stride = synth.blob_stride(H3, I3)
+    slots = int(32 * 2 ** 30 * L3 / 43) // stride
+    hp, dp = [], []
+    for layer in range(L3):
+        d = synth.gpu.layer_pool(H3, I3, E3, seed, layer)
+        h = torch.empty(d.numel(), dtype=torch.uint8).pin_memory()
+        h.copy_(d)
+        hp.append(h)
+        dp.append(d)
+    torch.cuda.synchronize()
+    sets = np.stack([synth.zipf_trace(seed, layer, n_tok, E3, k3, 1.0, 0.5) for layer in range(L3)], axis=1)
+    xb = synth.activations_bf16(seed, 1, 1, H3)
+    cache = Ctx(ft.make_desc(H3, I3, E3, k3, L3, 0, slots * stride, 1), hp, None)
+    res = Ctx(ft.make_desc(H3, I3, E3, k3, L3, 0, 0, 1), None, dp)
+    ref = olru.LRUCache(slots)
+    n_miss = 0
+    try:
+        x = x_dev(xb)
+        for p in range(n_tok):
+            if p == n_tok // 3:
+                ft.ft_expert_cache_resize(cache.h, (slots // 2) * stride)
+                assert oracle_events(ft.ft_cache_trace(cache.h, cap=1 << 16)) == ref.resize(slots // 2)
+            if p == 2 * n_tok // 3:
+                ft.ft_expert_cache_resize(cache.h, slots * stride)
+                assert ft.ft_cache_trace(cache.h) == []
+                ref.resize(slots)
+            for layer in range(L3):
+                lg = synth.logits_for_sets(seed, p * 100 + layer, sets[p, layer][None], E3)
+                lgd = torch.from_numpy(lg).cuda()
+                o1, o2 = torch.empty_like(x), torch.empty_like(x)
+                ft.ft_moe_layer_forward(cache.h, layer, x, 1, None, lgd, o1, ft.FT_ROUTE_RENORM)
+                ft.ft_moe_layer_forward(res.h, layer, x, 1, None, lgd, o2, ft.FT_ROUTE_RENORM)
+                torch.cuda.synchronize()
+                assert (bf16_bits(o1) == bf16_bits(o2)).all(), (p, layer)
+                ids, _ = routing.topk(lg, k3)
+                want = ref.step(layer, ids.reshape(-1))
+                n_miss += sum(1 for e in want if e[0] == olru.MISS)
+                assert oracle_events(ft.ft_cache_trace(cache.h, cap=1 << 16)) == want, (p, layer)
+                x = o1
+        st = ft.ft_cache_stats_get(cache.h)
+        assert st["misses"] == n_miss and st["evictions"] > 0 and st["moves"] > 0
+    finally:
+        cache.close()
+        res.close()

@@ -133,3 +133,38 @@ def test_injected_copy_failure_drops_the_key_and_a_retry_recovers():
     finally:
         cache.close()
         res.close()
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_tagged_words_are_zeroed_when_the_launch_counter_wraps(T):
+    """The persistent kernel's tagged hand-over words carry a tag (launch
+    counter << 7 | layer) that repeats every 2^25 launches.  Stale words of a
+    launch 2^25 earlier would pass for the current launch's; the routing
+    kernel zeroes every tagged word when the counter wraps.  Here each tagged
+    word is overwritten with a NaN under the exact tag the wrapping launch uses
+    for a layer, and the launches across the wrap must still equal the
+    per-layer kernels bit for bit."""
+    H, I, E, k, L = 2048, 512, 64, 8, 2
+    pools = [synth.gpu.layer_pool(H, I, E + 1, SEED, layer) for layer in range(L)]
+    sets = [np.stack([synth.zipf_trace(SEED, layer, 3, E, k, 1.1, 0.6, stream=t)[-1] for t in range(T)])
+            for layer in range(L)]
+    lg = torch.from_numpy(np.stack([synth.logits_for_sets(SEED, layer, sets[layer], E) for layer in range(L)])).cuda()
+    x = x_dev(synth.activations_bf16(SEED, 2, T, H))
+    with Ctx(ft.make_desc(H, I, E, k, L, 1, 0, 4), None, pools) as c:
+        want = torch.empty_like(x)
+        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, want, 1 | ft.FT_STACK_LAYERWISE)
+        ft.ft_sync_status(c.h)
+        want_b = bf16_bits(want)
+        for poison in range(L):
+            ft.ft_debug_stack_epoch(c.h, (1 << 25) - 1, poison)   # the next launch wraps
+            for rep in range(3):
+                got = torch.empty_like(x)
+                ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, got, 1)
+                ft.ft_sync_status(c.h)
+                assert (bf16_bits(got) == want_b).all(), (poison, rep)
+        ft.ft_debug_stack_epoch(c.h, (1 << 32) - 3)           # the 32-bit counter itself wraps too
+        for rep in range(4):
+            got = torch.empty_like(x)
+            ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, got, 1)
+            ft.ft_sync_status(c.h)
+            assert (bf16_bits(got) == want_b).all(), rep
