@@ -626,8 +626,9 @@ def main():
         warm, timed = min(args.warmup, 2), max(1, min(args.steps, 20))
         times, threads = oracle_layer_times(T, warm + timed, warm, float("inf"))
         v = statistics.median(T / (t * L) for t in times)
+        # a step is one oracle layer: ms_per_step x steps is the timed region
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * T / v,
+                "steps": len(times), "warmup": warm, "ms_per_step": 1e3 * statistics.mean(times),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": workload_config(T),
                 "cpu_baseline": {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",

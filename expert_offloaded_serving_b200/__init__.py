@@ -23,6 +23,7 @@ FT_ROUTE_RENORM = 1
 FT_ACT_BF16 = 0
 FT_ACT_MXFP4 = 2
 FT_STACK_LAYERWISE = 4
+FT_STACK_COUNTERS = 8
 FT_EV_HIT, FT_EV_MISS, FT_EV_EVICT, FT_EV_MOVE = range(4)
 
 EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft_destroy", "ft_sync_status",
@@ -31,7 +32,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
            "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry",
-           "ft_debug_stack_epoch")
+           "ft_debug_stack_epoch", "ft_flow_geometry")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -105,6 +106,7 @@ def lib() -> C.CDLL:
         "ft_debug_host_wait_limit": (ST, [P, C.c_double]),
         "ft_debug_fail_copy": (ST, [P, I64]),
         "ft_debug_stack_epoch": (ST, [P, U32, I32]),
+        "ft_flow_geometry": (ST, [I32, I32, I32, I32, I32, I32, I32, C.POINTER(I64)]),
         "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
     for name, (res, args) in sig.items():
@@ -267,6 +269,12 @@ def ft_debug_host_wait_limit(ctx, seconds: float) -> None:
 
 def ft_debug_fail_copy(ctx, n: int) -> None:
     _check(lib().ft_debug_fail_copy(ctx, n))
+
+
+def ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers) -> dict:
+    out = (I64 * 3)()
+    _check(lib().ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, out))
+    return {"ok": bool(out[0]), "rows_cap": out[1], "smem": out[2]}
 
 
 def ft_debug_stack_epoch(ctx, epoch: int, poison_layer: int = -1) -> None:

@@ -118,6 +118,32 @@ bool stack_supported(int H, int I, int n_layers);
 int stack_sync_stride(int H, int I);
 cudaError_t launch_dec_stack(const StackArgs& a, cudaStream_t s);
 
+// Dataflow decode over n_layers consecutive layers for one or two tokens
+// (ft_decode_flow.cu): one cooperative launch, one CTA per SM; h and the next
+// layer's x travel as tagged words, the down tiles span every unit and
+// combine their rows themselves.
+struct FlowArgs {
+  const uint16_t* x0;          // bf16 [T][H] input of the first layer
+  uint16_t* out;               // bf16 [T][H] output of the last layer
+  const Route* rec;            // [n_layers] routing records
+  const uint8_t* const* eptr;  // [n_layers][n_blobs] blob pointers
+  int n_layers, n_blobs;
+  int T, H, I, E, k, n_shared;
+  BlobLayout lay;
+  uint64_t* h_tagged;          // [T*k + n_shared*T][I] words: tag << 32 | fp32
+  uint64_t* x_tagged;          // [T][H/2] words: tag << 32 | two bf16
+  const uint32_t* epoch;       // advanced by the routing kernel before this launch
+  int rows_cap;                // down-tile rows over all units (flow_geometry)
+  int* status;
+};
+struct FlowGeom {
+  int rows_cap;
+  size_t smem;
+  bool ok;                     // the dataflow kernel takes this shape, batch and depth
+};
+FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers);
+cudaError_t launch_dec_flow(const FlowArgs& a, cudaStream_t s);
+
 // One CTA waiting, with the persistent kernel's bounded wait, for *flag >= 1;
 // sets the timeout bit of *status after limit_ns.
 cudaError_t launch_debug_wait(const int* flag, int* status, uint64_t limit_ns, cudaStream_t s);

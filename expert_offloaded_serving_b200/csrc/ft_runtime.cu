@@ -176,7 +176,9 @@ struct ft_ctx {
   int* d_sync = nullptr;       // persistent stack kernel counters [L][sync_stride]
   int sync_stride = 0;
   int* d_flag = nullptr;       // a device flag nothing sets (failure injection)
-  uint64_t* d_h_tagged = nullptr;  // persistent kernel, T <= 2: tagged h [T*k + S*T][I]
+  uint64_t* d_tagged = nullptr;    // persistent kernels, T <= 2: tagged h, then tagged x
+  uint64_t* d_h_tagged = nullptr;  // [T*k + S*T][I] words
+  uint64_t* d_x_tagged = nullptr;  // [T][H/2] words (dataflow kernel)
   int64_t tagged_words = 0;
   uint32_t* d_epoch = nullptr;     // launch counter for those tags
 
@@ -395,12 +397,15 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
     return bail(st);
   if (stack_supported(H, I, 1)) {
     c->sync_stride = stack_sync_stride(H, I);
-    const size_t hrows = (size_t)(std::min(c->decode_max_t, 2) * k + desc->n_shared * std::min(c->decode_max_t, 2));
-    if ((st = dev_alloc(&c->d_sync, (size_t)L * c->sync_stride)) || (st = dev_alloc(&c->d_h_tagged, hrows * I)) ||
-        (st = dev_alloc(&c->d_epoch, 1)))
+    const int t2 = std::min(c->decode_max_t, 2);
+    const size_t hrows = (size_t)(t2 * k + desc->n_shared * t2);
+    c->tagged_words = (int64_t)(hrows * I + (size_t)t2 * H / 2);
+    if ((st = dev_alloc(&c->d_sync, (size_t)L * c->sync_stride)) ||
+        (st = dev_alloc(&c->d_tagged, (size_t)c->tagged_words)) || (st = dev_alloc(&c->d_epoch, 1)))
       return bail(st);
-    c->tagged_words = (int64_t)(hrows * I);
-    if (cudaMemset(c->d_h_tagged, 0, hrows * I * sizeof(uint64_t)) != cudaSuccess ||
+    c->d_h_tagged = c->d_tagged;
+    c->d_x_tagged = c->d_tagged + hrows * I;
+    if (cudaMemset(c->d_tagged, 0, (size_t)c->tagged_words * sizeof(uint64_t)) != cudaSuccess ||
         cudaMemset(c->d_epoch, 0, sizeof(uint32_t)) != cudaSuccess)
       return bail(fail(FT_ERR_CUDA, "memset"));
   }
@@ -518,7 +523,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   cudaFree(c->d_xbuf[0]);
   cudaFree(c->d_xbuf[1]);
   cudaFree(c->d_sync);
-  cudaFree(c->d_h_tagged);
+  cudaFree(c->d_tagged);
   cudaFree(c->d_epoch);
   cudaFree(c->d_eptr_res);
   cudaFree(c->d_eptr_cache);
@@ -640,6 +645,19 @@ extern "C" ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n
   return FT_OK;
 }
 
+extern "C" ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
+                                      int32_t n_experts, int32_t n_layers, int64_t out[3]) {
+  if (!out) return fail(FT_ERR_INVALID, "out is NULL");
+  if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128 || top_k <= 0 || top_k > 16 || n_experts <= 0 ||
+      n_shared < 0 || n_shared > 1 || T <= 0 || n_layers <= 0)
+    return fail(FT_ERR_INVALID, "bad shape");
+  const FlowGeom fg = flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers);
+  out[0] = fg.ok ? 1 : 0;
+  out[1] = fg.rows_cap;
+  out[2] = (int64_t)fg.smem;
+  return FT_OK;
+}
+
 extern "C" ft_status ft_debug_device_wait(ft_ctx* c, int64_t timeout_us, void* stream) {
   if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
   if (timeout_us < 1 || timeout_us > 2000000) return fail(FT_ERR_INVALID, "timeout_us %lld outside [1, 2e6]", (long long)timeout_us);
@@ -658,7 +676,7 @@ extern "C" ft_status ft_debug_stack_epoch(ft_ctx* c, uint32_t epoch, int32_t poi
     const uint32_t tag = (next_epoch(epoch, nullptr) << 7) | (uint32_t)poison_layer;
     const uint64_t word = ((uint64_t)tag << 32) | 0x7fc00000ull;  // a NaN under the next launch's tag
     std::vector<uint64_t> w((size_t)c->tagged_words, word);
-    CUDA_TRY(cudaMemcpy(c->d_h_tagged, w.data(), w.size() * sizeof(uint64_t), cudaMemcpyHostToDevice));
+    CUDA_TRY(cudaMemcpy(c->d_tagged, w.data(), w.size() * sizeof(uint64_t), cudaMemcpyHostToDevice));
   }
   return FT_OK;
 }
@@ -1254,26 +1272,57 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   if (T == 0) return FT_OK;
   cudaStream_t s = (cudaStream_t)stream;
   const int Ti = (int)T;
-  const bool persistent =
-      !(flags & FT_STACK_LAYERWISE) && c->d_sync != nullptr && stack_supported(c->d.hidden, c->d.inter, n_layers);
-  // with one or two tokens the persistent kernel folds the combine into the
-  // next layer and hands h over tagged (the tag holds the layer in 7 bits)
+  const int H = c->d.hidden, I = c->d.inter;
+  const bool layerwise = (flags & FT_STACK_LAYERWISE) != 0;
+  // one or two tokens: the dataflow kernel (tagged h and x, down tiles over
+  // every unit); else, or with FT_STACK_COUNTERS, the counter-synchronised
+  // persistent kernel; else two kernels per layer
+  const FlowGeom fg = flow_geometry(H, I, Ti, c->d.top_k, c->d.n_shared, c->d.n_experts, n_layers);
+  const bool flow = !layerwise && !(flags & FT_STACK_COUNTERS) && c->d_tagged != nullptr && fg.ok;
+  const bool persistent = !layerwise && !flow && c->d_sync != nullptr && stack_supported(H, I, n_layers);
+  // with one or two tokens the counter-synchronised kernel folds the combine
+  // into the next layer and hands h over tagged (the tag holds the layer in 7 bits)
   const bool fused = persistent && Ti <= 2 && n_layers <= 128;
   // all layers' routing records in one launch (their logits are inputs); it
-  // also zeroes the persistent kernel's counters of those layers
+  // also zeroes the counter-synchronised kernel's counters of those layers
   {
     KTimer kt(c, FT_K_TOPK, s);
     RouteArgs ra = route_args(c, logits, Ti, n_layers, flags, c->d_routes + first_layer);
     if (persistent) {
       ra.sync = c->d_sync;
       ra.sync_stride = c->sync_stride;
-      if (fused) {
-        ra.epoch = c->d_epoch;
-        ra.tagged = c->d_h_tagged;
-        ra.tagged_words = c->tagged_words;
-      }
+    }
+    if (fused || flow) {
+      ra.epoch = c->d_epoch;
+      ra.tagged = c->d_tagged;
+      ra.tagged_words = c->tagged_words;
     }
     CUDA_TRY(launch_route(ra, s));
+  }
+  if (flow) {
+    FlowArgs a{};
+    a.x0 = (const uint16_t*)x;
+    a.out = (uint16_t*)out;
+    a.rec = c->d_routes + first_layer;
+    a.eptr = c->d_eptr_res + (size_t)first_layer * c->n_blobs;
+    a.n_layers = n_layers;
+    a.n_blobs = c->n_blobs;
+    a.T = Ti;
+    a.H = H;
+    a.I = I;
+    a.E = c->d.n_experts;
+    a.k = c->d.top_k;
+    a.n_shared = c->d.n_shared;
+    a.lay = c->lay;
+    a.h_tagged = c->d_h_tagged;
+    a.x_tagged = c->d_x_tagged;
+    a.epoch = c->d_epoch;
+    a.rows_cap = fg.rows_cap;
+    a.status = c->d_status;
+    KTimer kt(c, FT_K_DEC_STACK, s);
+    CUDA_TRY(launch_dec_flow(a, s));
+    c->last_stream = s;
+    return FT_OK;
   }
   if (persistent) {
     StackArgs a{};

@@ -82,7 +82,8 @@ typedef struct {
 #define FT_ROUTE_RENORM 1u    /* renormalise the k softmax weights to sum 1 (default on) */
 #define FT_ACT_BF16     0u    /* decode: bf16 activations, fp32 h, FP4 GEMV on CUDA cores */
 #define FT_ACT_MXFP4    2u    /* prefill: x and h quantised to MXFP4, tcgen05 grouped GEMM */
-#define FT_STACK_LAYERWISE 4u /* ft_moe_stack_forward: two kernels per layer, not the persistent kernel */
+#define FT_STACK_LAYERWISE 4u /* ft_moe_stack_forward: two kernels per layer, not a persistent kernel */
+#define FT_STACK_COUNTERS  8u /* ft_moe_stack_forward: the counter-synchronised persistent kernel, not the dataflow one */
 
 /* cache trace events */
 #define FT_EV_HIT   0
@@ -314,6 +315,14 @@ FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, fl
  * out[22] 1 if the persistent kernel takes a stack of n_layers layers of this
  * shape, out[23] its counter words per layer.  FT_ERR_INVALID on a bad shape. */
 FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_layers, int64_t out[24]);
+
+/* Geometry of the dataflow decode kernel that ft_moe_stack_forward runs for
+ * one or two tokens (host only, no device needed): out[0] = 1 if it takes
+ * this shape, batch T and stack depth (else the counter-synchronised or the
+ * per-layer kernels run), out[1] = rows of a down tile over all units,
+ * out[2] = shared memory of a CTA in bytes.  FT_ERR_INVALID on a bad shape. */
+FT_API ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
+                                  int32_t n_experts, int32_t n_layers, int64_t out[3]);
 
 /* Failure injection for tests: none of these fault or hang a GPU.
  *

@@ -61,3 +61,26 @@ def test_limits_are_refused():
     with pytest.raises(ft.FtError) as e:
         ft.ft_decode_geometry(2000, 512, 1)
     assert e.value.status == ft.FT_ERR_INVALID
+
+
+@pytest.mark.parametrize("shape", [(2048, 512, 256, 8, 1, 40), (4096, 2048, 256, 6, 0, 43), (6144, 2048, 256, 8, 0, 8),
+                                   (256, 128, 16, 2, 0, 4), (1024, 512, 64, 4, 0, 3), (1024, 768, 64, 4, 1, 3),
+                                   (256, 256, 16, 4, 1, 3)])
+@pytest.mark.parametrize("T", [1, 2])
+def test_dataflow_kernel_geometry(shape, T):
+    """The dataflow stack kernel takes the workload shapes at one and two
+    tokens: its CTA fits the opt-in shared memory, and a down tile has room
+    for two rows of every unit a layer can have (rb >= 2, even)."""
+    H, I, E, k, S, L = shape
+    g = ft.ft_flow_geometry(H, I, T, k, S, E, L)
+    assert g["ok"] and g["smem"] <= OPT_IN_SMEM
+    units = min(E, T * k) + S
+    assert g["rows_cap"] % 2 == 0 and g["rows_cap"] >= 2 * units
+
+
+def test_dataflow_kernel_limits():
+    """Three or more tokens, or more than 127 layers (the tag holds the layer
+    in 7 bits), go to the other kernels."""
+    assert not ft.ft_flow_geometry(2048, 512, 3, 8, 1, 256, 40)["ok"]
+    assert not ft.ft_flow_geometry(2048, 512, 1, 8, 1, 256, 128)["ok"]
+    assert ft.ft_flow_geometry(2048, 512, 1, 8, 1, 256, 127)["ok"]

@@ -134,6 +134,7 @@ def test_fused_routing_ties_and_no_renorm():
 
 STACK_SHAPES = {
     # name: H, I, E, k, S, seed
+    "tiny": (256, 128, 16, 2, 0, 1001),
     "35b": (2048, 512, 256, 8, 1, 1002),
     "no_shared": (1024, 512, 64, 4, 0, 1004),
     "narrow_down": (1024, 768, 64, 4, 1, 1005),   # down tile of 256 threads
@@ -151,10 +152,16 @@ def stack_case(name, T, L):
     return (H, I, E, k, S, seed), pools, lgs
 
 
-@pytest.mark.parametrize("name,T", [("35b", 1), ("35b", 4), ("35b", 16), ("no_shared", 1), ("no_shared", 16),
-                                    ("narrow_down", 3), ("dsv4", 2)])
-@pytest.mark.parametrize("flags", [1, 1 | ft.FT_STACK_LAYERWISE], ids=["persistent", "layerwise"])
+@pytest.mark.parametrize("name,T", [("tiny", 1), ("tiny", 2), ("35b", 1), ("35b", 2), ("35b", 4), ("35b", 16),
+                                    ("no_shared", 1), ("no_shared", 2), ("no_shared", 16), ("narrow_down", 1),
+                                    ("narrow_down", 2), ("narrow_down", 3), ("dsv4", 1), ("dsv4", 2)])
+@pytest.mark.parametrize("flags", [1, 1 | ft.FT_STACK_COUNTERS, 1 | ft.FT_STACK_LAYERWISE],
+                         ids=["default", "counters", "layerwise"])
 def test_stack_forward_matches_layer_by_layer(name, T, flags):
+    """Every stack mode equals the same layers run one ft_moe_layer_forward at
+    a time, bit for bit: the dataflow kernel (the default for one or two
+    tokens), the counter-synchronised persistent kernel, and two kernels per
+    layer."""
     L = 3
     (H, I, E, k, S, seed), pools, lgs = stack_case(name, T, L)
     lg_all = torch.from_numpy(np.stack(lgs)).cuda()
@@ -215,7 +222,8 @@ def test_stack_forward_repeated_and_sub_stacks():
         ft.ft_sync_status(c.h)
         torch.cuda.synchronize()
         assert (bf16_bits(a) == bf16_bits(b)).all()
-        ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, b, 1 | ft.FT_STACK_LAYERWISE)
-        ft.ft_sync_status(c.h)
-        torch.cuda.synchronize()
-        assert (bf16_bits(a) == bf16_bits(b)).all()
+        for other in (ft.FT_STACK_LAYERWISE, ft.FT_STACK_COUNTERS):
+            ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg_all, b, 1 | other)
+            ft.ft_sync_status(c.h)
+            torch.cuda.synchronize()
+            assert (bf16_bits(a) == bf16_bits(b)).all()

@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 H, I, E, K, S, L, SEED = 2048, 512, 256, 8, 1, 40, 1002
 
 
-@pytest.mark.parametrize("T", [1, 4])
+@pytest.mark.parametrize("T", [1, 2, 4])
 def test_35b_class_stack_at_full_size(T):
     pools = [synth.gpu.layer_pool(H, I, E + S, SEED, layer) for layer in range(L)]
     lgs = []
