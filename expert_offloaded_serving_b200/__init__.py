@@ -24,6 +24,7 @@ FT_ACT_BF16 = 0
 FT_ACT_MXFP4 = 2
 FT_STACK_LAYERWISE = 4
 FT_STACK_COUNTERS = 8
+FT_CACHE_SERIAL = 16
 FT_EV_HIT, FT_EV_MISS, FT_EV_EVICT, FT_EV_MOVE = range(4)
 
 EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft_destroy", "ft_sync_status",
@@ -57,7 +58,8 @@ class CacheEvent(C.Structure):
 
 class CacheStats(C.Structure):
     _fields_ = [("hits", C.c_int64), ("misses", C.c_int64), ("evictions", C.c_int64), ("moves", C.c_int64),
-                ("h2d_bytes", C.c_int64), ("h2d_ms", C.c_double), ("capacity_slots", C.c_int64),
+                ("h2d_bytes", C.c_int64), ("h2d_ms", C.c_double), ("hit_ms", C.c_double),
+                ("overlap_ms", C.c_double), ("capacity_slots", C.c_int64),
                 ("used_slots", C.c_int64), ("mapped_bytes", C.c_int64)]
 
 

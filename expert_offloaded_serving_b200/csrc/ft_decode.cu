@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
   uint8_t* base = smem + kTileOff;
   const Gv g = make_gv(a.H, a.I, 2);
   const int nrb = a.I / g.R;
-  const int rb = blockIdx.x % nrb, u = blockIdx.x / nrb;
+  const int rb = blockIdx.x % nrb, u = a.n_sel ? a.sel[blockIdx.x / nrb] : blockIdx.x / nrb;
   UnitInfo ui;
   if (!resolve_unit(a, a.rec, u, ui, hd.tok)) {
     pdl_trigger();
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
   uint8_t* base = smem + kTileOff;
   const Gv g = make_gv(a.I, a.H, 1);
   const int nrb = a.H / g.R;
-  const int rb = blockIdx.x % nrb, u = blockIdx.x / nrb;
+  const int rb = blockIdx.x % nrb, u = a.n_sel ? a.sel[blockIdx.x / nrb] : blockIdx.x / nrb;
   UnitInfo ui;
   if (!resolve_unit(a, a.rec, u, ui, hd.tok)) {
     pdl_trigger();
@@ -909,12 +909,14 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
 
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const Gv g = make_gv(a.H, a.I, 2);
-  return launch_one(k_dec_gate_up, a, g, a.I, (a.max_units + a.n_shared) * (a.I / g.R), pdl, s);
+  const int units = a.n_sel ? a.n_sel : a.max_units + a.n_shared;
+  return launch_one(k_dec_gate_up, a, g, a.I, units * (a.I / g.R), pdl, s);
 }
 
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
   const Gv g = make_gv(a.I, a.H, 1);
-  return launch_one(k_dec_down, a, g, a.H, (a.max_units + a.n_shared) * (a.H / g.R), pdl, s);
+  const int units = a.n_sel ? a.n_sel : a.max_units + a.n_shared;
+  return launch_one(k_dec_down, a, g, a.H, units * (a.H / g.R), pdl, s);
 }
 
 cudaError_t launch_dec_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int H, int I, float* out,

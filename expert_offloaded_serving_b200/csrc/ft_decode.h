@@ -66,6 +66,12 @@ struct DecodeArgs {
   uint16_t* out;           // bf16 [T][H]
   int* counters;           // [H/8] combine counters, zero before the first launch
   int* status;
+  // Units this launch takes: all (n_sel == 0), or the units sel[0 .. n_sel).
+  // The cache path runs the resident experts at once and each fetched expert
+  // after its own copy; the last down CTA of a row block, over all launches of
+  // the layer, does the combine.
+  int n_sel;
+  uint16_t sel[kMaxUnits];
 };
 
 // True when the decode kernels take this shape (hidden and inter multiples of

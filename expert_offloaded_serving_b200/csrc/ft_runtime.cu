@@ -209,8 +209,17 @@ struct ft_ctx {
   std::vector<ft_cache_event> trace;
   int64_t trace_dropped = 0;  // events not recorded because the trace was full
   ft_cache_stats stats{};
-  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> copy_timing;  // (start, end) of miss copies in flight
-  std::vector<cudaEvent_t> spare_events;                          // finished timing events, reused
+  // Timing of one cache step with misses: ref precedes everything of the step
+  // (recorded with the routed ids the host waited for), c0 / c1 bracket the
+  // step's copies on the copy stream, h0 / h1 the resident experts' kernels
+  // that run while the copies are in flight (NULL without such kernels).
+  struct StepTiming {
+    cudaEvent_t ref, c0, c1, h0, h1;
+  };
+  std::vector<StepTiming> copy_timing;   // steps whose events are still in flight
+  std::vector<cudaEvent_t> spare_events;  // finished timing events, reused
+  std::vector<cudaEvent_t> miss_events;   // one per miss copy of the current step (no timing)
+  std::vector<cudaEvent_t> spare_miss_events;
 
   // prefill staging
   uint8_t* d_stage[2] = {nullptr, nullptr};
@@ -499,11 +508,12 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
       cudaEventDestroy(m.second.first);
       cudaEventDestroy(m.second.second);
     }
-  for (auto& pr : c->copy_timing) {
-    cudaEventDestroy(pr.first);
-    cudaEventDestroy(pr.second);
-  }
+  for (auto& st : c->copy_timing)
+    for (cudaEvent_t e : {st.ref, st.c0, st.c1, st.h0, st.h1})
+      if (e) cudaEventDestroy(e);
   for (cudaEvent_t e : c->spare_events) cudaEventDestroy(e);
+  for (cudaEvent_t e : c->miss_events) cudaEventDestroy(e);
+  for (cudaEvent_t e : c->spare_miss_events) cudaEventDestroy(e);
   free_prefill_scratch(c->pf);
   cudaFree(c->d_status);
   cudaFree(c->d_flag);
@@ -738,12 +748,20 @@ static int32_t evict_one(ft_ctx* c, const std::vector<int64_t>& keep, int64_t* v
 static void fold_copy_timing(ft_ctx* c) {
   size_t n = 0;
   for (; n < c->copy_timing.size(); n++) {
-    const auto& pr = c->copy_timing[n];
-    if (cudaEventQuery(pr.second) != cudaSuccess) break;
-    float ms = 0.f;
-    if (cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess) c->stats.h2d_ms += ms;
-    c->spare_events.push_back(pr.first);
-    c->spare_events.push_back(pr.second);
+    const auto& st = c->copy_timing[n];
+    if (cudaEventQuery(st.c1) != cudaSuccess || (st.h1 && cudaEventQuery(st.h1) != cudaSuccess)) break;
+    float c0 = 0.f, c1 = 0.f;
+    if (cudaEventElapsedTime(&c0, st.ref, st.c0) == cudaSuccess && cudaEventElapsedTime(&c1, st.ref, st.c1) == cudaSuccess) {
+      c->stats.h2d_ms += c1 - c0;
+      float h0 = 0.f, h1 = 0.f;
+      if (st.h0 && cudaEventElapsedTime(&h0, st.ref, st.h0) == cudaSuccess &&
+          cudaEventElapsedTime(&h1, st.ref, st.h1) == cudaSuccess) {
+        c->stats.hit_ms += h1 - h0;
+        c->stats.overlap_ms += std::max(0.f, std::min(c1, h1) - std::max(c0, h0));
+      }
+    }
+    for (cudaEvent_t e : {st.ref, st.c0, st.c1, st.h0, st.h1})
+      if (e) c->spare_events.push_back(e);
   }
   c->copy_timing.erase(c->copy_timing.begin(), c->copy_timing.begin() + (std::ptrdiff_t)n);
 }
@@ -759,6 +777,19 @@ static cudaEvent_t copy_event(ft_ctx* c) {
   return e;
 }
 
+// An event (no timing) marking the end of one miss's copy on the copy stream.
+static cudaEvent_t miss_event(ft_ctx* c) {
+  cudaEvent_t e = nullptr;
+  if (!c->spare_miss_events.empty()) {
+    e = c->spare_miss_events.back();
+    c->spare_miss_events.pop_back();
+  } else {
+    cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+  }
+  c->miss_events.push_back(e);
+  return e;
+}
+
 // Issue the H2D copy of (layer, e) into `slot` on the copy stream.
 static ft_status fetch(ft_ctx* c, int layer, int e, int32_t slot) {
   if (c->fail_copy_in > 0 && --c->fail_copy_in == 0)
@@ -770,7 +801,11 @@ static ft_status fetch(ft_ctx* c, int layer, int e, int32_t slot) {
 }
 
 // One decode step of the cache for `layer` over the distinct experts S (ascending).
-static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, bool& any_miss, std::vector<int>& dirty) {
+// Misses are fetched in ascending expert id; for each, miss_units gets its
+// position in S and c->miss_events an event after its copy.  `ref` (a timing
+// event that precedes the step, or NULL) anchors the step's timing.
+static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, bool& any_miss, std::vector<int>& dirty,
+                            std::vector<int>* miss_units = nullptr, cudaEvent_t ref = nullptr) {
   any_miss = false;
   if ((int64_t)S.size() > c->lru.capacity)
     return fail(FT_ERR_NO_SPACE, "%zu experts in one step exceed the cache capacity of %lld slots", S.size(),
@@ -780,7 +815,8 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
   keep.reserve(S.size());
   for (int e : S) keep.push_back(key_of(c, layer, e));
   cudaEvent_t t0 = nullptr, t1 = nullptr;
-  for (int e : S) {
+  for (size_t si = 0; si < S.size(); si++) {
+    const int e = S[si];
     int64_t key = key_of(c, layer, e);
     auto m = c->lru.map.find(key);
     if (m != c->lru.map.end()) {
@@ -799,6 +835,10 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
       slot = c->lru.lowest_free();
     }
     if (!any_miss) {
+      if (!ref) {  // a step without a caller's anchor is anchored at its first copy
+        ref = copy_event(c);
+        cudaEventRecord(ref, c->copy_stream);
+      }
       t0 = copy_event(c);
       t1 = copy_event(c);
       cudaEventRecord(t0, c->copy_stream);
@@ -822,16 +862,22 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
       c->stats.evictions++;
       c->stats.used_slots = (int64_t)c->lru.map.size();
       cudaEventRecord(t1, c->copy_stream);
-      c->copy_timing.push_back({t0, t1});
+      c->copy_timing.push_back({ref, t0, t1, nullptr, nullptr});
       // a later step counts the earlier keys as hits and does not wait for
       // their copies: let them land now
       cudaStreamSynchronize(c->copy_stream);
       return fs;
     }
+    if (miss_units) {
+      miss_units->push_back((int)si);
+      cudaEventRecord(miss_event(c), c->copy_stream);
+    }
   }
   if (any_miss) {
     cudaEventRecord(t1, c->copy_stream);
-    c->copy_timing.push_back({t0, t1});
+    c->copy_timing.push_back({ref, t0, t1, nullptr, nullptr});
+  } else if (ref) {
+    c->spare_events.push_back(ref);
   }
   c->stats.used_slots = (int64_t)c->lru.map.size();
   return FT_OK;
@@ -889,7 +935,7 @@ extern "C" ft_status ft_expert_cache_insert(ft_ctx* c, int32_t layer, int32_t ex
   if (evicted_key && c->stats.evictions > before_evict) *evicted_key = victim;
   *slot = c->lru.map[key_of(c, layer, expert)].first;
   if (any_miss) {
-    cudaEvent_t done = c->copy_timing.back().second;
+    cudaEvent_t done = c->copy_timing.back().c1;
     CUDA_TRY(cudaStreamWaitEvent(s, done, 0));
   }
   FT_TRY(push_table_rows(c, dirty, s));
@@ -1107,6 +1153,8 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   // 4: weight source.  Prefill (MXFP4) reads resident or staged layers and
   // never touches the cache; decode reads resident layers or the cache.
   const uint8_t* const* eptr = nullptr;
+  std::vector<int> miss_units;  // cache path: units whose blobs are still being copied, in copy order
+  int n_routed_units = 0;
   const uint8_t* pool = nullptr;
   int stage_buf = -1;
   if (c->resident[layer]) {
@@ -1123,32 +1171,99 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     CUDA_TRY(cudaMemcpyAsync(c->h_ids, c->d_ids, (size_t)Ti * k * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaEventRecord(c->ev_ids, s));
-    FT_TRY(wait_event(c->ev_ids, "routing ids", c->host_wait_s));
+    // timing anchor of the step: everything below comes after it
+    cudaEvent_t ref = copy_event(c);
+    CUDA_TRY(cudaEventRecord(ref, s));
+    const ft_status ws = wait_event(c->ev_ids, "routing ids", c->host_wait_s);
+    if (ws != FT_OK) {
+      c->spare_events.push_back(ref);
+      return ws;
+    }
     if (*c->h_status) {
+      c->spare_events.push_back(ref);
       int st = *c->h_status;
       CUDA_TRY(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
       return status_to_ft(st);
     }
     std::vector<int> S(c->h_ids, c->h_ids + (size_t)Ti * k);
     for (int e : S)
-      if (e < 0 || e >= E) return fail(FT_ERR_INVALID, "expert id %d out of range", e);
+      if (e < 0 || e >= E) {
+        c->spare_events.push_back(ref);
+        return fail(FT_ERR_INVALID, "expert id %d out of range", e);
+      }
     std::sort(S.begin(), S.end());
     S.erase(std::unique(S.begin(), S.end()), S.end());
     std::vector<int> dirty{layer};
     bool any_miss = false;
     {
       NvtxRange step_range("cache_step");
-      FT_TRY(cache_step(c, layer, S, any_miss, dirty));
+      ft_status cs = cache_step(c, layer, S, any_miss, dirty, &miss_units, ref);
+      if (!any_miss && cs == FT_OK) ref = nullptr;  // returned to the pool by cache_step
+      if (cs != FT_OK) {
+        for (cudaEvent_t e : c->miss_events) c->spare_miss_events.push_back(e);
+        c->miss_events.clear();
+        return cs;
+      }
     }
-    if (any_miss) CUDA_TRY(cudaStreamWaitEvent(s, c->copy_timing.back().second, 0));
     FT_TRY(push_table_rows(c, dirty, s));
     eptr = c->d_eptr_cache + (size_t)layer * c->n_blobs;
+    if (any_miss && (flags & FT_CACHE_SERIAL)) {
+      // the serial order, for comparison: every copy lands before any expert runs
+      CUDA_TRY(cudaStreamWaitEvent(s, c->copy_timing.back().c1, 0));
+      miss_units.clear();
+    }
+    n_routed_units = (int)S.size();
   } else {
     return fail(FT_ERR_NOT_FOUND, "layer %d is neither resident nor cached", layer);
   }
 
   // 5: experts and combine
-  if (!mx) {
+  if (!mx && !miss_units.empty()) {
+    // cache path with misses: the resident experts (hits and the shared
+    // experts) run at once, while the misses' copies are in flight; each
+    // missed expert runs after its own copy ([no] experts fetched over PCIe;
+    // the copies overlap the compute of the experts already resident)
+    DecodeArgs a = decode_args(c, (const uint16_t*)x, rec, Ti, eptr, (uint16_t*)out);
+    std::vector<char> is_miss((size_t)n_routed_units, 0);
+    for (int u : miss_units) is_miss[u] = 1;
+    a.n_sel = 0;
+    for (int u = 0; u < n_routed_units; u++)
+      if (!is_miss[u]) a.sel[a.n_sel++] = (uint16_t)u;
+    for (int sx = 0; sx < c->d.n_shared; sx++) a.sel[a.n_sel++] = (uint16_t)(a.max_units + sx);
+    ft_ctx::StepTiming& stp = c->copy_timing.back();
+    if (a.n_sel > 0) {
+      stp.h0 = copy_event(c);
+      stp.h1 = copy_event(c);
+      CUDA_TRY(cudaEventRecord(stp.h0, s));
+      {
+        KTimer kt(c, FT_K_GATE_UP, s);
+        CUDA_TRY(launch_dec_gate_up(a, false, s));
+      }
+      {
+        KTimer kt(c, FT_K_DOWN_COMBINE, s);
+        CUDA_TRY(launch_dec_down(a, true, s));
+      }
+      CUDA_TRY(cudaEventRecord(stp.h1, s));
+    }
+    for (size_t mi = 0; mi < miss_units.size(); mi++) {
+      CUDA_TRY(cudaStreamWaitEvent(s, c->miss_events[mi], 0));
+      a.n_sel = 1;
+      a.sel[0] = (uint16_t)miss_units[mi];
+      {
+        KTimer kt(c, FT_K_GATE_UP, s);
+        CUDA_TRY(launch_dec_gate_up(a, false, s));
+      }
+      {
+        KTimer kt(c, FT_K_DOWN_COMBINE, s);
+        CUDA_TRY(launch_dec_down(a, true, s));
+      }
+    }
+    // the waits above hold the events' current records: they can be reused
+    for (cudaEvent_t e : c->miss_events) c->spare_miss_events.push_back(e);
+    c->miss_events.clear();
+  } else if (!mx) {
+    for (cudaEvent_t e : c->miss_events) c->spare_miss_events.push_back(e);
+    c->miss_events.clear();
     DecodeArgs a = decode_args(c, (const uint16_t*)x, rec, Ti, eptr, (uint16_t*)out);
     {
       KTimer kt(c, FT_K_GATE_UP, s);

@@ -84,6 +84,7 @@ typedef struct {
 #define FT_ACT_MXFP4    2u    /* prefill: x and h quantised to MXFP4, tcgen05 grouped GEMM */
 #define FT_STACK_LAYERWISE 4u /* ft_moe_stack_forward: two kernels per layer, not a persistent kernel */
 #define FT_STACK_COUNTERS  8u /* ft_moe_stack_forward: the counter-synchronised persistent kernel, not the dataflow one */
+#define FT_CACHE_SERIAL   16u /* cache path: every miss copy lands before any expert runs (for comparison) */
 
 /* cache trace events */
 #define FT_EV_HIT   0
@@ -102,6 +103,8 @@ typedef struct {
   int64_t hits, misses, evictions, moves;
   int64_t h2d_bytes;          /* bytes fetched from the host pool by misses */
   double  h2d_ms;             /* copy-stream time of those fetches (CUDA events) */
+  double  hit_ms;             /* time of the resident experts' kernels of steps with misses */
+  double  overlap_ms;         /* part of hit_ms that ran while that step's copies were in flight */
   int64_t capacity_slots, used_slots;
   int64_t mapped_bytes;       /* physical memory mapped under the slot arena */
 } ft_cache_stats;

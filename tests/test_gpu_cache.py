@@ -32,7 +32,13 @@ def oracle_events(ev):
     return [tuple(int(v) for v in e) for e in ev]
 
 
-def test_cache_trace_matches_oracle_and_resident_outputs():
+@pytest.mark.parametrize("serial", [False, True], ids=["overlapped", "serial"])
+def test_cache_trace_matches_oracle_and_resident_outputs(serial):
+    """The cache path against the oracle LRU (every event) and the resident
+    path (every output bit).  By default the resident experts run while the
+    misses' copies are in flight and each missed expert after its own copy;
+    FT_CACHE_SERIAL waits for every copy first.  Both give the same bits."""
+    flags = 1 | (ft.FT_CACHE_SERIAL if serial else 0)
     stride = synth.blob_stride(H, I)
     hp = host_pools(E)
     dp = [p.cuda() for p in hp]
@@ -61,7 +67,7 @@ def test_cache_trace_matches_oracle_and_resident_outputs():
             lgd = torch.from_numpy(lg).cuda()
             o1 = torch.empty_like(x)
             o2 = torch.empty_like(x)
-            ft.ft_moe_layer_forward(cache.h, layer, x, T, None, lgd, o1, 1)
+            ft.ft_moe_layer_forward(cache.h, layer, x, T, None, lgd, o1, flags)
             ft.ft_moe_layer_forward(res.h, layer, x, T, None, lgd, o2, 1)
             torch.cuda.synchronize()
             assert (bf16_bits(o1) == bf16_bits(o2)).all(), step
@@ -71,6 +77,9 @@ def test_cache_trace_matches_oracle_and_resident_outputs():
         st = ft.ft_cache_stats_get(cache.h)
         assert st["misses"] > 0 and st["hits"] > 0
         assert st["h2d_bytes"] == st["misses"] * ft.ft_blob_layout(H, I)["used"]
+        assert st["h2d_ms"] > 0 and 0 <= st["overlap_ms"] <= st["hit_ms"] + 1e-3
+        if serial:
+            assert st["hit_ms"] == 0
     finally:
         cache.close()
         res.close()
@@ -175,6 +184,8 @@ def test_cache_trace_dsv4_shape_matches_oracle():
                 x = o1
         st = ft.ft_cache_stats_get(cache.h)
         assert st["misses"] == n_miss and st["evictions"] > 0 and st["moves"] > 0
+        # steps with misses ran their resident experts during the copies
+        assert st["hit_ms"] > 0 and 0 < st["overlap_ms"] <= st["hit_ms"] + 1e-3
     finally:
         cache.close()
         res.close()
