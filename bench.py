@@ -44,7 +44,9 @@ def parse():
                     help="decode: the 35B-class decode stack (default line); prefill / miss: only that measurement")
     ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     ap.add_argument("--layerwise", action="store_true",
-                    help="decode with two kernels per layer instead of the persistent stack kernel")
+                    help="decode with two kernels per layer instead of a persistent stack kernel")
+    ap.add_argument("--counters", action="store_true",
+                    help="decode with the counter-synchronised persistent kernel instead of the dataflow kernel")
     return ap.parse_args()
 
 
@@ -217,7 +219,8 @@ def run_ours(args, world, rank):
     stream = torch.cuda.Stream()
     out_buf = torch.empty_like(x0)
 
-    flags = ft.FT_ROUTE_RENORM | (ft.FT_STACK_LAYERWISE if args.layerwise else 0)
+    flags = ft.FT_ROUTE_RENORM | (ft.FT_STACK_LAYERWISE if args.layerwise else 0) | \
+        (ft.FT_STACK_COUNTERS if getattr(args, "counters", False) else 0)
 
     def one_pass(src):
         ft.ft_moe_stack_forward(ctx, 0, L, src, T, logits_buf, out_buf, flags, stream.cuda_stream)
@@ -594,8 +597,16 @@ def measure_decode_batch(args, T, pk):
     return out
 
 
-def workload_config(T, layerwise=False):
-    return {"decode_kernels": "two per layer" if layerwise else "persistent stack kernel",
+def decode_kernel_name(T, layerwise=False, counters=False):
+    if layerwise:
+        return "two per layer"
+    if counters or T > 2:
+        return "persistent stack kernel, counter-synchronised"
+    return "persistent stack kernel, dataflow (tagged hand-overs)"
+
+
+def workload_config(T, layerwise=False, counters=False):
+    return {"decode_kernels": decode_kernel_name(T, layerwise, counters),
             "workload": f"35B-A3B-class MoE decode stack: hidden {H}, {E} routed experts top-{K_TOP} + {S_SHARED} shared, "
                         f"intermediate {I}, {L} layers, MXFP4 (e2m1 + UE8M0/32) weights resident in HBM, "
                         f"batch {T}, Zipf(1.1) routing traces with 0.6 adjacent-token reuse",
@@ -656,7 +667,7 @@ def main():
     line = {"metric": METRIC, "value": res["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(T, args.layerwise),
+            "config": workload_config(T, args.layerwise, args.counters),
             "roofline": {"bound": "hbm", "kernel": rk, "achieved": rk_gbs, "peak": pk["hbm"],
                          "peak_source": pk["src"], "unit": "GB/s", "frac": rk_gbs / pk["hbm"], "traffic": rk_traffic,
                          "algorithmic_bytes_per_launch": rk_bytes},
