@@ -322,43 +322,51 @@ def run_ours(args, world, rank):
 # ---------------------------------------------------------------------------
 # oracle timing (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_layer_times(T, max_layers, warm, budget_s):
-    """Time the oracle on one token position of the 40-layer stack, one layer
-    at a time (layers 0, 1, ...): `warm` untimed layers, then timed layers
-    until `max_layers` layers or `budget_s` seconds of timed oracle work.  The
-    synthetic inputs of a layer (its selected experts' blobs, logits) are
-    generated before its timed region.  Returns (seconds per timed layer,
-    threads the oracle's BLAS uses)."""
+def oracle_layer_times(T, n_layers, warm, budget_s, threads, distinct=4):
+    """Time the C++ oracle (oracle/ft_oracle.cpp) on one token position of the
+    40-layer stack, one layer per step, on `threads` OpenMP threads: the
+    synthetic inputs (selected experts' blobs, logits) of `distinct` layers are
+    generated first, outside any timed region; then `warm` untimed layers and
+    up to `n_layers` timed layers cycle through them, stopping early once
+    `budget_s` seconds of timed oracle work are done.  Returns (seconds per
+    timed layer, threads used)."""
     import numpy as np
     import synth
-    from oracle import layer as olayer
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
+    from oracle import cpp
     xb = synth.activations_bf16(SEED, 7, T, H)
-    times = []
-    for layer in range(max_layers):
+    inputs = []
+    for layer in range(distinct):
         sets = np.stack([synth.zipf_trace(SEED, layer, 4, E, K_TOP, 1.1, 0.6, stream=t)[-1] for t in range(T)])
         lg = synth.logits_for_sets(SEED, layer, sets, E)
         blobs = {int(e): synth.expert_blob(SEED, layer, int(e), H, I) for e in np.unique(sets)}
         blobs[E] = synth.expert_blob(SEED, layer, E, H, I)
+        inputs.append((lg, blobs))
+    times = []
+    for i in range(warm + n_layers):
+        lg, blobs = inputs[i % distinct]
         t0 = time.perf_counter()
-        olayer.moe_layer(xb, blobs.__getitem__, H, I, E, K_TOP, logits=lg, shared_blob=blobs[E])
+        cpp.moe_layer(xb, blobs.__getitem__, H, I, E, K_TOP, logits=lg, shared_blob=blobs[E], threads=threads)
         dt = time.perf_counter() - t0
-        if layer >= warm:
+        if i >= warm:
             times.append(dt)
             if sum(times) > budget_s:
                 break
     return times, threads
 
 
-def oracle_tok_s(T, budget_s=12.0, max_layers=12):
-    """CPU baseline: tok/s of the oracle over the 40-layer stack, from the mean
-    of its timed layers (one warm-up layer); returns (tok/s, layers, threads)."""
-    times, threads = oracle_layer_times(T, max_layers + 1, 1, budget_s)
-    return T / (statistics.mean(times) * L), len(times), threads
+def oracle_tok_s(T, threads, budget_s=8.0, max_layers=12):
+    """CPU baseline: tok/s of the C++ oracle over the 40-layer stack, from the
+    mean of its timed layers (one warm-up layer); returns (tok/s, layers)."""
+    times, _ = oracle_layer_times(T, max_layers, 1, budget_s, threads)
+    return T / (statistics.mean(times) * L), len(times)
+
+
+def host_cores():
+    """Cores this process may run on (the OpenMP threads the oracle is given)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 # ---------------------------------------------------------------------------
@@ -632,20 +640,21 @@ def main():
             print(json.dumps({"case": args.case, **r}))
         return
     if args.impl == "reference":
-        # one step = one oracle layer of the stack; at most 2 warm-up and 20
-        # timed layers, so that any --steps / --warmup ends within minutes
-        warm, timed = min(args.warmup, 2), max(1, min(args.steps, 20))
-        times, threads = oracle_layer_times(T, warm + timed, warm, float("inf"))
-        v = statistics.median(T / (t * L) for t in times)
-        # a step is one oracle layer: ms_per_step x steps is the timed region
+        # one step = one layer of the stack through the C++ oracle on every
+        # host core: W warm-up and exactly K timed steps (about 0.1 s each on
+        # 16 cores), so ms_per_step x steps is the timed region
+        threads = host_cores()
+        times, _ = oracle_layer_times(T, args.steps, args.warmup, float("inf"), threads)
+        v = T * len(times) / (sum(times) * L)
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1,
-                "steps": len(times), "warmup": warm, "ms_per_step": 1e3 * statistics.mean(times),
+                "steps": len(times), "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": workload_config(T),
                 "cpu_baseline": {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",
-                                 "sample": f"{len(times)} timed layers (after {warm} warm-up) of one token through "
-                                           f"the {L}-layer stack, each a step, median extrapolated to {L} layers; "
-                                           f"inputs generated outside the timed region"},
+                                 "sample": f"{len(times)} timed layers (after {args.warmup} warm-up) of one token "
+                                           f"through the {L}-layer stack, one layer a step, cycling over the "
+                                           f"inputs of 4 layers, mean extrapolated to {L} layers; C++ oracle on "
+                                           f"{threads} OpenMP threads; inputs generated outside the timed region"},
                 "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
@@ -692,11 +701,14 @@ def main():
             except Exception as ex:
                 line["decode_batch4"] = {"error": repr(ex)}
     if world == 1:
-        v, done, threads = oracle_tok_s(T)
-        line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": threads, "kind": "oracle",
-                                "sample": f"1 token through {done} layers of the {L}-layer stack (after one warm-up "
-                                          f"layer), mean extrapolated to {L}; inputs generated outside the timed "
-                                          f"region"}
+        cores = host_cores()
+        v, done = oracle_tok_s(T, cores)
+        v1, done1 = oracle_tok_s(T, 1)
+        line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                                "sample": f"C++ oracle on {cores} OpenMP threads: 1 token through {done} layers of the "
+                                          f"{L}-layer stack (after one warm-up layer), mean extrapolated to {L}; "
+                                          f"inputs generated outside the timed region",
+                                "single_thread": {"value": v1, "unit": "tok/s", "cores": 1, "layers": done1}}
     print(json.dumps(line))
 
 

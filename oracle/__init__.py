@@ -15,6 +15,10 @@ Plain, slow and fp64 throughout, written from the public write-ups of FreeToken
                MXFP4-activation mode).
 * ``lru``      the global LRU expert cache across layers, with resize.
 * ``formats``  BF16 and NVFP4 expert blobs (decode only), decoded to fp64.
+* ``cpp``      the same functions from ``ft_oracle.cpp``, a plain C++17
+               restatement (built by ``oracle/build.py`` into liboracle.so,
+               OpenMP over the experts of a layer for the timed CPU baseline).
+               The numpy modules are its cross-check (tests/test_oracle_cpp.py).
 
 Pins (tests/test_oracle_*.py, all CPU): exhaustive code x scale tables against
 the closed form, hand-computed scale-atom offsets, quantiser ties and
@@ -29,3 +33,4 @@ recency rules); each makes at least one of those pins fail.
 No function here is "parity unpinned".
 """
 from . import fp4, formats, routing, layer, lru  # noqa: F401
+# ``oracle.cpp`` is imported on use: it compiles liboracle.so on first load

@@ -30,7 +30,8 @@ def line(monkeypatch, capsys):
     monkeypatch.setattr(bench, "run_ours", fake_decode)
     monkeypatch.setattr(bench, "measure_prefill", lambda: {"workload": "prefill"})
     monkeypatch.setattr(bench, "measure_misses", lambda: {"workload": "miss"})
-    monkeypatch.setattr(bench, "oracle_tok_s", lambda T: (0.22, 12, 16))
+    monkeypatch.setattr(bench, "oracle_tok_s", lambda T, threads: (0.22 if threads > 1 else 0.05, 12))
+    monkeypatch.setattr(bench, "host_cores", lambda: 16)
     monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "10", "--warmup", "3"])
     bench.main()
     out = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
@@ -65,6 +66,7 @@ def test_derived_figures(line):
     assert line["value"] == pytest.approx(1e3 / 0.3238)
     assert line["gpu_launches"] == 20
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 16
+    assert line["cpu_baseline"]["value"] == 0.22 and line["cpu_baseline"]["single_thread"]["value"] == 0.05
 
 
 def test_layerwise_line_reports_the_gate_up_kernel(monkeypatch, capsys):
@@ -80,7 +82,7 @@ def test_layerwise_line_reports_the_gate_up_kernel(monkeypatch, capsys):
     monkeypatch.setattr(bench, "dist_setup", lambda args: (1, 0, 0))
     monkeypatch.setattr(bench, "run_ours", fake)
     monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "4", "--warmup", "3", "--layerwise", "--no-extra"])
-    monkeypatch.setattr(bench, "oracle_tok_s", lambda T: (0.22, 12, 16))
+    monkeypatch.setattr(bench, "oracle_tok_s", lambda T, threads: (0.22 if threads > 1 else 0.05, 12))
     bench.main()
     line = json.loads([ln for ln in capsys.readouterr().out.splitlines() if ln.strip()][0])
     r = line["roofline"]

@@ -27,7 +27,7 @@ def test_reference_line_has_the_contract_keys():
     assert d["impl"] == "reference" and d["unit"] == "tok/s" and d["higher_is_better"] is True
     assert d["steps"] == 2 and d["warmup"] == 1 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
-    assert "2 timed layers" in d["cpu_baseline"]["sample"]
+    assert "2 timed layers" in d["cpu_baseline"]["sample"] and "C++ oracle" in d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert "workload" in d["config"]
     # a step is one layer of the stack: the per-layer time, and tok/s extrapolates it to 40 layers
