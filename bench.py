@@ -373,7 +373,7 @@ def host_cores():
 # secondary measurements: prefill FP4 GEMM throughput with double-buffered
 # prefetch, expert-cache miss fetch bandwidth
 # ---------------------------------------------------------------------------
-FP4_DENSE_TFLOPS_NOMINAL = 9000.0   # B200 dense FP4 tensor peak, spec figure (not measured on this machine)
+FP4_DENSE_TFLOPS_NOMINAL = 9000.0   # B200 dense FP4 tensor peak, spec figure (quoted beside the measured one)
 EV_HIT, EV_MISS = 0, 1               # cache event kinds of the C ABI
 
 
@@ -393,14 +393,44 @@ def miss_phases(events, per_token, phases):
     return out
 
 
-def prefill_roofline(flops, weight_bytes, hbm_gbs, tflops):
+def prefill_roofline(flops, weight_bytes, hbm_gbs, tflops, fp4_peak=FP4_DENSE_TFLOPS_NOMINAL):
     """The prefill GEMM against its own roofline: min(FP4 dense peak, HBM
     bandwidth x arithmetic intensity over the weight bytes it must read)."""
     ai = flops / weight_bytes
-    roof = min(FP4_DENSE_TFLOPS_NOMINAL, hbm_gbs * ai / 1e3)
+    roof = min(fp4_peak, hbm_gbs * ai / 1e3)
     return {"flop_per_weight_byte": ai, "roofline_tflops": roof, "frac_of_roofline": tflops / roof,
-            "frac_of_fp4_nominal": tflops / FP4_DENSE_TFLOPS_NOMINAL,
-            "bound": "hbm" if roof < FP4_DENSE_TFLOPS_NOMINAL else "tensor"}
+            "frac_of_fp4_peak": tflops / fp4_peak, "frac_of_fp4_nominal": tflops / FP4_DENSE_TFLOPS_NOMINAL,
+            "bound": "hbm" if roof < fp4_peak else "tensor"}
+
+
+def measure_fp4_peak(iters=16384, reps=7):
+    """Dense FP4 tensor peak of this GPU: the library's tcgen05 kind::mxf4
+    probe (one CTA per SM, operands in shared memory, M = N = 128, K = 64),
+    timed by CUDA events per launch after two warm-up launches; the median
+    launch, with the SM clocks sampled meanwhile."""
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    sink = torch.zeros(1024, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        grid = ft.ft_fp4_mma_probe(iters, sink, status, stream.cuda_stream)
+    ms = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            grid = ft.ft_fp4_mma_probe(iters, sink, status, stream.cuda_stream)
+            b.record(stream)
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+    if int(status.item()) != 0:
+        raise RuntimeError("FP4 probe: the wait for the tensor pipe gave up")
+    flops = grid * iters * 4 * 2 * 128 * 128 * 64
+    t = statistics.median(ms)
+    return {"tflops": flops / (t * 1e-3) / 1e12, "ms": t, "ctas": grid, "iters": iters,
+            "instruction": "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32, M = N = 128, K = 64",
+            "clocks": clk.summary()}
 
 
 def overlap_fraction(copy_ms, compute_ms, total_ms, hideable_ms):
@@ -494,9 +524,13 @@ def measure_prefill(reps=3, layers=3):
     wbytes = E2 * ft.ft_blob_layout(H2, I2)["used"]
     res["gemm_weight_gbs"] = wbytes / (gemm_ms * 1e-3) / 1e9
     pk = peaks()
-    res["gemm_roofline"] = {**prefill_roofline(flops, wbytes, pk["hbm"], res["gemm_tflops"]),
+    fp4 = measure_fp4_peak()
+    res["fp4_peak"] = fp4
+    res["gemm_roofline"] = {**prefill_roofline(flops, wbytes, pk["hbm"], res["gemm_tflops"], fp4["tflops"]),
                             "hbm_peak_gbs": pk["hbm"], "hbm_peak_source": pk["src"],
-                            "fp4_peak_tflops": FP4_DENSE_TFLOPS_NOMINAL, "fp4_peak_source": "nominal"}
+                            "fp4_peak_tflops": fp4["tflops"], "fp4_peak_source": "measured (tcgen05 mxf4 probe)",
+                            "fp4_nominal_tflops": FP4_DENSE_TFLOPS_NOMINAL}
+    res["calibration"] = measure_prefill_calibration(fp4["tflops"])
     # (b) pinned host pools, double-buffered prefetch
     hp = host_layer_pools(H2, I2, E2, seed, layers)
     ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, layers, 0, 0, T2), hp, None)
@@ -527,63 +561,159 @@ def measure_prefill(reps=3, layers=3):
     return res
 
 
-def measure_misses(tokens=64, layers=8):
-    """DeepSeek-V4-Flash-class decode over a GPU LRU expert cache: hidden 4096,
-    256 experts top-6, intermediate 2048; `layers` of the 43 layers with their
-    full pools in pinned host memory and the cache budget scaled from 32 GB of
-    the 147 GB pool; batch 1; Zipf(1.0) traces with 0.5 adjacent reuse;
-    budget shrunk to half and restored mid-trace."""
+def host_pools_pageable(H, I, n_blobs, seed, layers):
+    """Host pools of `layers` layers in ordinary (pageable) host memory, filled
+    on the GPU by the seeded filler and copied down; ft_create pins them
+    (cudaHostRegister) without copying.  Pageable numpy buffers avoid the
+    power-of-two rounding of torch's pinned allocator at these sizes."""
+    import numpy as np
+    import torch
+    import synth.gpu
+    stride = synth.blob_stride(H, I)
+    pools = []
+    for layer in range(layers):
+        h = np.empty(n_blobs * stride, np.uint8)
+        d = synth.gpu.layer_pool(H, I, n_blobs, seed, layer)
+        torch.from_numpy(h).copy_(d)
+        del d
+        pools.append(h)
+    torch.cuda.synchronize()
+    return pools
+
+
+def available_host_bytes():
+    try:
+        import psutil
+        return psutil.virtual_memory().available
+    except Exception:
+        return os.sysconf("SC_AVPHYS_PAGES") * os.sysconf("SC_PAGE_SIZE")
+
+
+def measure_prefill_calibration(fp4_peak, T=65536, reps=2):
+    """The compute-bound calibration shape of the prefill GEMMs: the
+    DSV4-class layer (hidden 4096, 256 experts top-6, intermediate 2048) on a
+    65,536-token chunk, 1,536 tokens per expert on average (arithmetic
+    intensity ~5.8k FLOP per weight byte, above the HBM / FP4 ridge), through
+    the same path; GEMM TFLOP/s from the kernel timers against the measured
+    FP4 peak.  Not a workload of its own: it shows the GEMM where the tensor
+    pipe, not HBM, bounds it."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+    H2, I2, E2, k2, seed = 4096, 2048, 256, 6, 1005
+    flops = 2.0 * T * k2 * 3 * H2 * I2
+    pool = synth.gpu.layer_pool(H2, I2, E2, seed, 0)
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, 1, 0, 0, T), None, [pool])
+    x = torch.from_numpy(synth.activations_bf16(seed, 1, T, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    lg = torch.from_numpy(synth.logits_for_sets(seed, 3, synth.near_uniform_sets(seed, 0, T, E2, k2), E2)).cuda()
+    out = torch.empty_like(x)
+    flags = ft.FT_ACT_MXFP4 | ft.FT_ROUTE_RENORM
+    ft.ft_moe_layer_forward(ctx, 0, x, T, None, lg, out, flags)
+    torch.cuda.synchronize()
+    ft.ft_kernel_timing_enable(ctx, True)
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, x, T, None, lg, out, flags)
+    kt = ft.ft_kernel_timing_read(ctx)
+    ft.ft_kernel_timing_enable(ctx, False)
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    del pool, x, out, lg
+    torch.cuda.empty_cache()
+    gemm_ms = (kt["gemm_gate_up"][0] + kt["gemm_down"][0]) / reps
+    tf = flops / (gemm_ms * 1e-3) / 1e12
+    return {"workload": f"DSV4-class prefill GEMMs, {T} tokens top-{k2} over {E2} experts ({T * k2 // E2} tokens "
+                        "per expert on average)",
+            "flop": flops, "gemm_ms": gemm_ms, "gemm_tflops": tf, "frac_of_fp4_peak": tf / fp4_peak,
+            "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps}
+
+
+def measure_misses(tokens=512, layers=43, resize_at=(170, 340)):
+    """DeepSeek-V4-Flash-class decode over a GPU LRU expert cache (hidden
+    4096, 256 experts top-6, intermediate 2048): `layers` layers (43 = the
+    model) with their full pools in host memory pinned by the context, a
+    32 GiB cache budget (2570 slots) halved at token 170 and restored at token
+    340, batch 1 over a 512-token Zipf(1.0) trace with 0.5 adjacent reuse.
+    The run goes twice on fresh contexts with the same trace (the same LRU
+    events and copies): the default order, where the resident experts run
+    while the misses' copies are in flight and each missed expert after its
+    own copy, and FT_CACHE_SERIAL, where every copy lands first.  When the
+    host cannot hold the full pool, the largest layer count that fits runs
+    and the budget keeps its 32 GiB share of those layers (stated in the
+    workload); tok/s is measured, never extrapolated."""
     import numpy as np
     import torch
     import expert_offloaded_serving_b200 as ft
     import synth
     H3, I3, E3, k3, seed = 4096, 2048, 256, 6, 1003
     stride = ft.ft_blob_stride(H3, I3)
-    budget = int(32e9 * layers / 43) // stride * stride
-    hp = host_layer_pools(H3, I3, E3, seed, layers)
+    pool_bytes = E3 * stride
+    fit = int((available_host_bytes() - 24e9) // pool_bytes)
+    L3 = max(1, min(layers, fit))
+    budget = int(32 * 2 ** 30 * L3 / layers) // stride * stride
+    hp = host_pools_pageable(H3, I3, E3, seed, L3)
     h2d_peak = pinned_h2d_gbs()
-    ctx = ft.ft_create(ft.make_desc(H3, I3, E3, k3, layers, 0, budget, 1), hp, None)
-    sets = np.stack([synth.zipf_trace(seed, l, tokens, E3, k3, 1.0, 0.5) for l in range(layers)], axis=1)
+    sets = np.stack([synth.zipf_trace(seed, l, tokens, E3, k3, 1.0, 0.5) for l in range(L3)], axis=1)
     lg = torch.from_numpy(np.stack([[synth.logits_for_sets(seed, p * 100 + l, sets[p, l][None], E3)[0]
-                                     for l in range(layers)] for p in range(tokens)])).cuda()
+                                     for l in range(L3)] for p in range(tokens)])).cuda()
     x = torch.from_numpy(synth.activations_bf16(seed, 1, 1, H3).view(np.int16).copy()).cuda().view(torch.bfloat16)
     bufs = [torch.empty_like(x), torch.empty_like(x)]
-    ft.ft_cache_stats_get(ctx, reset=True)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    cur = x
-    for p in range(tokens):
-        if p == tokens // 3:
-            ft.ft_expert_cache_resize(ctx, budget // 2)
-        if p == 2 * tokens // 3:
-            ft.ft_expert_cache_resize(ctx, budget)
-        for l in range(layers):
-            nxt = bufs[(p * layers + l) % 2]
-            ft.ft_moe_layer_forward(ctx, l, cur, 1, None, lg[p, l], nxt, ft.FT_ROUTE_RENORM)
-            cur = nxt
-    b.record()
-    b.synchronize()
-    st = ft.ft_cache_stats_get(ctx)
-    ev = ft.ft_cache_trace(ctx, cap=1 << 16)
-    ft.ft_sync_status(ctx)
+
+    # one context (pinning the pool once); the second run starts from a cold
+    # cache again: a resize to 0 evicts every expert, the next restores the budget
+    ctx = ft.ft_create(ft.make_desc(H3, I3, E3, k3, L3, 0, budget, 1), hp, None)
+
+    def run(flags):
+        ft.ft_expert_cache_resize(ctx, 0)
+        ft.ft_expert_cache_resize(ctx, budget)
+        ft.ft_cache_trace(ctx, cap=1 << 22)
+        ft.ft_cache_stats_get(ctx, reset=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        cur = x
+        for p in range(tokens):
+            if p == resize_at[0]:
+                ft.ft_expert_cache_resize(ctx, budget // 2 // stride * stride)
+            if p == resize_at[1]:
+                ft.ft_expert_cache_resize(ctx, budget)
+            for l in range(L3):
+                nxt = bufs[(p * L3 + l) % 2]
+                ft.ft_moe_layer_forward(ctx, l, cur, 1, None, lg[p, l], nxt, flags)
+                cur = nxt
+        b.record()
+        b.synchronize()
+        st = ft.ft_cache_stats_get(ctx)
+        ev = ft.ft_cache_trace(ctx, cap=1 << 22)
+        ft.ft_sync_status(ctx)
+        return a.elapsed_time(b), st, ev
+
+    total_ms, st, ev = run(ft.FT_ROUTE_RENORM)
+    serial_ms, st_s, _ = run(ft.FT_ROUTE_RENORM | ft.FT_CACHE_SERIAL)
     ft.ft_destroy(ctx)
     del hp
-    total_ms = a.elapsed_time(b)
     lookups = st["hits"] + st["misses"]
     miss_gbs = st["h2d_bytes"] / (st["h2d_ms"] * 1e-3) / 1e9 if st["h2d_ms"] > 0 else None
-    t3 = tokens // 3
-    phases = miss_phases(ev, layers * k3, [("cold_first_token", (0, 1)), ("warm_full_budget", (1, t3)),
-                                          ("half_budget", (t3, 2 * t3)), ("restored_budget", (2 * t3, tokens))])
-    return {"workload": f"DSV4-class decode with expert cache: {layers} of 43 layers, pools in pinned host memory, "
-                        f"budget {budget / 1e9:.1f} GB (32 GB x {layers}/43), batch 1, {tokens} tokens, "
-                        "resize to half and back",
-            "tok_s": tokens / (total_ms * 1e-3) * layers / 43,
+    phases = miss_phases(ev, L3 * k3, [("cold_first_token", (0, 1)), ("warm_full_budget", (1, resize_at[0])),
+                                       ("half_budget", resize_at), ("restored_budget", (resize_at[1], tokens))])
+    return {"workload": f"DSV4-class decode with expert cache: {L3} of {layers} layers, "
+                        f"{L3 * pool_bytes / 1e9:.1f} GB pool in pinned host memory, budget "
+                        f"{budget / 2 ** 30:.2f} GiB ({budget // stride} slots) halved at token {resize_at[0]} and "
+                        f"restored at token {resize_at[1]}, batch 1, {tokens} tokens",
+            "layers": L3, "tokens": tokens, "host_bytes_available": available_host_bytes(),
+            "tok_s": tokens / (total_ms * 1e-3), "ms": total_ms,
             "miss_rate": st["misses"] / max(lookups, 1), "miss_rate_by_phase": phases,
+            "hits": st["hits"], "misses": st["misses"], "evictions": st["evictions"], "moves": st["moves"],
+            "miss_h2d_gbs": miss_gbs, "pinned_h2d_gbs": h2d_peak,
+            "miss_h2d_frac": (miss_gbs / h2d_peak) if miss_gbs else None,
             "copy_busy_share": st["h2d_ms"] / total_ms if total_ms > 0 else None,
-            "hits": st["hits"], "misses": st["misses"],
-            "evictions": st["evictions"], "moves": st["moves"], "miss_h2d_gbs": miss_gbs,
-            "pinned_h2d_gbs": h2d_peak, "miss_h2d_frac": (miss_gbs / h2d_peak) if miss_gbs else None}
-
+            # the resident experts' kernels of steps with misses, and the part of
+            # them that ran while those steps' copies were in flight
+            "overlap": {"resident_expert_ms": st["hit_ms"], "under_copies_ms": st["overlap_ms"],
+                        "frac_of_resident_compute_hidden": st["overlap_ms"] / st["hit_ms"] if st["hit_ms"] else None,
+                        "serial_order_tok_s": tokens / (serial_ms * 1e-3),
+                        "saved_ms": serial_ms - total_ms}}
 
 
 def measure_decode_batch(args, T, pk):

@@ -33,7 +33,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
            "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry",
-           "ft_debug_stack_epoch", "ft_flow_geometry")
+           "ft_debug_stack_epoch", "ft_flow_geometry", "ft_fp4_mma_probe")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -109,6 +109,7 @@ def lib() -> C.CDLL:
         "ft_debug_fail_copy": (ST, [P, I64]),
         "ft_debug_stack_epoch": (ST, [P, U32, I32]),
         "ft_flow_geometry": (ST, [I32, I32, I32, I32, I32, I32, I32, C.POINTER(I64)]),
+        "ft_fp4_mma_probe": (ST, [I64, P, P, C.POINTER(I32), P]),
         "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
     for name, (res, args) in sig.items():
@@ -271,6 +272,14 @@ def ft_debug_host_wait_limit(ctx, seconds: float) -> None:
 
 def ft_debug_fail_copy(ctx, n: int) -> None:
     _check(lib().ft_debug_fail_copy(ctx, n))
+
+
+def ft_fp4_mma_probe(iters: int, sink, status, stream=None) -> int:
+    """Launch the FP4 tensor-peak probe; returns the CTAs launched.  FLOPs =
+    CTAs * iters * 4 * 2 * 128 * 128 * 64."""
+    g = I32()
+    _check(lib().ft_fp4_mma_probe(iters, _ptr(sink, 4), _ptr(status, 4), C.byref(g), _stream(stream)))
+    return g.value
 
 
 def ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers) -> dict:

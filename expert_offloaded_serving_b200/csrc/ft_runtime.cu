@@ -655,6 +655,20 @@ extern "C" ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n
   return FT_OK;
 }
 
+namespace ft {
+size_t fp4_probe_smem();
+cudaError_t launch_fp4_probe(int64_t iters, float* sink, int* status, int* grid_out, cudaStream_t s);
+}  // namespace ft
+
+extern "C" ft_status ft_fp4_mma_probe(int64_t iters, float* sink, int32_t* status, int32_t* grid, void* stream) {
+  if (!sink || !status || !grid) return fail(FT_ERR_INVALID, "NULL argument");
+  if (iters < 1 || iters > 65536) return fail(FT_ERR_INVALID, "iters %lld outside [1, 65536]", (long long)iters);
+  int g = 0;
+  CUDA_TRY(launch_fp4_probe(iters, sink, status, &g, (cudaStream_t)stream));
+  *grid = g;
+  return FT_OK;
+}
+
 extern "C" ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
                                       int32_t n_experts, int32_t n_layers, int64_t out[3]) {
   if (!out) return fail(FT_ERR_INVALID, "out is NULL");

@@ -369,6 +369,17 @@ FT_API ft_status ft_debug_fail_copy(ft_ctx* ctx, int64_t n);
 /* measurement                                                             */
 /* ---------------------------------------------------------------------- */
 
+/* FP4 tensor-core peak probe: one CTA per SM issues iters (1 .. 65536)
+ * rounds of four tcgen05.mma kind::mxf4 (M = N = 128, K = 64, MXFP4 x MXFP4
+ * with UE8M0 block scales, the prefill GEMM's instruction) on operands held
+ * in shared memory, into a tensor-memory accumulator, on `stream`.  It
+ * performs (*grid) * iters * 4 * 2 * 128 * 128 * 64 floating-point operations
+ * and reads no global memory while it runs, so the launch time measures the
+ * tensor pipe.  sink: dev fp32 [number of SMs], one accumulator value per CTA;
+ * status: dev int32, bit 4 set if the wait for the tensor pipe gave up
+ * (200 ms).  *grid = CTAs launched.  Errors: FT_ERR_INVALID, FT_ERR_CUDA. */
+FT_API ft_status ft_fp4_mma_probe(int64_t iters, float* sink, int32_t* status, int32_t* grid, void* stream);
+
 /* Kernel classes of the per-kernel timers. */
 #define FT_K_ROUTER_LOGITS 0
 #define FT_K_TOPK          1
