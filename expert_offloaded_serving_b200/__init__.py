@@ -33,7 +33,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
            "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry",
-           "ft_debug_stack_epoch", "ft_flow_geometry", "ft_fp4_mma_probe")
+           "ft_debug_stack_epoch", "ft_flow_geometry", "ft_fp4_mma_probe", "ft_blob_layout_format")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -48,7 +48,7 @@ class FtError(RuntimeError):
 class ModelDesc(C.Structure):
     _fields_ = [("hidden", C.c_int32), ("inter", C.c_int32), ("n_experts", C.c_int32), ("top_k", C.c_int32),
                 ("n_layers", C.c_int32), ("n_shared", C.c_int32), ("cache_budget_bytes", C.c_int64),
-                ("max_tokens", C.c_int32), ("reserved", C.c_int32)]
+                ("max_tokens", C.c_int32), ("weight_format", C.c_int32)]
 
 
 class CacheEvent(C.Structure):
@@ -108,7 +108,8 @@ def lib() -> C.CDLL:
         "ft_debug_host_wait_limit": (ST, [P, C.c_double]),
         "ft_debug_fail_copy": (ST, [P, I64]),
         "ft_debug_stack_epoch": (ST, [P, U32, I32]),
-        "ft_flow_geometry": (ST, [I32, I32, I32, I32, I32, I32, I32, C.POINTER(I64)]),
+        "ft_flow_geometry": (ST, [I32, I32, I32, I32, I32, I32, I32, I32, C.POINTER(I64)]),
+        "ft_blob_layout_format": (ST, [I32, I32, I32, C.POINTER(I64)]),
         "ft_fp4_mma_probe": (ST, [I64, P, P, C.POINTER(I32), P]),
         "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
@@ -165,6 +166,15 @@ def ft_blob_layout(hidden: int, inter: int) -> dict:
     out = (I64 * 8)()
     _check(lib().ft_blob_layout(hidden, inter, out))
     return dict(zip(("wg", "wu", "wd", "wg_sf", "wu_sf", "wd_sf", "used", "stride"), list(out)))
+
+
+FT_FMT_MXFP4, FT_FMT_NVFP4, FT_FMT_BF16 = 0, 1, 2
+
+
+def ft_blob_layout_format(hidden: int, inter: int, fmt: int) -> dict:
+    out = (I64 * 9)()
+    _check(lib().ft_blob_layout_format(hidden, inter, fmt, out))
+    return dict(zip(("wg", "wu", "wd", "wg_sf", "wu_sf", "wd_sf", "used", "stride", "ts"), list(out)))
 
 
 def ft_create(desc: ModelDesc, host_layers=None, resident_layers=None) -> int:
@@ -282,9 +292,9 @@ def ft_fp4_mma_probe(iters: int, sink, status, stream=None) -> int:
     return g.value
 
 
-def ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers) -> dict:
+def ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, weight_format=0) -> dict:
     out = (I64 * 3)()
-    _check(lib().ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, out))
+    _check(lib().ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, weight_format, out))
     return {"ok": bool(out[0]), "rows_cap": out[1], "smem": out[2]}
 
 
@@ -325,5 +335,6 @@ def ft_moe_layer_forward_noalloc(hidden, inter, n_experts, top_k, n_shared, laye
 
 
 def make_desc(hidden, inter, n_experts, top_k, n_layers=1, n_shared=0, cache_budget_bytes=0,
-              max_tokens=16) -> ModelDesc:
-    return ModelDesc(hidden, inter, n_experts, top_k, n_layers, n_shared, cache_budget_bytes, max_tokens, 0)
+              max_tokens=16, weight_format=0) -> ModelDesc:
+    return ModelDesc(hidden, inter, n_experts, top_k, n_layers, n_shared, cache_budget_bytes, max_tokens,
+                     weight_format)

@@ -19,26 +19,65 @@ constexpr int kStMissing = 8;   // an expert pointer was NULL at kernel time
 
 __host__ __device__ inline int64_t pad_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
+// expert weight formats (ft_model_desc.weight_format)
+constexpr int kFmtMx = 0;    // MXFP4: e2m1 codes, one UE8M0 scale per 32 elements
+constexpr int kFmtNv = 1;    // NVFP4: e2m1 codes, one E4M3 scale per 16 elements, one fp32 scale per matrix
+constexpr int kFmtBf16 = 2;  // BF16 weights
+
 struct BlobLayout {
   int64_t wg, wu, wd, wg_sf, wu_sf, wd_sf, used, stride;
+  int64_t ts;  // NVFP4: the three fp32 matrix scales (Wg, Wu, Wd); else -1
+  int fmt;
 };
 
 // Region offsets of one expert blob (see ft_moe.h).
-__host__ __device__ inline BlobLayout blob_layout(int H, int I) {
+//   MXFP4: codes Wg [I][H/2], Wu [I][H/2], Wd [H][I/2], then UE8M0 scale
+//          regions (128-row x 4-block atoms, blocks of 32 along K).
+//   NVFP4: the same codes, then E4M3 scale regions in the same atoms with
+//          blocks of 16, then three fp32 matrix scales and 4 zero bytes.
+//   BF16:  Wg [I][H], Wu [I][H], Wd [H][I] as bf16 (no scales).
+// Each padded to a multiple of 256 bytes.
+__host__ __device__ inline BlobLayout blob_layout(int H, int I, int fmt = kFmtMx) {
   BlobLayout b;
+  b.fmt = fmt;
+  b.ts = -1;
+  if (fmt == kFmtBf16) {
+    b.wg = 0;
+    b.wu = 2 * (int64_t)I * H;
+    b.wd = 4 * (int64_t)I * H;
+    b.used = 6 * (int64_t)I * H;
+    b.wg_sf = b.wu_sf = b.wd_sf = b.used;
+    b.stride = pad_up(b.used, 256);
+    return b;
+  }
+  const int blk = fmt == kFmtNv ? 16 : 32;
   int64_t gu = (int64_t)I * H / 2;
   b.wg = 0;
   b.wu = gu;
   b.wd = 2 * gu;
   int64_t end = b.wd + (int64_t)H * I / 2;
-  int64_t sf_gu = pad_up(I, 128) * pad_up(H / 32, 4);
-  int64_t sf_d = pad_up(H, 128) * pad_up(I / 32, 4);
+  int64_t sf_gu = pad_up(I, 128) * pad_up(H / blk, 4);
+  int64_t sf_d = pad_up(H, 128) * pad_up(I / blk, 4);
   b.wg_sf = end;
   b.wu_sf = end + sf_gu;
   b.wd_sf = end + 2 * sf_gu;
   b.used = end + 2 * sf_gu + sf_d;
+  if (fmt == kFmtNv) {
+    b.ts = b.used;
+    b.used += 16;
+  }
   b.stride = pad_up(b.used, 256);
   return b;
+}
+
+// E4M3 byte (no infinities, S.1111.111 = NaN) -> fp32, exact: exponent 0 is
+// subnormal m/8 * 2^-6, else (1 + m/8) * 2^(e - 7).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  const uint32_t s = (b >> 7) & 1u, e = (b >> 3) & 15u, m = b & 7u;
+  if (e == 15u && m == 7u) return __uint_as_float(0x7fc00000u);
+  const uint32_t bits =
+      e == 0u ? (m == 0u ? 0u : __float_as_uint((float)m * 0.001953125f)) : (((e + 120u) << 23) | (m << 20));
+  return __uint_as_float(bits | (s << 31));
 }
 
 // Byte offset of the 4-byte scale word holding blocks 4a..4a+3 of `row` in a

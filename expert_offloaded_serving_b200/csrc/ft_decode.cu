@@ -56,8 +56,15 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 struct CtaHdr {
   int32_t tok[16];
   int32_t last;
-  int32_t pad[3];
+  float ts[2];  // NVFP4: the matrix scales of the tile's matrices (else unused)
+  int32_t pad;
 };
+static_assert(sizeof(CtaHdr) <= 128, "CtaHdr");
+
+// NVFP4: the fp32 scale of matrix `mat` (0 Wg, 1 Wu, 2 Wd) of a blob.
+__device__ __forceinline__ float nv_matrix_scale(const uint8_t* blob, const BlobLayout& lay, int mat) {
+  return reinterpret_cast<const float*>(blob + lay.ts)[mat];
+}
 constexpr size_t kTileOff = 128;
 
 // Order key of a logit: larger key = ranks first.  NaN -> 1 (below -inf),
@@ -218,11 +225,12 @@ __device__ __forceinline__ bool resolve_unit(const DecodeArgs& a, const Route* _
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU: CTA = (unit, block of R rows of Wg and Wu), full K = H
 // ---------------------------------------------------------------------------
+template <int F>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
   uint8_t* base = smem + kTileOff;
-  const Gv g = make_gv(a.H, a.I, 2);
+  const Gv g = make_gv(a.H, a.I, 2, F);
   const int nrb = a.I / g.R;
   const int rb = blockIdx.x % nrb, u = a.n_sel ? a.sel[blockIdx.x / nrb] : blockIdx.x / nrb;
   UnitInfo ui;
@@ -240,6 +248,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
   stage_mat(g, base, 0, blob + a.lay.wg, blob + a.lay.wg_sf, row0);
   stage_mat(g, base, 1, blob + a.lay.wu, blob + a.lay.wu_sf, row0);
   cp_async_commit();
+  if (F == kFmtNv && threadIdx.x < 2) hd.ts[threadIdx.x] = nv_matrix_scale(blob, a.lay, threadIdx.x);
   pdl_trigger();
   pdl_wait();  // x is the previous kernel's output when launched as a dependent
   const LaneMap m = lane_map(g);
@@ -249,12 +258,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
     stage_x<true>(g, base, a.x, hd.tok + t0, n);
     cp_async_wait_all();
     __syncthreads();
-    tile_dots(g, m, base, n);
+    tile_dots<F>(g, m, base, n);
     __syncthreads();
     if (threadIdx.x < g.R * n) {
       const int t = threadIdx.x >> g.rlog, r = threadIdx.x & (g.R - 1);
-      a.h[(size_t)(ui.hbase + t0 + t) * a.I + row0 + r] =
-          silu(row_value(g, base, 0, r, t)) * row_value(g, base, 1, r, t);
+      float gv = row_value(g, base, 0, r, t), uv = row_value(g, base, 1, r, t);
+      if (F == kFmtNv) {
+        gv *= hd.ts[0];
+        uv *= hd.ts[1];
+      }
+      a.h[(size_t)(ui.hbase + t0 + t) * a.I + row0 + r] = silu(gv) * uv;
     }
   }
 }
@@ -263,11 +276,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_gate_up(DecodeArgs a) {
 // down + combine: CTA = (unit, block of R rows of Wd), full K = I.  The last
 // CTA to finish a row block (one counter per block) does the weighted combine.
 // ---------------------------------------------------------------------------
+template <int F>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   CtaHdr& hd = *reinterpret_cast<CtaHdr*>(smem);
   uint8_t* base = smem + kTileOff;
-  const Gv g = make_gv(a.I, a.H, 1);
+  const Gv g = make_gv(a.I, a.H, 1, F);
   const int nrb = a.H / g.R;
   const int rb = blockIdx.x % nrb, u = a.n_sel ? a.sel[blockIdx.x / nrb] : blockIdx.x / nrb;
   UnitInfo ui;
@@ -283,6 +297,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
   const int row0 = rb * g.R;
   stage_mat(g, base, 0, blob + a.lay.wd, blob + a.lay.wd_sf, row0);
   cp_async_commit();
+  if (F == kFmtNv && threadIdx.x == 0) hd.ts[0] = nv_matrix_scale(blob, a.lay, 2);
   pdl_trigger();
   pdl_wait();  // h is written by the gate/up kernel
   if (threadIdx.x < 16) hd.tok[threadIdx.x] = ui.hbase + threadIdx.x;  // h rows of the unit's tokens
@@ -293,11 +308,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
     stage_x<false>(g, base, a.h, hd.tok + t0, n);
     cp_async_wait_all();
     __syncthreads();
-    tile_dots(g, m, base, n);
+    tile_dots<F>(g, m, base, n);
     __syncthreads();
     if (threadIdx.x < g.R * n) {
       const int t = threadIdx.x >> g.rlog, r = threadIdx.x & (g.R - 1);
-      a.y[(size_t)(ui.hbase + t0 + t) * a.H + row0 + r] = row_value(g, base, 0, r, t);
+      float yv = row_value(g, base, 0, r, t);
+      if (F == kFmtNv) yv *= hd.ts[0];
+      a.y[(size_t)(ui.hbase + t0 + t) * a.H + row0 + r] = yv;
     }
   }
   // last CTA of this row block combines
@@ -333,12 +350,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_down(DecodeArgs a) {
 // e2m1x8_to_f16x8, the conversion the dot products use; out = f16 value x
 // UE8M0 scale (exact in fp32 unless it overflows).
 // ---------------------------------------------------------------------------
+template <int F>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_dequant(const uint8_t* blob, BlobLayout lay, int mat, int H,
                                                                  int I, float* out) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* base = smem + kTileOff;
   const int K = mat < 2 ? H : I, rows = mat < 2 ? I : H;
-  const Gv g = make_gv(K, rows, 1);
+  const Gv g = make_gv(K, rows, 1, F);
   const int row0 = blockIdx.x * g.R;
   const int64_t co = mat == 0 ? lay.wg : mat == 1 ? lay.wu : lay.wd;
   const int64_t so = mat == 0 ? lay.wg_sf : mat == 1 ? lay.wu_sf : lay.wd_sf;
@@ -348,22 +366,44 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_dequant(const uint8_t* 
   __syncthreads();
   const uint8_t* codes = base + g.codes;
   const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
+  const float ts = F == kFmtNv ? nv_matrix_scale(blob, lay, mat) : 1.f;
   for (int i = threadIdx.x; i < g.R * g.chunks; i += kGemvThreads) {
     const int r = i / g.chunks, c = i - r * g.chunks;
-    uint4 q;
-    float s;
-    tile_chunk(g, codes, sc, r, c, q, s);
-    const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
     float* o = out + (size_t)(row0 + r) * K + c * 32;
+    if constexpr (F == kFmtBf16) {
+      uint4 q[4];
+      tile_chunk_bf16(g, codes, r, c, q);
 #pragma unroll
-    for (int wv = 0; wv < 4; wv++) {
-      uint32_t hv[4];
-      e2m1x8_to_f16x8(qs[wv], hv);
+      for (int i4 = 0; i4 < 4; i4++) {
+        const uint32_t ws[4] = {q[i4].x, q[i4].y, q[i4].z, q[i4].w};
 #pragma unroll
-      for (int j = 0; j < 4; j++) {
-        const float2 f = f16x2_to_f32x2(hv[j]);
-        o[8 * wv + 2 * j] = f.x * s;
-        o[8 * wv + 2 * j + 1] = f.y * s;
+        for (int j = 0; j < 4; j++) {
+          o[8 * i4 + 2 * j] = __uint_as_float(ws[j] << 16);
+          o[8 * i4 + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+        }
+      }
+    } else {
+      uint4 q;
+      float s0, s1;
+      if constexpr (F == kFmtNv) {
+        tile_chunk_nv(g, codes, sc, r, c, q, s0, s1);
+      } else {
+        tile_chunk(g, codes, sc, r, c, q, s0);
+        s1 = s0;
+      }
+      const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int wv = 0; wv < 4; wv++) {
+        uint32_t hv[4];
+        e2m1x8_to_f16x8(qs[wv], hv);
+        const float s = wv < 2 ? s0 : s1;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const float2 f = f16x2_to_f32x2(hv[j]);
+          // NVFP4: (code x block scale) is exact; the matrix scale rounds once
+          o[8 * wv + 2 * j] = F == kFmtNv ? (f.x * s) * ts : f.x * s;
+          o[8 * wv + 2 * j + 1] = F == kFmtNv ? (f.y * s) * ts : f.y * s;
+        }
       }
     }
   }
@@ -715,7 +755,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
           drain();
           return;
         }
-        tile_dots(gA, lmA, baseA, n);
+        tile_dots<kFmtMx>(gA, lmA, baseA, n);
         __syncthreads();
         if (threadIdx.x < gA.R * n) {
           const int t = threadIdx.x >> gA.rlog, r = threadIdx.x & (gA.R - 1);
@@ -769,7 +809,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
             drain();
             return;
           }
-          tile_dots(gB, lmB, baseB, n);
+          tile_dots<kFmtMx>(gB, lmB, baseB, n);
           __syncthreads();
           if (threadIdx.x < gB.R * n) {
             const int t = threadIdx.x >> gB.rlog, r = threadIdx.x & (gB.R - 1);
@@ -908,30 +948,39 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dec_gate_up(const DecodeArgs& a, bool pdl, cudaStream_t s) {
-  const Gv g = make_gv(a.H, a.I, 2);
+  const int F = a.lay.fmt;
+  const Gv g = make_gv(a.H, a.I, 2, F);
   const int units = a.n_sel ? a.n_sel : a.max_units + a.n_shared;
-  return launch_one(k_dec_gate_up, a, g, a.I, units * (a.I / g.R), pdl, s);
+  void (*kern)(DecodeArgs) =
+      F == kFmtNv ? k_dec_gate_up<kFmtNv> : F == kFmtBf16 ? k_dec_gate_up<kFmtBf16> : k_dec_gate_up<kFmtMx>;
+  return launch_one(kern, a, g, a.I, units * (a.I / g.R), pdl, s);
 }
 
 cudaError_t launch_dec_down(const DecodeArgs& a, bool pdl, cudaStream_t s) {
-  const Gv g = make_gv(a.I, a.H, 1);
+  const int F = a.lay.fmt;
+  const Gv g = make_gv(a.I, a.H, 1, F);
   const int units = a.n_sel ? a.n_sel : a.max_units + a.n_shared;
-  return launch_one(k_dec_down, a, g, a.H, units * (a.H / g.R), pdl, s);
+  void (*kern)(DecodeArgs) = F == kFmtNv ? k_dec_down<kFmtNv> : F == kFmtBf16 ? k_dec_down<kFmtBf16> : k_dec_down<kFmtMx>;
+  return launch_one(kern, a, g, a.H, units * (a.H / g.R), pdl, s);
 }
 
 cudaError_t launch_dec_dequant(const uint8_t* blob, const BlobLayout& lay, int mat, int H, int I, float* out,
                                cudaStream_t s) {
   const int K = mat < 2 ? H : I, rows = mat < 2 ? I : H;
-  const Gv g = make_gv(K, rows, 1);
+  const Gv g = make_gv(K, rows, 1, lay.fmt);
   if (!gv_ok(g, rows)) return cudaErrorInvalidValue;
   const size_t smem = kTileOff + g.total;
-  cudaError_t e = cudaFuncSetAttribute(k_dec_dequant, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  void (*kern)(const uint8_t*, BlobLayout, int, int, int, float*) =
+      lay.fmt == kFmtNv ? k_dec_dequant<kFmtNv> : lay.fmt == kFmtBf16 ? k_dec_dequant<kFmtBf16> : k_dec_dequant<kFmtMx>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_dec_dequant<<<rows / g.R, kGemvThreads, smem, s>>>(blob, lay, mat, H, I, out);
+  kern<<<rows / g.R, kGemvThreads, smem, s>>>(blob, lay, mat, H, I, out);
   return cudaGetLastError();
 }
 
-bool decode_supported(int H, int I) { return gv_ok(make_gv(H, I, 2), I) && gv_ok(make_gv(I, H, 1), H); }
+bool decode_supported(int H, int I, int fmt) {
+  return gv_ok(make_gv(H, I, 2, fmt), I) && gv_ok(make_gv(I, H, 1, fmt), H);
+}
 
 void decode_geometry(int H, int I, int64_t* out) {
   const Gv gs[2] = {make_gv(H, I, 2), make_gv(I, H, 1)};

@@ -74,9 +74,9 @@ struct DecodeArgs {
   uint16_t sel[kMaxUnits];
 };
 
-// True when the decode kernels take this shape (hidden and inter multiples of
-// 128, both at most 16384).
-bool decode_supported(int H, int I);
+// True when the decode kernels take this shape in weight format fmt (hidden
+// and inter multiples of 128, both at most 16384).
+bool decode_supported(int H, int I, int fmt = kFmtMx);
 // Tile geometry of the decode kernels for hidden H and intermediate I:
 // out[0..9] gate/up tile, out[10..19] down tile, each K, chunks, lpr, rpw,
 // parts, rsets, groups, R, shared bytes of a per-layer CTA, taken (0/1);
@@ -147,7 +147,7 @@ struct FlowGeom {
   size_t smem;
   bool ok;                     // the dataflow kernel takes this shape, batch and depth
 };
-FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers);
+FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers, int fmt = kFmtMx);
 cudaError_t launch_dec_flow(const FlowArgs& a, cudaStream_t s);
 
 // One CTA waiting, with the persistent kernel's bounded wait, for *flag >= 1;

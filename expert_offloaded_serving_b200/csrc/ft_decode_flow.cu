@@ -55,8 +55,10 @@ struct FlowUnit {
   int8_t m;             // tokens of the unit (1 or 2)
   int8_t tok[2];        // their token ids
   int8_t pad[3];
+  float ts[3];          // NVFP4: the fp32 scales of Wg, Wu, Wd (else 1)
+  int32_t pad2;
 };
-static_assert(sizeof(FlowUnit) == 16, "FlowUnit");
+static_assert(sizeof(FlowUnit) == 32, "FlowUnit");
 
 // One (token, rank) pair of a layer, for the combine.
 struct FlowPair {
@@ -87,15 +89,15 @@ struct FlowHdr {
 
 // Down-tile geometry: the GEMV lane mapping for K = I, with rows_cap rows (all
 // units) and nh activation rows staged at once.
-__host__ __device__ inline Gv make_gd(int I, int rows_cap, int nh) {
-  Gv g = make_gv(I, 1 << 30, 1);
+__host__ __device__ inline Gv make_gd(int I, int rows_cap, int nh, int fmt) {
+  Gv g = make_gv(I, 1 << 30, 1, fmt);
   g.R = rows_cap;
   g.rlog = 0;
   g.codes = 0;
-  g.scales = (size_t)rows_cap * I / 2;
+  g.scales = (size_t)rows_cap * g.rowb;
   g.xh = g.scales + (size_t)rows_cap * g.atoms * 4;
-  g.xinv = g.xh + (size_t)nh * I * 2;
-  g.red = g.xinv + (((size_t)nh * g.chunks * 4 + 15) & ~(size_t)15);
+  g.xinv = g.xh + (size_t)nh * I * (fmt == kFmtBf16 ? 4 : 2);
+  g.red = g.xinv + (fmt == kFmtBf16 ? 0 : (((size_t)nh * g.chunks * 4 + 15) & ~(size_t)15));
   g.total = (g.red + (size_t)g.parts * rows_cap * kMT * 4 + 127) & ~(size_t)127;
   return g;
 }
@@ -187,14 +189,12 @@ __device__ __forceinline__ void stage_h_all(const Gv& g, uint8_t* base, const ui
 // [g*ppg, (g+1)*ppg).  Every lane of a warp runs the same number of steps, so
 // the reduction's shuffles see the whole warp; pairs past the end compute
 // zeros and are not stored.  NT = tokens per pass (2 when any unit has two).
-template <int NT>
+template <int NT, int F>
 __device__ __forceinline__ void dtile_dots(const Gv& g, const LaneMap& m, uint8_t* base, const FlowUnit* un, int U,
                                            int rb) {
   if (!m.on) return;
   const uint8_t* codes = base + g.codes;
   const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
-  const uint4* xh = reinterpret_cast<const uint4*>(base + g.xh);
-  const float* xinv = reinterpret_cast<const float*>(base + g.xinv);
   float* red = reinterpret_cast<float*>(base + g.red);
   const bool cv = m.c < g.chunks;
   const int npairs = U * rb / 2;
@@ -203,10 +203,9 @@ __device__ __forceinline__ void dtile_dots(const Gv& g, const LaneMap& m, uint8_
   int cur = -1;
   uint32_t x[kMT][16];
   float xi[kMT] = {0.f, 0.f};
+  float xf[kMT][32];
 #pragma unroll
-  for (int t = 0; t < kMT; t++)
-#pragma unroll
-    for (int i = 0; i < 16; i++) x[t][i] = 0u;
+  for (int t = 0; t < kMT; t++) zero_act<F>(x[t], xi[t], xf[t]);
   for (int jp = 0; jp < ppg; jp++) {
     const int p = m.grp * ppg + jp;
     const bool pv = p < npairs;
@@ -217,37 +216,15 @@ __device__ __forceinline__ void dtile_dots(const Gv& g, const LaneMap& m, uint8_
       const FlowUnit f = un[u];
 #pragma unroll
       for (int t = 0; t < NT; t++) {
-        if (t < f.m) {
-          const int hr = f.hrow + t;
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            const uint4 w = xh[(size_t)hr * (g.K / 8) + (size_t)i * g.chunks + m.c];
-            x[t][4 * i] = w.x;
-            x[t][4 * i + 1] = w.y;
-            x[t][4 * i + 2] = w.z;
-            x[t][4 * i + 3] = w.w;
-          }
-          xi[t] = xinv[hr * g.chunks + m.c];
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; i++) x[t][i] = 0u;
-          xi[t] = 0.f;
-        }
+        if (t < f.m) load_act<F>(g, base, f.hrow + t, m.c, x[t], xi[t], xf[t]);
+        else zero_act<F>(x[t], xi[t], xf[t]);
       }
     }
     float v[4][kMT];
 #pragma unroll
     for (int uu = 0; uu < 2; uu++) {
       v[uu][0] = v[uu][1] = 0.f;
-      if (cv && pv) {
-        uint4 q;
-        float s;
-        tile_chunk(g, codes, sc, row + uu, m.c, q, s);
-        float d[NT];
-        chunk_dot<NT>(q, x, d);
-#pragma unroll
-        for (int t = 0; t < NT; t++) v[uu][t] = d[t] * (s * xi[t]);
-      }
+      if (cv && pv) chunk_value<NT, F>(g, codes, sc, row + uu, m.c, x, xi, xf, v[uu]);
     }
     const int sel = group_reduce<2, NT>(v, g.lpr);
     if (pv && ((threadIdx.x & 31) & lmask) == 0) {
@@ -270,14 +247,14 @@ __device__ __forceinline__ float dtile_y(const Gv& g, const uint8_t* base, int r
 
 // See the file comment.  HS, IS: hidden and intermediate size fixed at compile
 // time (the tile geometry then folds to constants), or 0, 0 for any shape.
-template <int HS, int IS>
+template <int HS, int IS, int F>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = HS ? HS : a.H, I = IS ? IS : a.I;
   const int T = a.T, k = a.k, S = a.n_shared, P = T * k, NH = P + S * T;
   const int umax = min(a.E, P) + S;
-  const Gv gA = make_gv(H, I, 2);
-  const Gv gB = make_gd(I, a.rows_cap, NH);
+  const Gv gA = make_gv(H, I, 2, F);
+  const Gv gB = make_gd(I, a.rows_cap, NH, F);
   uint8_t* baseA = smem;
   uint8_t* baseB = smem + round128(gA.total);
   FlowHdr& hd = *reinterpret_cast<FlowHdr*>(baseB + gB.total);
@@ -330,6 +307,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         }
         f.blob = eptr[e];
         f.pad[0] = f.pad[1] = f.pad[2] = 0;
+        f.pad2 = 0;
+        for (int q = 0; q < 3; q++)
+          f.ts[q] = (F == kFmtNv && f.blob) ? reinterpret_cast<const float*>(f.blob + a.lay.ts)[q] : 1.f;
         if (!f.blob) set_status(a.status, kStMissing);
         un[u] = f;
       }
@@ -366,12 +346,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
     const FlowUnit f = lunits(l)[i / nrbA];
     const int row0 = (i % nrbA) * gA.R;
     if (threadIdx.x == kIssuerF) {
-      const uint32_t bytes = (uint32_t)gA.R * (uint32_t)(gA.K / 2);
+      const uint32_t bytes = (uint32_t)gA.R * (uint32_t)gA.rowb;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_expect_tx(&hd.bar[0], f.blob ? 2u * bytes : 0u);
       if (f.blob) {
-        bulk_g2s(baseA + gA.codes, f.blob + a.lay.wg + (size_t)row0 * (gA.K / 2), bytes, &hd.bar[0]);
-        bulk_g2s(baseA + gA.codes + bytes, f.blob + a.lay.wu + (size_t)row0 * (gA.K / 2), bytes, &hd.bar[0]);
+        bulk_g2s(baseA + gA.codes, f.blob + a.lay.wg + (size_t)row0 * gA.rowb, bytes, &hd.bar[0]);
+        bulk_g2s(baseA + gA.codes + bytes, f.blob + a.lay.wu + (size_t)row0 * gA.rowb, bytes, &hd.bar[0]);
       }
     }
     if (f.blob) {
@@ -386,7 +366,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
     const FlowLayerHdr lh = lhdr(l);
     const FlowUnit* un = lunits(l);
     const int rb = lh.rb, n0 = d * rb, nv = min(rb, H - n0);
-    const uint32_t rbytes = (uint32_t)nv * (uint32_t)(I / 2);
+    const uint32_t rbytes = (uint32_t)nv * (uint32_t)gB.rowb;
     if (threadIdx.x == kIssuerF) {
       uint32_t total = 0;
       for (int u = 0; u < lh.units; u++)
@@ -395,11 +375,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
       mbar_expect_tx(&hd.bar[1], total);
       for (int u = 0; u < lh.units; u++)
         if (un[u].blob)
-          bulk_g2s(baseB + gB.codes + (size_t)u * rb * (I / 2), un[u].blob + a.lay.wd + (size_t)n0 * (I / 2), rbytes,
+          bulk_g2s(baseB + gB.codes + (size_t)u * rb * gB.rowb, un[u].blob + a.lay.wd + (size_t)n0 * gB.rowb, rbytes,
                    &hd.bar[1]);
     }
     uint32_t* sd = reinterpret_cast<uint32_t*>(baseB + gB.scales);
-    const int per_u = nv * gB.atoms;
+    const int per_u = nv * gB.atoms;  // 0 for BF16: no scales
     for (int i = threadIdx.x; i < lh.units * per_u; i += kGemvThreads) {
       const int u = i / per_u, j = i - u * per_u, r = j / gB.atoms, at = j - r * gB.atoms;
       const uint8_t* bl = un[u].blob;
@@ -449,13 +429,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         drain();
         return;
       }
-      tile_dots(gA, lmA, baseA, f.m);
+      tile_dots<F>(gA, lmA, baseA, f.m);
       __syncthreads();
       if (threadIdx.x < gA.R * f.m) {
         const int t = threadIdx.x >> gA.rlog, r = threadIdx.x & (gA.R - 1);
+        float gv = row_value(gA, baseA, 0, r, t), uv = row_value(gA, baseA, 1, r, t);
+        if (F == kFmtNv) {
+          gv *= f.ts[0];
+          uv *= f.ts[1];
+        }
         // a missing expert still delivers (zeros), so no reader waits for it
-        st_tagged(a.h_tagged + (size_t)(f.hrow + t) * I + row0 + r,
-                  f.blob ? silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t) : 0.f, tag);
+        st_tagged(a.h_tagged + (size_t)(f.hrow + t) * I + row0 + r, f.blob ? silu(gv) * uv : 0.f, tag);
       }
       __syncthreads();
     }
@@ -474,8 +458,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
           drain();
           return;
         }
-        if (T > 1) dtile_dots<2>(gB, lmB, baseB, un, lh.units, rb);
-        else dtile_dots<1>(gB, lmB, baseB, un, lh.units, rb);
+        if (T > 1) dtile_dots<2, F>(gB, lmB, baseB, un, lh.units, rb);
+        else dtile_dots<1, F>(gB, lmB, baseB, un, lh.units, rb);
         __syncthreads();
         const int n0 = d * rb, nv = min(rb, H - n0), half = nv / 2;
         for (int i = threadIdx.x; i < T * half; i += kGemvThreads) {
@@ -486,12 +470,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
             float acc = 0.f;
             for (int j = 0; j < k; j++) {
               const FlowPair q = pr[t * k + j];
-              const float y = un[q.unit].blob ? dtile_y(gB, baseB, q.unit * rb + nl + e, q.slot) : 0.f;
+              float y = un[q.unit].blob ? dtile_y(gB, baseB, q.unit * rb + nl + e, q.slot) : 0.f;
+              if (F == kFmtNv) y *= un[q.unit].ts[2];
               acc = fmaf(q.w, y, acc);
             }
             for (int s2 = 0; s2 < S; s2++) {
               const int u = na + s2;
-              acc += un[u].blob ? dtile_y(gB, baseB, u * rb + nl + e, t) : 0.f;
+              float y = un[u].blob ? dtile_y(gB, baseB, u * rb + nl + e, t) : 0.f;
+              if (F == kFmtNv) y *= un[u].ts[2];
+              acc += y;
             }
             o[e] = acc;
           }
@@ -513,20 +500,20 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers) {
+FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers, int fmt) {
   FlowGeom fg{};
   if (T < 1 || T > 2 || n_layers < 1 || n_layers > 127) return fg;
-  const Gv gA = make_gv(H, I, 2);
+  const Gv gA = make_gv(H, I, 2, fmt);
   if (!gv_ok(gA, I)) return fg;
-  const Gv l = make_gv(I, 1 << 30, 1);
+  const Gv l = make_gv(I, 1 << 30, 1, fmt);
   if (l.rsets <= 0 || I % 128) return fg;
   const int P = T * k, NH = P + S * T, umax = std::min(E, P) + S;
   if (umax > 255) return fg;
   // down-tile rows over all units: up to 256, and about 64 KB of codes
-  int rows_cap = std::min(256, (int)(65536 / (I / 2)));
+  int rows_cap = std::min(256, (int)(65536 / l.rowb));
   rows_cap &= ~1;
   if (rows_cap < 2 * umax) rows_cap = 2 * umax;
-  const Gv gB = make_gd(I, rows_cap, NH);
+  const Gv gB = make_gd(I, rows_cap, NH, fmt);
   const size_t smem = round128(gA.total) + gB.total + sizeof(FlowHdr) + (size_t)n_layers * flow_layer_bytes(umax, P);
   fg.rows_cap = rows_cap;
   fg.smem = smem;
@@ -535,9 +522,14 @@ FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers) {
 }
 
 cudaError_t launch_dec_flow(const FlowArgs& a, cudaStream_t s) {
-  const FlowGeom fg = flow_geometry(a.H, a.I, a.T, a.k, a.n_shared, a.E, a.n_layers);
+  const int F = a.lay.fmt;
+  const FlowGeom fg = flow_geometry(a.H, a.I, a.T, a.k, a.n_shared, a.E, a.n_layers, F);
   if (!fg.ok || a.rows_cap != fg.rows_cap) return cudaErrorInvalidValue;
-  void (*kern)(FlowArgs) = (a.H == 2048 && a.I == 512) ? k_dec_flow<2048, 512> : k_dec_flow<0, 0>;
+  // the 35B-class shape (hidden 2048, intermediate 512) has its own builds
+  const bool s35 = a.H == 2048 && a.I == 512;
+  void (*kern)(FlowArgs) = F == kFmtNv ? (s35 ? k_dec_flow<2048, 512, kFmtNv> : k_dec_flow<0, 0, kFmtNv>)
+                           : F == kFmtBf16 ? (s35 ? k_dec_flow<2048, 512, kFmtBf16> : k_dec_flow<0, 0, kFmtBf16>)
+                                           : (s35 ? k_dec_flow<2048, 512, kFmtMx> : k_dec_flow<0, 0, kFmtMx>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fg.smem);
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 0, occ = 0;

@@ -274,13 +274,23 @@ static ft_status check_desc(const ft_model_desc* d) {
   if (d->n_shared < 0 || d->n_shared > 1) return fail(FT_ERR_INVALID, "n_shared %d not 0 or 1", d->n_shared);
   if (d->cache_budget_bytes < 0) return fail(FT_ERR_INVALID, "negative cache budget");
   if (d->max_tokens <= 0) return fail(FT_ERR_INVALID, "max_tokens %d", d->max_tokens);
-  if (d->reserved != 0) return fail(FT_ERR_INVALID, "reserved field %d is not 0", d->reserved);
+  if (d->weight_format < FT_FMT_MXFP4 || d->weight_format > FT_FMT_BF16)
+    return fail(FT_ERR_INVALID, "weight_format %d is not FT_FMT_MXFP4, FT_FMT_NVFP4 or FT_FMT_BF16", d->weight_format);
   return FT_OK;
 }
 
 extern "C" int64_t ft_blob_stride(int32_t hidden, int32_t inter) {
   if (hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return -1;
   return blob_layout(hidden, inter).stride;
+}
+
+extern "C" ft_status ft_blob_layout_format(int32_t hidden, int32_t inter, int32_t fmt, int64_t out[9]) {
+  if (!out || hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return fail(FT_ERR_INVALID, "bad shape");
+  if (fmt < FT_FMT_MXFP4 || fmt > FT_FMT_BF16) return fail(FT_ERR_INVALID, "bad weight format %d", fmt);
+  BlobLayout b = blob_layout(hidden, inter, fmt);
+  int64_t v[9] = {b.wg, b.wu, b.wd, b.wg_sf, b.wu_sf, b.wd_sf, b.used, b.stride, b.ts};
+  memcpy(out, v, sizeof v);
+  return FT_OK;
 }
 
 extern "C" ft_status ft_blob_layout(int32_t hidden, int32_t inter, int64_t out[8]) {
@@ -356,7 +366,7 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
   ft_ctx* c = new ft_ctx();
   c->d = *desc;
   const int H = desc->hidden, I = desc->inter, E = desc->n_experts, k = desc->top_k, L = desc->n_layers;
-  c->lay = blob_layout(H, I);
+  c->lay = blob_layout(H, I, desc->weight_format);
   c->stride = c->lay.stride;
   c->n_blobs = E + desc->n_shared;
   c->max_tokens = desc->max_tokens;
@@ -670,12 +680,12 @@ extern "C" ft_status ft_fp4_mma_probe(int64_t iters, float* sink, int32_t* statu
 }
 
 extern "C" ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
-                                      int32_t n_experts, int32_t n_layers, int64_t out[3]) {
+                                      int32_t n_experts, int32_t n_layers, int32_t weight_format, int64_t out[3]) {
   if (!out) return fail(FT_ERR_INVALID, "out is NULL");
   if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128 || top_k <= 0 || top_k > 16 || n_experts <= 0 ||
-      n_shared < 0 || n_shared > 1 || T <= 0 || n_layers <= 0)
+      n_shared < 0 || n_shared > 1 || T <= 0 || n_layers <= 0 || weight_format < 0 || weight_format > 2)
     return fail(FT_ERR_INVALID, "bad shape");
-  const FlowGeom fg = flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers);
+  const FlowGeom fg = flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, weight_format);
   out[0] = fg.ok ? 1 : 0;
   out[1] = fg.rows_cap;
   out[2] = (int64_t)fg.smem;
@@ -1133,9 +1143,11 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   const bool mx = (flags & FT_ACT_MXFP4) != 0;
   if (mx && (c->d.hidden % 256 || c->d.inter % 256))
     return fail(FT_ERR_INVALID, "the MXFP4 prefill path needs hidden and inter to be multiples of 256");
+  if (mx && c->d.weight_format != FT_FMT_MXFP4)
+    return fail(FT_ERR_INVALID, "the prefill path (FT_ACT_MXFP4) takes MXFP4 weights only");
   if (!mx && T > c->decode_max_t)
     return fail(FT_ERR_INVALID, "decode GEMV path takes T <= %d (use FT_ACT_MXFP4 for prefill)", c->decode_max_t);
-  if (!mx && !decode_supported(c->d.hidden, c->d.inter))
+  if (!mx && !decode_supported(c->d.hidden, c->d.inter, c->d.weight_format))
     return fail(FT_ERR_INVALID, "decode GEMV path takes hidden and inter up to 16384 (use FT_ACT_MXFP4)");
   if (T == 0) return FT_OK;
   cudaStream_t s = (cudaStream_t)stream;
@@ -1392,7 +1404,7 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   if (n_layers <= 0 || first_layer < 0 || first_layer + n_layers > c->d.n_layers)
     return fail(FT_ERR_INVALID, "layers [%d, %d) outside [0, %d)", first_layer, first_layer + n_layers, c->d.n_layers);
   if (T < 0 || T > c->decode_max_t) return fail(FT_ERR_INVALID, "T=%lld outside [0, %d]", (long long)T, c->decode_max_t);
-  if (!decode_supported(c->d.hidden, c->d.inter))
+  if (!decode_supported(c->d.hidden, c->d.inter, c->d.weight_format))
     return fail(FT_ERR_INVALID, "decode kernels take hidden and inter up to 16384");
   if (flags & FT_ACT_MXFP4) return fail(FT_ERR_INVALID, "the stacked forward is the decode path (FT_ACT_BF16)");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
@@ -1406,9 +1418,11 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   // one or two tokens: the dataflow kernel (tagged h and x, down tiles over
   // every unit); else, or with FT_STACK_COUNTERS, the counter-synchronised
   // persistent kernel; else two kernels per layer
-  const FlowGeom fg = flow_geometry(H, I, Ti, c->d.top_k, c->d.n_shared, c->d.n_experts, n_layers);
+  const FlowGeom fg = flow_geometry(H, I, Ti, c->d.top_k, c->d.n_shared, c->d.n_experts, n_layers, c->d.weight_format);
   const bool flow = !layerwise && !(flags & FT_STACK_COUNTERS) && c->d_tagged != nullptr && fg.ok;
-  const bool persistent = !layerwise && !flow && c->d_sync != nullptr && stack_supported(H, I, n_layers);
+  // the counter-synchronised kernel computes MXFP4 weights only
+  const bool persistent = !layerwise && !flow && c->d_sync != nullptr && c->d.weight_format == FT_FMT_MXFP4 &&
+                          stack_supported(H, I, n_layers);
   // with one or two tokens the counter-synchronised kernel folds the combine
   // into the next layer and hands h over tagged (the tag holds the layer in 7 bits)
   const bool fused = persistent && Ti <= 2 && n_layers <= 128;

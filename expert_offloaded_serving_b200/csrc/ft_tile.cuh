@@ -47,11 +47,23 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // chunks' values: the lanes of a group add theirs with xor shuffles, then the
 // parts are added in ascending order through shared memory.
 //
+// Other weight formats (fmt):
+//   NVFP4  the same codes; a chunk has two E4M3 scales (16 elements each),
+//          so its two halves keep separate sums, each times its scale; the
+//          matrix's fp32 scale multiplies a row's value once, after the
+//          reduction (by the caller).
+//   BF16   a chunk is 32 bf16 weights (64 bytes); activations stay fp32 in
+//          shared memory (no re-encoding: x and h enter exactly); each weight
+//          widens to fp32 exactly and the products are summed by packed fp32
+//          fused multiply-adds (fma.rn.f32x2) into two accumulators.
+//
 // Shared memory, from the tile's base:
-//   codes  [nmat][R][K/2]        as in global memory (16-byte cp.async copies)
-//   scales [nmat][R][K/128]      words of four blocks' UE8M0 bytes
+//   codes  [nmat][R][rowb]       as in global memory (rowb = K/2, or 2K for BF16)
+//   scales [nmat][R][atoms]      words of four scale bytes (K/128 words for
+//                                MXFP4, K/64 for NVFP4, none for BF16)
 //   xh     [kMT][4][K/32] x 16 B  activations, f16: quad i of chunk c at [t][i][c]
-//   xinv   [kMT][K/32]           inverse block factors
+//          (BF16: [kMT][8][K/32] x 16 B of fp32)
+//   xinv   [kMT][K/32]           inverse block factors (not for BF16)
 //   red    [parts][nmat][R][kMT] partial sums
 // ---------------------------------------------------------------------------
 constexpr int kMT = 2;                      // tokens per pass over the tile
@@ -63,32 +75,36 @@ struct Gv {
   int K, chunks, atoms;
   int lpr, rpw, parts, rsets, groups;
   int R, rlog, nmat;  // rows per tile, a power of two (R = 1 << rlog)
+  int fmt, rowb;      // weight format, bytes of a row's codes
   size_t codes, scales, xh, xinv, red, total;
 };
 
-__host__ __device__ inline Gv make_gv(int K, int rows, int nmat) {
+__host__ __device__ inline Gv make_gv(int K, int rows, int nmat, int fmt = kFmtMx) {
   Gv g;
   g.K = K;
   g.nmat = nmat;
+  g.fmt = fmt;
+  g.rowb = fmt == kFmtBf16 ? 2 * K : K / 2;
   g.chunks = K / 32;
-  g.atoms = K / 128;
+  g.atoms = fmt == kFmtMx ? K / 128 : fmt == kFmtNv ? K / 64 : 0;
   g.lpr = 1;
   while (g.lpr < 32 && g.lpr < g.chunks) g.lpr <<= 1;
   g.rpw = 32 / g.lpr;
   g.parts = (g.chunks + g.lpr - 1) / g.lpr;
   g.rsets = kWarps / g.parts;  // 0 for K > 16384: not supported
   g.groups = g.rsets * g.rpw;
+  const int rmin = fmt == kFmtBf16 ? 2 : 8;
   int R = 128;
-  while (R > 8 && (size_t)R * nmat * K / 2 > kTileBytes) R >>= 1;
+  while (R > rmin && (size_t)R * nmat * g.rowb > kTileBytes) R >>= 1;
   if (R > rows) R = rows;
   for (;;) {
     g.codes = 0;
-    g.scales = (size_t)nmat * R * K / 2;
+    g.scales = (size_t)nmat * R * g.rowb;
     g.xh = g.scales + (size_t)nmat * R * g.atoms * 4;
-    g.xinv = g.xh + (size_t)kMT * K * 2;
-    g.red = g.xinv + (((size_t)kMT * g.chunks * 4 + 15) & ~(size_t)15);
+    g.xinv = g.xh + (size_t)kMT * K * (fmt == kFmtBf16 ? 4 : 2);
+    g.red = g.xinv + (fmt == kFmtBf16 ? 0 : (((size_t)kMT * g.chunks * 4 + 15) & ~(size_t)15));
     g.total = g.red + (size_t)g.parts * nmat * R * kMT * 4;
-    if (g.total <= kSmemLimit || R <= 8) break;
+    if (g.total <= kSmemLimit || R <= rmin) break;
     R >>= 1;
   }
   g.R = R;
@@ -126,6 +142,7 @@ __device__ __forceinline__ LaneMap lane_map(const Gv& g) {
 // Scale words of rows [row0, row0 + R) of matrix `mat` (scale region sc_g),
 // one 4-byte cp.async each.
 __device__ __forceinline__ void stage_scales(const Gv& g, uint8_t* base, int mat, const uint8_t* sc_g, int row0) {
+  if (g.atoms == 0) return;  // BF16: no scales
   uint32_t* sd = reinterpret_cast<uint32_t*>(base + g.scales) + (size_t)mat * g.R * g.atoms;
   for (int i = threadIdx.x; i < g.R * g.atoms; i += kGemvThreads) {
     const int r = i / g.atoms, at = i - r * g.atoms;
@@ -134,20 +151,33 @@ __device__ __forceinline__ void stage_scales(const Gv& g, uint8_t* base, int mat
 }
 
 // Stage rows [row0, row0 + R) of matrix `mat` (codes at codes_g, row pitch
-// K/2; scale region sc_g) into the tile with cp.async.
+// rowb; scale region sc_g) into the tile with cp.async.
 __device__ __forceinline__ void stage_mat(const Gv& g, uint8_t* base, int mat, const uint8_t* codes_g,
                                           const uint8_t* sc_g, int row0) {
-  uint8_t* dst = base + g.codes + (size_t)mat * g.R * (g.K / 2);
-  const uint8_t* src = codes_g + (size_t)row0 * (g.K / 2);
-  const int n16 = g.R * g.chunks;
+  uint8_t* dst = base + g.codes + (size_t)mat * g.R * g.rowb;
+  const uint8_t* src = codes_g + (size_t)row0 * g.rowb;
+  const int n16 = g.R * (g.rowb / 16);
   for (int i = threadIdx.x; i < n16; i += kGemvThreads) cp_async16(dst + (size_t)i * 16, src + (size_t)i * 16);
   stage_scales(g, base, mat, sc_g, row0);
 }
 
+// BF16 weights: 4 consecutive fp32 activations (group q of token t) stored as
+// they are; quad i of chunk c sits at [t][i][c], 8 quads a chunk.
+__device__ __forceinline__ void store4f(const Gv& g, uint8_t* base, int t, int q, const float (&v)[4]) {
+  float4* xf = reinterpret_cast<float4*>(base + g.xh);
+  const int c = q >> 3, i = q & 7;
+  xf[((size_t)t * 8 + i) * g.chunks + c] = make_float4(v[0], v[1], v[2], v[3]);
+}
+
 // Encode 4 consecutive activations v (group q of token t) into the tile's f16
 // activations; the 8 lanes of a 32-element block agree on its factor by
-// shuffles, so all 32 lanes of the warp must call this together.
+// shuffles, so all 32 lanes of the warp must call this together.  (BF16
+// weights: stored as fp32, see store4f.)
 __device__ __forceinline__ void encode4(const Gv& g, uint8_t* base, int t, int q, const float (&v)[4]) {
+  if (g.fmt == kFmtBf16) {
+    store4f(g, base, t, q, v);
+    return;
+  }
   uint2* xh = reinterpret_cast<uint2*>(base + g.xh);
   float* xinv = reinterpret_cast<float*>(base + g.xinv);
   uint32_t e = 0;
@@ -221,9 +251,26 @@ __device__ __forceinline__ float fma_f16x2(uint32_t w, uint32_t x, float acc) {
 // staged row `row` (rows of all matrices of the tile counted in order).
 __device__ __forceinline__ void tile_chunk(const Gv& g, const uint8_t* codes, const uint32_t* sc, int row, int c,
                                            uint4& q, float& s) {
-  q = *reinterpret_cast<const uint4*>(codes + (size_t)row * (g.K / 2) + c * 16);
+  q = *reinterpret_cast<const uint4*>(codes + (size_t)row * g.rowb + c * 16);
   const uint32_t sw = sc[(size_t)row * g.atoms + (c >> 2)];
   s = ue8m0_to_f32((sw >> (8 * (c & 3))) & 0xffu);
+}
+
+// NVFP4: the codes of chunk c and the E4M3 scales of its two 16-element
+// halves (adjacent bytes of one scale word: blocks 2c and 2c + 1).
+__device__ __forceinline__ void tile_chunk_nv(const Gv& g, const uint8_t* codes, const uint32_t* sc, int row, int c,
+                                              uint4& q, float& s0, float& s1) {
+  q = *reinterpret_cast<const uint4*>(codes + (size_t)row * g.rowb + c * 16);
+  const uint32_t sw = sc[(size_t)row * g.atoms + (c >> 1)] >> (16 * (c & 1));
+  s0 = e4m3_to_f32(sw & 0xffu);
+  s1 = e4m3_to_f32((sw >> 8) & 0xffu);
+}
+
+// BF16: the 32 weights (64 bytes) of chunk c of staged row `row`.
+__device__ __forceinline__ void tile_chunk_bf16(const Gv& g, const uint8_t* codes, int row, int c, uint4 (&q)[4]) {
+  const uint4* p = reinterpret_cast<const uint4*>(codes + (size_t)row * g.rowb + c * 64);
+#pragma unroll
+  for (int i = 0; i < 4; i++) q[i] = p[i];
 }
 
 // Dot of one chunk of 32 e2m1 codes with NT tokens' f16 activations x[t][i]
@@ -246,6 +293,53 @@ __device__ __forceinline__ void chunk_dot(uint4 q, const uint32_t (&x)[kMT][16],
   }
 #pragma unroll
   for (int t = 0; t < NT; t++) d[t] = acc[t][0] + acc[t][1];
+}
+
+// NVFP4: the dot of a chunk's two 16-element halves, kept apart (words 0-1
+// and 2-3 of the codes), each a chain of fused multiply-adds in fixed order.
+template <int NT>
+__device__ __forceinline__ void chunk_dot_nv(uint4 q, const uint32_t (&x)[kMT][16], float* d0, float* d1) {
+  float acc[NT][2];
+#pragma unroll
+  for (int t = 0; t < NT; t++) acc[t][0] = acc[t][1] = 0.f;
+  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int wv = 0; wv < 4; wv++) {
+    uint32_t h[4];
+    e2m1x8_to_f16x8(qs[wv], h);
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+#pragma unroll
+      for (int t = 0; t < NT; t++) acc[t][wv >> 1] = fma_f16x2(h[j], x[t][4 * wv + j], acc[t][wv >> 1]);
+  }
+#pragma unroll
+  for (int t = 0; t < NT; t++) {
+    d0[t] = acc[t][0];
+    d1[t] = acc[t][1];
+  }
+}
+
+// BF16: the dot of a chunk's 32 weights with NT tokens' fp32 activations
+// xf[t][0..31]: each bf16 widens exactly to fp32, pairs meet their
+// activations in packed fp32 fused multiply-adds (two accumulator lanes).
+template <int NT>
+__device__ __forceinline__ void chunk_dot_bf16(const uint4 (&q)[4], const float (&xf)[kMT][32], float* d) {
+  float2 acc[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++) acc[t] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const uint32_t ws[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const float2 w = make_float2(__uint_as_float(ws[j] << 16), __uint_as_float(ws[j] & 0xffff0000u));
+      const int e = 8 * i + 2 * j;
+#pragma unroll
+      for (int t = 0; t < NT; t++) acc[t] = ffma2(w, make_float2(xf[t][e], xf[t][e + 1]), acc[t]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NT; t++) d[t] = acc[t].x + acc[t].y;
 }
 
 // Sum over the lpr lanes of a group of RU rows' partial sums v[u][t] (RU = 1,
@@ -285,11 +379,83 @@ __device__ __forceinline__ int group_reduce(float (&v)[4][kMT], int lpr) {
   return row;
 }
 
+// Value of chunk c of staged row `row` for NT tokens, before the row's
+// reduction over its lanes: MXFP4 chunk sum x (scale x inverse factor);
+// NVFP4 (half sum x scale, added) x inverse factor; BF16 the fp32 dot.
+template <int NT, int F>
+__device__ __forceinline__ void chunk_value(const Gv& g, const uint8_t* codes, const uint32_t* sc, int row, int c,
+                                            const uint32_t (&x)[kMT][16], const float (&xi)[kMT],
+                                            const float (&xf)[kMT][32], float* v) {
+  if constexpr (F == kFmtMx) {
+    uint4 q;
+    float s;
+    tile_chunk(g, codes, sc, row, c, q, s);
+    float d[NT];
+    chunk_dot<NT>(q, x, d);
+#pragma unroll
+    for (int t = 0; t < NT; t++) v[t] = d[t] * (s * xi[t]);
+  } else if constexpr (F == kFmtNv) {
+    uint4 q;
+    float s0, s1;
+    tile_chunk_nv(g, codes, sc, row, c, q, s0, s1);
+    float d0[NT], d1[NT];
+    chunk_dot_nv<NT>(q, x, d0, d1);
+#pragma unroll
+    for (int t = 0; t < NT; t++) v[t] = fmaf(d0[t], s0, d1[t] * s1) * xi[t];
+  } else {
+    uint4 q[4];
+    tile_chunk_bf16(g, codes, row, c, q);
+    chunk_dot_bf16<NT>(q, xf, v);
+  }
+}
+
+// Activations of staged row srow, chunk c, into one token slot of the lane's
+// registers (f16 pairs and the inverse factor; fp32 for BF16 weights).
+template <int F>
+__device__ __forceinline__ void load_act(const Gv& g, const uint8_t* base, int srow, int c, uint32_t (&x)[16],
+                                         float& xi, float (&xf)[32]) {
+  if constexpr (F == kFmtBf16) {
+    const float4* p = reinterpret_cast<const float4*>(base + g.xh);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float4 f = p[((size_t)srow * 8 + i) * g.chunks + c];
+      xf[4 * i] = f.x;
+      xf[4 * i + 1] = f.y;
+      xf[4 * i + 2] = f.z;
+      xf[4 * i + 3] = f.w;
+    }
+  } else {
+    const uint4* xh = reinterpret_cast<const uint4*>(base + g.xh);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const uint4 u = xh[(size_t)srow * (g.K / 8) + (size_t)i * g.chunks + c];
+      x[4 * i] = u.x;
+      x[4 * i + 1] = u.y;
+      x[4 * i + 2] = u.z;
+      x[4 * i + 3] = u.w;
+    }
+    xi = reinterpret_cast<const float*>(base + g.xinv)[srow * g.chunks + c];
+  }
+}
+
+template <int F>
+__device__ __forceinline__ void zero_act(uint32_t (&x)[16], float& xi, float (&xf)[32]) {
+  if constexpr (F == kFmtBf16) {
+#pragma unroll
+    for (int i = 0; i < 32; i++) xf[i] = 0.f;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; i++) x[i] = 0u;
+    xi = 0.f;
+  }
+}
+
 // Partial sums of the staged tile's rows for NT tokens into red.  Lane group
 // grp takes rows grp + j*groups, RU of them at a time.
-template <int RU, int NT>
+template <int RU, int NT, int F>
 __device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8_t* base,
-                                            const uint32_t (&x)[kMT][16], const float (&xi)[kMT]) {
+                                            const uint32_t (&x)[kMT][16], const float (&xi)[kMT],
+                                            const float (&xf)[kMT][32]) {
   const uint8_t* codes = base + g.codes;
   const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
   float* red = reinterpret_cast<float*>(base + g.red);
@@ -303,16 +469,7 @@ __device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8
 #pragma unroll
       for (int u = 0; u < RU; u++) {
         v[u][0] = v[u][1] = 0.f;
-        if (cv) {
-          const int row = mat * g.R + m.grp + (j0 + u) * g.groups;
-          uint4 q;
-          float s;
-          tile_chunk(g, codes, sc, row, m.c, q, s);
-          float d[NT];
-          chunk_dot<NT>(q, x, d);
-#pragma unroll
-          for (int t = 0; t < NT; t++) v[u][t] = d[t] * (s * xi[t]);
-        }
+        if (cv) chunk_value<NT, F>(g, codes, sc, mat * g.R + m.grp + (j0 + u) * g.groups, m.c, x, xi, xf, v[u]);
       }
       const int u = group_reduce<RU, NT>(v, g.lpr);
       if (((threadIdx.x & 31) & lmask) == 0) {
@@ -326,47 +483,32 @@ __device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8
 }
 
 // Partial sums of every row of the staged tile for n (<= kMT) tokens into red.
+template <int F = kFmtMx>
 __device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t* base, int n) {
   if (!m.on) return;
   uint32_t x[kMT][16];
   float xi[kMT] = {0.f, 0.f};
-  if (m.c < g.chunks) {
-    const uint4* xh = reinterpret_cast<const uint4*>(base + g.xh);
-    const float* xinv = reinterpret_cast<const float*>(base + g.xinv);
+  float xf[kMT][32];
 #pragma unroll
-    for (int t = 0; t < kMT; t++) {
-      if (t < n) {
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-          const uint4 u = xh[(size_t)t * (g.K / 8) + (size_t)i * g.chunks + m.c];
-          x[t][4 * i] = u.x;
-          x[t][4 * i + 1] = u.y;
-          x[t][4 * i + 2] = u.z;
-          x[t][4 * i + 3] = u.w;
-        }
-        xi[t] = xinv[t * g.chunks + m.c];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; i++) x[t][i] = 0u;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int t = 0; t < kMT; t++)
-#pragma unroll
-      for (int i = 0; i < 16; i++) x[t][i] = 0u;
+  for (int t = 0; t < kMT; t++) {
+    if (m.c < g.chunks && t < n) load_act<F>(g, base, t, m.c, x[t], xi[t], xf[t]);
+    else zero_act<F>(x[t], xi[t], xf[t]);
   }
   // rows per lane group and matrix; groups of 4 or 2 when they divide it
+  // (BF16 holds 32 fp32 activations per token: at most 2 rows at a time, so
+  // that the registers suffice; the reduction tree does not depend on it)
   const int per = g.R % g.groups == 0 ? g.R / g.groups : 0;
-  const int ru = (per % 4 == 0 && per > 0 && g.lpr >= 4) ? 4 : (per % 2 == 0 && per > 0 && g.lpr >= 2) ? 2 : 1;
+  const int ru = (F != kFmtBf16 && per % 4 == 0 && per > 0 && g.lpr >= 4) ? 4
+                 : (per % 2 == 0 && per > 0 && g.lpr >= 2)                ? 2
+                                                                           : 1;
   if (n > 1) {
-    if (ru == 4) tile_dots_t<4, 2>(g, m, base, x, xi);
-    else if (ru == 2) tile_dots_t<2, 2>(g, m, base, x, xi);
-    else tile_dots_t<1, 2>(g, m, base, x, xi);
+    if (ru == 4) tile_dots_t<4, 2, F>(g, m, base, x, xi, xf);
+    else if (ru == 2) tile_dots_t<2, 2, F>(g, m, base, x, xi, xf);
+    else tile_dots_t<1, 2, F>(g, m, base, x, xi, xf);
   } else {
-    if (ru == 4) tile_dots_t<4, 1>(g, m, base, x, xi);
-    else if (ru == 2) tile_dots_t<2, 1>(g, m, base, x, xi);
-    else tile_dots_t<1, 1>(g, m, base, x, xi);
+    if (ru == 4) tile_dots_t<4, 1, F>(g, m, base, x, xi, xf);
+    else if (ru == 2) tile_dots_t<2, 1, F>(g, m, base, x, xi, xf);
+    else tile_dots_t<1, 1, F>(g, m, base, x, xi, xf);
   }
 }
 

@@ -75,8 +75,23 @@ typedef struct {
   int32_t n_shared;           /* always-on shared experts per layer (weight 1), 0 or 1 */
   int64_t cache_budget_bytes; /* GPU expert-cache budget (0 = no cache) */
   int32_t max_tokens;         /* largest T any forward call passes; sizes scratch */
-  int32_t reserved;           /* must be 0 */
+  int32_t weight_format;      /* FT_FMT_MXFP4 (0), FT_FMT_NVFP4 or FT_FMT_BF16 */
 } ft_model_desc;
+
+/* Expert weight formats ([no] "Hvor raskt kjører modellene?": MXFP4 for
+ * DeepSeek-V4-Flash, BF16 and NVFP4 builds of Qwen3.6-35B-A3B).  Blob layouts
+ * (each matrix K-contiguous, padded to a multiple of 256 bytes):
+ *   MXFP4  as described above (ft_blob_stride);
+ *   NVFP4  the same e2m1 code regions; then E4M3 block scales (one per 16
+ *          elements along K; no infinities, S.1111.111 is NaN) in the same
+ *          128-row x 4-block atoms; then the fp32 scales of Wg, Wu, Wd and 4
+ *          zero bytes.  A weight is code value x block scale x matrix scale.
+ *   BF16   Wg [I][H], Wu [I][H], Wd [H][I] as little-endian bf16.
+ * The decode paths (FT_ACT_BF16) take every format; the prefill path
+ * (FT_ACT_MXFP4) takes MXFP4 weights only. */
+#define FT_FMT_MXFP4 0
+#define FT_FMT_NVFP4 1
+#define FT_FMT_BF16  2
 
 /* forward / route flags */
 #define FT_ROUTE_RENORM 1u    /* renormalise the k softmax weights to sum 1 (default on) */
@@ -120,6 +135,11 @@ FT_API int64_t ft_blob_stride(int32_t hidden, int32_t inter);
 /* Byte offsets of the regions of a blob: out[0..7] = Wg, Wu, Wd codes,
  * Wg, Wu, Wd scales, used bytes, stride.  FT_ERR_INVALID on a bad shape. */
 FT_API ft_status ft_blob_layout(int32_t hidden, int32_t inter, int64_t out[8]);
+
+/* The same for weight format fmt (FT_FMT_*): out[0..7] as ft_blob_layout
+ * (for BF16 the scale offsets equal the used bytes), out[8] the NVFP4 matrix
+ * scales' offset (-1 otherwise).  FT_ERR_INVALID on a bad shape or format. */
+FT_API ft_status ft_blob_layout_format(int32_t hidden, int32_t inter, int32_t fmt, int64_t out[9]);
 
 /* Message of the last error on this thread ("" if none). */
 FT_API const char* ft_last_error(void);
@@ -321,11 +341,11 @@ FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_lay
 
 /* Geometry of the dataflow decode kernel that ft_moe_stack_forward runs for
  * one or two tokens (host only, no device needed): out[0] = 1 if it takes
- * this shape, batch T and stack depth (else the counter-synchronised or the
- * per-layer kernels run), out[1] = rows of a down tile over all units,
+ * this shape, batch T, stack depth and weight format (else the
+ * counter-synchronised or the per-layer kernels run), out[1] = rows of a down tile over all units,
  * out[2] = shared memory of a CTA in bytes.  FT_ERR_INVALID on a bad shape. */
 FT_API ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
-                                  int32_t n_experts, int32_t n_layers, int64_t out[3]);
+                                  int32_t n_experts, int32_t n_layers, int32_t weight_format, int64_t out[3]);
 
 /* Failure injection for tests: none of these fault or hang a GPU.
  *

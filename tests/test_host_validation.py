@@ -23,16 +23,17 @@ POOL, X, OUT, LG, WR = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000
     (dict(n_shared=2), "n_shared"),
     (dict(cache_budget_bytes=-1), "budget"),
     (dict(max_tokens=0), "max_tokens"),
-    (dict(reserved=1), "reserved"),
+    (dict(weight_format=3), "weight_format"),
+    (dict(weight_format=-1), "weight_format"),
 ])
 def test_create_refuses_each_bad_descriptor_field(desc, what):
     base = dict(hidden=256, inter=128, n_experts=16, top_k=2, n_layers=1, n_shared=0, cache_budget_bytes=0,
                 max_tokens=16)
     desc = dict(desc)
-    reserved = desc.pop("reserved", 0)
+    fmt = desc.pop("weight_format", 0)
     base.update(desc)
     d = ft.make_desc(**base)
-    d.reserved = reserved
+    d.weight_format = fmt
     with pytest.raises(ft.FtError) as e:
         ft.ft_create(d)
     assert e.value.status == ft.FT_ERR_INVALID
