@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     ap.add_argument("--layerwise", action="store_true",
                     help="decode with two kernels per layer instead of a persistent stack kernel")
+    ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4", "bf16"],
+                    help="expert weight format of the decode stack")
     ap.add_argument("--counters", action="store_true",
                     help="decode with the counter-synchronised persistent kernel instead of the dataflow kernel")
     return ap.parse_args()
@@ -201,13 +203,15 @@ def run_ours(args, world, rank):
     import synth.gpu
 
     T = args.tokens
-    lay = ft.ft_blob_layout(H, I)
+    fmt = getattr(args, "format", "mxfp4")
+    fcode = {"mxfp4": ft.FT_FMT_MXFP4, "nvfp4": ft.FT_FMT_NVFP4, "bf16": ft.FT_FMT_BF16}[fmt]
+    lay = ft.ft_blob_layout_format(H, I, fcode)
     used = lay["used"]
-    gu_bytes = lay["wd"] + (lay["wd_sf"] - lay["wg_sf"])          # Wg + Wu codes and scales
-    d_bytes = (lay["wd"] - lay["wu"]) + (lay["used"] - lay["wd_sf"])  # Wd codes and scales
-    pools = [synth.gpu.layer_pool(H, I, E + S_SHARED, SEED, layer) for layer in range(L)]
+    gu_bytes = (lay["wd"] - lay["wg"]) + (lay["wd_sf"] - lay["wg_sf"])   # Wg + Wu codes and scales
+    d_bytes = used - gu_bytes                                            # Wd codes, scales (and matrix scales)
+    pools = [synth.gpu.layer_pool(H, I, E + S_SHARED, SEED, layer, fmt=fmt) for layer in range(L)]
     torch.cuda.synchronize()
-    ctx = ft.ft_create(ft.make_desc(H, I, E, K_TOP, L, S_SHARED, 0, T), None, pools)
+    ctx = ft.ft_create(ft.make_desc(H, I, E, K_TOP, L, S_SHARED, 0, T, weight_format=fcode), None, pools)
     sets = decode_routing(T)
     logits_all = torch.from_numpy(decode_logits(sets)).cuda()        # [P][L][T][E]
     logits_buf = torch.empty_like(logits_all[0])
@@ -316,6 +320,8 @@ def run_ours(args, world, rank):
                   "d2h_bytes_per_step": int(host_out.numel() * 2)}
     del g, g2, final, final2
     ft.ft_destroy(ctx)
+    del pools
+    torch.cuda.empty_cache()
     return res
 
 
@@ -716,6 +722,28 @@ def measure_misses(tokens=512, layers=43, resize_at=(170, 340)):
                         "saved_ms": serial_ms - total_ms}}
 
 
+def measure_decode_formats(args, pk, steps=300, warmup=20):
+    """The same 35B-class decode stack at batch 1 with NVFP4 and with BF16
+    experts (the pages' other formats of this model): tokens/s, the
+    persistent kernel's bandwidth on the format's algorithmic bytes (whole
+    blobs of the routed and shared experts) and its fraction of the HBM
+    peak."""
+    import copy
+    out = {}
+    for fmt in ("nvfp4", "bf16"):
+        a = copy.copy(args)
+        a.tokens, a.format, a.steps, a.warmup = 1, fmt, steps, warmup
+        res = run_ours(a, 1, 0)
+        o = {"workload": workload_config(1, fmt=fmt)["workload"], "tok_s": res["tok_s"], "ms_per_step": res["ms"] / steps,
+             "e2e_tok_s": res["e2e"]["value"], "algorithmic_bytes_per_step": res["stack_bytes"], "clocks": res["clocks"]}
+        st = res["kernels"].get("dec_stack")
+        if st:
+            gbs = res["stack_bytes"] / (st["us_avg"] * 1e-6) / 1e9
+            o.update(kernel_us=st["us_avg"], kernel_gbs=gbs, kernel_frac=gbs / pk["hbm"])
+        out[fmt] = o
+    return out
+
+
 def measure_decode_batch(args, T, pk):
     """The same 35B-class decode stack at batch T (the workload's other batch
     size): tokens/s, ms per step, end-to-end tokens/s and the persistent
@@ -743,10 +771,14 @@ def decode_kernel_name(T, layerwise=False, counters=False):
     return "persistent stack kernel, dataflow (tagged hand-overs)"
 
 
-def workload_config(T, layerwise=False, counters=False):
+FORMAT_NAMES = {"mxfp4": "MXFP4 (e2m1 + UE8M0/32)", "nvfp4": "NVFP4 (e2m1 + E4M3/16 + fp32 per matrix)",
+                "bf16": "BF16"}
+
+
+def workload_config(T, layerwise=False, counters=False, fmt="mxfp4"):
     return {"decode_kernels": decode_kernel_name(T, layerwise, counters),
             "workload": f"35B-A3B-class MoE decode stack: hidden {H}, {E} routed experts top-{K_TOP} + {S_SHARED} shared, "
-                        f"intermediate {I}, {L} layers, MXFP4 (e2m1 + UE8M0/32) weights resident in HBM, "
+                        f"intermediate {I}, {L} layers, {FORMAT_NAMES[fmt]} weights resident in HBM, "
                         f"batch {T}, Zipf(1.1) routing traces with 0.6 adjacent-token reuse",
             "global_batch": T, "layers": L, "l2": "inputs larger than L2 (~600 MB of distinct expert weights per step)"}
 
@@ -806,7 +838,7 @@ def main():
     line = {"metric": METRIC, "value": res["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(T, args.layerwise, args.counters),
+            "config": workload_config(T, args.layerwise, args.counters, args.format),
             "roofline": {"bound": "hbm", "kernel": rk, "achieved": rk_gbs, "peak": pk["hbm"],
                          "peak_source": pk["src"], "unit": "GB/s", "frac": rk_gbs / pk["hbm"], "traffic": rk_traffic,
                          "algorithmic_bytes_per_launch": rk_bytes},
@@ -830,6 +862,11 @@ def main():
                 line["decode_batch4"] = measure_decode_batch(args, 4, pk)
             except Exception as ex:
                 line["decode_batch4"] = {"error": repr(ex)}
+            if args.format == "mxfp4":
+                try:
+                    line["decode_formats"] = measure_decode_formats(args, pk)
+                except Exception as ex:
+                    line["decode_formats"] = {"error": repr(ex)}
     if world == 1:
         cores = host_cores()
         v, done = oracle_tok_s(T, cores)

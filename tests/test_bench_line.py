@@ -14,7 +14,7 @@ STACK_BYTES = 601_620_480.0          # 40 layers x 9 units x 1,671,168 B at batc
 
 
 def fake_decode(args, world, rank):
-    assert world == 1 and args.tokens in (1, 4)
+    assert world == 1 and args.tokens in (1, 4) and args.format in ("mxfp4", "nvfp4", "bf16")
     us = 316.0
     return dict(ms=args.steps * 0.3238, tok_s=1e3 / 0.3238, hbm_gbs=1858.0, step_bytes=STACK_BYTES,
                 launches=2 * args.steps, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 40},
@@ -54,6 +54,9 @@ def test_contract_keys(line):
     assert line["prefill"] == {"workload": "prefill"} and line["miss"] == {"workload": "miss"}
     b4 = line["decode_batch4"]
     assert "batch 4" in b4["workload"] and b4["tok_s"] > 0 and 0 < b4["kernel_frac"] < 1.5
+    fm = line["decode_formats"]
+    assert set(fm) == {"nvfp4", "bf16"} and "NVFP4" in fm["nvfp4"]["workload"] and "BF16" in fm["bf16"]["workload"]
+    assert "MXFP4" in line["config"]["workload"]
 
 
 def test_derived_figures(line):

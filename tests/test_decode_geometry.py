@@ -84,3 +84,28 @@ def test_dataflow_kernel_limits():
     assert not ft.ft_flow_geometry(2048, 512, 3, 8, 1, 256, 40)["ok"]
     assert not ft.ft_flow_geometry(2048, 512, 1, 8, 1, 256, 128)["ok"]
     assert ft.ft_flow_geometry(2048, 512, 1, 8, 1, 256, 127)["ok"]
+
+
+@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("T", [1, 2])
+def test_dataflow_kernel_geometry_other_formats(fmt, T):
+    """NVFP4 and BF16 experts at the 35B-class shape (the formats' decode
+    benchmark) fit the dataflow kernel at one and two tokens."""
+    g = ft.ft_flow_geometry(2048, 512, T, 8, 1, 256, 40, fmt)
+    assert g["ok"] and g["smem"] <= OPT_IN_SMEM
+
+
+def test_blob_layout_formats():
+    """Blob sizes of the three formats at the 35B-class shape, from the
+    definitions: MXFP4 3HI(1/2 + 1/32); NVFP4 3HI(1/2 + 1/16) + 16 bytes of
+    matrix scales, padded to 256; BF16 6HI."""
+    H, I = 2048, 512
+    mx = ft.ft_blob_layout_format(H, I, 0)
+    nv = ft.ft_blob_layout_format(H, I, 1)
+    bf = ft.ft_blob_layout_format(H, I, 2)
+    assert mx["stride"] == 3 * H * I * 17 // 32 and mx["ts"] == -1
+    assert nv["ts"] == 3 * H * I * 9 // 16 and nv["used"] == nv["ts"] + 16 and nv["stride"] == nv["used"] + 240
+    assert bf["used"] == bf["stride"] == 6 * H * I
+    import synth
+    assert synth.nvfp4_blob_regions(H, I)["stride"] == nv["stride"]
+    assert synth.bf16_blob_regions(H, I)["stride"] == bf["stride"]
