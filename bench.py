@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 or 4)")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
-    ap.add_argument("--case", default="decode", choices=["decode", "prefill", "miss"],
+    ap.add_argument("--case", default="decode", choices=["decode", "prefill", "miss", "glm"],
                     help="decode: the 35B-class decode stack (default line); prefill / miss: only that measurement")
     ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     ap.add_argument("--layerwise", action="store_true",
@@ -744,6 +744,85 @@ def measure_decode_formats(args, pk, steps=300, warmup=20):
     return out
 
 
+def measure_glm(tokens=256, layers=8, prefill_tokens=2048, reps=3):
+    """GLM-5.2-class slice (hidden 6144, 256 experts top-8, intermediate
+    2048, 20 MB blobs): 8 of the 78 layers with their pools (41 GB) in pinned
+    host memory, a 24 GiB cache (1285 slots), batch-1 decode over a 256-token
+    Zipf(1.1) / 0.6-overlap trace through the cache path (tok/s, miss rate,
+    miss H2D GB/s); and one 2048-token prefill chunk of a resident layer (GEMM
+    TFLOP/s and layer time)."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+    H5, I5, E5, k5, seed = 6144, 2048, 256, 8, 1006
+    stride = ft.ft_blob_stride(H5, I5)
+    budget = (24 * 2 ** 30) // stride * stride
+    hp = host_pools_pageable(H5, I5, E5, seed, layers)
+    sets = np.stack([synth.zipf_trace(seed, l, tokens, E5, k5, 1.1, 0.6) for l in range(layers)], axis=1)
+    lg = torch.from_numpy(np.stack([[synth.logits_for_sets(seed, p * 100 + l, sets[p, l][None], E5)[0]
+                                     for l in range(layers)] for p in range(tokens)])).cuda()
+    x = torch.from_numpy(synth.activations_bf16(seed, 1, 1, H5).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    bufs = [torch.empty_like(x), torch.empty_like(x)]
+    ctx = ft.ft_create(ft.make_desc(H5, I5, E5, k5, layers, 0, budget, 1), hp, None)
+    ft.ft_cache_stats_get(ctx, reset=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    cur = x
+    for p in range(tokens):
+        for l in range(layers):
+            nxt = bufs[(p * layers + l) % 2]
+            ft.ft_moe_layer_forward(ctx, l, cur, 1, None, lg[p, l], nxt, ft.FT_ROUTE_RENORM)
+            cur = nxt
+    b.record()
+    b.synchronize()
+    st = ft.ft_cache_stats_get(ctx)
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    del hp
+    ms = a.elapsed_time(b)
+    lookups = st["hits"] + st["misses"]
+    dec = {"workload": f"GLM-class decode: {layers} of 78 layers, {layers * E5 * stride / 1e9:.1f} GB pool in pinned "
+                       f"host memory, 24 GiB cache ({budget // stride} slots), batch 1, {tokens} tokens",
+           "tok_s_over_these_layers": tokens / (ms * 1e-3), "ms": ms, "miss_rate": st["misses"] / max(lookups, 1),
+           "hits": st["hits"], "misses": st["misses"], "evictions": st["evictions"],
+           "miss_h2d_gbs": st["h2d_bytes"] / (st["h2d_ms"] * 1e-3) / 1e9 if st["h2d_ms"] > 0 else None,
+           "overlap": {"resident_expert_ms": st["hit_ms"], "under_copies_ms": st["overlap_ms"]}}
+    # prefill: one resident layer, one 2048-token chunk through the router GEMV
+    T = prefill_tokens
+    pool = synth.gpu.layer_pool(H5, I5, E5, seed, 0)
+    ctx = ft.ft_create(ft.make_desc(H5, I5, E5, k5, 1, 0, 0, T), None, [pool])
+    xp = torch.from_numpy(synth.activations_bf16(seed, 2, T, H5).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    wr = torch.from_numpy(synth.router_weights(seed, 0, E5, H5)).cuda()
+    out = torch.empty_like(xp)
+    flags = ft.FT_ACT_MXFP4 | ft.FT_ROUTE_RENORM
+    ft.ft_moe_layer_forward(ctx, 0, xp, T, wr, None, out, flags)
+    torch.cuda.synchronize()
+    ft.ft_kernel_timing_enable(ctx, True)
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, xp, T, wr, None, out, flags)
+    kt = ft.ft_kernel_timing_read(ctx)
+    ft.ft_kernel_timing_enable(ctx, False)
+    a.record()
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, xp, T, wr, None, out, flags)
+    b.record()
+    b.synchronize()
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    del pool
+    torch.cuda.empty_cache()
+    flops = 2.0 * T * k5 * 3 * H5 * I5
+    gemm_ms = (kt["gemm_gate_up"][0] + kt["gemm_down"][0]) / reps
+    pre = {"workload": f"GLM-class prefill layer: {T} tokens, router GEMV, weights resident", "flop": flops,
+           "gemm_ms": gemm_ms, "gemm_tflops": flops / (gemm_ms * 1e-3) / 1e12, "layer_ms": a.elapsed_time(b) / reps,
+           "kernels_ms": {k_: v[0] / reps for k_, v in kt.items() if v[1]},
+           "gemm_weight_gbs": E5 * ft.ft_blob_layout(H5, I5)["used"] / (gemm_ms * 1e-3) / 1e9}
+    return {"decode": dec, "prefill": pre}
+
+
 def measure_decode_batch(args, T, pk):
     """The same 35B-class decode stack at batch T (the workload's other batch
     size): tokens/s, ms per step, end-to-end tokens/s and the persistent
@@ -798,7 +877,8 @@ def main():
         world, rank, local = dist_setup(args)
     if args.case != "decode":
         if rank == 0:
-            r = measure_prefill(reps=max(args.steps, 1)) if args.case == "prefill" else measure_misses()
+            r = {"prefill": lambda: measure_prefill(reps=max(args.steps, 1)), "miss": measure_misses,
+                 "glm": measure_glm}[args.case]()
             print(json.dumps({"case": args.case, **r}))
         return
     if args.impl == "reference":
@@ -867,6 +947,10 @@ def main():
                     line["decode_formats"] = measure_decode_formats(args, pk)
                 except Exception as ex:
                     line["decode_formats"] = {"error": repr(ex)}
+        try:
+            line["glm"] = measure_glm()
+        except Exception as ex:
+            line["glm"] = {"error": repr(ex)}
     if world == 1:
         cores = host_cores()
         v, done = oracle_tok_s(T, cores)
