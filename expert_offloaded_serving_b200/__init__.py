@@ -25,7 +25,7 @@ FT_ACT_MXFP4 = 2
 FT_STACK_LAYERWISE = 4
 FT_STACK_COUNTERS = 8
 FT_CACHE_SERIAL = 16
-FT_EV_HIT, FT_EV_MISS, FT_EV_EVICT, FT_EV_MOVE = range(4)
+FT_EV_HIT, FT_EV_MISS, FT_EV_EVICT, FT_EV_MOVE, FT_EV_PREFETCH = range(5)
 
 EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft_destroy", "ft_sync_status",
            "ft_router_logits", "ft_moe_route", "ft_moe_permute", "ft_quantize_mxfp4", "ft_moe_layer_forward",
@@ -33,7 +33,8 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
            "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry",
-           "ft_debug_stack_epoch", "ft_flow_geometry", "ft_fp4_mma_probe", "ft_blob_layout_format")
+           "ft_debug_stack_epoch", "ft_flow_geometry", "ft_fp4_mma_probe", "ft_blob_layout_format",
+           "ft_cache_prefetch")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -60,7 +61,8 @@ class CacheStats(C.Structure):
     _fields_ = [("hits", C.c_int64), ("misses", C.c_int64), ("evictions", C.c_int64), ("moves", C.c_int64),
                 ("h2d_bytes", C.c_int64), ("h2d_ms", C.c_double), ("hit_ms", C.c_double),
                 ("overlap_ms", C.c_double), ("capacity_slots", C.c_int64),
-                ("used_slots", C.c_int64), ("mapped_bytes", C.c_int64)]
+                ("used_slots", C.c_int64), ("mapped_bytes", C.c_int64), ("prefetches", C.c_int64),
+                ("prefetch_hits", C.c_int64), ("prefetch_bytes", C.c_int64)]
 
 
 _lib = None
@@ -110,6 +112,7 @@ def lib() -> C.CDLL:
         "ft_debug_stack_epoch": (ST, [P, U32, I32]),
         "ft_flow_geometry": (ST, [I32, I32, I32, I32, I32, I32, I32, I32, C.POINTER(I64)]),
         "ft_blob_layout_format": (ST, [I32, I32, I32, C.POINTER(I64)]),
+        "ft_cache_prefetch": (ST, [P, I32]),
         "ft_fp4_mma_probe": (ST, [I64, P, P, C.POINTER(I32), P]),
         "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
@@ -256,6 +259,10 @@ def ft_cache_trace(ctx, cap: int = 1 << 20) -> list[tuple]:
     n = I64()
     _check(lib().ft_cache_trace(ctx, buf, cap, C.byref(n)))
     return [(buf[i].kind, buf[i].layer, buf[i].expert, buf[i].slot, buf[i].from_slot) for i in range(n.value)]
+
+
+def ft_cache_prefetch(ctx, per_layer: int) -> None:
+    _check(lib().ft_cache_prefetch(ctx, per_layer))
 
 
 def ft_cache_stats_get(ctx, reset: bool = False) -> dict:

@@ -23,6 +23,7 @@
 #include <string>
 #include <thread>
 #include <unordered_map>
+#include <unordered_set>
 #include <vector>
 
 #include "ft_common.cuh"
@@ -220,6 +221,11 @@ struct ft_ctx {
   std::vector<cudaEvent_t> spare_events;  // finished timing events, reused
   std::vector<cudaEvent_t> miss_events;   // one per miss copy of the current step (no timing)
   std::vector<cudaEvent_t> spare_miss_events;
+  // next-layer prefetch
+  int prefetch_per_layer = 0;
+  std::vector<int64_t> sel_count;                     // [L][E] steps whose set held the expert
+  std::unordered_map<int64_t, cudaEvent_t> pending;   // prefetched keys whose copy may be in flight
+  std::unordered_set<int64_t> unused_prefetch;        // prefetched keys not hit yet
 
   // prefill staging
   uint8_t* d_stage[2] = {nullptr, nullptr};
@@ -478,6 +484,7 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
     if (c->drv.memAddressReserve(&c->va, c->va_size, c->chunk, 0, 0) != CUDA_SUCCESS)
       return bail(fail(FT_ERR_CUDA, "cuMemAddressReserve of %zu bytes failed", c->va_size));
     c->cache_on = true;
+    c->sel_count.assign((size_t)L * E, 0);
     int64_t cap = desc->cache_budget_bytes / c->stride;
     c->lru.set_capacity(cap);
     if ((st = arena_map(c, cap))) return bail(st);
@@ -524,6 +531,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   for (cudaEvent_t e : c->spare_events) cudaEventDestroy(e);
   for (cudaEvent_t e : c->miss_events) cudaEventDestroy(e);
   for (cudaEvent_t e : c->spare_miss_events) cudaEventDestroy(e);
+  for (auto& kv : c->pending) cudaEventDestroy(kv.second);
   free_prefill_scratch(c->pf);
   cudaFree(c->d_status);
   cudaFree(c->d_flag);
@@ -746,11 +754,19 @@ static int64_t key_of(ft_ctx* c, int layer, int expert) { return (int64_t)layer 
 
 // Evict the least recent key not in `keep` (may be empty); returns its slot
 // (-1 if none) and the evicted key in *victim.
-static int32_t evict_one(ft_ctx* c, const std::vector<int64_t>& keep, int64_t* victim = nullptr) {
+static int32_t evict_one(ft_ctx* c, const std::vector<int64_t>& keep, int64_t* victim = nullptr,
+                         int skip_layer = -1) {
   for (auto it = c->lru.order.begin(); it != c->lru.order.end(); ++it) {
     int64_t key = *it;
     if (std::find(keep.begin(), keep.end(), key) != keep.end()) continue;
+    if (skip_layer >= 0 && key / c->d.n_experts == skip_layer) continue;
     auto m = c->lru.map.find(key);
+    c->unused_prefetch.erase(key);
+    auto pe = c->pending.find(key);
+    if (pe != c->pending.end()) {  // a later copy into the slot is ordered after it on the copy stream
+      c->spare_miss_events.push_back(pe->second);
+      c->pending.erase(pe);
+    }
     int32_t slot = m->second.first;
     c->lru.order.erase(it);
     c->lru.map.erase(m);
@@ -847,6 +863,20 @@ static ft_status cache_step(ft_ctx* c, int layer, const std::vector<int>& S, boo
       c->lru.order.splice(c->lru.order.end(), c->lru.order, m->second.second);
       record(c, FT_EV_HIT, layer, e, m->second.first, -1);
       c->stats.hits++;
+      if (c->unused_prefetch.erase(key)) c->stats.prefetch_hits++;
+      auto pe = c->pending.find(key);
+      if (pe != c->pending.end()) {
+        if (cudaEventQuery(pe->second) == cudaSuccess) {
+          c->spare_miss_events.push_back(pe->second);
+        } else if (miss_units) {  // its prefetch copy is still in flight: the expert waits for it
+          miss_units->push_back((int)si);
+          c->miss_events.push_back(pe->second);
+        } else {
+          cudaEventSynchronize(pe->second);
+          c->spare_miss_events.push_back(pe->second);
+        }
+        c->pending.erase(pe);
+      }
       continue;
     }
     int32_t slot;
@@ -917,6 +947,76 @@ static ft_status push_table_rows(ft_ctx* c, const std::vector<int>& rows, cudaSt
   return FT_OK;
 }
 
+// Decode-time next-layer prefetch (see ft_cache_prefetch in ft_moe.h).
+static ft_status prefetch_next(ft_ctx* c, int layer, const std::vector<int>& S) {
+  const int E = c->d.n_experts, L = c->d.n_layers;
+  for (int e : S) c->sel_count[(size_t)layer * E + e]++;
+  if (c->prefetch_per_layer <= 0) return FT_OK;
+  const int n = (layer + 1) % L;
+  if (!c->host_layers[n] || c->resident[n]) return FT_OK;
+  std::vector<int> cand;
+  for (int e = 0; e < E; e++)
+    if (c->sel_count[(size_t)n * E + e] > 0) cand.push_back(e);
+  const int64_t* cnt = c->sel_count.data() + (size_t)n * E;
+  std::stable_sort(cand.begin(), cand.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  std::vector<int64_t> keep;
+  for (int e : S) keep.push_back(key_of(c, layer, e));
+  int done = 0;
+  for (int e : cand) {
+    if (done >= c->prefetch_per_layer) break;
+    const int64_t key = key_of(c, n, e);
+    if (c->lru.map.count(key)) continue;
+    if (c->lru.capacity <= 0) break;
+    int32_t slot;
+    if ((int64_t)c->lru.map.size() >= c->lru.capacity) {
+      slot = evict_one(c, keep, nullptr, n);
+      if (slot < 0) break;
+    } else {
+      slot = c->lru.lowest_free();
+    }
+    c->lru.order.push_back(key);
+    c->lru.map[key] = {slot, std::prev(c->lru.order.end())};
+    c->lru.slot_used[slot] = 1;
+    c->h_eptr_cache[(size_t)n * c->n_blobs + e] = slot_ptr(c, slot);
+    record(c, FT_EV_PREFETCH, n, e, slot, -1);
+    const ft_status fs = fetch(c, n, e, slot);
+    c->stats.h2d_bytes -= fs == FT_OK ? c->lay.used : 0;  // demand-miss bytes only; counted below
+    if (fs != FT_OK) {  // the key never became resident
+      c->lru.order.pop_back();
+      c->lru.map.erase(key);
+      c->lru.slot_used[slot] = 0;
+      c->h_eptr_cache[(size_t)n * c->n_blobs + e] = nullptr;
+      record(c, FT_EV_EVICT, n, e, slot, -1);
+      c->stats.evictions++;
+      cudaStreamSynchronize(c->copy_stream);
+      return fs;
+    }
+    cudaEvent_t ev = nullptr;
+    if (!c->spare_miss_events.empty()) {
+      ev = c->spare_miss_events.back();
+      c->spare_miss_events.pop_back();
+    } else {
+      CUDA_TRY(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    }
+    CUDA_TRY(cudaEventRecord(ev, c->copy_stream));
+    c->pending[key] = ev;
+    c->unused_prefetch.insert(key);
+    c->stats.prefetches++;
+    c->stats.prefetch_bytes += c->lay.used;
+    done++;
+  }
+  c->stats.used_slots = (int64_t)c->lru.map.size();
+  return FT_OK;
+}
+
+extern "C" ft_status ft_cache_prefetch(ft_ctx* c, int32_t per_layer) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
+  if (per_layer < 0 || per_layer > 16) return fail(FT_ERR_INVALID, "per_layer %d outside [0, 16]", per_layer);
+  c->prefetch_per_layer = per_layer;
+  return FT_OK;
+}
+
 extern "C" ft_status ft_expert_cache_lookup(ft_ctx* c, int32_t layer, int32_t expert, int32_t* slot) {
   if (!c || !slot) return fail(FT_ERR_INVALID, "NULL argument");
   if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
@@ -973,6 +1073,8 @@ extern "C" ft_status ft_expert_cache_resize(ft_ctx* c, int64_t new_budget) {
   if (new_budget < 0) return fail(FT_ERR_INVALID, "negative budget");
   if (!c->cache_on) return fail(FT_ERR_INVALID, "context has no expert cache");
   CUDA_TRY(cudaDeviceSynchronize());
+  for (auto& kv : c->pending) c->spare_miss_events.push_back(kv.second);  // every copy has landed
+  c->pending.clear();
   int64_t cap = new_budget / c->stride;
   if ((size_t)cap * c->stride > c->va_size) return fail(FT_ERR_NO_SPACE, "budget larger than the reserved arena");
   const int64_t old_cap = c->lru.capacity;
@@ -1181,6 +1283,9 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   const uint8_t* const* eptr = nullptr;
   std::vector<int> miss_units;  // cache path: units whose blobs are still being copied, in copy order
   int n_routed_units = 0;
+  bool step_timed = false;      // cache path: this step's copies have a timing entry
+  bool cache_layer = false;     // cache path taken
+  std::vector<int> step_set;    // cache path: the step's distinct experts
   const uint8_t* pool = nullptr;
   int stage_buf = -1;
   if (c->resident[layer]) {
@@ -1233,12 +1338,15 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     }
     FT_TRY(push_table_rows(c, dirty, s));
     eptr = c->d_eptr_cache + (size_t)layer * c->n_blobs;
-    if (any_miss && (flags & FT_CACHE_SERIAL)) {
+    if (!miss_units.empty() && (flags & FT_CACHE_SERIAL)) {
       // the serial order, for comparison: every copy lands before any expert runs
-      CUDA_TRY(cudaStreamWaitEvent(s, c->copy_timing.back().c1, 0));
+      for (cudaEvent_t e : c->miss_events) CUDA_TRY(cudaStreamWaitEvent(s, e, 0));
       miss_units.clear();
     }
     n_routed_units = (int)S.size();
+    step_timed = any_miss;
+    cache_layer = true;
+    step_set = S;
   } else {
     return fail(FT_ERR_NOT_FOUND, "layer %d is neither resident nor cached", layer);
   }
@@ -1256,11 +1364,13 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     for (int u = 0; u < n_routed_units; u++)
       if (!is_miss[u]) a.sel[a.n_sel++] = (uint16_t)u;
     for (int sx = 0; sx < c->d.n_shared; sx++) a.sel[a.n_sel++] = (uint16_t)(a.max_units + sx);
-    ft_ctx::StepTiming& stp = c->copy_timing.back();
+    ft_ctx::StepTiming* stp = step_timed ? &c->copy_timing.back() : nullptr;
     if (a.n_sel > 0) {
-      stp.h0 = copy_event(c);
-      stp.h1 = copy_event(c);
-      CUDA_TRY(cudaEventRecord(stp.h0, s));
+      if (stp) {
+        stp->h0 = copy_event(c);
+        stp->h1 = copy_event(c);
+        CUDA_TRY(cudaEventRecord(stp->h0, s));
+      }
       {
         KTimer kt(c, FT_K_GATE_UP, s);
         CUDA_TRY(launch_dec_gate_up(a, false, s));
@@ -1269,7 +1379,7 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
         KTimer kt(c, FT_K_DOWN_COMBINE, s);
         CUDA_TRY(launch_dec_down(a, true, s));
       }
-      CUDA_TRY(cudaEventRecord(stp.h1, s));
+      if (stp) CUDA_TRY(cudaEventRecord(stp->h1, s));
     }
     for (size_t mi = 0; mi < miss_units.size(); mi++) {
       CUDA_TRY(cudaStreamWaitEvent(s, c->miss_events[mi], 0));
@@ -1341,6 +1451,9 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   }
   if (stage_buf >= 0) CUDA_TRY(cudaEventRecord(c->ev_done[stage_buf], s));
   c->last_stream = s;
+  // cache path: count the step's experts; the next layer's prefetch follows
+  // the step's own copies on the copy stream
+  if (cache_layer) FT_TRY(prefetch_next(c, layer, step_set));
   return FT_OK;
 }
 

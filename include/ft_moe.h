@@ -106,6 +106,7 @@ typedef struct {
 #define FT_EV_MISS  1
 #define FT_EV_EVICT 2
 #define FT_EV_MOVE  3
+#define FT_EV_PREFETCH 4   /* inserted ahead of use by ft_cache_prefetch's policy */
 typedef struct {
   int32_t kind;      /* FT_EV_* */
   int32_t layer;
@@ -122,6 +123,9 @@ typedef struct {
   double  overlap_ms;         /* part of hit_ms that ran while that step's copies were in flight */
   int64_t capacity_slots, used_slots;
   int64_t mapped_bytes;       /* physical memory mapped under the slot arena */
+  int64_t prefetches;         /* keys inserted by the next-layer prefetch */
+  int64_t prefetch_hits;      /* prefetched keys later hit (each counted once) */
+  int64_t prefetch_bytes;     /* bytes copied by those prefetches */
 } ft_cache_stats;
 
 /* ---------------------------------------------------------------------- */
@@ -293,6 +297,20 @@ FT_API ft_status ft_expert_cache_insert(ft_ctx* ctx, int32_t layer, int32_t expe
  * not touched.  FT_ERR_INVALID for a negative budget; FT_ERR_CUDA if physical
  * memory cannot be mapped. */
 FT_API ft_status ft_expert_cache_resize(ft_ctx* ctx, int64_t new_budget_bytes);
+
+/* Decode-time next-layer prefetch ([ro] predictive preloading of the
+ * experts the coming tokens will likely use; [fa] adjacent tokens' expert
+ * paths overlap).  With per_layer > 0 (at most 16), after each cache step at
+ * layer l the context counts that step's experts, then copies up to per_layer
+ * experts of layer (l + 1) mod n_layers into the cache: those selected at
+ * least once so far, most often first (ties to the lower id), skipping
+ * resident ones.  Each is inserted as most recent (a FT_EV_PREFETCH event),
+ * evicting when full the least recent key that is neither in the step's set
+ * nor of layer l + 1.  The copies run on the copy stream behind the step's
+ * own misses; an expert hit before its prefetch copy landed waits for that
+ * copy.  0 turns it off (the default).  FT_ERR_INVALID outside [0, 16] or
+ * without a cache. */
+FT_API ft_status ft_cache_prefetch(ft_ctx* ctx, int32_t per_layer);
 
 /* Copy out the cache events recorded since the last call (HIT, MISS, EVICT,
  * MOVE in order) and clear them.  *n = events written (<= cap); if more were

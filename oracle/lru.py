@@ -26,7 +26,7 @@ HIT, MISS, EVICT, MOVE; from_slot is the old slot for MOVE and -1 otherwise.
 """
 from __future__ import annotations
 
-HIT, MISS, EVICT, MOVE = 0, 1, 2, 3
+HIT, MISS, EVICT, MOVE, PREFETCH = 0, 1, 2, 3, 4
 
 
 class NoSpace(Exception):
@@ -95,3 +95,82 @@ class LRUCache:
         self.order.remove(key)
         self.order.append(key)
         return self.slot[key]
+
+
+class PrefetchingLRUCache(LRUCache):
+    """The global LRU with decode-time next-layer prefetch.
+
+    Pages: the engine preloads the experts the coming tokens are likely to
+    use, judged from their activation patterns (world.tibi.club, "Cum
+    reușește FreeToken să ruleze 753B pe un singur GPU?", predictive
+    scheduling; low-reliability page), and the shared LRU exploits the
+    overlap of adjacent tokens' expert paths (aipolix.com, paragraph on
+    semantic-aware caching).  The pages give no rule; the reading used here:
+
+    * every step adds 1 to the count of each expert of its set S at its layer;
+    * after the step at layer l, the next layer n = (l + 1) mod n_layers gets
+      up to ``per_layer`` prefetches: its experts selected at least once,
+      ranked by count (descending, ties to the lower id), resident ones
+      skipped; each is inserted like a miss (evicting, when full, the least
+      recent key that is neither in the step's S at layer l nor of layer n,
+      else the lowest free slot) and recorded as PREFETCH;
+    * a later HIT on a prefetched key counts as a prefetch hit (once).
+    """
+
+    def __init__(self, capacity: int, n_layers: int, n_experts: int, per_layer: int):
+        super().__init__(capacity)
+        self.n_layers, self.n_experts, self.per_layer = n_layers, n_experts, per_layer
+        self.count = [[0] * n_experts for _ in range(n_layers)]
+        self.unused = set()
+        self.prefetches = 0
+        self.prefetch_hits = 0
+
+    def step(self, layer, experts) -> list[tuple]:
+        ev = super().step(layer, experts)
+        S = sorted(set(int(e) for e in experts))
+        for kind, l, e, _, _ in ev:
+            if kind == HIT and (l, e) in self.unused:
+                self.unused.discard((l, e))
+                self.prefetch_hits += 1
+            if kind == EVICT:
+                self.unused.discard((l, e))
+        for e in S:
+            self.count[layer][e] += 1
+        if self.per_layer <= 0:
+            return ev
+        n = (layer + 1) % self.n_layers
+        keep = {(layer, e) for e in S}
+        ranked = sorted((e for e in range(self.n_experts) if self.count[n][e] > 0),
+                        key=lambda e: (-self.count[n][e], e))
+        done = 0
+        for e in ranked:
+            if done >= self.per_layer:
+                break
+            key = (n, e)
+            if key in self.slot:
+                continue
+            if len(self.order) == self.capacity:
+                cands = [k for k in self.order if k not in keep and k[0] != n]
+                if not cands:
+                    break
+                victim = cands[0]
+                self.order.remove(victim)
+                s = self.slot.pop(victim)
+                self.unused.discard(victim)
+                ev.append((EVICT, victim[0], victim[1], s, -1))
+            else:
+                s = min(self._free_slots())
+            self.slot[key] = s
+            self.order.append(key)
+            self.unused.add(key)
+            self.prefetches += 1
+            ev.append((PREFETCH, n, e, s, -1))
+            done += 1
+        return ev
+
+    def resize(self, capacity: int) -> list[tuple]:
+        ev = super().resize(capacity)
+        for kind, l, e, _, _ in ev:
+            if kind == EVICT:
+                self.unused.discard((l, e))
+        return ev

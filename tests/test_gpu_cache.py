@@ -189,3 +189,44 @@ def test_cache_trace_dsv4_shape_matches_oracle():
     finally:
         cache.close()
         res.close()
+
+
+@pytest.mark.parametrize("per_layer", [1, 2])
+def test_cache_prefetch_matches_oracle_and_resident_outputs(per_layer):
+    """Decode-time next-layer prefetch: the event sequence, PREFETCH events
+    included, equals the oracle's prefetching LRU step by step; prefetch and
+    prefetch-hit counts agree; every output equals the resident path's (a
+    prefetched expert hit before its copy landed waits for the copy)."""
+    stride = synth.blob_stride(H, I)
+    hp = host_pools(E)
+    dp = [p.cuda() for p in hp]
+    cap = 10
+    cache = Ctx(ft.make_desc(H, I, E, K, L, 0, cap * stride, 4), hp, None)
+    res = Ctx(ft.make_desc(H, I, E, K, L, 0, 0, 4), None, dp)
+    ref = olru.PrefetchingLRUCache(cap, L, E, per_layer)
+    traces = [[synth.zipf_trace(SEED, layer, 80, E, K, 1.0, 0.5, stream=s) for s in range(2)] for layer in range(L)]
+    try:
+        ft.ft_cache_prefetch(cache.h, per_layer)
+        for step in range(80):
+            if step == 40:
+                ft.ft_expert_cache_resize(cache.h, 6 * stride)
+                assert oracle_events(ft.ft_cache_trace(cache.h)) == ref.resize(6)
+            layer = step % L
+            T = 1 + (step % 2)
+            sets = np.stack([traces[layer][t][step] for t in range(T)])
+            lg = synth.logits_for_sets(SEED, 500 + step, sets, E)
+            x = x_dev(synth.activations_bf16(SEED, 500 + step, T, H))
+            lgd = torch.from_numpy(lg).cuda()
+            o1, o2 = torch.empty_like(x), torch.empty_like(x)
+            ft.ft_moe_layer_forward(cache.h, layer, x, T, None, lgd, o1, 1)
+            ft.ft_moe_layer_forward(res.h, layer, x, T, None, lgd, o2, 1)
+            torch.cuda.synchronize()
+            assert (bf16_bits(o1) == bf16_bits(o2)).all(), step
+            ids, _ = routing.topk(lg, K)
+            assert oracle_events(ft.ft_cache_trace(cache.h)) == ref.step(layer, ids.reshape(-1)), step
+        st = ft.ft_cache_stats_get(cache.h)
+        assert st["prefetches"] == ref.prefetches > 0 and st["prefetch_hits"] == ref.prefetch_hits
+        assert st["prefetch_bytes"] == st["prefetches"] * ft.ft_blob_layout(H, I)["used"]
+    finally:
+        cache.close()
+        res.close()

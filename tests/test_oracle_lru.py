@@ -124,3 +124,53 @@ def test_lookup_touches_a_hit_and_leaves_a_miss_alone():
     d.step(0, [1])
     d.step(0, [2])
     assert d.step(0, [3]) == [(lru.EVICT, 0, 1, 0, -1), (lru.MISS, 0, 3, 0, -1)]   # without the lookup
+
+
+def test_prefetch_hand_sequence():
+    """Capacity 6, 3 layers, 8 experts, one prefetch per step, worked by hand
+    from the stated rule (counts of each layer's selections; after a step at
+    layer l, the most-counted non-resident expert of layer l+1 is inserted,
+    evicting the least recent key outside the step's set and outside layer
+    l+1)."""
+    H_, M_, E_, P_ = lru.HIT, lru.MISS, lru.EVICT, lru.PREFETCH
+    c = lru.PrefetchingLRUCache(6, 3, 8, 1)
+    assert c.step(0, [1, 2]) == [(M_, 0, 1, 0, -1), (M_, 0, 2, 1, -1)]      # layer 1 has no counts yet
+    assert c.step(1, [3]) == [(M_, 1, 3, 2, -1)]
+    assert c.step(2, [1]) == [(M_, 2, 1, 3, -1)]                             # layer 0's counted experts resident
+    assert c.step(0, [1, 5]) == [(H_, 0, 1, 0, -1), (M_, 0, 5, 4, -1)]
+    assert c.step(1, [3, 4]) == [(H_, 1, 3, 2, -1), (M_, 1, 4, 5, -1)]      # now full
+    # (2,6) evicts the least recent (0,2); then layer 0's counts 1:2, 2:1, 5:1
+    # pick (0,2), evicting the least recent key outside {(2,1),(2,6)} and layer 0: (1,3)
+    assert c.step(2, [1, 6]) == [(H_, 2, 1, 3, -1), (E_, 0, 2, 1, -1), (M_, 2, 6, 1, -1),
+                                 (E_, 1, 3, 2, -1), (P_, 0, 2, 2, -1)]
+    # (0,2) is a prefetch hit; layer 1's counts 3:2, 4:1 pick (1,3), evicting (0,1)
+    assert c.step(0, [2, 5]) == [(H_, 0, 2, 2, -1), (H_, 0, 5, 4, -1), (E_, 0, 1, 0, -1), (P_, 1, 3, 0, -1)]
+    assert c.prefetches == 2 and c.prefetch_hits == 1
+    # (1,3) is the second prefetch hit; layer 2's counted experts 1, 6 are resident
+    assert c.step(1, [3]) == [(H_, 1, 3, 0, -1)]
+    assert c.prefetch_hits == 2
+
+
+def test_prefetch_off_is_the_plain_lru_and_counts_are_consistent():
+    import numpy as np
+    rng = np.random.default_rng(11)
+    a, b = lru.LRUCache(10), lru.PrefetchingLRUCache(10, 4, 16, 0)
+    p = lru.PrefetchingLRUCache(10, 4, 16, 2)
+    for step in range(300):
+        if step == 120:
+            assert a.resize(5) == b.resize(5)
+            p.resize(5)
+        if step == 200:
+            assert a.resize(10) == b.resize(10)
+            p.resize(10)
+        layer = step % 4
+        e = rng.choice(16, 2, replace=False)
+        assert a.step(layer, e) == b.step(layer, e)
+        ev = p.step(layer, e)
+        # a prefetch never evicts the step's own keys nor keys of the layer it fills
+        pf = [x for x in ev if x[0] == lru.PREFETCH]
+        for x in ev:
+            if x[0] == lru.EVICT and pf:
+                assert (x[1], x[2]) not in {(layer, int(v)) for v in e}
+        assert len(p.slot) <= p.capacity
+    assert b.prefetches == 0 and 0 < p.prefetch_hits <= p.prefetches
