@@ -670,9 +670,10 @@ def measure_misses(tokens=512, layers=43, resize_at=(170, 340)):
     # cache again: a resize to 0 evicts every expert, the next restores the budget
     ctx = ft.ft_create(ft.make_desc(H3, I3, E3, k3, L3, 0, budget, 1), hp, None)
 
-    def run(flags):
+    def run(flags, prefetch=0):
         ft.ft_expert_cache_resize(ctx, 0)
         ft.ft_expert_cache_resize(ctx, budget)
+        ft.ft_cache_prefetch(ctx, prefetch)
         ft.ft_cache_trace(ctx, cap=1 << 22)
         ft.ft_cache_stats_get(ctx, reset=True)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -697,6 +698,7 @@ def measure_misses(tokens=512, layers=43, resize_at=(170, 340)):
 
     total_ms, st, ev = run(ft.FT_ROUTE_RENORM)
     serial_ms, st_s, _ = run(ft.FT_ROUTE_RENORM | ft.FT_CACHE_SERIAL)
+    pf_ms, st_p, _ = run(ft.FT_ROUTE_RENORM, prefetch=2)
     ft.ft_destroy(ctx)
     del hp
     lookups = st["hits"] + st["misses"]
@@ -719,7 +721,13 @@ def measure_misses(tokens=512, layers=43, resize_at=(170, 340)):
             "overlap": {"resident_expert_ms": st["hit_ms"], "under_copies_ms": st["overlap_ms"],
                         "frac_of_resident_compute_hidden": st["overlap_ms"] / st["hit_ms"] if st["hit_ms"] else None,
                         "serial_order_tok_s": tokens / (serial_ms * 1e-3),
-                        "saved_ms": serial_ms - total_ms}}
+                        "saved_ms": serial_ms - total_ms},
+            # the same trace with decode-time next-layer prefetch (2 per layer step)
+            "prefetch": {"per_layer": 2, "tok_s": tokens / (pf_ms * 1e-3), "prefetches": st_p["prefetches"],
+                         "prefetch_hits": st_p["prefetch_hits"],
+                         "hit_rate": st_p["prefetch_hits"] / st_p["prefetches"] if st_p["prefetches"] else None,
+                         "miss_rate": st_p["misses"] / max(st_p["hits"] + st_p["misses"], 1),
+                         "gain_vs_default": total_ms / pf_ms - 1.0}}
 
 
 def measure_decode_formats(args, pk, steps=300, warmup=20):
