@@ -34,7 +34,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
            "ft_debug_device_wait", "ft_debug_host_wait_limit", "ft_debug_fail_copy", "ft_decode_geometry",
            "ft_debug_stack_epoch", "ft_flow_geometry", "ft_fp4_mma_probe", "ft_blob_layout_format",
-           "ft_cache_prefetch")
+           "ft_cache_prefetch", "ft_debug_stack_timeline")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
            "combine", "dec_stack")
@@ -113,6 +113,7 @@ def lib() -> C.CDLL:
         "ft_flow_geometry": (ST, [I32, I32, I32, I32, I32, I32, I32, I32, C.POINTER(I64)]),
         "ft_blob_layout_format": (ST, [I32, I32, I32, C.POINTER(I64)]),
         "ft_cache_prefetch": (ST, [P, I32]),
+        "ft_debug_stack_timeline": (ST, [P, P, I64]),
         "ft_fp4_mma_probe": (ST, [I64, P, P, C.POINTER(I32), P]),
         "ft_decode_geometry": (ST, [I32, I32, I32, C.POINTER(I64)]),
     }
@@ -259,6 +260,10 @@ def ft_cache_trace(ctx, cap: int = 1 << 20) -> list[tuple]:
     n = I64()
     _check(lib().ft_cache_trace(ctx, buf, cap, C.byref(n)))
     return [(buf[i].kind, buf[i].layer, buf[i].expert, buf[i].slot, buf[i].from_slot) for i in range(n.value)]
+
+
+def ft_debug_stack_timeline(ctx, buf=None) -> None:
+    _check(lib().ft_debug_stack_timeline(ctx, _ptr(buf, 8), buf.numel() if buf is not None else 0))
 
 
 def ft_cache_prefetch(ctx, per_layer: int) -> None:

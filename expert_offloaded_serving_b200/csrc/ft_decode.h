@@ -141,6 +141,10 @@ struct FlowArgs {
   const uint32_t* epoch;       // advanced by the routing kernel before this launch
   int rows_cap;                // down-tile rows over all units (flow_geometry)
   int* status;
+  // NULL, or [n_layers][gridDim][8] %globaltimer stamps of each CTA: gate/up
+  // start, x staged, h published, down h staged, x published (0 where the CTA
+  // had no tile of the phase)
+  uint64_t* timeline;
 };
 struct FlowGeom {
   int rows_cap;

@@ -406,11 +406,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
   if (b < lhdr(0).tiles_a) issue_A(0, b);
   if (b < lhdr(0).nd) issue_B(0, b);
 
+  uint64_t* tl = nullptr;  // this CTA's stamps of the current layer (timeline attached)
+  auto stamp = [&](int i) {
+    if (tl && threadIdx.x == 0) tl[i] = gclock();
+  };
   for (int l = 0; l < a.n_layers; l++) {
     const FlowLayerHdr lh = lhdr(l);
     const FlowUnit* un = lunits(l);
     const uint32_t tag = (epoch << 7) | (uint32_t)l;
     const bool last = l + 1 == a.n_layers;
+    tl = a.timeline ? a.timeline + ((size_t)l * G + b) * 8 : nullptr;
+    stamp(0);
     // ---------------- gate/up + SwiGLU ----------------
     for (int i = b; i < lh.tiles_a; i += G) {
       if (i != b) issue_A(l, i);  // buffer A is free since the previous tile's compute
@@ -429,6 +435,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         drain();
         return;
       }
+      if (i == b) stamp(1);
       tile_dots<F>(gA, lmA, baseA, f.m);
       __syncthreads();
       if (threadIdx.x < gA.R * f.m) {
@@ -443,6 +450,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
       }
       __syncthreads();
     }
+    if (b < lh.tiles_a) stamp(2);
     // buffer A is free: the next layer's first gate/up tile streams in now
     if (!last && b < lhdr(l + 1).tiles_a) issue_A(l + 1, b);
     // ---------------- down + combine, over every unit ----------------
@@ -458,6 +466,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
           drain();
           return;
         }
+        if (d == b) stamp(3);
         if (T > 1) dtile_dots<2, F>(gB, lmB, baseB, un, lh.units, rb);
         else dtile_dots<1, F>(gB, lmB, baseB, un, lh.units, rb);
         __syncthreads();
@@ -491,6 +500,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         __syncthreads();
       }
     }
+    if (b < lh.nd) stamp(4);
     // buffer B is free: the next layer's first down tile streams in now
     if (!last && b < lhdr(l + 1).nd) issue_B(l + 1, b);
   }

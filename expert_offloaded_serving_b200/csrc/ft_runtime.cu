@@ -182,6 +182,8 @@ struct ft_ctx {
   uint64_t* d_x_tagged = nullptr;  // [T][H/2] words (dataflow kernel)
   int64_t tagged_words = 0;
   uint32_t* d_epoch = nullptr;     // launch counter for those tags
+  uint64_t* timeline = nullptr;    // dataflow kernel phase stamps (caller's device buffer) or NULL
+  int64_t timeline_words = 0;
 
   // failure injection
   double host_wait_s = kHostWaitSeconds;  // limit of the bounded host waits
@@ -720,6 +722,14 @@ extern "C" ft_status ft_debug_stack_epoch(ft_ctx* c, uint32_t epoch, int32_t poi
     std::vector<uint64_t> w((size_t)c->tagged_words, word);
     CUDA_TRY(cudaMemcpy(c->d_tagged, w.data(), w.size() * sizeof(uint64_t), cudaMemcpyHostToDevice));
   }
+  return FT_OK;
+}
+
+extern "C" ft_status ft_debug_stack_timeline(ft_ctx* c, uint64_t* buf, int64_t n_words) {
+  if (!c) return fail(FT_ERR_INVALID, "ctx is NULL");
+  if (buf && n_words <= 0) return fail(FT_ERR_INVALID, "n_words must be positive");
+  c->timeline = buf;
+  c->timeline_words = buf ? n_words : 0;
   return FT_OK;
 }
 
@@ -1575,6 +1585,10 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     a.epoch = c->d_epoch;
     a.rows_cap = fg.rows_cap;
     a.status = c->d_status;
+    int dev = 0, nsm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    a.timeline = c->timeline && c->timeline_words >= (int64_t)n_layers * nsm * 8 ? c->timeline : nullptr;
     KTimer kt(c, FT_K_DEC_STACK, s);
     CUDA_TRY(launch_dec_flow(a, s));
     c->last_stream = s;

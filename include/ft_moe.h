@@ -400,6 +400,16 @@ FT_API ft_status ft_debug_device_wait(ft_ctx* ctx, int64_t timeout_us, void* str
  * Errors: FT_ERR_INVALID, FT_ERR_STATE (no persistent kernel in this
  * context), FT_ERR_CUDA. */
 FT_API ft_status ft_debug_stack_epoch(ft_ctx* ctx, uint32_t epoch, int32_t poison_layer);
+
+/* Phase timeline of the dataflow stack kernel, for profiling: with buf (dev
+ * uint64 [n_words]) attached, each later ft_moe_stack_forward that runs the
+ * dataflow kernel over n layers with at least n * (number of SMs) * 8 words
+ * writes, at [layer][CTA][0..4], the %globaltimer nanoseconds at which the
+ * CTA began the layer, had its first gate/up tile's input and weights, had
+ * published its h, had its first down tile's h and weights, and had
+ * published its part of the next layer's input (0 where the CTA had no tile
+ * of that phase).  NULL detaches it.  The kernel's results do not change. */
+FT_API ft_status ft_debug_stack_timeline(ft_ctx* ctx, uint64_t* buf, int64_t n_words);
 FT_API ft_status ft_debug_host_wait_limit(ft_ctx* ctx, double seconds);
 FT_API ft_status ft_debug_fail_copy(ft_ctx* ctx, int64_t n);
 
