@@ -51,6 +51,80 @@ __global__ void __launch_bounds__(256) k_router_logits(const uint16_t* __restric
   }
 }
 
+// ---------------------------------------------------------------------------
+// router logits for many tokens: the same summation order, tiled.  A CTA of 8
+// warps takes 8 tokens x 32 experts; per 128-element block of K it stages the
+// block of x and of Wr in shared memory, converted to fp64 once (each x value
+// then serves 32 experts, each Wr value 8 tokens), element 4j + v of the block
+// at [v][j] so that lane j's reads are consecutive.  Warp w computes experts
+// 4w .. 4w+3 for all 8 tokens; lane j holds partial sum j of each of those
+// 32 (token, expert) pairs and adds its block elements 4j, 4j+1, 4j+2, 4j+3 in
+// ascending order, so every partial sum sees the same terms in the same
+// order as in k_router_logits; the butterfly and the rounding are the same.
+// ---------------------------------------------------------------------------
+constexpr int kRtT = 8, kRtE = 32;
+
+__global__ void __launch_bounds__(256) k_router_logits_tiled(const uint16_t* __restrict__ x,
+                                                             const float* __restrict__ wr, int T, int H, int E,
+                                                             float* __restrict__ logits) {
+  __shared__ double xs[kRtT][4][32];
+  __shared__ double ws[kRtE][4][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+  double acc[4][kRtT];
+#pragma unroll
+  for (int i = 0; i < 4; i++)
+#pragma unroll
+    for (int t = 0; t < kRtT; t++) acc[i][t] = 0.0;
+  const int C = H >> 7;
+  for (int c = 0; c < C; c++) {
+    __syncthreads();
+    {  // x: 8 tokens x 128 elements, 4 per thread
+      const int t = threadIdx.x >> 5, q = threadIdx.x & 31;  // elements 4q .. 4q+3 of token t
+      uint2 xv = make_uint2(0u, 0u);
+      if (t0 + t < T) xv = __ldg(reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H + c * 128) + q);
+      xs[t][0][q] = (double)bf16_bits_to_f32((uint16_t)(xv.x & 0xffff));
+      xs[t][1][q] = (double)bf16_bits_to_f32((uint16_t)(xv.x >> 16));
+      xs[t][2][q] = (double)bf16_bits_to_f32((uint16_t)(xv.y & 0xffff));
+      xs[t][3][q] = (double)bf16_bits_to_f32((uint16_t)(xv.y >> 16));
+    }
+#pragma unroll
+    for (int r = 0; r < 4; r++) {  // Wr: 32 experts x 128 elements, 16 per thread
+      const int idx = threadIdx.x + 256 * r, e = idx >> 5, q = idx & 31;
+      float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0 + e < E) w4 = __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + e) * H + c * 128) + q);
+      ws[e][0][q] = (double)w4.x;
+      ws[e][1][q] = (double)w4.y;
+      ws[e][2][q] = (double)w4.z;
+      ws[e][3][q] = (double)w4.w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int v = 0; v < 4; v++) {
+      double xr[kRtT], wv[4];
+#pragma unroll
+      for (int t = 0; t < kRtT; t++) xr[t] = xs[t][v][lane];
+#pragma unroll
+      for (int i = 0; i < 4; i++) wv[i] = ws[4 * warp + i][v][lane];
+#pragma unroll
+      for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int t = 0; t < kRtT; t++) acc[i][t] = fma(xr[t], wv[i], acc[i][t]);  // exact product: fma == add
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const int e = e0 + 4 * warp + i;
+#pragma unroll
+    for (int t = 0; t < kRtT; t++) {
+      double a = acc[i][t];
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) a = a + __shfl_xor_sync(0xffffffffu, a, d);
+      if (lane == 0 && e < E && t0 + t < T) logits[(size_t)(t0 + t) * E + e] = __double2float_rn(a);
+    }
+  }
+}
+
 cudaError_t launch_router_logits(const uint16_t* x, const float* wr, int T, int H, int E, float* logits,
                                  cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
@@ -58,9 +132,12 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* wr, int T, int 
   if (T <= 4) {
     dim3 grid((T + 3) / 4, (E + 7) / 8);
     k_router_logits<4><<<grid, block, 0, s>>>(x, wr, T, H, E, logits);
-  } else {
+  } else if (T < 64) {
     dim3 grid((T + 7) / 8, (E + 7) / 8);
     k_router_logits<8><<<grid, block, 0, s>>>(x, wr, T, H, E, logits);
+  } else {
+    dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
+    k_router_logits_tiled<<<grid, block, 0, s>>>(x, wr, T, H, E, logits);
   }
   return cudaGetLastError();
 }

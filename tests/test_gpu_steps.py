@@ -54,7 +54,7 @@ def test_gpu_dequant_bit_exact(H, I):
         c.close()
 
 
-@pytest.mark.parametrize("T", [1, 2, 3, 4, 7, 8, 33, 300])
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 7, 8, 33, 63, 64, 300])
 @pytest.mark.parametrize("H,E", [(256, 16), (2048, 256), (4096, 256)])
 def test_gpu_router_logits_bit_exact(ctx, T, H, E):
     xb = synth.activations_bf16(11, T, T, H)
