@@ -16,9 +16,10 @@
 //   k_dec_stack     persistent and cooperative: one launch runs a stack of
 //                   layers; each CTA takes the gate/up and the down tiles with
 //                   its index modulo the grid, layer after layer; layers hand
-//                   over through bounded counters in global memory (and, for
-//                   one or two tokens, h through tagged words) instead of
+//                   over through bounded counters in global memory instead of
 //                   kernel boundaries; same arithmetic as the two kernels above.
+//                   (One or two tokens go to the dataflow kernel of
+//                   ft_decode_flow.cu unless FT_STACK_COUNTERS asks for this one.)
 //
 // All three share the GEMV tile: lanes own 32-code chunks of K and hold their
 // chunk's activations (re-encoded per 32-element block as f16) in registers,
@@ -466,102 +467,6 @@ __device__ __forceinline__ void cta_arrive(int* p) {
   }
 }
 
-// out[t][n] = bf16( sum_j w[t][j] * y[pos[t][j]][n]  (j ascending, fused)
-//                   + sum_s y[T*k + s*T + t][n] ) for 4 consecutive n (group q)
-// of row length H; the same arithmetic as the combine of the per-layer kernels.
-__device__ __forceinline__ void combine4(const float* y, const float* cw, const int* cpos, int tok, int q, int H, int T,
-                                         int k, int S, float (&v)[4]) {
-  constexpr int kBatch = 8;  // rows in flight at once
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  // the shared expert's row is loaded with the first batch and added last
-  float4 sh = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (S > 0) sh = __ldcg(reinterpret_cast<const float4*>(y + (size_t)(T * k + tok) * H) + q);
-  for (int j0 = 0; j0 < k; j0 += kBatch) {
-    float4 u[kBatch];
-    float w[kBatch];
-#pragma unroll
-    for (int j = 0; j < kBatch; j++) {
-      if (j0 + j < k) {
-        const int f = tok * k + j0 + j;
-        w[j] = cw[f];
-        u[j] = __ldcg(reinterpret_cast<const float4*>(y + (size_t)cpos[f] * H) + q);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kBatch; j++) {
-      if (j0 + j < k) {
-        acc[0] = fmaf(w[j], u[j].x, acc[0]);
-        acc[1] = fmaf(w[j], u[j].y, acc[1]);
-        acc[2] = fmaf(w[j], u[j].z, acc[2]);
-        acc[3] = fmaf(w[j], u[j].w, acc[3]);
-      }
-    }
-  }
-  for (int s2 = 0; s2 < S; s2++) {
-    const float4 u = s2 == 0 ? sh : __ldcg(reinterpret_cast<const float4*>(y + (size_t)(T * k + s2 * T + tok) * H) + q);
-    acc[0] += u.x;
-    acc[1] += u.y;
-    acc[2] += u.z;
-    acc[3] += u.w;
-  }
-#pragma unroll
-  for (int e = 0; e < 4; e++) v[e] = __bfloat162float(__float2bfloat16_rn(acc[e]));
-}
-
-// The gate/up activations of tokens toks[0 .. n) rebuilt from the previous
-// layer's y (the layer input is that layer's combined output), re-encoded like
-// stage_x.
-__device__ __forceinline__ void stage_comb(const Gv& g, uint8_t* base, const StackArgs& a, int H, const float* cw,
-                                           const int* cpos, const int* toks, int n) {
-  const int per = g.K / 4;
-  const int items = (n > 1 ? kMT : 1) * per;
-  for (int i = threadIdx.x; i < items; i += kGemvThreads) {
-    const int t = i / per, q = i - t * per;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (t < n) combine4(a.y, cw, cpos, toks[t], q, H, a.T, a.k, a.n_shared, v);
-    encode4(g, base, t, q, v);
-  }
-}
-
-// The down tile's activations from the tagged h: a word whose tag is not
-// this layer's has not arrived yet and is read again, for at most 2 s (then
-// the timeout bit and the CTA's abort flag are set).  Re-encoded like
-// stage_x.
-__device__ __forceinline__ void stage_h_tagged(const Gv& g, uint8_t* base, const uint64_t* ht, const int* rows, int n,
-                                               uint32_t tag, int& abort, int* status) {
-  const int per = g.K / 4;
-  const int items = (n > 1 ? kMT : 1) * per;
-  for (int i = threadIdx.x; i < items; i += kGemvThreads) {
-    const int t = i / per, q = i - t * per;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (t < n) {
-      const uint64_t* p = ht + (size_t)rows[t] * g.K + 4 * q;
-      uint64_t w[4];
-      ld_tagged4(p, w);
-      auto ready = [&]() {
-        return (uint32_t)(w[0] >> 32) == tag && (uint32_t)(w[1] >> 32) == tag && (uint32_t)(w[2] >> 32) == tag &&
-               (uint32_t)(w[3] >> 32) == tag;
-      };
-      if (!ready()) {
-        const uint64_t t0 = gclock();
-        for (;;) {
-          __nanosleep(20);
-          ld_tagged4(p, w);
-          if (ready()) break;
-          if (gclock() - t0 > kSpinNs) {
-            set_status(status, kStTimeout);
-            abort = 1;
-            break;
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; j++) v[j] = __uint_as_float((uint32_t)w[j]);
-    }
-    encode4(g, base, t, q, v);
-  }
-}
-
 // One warp resolves tile i of a phase (nrb row blocks of R rows per unit) of
 // layer `rec` into m; the caller synchronises before the CTA reads it.
 __device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* rec, const uint8_t* const* eptr, int i,
@@ -598,12 +503,8 @@ __device__ __forceinline__ void resolve_tile(const StackArgs& a, const Route* re
 // Wu) and then its down tiles (unit x R rows of Wd); tile i of a phase goes to
 // CTA i mod gridDim.  Dependencies between CTAs go through counters in global
 // memory.  Per layer: [0] gate/up tiles done (down waits for all of them);
-// [1] down tiles done (fused mode) or row blocks combined; [2 + rb] down
-// tiles done in row block rb.  In the fused mode (a.fused, one or two tokens)
-// the next layer's gate/up tiles rebuild their input from y themselves, so a
-// layer hands over after its last down tile, and h goes from gate/up to down
-// as tagged words that the down tiles poll, without counter [0]; otherwise
-// the last down tile of a row block combines that block into the layer output
+// [1] row blocks combined; [2 + rb] down tiles done in row block rb.  The
+// last down tile of a row block combines that block into the layer output
 // and the next layer waits for every row block.  A CTA streams its next
 // tiles' weights during a compute phase: the layer's first down tile during
 // gate/up, the next layer's first gate/up tile during down.  Activations
@@ -623,8 +524,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   const LaneMap lmA = lane_map(gA), lmB = lane_map(gB);
   const int G = gridDim.x, b = blockIdx.x;
   const int nrbA = I / gA.R, nrbB = H / gB.R;
-  const bool fused = a.fused != 0;
-  const uint32_t epoch = fused ? *a.epoch : 0u;  // tag of layer l: epoch << 7 | l
 
   // A tile's codes (R contiguous rows per matrix) arrive by bulk copies that
   // one thread issues and that complete on the buffer's mbarrier; its scale
@@ -712,9 +611,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     int* sy = a.sync + (size_t)l * a.sync_stride;
     const int units_n = l + 1 < a.n_layers ? units_of[l + 1] : 0;
     const bool nextA = b < units_n * nrbA;
-    // the combine weights this layer uses: the previous layer's for the fused
-    // gate/up input, else this layer's for its row-block combines
-    if (fused ? l > 0 : haveB) load_combine(fused ? rec - 1 : rec);
+    // the combine weights of this layer's row-block combines
+    if (haveB) load_combine(rec);
     if (haveB && !haveA && !issuedB) {
       issue_B(first[2 * l + 1]);
       issuedB = true;
@@ -725,7 +623,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         // the first tile was issued ahead: wait for the previous layer
         if (l > 0) {
           const int* prev = a.sync + (size_t)(l - 1) * a.sync_stride + 1;
-          if (!cta_wait_geq(prev, fused ? units_of[l - 1] * nrbB : nrbB, hd.abort, a.status)) {
+          if (!cta_wait_geq(prev, nrbB, hd.abort, a.status)) {
             drain();
             return;
           }
@@ -739,8 +637,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
       for (int t0 = 0; t0 < m.m; t0 += kMT) {
         const int n = min(kMT, m.m - t0);
         if (t0 > 0) __syncthreads();
-        if (fused && l > 0) stage_comb(gA, baseA, a, H, hd.cw, hd.cpos, m.tok + t0, n);
-        else stage_x<true>(gA, baseA, xin, m.tok + t0, n);
+        stage_x<true>(gA, baseA, xin, m.tok + t0, n);
         // the layer's first down tile streams in during the gate/up compute;
         // issued after the staging loads so as not to queue ahead of them
         if (i == b && t0 == 0 && haveB && !issuedB) {
@@ -760,16 +657,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         if (threadIdx.x < gA.R * n) {
           const int t = threadIdx.x >> gA.rlog, r = threadIdx.x & (gA.R - 1);
           const size_t at = (size_t)(m.hbase + t0 + t) * I + m.row0 + r;
-          if (fused)  // a missing expert still delivers (zeros), so no reader waits for it
-            st_tagged(a.h_tagged + at,
-                      m.blob ? silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t) : 0.f,
-                      (epoch << 7) | (uint32_t)l);
-          else if (m.blob)
-            a.h[at] = silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t);
+          if (m.blob) a.h[at] = silu(row_value(gA, baseA, 0, r, t)) * row_value(gA, baseA, 1, r, t);
         }
       }
-      // the fused mode's h carries its own tag: no counter to publish
-      if (fused) __syncthreads(); else cta_arrive(&sy[0]);
+      cta_arrive(&sy[0]);
     }
     // without a down phase, the next layer's first gate/up tile goes out now
     if (!haveB && nextA) {
@@ -778,9 +669,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     }
     // ---------------- down (+ row-block combine) ----------------
     if (haveB) {
-      // every gate/up tile of this layer is done (the fused mode polls its
-      // tagged h instead)
-      if (!fused && !cta_wait_geq(&sy[0], tilesA, hd.abort, a.status)) {
+      // every gate/up tile of this layer is done
+      if (!cta_wait_geq(&sy[0], tilesA, hd.abort, a.status)) {
         drain();
         return;
       }
@@ -796,8 +686,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
         for (int t0 = 0; t0 < mb.m; t0 += kMT) {
           const int n = min(kMT, mb.m - t0);
           if (t0 > 0) __syncthreads();
-          if (fused) stage_h_tagged(gB, baseB, a.h_tagged, mb.tok + t0, n, (epoch << 7) | (uint32_t)l, hd.abort, a.status);
-          else stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
+          stage_x<false>(gB, baseB, a.h, mb.tok + t0, n);
           // buffer A is free since the gate/up phase: the next layer's first
           // gate/up tile streams in during the down compute
           if (i == b && t0 == 0 && nextA) issue_A(first[2 * (l + 1)]);
@@ -815,10 +704,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
             const int t = threadIdx.x >> gB.rlog, r = threadIdx.x & (gB.R - 1);
             a.y[(size_t)(mb.hbase + t0 + t) * H + mb.row0 + r] = mb.blob ? row_value(gB, baseB, 0, r, t) : 0.f;
           }
-        }
-        if (fused) {
-          cta_arrive(&sy[1]);
-          continue;
         }
         __syncthreads();
         if (threadIdx.x == kArriver) {
@@ -850,22 +735,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
     units = units_n;
   }
   cp_async_wait_all();
-  // fused combine: CTA 0 writes the last layer's output once its down tiles are done
-  if (fused && b == 0) {
-    const int L = a.n_layers;
-    __syncthreads();
-    load_combine(a.rec + L - 1);
-    if (!cta_wait_geq(a.sync + (size_t)(L - 1) * a.sync_stride + 1, units_of[L - 1] * nrbB, hd.abort, a.status)) return;
-    const int per = H / 4;
-    for (int i = threadIdx.x; i < a.T * per; i += kGemvThreads) {
-      const int t = i / per, q = i - t * per;
-      float v[4];
-      combine4(a.y, hd.cw, hd.cpos, t, q, H, a.T, a.k, a.n_shared, v);
-      __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-      reinterpret_cast<uint2*>(a.out + (size_t)t * H)[q] =
-          make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------

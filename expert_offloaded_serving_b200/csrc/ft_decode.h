@@ -110,11 +110,6 @@ struct StackArgs {
   float* y;                // [T*k + n_shared*T][H]
   int* sync;               // [n_layers][sync_stride], zero at launch
   int sync_stride;         // >= stack_sync_stride(H, I)
-  int fused;               // 1: each gate/up tile rebuilds its input from the previous layer's y (T <= 2)
-  // With fused: h travels tagged, [T*k + n_shared*T][I] words (tag << 32 | fp32 bits), and
-  // the down tiles poll it instead of a counter; the tag is (*epoch << 7) | layer.
-  uint64_t* h_tagged;
-  const uint32_t* epoch;   // advanced by the routing kernel before this launch
   int* status;
 };
 

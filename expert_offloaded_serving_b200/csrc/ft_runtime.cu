@@ -1546,9 +1546,6 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   // the counter-synchronised kernel computes MXFP4 weights only
   const bool persistent = !layerwise && !flow && c->d_sync != nullptr && c->d.weight_format == FT_FMT_MXFP4 &&
                           stack_supported(H, I, n_layers);
-  // with one or two tokens the counter-synchronised kernel folds the combine
-  // into the next layer and hands h over tagged (the tag holds the layer in 7 bits)
-  const bool fused = persistent && Ti <= 2 && n_layers <= 128;
   // all layers' routing records in one launch (their logits are inputs); it
   // also zeroes the counter-synchronised kernel's counters of those layers
   {
@@ -1558,7 +1555,7 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
       ra.sync = c->d_sync;
       ra.sync_stride = c->sync_stride;
     }
-    if (fused || flow) {
+    if (flow) {
       ra.epoch = c->d_epoch;
       ra.tagged = c->d_tagged;
       ra.tagged_words = c->tagged_words;
@@ -1615,9 +1612,6 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     a.y = c->d_y;
     a.sync = c->d_sync;
     a.sync_stride = c->sync_stride;
-    a.fused = fused ? 1 : 0;  // beyond two tokens the per-tile recombination costs more L2 reads than a hand-over
-    a.h_tagged = c->d_h_tagged;
-    a.epoch = c->d_epoch;
     a.status = c->d_status;
     KTimer kt(c, FT_K_DEC_STACK, s);
     CUDA_TRY(launch_dec_stack(a, s));

@@ -211,15 +211,16 @@ def expert_blob_nvfp4(seed: int, layer: int, expert: int, hidden: int, inter: in
 # wide-range MXFP4 blobs (parity tests of the extremes of the format)
 # ---------------------------------------------------------------------------
 # The matrices named in ``wide`` get codes uniform over all 16 e2m1 codes and
-# UE8M0 scale bytes uniform over 0 .. 254 (every finite scale, 2^-127 ..
-# 2^127); the other matrices keep the usual code histogram with their scale
-# bytes moved from SCALE_BASE +- 1 to ``narrow_base`` +- 1.  Pure byte draws
+# UE8M0 scale bytes uniform over ``wide_range`` (by default 0 .. 254: every
+# finite scale, 2^-127 .. 2^127); the other matrices keep the usual code
+# histogram with their scale bytes moved from SCALE_BASE +- 1 to
+# ``narrow_base`` +- 1.  Pure byte draws
 # from the same counter-based generator (stream region REGION_WIDE).
 REGION_WIDE = 4
 
 
 def expert_blob_wide(seed: int, layer: int, expert: int, hidden: int, inter: int,
-                     wide=("wg", "wu"), narrow_base: int = SCALE_BASE) -> np.ndarray:
+                     wide=("wg", "wu"), narrow_base: int = SCALE_BASE, wide_range=(0, 254)) -> np.ndarray:
     r = blob_regions(hidden, inter)
     blob = expert_blob(seed, layer, expert, hidden, inter)
     code_rng = {"wg": (r["wg"], r["wu"]), "wu": (r["wu"], r["wd"]), "wd": (r["wd"], r["codes_end"])}
@@ -239,7 +240,8 @@ def expert_blob_wide(seed: int, layer: int, expert: int, hidden: int, inter: int
             if (a, b) == code_rng[name]:
                 blob[a:b] = (f & np.uint64(0xFF)).astype(np.uint8)       # two uniform 4-bit codes
             else:
-                blob[a:b] = (f % np.uint64(255)).astype(np.uint8)        # 0 .. 254
+                lo, hi = wide_range                                       # 0 .. 254 by default
+                blob[a:b] = (np.uint64(lo) + f % np.uint64(hi - lo + 1)).astype(np.uint8)
     return blob
 
 

@@ -136,9 +136,8 @@ def test_injected_copy_failure_drops_the_key_and_a_retry_recovers():
 
 
 @pytest.mark.parametrize("T", [1, 2])
-@pytest.mark.parametrize("kernel", [0, ft.FT_STACK_COUNTERS], ids=["dataflow", "counters"])
-def test_tagged_words_are_zeroed_when_the_launch_counter_wraps(T, kernel):
-    """The persistent kernel's tagged hand-over words carry a tag (launch
+def test_tagged_words_are_zeroed_when_the_launch_counter_wraps(T):
+    """The dataflow stack kernel's tagged hand-over words carry a tag (launch
     counter << 7 | layer) that repeats every 2^25 launches.  Stale words of a
     launch 2^25 earlier would pass for the current launch's; the routing
     kernel zeroes every tagged word when the counter wraps.  Here each tagged
@@ -160,12 +159,12 @@ def test_tagged_words_are_zeroed_when_the_launch_counter_wraps(T, kernel):
             ft.ft_debug_stack_epoch(c.h, (1 << 25) - 1, poison)   # the next launch wraps
             for rep in range(3):
                 got = torch.empty_like(x)
-                ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, got, 1 | kernel)
+                ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, got, 1)
                 ft.ft_sync_status(c.h)
                 assert (bf16_bits(got) == want_b).all(), (poison, rep)
         ft.ft_debug_stack_epoch(c.h, (1 << 32) - 3)           # the 32-bit counter itself wraps too
         for rep in range(4):
             got = torch.empty_like(x)
-            ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, got, 1 | kernel)
+            ft.ft_moe_stack_forward(c.h, 0, L, x, T, lg, got, 1)
             ft.ft_sync_status(c.h)
             assert (bf16_bits(got) == want_b).all(), rep

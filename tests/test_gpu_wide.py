@@ -9,10 +9,11 @@ Two variants keep the outputs finite:
 * "gate_up": wide Wg and Wu; x ~ N(0, 1) * 2^-127 (mostly bf16 subnormals), so
   that a block scaled by 2^127 meets x of order 2^-127; Wd keeps the usual
   code histogram with scale bytes 109 .. 111.
-* "down": wide Wd; x ~ N(0, 1); Wg and Wu scale bytes 52 .. 54, so that h is
-  near 2^-110 and a Wd block scaled by 2^127 gives outputs of order 1.  The
-  prefill variant uses scale bytes 59 .. 61: MXFP4 cannot encode h much below
-  2^-127 (the block scale byte clamps at 0), and smaller h quantises to zero.
+* "down": wide Wd; x ~ N(0, 1); Wg and Wu scale bytes 65 .. 67, so that h
+  lies in 2^-120 .. 2^-106 (normal fp32 values: fp32 arithmetic would lose
+  bits below 2^-126) and a Wd block scaled by up to 2^127 meets it.  The
+  prefill variant uses scale bytes 69 .. 71 (h in 2^-111 .. 2^-94, within
+  MXFP4's range, whose block scale byte clamps at 0, i.e. 2^-127).
 One block near the top of the scale range dominates each row, so outputs span
 many binades; the layer tolerance is applied to the outputs divided by their
 largest magnitude (``assert_close_scaled``).
@@ -37,9 +38,9 @@ pytestmark = pytest.mark.gpu
 H, I, E, K, S = 2048, 512, 16, 8, 1
 VARIANTS = {
     "gate_up": dict(wide=("wg", "wu"), narrow_base=110, xstd=2.0 ** -127, seed=5101),
-    "down": dict(wide=("wd",), narrow_base=53, xstd=1.0, seed=5102),
+    "down": dict(wide=("wd",), narrow_base=66, xstd=1.0, seed=5102),
 }
-PREFILL_BASE = {"gate_up": 110, "down": 60}
+PREFILL_BASE = {"gate_up": 110, "down": 70}
 
 
 def blobs_of(variant, layer, narrow_base=None):
