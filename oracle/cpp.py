@@ -44,6 +44,8 @@ def lib() -> C.CDLL:
             "fto_lru_step": (C.c_int64, [P, C.c_int, P, C.c_int, P, C.c_int64]),
             "fto_lru_resize": (C.c_int64, [P, C.c_int64, P, C.c_int64]),
             "fto_lru_lookup": (C.c_int, [P, C.c_int, C.c_int]),
+            "fto_lru_set_prefetch": (None, [P, C.c_int, C.c_int, C.c_int]),
+            "fto_lru_prefetch_counts": (None, [P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -217,7 +219,7 @@ class LRUCache:
 
     def step(self, layer, experts) -> list[tuple]:
         e = np.ascontiguousarray(np.asarray(experts).reshape(-1), dtype=np.int32)
-        buf = np.empty((3 * e.size + 4, 5), np.int32)
+        buf = np.empty((3 * e.size + 4 + 2 * 16, 5), np.int32)
         n = lib().fto_lru_step(self.h, int(layer), _p(e), e.size, _p(buf), buf.shape[0])
         if n < 0:
             raise RuntimeError("more experts in one step than cache slots")
@@ -232,3 +234,24 @@ class LRUCache:
 
     def lookup(self, layer: int, expert: int) -> int:
         return lib().fto_lru_lookup(self.h, int(layer), int(expert))
+
+
+class PrefetchingLRUCache(LRUCache):
+    """``oracle.lru.PrefetchingLRUCache`` from the C++ oracle."""
+
+    def __init__(self, capacity: int, n_layers: int, n_experts: int, per_layer: int):
+        super().__init__(capacity)
+        lib().fto_lru_set_prefetch(self.h, n_layers, n_experts, per_layer)
+
+    def _counts(self):
+        out = np.zeros(2, np.int64)
+        lib().fto_lru_prefetch_counts(self.h, _p(out))
+        return int(out[0]), int(out[1])
+
+    @property
+    def prefetches(self) -> int:
+        return self._counts()[0]
+
+    @property
+    def prefetch_hits(self) -> int:
+        return self._counts()[1]

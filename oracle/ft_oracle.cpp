@@ -350,6 +350,11 @@ struct Lru {
   int64_t capacity;
   std::list<std::pair<int, int>> order;          // least recent first
   std::map<std::pair<int, int>, int> slot;
+  // decode-time next-layer prefetch (off while per_layer == 0)
+  int n_layers = 0, n_experts = 0, per_layer = 0;
+  std::vector<int64_t> count;                    // [layer][expert] steps whose set held the expert
+  std::map<std::pair<int, int>, int> unused;     // prefetched keys not hit yet
+  int64_t prefetches = 0, prefetch_hits = 0;
 };
 
 }  // namespace
@@ -510,7 +515,31 @@ FTO_API int fto_moe_layer(const uint16_t* x_bits, int T, int H, int I, int E, in
 // Events: (kind, layer, expert, slot, from_slot) with kind 0 HIT, 1 MISS,
 // 2 EVICT, 3 MOVE.
 
-FTO_API void* fto_lru_new(int64_t capacity) { return new Lru{capacity, {}, {}}; }
+FTO_API void* fto_lru_new(int64_t capacity) {
+  Lru* c = new Lru();
+  c->capacity = capacity;
+  return c;
+}
+
+// Decode-time next-layer prefetch (the numpy oracle's PrefetchingLRUCache):
+// after each step at layer l, the experts of layer (l + 1) % n_layers that
+// were selected at least once, most often first (ties to the lower id), are
+// inserted, up to per_layer of them, skipping resident ones; when full, the
+// victim is the least recent key neither in the step's set nor of that layer.
+// Events of kind 4 (PREFETCH).
+FTO_API void fto_lru_set_prefetch(void* h, int n_layers, int n_experts, int per_layer) {
+  Lru& c = *static_cast<Lru*>(h);
+  c.n_layers = n_layers;
+  c.n_experts = n_experts;
+  c.per_layer = per_layer;
+  c.count.assign((size_t)n_layers * n_experts, 0);
+}
+
+FTO_API void fto_lru_prefetch_counts(void* h, int64_t* out2) {
+  Lru& c = *static_cast<Lru*>(h);
+  out2[0] = c.prefetches;
+  out2[1] = c.prefetch_hits;
+}
 
 FTO_API void fto_lru_free(void* h) { delete static_cast<Lru*>(h); }
 
@@ -549,6 +578,7 @@ FTO_API int64_t fto_lru_step(void* h, int layer, const int32_t* experts, int n, 
       c.order.remove(key);
       c.order.push_back(key);
       emit(0, layer, e, it->second, -1);
+      if (c.unused.erase(key)) c.prefetch_hits++;
       continue;
     }
     int s;
@@ -559,6 +589,7 @@ FTO_API int64_t fto_lru_step(void* h, int layer, const int32_t* experts, int n, 
       c.order.erase(v);
       s = c.slot[victim];
       c.slot.erase(victim);
+      c.unused.erase(victim);
       emit(2, victim.first, victim.second, s, -1);
     } else {
       s = lowest_free(c);
@@ -566,6 +597,43 @@ FTO_API int64_t fto_lru_step(void* h, int layer, const int32_t* experts, int n, 
     c.slot[key] = s;
     c.order.push_back(key);
     emit(1, layer, e, s, -1);
+  }
+  if (c.n_layers <= 0) return ne;
+  for (int e : S) c.count[(size_t)layer * c.n_experts + e]++;
+  if (c.per_layer <= 0) return ne;
+  const int nl = (layer + 1) % c.n_layers;
+  std::vector<int> cand;
+  for (int e = 0; e < c.n_experts; e++)
+    if (c.count[(size_t)nl * c.n_experts + e] > 0) cand.push_back(e);
+  const int64_t* cnt = c.count.data() + (size_t)nl * c.n_experts;
+  std::stable_sort(cand.begin(), cand.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  int done = 0;
+  for (int e : cand) {
+    if (done >= c.per_layer) break;
+    const std::pair<int, int> key{nl, e};
+    if (c.slot.count(key)) continue;
+    int s;
+    if ((int64_t)c.order.size() == c.capacity) {
+      auto v = c.order.begin();
+      while (v != c.order.end() &&
+             ((v->first == layer && std::binary_search(S.begin(), S.end(), v->second)) || v->first == nl))
+        ++v;
+      if (v == c.order.end()) break;
+      const std::pair<int, int> victim = *v;
+      c.order.erase(v);
+      s = c.slot[victim];
+      c.slot.erase(victim);
+      c.unused.erase(victim);
+      emit(2, victim.first, victim.second, s, -1);
+    } else {
+      s = lowest_free(c);
+    }
+    c.slot[key] = s;
+    c.order.push_back(key);
+    c.unused[key] = 1;
+    c.prefetches++;
+    emit(4, nl, e, s, -1);
+    done++;
   }
   return ne;
 }
@@ -589,6 +657,7 @@ FTO_API int64_t fto_lru_resize(void* h, int64_t capacity, int32_t* ev, int64_t c
     c.order.pop_front();
     const int s = c.slot[victim];
     c.slot.erase(victim);
+    c.unused.erase(victim);
     emit(2, victim.first, victim.second, s, -1);
   }
   const int64_t old = c.capacity;

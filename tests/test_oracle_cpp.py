@@ -296,3 +296,18 @@ def test_lru_hit_rate_one_when_everything_fits():
         assert all(ev[0] == lru.HIT for ev in c.step(layer_, e))
     with pytest.raises(RuntimeError):
         cpp.LRUCache(2).step(0, [1, 2, 3])
+
+
+@pytest.mark.parametrize("per_layer", [0, 1, 2])
+def test_prefetching_lru_equals_the_numpy_oracle(per_layer):
+    rng = np.random.default_rng(12 + per_layer)
+    a = cpp.PrefetchingLRUCache(10, 4, 16, per_layer)
+    b = lru.PrefetchingLRUCache(10, 4, 16, per_layer)
+    for step in range(400):
+        if step == 150:
+            assert a.resize(5) == b.resize(5)
+        if step == 260:
+            assert a.resize(10) == b.resize(10)
+        experts = rng.choice(16, int(rng.integers(1, 4)), replace=False)
+        assert a.step(step % 4, experts) == b.step(step % 4, experts), step
+    assert (a.prefetches, a.prefetch_hits) == (b.prefetches, b.prefetch_hits)
