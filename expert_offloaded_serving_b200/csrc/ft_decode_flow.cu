@@ -65,7 +65,8 @@ struct FlowPair {
   float w;        // combine weight
   uint8_t unit;   // unit holding the pair's expert
   uint8_t slot;   // the pair's token slot within that unit
-  uint8_t pad[2];
+  uint8_t on;     // the expert's blob is present (else its y counts as zero)
+  uint8_t pad;
 };
 static_assert(sizeof(FlowPair) == 8, "FlowPair");
 
@@ -149,37 +150,49 @@ __device__ __forceinline__ void stage_x_tagged(const Gv& g, uint8_t* base, const
 }
 
 // The down tile's activations: every h row 0 .. nh-1 of the layer (all
-// units), from the tagged h words, re-encoded like stage_x.
+// units), from the tagged h words, re-encoded like stage_x.  Each thread
+// loads up to kHBatch items before it looks at any tag, so the L2 round
+// trips of its items overlap.
+constexpr int kHBatch = 4;
 __device__ __forceinline__ void stage_h_all(const Gv& g, uint8_t* base, const uint64_t* ht, int nh, uint32_t tag,
                                             int& abort, int* status) {
   const int per = g.K / 4;
   const int items = nh * per;  // a multiple of 32: warps stay whole for encode4's shuffles
-  for (int i = threadIdx.x; i < items; i += kGemvThreads) {
-    const int t = i / per, q = i - t * per;
-    const uint64_t* p = ht + (size_t)t * g.K + 4 * q;
-    uint64_t w[4];
-    ld_tagged4(p, w);
-    auto ready = [&]() {
-      return (uint32_t)(w[0] >> 32) == tag && (uint32_t)(w[1] >> 32) == tag && (uint32_t)(w[2] >> 32) == tag &&
-             (uint32_t)(w[3] >> 32) == tag;
-    };
-    if (!ready()) {
-      const uint64_t t0 = gclock();
-      for (;;) {
-        __nanosleep(20);
-        ld_tagged4(p, w);
-        if (ready()) break;
-        if (gclock() - t0 > kSpinNs) {
-          set_status(status, kStTimeout);
-          abort = 1;
-          break;
+  for (int i0 = 0; i0 < items; i0 += kHBatch * kGemvThreads) {
+    uint64_t w[kHBatch][4];
+#pragma unroll
+    for (int j = 0; j < kHBatch; j++) {
+      const int i = i0 + j * kGemvThreads + threadIdx.x;
+      if (i < items) ld_tagged4(ht + (size_t)(i / per) * g.K + 4 * (i % per), w[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kHBatch; j++) {
+      const int i = i0 + j * kGemvThreads + threadIdx.x;
+      if (i >= items) break;
+      const int t = i / per, q = i - t * per;
+      auto ready = [&]() {
+        return (uint32_t)(w[j][0] >> 32) == tag && (uint32_t)(w[j][1] >> 32) == tag &&
+               (uint32_t)(w[j][2] >> 32) == tag && (uint32_t)(w[j][3] >> 32) == tag;
+      };
+      if (!ready()) {
+        const uint64_t* p = ht + (size_t)t * g.K + 4 * q;
+        const uint64_t t0 = gclock();
+        for (;;) {
+          __nanosleep(20);
+          ld_tagged4(p, w[j]);
+          if (ready()) break;
+          if (gclock() - t0 > kSpinNs) {
+            set_status(status, kStTimeout);
+            abort = 1;
+            break;
+          }
         }
       }
-    }
-    float v[4];
+      float v[4];
 #pragma unroll
-    for (int j = 0; j < 4; j++) v[j] = __uint_as_float((uint32_t)w[j]);
-    encode4(g, base, t, q, v);
+      for (int e = 0; e < 4; e++) v[e] = __uint_as_float((uint32_t)w[j][e]);
+      encode4(g, base, t, q, v);
+    }
   }
 }
 
@@ -321,7 +334,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         q.w = rec->w[f];
         q.unit = (uint8_t)u;
         q.slot = (uint8_t)(pos - rec->unit_p0[u]);
-        q.pad[0] = q.pad[1] = 0;
+        q.on = eptr[rec->unit_e[u]] != nullptr;
+        q.pad = 0;
         pr[f] = q;
       }
       if (lane == 0) {
@@ -438,6 +452,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
       if (i == b) stamp(1);
       tile_dots<F>(gA, lmA, baseA, f.m);
       __syncthreads();
+      if (i == b) stamp(7);
       if (threadIdx.x < gA.R * f.m) {
         const int t = threadIdx.x >> gA.rlog, r = threadIdx.x & (gA.R - 1);
         float gv = row_value(gA, baseA, 0, r, t), uv = row_value(gA, baseA, 1, r, t);
@@ -470,26 +485,47 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         if (T > 1) dtile_dots<2, F>(gB, lmB, baseB, un, lh.units, rb);
         else dtile_dots<1, F>(gB, lmB, baseB, un, lh.units, rb);
         __syncthreads();
+        if (d == b) stamp(5);
         const int n0 = d * rb, nv = min(rb, H - n0), half = nv / 2;
         for (int i = threadIdx.x; i < T * half; i += kGemvThreads) {
           const int t = i / half, nl = 2 * (i - t * half);
-          float o[2];
+          float o[2] = {0.f, 0.f};
+          // the routed pairs four at a time: their loads first, then the
+          // multiply-adds in ascending j
+          for (int j0 = 0; j0 < k; j0 += 4) {
+            float w4[4], y4[4][2];
 #pragma unroll
-          for (int e = 0; e < 2; e++) {
-            float acc = 0.f;
-            for (int j = 0; j < k; j++) {
-              const FlowPair q = pr[t * k + j];
-              float y = un[q.unit].blob ? dtile_y(gB, baseB, q.unit * rb + nl + e, q.slot) : 0.f;
-              if (F == kFmtNv) y *= un[q.unit].ts[2];
-              acc = fmaf(q.w, y, acc);
+            for (int jj = 0; jj < 4; jj++) {
+              w4[jj] = 0.f;
+              y4[jj][0] = y4[jj][1] = 0.f;
+              if (j0 + jj < k) {
+                const FlowPair q = pr[t * k + j0 + jj];
+                w4[jj] = q.w;
+                const float ts = F == kFmtNv ? un[q.unit].ts[2] : 1.f;
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                  float y = q.on ? dtile_y(gB, baseB, q.unit * rb + nl + e, q.slot) : 0.f;
+                  if (F == kFmtNv) y *= ts;
+                  y4[jj][e] = y;
+                }
+              }
             }
-            for (int s2 = 0; s2 < S; s2++) {
-              const int u = na + s2;
-              float y = un[u].blob ? dtile_y(gB, baseB, u * rb + nl + e, t) : 0.f;
-              if (F == kFmtNv) y *= un[u].ts[2];
-              acc += y;
+#pragma unroll
+            for (int jj = 0; jj < 4; jj++)
+              if (j0 + jj < k)
+#pragma unroll
+                for (int e = 0; e < 2; e++) o[e] = fmaf(w4[jj], y4[jj][e], o[e]);
+          }
+          for (int s2 = 0; s2 < S; s2++) {
+            const int u = na + s2;
+            const bool on = un[u].blob != nullptr;
+            const float ts = F == kFmtNv ? un[u].ts[2] : 1.f;
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+              float y = on ? dtile_y(gB, baseB, u * rb + nl + e, t) : 0.f;
+              if (F == kFmtNv) y *= ts;
+              o[e] += y;
             }
-            o[e] = acc;
           }
           __nv_bfloat162 bb = __floats2bfloat162_rn(o[0], o[1]);
           const uint32_t pairbits = *reinterpret_cast<uint32_t*>(&bb);
@@ -497,6 +533,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
           if (last) reinterpret_cast<uint32_t*>(a.out)[at / 2] = pairbits;
           else st_tagged_raw(a.x_tagged + at / 2, ((uint64_t)((epoch << 7) | (uint32_t)(l + 1)) << 32) | pairbits);
         }
+        if (d == b) stamp(6);
         __syncthreads();
       }
     }

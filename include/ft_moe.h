@@ -404,11 +404,13 @@ FT_API ft_status ft_debug_stack_epoch(ft_ctx* ctx, uint32_t epoch, int32_t poiso
 /* Phase timeline of the dataflow stack kernel, for profiling: with buf (dev
  * uint64 [n_words]) attached, each later ft_moe_stack_forward that runs the
  * dataflow kernel over n layers with at least n * (number of SMs) * 8 words
- * writes, at [layer][CTA][0..4], the %globaltimer nanoseconds at which the
- * CTA began the layer, had its first gate/up tile's input and weights, had
- * published its h, had its first down tile's h and weights, and had
- * published its part of the next layer's input (0 where the CTA had no tile
- * of that phase).  NULL detaches it.  The kernel's results do not change. */
+ * writes, at [layer][CTA][0..7], the %globaltimer nanoseconds at which the
+ * CTA began the layer [0], had its first gate/up tile's input and weights
+ * [1], had that tile's dot products [7], had published its h [2], had its
+ * first down tile's h and weights [3], had that tile's dot products [5],
+ * had stored its combined rows [6] and had left the down phase [4] (0 where
+ * the CTA had no tile of that phase).  NULL detaches it.  The kernel's
+ * results do not change. */
 FT_API ft_status ft_debug_stack_timeline(ft_ctx* ctx, uint64_t* buf, int64_t n_words);
 FT_API ft_status ft_debug_host_wait_limit(ft_ctx* ctx, double seconds);
 FT_API ft_status ft_debug_fail_copy(ft_ctx* ctx, int64_t n);

@@ -46,7 +46,9 @@ def test_glm_class_prefill_2048_tokens_every_row():
 def test_glm_class_cache_trace_and_outputs():
     """3 layers with the slice's slot share (24 GiB = 1285 slots over 8
     layers, scaled to 3: 481 slots), 32 tokens of a Zipf(1.1) / 0.6-overlap
-    trace, budget halved at token 12 and restored at token 24; the last step's
+    trace.  The 32 tokens touch fewer distinct experts than that share, so the
+    budget is cut to 48 slots at token 12 (evicting down to the 48 most recent
+    keys, then every miss evicts) and restored at token 24; the last step's
     output against the oracle on its own input."""
     L, n_tok = 3, 32
     stride = synth.blob_stride(H, I)
