@@ -129,11 +129,11 @@ __device__ __forceinline__ void stage_x_tagged(const Gv& g, uint8_t* base, const
       ld_tagged2(p, w0, w1);
       if ((uint32_t)(w0 >> 32) != tag || (uint32_t)(w1 >> 32) != tag) {
         const uint64_t t0 = gclock();
-        for (;;) {
+        for (uint32_t n = 1;; n++) {
           __nanosleep(20);
           ld_tagged2(p, w0, w1);
           if ((uint32_t)(w0 >> 32) == tag && (uint32_t)(w1 >> 32) == tag) break;
-          if (gclock() - t0 > kSpinNs) {
+          if ((n & 15) == 0 && gclock() - t0 > kSpinNs) {
             set_status(status, kStTimeout);
             abort = 1;
             break;
@@ -177,11 +177,11 @@ __device__ __forceinline__ void stage_h_all(const Gv& g, uint8_t* base, const ui
       if (!ready()) {
         const uint64_t* p = ht + (size_t)t * g.K + 4 * q;
         const uint64_t t0 = gclock();
-        for (;;) {
+        for (uint32_t n = 1;; n++) {
           __nanosleep(20);
           ld_tagged4(p, w[j]);
           if (ready()) break;
-          if (gclock() - t0 > kSpinNs) {
+          if ((n & 15) == 0 && gclock() - t0 > kSpinNs) {
             set_status(status, kStTimeout);
             abort = 1;
             break;

@@ -4,21 +4,31 @@
 //
 // Swap-AB: weights are the M = 128 side (rows of Wg/Wu or Wd), tokens the
 // N = 128 side, so experts with ~100 tokens fill an MMA without padding the
-// large weight dimension.  Per CTA (128 weight rows x 128 padded token rows of
-// one expert):
+// large weight dimension.  A tile is (128 weight rows) x (128 padded token
+// rows of one expert).
+//
+// Persistent: one CTA per SM walks the tiles i = CTA, CTA + grid, ...; tile i
+// is token tile i / (M/128) and weight tile i % (M/128), so the CTAs running
+// at the same time share a few token tiles and the weight tiles of one or two
+// experts through L2.  Roles, one CTA of 18 warps:
 //   warp 0, one thread   TMA loads of the K-stage tiles (128B-swizzled,
 //                        cp.async.bulk.tensor) and bulk copies of the matching
-//                        scale atoms, on a ring of kStages shared-memory stages
+//                        scale atoms into a ring of kStages shared-memory
+//                        stages; it runs ahead across tile boundaries
 //   warp 1, one thread   tcgen05.cp of the scale atoms into tensor memory and
 //                        tcgen05.mma (K = 64 per instruction); tcgen05.commit
-//                        frees a stage and finally signals the accumulators
-//   warps 0..15          epilogue from tensor memory (tcgen05.ld): warp w reads
-//                        TMEM lanes 32(w%4).. (its weight rows) and every
-//                        fourth 16-column group of tokens from 16(w/4): SwiGLU
-//                        and MXFP4 quantisation of h (gate/up), or fp32 y (down)
-// All mbarrier waits are bounded; on a timeout the CTA records the TIMEOUT
-// status, stops issuing, waits (bounded) for its copies still in flight, frees
-// its tensor memory and returns.
+//                        frees a stage, and marks a tile's accumulators full
+//   warps 2..17          epilogue: warp w reads TMEM lanes 32(w%4).. (its 32
+//                        weight rows) and 32 token columns from
+//                        32((w-2)/4), frees the accumulators as soon as its
+//                        values are in registers, then SwiGLU and MXFP4
+//                        quantisation of h (gate/up), or fp32 y (down)
+// The down GEMM double-buffers its accumulator in tensor memory; gate/up (two
+// 128-column accumulators) has one buffer, which its epilogue releases right
+// after the tensor-memory loads, so the next tile's MMAs wait only for those
+// loads.  All mbarrier waits are bounded; on a timeout the CTA records the
+// TIMEOUT status, stops issuing, waits (bounded) for its copies and tensor
+// operations still in flight, frees its tensor memory and returns.
 //
 // Pages: prefill computes a whole layer's experts over many tokens while the
 // next layer's experts cross PCIe (aipolix.com, paragraph on bandwidth-
@@ -34,13 +44,59 @@ namespace ft {
 using namespace tc;
 namespace {
 
-constexpr int kThreads = 512;    // 16 warps: warps w, w+4, w+8, w+12 share TMEM lanes 32(w%4).. in the epilogue
-constexpr int kEpiGroups = kThreads / 128;  // column groups of the epilogue
-constexpr int kStagesGU = 3;     // gate/up: 2 weight tiles + 1 token tile per stage
-constexpr int kStagesDn = 4;     // down: 1 + 1
+constexpr int kWarps = 18;                 // producer, MMA issuer, 16 epilogue warps
+constexpr int kThreads = 32 * kWarps;
+constexpr int kEpiWarp0 = 2;               // first epilogue warp
+constexpr int kEpiWarps = kWarps - kEpiWarp0;
+constexpr int kStagesGU = 4;     // gate/up: 2 weight tiles + 1 token tile per stage (51 KB)
+constexpr int kStagesDn = 6;     // down: 1 + 1 (34 KB)
 constexpr int kTileBytes = kGemmBM * kGemmBK / 2;   // 16 KB of e2m1 codes
 constexpr int kSfBytes = 1024;                      // two 512-byte scale atoms
 constexpr int kTmemCols = 512;
+constexpr int kAccCols = 2 * kGemmBN;               // accumulator columns: gate + up, or two down buffers
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s_u32(b)) : "memory");
+}
+
+// 16 columns of 32-bit TMEM values of this warp's lanes, without the wait.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// Wait for this thread's tensor-memory loads; the registers are tied to the
+// wait so that no use of them moves above it.
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+
+// silu(z) = z / (1 + e^-z) with the fast exponential and division (h is
+// quantised to MXFP4 right after, so a few ulp do not matter).
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// Lane-wise unsigned maximum of two 16-bit halves.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Expert segment holding padded token row row0 (segments are 128-row aligned).
+__device__ __forceinline__ int segment_of(const GemmArgs& a, int row0) {
+  int lo = 0, hi = a.n_segments - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.pad_offs[mid] <= row0) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
 
 // ---------------------------------------------------------------------------
 // the kernel.  MODE 0: gate/up (two weight matrices, SwiGLU, MXFP4 h);
@@ -51,6 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
                                                       const __grid_constant__ GemmMaps maps) {
   constexpr int S = MODE == 0 ? kStagesGU : kStagesDn;
   constexpr int NA = MODE == 0 ? 2 : 1;
+  constexpr int NB = MODE == 0 ? 1 : 2;   // accumulator buffers
+  constexpr int SFC = 8 * (NA + 1);       // scale columns per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tileA = smem;                              // [S][NA] 16 KB, 1024-aligned
@@ -59,20 +117,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
   uint8_t* sfB = sfA + S * NA * kSfBytes;             // [S] 1 KB
   uint64_t* full = reinterpret_cast<uint64_t*>(sfB + S * kSfBytes);
   uint64_t* empty = full + S;
-  uint64_t* accb = empty + S;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accb + 1);
+  uint64_t* acc_full = empty + S;                     // [NB] MMA -> epilogue
+  uint64_t* acc_empty = acc_full + NB;                // [NB] epilogue (one arrive per warp) -> MMA
+  uint64_t* fin = acc_empty + NB;                     // the MMA thread's last operations
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fin + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, jt = blockIdx.y;
-  const int row0 = jt * kGemmBN;
-  if (row0 >= a.pad_offs[a.n_segments]) return;
-  // expert segment holding this token tile (segments are 128-row aligned)
-  int lo = 0, hi = a.n_segments - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.pad_offs[mid] <= row0) lo = mid; else hi = mid - 1;
-  }
-  const int e = lo;
+  const int n_mt = a.M / kGemmBM;
+  const int n_jt = min(a.n_tiles_max, a.pad_offs[a.n_segments] / kGemmBN);
+  const int n_tiles = n_mt * n_jt;
+  if ((int)blockIdx.x >= n_tiles) return;  // the whole CTA, before any barrier or allocation
   const int KT = a.K / kGemmBK;
   const int atoms_k = a.K / 128;
 
@@ -81,7 +136,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accb, 1);
+    for (int b = 0; b < NB; b++) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    mbar_init(fin, 1);
+    *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -94,116 +154,182 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t d0 = tmem;                 // accumulator of matrix 0: columns [0, 128)
-  const uint32_t d1 = tmem + kGemmBN;       // accumulator of matrix 1: [128, 256)
-  const uint32_t sf0 = tmem + 2 * kGemmBN;  // per stage 24 scale columns: A0 +0, A1 +8, B +16
+  const uint32_t sf0 = tmem + kAccCols;  // per stage SFC scale columns: A0 +0, A1 +8 (gate/up), B +8*NA
 
-  if (warp == 0 && lane == 0) {
-    // ---- producer ----
-    const uint8_t* blob = a.pool + (int64_t)e * a.blob_stride;
-    const uint32_t bytes = (NA + 1) * (kTileBytes + kSfBytes);
-    int issued = 0;  // K stages whose copies went out
-    for (int kt = 0; kt < KT; kt++) {
-      const int s = kt % S;
-      if (kt >= S && !mbar_wait(&empty[s], ((kt / S) - 1) & 1)) {
-        set_status(a.status, kStTimeout);
-        break;
-      }
-      mbar_expect(&full[s], bytes);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer ----
+      const uint32_t bytes = (NA + 1) * (kTileBytes + kSfBytes);
+      int issued = 0;  // K stages whose copies went out, over all tiles
+      for (int i = blockIdx.x; i < n_tiles && !*abort_flag; i += gridDim.x) {
+        const int jt = i / n_mt, mt = i - jt * n_mt, row0 = jt * kGemmBN;
+        const int e = segment_of(a, row0);
+        const uint8_t* blob = a.pool + (int64_t)e * a.blob_stride;
+        bool ok = true;
+        for (int kt = 0; kt < KT; kt++) {
+          const int s = issued % S;
+          if (issued >= S && !mbar_wait(&empty[s], ((issued / S) - 1) & 1)) {
+            set_status(a.status, kStTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          mbar_expect(&full[s], bytes);
 #pragma unroll
-      for (int q = 0; q < NA; q++) {
-        tma_3d(tileA + (s * NA + q) * kTileBytes, &maps.a[q], kt * (kGemmBK / 2), mt * kGemmBM, e, &full[s]);
-        bulk_g2s(sfA + (s * NA + q) * kSfBytes, blob + a.sfa_off[q] + ((int64_t)mt * atoms_k + 2 * kt) * 512,
-                 kSfBytes, &full[s]);
+          for (int q = 0; q < NA; q++) {
+            tma_3d(tileA + (s * NA + q) * kTileBytes, &maps.a[q], kt * (kGemmBK / 2), mt * kGemmBM, e, &full[s]);
+            bulk_g2s(sfA + (s * NA + q) * kSfBytes, blob + a.sfa_off[q] + ((int64_t)mt * atoms_k + 2 * kt) * 512,
+                     kSfBytes, &full[s]);
+          }
+          tma_2d(tileB + s * kTileBytes, &maps.b, kt * (kGemmBK / 2), row0, &full[s]);
+          bulk_g2s(sfB + s * kSfBytes, a.sfb + ((int64_t)jt * atoms_k + 2 * kt) * 512, kSfBytes, &full[s]);
+          issued++;
+        }
+        if (!ok) break;
       }
-      tma_2d(tileB + s * kTileBytes, &maps.b, kt * (kGemmBK / 2), row0, &full[s]);
-      bulk_g2s(sfB + s * kSfBytes, a.sfb + ((int64_t)jt * atoms_k + 2 * kt) * 512, kSfBytes, &full[s]);
-      issued = kt + 1;
+      // No copy may still be writing this CTA's shared memory when it exits,
+      // also after a timeout of any role.  A stage is reissued only after the
+      // MMA consumed its previous round, so only the last S issued stages can
+      // be in flight; without a timeout the MMA thread has waited for the
+      // same phases, so these waits succeed at once.
+      for (int n = issued > S ? issued - S : 0; n < issued; n++) mbar_wait(&full[n % S], (n / S) & 1);
     }
-    // No copy may still be writing this CTA's shared memory when it exits,
-    // also after a timeout of either role.  A stage is reissued only after
-    // the MMA consumed its previous round, so only the last S issued stages
-    // can be in flight; without a timeout the MMA thread has waited for the
-    // same phases, so these waits succeed at once.
-    for (int kt = issued > S ? issued - S : 0; kt < issued; kt++) mbar_wait(&full[kt % S], (kt / S) & 1);
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ----
-    for (int kt = 0; kt < KT; kt++) {
-      const int s = kt % S;
-      if (!mbar_wait(&full[s], (kt / S) & 1)) {
-        set_status(a.status, kStTimeout);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      int consumed = 0, tcount = 0;
+      for (int i = blockIdx.x; i < n_tiles && !*abort_flag; i += gridDim.x, tcount++) {
+        const int b = tcount % NB, use = tcount / NB;
+        if (use > 0 && !mbar_wait(&acc_empty[b], (use - 1) & 1)) {
+          set_status(a.status, kStTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem + (uint32_t)(b * kGemmBN);  // gate/up: d0 = gate, d0 + 128 = up
+        bool ok = true;
+        for (int kt = 0; kt < KT; kt++) {
+          const int s = consumed % S;
+          if (!mbar_wait(&full[s], (consumed / S) & 1)) {
+            set_status(a.status, kStTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfs = sf0 + s * SFC;
+#pragma unroll
+          for (int q = 0; q < NA; q++)
+#pragma unroll
+            for (int at = 0; at < 2; at++)
+              utccp_32x128(sfs + q * 8 + 4 * at, desc_sf(sfA + (s * NA + q) * kSfBytes + at * 512));
+#pragma unroll
+          for (int at = 0; at < 2; at++) utccp_32x128(sfs + 8 * NA + 4 * at, desc_sf(sfB + s * kSfBytes + at * 512));
+          const uint64_t bd = desc_sw128(tileB + s * kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 64; kk++) {
+            const uint32_t byte = 2u * (kk & 1), col = 4u * (kk >> 1);
+            const uint32_t idesc = idesc_mxf4(byte, byte, kGemmBM, kGemmBN);
+#pragma unroll
+            for (int q = 0; q < NA; q++) {
+              const uint64_t ad = desc_sw128(tileA + (s * NA + q) * kTileBytes) + (uint64_t)(kk * 2);  // +32 B of K
+              mma_mxf4(d0 + (uint32_t)(q * kGemmBN), ad, bd + (uint64_t)(kk * 2), idesc,
+                       (sfs + q * 8 + col) | (byte << 30), (sfs + 8 * NA + col) | (byte << 30),
+                       (kt | kk) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty[s]);
+          consumed++;
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[b]);
+      }
+      // every tensor operation this thread issued has completed before the
+      // CTA frees its tensor memory
+      umma_commit(fin);
+      mbar_wait(fin, 0);
+    }
+  } else {
+    // ---- epilogue: warp w owns TMEM lanes 32(w%4).. = weight rows, and the
+    // token columns [32 cg, 32 cg + 32), cg = (w - 2) / 4 ----
+    const int quad = warp & 3, cg = (warp - kEpiWarp0) >> 2;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    int tcount = 0;
+    for (int i = blockIdx.x; i < n_tiles; i += gridDim.x, tcount++) {
+      const int b = tcount % NB, use = tcount / NB;
+      if (!mbar_wait_warp(&acc_full[b], use & 1)) {
+        if (lane == 0) set_status(a.status, kStTimeout);
         break;
       }
       tc_fence_after();
-      const uint32_t sfs = sf0 + s * 24;
+      const int jt = i / n_mt, mt = i - jt * n_mt, row0 = jt * kGemmBN;
+      const uint32_t d0 = tmem + (uint32_t)(b * kGemmBN) + lane_off + (uint32_t)(32 * cg);
+      if (MODE == 0) {
+        uint32_t g0[16], g1[16], u0[16], u1[16];
+        tmem_ld16_async(d0, g0);
+        tmem_ld16_async(d0 + 16, g1);
+        tmem_ld16_async(d0 + kGemmBN, u0);
+        tmem_ld16_async(d0 + kGemmBN + 16, u1);
+        tmem_wait16(g0);
+        tmem_wait16(g1);
+        tmem_wait16(u0);
+        tmem_wait16(u1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        const int I = a.M;
+        const int irow = mt * kGemmBM + quad * 32 + lane;
+        const int atoms_i = I / 128;
+        // column q is padded row p = row0 + 32 cg + q: its codes at p * I/2 +
+        // irow/2, the scale of its block 4 mt + quad at atom (jt, mt), byte
+        // (p % 32) * 16 + ((p / 32) % 4) * 4 + quad = q * 16 + cg * 4 + quad
+        uint8_t* hq_col = a.hq + (size_t)(row0 + 32 * cg) * (I / 2) + (irow >> 1);
+        uint8_t* sf_col = a.hq_sf + ((int64_t)jt * atoms_i + mt) * 512 + cg * 4 + quad;
 #pragma unroll
-      for (int q = 0; q < NA; q++)
+        for (int q = 0; q < 32; q += 2) {
+          float hv[2];
 #pragma unroll
-        for (int at = 0; at < 2; at++) utccp_32x128(sfs + q * 8 + 4 * at, desc_sf(sfA + (s * NA + q) * kSfBytes + at * 512));
+          for (int e = 0; e < 2; e++) {
+            const int c = q + e;
+            const float g = __uint_as_float(c < 16 ? g0[c & 15] : g1[c & 15]);
+            const float u = __uint_as_float(c < 16 ? u0[c & 15] : u1[c & 15]);
+            hv[e] = silu_fast(g) * u;
+          }
+          // the block maxima of both columns at once: the top 16 bits of |h|
+          // keep its exponent field, which is all the scale rule reads
+          uint32_t m = ((__float_as_uint(hv[0]) >> 16) & 0x7fffu) | (__float_as_uint(hv[1]) & 0x7fff0000u);
 #pragma unroll
-      for (int at = 0; at < 2; at++) utccp_32x128(sfs + 16 + 4 * at, desc_sf(sfB + s * kSfBytes + at * 512));
-      const uint64_t bd = desc_sw128(tileB + s * kTileBytes);
+          for (int d = 16; d >= 1; d >>= 1) m = max_u16x2(m, __shfl_xor_sync(0xffffffffu, m, d));
 #pragma unroll
-      for (int kk = 0; kk < kGemmBK / 64; kk++) {
-        const uint32_t byte = 2u * (kk & 1), col = 4u * (kk >> 1);
-        const uint32_t idesc = idesc_mxf4(byte, byte, kGemmBM, kGemmBN);
-#pragma unroll
-        for (int q = 0; q < NA; q++) {
-          const uint64_t ad = desc_sw128(tileA + (s * NA + q) * kTileBytes) + (uint64_t)(kk * 2);  // +32 bytes of K
-          mma_mxf4(q == 0 ? d0 : d1, ad, bd + (uint64_t)(kk * 2), idesc, (sfs + q * 8 + col) | (byte << 30),
-                   (sfs + 16 + col) | (byte << 30), (kt | kk) != 0 ? 1u : 0u);
+          for (int e = 0; e < 2; e++) {
+            const int be = (int)(((e ? m >> 16 : m) & 0x7fffu) >> 7);  // biased exponent of the block maximum
+            const int e8 = min(max(be - 2, 0), 254);
+            const float v = hv[e] * mx_inv_scale(e8);
+            const float nb = __shfl_xor_sync(0xffffffffu, v, 1);
+            if ((lane & 1) == 0) hq_col[(size_t)(q + e) * (I / 2)] = (uint8_t)cvt_e2m1x2(v, nb);
+            if (lane == 0) sf_col[(q + e) * 16] = (uint8_t)e8;
+          }
         }
-      }
-      umma_commit(&empty[s]);
-    }
-    umma_commit(accb);
-  }
-  __syncwarp();
-
-  // ---- epilogue: warp w owns TMEM lanes 32(w%4).. = weight rows and the
-  // token columns 16 * (w/4 + kEpiGroups * j) ----
-  const bool have = mbar_wait_warp(accb, 0);
-  if (!have && threadIdx.x == 0) set_status(a.status, kStTimeout);
-  const int quad = warp & 3, cg = warp >> 2;
-  if (have) {
-    tc_fence_after();
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    if (MODE == 0) {
-      const int I = a.M;
-      const int irow = mt * kGemmBM + quad * 32 + lane;
-      const int atoms_i = I / 128;
-      for (int c0 = 16 * cg; c0 < kGemmBN; c0 += 16 * kEpiGroups) {
-        float g[16], u[16];
-        tmem_ld16(d0 + lane_off + c0, g);
-        tmem_ld16(d1 + lane_off + c0, u);
+      } else {
+        uint32_t v0[16], v1[16];
+        tmem_ld16_async(d0, v0);
+        tmem_ld16_async(d0 + 16, v1);
+        tmem_wait16(v0);
+        tmem_wait16(v1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        const int H = a.M;
+        const int hrow = mt * kGemmBM + quad * 32 + lane;
+        const int e = segment_of(a, row0);
+        const bool shared = e >= a.E;
+        const int valid = shared ? a.T : a.offs[e + 1] - a.offs[e];
+        const int base_pos = shared ? a.T * a.k + (e - a.E) * a.T : a.offs[e];
+        const int r0 = row0 - a.pad_offs[e] + 32 * cg;
 #pragma unroll
-        for (int q = 0; q < 16; q++) {
-          const int p = row0 + c0 + q;
-          const float hv = silu(g[q]) * u[q];
-          float amax = fabsf(hv);
-#pragma unroll
-          for (int d = 16; d >= 1; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-          const int e8 = mx_scale_byte(amax);
-          const float v = hv * mx_inv_scale(e8);
-          const float nb = __shfl_xor_sync(0xffffffffu, v, 1);
-          if ((lane & 1) == 0) a.hq[(size_t)p * (I / 2) + (irow >> 1)] = (uint8_t)cvt_e2m1x2(v, nb);
-          if (lane == 0) a.hq_sf[sf_word(p, mt, atoms_i) + quad] = (uint8_t)e8;
-        }
-      }
-    } else {
-      const int H = a.M;
-      const int hrow = mt * kGemmBM + quad * 32 + lane;
-      const bool shared = e >= a.E;
-      const int valid = shared ? a.T : a.offs[e + 1] - a.offs[e];
-      const int base_pos = shared ? a.T * a.k + (e - a.E) * a.T : a.offs[e];
-      const int r0 = row0 - a.pad_offs[e];
-      for (int c0 = 16 * cg; c0 < kGemmBN; c0 += 16 * kEpiGroups) {
-        float v[16];
-        tmem_ld16(d0 + lane_off + c0, v);
-#pragma unroll
-        for (int q = 0; q < 16; q++) {
-          const int r = r0 + c0 + q;
-          if (r < valid) a.y[(size_t)(base_pos + r) * H + hrow] = v[q];
+        for (int q = 0; q < 32; q++) {
+          const int r = r0 + q;
+          if (r < valid) a.y[(size_t)(base_pos + r) * H + hrow] = __uint_as_float(q < 16 ? v0[q & 15] : v1[q & 15]);
         }
       }
     }
@@ -219,20 +345,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
 }  // namespace
 
 size_t gemm_smem_bytes(int mode) {
-  const int S = mode == 0 ? kStagesGU : kStagesDn, NA = mode == 0 ? 2 : 1;
-  return 1024 + (size_t)S * (NA + 1) * (kTileBytes + kSfBytes) + (2 * S + 1) * 8 + 16;
+  const int S = mode == 0 ? kStagesGU : kStagesDn, NA = mode == 0 ? 2 : 1, NB = mode == 0 ? 1 : 2;
+  return 1024 + (size_t)S * (NA + 1) * (kTileBytes + kSfBytes) + (2 * S + 2 * NB + 1) * 8 + 16;
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, const GemmMaps& maps, cudaStream_t s) {
-  dim3 grid(a.M / kGemmBM, a.n_tiles_max);
   if (a.n_tiles_max <= 0) return cudaSuccess;
+  int dev = 0, nsm = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const int tiles = (a.M / kGemmBM) * a.n_tiles_max;
+  const dim3 grid(tiles < nsm ? tiles : nsm);
   if (a.mode == 0) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(0));
-    if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(0))) !=
+        cudaSuccess)
+      return e;
     k_gemm<0><<<grid, kThreads, gemm_smem_bytes(0), s>>>(a, maps);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(1));
-    if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(1))) !=
+        cudaSuccess)
+      return e;
     k_gemm<1><<<grid, kThreads, gemm_smem_bytes(1), s>>>(a, maps);
   }
   return cudaGetLastError();

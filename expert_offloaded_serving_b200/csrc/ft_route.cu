@@ -52,77 +52,106 @@ __global__ void __launch_bounds__(256) k_router_logits(const uint16_t* __restric
 }
 
 // ---------------------------------------------------------------------------
-// router logits for many tokens: the same summation order, tiled.  A CTA of 8
-// warps takes 8 tokens x 32 experts; per 128-element block of K it stages the
-// block of x and of Wr in shared memory, converted to fp64 once (each x value
-// then serves 32 experts, each Wr value 8 tokens), element 4j + v of the block
-// at [v][j] so that lane j's reads are consecutive.  Warp w computes experts
-// 4w .. 4w+3 for all 8 tokens; lane j holds partial sum j of each of those
-// 32 (token, expert) pairs and adds its block elements 4j, 4j+1, 4j+2, 4j+3 in
-// ascending order, so every partial sum sees the same terms in the same
-// order as in k_router_logits; the butterfly and the rounding are the same.
+// router logits for many tokens: the same summation order, register-tiled.
+// A CTA of 8 warps takes 32 tokens x 16 experts; warp w takes tokens
+// 8(w/2) .. +7 and experts 8(w%2) .. +7, and lane j holds partial sum j of
+// each of its warp's 64 (token, expert) pairs in registers.  Per 128-element
+// block of K the CTA stages x (converted to fp64 once) and Wr (fp32, widened
+// at use) in shared memory, element 4j + v of the block at [v][j] so that
+// lane j's reads are consecutive; the next block's global loads are in
+// flight while the current one is used (two buffers).  Lane j adds its block
+// elements 4j, 4j+1, 4j+2, 4j+3 in ascending order, so every partial sum
+// sees the same terms in the same order as in k_router_logits; the
+// butterfly and the rounding are the same.
 // ---------------------------------------------------------------------------
-constexpr int kRtT = 8, kRtE = 32;
+constexpr int kRtT = 32, kRtE = 16;
+constexpr size_t kRtSmem = 2 * (size_t)(kRtT * 128 * 8 + kRtE * 128 * 4);
 
-__global__ void __launch_bounds__(256) k_router_logits_tiled(const uint16_t* __restrict__ x,
-                                                             const float* __restrict__ wr, int T, int H, int E,
-                                                             float* __restrict__ logits) {
-  __shared__ double xs[kRtT][4][32];
-  __shared__ double ws[kRtE][4][32];
+__global__ void __launch_bounds__(256, 1) k_router_logits_tiled(const uint16_t* __restrict__ x,
+                                                                const float* __restrict__ wr, int T, int H, int E,
+                                                                float* __restrict__ logits) {
+  extern __shared__ __align__(16) uint8_t rt_smem[];
+  double* xs = reinterpret_cast<double*>(rt_smem);                      // [2][kRtT][4][32]
+  float* ws = reinterpret_cast<float*>(rt_smem + 2 * kRtT * 128 * 8);   // [2][kRtE][4][32]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tw = warp >> 1, ew = warp & 1;
   const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
-  double acc[4][kRtT];
+  // staging: thread i loads elements 16(i%8) .. +15 of token i/8, and
+  // elements 8(i%16) .. +7 of expert i/16
+  const int st = threadIdx.x >> 3, sp = threadIdx.x & 7;
+  const int se = threadIdx.x >> 4, sq = threadIdx.x & 15;
+  const bool tok_ok = t0 + st < T, exp_ok = e0 + se < E;
+  const uint4* xg = reinterpret_cast<const uint4*>(x + (size_t)(tok_ok ? t0 + st : 0) * H) + 2 * sp;
+  const float4* wg = reinterpret_cast<const float4*>(wr + (size_t)(exp_ok ? e0 + se : 0) * H) + 2 * sq;
+  uint4 xr[2];
+  float4 wq[2];
+  auto gload = [&](int c) {
 #pragma unroll
-  for (int i = 0; i < 4; i++)
+    for (int i = 0; i < 2; i++) {
+      xr[i] = tok_ok ? __ldg(xg + c * 16 + i) : make_uint4(0u, 0u, 0u, 0u);
+      wq[i] = exp_ok ? __ldg(wg + c * 32 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto sstore = [&](int buf) {
+    double* xd = xs + ((size_t)buf * kRtT + st) * 128;
+    float* wd = ws + ((size_t)buf * kRtE + se) * 128;
 #pragma unroll
-    for (int t = 0; t < kRtT; t++) acc[i][t] = 0.0;
+    for (int i = 0; i < 2; i++) {
+      const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
+#pragma unroll
+      for (int h = 0; h < 8; h++) {
+        const int kk = 16 * sp + 8 * i + h;  // element of the block
+        const uint16_t b = (uint16_t)((h & 1) ? (u[h >> 1] >> 16) : (u[h >> 1] & 0xffffu));
+        xd[(kk & 3) * 32 + (kk >> 2)] = (double)bf16_bits_to_f32(b);
+      }
+      const float f[4] = {wq[i].x, wq[i].y, wq[i].z, wq[i].w};
+#pragma unroll
+      for (int h = 0; h < 4; h++) {
+        const int kk = 8 * sq + 4 * i + h;
+        wd[(kk & 3) * 32 + (kk >> 2)] = f[h];
+      }
+    }
+  };
+  double acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; i++)
+#pragma unroll
+    for (int j = 0; j < 8; j++) acc[i][j] = 0.0;
   const int C = H >> 7;
+  gload(0);
+  sstore(0);
+  __syncthreads();
   for (int c = 0; c < C; c++) {
-    __syncthreads();
-    {  // x: 8 tokens x 128 elements, 4 per thread
-      const int t = threadIdx.x >> 5, q = threadIdx.x & 31;  // elements 4q .. 4q+3 of token t
-      uint2 xv = make_uint2(0u, 0u);
-      if (t0 + t < T) xv = __ldg(reinterpret_cast<const uint2*>(x + (size_t)(t0 + t) * H + c * 128) + q);
-      xs[t][0][q] = (double)bf16_bits_to_f32((uint16_t)(xv.x & 0xffff));
-      xs[t][1][q] = (double)bf16_bits_to_f32((uint16_t)(xv.x >> 16));
-      xs[t][2][q] = (double)bf16_bits_to_f32((uint16_t)(xv.y & 0xffff));
-      xs[t][3][q] = (double)bf16_bits_to_f32((uint16_t)(xv.y >> 16));
-    }
-#pragma unroll
-    for (int r = 0; r < 4; r++) {  // Wr: 32 experts x 128 elements, 16 per thread
-      const int idx = threadIdx.x + 256 * r, e = idx >> 5, q = idx & 31;
-      float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e0 + e < E) w4 = __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + e) * H + c * 128) + q);
-      ws[e][0][q] = (double)w4.x;
-      ws[e][1][q] = (double)w4.y;
-      ws[e][2][q] = (double)w4.z;
-      ws[e][3][q] = (double)w4.w;
-    }
-    __syncthreads();
+    const int buf = c & 1;
+    if (c + 1 < C) gload(c + 1);
+    const double* xb = xs + ((size_t)buf * kRtT + 8 * tw) * 128 + lane;
+    const float* wb = ws + ((size_t)buf * kRtE + 8 * ew) * 128 + lane;
 #pragma unroll
     for (int v = 0; v < 4; v++) {
-      double xr[kRtT], wv[4];
+      double xv[8], wv[8];
 #pragma unroll
-      for (int t = 0; t < kRtT; t++) xr[t] = xs[t][v][lane];
+      for (int i = 0; i < 8; i++) xv[i] = xb[i * 128 + v * 32];
 #pragma unroll
-      for (int i = 0; i < 4; i++) wv[i] = ws[4 * warp + i][v][lane];
+      for (int j = 0; j < 8; j++) wv[j] = (double)wb[j * 128 + v * 32];
+      // products bf16 * fp32 are exact in fp64: fma == add of the product
 #pragma unroll
-      for (int i = 0; i < 4; i++)
+      for (int i = 0; i < 8; i++)
 #pragma unroll
-        for (int t = 0; t < kRtT; t++) acc[i][t] = fma(xr[t], wv[i], acc[i][t]);  // exact product: fma == add
+        for (int j = 0; j < 8; j++) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
     }
+    if (c + 1 < C) sstore(buf ^ 1);
+    __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; i++) {
-    const int e = e0 + 4 * warp + i;
+  for (int i = 0; i < 8; i++)
 #pragma unroll
-    for (int t = 0; t < kRtT; t++) {
-      double a = acc[i][t];
+    for (int j = 0; j < 8; j++) {
+      double a = acc[i][j];
 #pragma unroll
       for (int d = 16; d >= 1; d >>= 1) a = a + __shfl_xor_sync(0xffffffffu, a, d);
-      if (lane == 0 && e < E && t0 + t < T) logits[(size_t)(t0 + t) * E + e] = __double2float_rn(a);
+      const int t = t0 + 8 * tw + i, e = e0 + 8 * ew + j;
+      if (lane == ((i * 8 + j) & 31) && t < T && e < E) logits[(size_t)t * E + e] = __double2float_rn(a);
     }
-  }
 }
 
 cudaError_t launch_router_logits(const uint16_t* x, const float* wr, int T, int H, int E, float* logits,
@@ -137,7 +166,10 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* wr, int T, int 
     k_router_logits<8><<<grid, block, 0, s>>>(x, wr, T, H, E, logits);
   } else {
     dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
-    k_router_logits_tiled<<<grid, block, 0, s>>>(x, wr, T, H, E, logits);
+    cudaError_t e = cudaFuncSetAttribute(k_router_logits_tiled, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kRtSmem);
+    if (e != cudaSuccess) return e;
+    k_router_logits_tiled<<<grid, block, kRtSmem, s>>>(x, wr, T, H, E, logits);
   }
   return cudaGetLastError();
 }

@@ -25,7 +25,7 @@ __device__ __forceinline__ uint64_t gtime() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// One lane of the warp waits for phase `parity` with a sleep between polls
+// One lane of the warp waits for phase `parity` with a short sleep between polls
 // (the warps that only wait for the accumulators do not compete for issue
 // slots with the producer and MMA threads), then the warp reconverges; false
 // after kWaitNs of wall time.
@@ -34,13 +34,13 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity) {
   if ((threadIdx.x & 31) == 0) {
     const uint32_t a = s_u32(b);
     const uint64_t t0 = gtime();
-    for (;;) {
+    for (uint32_t n = 1;; n++) {
       asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
                    : "=r"(ok)
                    : "r"(a), "r"(parity)
                    : "memory");
-      if (ok || gtime() - t0 > kWaitNs) break;
-      __nanosleep(256);
+      if (ok || ((n & 15) == 0 && gtime() - t0 > kWaitNs)) break;
+      __nanosleep(64);
     }
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -55,18 +55,19 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 
-// wait for phase `parity`, giving up after kWaitNs of wall time
+// wait for phase `parity`, giving up after about kWaitNs of wall time
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
   const uint32_t a = s_u32(b);
   const uint64_t t0 = gtime();
-  for (;;) {
+  for (uint32_t n = 1;; n++) {
     uint32_t ok;
     asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
                  : "=r"(ok)
                  : "r"(a), "r"(parity)
                  : "memory");
     if (ok) return true;
-    if (gtime() - t0 > kWaitNs) return false;
+    // the global timer is read on every 32nd poll only
+    if ((n & 31) == 0 && gtime() - t0 > kWaitNs) return false;
   }
 }
 

@@ -560,13 +560,14 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = gclock();
-  while (!mbar_try(bar, parity)) {
-    if (gclock() - t0 > kSpinNs) {
+  for (uint32_t n = 1;; n++) {
+    if (mbar_try(bar, parity)) return true;
+    // the global timer is read on every 32nd poll only
+    if ((n & 31) == 0 && gclock() - t0 > kSpinNs) {
       set_status(status, kStTimeout);
       return false;
     }
   }
-  return true;
 }
 // One contiguous global -> shared copy by the bulk-copy engine, completing on bar.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -582,8 +583,8 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 __device__ inline bool cta_wait_geq(const int* p, int target, int& abort, int* status, uint64_t limit_ns = kSpinNs) {
   if (threadIdx.x == 0 && ld_acquire(p) < target) {
     const uint64_t t0 = gclock();
-    while (ld_acquire(p) < target) {
-      if (gclock() - t0 > limit_ns) {
+    for (uint32_t n = 1; ld_acquire(p) < target; n++) {
+      if ((n & 15) == 0 && gclock() - t0 > limit_ns) {
         set_status(status, kStTimeout);
         abort = 1;
         break;

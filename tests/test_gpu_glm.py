@@ -69,8 +69,8 @@ def test_glm_class_cache_trace_and_outputs():
         x = x_dev(synth.activations_bf16(SEED, 2, 1, H))
         for p in range(n_tok):
             if p == 12:
-                ft.ft_expert_cache_resize(cache.h, (slots // 2) * stride)
-                assert [tuple(int(v) for v in e) for e in ft.ft_cache_trace(cache.h)] == ref.resize(slots // 2)
+                ft.ft_expert_cache_resize(cache.h, 48 * stride)
+                assert [tuple(int(v) for v in e) for e in ft.ft_cache_trace(cache.h)] == ref.resize(48)
             if p == 24:
                 ft.ft_expert_cache_resize(cache.h, slots * stride)
                 ft.ft_cache_trace(cache.h)
