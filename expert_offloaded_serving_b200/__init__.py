@@ -305,16 +305,16 @@ def ft_fp4_mma_probe(iters: int, sink, status, stream=None) -> int:
 
 
 def ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, weight_format=0) -> dict:
-    out = (I64 * 4)()
+    out = (I64 * 3)()
     _check(lib().ft_flow_geometry(hidden, inter, T, top_k, n_shared, n_experts, n_layers, weight_format, out))
-    return {"ok": bool(out[0]), "rows_cap": out[1], "smem": out[2], "a_rows": out[3]}
+    return {"ok": bool(out[0]), "rows_cap": out[1], "smem": out[2]}
 
 
 def ft_debug_stack_epoch(ctx, epoch: int, poison_layer: int = -1) -> None:
     _check(lib().ft_debug_stack_epoch(ctx, epoch & 0xFFFFFFFF, poison_layer))
 
 
-GEOMETRY_FIELDS = ("K", "chunks", "pblk", "parts", "tasks", "rstride", "sstride", "R", "smem", "taken")
+GEOMETRY_FIELDS = ("K", "chunks", "lpr", "rpw", "parts", "rsets", "groups", "R", "smem", "taken")
 
 
 def ft_decode_geometry(hidden: int, inter: int, n_layers: int = 1) -> dict:

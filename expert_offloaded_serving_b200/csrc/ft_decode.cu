@@ -531,14 +531,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_stack(StackArgs a) {
   uint32_t phase[2] = {0u, 0u};     // parity of each buffer's next phase
   bool pending[2] = {false, false};  // a tile issued into the buffer and not waited for
   auto issue_codes = [&](int buf, const Gv& g, uint8_t* base, const uint8_t* m0, const uint8_t* m1, int row0) {
-    if ((threadIdx.x >> 5) == (kIssuer >> 5)) {
-      const uint32_t bytes = (uint32_t)g.R * (uint32_t)g.rowb;
+    if (threadIdx.x == kIssuer) {
+      const uint32_t bytes = (uint32_t)g.R * (uint32_t)(g.K / 2);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if ((threadIdx.x & 31) == 0) mbar_expect_tx(&hd.bar[buf], m0 ? bytes * (m1 ? 2u : 1u) : 0u);
-      __syncwarp();
-      if (m0) bulk_rows_warp(g, base + g.codes, m0 + (size_t)row0 * g.rowb, g.R, &hd.bar[buf]);
-      if (m0 && m1) bulk_rows_warp(g, base + g.codes + (size_t)g.R * g.rstride, m1 + (size_t)row0 * g.rowb, g.R,
-                                   &hd.bar[buf]);
+      mbar_expect_tx(&hd.bar[buf], m0 ? bytes * (m1 ? 2u : 1u) : 0u);
+      if (m0) bulk_g2s(base + g.codes, m0 + (size_t)row0 * (g.K / 2), bytes, &hd.bar[buf]);
+      if (m0 && m1) bulk_g2s(base + g.codes + bytes, m1 + (size_t)row0 * (g.K / 2), bytes, &hd.bar[buf]);
     }
     pending[buf] = true;
   };
@@ -861,11 +859,11 @@ void decode_geometry(int H, int I, int64_t* out) {
     int64_t* o = out + 10 * p;
     o[0] = g.K;
     o[1] = g.chunks;
-    o[2] = g.pblk;
-    o[3] = g.parts;
-    o[4] = (int64_t)(g.nmat * g.R / 16) * g.parts;
-    o[5] = g.rstride;
-    o[6] = g.sstride;
+    o[2] = g.lpr;
+    o[3] = g.rpw;
+    o[4] = g.parts;
+    o[5] = g.rsets;
+    o[6] = g.groups;
     o[7] = g.R;
     o[8] = (int64_t)(kTileOff + g.total);
     o[9] = gv_ok(g, rows[p]) ? 1 : 0;

@@ -135,7 +135,6 @@ struct FlowArgs {
   uint64_t* x_tagged;          // [T][H/2] words: tag << 32 | two bf16
   const uint32_t* epoch;       // advanced by the routing kernel before this launch
   int rows_cap;                // down-tile rows over all units (flow_geometry)
-  int a_rows;                  // rows of each matrix in a gate/up tile (flow_geometry)
   int* status;
   // NULL, or [n_layers][gridDim][8] %globaltimer stamps of each CTA: gate/up
   // start, x staged, h published, down h staged, x published (0 where the CTA
@@ -144,7 +143,6 @@ struct FlowArgs {
 };
 struct FlowGeom {
   int rows_cap;
-  int a_rows;
   size_t smem;
   bool ok;                     // the dataflow kernel takes this shape, batch and depth
 };

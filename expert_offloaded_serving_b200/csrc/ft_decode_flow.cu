@@ -46,7 +46,7 @@ using namespace tile;
 namespace {
 
 constexpr int kWarpsF = kGemvThreads / 32;
-constexpr int kIssuerWarp = 1;  // warp 1 issues the bulk weight copies
+constexpr int kIssuerF = 32;  // lane 0 of warp 1 issues the bulk weight copies
 
 // One unit of a layer (a distinct routed expert or a shared expert).
 struct FlowUnit {
@@ -88,16 +88,16 @@ struct FlowHdr {
   int32_t pad[3];
 };
 
-// Down-tile geometry for K = I: rows_cap staged rows (all units), nh
-// activation rows staged at once.
+// Down-tile geometry: the GEMV lane mapping for K = I, with rows_cap rows (all
+// units) and nh activation rows staged at once.
 __host__ __device__ inline Gv make_gd(int I, int rows_cap, int nh, int fmt) {
   Gv g = make_gv(I, 1 << 30, 1, fmt);
   g.R = rows_cap;
   g.rlog = 0;
   g.codes = 0;
-  g.scales = (size_t)rows_cap * g.rstride;
-  g.xh = g.scales + (size_t)rows_cap * g.sstride * 4;
-  g.xinv = g.xh + (fmt == kFmtBf16 ? (size_t)nh * I * 4 : (size_t)nh * g.xstride);
+  g.scales = (size_t)rows_cap * g.rowb;
+  g.xh = g.scales + (size_t)rows_cap * g.atoms * 4;
+  g.xinv = g.xh + (size_t)nh * I * (fmt == kFmtBf16 ? 4 : 2);
   g.red = g.xinv + (fmt == kFmtBf16 ? 0 : (((size_t)nh * g.chunks * 4 + 15) & ~(size_t)15));
   g.total = (g.red + (size_t)g.parts * rows_cap * kMT * 4 + 127) & ~(size_t)127;
   return g;
@@ -197,63 +197,53 @@ __device__ __forceinline__ void stage_h_all(const Gv& g, uint8_t* base, const ui
 }
 
 // Partial sums of the down tile: unit u's rows u*rb .. u*rb + rb - 1 against
-// the unit's h rows.  MXFP4/NVFP4: the tensor-core tasks of the tile, each
-// 16-row group inside one unit (rb is a multiple of 16).  BF16: the tile's
-// rows, unit-major, are taken two at a time (rb is even, so a pair never
-// straddles units); lane group g takes the pairs [g*ppg, (g+1)*ppg).  Every
-// lane of a warp runs the same number of steps, so the reduction's shuffles
-// see the whole warp; pairs past the end compute zeros and are not stored.
-// NT = tokens per pass (2 when any unit has two).
+// the unit's h rows.  The tile's rows, unit-major, are taken two at a time
+// (rb is even, so a pair never straddles units); lane group g takes the pairs
+// [g*ppg, (g+1)*ppg).  Every lane of a warp runs the same number of steps, so
+// the reduction's shuffles see the whole warp; pairs past the end compute
+// zeros and are not stored.  NT = tokens per pass (2 when any unit has two).
 template <int NT, int F>
 __device__ __forceinline__ void dtile_dots(const Gv& g, const LaneMap& m, uint8_t* base, const FlowUnit* un, int U,
                                            int rb) {
-  if constexpr (F != kFmtBf16) {
-    mma_dots<F>(g, base, U * rb, g.R, [&](int q) {
-      const FlowUnit& f = un[(16 * q) / rb];
-      return make_int2(f.hrow, f.m);
-    });
-  } else {
-    if (!m.on) return;
-    const uint8_t* codes = base + g.codes;
-    float* red = reinterpret_cast<float*>(base + g.red);
-    const bool cv = m.c < g.chunks;
-    const int npairs = U * rb / 2;
-    const int ppg = (npairs + g.groups - 1) / g.groups;
-    const int lmask = (g.lpr >> 1) - 1;
-    int cur = -1;
-    float xf[kMT][32];
+  if (!m.on) return;
+  const uint8_t* codes = base + g.codes;
+  const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
+  float* red = reinterpret_cast<float*>(base + g.red);
+  const bool cv = m.c < g.chunks;
+  const int npairs = U * rb / 2;
+  const int ppg = (npairs + g.groups - 1) / g.groups;
+  const int lmask = (g.lpr >> 1) - 1;
+  int cur = -1;
+  uint32_t x[kMT][16];
+  float xi[kMT] = {0.f, 0.f};
+  float xf[kMT][32];
 #pragma unroll
-    for (int t = 0; t < kMT; t++) zero_act_bf16(xf[t]);
-    for (int jp = 0; jp < ppg; jp++) {
-      const int p = m.grp * ppg + jp;
-      const bool pv = p < npairs;
-      const int row = 2 * p;
-      const int u = pv ? row / rb : cur;
-      if (pv && u != cur && cv) {
-        cur = u;
-        const FlowUnit f = un[u];
+  for (int t = 0; t < kMT; t++) zero_act<F>(x[t], xi[t], xf[t]);
+  for (int jp = 0; jp < ppg; jp++) {
+    const int p = m.grp * ppg + jp;
+    const bool pv = p < npairs;
+    const int row = 2 * p;
+    const int u = pv ? row / rb : cur;
+    if (pv && u != cur && cv) {
+      cur = u;
+      const FlowUnit f = un[u];
 #pragma unroll
-        for (int t = 0; t < NT; t++) {
-          if (t < f.m) load_act_bf16(g, base, f.hrow + t, m.c, xf[t]);
-          else zero_act_bf16(xf[t]);
-        }
+      for (int t = 0; t < NT; t++) {
+        if (t < f.m) load_act<F>(g, base, f.hrow + t, m.c, x[t], xi[t], xf[t]);
+        else zero_act<F>(x[t], xi[t], xf[t]);
       }
-      float v[4][kMT];
+    }
+    float v[4][kMT];
 #pragma unroll
-      for (int uu = 0; uu < 2; uu++) {
-        v[uu][0] = v[uu][1] = 0.f;
-        if (cv && pv) {
-          uint4 q[4];
-          tile_chunk_bf16(g, codes, row + uu, m.c, q);
-          chunk_dot_bf16<NT>(q, xf, v[uu]);
-        }
-      }
-      const int sel = group_reduce<2, NT>(v, g.lpr);
-      if (pv && ((threadIdx.x & 31) & lmask) == 0) {
-        float* o = red + ((size_t)m.part * g.R + row + sel) * kMT;
+    for (int uu = 0; uu < 2; uu++) {
+      v[uu][0] = v[uu][1] = 0.f;
+      if (cv && pv) chunk_value<NT, F>(g, codes, sc, row + uu, m.c, x, xi, xf, v[uu]);
+    }
+    const int sel = group_reduce<2, NT>(v, g.lpr);
+    if (pv && ((threadIdx.x & 31) & lmask) == 0) {
+      float* o = red + ((size_t)m.part * g.R + row + sel) * kMT;
 #pragma unroll
-        for (int t = 0; t < NT; t++) o[t] = v[0][t];
-      }
+      for (int t = 0; t < NT; t++) o[t] = v[0][t];
     }
   }
 }
@@ -276,7 +266,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
   const int H = HS ? HS : a.H, I = IS ? IS : a.I;
   const int T = a.T, k = a.k, S = a.n_shared, P = T * k, NH = P + S * T;
   const int umax = min(a.E, P) + S;
-  const Gv gA = make_gv(H, HS ? IS : a.a_rows, 2, F);
+  const Gv gA = make_gv(H, I, 2, F);
   const Gv gB = make_gd(I, a.rows_cap, NH, F);
   uint8_t* baseA = smem;
   uint8_t* baseB = smem + round128(gA.total);
@@ -303,9 +293,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
   {
     const int lane = threadIdx.x & 31;
     // down rows per unit: about H / G rows per tile (one tile per CTA), at most
-    // rows_cap over all units, in steps of 16 (a tensor-core task) or 2 (BF16)
-    constexpr int RQ = F == kFmtBf16 ? 2 : 16;
-    const int rb_g = RQ * ((H + RQ * G - 1) / (RQ * G));
+    // rows_cap over all units
+    const int rb_g = 2 * ((H + 2 * G - 1) / (2 * G));
     for (int l = threadIdx.x >> 5; l < a.n_layers; l += kWarpsF) {
       const Route* rec = a.rec + l;
       const uint8_t* const* eptr = a.eptr + (size_t)l * a.n_blobs;
@@ -352,7 +341,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
       if (lane == 0) {
         FlowLayerHdr h;
         h.units = U;
-        h.rb = max(RQ, min(rb_g, RQ * (a.rows_cap / (RQ * U))));
+        h.rb = max(2, min(rb_g, 2 * (a.rows_cap / (2 * U))));
         h.nd = (H + h.rb - 1) / h.rb;
         h.tiles_a = U * nrbA;
         *reinterpret_cast<FlowLayerHdr*>(L) = h;
@@ -370,15 +359,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
   auto issue_A = [&](int l, int i) {
     const FlowUnit f = lunits(l)[i / nrbA];
     const int row0 = (i % nrbA) * gA.R;
-    if ((threadIdx.x >> 5) == kIssuerWarp) {
+    if (threadIdx.x == kIssuerF) {
       const uint32_t bytes = (uint32_t)gA.R * (uint32_t)gA.rowb;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if ((threadIdx.x & 31) == 0) mbar_expect_tx(&hd.bar[0], f.blob ? 2u * bytes : 0u);
-      __syncwarp();
+      mbar_expect_tx(&hd.bar[0], f.blob ? 2u * bytes : 0u);
       if (f.blob) {
-        bulk_rows_warp(gA, baseA + gA.codes, f.blob + a.lay.wg + (size_t)row0 * gA.rowb, gA.R, &hd.bar[0]);
-        bulk_rows_warp(gA, baseA + gA.codes + (size_t)gA.R * gA.rstride, f.blob + a.lay.wu + (size_t)row0 * gA.rowb,
-                       gA.R, &hd.bar[0]);
+        bulk_g2s(baseA + gA.codes, f.blob + a.lay.wg + (size_t)row0 * gA.rowb, bytes, &hd.bar[0]);
+        bulk_g2s(baseA + gA.codes + bytes, f.blob + a.lay.wu + (size_t)row0 * gA.rowb, bytes, &hd.bar[0]);
       }
     }
     if (f.blob) {
@@ -394,24 +381,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
     const FlowUnit* un = lunits(l);
     const int rb = lh.rb, n0 = d * rb, nv = min(rb, H - n0);
     const uint32_t rbytes = (uint32_t)nv * (uint32_t)gB.rowb;
-    if ((threadIdx.x >> 5) == kIssuerWarp) {
+    if (threadIdx.x == kIssuerF) {
       uint32_t total = 0;
       for (int u = 0; u < lh.units; u++)
         if (un[u].blob) total += rbytes;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if ((threadIdx.x & 31) == 0) mbar_expect_tx(&hd.bar[1], total);
-      __syncwarp();
+      mbar_expect_tx(&hd.bar[1], total);
       for (int u = 0; u < lh.units; u++)
         if (un[u].blob)
-          bulk_rows_warp(gB, baseB + gB.codes + (size_t)u * rb * gB.rstride, un[u].blob + a.lay.wd + (size_t)n0 * gB.rowb,
-                         nv, &hd.bar[1]);
+          bulk_g2s(baseB + gB.codes + (size_t)u * rb * gB.rowb, un[u].blob + a.lay.wd + (size_t)n0 * gB.rowb, rbytes,
+                   &hd.bar[1]);
     }
     uint32_t* sd = reinterpret_cast<uint32_t*>(baseB + gB.scales);
     const int per_u = nv * gB.atoms;  // 0 for BF16: no scales
     for (int i = threadIdx.x; i < lh.units * per_u; i += kGemvThreads) {
       const int u = i / per_u, j = i - u * per_u, r = j / gB.atoms, at = j - r * gB.atoms;
       const uint8_t* bl = un[u].blob;
-      if (bl) cp_async4(sd + (size_t)(u * rb + r) * gB.sstride + at, bl + a.lay.wd_sf + sf_word(n0 + r, at, gB.atoms));
+      if (bl) cp_async4(sd + (size_t)(u * rb + r) * gB.atoms + at, bl + a.lay.wd_sf + sf_word(n0 + r, at, gB.atoms));
     }
     cp_async_commit();
     seqbuf[1] = seq++;
@@ -564,40 +550,30 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
 FlowGeom flow_geometry(int H, int I, int T, int k, int S, int E, int n_layers, int fmt) {
   FlowGeom fg{};
   if (T < 1 || T > 2 || n_layers < 1 || n_layers > 127) return fg;
+  const Gv gA = make_gv(H, I, 2, fmt);
+  if (!gv_ok(gA, I)) return fg;
   const Gv l = make_gv(I, 1 << 30, 1, fmt);
   if (l.rsets <= 0 || I % 128) return fg;
   const int P = T * k, NH = P + S * T, umax = std::min(E, P) + S;
   if (umax > 255) return fg;
-  // down-tile rows over all units: up to 256 and about 64 KB of codes, in
-  // whole 16-row tensor-core tasks (MXFP4, NVFP4) or row pairs (BF16), at
-  // least one such step per unit
-  const int rq = fmt == kFmtBf16 ? 2 : 16;
+  // down-tile rows over all units: up to 256, and about 64 KB of codes
   int rows_cap = std::min(256, (int)(65536 / l.rowb));
-  rows_cap -= rows_cap % rq;
-  if (rows_cap < rq * umax) rows_cap = rq * umax;
+  rows_cap &= ~1;
+  if (rows_cap < 2 * umax) rows_cap = 2 * umax;
   const Gv gB = make_gd(I, rows_cap, NH, fmt);
-  // the gate/up tile: about 64 KB of codes, or 32 or 16 KB when the down tile
-  // and the layer table need the room (a smaller tile only means more tiles)
-  for (size_t tb = kTileBytes; tb >= kTileBytes / 4; tb /= 2) {
-    const Gv gA = make_gv(H, I, 2, fmt, tb);
-    if (!gv_ok(gA, I)) continue;
-    const size_t smem = round128(gA.total) + gB.total + sizeof(FlowHdr) + (size_t)n_layers * flow_layer_bytes(umax, P);
-    fg.rows_cap = rows_cap;
-    fg.a_rows = gA.R;
-    fg.smem = smem;
-    fg.ok = smem <= 227 * 1024;
-    if (fg.ok) break;
-  }
+  const size_t smem = round128(gA.total) + gB.total + sizeof(FlowHdr) + (size_t)n_layers * flow_layer_bytes(umax, P);
+  fg.rows_cap = rows_cap;
+  fg.smem = smem;
+  fg.ok = smem <= 227 * 1024;
   return fg;
 }
 
 cudaError_t launch_dec_flow(const FlowArgs& a, cudaStream_t s) {
   const int F = a.lay.fmt;
   const FlowGeom fg = flow_geometry(a.H, a.I, a.T, a.k, a.n_shared, a.E, a.n_layers, F);
-  if (!fg.ok || a.rows_cap != fg.rows_cap || a.a_rows != fg.a_rows) return cudaErrorInvalidValue;
-  // the 35B-class shape (hidden 2048, intermediate 512) has its own builds,
-  // whose gate/up tile is the full one (R = 32)
-  const bool s35 = a.H == 2048 && a.I == 512 && fg.a_rows == make_gv(2048, 512, 2, F).R;
+  if (!fg.ok || a.rows_cap != fg.rows_cap) return cudaErrorInvalidValue;
+  // the 35B-class shape (hidden 2048, intermediate 512) has its own builds
+  const bool s35 = a.H == 2048 && a.I == 512;
   void (*kern)(FlowArgs) = F == kFmtNv ? (s35 ? k_dec_flow<2048, 512, kFmtNv> : k_dec_flow<0, 0, kFmtNv>)
                            : F == kFmtBf16 ? (s35 ? k_dec_flow<2048, 512, kFmtBf16> : k_dec_flow<0, 0, kFmtBf16>)
                                            : (s35 ? k_dec_flow<2048, 512, kFmtMx> : k_dec_flow<0, 0, kFmtMx>);

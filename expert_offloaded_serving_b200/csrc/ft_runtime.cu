@@ -690,7 +690,7 @@ extern "C" ft_status ft_fp4_mma_probe(int64_t iters, float* sink, int32_t* statu
 }
 
 extern "C" ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
-                                      int32_t n_experts, int32_t n_layers, int32_t weight_format, int64_t out[4]) {
+                                      int32_t n_experts, int32_t n_layers, int32_t weight_format, int64_t out[3]) {
   if (!out) return fail(FT_ERR_INVALID, "out is NULL");
   if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128 || top_k <= 0 || top_k > 16 || n_experts <= 0 ||
       n_shared < 0 || n_shared > 1 || T <= 0 || n_layers <= 0 || weight_format < 0 || weight_format > 2)
@@ -699,7 +699,6 @@ extern "C" ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, 
   out[0] = fg.ok ? 1 : 0;
   out[1] = fg.rows_cap;
   out[2] = (int64_t)fg.smem;
-  out[3] = fg.a_rows;
   return FT_OK;
 }
 
@@ -1582,7 +1581,6 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
     a.x_tagged = c->d_x_tagged;
     a.epoch = c->d_epoch;
     a.rows_cap = fg.rows_cap;
-    a.a_rows = fg.a_rows;
     a.status = c->d_status;
     int dev = 0, nsm = 0;
     cudaGetDevice(&dev);

@@ -347,13 +347,12 @@ FT_API ft_status ft_prefetch_layer(ft_ctx* ctx, int32_t layer, void* compute_str
  * products use.  FT_ERR_INVALID for a shape the decode kernels do not take. */
 FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, float* out, void* stream);
 
-/* Tile geometry the MXFP4 decode kernels use for hidden H and intermediate I
+/* Tile geometry the decode kernels use for hidden H and intermediate I
  * (host only, no device needed).  out[0..9] describe the gate/up tile and
- * out[10..19] the down tile, each: K, 32-code blocks of K, blocks per K part,
- * K parts, tensor-core tasks per tile (16-row groups x parts), bytes per
- * staged code row, scale words per staged row, R rows per tile, shared-memory
- * bytes of a per-layer CTA, 1 if the tile is taken; out[20] threads per CTA,
- * out[21] the shared-memory limit of a tile,
+ * out[10..19] the down tile, each: K, 32-code chunks of K, lanes per row group
+ * (lpr), row groups per warp (rpw), K parts, row sets, lane groups per CTA, R
+ * rows per tile, shared-memory bytes of a per-layer CTA, 1 if the tile is
+ * taken; out[20] threads per CTA, out[21] the shared-memory limit of a tile,
  * out[22] 1 if the persistent kernel takes a stack of n_layers layers of this
  * shape, out[23] its counter words per layer.  FT_ERR_INVALID on a bad shape. */
 FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_layers, int64_t out[24]);
@@ -362,10 +361,9 @@ FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_lay
  * one or two tokens (host only, no device needed): out[0] = 1 if it takes
  * this shape, batch T, stack depth and weight format (else the
  * counter-synchronised or the per-layer kernels run), out[1] = rows of a down tile over all units,
- * out[2] = shared memory of a CTA in bytes, out[3] = rows of each matrix in
- * a gate/up tile.  FT_ERR_INVALID on a bad shape. */
+ * out[2] = shared memory of a CTA in bytes.  FT_ERR_INVALID on a bad shape. */
 FT_API ft_status ft_flow_geometry(int32_t hidden, int32_t inter, int32_t T, int32_t top_k, int32_t n_shared,
-                                  int32_t n_experts, int32_t n_layers, int32_t weight_format, int64_t out[4]);
+                                  int32_t n_experts, int32_t n_layers, int32_t weight_format, int64_t out[3]);
 
 /* Failure injection for tests: none of these fault or hang a GPU.
  *

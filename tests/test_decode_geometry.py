@@ -1,7 +1,8 @@
 """Tile geometry of the decode GEMV kernels (host logic, no GPU): for every
 shape the kernels take, the tile fits shared memory, covers K and the rows
-exactly in whole 16-row tensor-core tasks, and its staged rows fall in
-distinct shared-memory banks; shapes past the limits are refused."""
+exactly, and keeps the row loop's trip count equal for all lanes of a warp
+(the xor-shuffle reductions need the whole warp); shapes past the limits are
+refused."""
 import pytest
 
 import expert_offloaded_serving_b200 as ft
@@ -14,18 +15,20 @@ def is_pow2(v):
     return v > 0 and (v & (v - 1)) == 0
 
 
-def check_tile(t, K, rows, nmat, threads, limit):
+def check_tile(t, K, rows, threads, limit):
+    warps = threads // 32
     assert t["K"] == K and t["chunks"] == K // 32
-    # K parts of 8 blocks of 32 when K allows, else of 4; they cover K exactly
-    assert t["pblk"] == (8 if K % 256 == 0 else 4) and t["parts"] * t["pblk"] == t["chunks"]
+    assert is_pow2(t["lpr"]) and t["lpr"] <= 32 and t["lpr"] * t["rpw"] == 32
+    assert t["lpr"] >= min(t["chunks"], 32)            # a lane group spans all chunks it can
+    assert t["parts"] * t["lpr"] >= t["chunks"] > (t["parts"] - 1) * t["lpr"]
+    assert 1 <= t["rsets"] and t["rsets"] * t["parts"] <= warps
+    assert t["groups"] == t["rsets"] * t["rpw"]
     assert is_pow2(t["R"]) and 8 <= t["R"] <= 128 and rows % t["R"] == 0
-    assert (nmat * t["R"]) % 16 == 0 and t["tasks"] == nmat * t["R"] // 16 * t["parts"]
-    # a staged row holds the row's codes; consecutive rows start 64 bytes apart
-    # modulo 128 (the 16-byte loads of 8 rows hit distinct banks); an odd count
-    # of scale words per row
-    assert t["rstride"] >= K // 2 and t["rstride"] % 128 == 64 and t["rstride"] % 16 == 0
-    assert t["sstride"] % 2 == 1 and t["sstride"] >= K // 128
     assert t["smem"] <= 128 + limit <= OPT_IN_SMEM
+    # several lane groups share a warp only with one K part, and then R is a
+    # multiple of the groups per warp: every lane of a warp runs the same rows loop
+    if t["rpw"] > 1:
+        assert t["parts"] == 1 and t["R"] % t["rpw"] == 0
 
 
 @pytest.mark.parametrize("H", SIZES)
@@ -34,16 +37,16 @@ def test_tiles_of_every_supported_shape(H, I):
     g = ft.ft_decode_geometry(H, I, 40)
     assert g["threads"] == 512
     assert g["gate_up"]["taken"] and g["down"]["taken"]
-    check_tile(g["gate_up"], H, I, 2, g["threads"], g["smem_limit"])
-    check_tile(g["down"], I, H, 1, g["threads"], g["smem_limit"])
+    check_tile(g["gate_up"], H, I, g["threads"], g["smem_limit"])
+    check_tile(g["down"], I, H, g["threads"], g["smem_limit"])
     if g["stack"]:
         assert g["sync_stride"] == 2 + H // g["down"]["R"]
 
 
 def test_35b_class_tiles_and_stack():
     g = ft.ft_decode_geometry(2048, 512, 40)
-    assert (g["gate_up"]["R"], g["gate_up"]["parts"], g["gate_up"]["tasks"]) == (32, 8, 32)
-    assert (g["down"]["R"], g["down"]["parts"], g["down"]["tasks"]) == (128, 2, 16)
+    assert (g["gate_up"]["R"], g["gate_up"]["lpr"], g["gate_up"]["parts"]) == (32, 32, 2)
+    assert (g["down"]["R"], g["down"]["lpr"], g["down"]["rpw"]) == (128, 16, 2)
     # 9 units (8 routed + shared) x I/R = 144 gate/up tiles and x H/R = 144 down
     # tiles: one of each per CTA on 148 SMs
     assert 9 * 512 // g["gate_up"]["R"] == 144 and 9 * 2048 // g["down"]["R"] == 144
@@ -60,31 +63,19 @@ def test_limits_are_refused():
     assert e.value.status == ft.FT_ERR_INVALID
 
 
-FLOW_SHAPES = [(2048, 512, 256, 8, 1, 40), (4096, 2048, 256, 6, 0, 43), (6144, 2048, 256, 8, 0, 8),
-               (256, 128, 16, 2, 0, 4), (1024, 512, 64, 4, 0, 3), (1024, 768, 64, 4, 1, 3), (256, 256, 16, 4, 1, 3)]
-# shapes whose down tile (16 rows of every unit over the full intermediate
-# size) and gate/up tile together outgrow a CTA's shared memory: the
-# counter-synchronised persistent kernel takes their stacks
-FLOW_TOO_BIG = {((4096, 2048, 256, 6, 0, 43), 2), ((6144, 2048, 256, 8, 0, 8), 1), ((6144, 2048, 256, 8, 0, 8), 2)}
-
-
-@pytest.mark.parametrize("shape", FLOW_SHAPES)
+@pytest.mark.parametrize("shape", [(2048, 512, 256, 8, 1, 40), (4096, 2048, 256, 6, 0, 43), (6144, 2048, 256, 8, 0, 8),
+                                   (256, 128, 16, 2, 0, 4), (1024, 512, 64, 4, 0, 3), (1024, 768, 64, 4, 1, 3),
+                                   (256, 256, 16, 4, 1, 3)])
 @pytest.mark.parametrize("T", [1, 2])
 def test_dataflow_kernel_geometry(shape, T):
     """The dataflow stack kernel takes the workload shapes at one and two
-    tokens where they fit: its CTA fits the opt-in shared memory, a down tile
-    has room for one 16-row tensor-core task of every unit a layer can have,
-    and the gate/up tile whole tasks (8 rows of each matrix at least).  The
-    rest go to the counter-synchronised kernel."""
+    tokens: its CTA fits the opt-in shared memory, and a down tile has room
+    for two rows of every unit a layer can have (rb >= 2, even)."""
     H, I, E, k, S, L = shape
     g = ft.ft_flow_geometry(H, I, T, k, S, E, L)
-    if (shape, T) in FLOW_TOO_BIG:
-        assert not g["ok"] and ft.ft_decode_geometry(H, I, L)["stack"]
-        return
     assert g["ok"] and g["smem"] <= OPT_IN_SMEM
     units = min(E, T * k) + S
-    assert g["rows_cap"] % 16 == 0 and g["rows_cap"] >= 16 * units
-    assert g["a_rows"] >= 8 and I % g["a_rows"] == 0
+    assert g["rows_cap"] % 2 == 0 and g["rows_cap"] >= 2 * units
 
 
 def test_dataflow_kernel_limits():
