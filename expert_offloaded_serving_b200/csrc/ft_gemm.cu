@@ -77,10 +77,6 @@ __device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
                : "memory");
 }
 
-// silu(z) = z / (1 + e^-z) with the fast exponential and division (h is
-// quantised to MXFP4 right after, so a few ulp do not matter).
-__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
-
 // Lane-wise unsigned maximum of two 16-bit halves.
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -293,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
             const int c = q + e;
             const float g = __uint_as_float(c < 16 ? g0[c & 15] : g1[c & 15]);
             const float u = __uint_as_float(c < 16 ? u0[c & 15] : u1[c & 15]);
-            hv[e] = silu_fast(g) * u;
+            hv[e] = silu(g) * u;
           }
           // the block maxima of both columns at once: the top 16 bits of |h|
           // keep its exponent field, which is all the scale rule reads

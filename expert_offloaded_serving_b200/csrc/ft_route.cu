@@ -56,23 +56,32 @@ __global__ void __launch_bounds__(256) k_router_logits(const uint16_t* __restric
 // A CTA of 8 warps takes 32 tokens x 16 experts; warp w takes tokens
 // 8(w/2) .. +7 and experts 8(w%2) .. +7, and lane j holds partial sum j of
 // each of its warp's 64 (token, expert) pairs in registers.  Per 128-element
-// block of K the CTA stages x (converted to fp64 once) and Wr (fp32, widened
-// at use) in shared memory, element 4j + v of the block at [v][j] so that
-// lane j's reads are consecutive; the next block's global loads are in
-// flight while the current one is used (two buffers).  Lane j adds its block
-// elements 4j, 4j+1, 4j+2, 4j+3 in ascending order, so every partial sum
-// sees the same terms in the same order as in k_router_logits; the
-// butterfly and the rounding are the same.
+// block of K the CTA stages x and Wr in shared memory as fp64 (each value
+// converted once), element 4j + v of the block at [v][j] so that lane j's
+// reads are consecutive; the global loads run two blocks ahead.  Lane j adds
+// its block elements 4j, 4j+1, 4j+2, 4j+3 in ascending order, so every
+// partial sum sees the same terms in the same order as in k_router_logits;
+// the butterfly and the rounding are the same.
 // ---------------------------------------------------------------------------
 constexpr int kRtT = 32, kRtE = 16;
-constexpr size_t kRtSmem = 2 * (size_t)(kRtT * 128 * 8 + kRtE * 128 * 4);
+constexpr size_t kRtSmem = 2 * (size_t)(kRtT + kRtE) * 128 * 8;
+
+// fp32 -> fp64, exact: normal values by moving the fields (rebiased
+// exponent, mantissa widened), zeros, subnormals, infinities and NaNs by the
+// conversion instruction.
+__device__ __forceinline__ double f32_to_f64(float f) {
+  const uint32_t u = __float_as_uint(f), e = (u >> 23) & 0xffu;
+  if (e == 0u || e == 255u) return (double)f;
+  const uint32_t hi = (u & 0x80000000u) | ((e + 896u) << 20) | ((u >> 3) & 0xfffffu);
+  return __hiloint2double((int)hi, (int)(u << 29));
+}
 
 __global__ void __launch_bounds__(256, 1) k_router_logits_tiled(const uint16_t* __restrict__ x,
                                                                 const float* __restrict__ wr, int T, int H, int E,
                                                                 float* __restrict__ logits) {
   extern __shared__ __align__(16) uint8_t rt_smem[];
-  double* xs = reinterpret_cast<double*>(rt_smem);                      // [2][kRtT][4][32]
-  float* ws = reinterpret_cast<float*>(rt_smem + 2 * kRtT * 128 * 8);   // [2][kRtE][4][32]
+  double* xs = reinterpret_cast<double*>(rt_smem);  // [2][kRtT][4][32]
+  double* ws = xs + 2 * kRtT * 128;                 // [2][kRtE][4][32]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tw = warp >> 1, ew = warp & 1;
   const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
@@ -83,18 +92,24 @@ __global__ void __launch_bounds__(256, 1) k_router_logits_tiled(const uint16_t* 
   const bool tok_ok = t0 + st < T, exp_ok = e0 + se < E;
   const uint4* xg = reinterpret_cast<const uint4*>(x + (size_t)(tok_ok ? t0 + st : 0) * H) + 2 * sp;
   const float4* wg = reinterpret_cast<const float4*>(wr + (size_t)(exp_ok ? e0 + se : 0) * H) + 2 * sq;
-  uint4 xr[2];
-  float4 wq[2];
-  auto gload = [&](int c) {
+  // two register sets of staged loads, named apart so that a set chosen at
+  // run time still lives in registers
+  uint4 xr0[2], xr1[2];
+  float4 wq0[2], wq1[2];
+  auto gload_into = [&](int c, uint4 (&xr)[2], float4 (&wq)[2]) {
 #pragma unroll
     for (int i = 0; i < 2; i++) {
       xr[i] = tok_ok ? __ldg(xg + c * 16 + i) : make_uint4(0u, 0u, 0u, 0u);
       wq[i] = exp_ok ? __ldg(wg + c * 32 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
-  auto sstore = [&](int buf) {
+  auto gload = [&](int c, int set) {
+    if (set == 0) gload_into(c, xr0, wq0);
+    else gload_into(c, xr1, wq1);
+  };
+  auto sstore_from = [&](int buf, const uint4 (&xr)[2], const float4 (&wq)[2]) {
     double* xd = xs + ((size_t)buf * kRtT + st) * 128;
-    float* wd = ws + ((size_t)buf * kRtE + se) * 128;
+    double* wd = ws + ((size_t)buf * kRtE + se) * 128;
 #pragma unroll
     for (int i = 0; i < 2; i++) {
       const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
@@ -102,15 +117,19 @@ __global__ void __launch_bounds__(256, 1) k_router_logits_tiled(const uint16_t* 
       for (int h = 0; h < 8; h++) {
         const int kk = 16 * sp + 8 * i + h;  // element of the block
         const uint16_t b = (uint16_t)((h & 1) ? (u[h >> 1] >> 16) : (u[h >> 1] & 0xffffu));
-        xd[(kk & 3) * 32 + (kk >> 2)] = (double)bf16_bits_to_f32(b);
+        xd[(kk & 3) * 32 + (kk >> 2)] = f32_to_f64(bf16_bits_to_f32(b));
       }
       const float f[4] = {wq[i].x, wq[i].y, wq[i].z, wq[i].w};
 #pragma unroll
       for (int h = 0; h < 4; h++) {
         const int kk = 8 * sq + 4 * i + h;
-        wd[(kk & 3) * 32 + (kk >> 2)] = f[h];
+        wd[(kk & 3) * 32 + (kk >> 2)] = f32_to_f64(f[h]);
       }
     }
+  };
+  auto sstore = [&](int buf, int set) {
+    if (set == 0) sstore_from(buf, xr0, wq0);
+    else sstore_from(buf, xr1, wq1);
   };
   double acc[8][8];
 #pragma unroll
@@ -118,28 +137,32 @@ __global__ void __launch_bounds__(256, 1) k_router_logits_tiled(const uint16_t* 
 #pragma unroll
     for (int j = 0; j < 8; j++) acc[i][j] = 0.0;
   const int C = H >> 7;
-  gload(0);
-  sstore(0);
+  // register set s holds the global loads of block c with c & 1 == s; block
+  // c + 1 is stored while block c is used, block c + 3 loaded
+  gload(0, 0);
+  if (C > 1) gload(1, 1);
+  sstore(0, 0);
+  if (C > 2) gload(2, 0);
   __syncthreads();
   for (int c = 0; c < C; c++) {
     const int buf = c & 1;
-    if (c + 1 < C) gload(c + 1);
     const double* xb = xs + ((size_t)buf * kRtT + 8 * tw) * 128 + lane;
-    const float* wb = ws + ((size_t)buf * kRtE + 8 * ew) * 128 + lane;
+    const double* wb = ws + ((size_t)buf * kRtE + 8 * ew) * 128 + lane;
 #pragma unroll
     for (int v = 0; v < 4; v++) {
       double xv[8], wv[8];
 #pragma unroll
       for (int i = 0; i < 8; i++) xv[i] = xb[i * 128 + v * 32];
 #pragma unroll
-      for (int j = 0; j < 8; j++) wv[j] = (double)wb[j * 128 + v * 32];
+      for (int j = 0; j < 8; j++) wv[j] = wb[j * 128 + v * 32];
       // products bf16 * fp32 are exact in fp64: fma == add of the product
 #pragma unroll
       for (int i = 0; i < 8; i++)
 #pragma unroll
         for (int j = 0; j < 8; j++) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
     }
-    if (c + 1 < C) sstore(buf ^ 1);
+    if (c + 1 < C) sstore(buf ^ 1, (c + 1) & 1);
+    if (c + 3 < C) gload(c + 3, (c + 1) & 1);
     __syncthreads();
   }
 #pragma unroll
