@@ -260,11 +260,14 @@ __device__ __forceinline__ float dtile_y(const Gv& g, const uint8_t* base, int r
 
 // See the file comment.  HS, IS: hidden and intermediate size fixed at compile
 // time (the tile geometry then folds to constants), or 0, 0 for any shape.
-template <int HS, int IS, int F>
+// TT: 1 for a build that takes one token only (its dot-product loops are
+// the one-token ones), 0 for one or two tokens.  RUG: rows per step of the
+// gate/up tile fixed at compile time (the shape-specific builds), or 0.
+template <int HS, int IS, int F, int TT, int RUG>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = HS ? HS : a.H, I = IS ? IS : a.I;
-  const int T = a.T, k = a.k, S = a.n_shared, P = T * k, NH = P + S * T;
+  const int T = TT ? TT : a.T, k = a.k, S = a.n_shared, P = T * k, NH = P + S * T;
   const int umax = min(a.E, P) + S;
   const Gv gA = make_gv(H, I, 2, F);
   const Gv gB = make_gd(I, a.rows_cap, NH, F);
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         return;
       }
       if (i == b) stamp(1);
-      tile_dots<F>(gA, lmA, baseA, f.m);
+      tile_dots<F, TT, RUG>(gA, lmA, baseA, f.m);
       __syncthreads();
       if (i == b) stamp(7);
       if (threadIdx.x < gA.R * f.m) {
@@ -482,7 +485,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
           return;
         }
         if (d == b) stamp(3);
-        if (T > 1) dtile_dots<2, F>(gB, lmB, baseB, un, lh.units, rb);
+        if (TT != 1 && T > 1) dtile_dots<2, F>(gB, lmB, baseB, un, lh.units, rb);
         else dtile_dots<1, F>(gB, lmB, baseB, un, lh.units, rb);
         __syncthreads();
         if (d == b) stamp(5);
@@ -572,11 +575,15 @@ cudaError_t launch_dec_flow(const FlowArgs& a, cudaStream_t s) {
   const int F = a.lay.fmt;
   const FlowGeom fg = flow_geometry(a.H, a.I, a.T, a.k, a.n_shared, a.E, a.n_layers, F);
   if (!fg.ok || a.rows_cap != fg.rows_cap) return cudaErrorInvalidValue;
-  // the 35B-class shape (hidden 2048, intermediate 512) has its own builds
+  // the 35B-class shape (hidden 2048, intermediate 512) has its own builds;
+  // MXFP4 at one token also a build with only the one-token loops, whose
+  // gate/up tile (32 rows of each matrix, 8 lane groups) steps 4 rows
   const bool s35 = a.H == 2048 && a.I == 512;
-  void (*kern)(FlowArgs) = F == kFmtNv ? (s35 ? k_dec_flow<2048, 512, kFmtNv> : k_dec_flow<0, 0, kFmtNv>)
-                           : F == kFmtBf16 ? (s35 ? k_dec_flow<2048, 512, kFmtBf16> : k_dec_flow<0, 0, kFmtBf16>)
-                                           : (s35 ? k_dec_flow<2048, 512, kFmtMx> : k_dec_flow<0, 0, kFmtMx>);
+  void (*kern)(FlowArgs) =
+      F == kFmtNv     ? (s35 ? k_dec_flow<2048, 512, kFmtNv, 0, 0> : k_dec_flow<0, 0, kFmtNv, 0, 0>)
+      : F == kFmtBf16 ? (s35 ? k_dec_flow<2048, 512, kFmtBf16, 0, 0> : k_dec_flow<0, 0, kFmtBf16, 0, 0>)
+      : s35           ? (a.T == 1 ? k_dec_flow<2048, 512, kFmtMx, 1, 4> : k_dec_flow<2048, 512, kFmtMx, 0, 0>)
+                      : k_dec_flow<0, 0, kFmtMx, 0, 0>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fg.smem);
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 0, occ = 0;

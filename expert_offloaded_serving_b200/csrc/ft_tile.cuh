@@ -483,7 +483,10 @@ __device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8
 }
 
 // Partial sums of every row of the staged tile for n (<= kMT) tokens into red.
-template <int F = kFmtMx>
+// NTF, RUF: tokens per pass and rows per step fixed at compile time (a build
+// for one tile shape and batch carries only that loop), or 0 for the choice
+// at run time; a fixed NTF = 1 takes n = 1 only.
+template <int F = kFmtMx, int NTF = 0, int RUF = 0>
 __device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t* base, int n) {
   if (!m.on) return;
   uint32_t x[kMT][16];
@@ -498,10 +501,15 @@ __device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t
   // (BF16 holds 32 fp32 activations per token: at most 2 rows at a time, so
   // that the registers suffice; the reduction tree does not depend on it)
   const int per = g.R % g.groups == 0 ? g.R / g.groups : 0;
-  const int ru = (F != kFmtBf16 && per % 4 == 0 && per > 0 && g.lpr >= 4) ? 4
+  const int ru = RUF ? RUF
+                 : (F != kFmtBf16 && per % 4 == 0 && per > 0 && g.lpr >= 4) ? 4
                  : (per % 2 == 0 && per > 0 && g.lpr >= 2)                ? 2
                                                                            : 1;
-  if (n > 1) {
+  if constexpr (NTF == 1 && RUF != 0) {
+    tile_dots_t<RUF, 1, F>(g, m, base, x, xi, xf);
+    return;
+  }
+  if (NTF != 1 && n > 1) {
     if (ru == 4) tile_dots_t<4, 2, F>(g, m, base, x, xi, xf);
     else if (ru == 2) tile_dots_t<2, 2, F>(g, m, base, x, xi, xf);
     else tile_dots_t<1, 2, F>(g, m, base, x, xi, xf);
