@@ -490,46 +490,49 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_dec_flow(FlowArgs a) {
         __syncthreads();
         if (d == b) stamp(5);
         const int n0 = d * rb, nv = min(rb, H - n0), half = nv / 2;
-        for (int i = threadIdx.x; i < T * half; i += kGemvThreads) {
+        // warp w combines output pairs w, w + 16, ...: lane j < k loads routed
+        // pair j's two y values, lane k + s the shared expert s's; the sum is
+        // taken in the fixed order (routed pairs ascending by fused
+        // multiply-add, then the shared experts) from the lanes' values
+        const int lane = threadIdx.x & 31;
+        for (int i = threadIdx.x >> 5; i < T * half; i += kWarpsF) {
           const int t = i / half, nl = 2 * (i - t * half);
-          float o[2] = {0.f, 0.f};
-          // the routed pairs four at a time: their loads first, then the
-          // multiply-adds in ascending j
-          for (int j0 = 0; j0 < k; j0 += 4) {
-            float w4[4], y4[4][2];
-#pragma unroll
-            for (int jj = 0; jj < 4; jj++) {
-              w4[jj] = 0.f;
-              y4[jj][0] = y4[jj][1] = 0.f;
-              if (j0 + jj < k) {
-                const FlowPair q = pr[t * k + j0 + jj];
-                w4[jj] = q.w;
-                const float ts = F == kFmtNv ? un[q.unit].ts[2] : 1.f;
-#pragma unroll
-                for (int e = 0; e < 2; e++) {
-                  float y = q.on ? dtile_y(gB, baseB, q.unit * rb + nl + e, q.slot) : 0.f;
-                  if (F == kFmtNv) y *= ts;
-                  y4[jj][e] = y;
-                }
+          float w = 0.f, y0 = 0.f, y1 = 0.f;
+          if (lane < k) {
+            const FlowPair q = pr[t * k + lane];
+            w = q.w;
+            if (q.on) {
+              const float ts = F == kFmtNv ? un[q.unit].ts[2] : 1.f;
+              y0 = dtile_y(gB, baseB, q.unit * rb + nl, q.slot);
+              y1 = dtile_y(gB, baseB, q.unit * rb + nl + 1, q.slot);
+              if (F == kFmtNv) {
+                y0 *= ts;
+                y1 *= ts;
               }
             }
-#pragma unroll
-            for (int jj = 0; jj < 4; jj++)
-              if (j0 + jj < k)
-#pragma unroll
-                for (int e = 0; e < 2; e++) o[e] = fmaf(w4[jj], y4[jj][e], o[e]);
-          }
-          for (int s2 = 0; s2 < S; s2++) {
-            const int u = na + s2;
-            const bool on = un[u].blob != nullptr;
-            const float ts = F == kFmtNv ? un[u].ts[2] : 1.f;
-#pragma unroll
-            for (int e = 0; e < 2; e++) {
-              float y = on ? dtile_y(gB, baseB, u * rb + nl + e, t) : 0.f;
-              if (F == kFmtNv) y *= ts;
-              o[e] += y;
+          } else if (lane < k + S) {
+            const int u = na + (lane - k);
+            if (un[u].blob) {
+              const float ts = F == kFmtNv ? un[u].ts[2] : 1.f;
+              y0 = dtile_y(gB, baseB, u * rb + nl, t);
+              y1 = dtile_y(gB, baseB, u * rb + nl + 1, t);
+              if (F == kFmtNv) {
+                y0 *= ts;
+                y1 *= ts;
+              }
             }
           }
+          float o[2] = {0.f, 0.f};
+          for (int j = 0; j < k; j++) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            o[0] = fmaf(wj, __shfl_sync(0xffffffffu, y0, j), o[0]);
+            o[1] = fmaf(wj, __shfl_sync(0xffffffffu, y1, j), o[1]);
+          }
+          for (int s2 = 0; s2 < S; s2++) {
+            o[0] += __shfl_sync(0xffffffffu, y0, k + s2);
+            o[1] += __shfl_sync(0xffffffffu, y1, k + s2);
+          }
+          if (lane != 0) continue;
           __nv_bfloat162 bb = __floats2bfloat162_rn(o[0], o[1]);
           const uint32_t pairbits = *reinterpret_cast<uint32_t*>(&bb);
           const size_t at = (size_t)t * H + n0 + nl;
