@@ -80,7 +80,8 @@ def test_a_35b_class_layer_under_the_decode_arithmetic_stays_inside_the_toleranc
     per block, fp32 block sums, h = silu(g) * u in fp32 re-encoded to 11 bits,
     the combine in fp32 over the ranks in order, one bf16 rounding.  Against
     the fp64 oracle the error before that rounding is about 2e-4 (relative
-    L2; mostly the 11-bit h), while rounding the exact result to bf16 alone
+    L2; mostly the 11-bit h, as the A/B with h kept in fp32 shows), while
+    rounding the exact result to bf16 alone
     gives about 1.6e-3: the arithmetic raises the output's error by under 5 %
     over that floor, and the output meets the layer tolerance (max abs 2e-2,
     relative L2 2e-3)."""
@@ -95,18 +96,26 @@ def test_a_35b_class_layer_under_the_decode_arithmetic_stays_inside_the_toleranc
     x = reencode_rows(fp4.bf16_to_f64(xb))[0]
     assert np.array_equal(x, fp4.bf16_to_f64(xb)[0])             # bf16 x passes exactly
 
-    def expert(blob):
+    def expert(blob, h11=True):
         g = gemv_fp32(formats.weight_matrix(blob, "wg", H, I), x)
         u = gemv_fp32(formats.weight_matrix(blob, "wu", H, I), x)
         h = (g / (np.float32(1) + np.exp(-g))) * u                 # fp32
-        return gemv_fp32(formats.weight_matrix(blob, "wd", H, I), reencode_rows(h[None, :])[0])
-    acc = np.zeros(H, np.float32)
-    for j in range(k):
-        acc = np.float32(r["w"][0, j]) * expert(blobs[int(r["ids"][0, j])]) + acc
-    acc = acc + expert(blobs[E])
+        hq = reencode_rows(h[None, :])[0] if h11 else h.astype(np.float64)
+        return gemv_fp32(formats.weight_matrix(blob, "wd", H, I), hq)
+
+    def layer_out(h11):
+        acc = np.zeros(H, np.float32)
+        for j in range(k):
+            acc = np.float32(r["w"][0, j]) * expert(blobs[int(r["ids"][0, j])], h11) + acc
+        return acc + expert(blobs[E], h11)
+    acc = layer_out(True)
     want = r["out_f64"][0]
     nrm = np.linalg.norm(want)
     pre = np.linalg.norm(acc.astype(np.float64) - want) / nrm
+    # the A/B: the same arithmetic with h kept in fp32 (no 11-bit rounding)
+    pre_exact_h = np.linalg.norm(layer_out(False).astype(np.float64) - want) / nrm
+    print(f"relative L2 before the bf16 rounding: 11-bit h {pre:.2e}, fp32 h {pre_exact_h:.2e}")
+    assert pre_exact_h < pre
     out = fp4.bf16_to_f64(fp4.round_bf16(acc.astype(np.float64)))
     rel = np.linalg.norm(out - want) / nrm
     floor = np.linalg.norm(fp4.bf16_to_f64(r["out_bits"][0]) - want) / nrm   # the exact result, rounded
