@@ -172,6 +172,13 @@ TRACE_LEN = 512
 STACK_TRAFFIC_PER_BYTE = (60254976 + 1071616) / 60162048
 
 
+# The arithmetic of the decode GEMVs: MXFP4 and NVFP4 weights decode exactly
+# to f16 and meet f16-encoded activations (x exact, h to 11 bits) in fused
+# multiply-adds that accumulate in fp32; BF16 weights widen exactly to fp32
+# and meet fp32 activations.
+DECODE_DTYPE = {"mxfp4": "f16*f16+f32", "nvfp4": "f16*f16+f32", "bf16": "f32"}
+
+
 def decode_routing(T):
     """Per token position p < TRACE_LEN: sets [L][T][k] of T independent sequences."""
     import numpy as np
@@ -925,7 +932,7 @@ def main():
     rk_gbs = rk_bytes / (rk_us * 1e-6) / 1e9
     line = {"metric": METRIC, "value": res["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": DECODE_DTYPE[args.format], "data": "synthetic",
             "config": workload_config(T, args.layerwise, args.counters, args.format),
             "roofline": {"bound": "hbm", "kernel": rk, "achieved": rk_gbs, "peak": pk["hbm"],
                          "peak_source": pk["src"], "unit": "GB/s", "frac": rk_gbs / pk["hbm"], "traffic": rk_traffic,

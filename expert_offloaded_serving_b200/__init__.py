@@ -126,7 +126,8 @@ def lib() -> C.CDLL:
 
 
 def _ptr(t, size: int | None = None) -> int | None:
-    """Device/host pointer of a torch tensor, an int, or None.  The ABI takes
+    """Device/host pointer of a torch tensor, a numpy array (host), an int, or
+    None.  The ABI takes
     dense row-major buffers, so a strided view is refused rather than read
     with the wrong layout; `size` is the element size in bytes the argument
     holds (2 for bf16 activations, 4 for fp32 / int32, 1 for codes), checked
@@ -135,6 +136,13 @@ def _ptr(t, size: int | None = None) -> int | None:
         return None
     if isinstance(t, int):
         return t
+    if hasattr(t, "__array_interface__") and not hasattr(t, "is_contiguous"):  # a numpy host buffer
+        if not t.flags["C_CONTIGUOUS"]:
+            raise ValueError(f"array of shape {t.shape} is not C-contiguous; the C ABI takes dense row-major buffers")
+        if size is not None and t.itemsize != size:
+            raise ValueError(f"array of dtype {t.dtype} has {t.itemsize}-byte elements where the C ABI "
+                             f"takes {size}-byte ones")
+        return t.ctypes.data
     if not t.is_contiguous():
         raise ValueError(f"tensor of shape {tuple(t.shape)} and strides {t.stride()} is not contiguous; "
                          "the C ABI takes dense row-major buffers")

@@ -106,3 +106,17 @@ def test_binding_refuses_wrong_element_sizes():
     with pytest.raises(ValueError, match="4-byte"):
         ft.ft_moe_route(0, torch.zeros(4, 16), 4, 16, 2, 1, torch.zeros(4, 2, dtype=torch.int64), torch.zeros(4, 2),
                         0)
+
+
+def test_binding_takes_numpy_host_buffers():
+    """Host pools may be numpy arrays (pageable memory the context pins): the
+    binding passes their data pointer, and refuses strided ones like tensors."""
+    import numpy as np
+    a = np.zeros(64, np.uint8)
+    assert ft._ptr(a) == a.ctypes.data
+    f = np.zeros(4, np.float32)
+    assert ft._ptr(f, 4) == f.ctypes.data
+    with pytest.raises(ValueError, match="not C-contiguous"):
+        ft._ptr(np.zeros((4, 4), np.uint8)[:, ::2])
+    with pytest.raises(ValueError, match="4-byte"):
+        ft._ptr(np.zeros(4, np.float64), 4)
