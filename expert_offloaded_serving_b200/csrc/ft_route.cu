@@ -85,46 +85,56 @@ __global__ void __launch_bounds__(256, 1) k_router_logits_tiled(const uint16_t* 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tw = warp >> 1, ew = warp & 1;
   const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
-  // staging: thread i loads elements 16(i%8) .. +15 of token i/8, and
-  // elements 8(i%16) .. +7 of expert i/16
-  const int st = threadIdx.x >> 3, sp = threadIdx.x & 7;
-  const int se = threadIdx.x >> 4, sq = threadIdx.x & 15;
-  const bool tok_ok = t0 + st < T, exp_ok = e0 + se < E;
-  const uint4* xg = reinterpret_cast<const uint4*>(x + (size_t)(tok_ok ? t0 + st : 0) * H) + 2 * sp;
-  const float4* wg = reinterpret_cast<const float4*>(wr + (size_t)(exp_ok ? e0 + se : 0) * H) + 2 * sq;
+  // staging: lane j of warp w loads elements 4j .. 4j+3 of tokens w, w + 8,
+  // w + 16, w + 24 and of experts w, w + 8, and stores element 4j + v at
+  // [v][j]: a warp's loads are contiguous and its stores 32 consecutive
+  // doubles (no bank conflicts)
+  const uint2* xg[4];
+  bool tok_ok[4];
+#pragma unroll
+  for (int m = 0; m < 4; m++) {
+    const int t = t0 + warp + 8 * m;
+    tok_ok[m] = t < T;
+    xg[m] = reinterpret_cast<const uint2*>(x + (size_t)(tok_ok[m] ? t : 0) * H) + lane;
+  }
+  const float4* wg[2];
+  bool exp_ok[2];
+#pragma unroll
+  for (int m = 0; m < 2; m++) {
+    const int e = e0 + warp + 8 * m;
+    exp_ok[m] = e < E;
+    wg[m] = reinterpret_cast<const float4*>(wr + (size_t)(exp_ok[m] ? e : 0) * H) + lane;
+  }
   // two register sets of staged loads, named apart so that a set chosen at
   // run time still lives in registers
-  uint4 xr0[2], xr1[2];
+  uint2 xr0[4], xr1[4];
   float4 wq0[2], wq1[2];
-  auto gload_into = [&](int c, uint4 (&xr)[2], float4 (&wq)[2]) {
+  auto gload_into = [&](int c, uint2 (&xr)[4], float4 (&wq)[2]) {
 #pragma unroll
-    for (int i = 0; i < 2; i++) {
-      xr[i] = tok_ok ? __ldg(xg + c * 16 + i) : make_uint4(0u, 0u, 0u, 0u);
-      wq[i] = exp_ok ? __ldg(wg + c * 32 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int m = 0; m < 4; m++) xr[m] = tok_ok[m] ? __ldg(xg[m] + c * 32) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int m = 0; m < 2; m++) wq[m] = exp_ok[m] ? __ldg(wg[m] + c * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   auto gload = [&](int c, int set) {
     if (set == 0) gload_into(c, xr0, wq0);
     else gload_into(c, xr1, wq1);
   };
-  auto sstore_from = [&](int buf, const uint4 (&xr)[2], const float4 (&wq)[2]) {
-    double* xd = xs + ((size_t)buf * kRtT + st) * 128;
-    double* wd = ws + ((size_t)buf * kRtE + se) * 128;
+  auto sstore_from = [&](int buf, const uint2 (&xr)[4], const float4 (&wq)[2]) {
 #pragma unroll
-    for (int i = 0; i < 2; i++) {
-      const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
+    for (int m = 0; m < 4; m++) {
+      double* xd = xs + ((size_t)buf * kRtT + warp + 8 * m) * 128 + lane;
+      xd[0] = f32_to_f64(bf16_bits_to_f32((uint16_t)(xr[m].x & 0xffffu)));
+      xd[32] = f32_to_f64(bf16_bits_to_f32((uint16_t)(xr[m].x >> 16)));
+      xd[64] = f32_to_f64(bf16_bits_to_f32((uint16_t)(xr[m].y & 0xffffu)));
+      xd[96] = f32_to_f64(bf16_bits_to_f32((uint16_t)(xr[m].y >> 16)));
+    }
 #pragma unroll
-      for (int h = 0; h < 8; h++) {
-        const int kk = 16 * sp + 8 * i + h;  // element of the block
-        const uint16_t b = (uint16_t)((h & 1) ? (u[h >> 1] >> 16) : (u[h >> 1] & 0xffffu));
-        xd[(kk & 3) * 32 + (kk >> 2)] = f32_to_f64(bf16_bits_to_f32(b));
-      }
-      const float f[4] = {wq[i].x, wq[i].y, wq[i].z, wq[i].w};
-#pragma unroll
-      for (int h = 0; h < 4; h++) {
-        const int kk = 8 * sq + 4 * i + h;
-        wd[(kk & 3) * 32 + (kk >> 2)] = f32_to_f64(f[h]);
-      }
+    for (int m = 0; m < 2; m++) {
+      double* wd = ws + ((size_t)buf * kRtE + warp + 8 * m) * 128 + lane;
+      wd[0] = f32_to_f64(wq[m].x);
+      wd[32] = f32_to_f64(wq[m].y);
+      wd[64] = f32_to_f64(wq[m].z);
+      wd[96] = f32_to_f64(wq[m].w);
     }
   };
   auto sstore = [&](int buf, int set) {
