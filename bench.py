@@ -40,8 +40,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 or 4)")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
-    ap.add_argument("--case", default="decode", choices=["decode", "prefill", "miss", "glm"],
-                    help="decode: the 35B-class decode stack (default line); prefill / miss: only that measurement")
+    ap.add_argument("--case", default="decode", choices=["decode", "prefill", "miss", "glm", "gemm", "router"],
+                    help="decode: the 35B-class decode stack (default line); prefill / miss / glm: only that "
+                         "measurement; gemm / router: the prefill GEMMs or router GEMV alone on a small case "
+                         "(the ncu captures' workloads)")
     ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     ap.add_argument("--layerwise", action="store_true",
                     help="decode with two kernels per layer instead of a persistent stack kernel")
@@ -642,6 +644,67 @@ def measure_prefill_calibration(fp4_peak, T=65536, reps=2):
             "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps}
 
 
+def measure_gemm_small(reps=2, T=16384, E2=64):
+    """The prefill GEMMs at the calibration case's 1,536 tokens per expert on
+    a small pool: the DSV4-class expert shape (hidden 4096, intermediate
+    2048, top-6) with 64 experts and 16,384 tokens (0.8 GB of experts), one
+    warm forward and `reps` timed ones through the MXFP4-activation path.
+    The workload of the GEMMs' ncu capture (a few GB on the device)."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+    H2, I2, k2, seed = 4096, 2048, 6, 1005
+    pool = synth.gpu.layer_pool(H2, I2, E2, seed, 0)
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, 1, 0, 0, T), None, [pool])
+    x = torch.from_numpy(synth.activations_bf16(seed, 1, T, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    lg = torch.from_numpy(synth.logits_for_sets(seed, 3, synth.near_uniform_sets(seed, 0, T, E2, k2), E2)).cuda()
+    out = torch.empty_like(x)
+    flags = ft.FT_ACT_MXFP4 | ft.FT_ROUTE_RENORM
+    ft.ft_moe_layer_forward(ctx, 0, x, T, None, lg, out, flags)
+    torch.cuda.synchronize()
+    ft.ft_kernel_timing_enable(ctx, True)
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, x, T, None, lg, out, flags)
+    kt = ft.ft_kernel_timing_read(ctx)
+    ft.ft_kernel_timing_enable(ctx, False)
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    gemm_ms = (kt["gemm_gate_up"][0] + kt["gemm_down"][0]) / reps
+    flops = 2.0 * T * k2 * 3 * H2 * I2
+    return {"workload": f"DSV4-shape prefill GEMMs, {E2} experts, {T} tokens top-{k2} ({T * k2 // E2} per expert)",
+            "gemm_ms": gemm_ms, "gemm_tflops": flops / (gemm_ms * 1e-3) / 1e12,
+            "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps}
+
+
+def measure_router(reps=5, T=4096, H2=4096, E2=256):
+    """The router GEMV of the DSV4-class prefill layer alone (4096 tokens x
+    256 experts x hidden 4096, fp64 fixed order), through ft_router_logits:
+    one warm call and `reps` timed ones.  The workload of its ncu capture."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    ctx = ft.ft_create(ft.make_desc(H2, 2048, E2, 6, 1, 0, 0, T))
+    x = torch.from_numpy(synth.activations_bf16(1, 1, T, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    wr = torch.from_numpy(synth.router_weights(1, 0, E2, H2)).cuda()
+    lg = torch.empty((T, E2), dtype=torch.float32, device="cuda")
+    ft.ft_router_logits(ctx, x, T, H2, wr, E2, lg)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ft.ft_router_logits(ctx, x, T, H2, wr, E2, lg)
+    e1.record()
+    torch.cuda.synchronize()
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    ms = e0.elapsed_time(e1) / reps
+    return {"workload": f"router logits, {T} tokens x {E2} experts x hidden {H2}, fp64 fixed order",
+            "ms": ms, "fp64_fma_per_s": T * E2 * H2 / (ms * 1e-3)}
+
+
 def measure_misses(tokens=512, layers=43, resize_at=(170, 340)):
     """DeepSeek-V4-Flash-class decode over a GPU LRU expert cache (hidden
     4096, 256 experts top-6, intermediate 2048): `layers` layers (43 = the
@@ -893,7 +956,8 @@ def main():
     if args.case != "decode":
         if rank == 0:
             r = {"prefill": lambda: measure_prefill(reps=max(args.steps, 1)), "miss": measure_misses,
-                 "glm": measure_glm}[args.case]()
+                 "glm": measure_glm, "gemm": lambda: measure_gemm_small(reps=max(args.steps, 1)),
+                 "router": lambda: measure_router(reps=max(args.steps, 1))}[args.case]()
             print(json.dumps({"case": args.case, **r}))
         return
     if args.impl == "reference":

@@ -580,12 +580,13 @@ cudaError_t launch_dec_flow(const FlowArgs& a, cudaStream_t s) {
   if (!fg.ok || a.rows_cap != fg.rows_cap) return cudaErrorInvalidValue;
   // the 35B-class shape (hidden 2048, intermediate 512) has its own builds;
   // MXFP4 at one token also a build with only the one-token loops, whose
-  // gate/up tile (32 rows of each matrix, 8 lane groups) steps 4 rows
+  // gate/up tile (32 rows of each matrix, 8 lane groups) takes 4 rows of
+  // each matrix in one step
   const bool s35 = a.H == 2048 && a.I == 512;
   void (*kern)(FlowArgs) =
       F == kFmtNv     ? (s35 ? k_dec_flow<2048, 512, kFmtNv, 0, 0> : k_dec_flow<0, 0, kFmtNv, 0, 0>)
       : F == kFmtBf16 ? (s35 ? k_dec_flow<2048, 512, kFmtBf16, 0, 0> : k_dec_flow<0, 0, kFmtBf16, 0, 0>)
-      : s35           ? (a.T == 1 ? k_dec_flow<2048, 512, kFmtMx, 1, 4> : k_dec_flow<2048, 512, kFmtMx, 0, 0>)
+      : s35           ? (a.T == 1 ? k_dec_flow<2048, 512, kFmtMx, 1, 8> : k_dec_flow<2048, 512, kFmtMx, 0, 0>)
                       : k_dec_flow<0, 0, kFmtMx, 0, 0>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fg.smem);
   if (e != cudaSuccess) return e;

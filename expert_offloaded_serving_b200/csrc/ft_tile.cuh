@@ -379,6 +379,52 @@ __device__ __forceinline__ int group_reduce(float (&v)[4][kMT], int lpr) {
   return row;
 }
 
+// The same reduction over eight rows v[0..7]: a first exchange step keeps
+// four of them, then the four-row steps.  Lanes pair by the same bits in the
+// same order as above, so every row's sum is bit for bit the one a smaller
+// step gives.  Needs lpr >= 8; returns the row this lane holds.
+template <int NT>
+__device__ __forceinline__ int group_reduce8(float (&v)[8][kMT], int lpr) {
+  const int lane = threadIdx.x & 31;
+  int d = lpr >> 1;
+  const bool hi = lane & d;
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const float sd = hi ? v[i][t] : v[4 + i][t], kp = hi ? v[4 + i][t] : v[i][t];
+      v[i][t] = kp + __shfl_xor_sync(0xffffffffu, sd, d);
+    }
+  int row = hi ? 4 : 0;
+  d >>= 1;
+  {
+    const bool h2 = lane & d;
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const float s0 = h2 ? v[0][t] : v[2][t], s1 = h2 ? v[1][t] : v[3][t];
+      const float k0 = h2 ? v[2][t] : v[0][t], k1 = h2 ? v[3][t] : v[1][t];
+      v[0][t] = k0 + __shfl_xor_sync(0xffffffffu, s0, d);
+      v[1][t] = k1 + __shfl_xor_sync(0xffffffffu, s1, d);
+    }
+    row += h2 ? 2 : 0;
+    d >>= 1;
+  }
+  {
+    const bool h3 = lane & d;
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const float sd = h3 ? v[0][t] : v[1][t], kp = h3 ? v[1][t] : v[0][t];
+      v[0][t] = kp + __shfl_xor_sync(0xffffffffu, sd, d);
+    }
+    row += h3 ? 1 : 0;
+    d >>= 1;
+  }
+  for (; d >= 1; d >>= 1)
+#pragma unroll
+    for (int t = 0; t < NT; t++) v[0][t] += __shfl_xor_sync(0xffffffffu, v[0][t], d);
+  return row;
+}
+
 // Value of chunk c of staged row `row` for NT tokens, before the row's
 // reduction over its lanes: MXFP4 chunk sum x (scale x inverse factor);
 // NVFP4 (half sum x scale, added) x inverse factor; BF16 the fp32 dot.
@@ -482,10 +528,36 @@ __device__ __forceinline__ void tile_dots_t(const Gv& g, const LaneMap& m, uint8
   }
 }
 
+// A two-matrix tile with R = 4 * groups in one step of eight rows per lane
+// group (rows grp + j*groups of both matrices, j < 4).
+template <int NT, int F>
+__device__ __forceinline__ void tile_dots_fused8(const Gv& g, const LaneMap& m, uint8_t* base,
+                                                 const uint32_t (&x)[kMT][16], const float (&xi)[kMT],
+                                                 const float (&xf)[kMT][32]) {
+  const uint8_t* codes = base + g.codes;
+  const uint32_t* sc = reinterpret_cast<const uint32_t*>(base + g.scales);
+  float* red = reinterpret_cast<float*>(base + g.red);
+  const bool cv = m.c < g.chunks;
+  float v[8][kMT];
+#pragma unroll
+  for (int u = 0; u < 8; u++) {
+    v[u][0] = v[u][1] = 0.f;
+    if (cv) chunk_value<NT, F>(g, codes, sc, (u >> 2) * g.R + m.grp + (u & 3) * g.groups, m.c, x, xi, xf, v[u]);
+  }
+  const int u = group_reduce8<NT>(v, g.lpr);
+  if (((threadIdx.x & 31) & ((g.lpr >> 3) - 1)) == 0) {
+    const int mat = u >> 2, r = m.grp + (u & 3) * g.groups;
+    float* o = red + ((size_t)(m.part * g.nmat + mat) * g.R + r) * kMT;
+#pragma unroll
+    for (int t = 0; t < NT; t++) o[t] = v[0][t];
+  }
+}
+
 // Partial sums of every row of the staged tile for n (<= kMT) tokens into red.
 // NTF, RUF: tokens per pass and rows per step fixed at compile time (a build
 // for one tile shape and batch carries only that loop), or 0 for the choice
-// at run time; a fixed NTF = 1 takes n = 1 only.
+// at run time; a fixed NTF = 1 takes n = 1 only; RUF = 8 takes a two-matrix
+// tile with R = 4 * groups in one step.
 template <int F = kFmtMx, int NTF = 0, int RUF = 0>
 __device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t* base, int n) {
   if (!m.on) return;
@@ -505,7 +577,10 @@ __device__ __forceinline__ void tile_dots(const Gv& g, const LaneMap& m, uint8_t
                  : (F != kFmtBf16 && per % 4 == 0 && per > 0 && g.lpr >= 4) ? 4
                  : (per % 2 == 0 && per > 0 && g.lpr >= 2)                ? 2
                                                                            : 1;
-  if constexpr (NTF == 1 && RUF != 0) {
+  if constexpr (NTF == 1 && RUF == 8) {  // both matrices of a gate/up tile in one step
+    tile_dots_fused8<1, F>(g, m, base, x, xi, xf);
+    return;
+  } else if constexpr (NTF == 1 && RUF != 0) {
     tile_dots_t<RUF, 1, F>(g, m, base, x, xi, xf);
     return;
   }
