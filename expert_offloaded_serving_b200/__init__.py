@@ -189,9 +189,16 @@ def ft_blob_layout_format(hidden: int, inter: int, fmt: int) -> dict:
     return dict(zip(("wg", "wu", "wd", "wg_sf", "wu_sf", "wd_sf", "used", "stride", "ts"), list(out)))
 
 
+# Buffers a context borrows (its host and resident pools), held here from
+# ft_create until ft_destroy: the library keeps their addresses, so a tensor
+# the caller dropped must not return to torch's allocator meanwhile.
+_borrowed: dict[int, tuple] = {}
+
+
 def ft_create(desc: ModelDesc, host_layers=None, resident_layers=None) -> int:
     """Returns the context handle.  host_layers / resident_layers: sequences of
-    per-layer pointers (tensors, ints or None) or None."""
+    per-layer pointers (tensors, numpy arrays, ints or None) or None; the
+    objects are held until ft_destroy of the handle."""
     L = desc.n_layers
 
     def arr(seq):
@@ -205,11 +212,16 @@ def ft_create(desc: ModelDesc, host_layers=None, resident_layers=None) -> int:
     out = P()
     _check(lib().ft_create(C.byref(desc), C.cast(h, P) if h is not None else None,
                            C.cast(r, P) if r is not None else None, C.byref(out)))
+    _borrowed[out.value] = (None if host_layers is None else list(host_layers),
+                            None if resident_layers is None else list(resident_layers))
     return out.value
 
 
 def ft_destroy(ctx: int) -> None:
-    _check(lib().ft_destroy(ctx))
+    try:
+        _check(lib().ft_destroy(ctx))
+    finally:
+        _borrowed.pop(ctx, None)
 
 
 def ft_sync_status(ctx: int, stream=None) -> None:

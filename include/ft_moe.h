@@ -161,7 +161,8 @@ FT_API const char* ft_last_error(void);
  *                   ([fa] elastic memory management).
  *   resident_layers host [L] pointers (or NULL): per-layer device copies of
  *                   the same pools; a layer with a non-NULL entry is served
- *                   from it and never touches the cache.
+ *                   from it and never touches the cache.  The context
+ *                   borrows them: they must outlive it as well.
  *   The library allocates the cache slot arena (CUDA virtual memory, sized by
  *   desc->cache_budget_bytes), device scratch for desc->max_tokens tokens,
  *   a copy stream and events.  Prefill staging buffers (2 layer pools) are

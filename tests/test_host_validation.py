@@ -120,3 +120,35 @@ def test_binding_takes_numpy_host_buffers():
         ft._ptr(np.zeros((4, 4), np.uint8)[:, ::2])
     with pytest.raises(ValueError, match="4-byte"):
         ft._ptr(np.zeros(4, np.float64), 4)
+
+
+def test_binding_holds_borrowed_pools_until_destroy(monkeypatch):
+    """The context keeps the addresses of its host and resident pools, so the
+    binding holds the objects from ft_create to ft_destroy: a pool passed
+    inline and dropped by the caller must not go back to the allocator (and
+    be reused under the context) meanwhile.  A fake library stands in for the
+    C calls."""
+    import gc
+    import weakref
+
+    import numpy as np
+
+    class FakeLib:
+        def ft_create(self, desc, host, res, out):
+            out._obj.value = 0x7000
+            return ft.FT_OK
+
+        def ft_destroy(self, ctx):
+            return ft.FT_OK
+
+    monkeypatch.setattr(ft, "lib", lambda: FakeLib())
+    host, res = np.zeros(64, np.uint8), np.zeros(64, np.uint8)
+    wh, wr = weakref.ref(host), weakref.ref(res)
+    d = ft.make_desc(256, 128, 16, 2, 1, 0, 0, 16)
+    h = ft.ft_create(d, [host], [res])
+    del host, res
+    gc.collect()
+    assert wh() is not None and wr() is not None
+    ft.ft_destroy(h)
+    gc.collect()
+    assert wh() is None and wr() is None
