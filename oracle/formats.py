@@ -157,3 +157,83 @@ def weight_matrix(blob: np.ndarray, which: str, hidden: int, inter: int, weights
     if weights == "bf16":
         return bf16_matrix(blob, which, hidden, inter)
     raise ValueError(f"unknown weight format {weights!r}")
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 activations (the prefill path of NVFP4 experts)
+# ---------------------------------------------------------------------------
+#
+# The pages name NVFP4 and do not define how activations are scaled.  The
+# reading taken is the usual two-level one for a block-scaled FP4 product: a
+# per-tensor fp32 scale s = amax / (448 * 6) over the whole matrix the GEMM
+# reads (all tokens of x; all h rows of the layer), so that the block scale of
+# the largest block lands on E4M3's largest value; per 16 values a block scale
+# E4M3(amax_block / (6 s)); codes e2m1(v / (block scale * s)).  Each of those
+# steps is a rounding that decides a byte, so it is taken in fp32, as the
+# kernel takes it: one fp32 multiply or divide per step, rounded to nearest
+# even.  A block whose scale is zero (or whose block scale times s underflows
+# to zero) has all codes +0.  Dequantised value: code x block scale x s.
+
+NVFP4_GLOBAL_DIV = np.float32(448.0 * 6.0)
+_E4M3_POS = E4M3_TABLE[:0x7F]          # bytes 0x00 .. 0x7e: 0 .. 448, ascending
+
+
+def e4m3_round(v: float) -> int:
+    """E4M3 byte of v >= 0 by brute force: the nearest of the 127 finite
+    non-negative values, ties to the even byte (even mantissa), values at or
+    above 448 saturating to 448 (0x7e)."""
+    if v >= 448.0:
+        return 0x7E
+    best = None
+    for b in range(0x7F):
+        d = abs(v - _E4M3_POS[b])
+        if best is None or d < best[0] or (d == best[0] and b % 2 == 0):
+            best = (d, b)
+    return best[1]
+
+
+def e4m3_round_vec(v: np.ndarray) -> np.ndarray:
+    """Vectorised ``e4m3_round`` (v >= 0): the two table neighbours of each
+    value, the nearer one, ties to the even byte."""
+    v = np.asarray(v, dtype=np.float64)
+    hi = np.clip(np.searchsorted(_E4M3_POS, v, side="left"), 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    dl = np.abs(v - _E4M3_POS[lo])
+    dh = np.abs(_E4M3_POS[hi] - v)
+    pick = np.where(dl < dh, lo, np.where(dh < dl, hi, np.where(lo % 2 == 0, lo, hi)))
+    return np.where(v >= 448.0, 0x7E, pick).astype(np.uint8)
+
+
+def nvfp4_global_scale(amax) -> np.float32:
+    """Per-tensor scale: fp32(amax) / 2688, one fp32 division."""
+    with np.errstate(all="ignore"):
+        return np.float32(np.float32(amax) / NVFP4_GLOBAL_DIV)
+
+
+def nvfp4_quantize_rows(v: np.ndarray, s=None) -> tuple[np.ndarray, np.ndarray, np.float32]:
+    """Quantise v [R, K] (values exact in fp32) to NVFP4: element codes [R, K],
+    E4M3 block-scale bytes [R, K/16] and the per-tensor scale s (fp32; None:
+    from the maximum magnitude of v)."""
+    v32 = np.asarray(v, dtype=np.float32)
+    R, K = v32.shape
+    if s is None:
+        s = nvfp4_global_scale(np.abs(v32).max() if v32.size else 0.0)
+    s = np.float32(s)
+    blocks = v32.reshape(R, K // 16, 16)
+    if s == 0:
+        return np.zeros((R, K), np.uint8), np.zeros((R, K // 16), np.uint8), s
+    with np.errstate(all="ignore"):
+        t = np.float32(s * np.float32(6.0))
+        b = (np.abs(blocks).max(axis=-1) / t).astype(np.float32)
+        e = e4m3_round_vec(b)
+        dq = (E4M3_TABLE[e].astype(np.float32) * s).astype(np.float32)
+        q = (blocks / np.where(dq > 0, dq, np.float32(1.0))[..., None]).astype(np.float32)
+    mag = fp4.round_to_grid_vec(np.abs(q).astype(np.float64))
+    codes = mag | np.where(np.signbit(q), 8, 0)
+    codes = np.where((dq > 0)[..., None], codes, 0).astype(np.uint8).reshape(R, K)
+    return codes, e.astype(np.uint8), s
+
+
+def nvfp4_dequant_rows(codes: np.ndarray, scales: np.ndarray, s) -> np.ndarray:
+    """Inverse of ``nvfp4_quantize_rows`` in fp64 (exact products)."""
+    return fp4.E2M1_TABLE[codes] * np.repeat(E4M3_TABLE[scales], 16, axis=1) * float(np.float32(s))

@@ -1,0 +1,125 @@
+"""Pins of the oracle's NVFP4 activation quantiser and of the NVFP4-activation
+layer mode: E4M3 rounding against torch's float8_e4m3fn cast and the format's
+own values, a block quantised by hand on power-of-two scales (every code and
+scale byte worked out below, ties included), the zero, underflow and all-zero
+cases, the dequantisation error bound on random data, and the layer's output
+within its quantisation error of the exact layer.
+
+Pages: the NVFP4 build of Qwen3.6-35B-A3B (jansverre.net, "Hvor raskt kjører
+modellene?"); the two-level scaling is the reading stated in the oracle."""
+import numpy as np
+import torch
+
+import synth
+from oracle import formats, fp4, layer
+
+
+def test_e4m3_round_against_torch_below_saturation():
+    rng = np.random.default_rng(7)
+    pos = formats.E4M3_TABLE[:0x7F]
+    mids = (pos[1:] + pos[:-1]) / 2
+    v = np.concatenate([pos, mids, rng.random(20000) * 448.0, rng.random(20000) * 2.0 ** -5,
+                        np.nextafter(mids, 0.0), np.nextafter(mids, 1e9)])
+    v = v[v < 448.0].astype(np.float32)
+    ref = torch.tensor(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(formats.e4m3_round_vec(v.astype(np.float64)), ref)
+    assert all(formats.e4m3_round(float(x)) == r for x, r in zip(v[::97], ref[::97]))
+
+
+def test_e4m3_round_spec_values_and_saturation():
+    cases = {448.0: 0x7E, 464.0: 0x7E, 1e30: 0x7E, 2.0 ** -9: 0x01, 2.0 ** -10: 0x00,  # tie 0 | 2^-9 -> even
+             1.0: 0x38, 1.0625: 0x38, 1.1875: 0x3A, 2.0 ** -6: 0x08, 0.0: 0x00}    # ties to the even byte
+    for v, b in cases.items():
+        assert formats.e4m3_round(v) == b, v
+        assert formats.e4m3_round_vec(np.array([v]))[0] == b, v
+
+
+def test_quantiser_worked_block():
+    """amax = 2688 makes s = 2688 / 2688 = 1 exactly.
+    Block 0 holds 2688: block scale 2688 / 6 = 448 -> 0x7e; 2688 / 448 = 6 ->
+    code 7; 224 / 448 = 0.5 -> code 1; -672 / 448 = -1.5 -> code 8|3.
+    Block 1 has amax 12: 12 / 6 = 2 -> 0x40 (2.0); its values / 2:
+    12 -> 6 (7), 3 -> 1.5 (3), -1.5 -> -0.75, the tie 0.5 | 1.0 -> 1.0 (8|2),
+    5 -> 2.5, the tie 2 | 3 -> 2 (4), 7 -> 3.5, the tie 3 | 4 -> 4 (6),
+    0.4 -> 0.2 -> 0 (0), -0.6 -> -0.3 -> -0.5 (8|1), -0.0 -> -0 (8).
+    Block 2 is zero: scale 0, codes 0.  Block 3 has amax 1e-6: 1e-6 / 6 is
+    below half of E4M3's smallest value 2^-9, so its scale is 0 and its
+    codes are +0."""
+    x = np.zeros((1, 64), np.float32)
+    x[0, 0:3] = [2688.0, 224.0, -672.0]
+    x[0, 16:25] = [12.0, 3.0, -1.5, 5.0, 7.0, 0.4, -0.6, -0.0, 1.0]
+    x[0, 48] = 1e-6
+    x[0, 49] = -1e-6
+    codes, scales, s = formats.nvfp4_quantize_rows(x)
+    assert s == np.float32(1.0)
+    assert list(scales[0]) == [0x7E, 0x40, 0x00, 0x00]
+    assert list(codes[0, 0:3]) == [7, 1, 8 | 3] and not codes[0, 3:16].any()
+    assert list(codes[0, 16:25]) == [7, 3, 8 | 2, 4, 6, 0, 8 | 1, 8, 1]  # 1 / 2 = 0.5 -> code 1
+    assert not codes[0, 25:].any()
+    deq = formats.nvfp4_dequant_rows(codes, scales, s)
+    assert list(deq[0, 16:24]) == [12.0, 3.0, -2.0, 4.0, 8.0, 0.0, -1.0, 0.0]
+
+
+def test_quantiser_zero_tensor_and_scale_of_the_largest_block():
+    c, b, s = formats.nvfp4_quantize_rows(np.zeros((3, 32), np.float32))
+    assert s == 0 and not c.any() and not b.any()
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((8, 128)) * 3).astype(np.float32)
+    c, b, s = formats.nvfp4_quantize_rows(x)
+    # the block holding the tensor's largest magnitude takes (close to) 448
+    r, k = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert formats.E4M3_TABLE[b[r, k // 16]] == 448.0
+    assert formats.E4M3_TABLE[b].max() == 448.0
+
+
+def test_quantiser_error_bound():
+    """Every value dequantises to within half a grid step of its scaled
+    value, unless it is beyond 6 scaled units (the block scale rounded
+    down), where it saturates to 6."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((16, 256)) * np.exp(rng.standard_normal((16, 1)) * 3)).astype(np.float32)
+    c, b, s = formats.nvfp4_quantize_rows(x)
+    deq = formats.nvfp4_dequant_rows(c, b, s)
+    dq = np.repeat(formats.E4M3_TABLE[b] * float(s), 16, axis=1)
+    q = np.abs(x.astype(np.float64)) / np.where(dq > 0, dq, 1.0)
+    grid = np.array(fp4.E2M1_TABLE[:8])
+    half_step = np.where(q < 2, 0.25, np.where(q < 4, 0.5, 1.0))
+    err = np.abs(deq - x) / np.where(dq > 0, dq, 1.0)
+    inside = q <= 6.0
+    assert (err[inside] <= half_step[inside] * (1 + 1e-6)).all()
+    assert np.allclose(np.abs(deq[~inside]), 6.0 * dq[~inside])
+    assert set(np.unique(np.abs(deq / np.where(dq > 0, dq, 1.0)))) <= set(grid)
+
+
+def test_nvfp4_layer_within_quantisation_error_of_the_exact_layer():
+    H, I, E, K, T, seed = 256, 128, 8, 2, 24, 77
+    blobs = {e: synth.expert_blob_nvfp4(seed, 0, e, H, I) for e in range(E + 1)}
+    xb = synth.activations_bf16(seed, 1, T, H)
+    lg = synth.logits_for_sets(seed, 2, synth.near_uniform_sets(seed, 0, T, E, K), E)
+    kw = dict(logits=lg, weights="nvfp4", shared_blob=blobs[E])
+    exact = layer.moe_layer(xb, blobs.__getitem__, H, I, E, K, **kw)["out_f64"]
+    q = layer.moe_layer(xb, blobs.__getitem__, H, I, E, K, nvfp4=True, **kw)["out_f64"]
+    rel = np.linalg.norm(q - exact) / np.linalg.norm(exact)
+    # two 4-bit roundings (x, h): 17 % here; MXFP4 activations on the same
+    # layer (MXFP4 blobs of the same seed) lose 21 %.  A transposed operand or
+    # a wrong scale lands near 100 %.
+    assert 0.05 < rel < 0.3, rel
+
+
+def test_nvfp4_layer_scale_spans_the_whole_batch():
+    """x's per-tensor scale comes from every token: making the last token the
+    largest (x 64) changes the quantisation, hence the output, of the others;
+    the exact layer's outputs of the others do not change."""
+    H, I, E, K, T, seed = 256, 128, 8, 2, 12, 78
+    blobs = {e: synth.expert_blob_nvfp4(seed, 0, e, H, I) for e in range(E)}
+    xb = synth.activations_bf16(seed, 1, T, H)
+    big = xb.copy()
+    big[-1] = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(xb[-1]) * 64.0)
+    lg = synth.logits_for_sets(seed, 2, synth.near_uniform_sets(seed, 0, T, E, K), E)
+    kw = dict(logits=lg, weights="nvfp4")
+    a = layer.moe_layer(xb, blobs.__getitem__, H, I, E, K, nvfp4=True, **kw)["out_f64"]
+    b = layer.moe_layer(big, blobs.__getitem__, H, I, E, K, nvfp4=True, **kw)["out_f64"]
+    assert not np.allclose(a[:-1], b[:-1], rtol=0, atol=0)
+    ea = layer.moe_layer(xb, blobs.__getitem__, H, I, E, K, **kw)["out_f64"]
+    eb = layer.moe_layer(big, blobs.__getitem__, H, I, E, K, **kw)["out_f64"]
+    assert np.array_equal(ea[:-1], eb[:-1])
