@@ -166,12 +166,12 @@ def replica_throughput(units_per_rank_step, steps, ms_max, world):
 # ---------------------------------------------------------------------------
 H, I, E, K_TOP, S_SHARED, L = 2048, 512, 256, 8, 1, 40
 TRACE_LEN = 512
-# DRAM bytes (read + write) of k_dec_stack per algorithmic byte, from an ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum) of a 4-layer launch of
-# this workload: 60,254,976 B read + 1,071,616 B written against 60,162,048 B.
-# The full 40-layer launch is too large to capture; its traffic grows with the
-# layers.
-STACK_TRAFFIC_PER_BYTE = (60254976 + 1071616) / 60162048
+# DRAM bytes (read + write) of the dataflow kernel k_dec_flow per algorithmic
+# byte, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# 4-layer launch of this workload: 60,285,440 B read + 1,479,168 B written
+# against 60,162,048 B.  The full 40-layer launch is too large to capture; its
+# traffic grows with the layers.
+STACK_TRAFFIC_PER_BYTE = (60285440 + 1479168) / 60162048
 
 
 # The arithmetic of the decode GEMVs: MXFP4 and NVFP4 weights decode exactly
