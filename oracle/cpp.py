@@ -32,6 +32,7 @@ def lib() -> C.CDLL:
             "fto_weight_matrix": (None, [P, C.c_int, C.c_int, C.c_int, C.c_int, P]),
             "fto_quantize_rows": (None, [P, C.c_int64, C.c_int, P, P]),
             "fto_round_bf16": (None, [P, C.c_int64, P]),
+            "fto_nvfp4_quantize_rows": (C.c_float, [P, C.c_int64, C.c_int, C.c_float, P, P]),
             "fto_router_logits": (None, [P, P, C.c_int, C.c_int, C.c_int, P]),
             "fto_topk": (C.c_int, [P, C.c_int, C.c_int, C.c_int, P]),
             "fto_softmax_weights": (None, [P, P, C.c_int, C.c_int, C.c_int, C.c_int, P]),
@@ -120,6 +121,17 @@ def quantize_rows(v: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     return codes, scales
 
 
+def nvfp4_quantize_rows(v: np.ndarray, s=None) -> tuple[np.ndarray, np.ndarray, np.float32]:
+    """As ``oracle.formats.nvfp4_quantize_rows``: codes [R, K], E4M3 scale
+    bytes [R, K/16] and the per-tensor scale."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    R, K = v.shape
+    codes = np.empty((R, K), np.uint8)
+    scales = np.empty((R, K // 16), np.uint8)
+    st = lib().fto_nvfp4_quantize_rows(_p(v), R, K, -1.0 if s is None else float(s), _p(codes), _p(scales))
+    return codes, scales, np.float32(st)
+
+
 def round_bf16(v: np.ndarray) -> np.ndarray:
     v = np.ascontiguousarray(v, dtype=np.float64)
     out = np.empty(v.shape, np.uint16)
@@ -176,7 +188,7 @@ def expert_ffn(blob, hidden, inter, x, mxfp4=False, weights="mxfp4") -> np.ndarr
 
 
 def moe_layer(x_bits, blob_of, hidden, inter, n_experts, top_k, logits=None, router_w=None, renorm=True,
-              mxfp4=False, shared_blob=None, weights="mxfp4", threads=1) -> dict:
+              mxfp4=False, shared_blob=None, weights="mxfp4", threads=1, nvfp4=False) -> dict:
     """One MoE layer on T tokens, as ``oracle.layer.moe_layer`` (blob_of is
     called for the selected experts only).  Returns dict with ids, w, out_f64,
     out_bits and nonfinite."""
@@ -198,7 +210,8 @@ def moe_layer(x_bits, blob_of, hidden, inter, n_experts, top_k, logits=None, rou
     ids = np.empty((T, k), np.int32)
     w = np.empty((T, k))
     bad = lib().fto_moe_layer(_p(x), T, H, inter, E, k, ptrs, _p(sb), _p(lg), None, 1 if renorm else 0,
-                              1 if mxfp4 else 0, FORMATS[weights], threads, _p(out), _p(bits), _p(ids), _p(w))
+                              2 if nvfp4 else (1 if mxfp4 else 0), FORMATS[weights], threads, _p(out), _p(bits),
+                              _p(ids), _p(w))
     return dict(ids=ids, w=w, out_f64=out, out_bits=bits, nonfinite=bool(bad), logits=lg)
 
 

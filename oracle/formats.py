@@ -168,11 +168,19 @@ def weight_matrix(blob: np.ndarray, which: str, hidden: int, inter: int, weights
 # per-tensor fp32 scale s = amax / (448 * 6) over the whole matrix the GEMM
 # reads (all tokens of x; all h rows of the layer), so that the block scale of
 # the largest block lands on E4M3's largest value; per 16 values a block scale
-# E4M3(amax_block / (6 s)); codes e2m1(v / (block scale * s)).  Each of those
-# steps is a rounding that decides a byte, so it is taken in fp32, as the
-# kernel takes it: one fp32 multiply or divide per step, rounded to nearest
-# even.  A block whose scale is zero (or whose block scale times s underflows
-# to zero) has all codes +0.  Dequantised value: code x block scale x s.
+# E4M3(amax_block / (6 s)); codes e2m1(v / (block scale * s)).  The two
+# divisions are taken as multiplications by rounded reciprocals, one per
+# tensor and one per block.  Each step is a rounding that decides a byte, so
+# it is taken in fp32, as the kernel takes it, every operation rounded to
+# nearest even:
+#   s  = amax / 2688                   g = 1 / (s * 6)
+#   b  = amax_block * g                e = E4M3(b), ties to even, at most 448
+#   dq = E4M3 value of e * s           r = 1 / dq
+#   code = e2m1(v * r), ties to even, saturating at 6, sign kept
+# A tensor whose largest magnitude is below 2^-100 quantises to zero (s = 0,
+# every byte 0), which keeps g, r and the products finite; a block with
+# dq == 0 has all codes +0.
+# Dequantised value: code x block scale x s.
 
 NVFP4_GLOBAL_DIV = np.float32(448.0 * 6.0)
 _E4M3_POS = E4M3_TABLE[:0x7F]          # bytes 0x00 .. 0x7e: 0 .. 448, ascending
@@ -204,10 +212,15 @@ def e4m3_round_vec(v: np.ndarray) -> np.ndarray:
     return np.where(v >= 448.0, 0x7E, pick).astype(np.uint8)
 
 
+NVFP4_MIN_AMAX = 2.0 ** -100
+
+
 def nvfp4_global_scale(amax) -> np.float32:
-    """Per-tensor scale: fp32(amax) / 2688, one fp32 division."""
-    with np.errstate(all="ignore"):
-        return np.float32(np.float32(amax) / NVFP4_GLOBAL_DIV)
+    """Per-tensor scale: fp32(amax) / 2688, one fp32 division; 0 below 2^-100."""
+    a = np.float32(amax)
+    if not a >= NVFP4_MIN_AMAX:
+        return np.float32(0.0)
+    return np.float32(a / NVFP4_GLOBAL_DIV)
 
 
 def nvfp4_quantize_rows(v: np.ndarray, s=None) -> tuple[np.ndarray, np.ndarray, np.float32]:
@@ -223,11 +236,12 @@ def nvfp4_quantize_rows(v: np.ndarray, s=None) -> tuple[np.ndarray, np.ndarray, 
     if s == 0:
         return np.zeros((R, K), np.uint8), np.zeros((R, K // 16), np.uint8), s
     with np.errstate(all="ignore"):
-        t = np.float32(s * np.float32(6.0))
-        b = (np.abs(blocks).max(axis=-1) / t).astype(np.float32)
+        g = np.float32(np.float32(1.0) / np.float32(s * np.float32(6.0)))
+        b = (np.abs(blocks).max(axis=-1) * g).astype(np.float32)
         e = e4m3_round_vec(b)
         dq = (E4M3_TABLE[e].astype(np.float32) * s).astype(np.float32)
-        q = (blocks / np.where(dq > 0, dq, np.float32(1.0))[..., None]).astype(np.float32)
+        r = (np.float32(1.0) / np.where(dq > 0, dq, np.float32(1.0))).astype(np.float32)
+        q = (blocks * r[..., None]).astype(np.float32)
     mag = fp4.round_to_grid_vec(np.abs(q).astype(np.float64))
     codes = mag | np.where(np.signbit(q), 8, 0)
     codes = np.where((dq > 0)[..., None], codes, 0).astype(np.uint8).reshape(R, K)

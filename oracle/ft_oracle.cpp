@@ -203,6 +203,69 @@ void mx_roundtrip(double* v, int K) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 activations (the prefill path of NVFP4 experts).  The pages leave
+// activation scaling open; the reading is the two-level one: a per-tensor
+// scale s = amax / 2688 over the matrix a GEMM reads (all tokens of x; every
+// h row of the layer), E4M3 block scales per 16 values, e2m1 codes.  Each
+// step decides a byte, so each is one fp32 operation rounded to nearest even:
+//   s = amax / 2688 (0 when amax < 2^-100: every byte 0), g = 1 / (s * 6);
+//   per block e = E4M3(amax_block * g) (nearest, ties to the even byte, at
+//   most 448), dq = value(e) * s, r = 1 / dq, code = e2m1(v * r) (dq == 0:
+//   codes 0).  Dequantised value: code x value(e) x s.
+// ---------------------------------------------------------------------------
+int e4m3_round(float v) {
+  if (v >= 448.0f) return 0x7E;
+  int best = 0;
+  double bd = std::fabs((double)v - e4m3(0));
+  for (int b = 1; b < 0x7F; b++) {
+    const double d = std::fabs((double)v - e4m3(b));
+    if (d < bd || (d == bd && (b & 1) == 0 && (best & 1) != 0)) {
+      bd = d;
+      best = b;
+    }
+  }
+  return best;
+}
+
+struct NvScale {
+  float s, g;
+};
+
+NvScale nv_tensor_scale(float amax) {
+  NvScale t{0.0f, 0.0f};
+  if (amax >= 0x1p-100f) {
+    t.s = amax / 2688.0f;
+    t.g = 1.0f / (t.s * 6.0f);
+  }
+  return t;
+}
+
+// One row of K values (exact in fp32): codes [K] and scale bytes [K/16] (each
+// optional) and the dequantised row in fp64.
+void nv_quantize_row(const float* v, int K, NvScale t, uint8_t* codes, uint8_t* scales, double* deq) {
+  for (int b = 0; b < K; b += 16) {
+    int e = 0;
+    if (t.s != 0.0f) {
+      float amax = 0.0f;
+      for (int i = 0; i < 16; i++) amax = std::max(amax, std::fabs(v[b + i]));
+      e = e4m3_round(amax * t.g);
+    }
+    const float dq = (float)e4m3(e) * t.s;
+    const float r = dq > 0.0f ? 1.0f / dq : 0.0f;
+    for (int i = 0; i < 16; i++) {
+      int code = 0;
+      if (dq > 0.0f) {
+        const float q = v[b + i] * r;
+        code = round_to_grid(std::fabs((double)q)) | (std::signbit(q) ? 8 : 0);
+      }
+      if (codes) codes[b + i] = (uint8_t)code;
+      if (deq) deq[b + i] = e2m1(code) * e4m3(e) * (double)t.s;
+    }
+    if (scales) scales[b / 16] = (uint8_t)e;
+  }
+}
+
 // fp64 -> bf16 bits, nearest with ties to even, directly (no fp32 step).
 uint16_t round_bf16(double x) {
   if (std::isnan(x)) return 0x7FC0;
@@ -413,6 +476,22 @@ FTO_API void fto_quantize_rows(const double* x, int64_t R, int K, uint8_t* codes
     }
 }
 
+// NVFP4 rows: x [R][K] (values exact in fp32) -> codes [R][K] (one code per
+// element), scale bytes [R][K/16]; returns the per-tensor scale (from the
+// largest |x| when s_in < 0, else s_in).
+FTO_API float fto_nvfp4_quantize_rows(const double* x, int64_t R, int K, float s_in, uint8_t* codes, uint8_t* scales) {
+  std::vector<float> v((size_t)R * K);
+  float amax = 0.0f;
+  for (size_t i = 0; i < v.size(); i++) {
+    v[i] = (float)x[i];
+    amax = std::max(amax, std::fabs(v[i]));
+  }
+  NvScale t = nv_tensor_scale(amax);
+  if (s_in >= 0.0f) t = s_in > 0.0f ? NvScale{s_in, 1.0f / (s_in * 6.0f)} : NvScale{0.0f, 0.0f};
+  for (int64_t r = 0; r < R; r++) nv_quantize_row(v.data() + r * K, K, t, codes + r * K, scales + r * (K / 16), nullptr);
+  return t.s;
+}
+
 FTO_API void fto_round_bf16(const double* v, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = round_bf16(v[i]);
 }
@@ -442,6 +521,9 @@ FTO_API void fto_expert_ffn(const uint8_t* blob, int H, int I, const double* x, 
 //   a blob; logits [T][E] or NULL (then router_w [E][H] and router_logits).
 //   Experts run in parallel on `threads` OpenMP threads (1 = serial; the sum
 //   order of the combine does not depend on it).  ids / w outputs may be NULL.
+//   mxfp4 selects the activations: 0 as given (decode), 1 MXFP4 per row, 2
+//   NVFP4 with the per-tensor scales of x (all T tokens) and of h (every h
+//   row of the layer, so all units' h come before any down projection).
 // Returns 1 if the routing saw a NaN / +inf logit (as topk), else 0.
 FTO_API int fto_moe_layer(const uint16_t* x_bits, int T, int H, int I, int E, int k, const uint8_t* const* blobs,
                           const uint8_t* shared, const float* logits, const float* router_w, int renorm, int mxfp4,
@@ -473,16 +555,71 @@ FTO_API int fto_moe_layer(const uint16_t* x_bits, int T, int H, int I, int E, in
     for (int t = 0; t < T; t++) toks[n_routed].push_back(t);
   std::vector<std::vector<double>> y(units.size());
   const int nu = (int)units.size();
+  if (mxfp4 == 2) {
+    // NVFP4 activations: x with its per-tensor scale over the T tokens; then
+    // every unit's h before h's per-tensor scale (over all of them)
+    float ax = 0.0f;
+    for (double v : x) ax = std::max(ax, (float)std::fabs(v));
+    const NvScale sx = nv_tensor_scale(ax);
+    std::vector<float> xf(x.begin(), x.end());
+    for (int t = 0; t < T; t++) nv_quantize_row(xf.data() + (size_t)t * H, H, sx, nullptr, nullptr, x.data() + (size_t)t * H);
+    std::vector<std::vector<double>> h(units.size());
 #ifdef _OPENMP
 #pragma omp parallel for schedule(dynamic, 1) num_threads(std::max(threads, 1))
 #endif
-  for (int u = 0; u < nu; u++) {
-    const int m = (int)toks[u].size();
-    std::vector<double> xu((size_t)m * H);
-    for (int i = 0; i < m; i++) std::copy(x.begin() + (size_t)toks[u][i] * H, x.begin() + (size_t)(toks[u][i] + 1) * H,
-                                          xu.begin() + (size_t)i * H);
-    y[u].assign((size_t)m * H, 0.0);
-    expert_ffn(units[u] < 0 ? shared : blobs[units[u]], H, I, xu.data(), m, mxfp4, fmt, y[u].data());
+    for (int u = 0; u < nu; u++) {
+      const uint8_t* blob = units[u] < 0 ? shared : blobs[units[u]];
+      const std::vector<double> wg = weight_matrix(blob, H, I, 0, fmt), wu = weight_matrix(blob, H, I, 1, fmt);
+      const int m = (int)toks[u].size();
+      h[u].assign((size_t)m * I, 0.0);
+      for (int i = 0; i < m; i++) {
+        const double* xs = x.data() + (size_t)toks[u][i] * H;
+        for (int r = 0; r < I; r++) {
+          double g = 0.0, uu = 0.0;
+          for (int kk = 0; kk < H; kk++) {
+            g += wg[(size_t)r * H + kk] * xs[kk];
+            uu += wu[(size_t)r * H + kk] * xs[kk];
+          }
+          h[u][(size_t)i * I + r] = silu(g) * uu;
+        }
+      }
+    }
+    double ah = 0.0;
+    for (const auto& hu : h)
+      for (double v : hu) ah = std::max(ah, std::fabs(v));
+    const NvScale sh = nv_tensor_scale((float)ah);
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(std::max(threads, 1))
+#endif
+    for (int u = 0; u < nu; u++) {
+      const uint8_t* blob = units[u] < 0 ? shared : blobs[units[u]];
+      const std::vector<double> wd = weight_matrix(blob, H, I, 2, fmt);
+      const int m = (int)toks[u].size();
+      y[u].assign((size_t)m * H, 0.0);
+      std::vector<float> hf(I);
+      std::vector<double> hq(I);
+      for (int i = 0; i < m; i++) {
+        for (int r = 0; r < I; r++) hf[r] = (float)h[u][(size_t)i * I + r];
+        nv_quantize_row(hf.data(), I, sh, nullptr, nullptr, hq.data());
+        for (int n = 0; n < H; n++) {
+          double acc = 0.0;
+          for (int r = 0; r < I; r++) acc += wd[(size_t)n * I + r] * hq[r];
+          y[u][(size_t)i * H + n] = acc;
+        }
+      }
+    }
+  } else {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(std::max(threads, 1))
+#endif
+    for (int u = 0; u < nu; u++) {
+      const int m = (int)toks[u].size();
+      std::vector<double> xu((size_t)m * H);
+      for (int i = 0; i < m; i++) std::copy(x.begin() + (size_t)toks[u][i] * H, x.begin() + (size_t)(toks[u][i] + 1) * H,
+                                            xu.begin() + (size_t)i * H);
+      y[u].assign((size_t)m * H, 0.0);
+      expert_ffn(units[u] < 0 ? shared : blobs[units[u]], H, I, xu.data(), m, mxfp4, fmt, y[u].data());
+    }
   }
   auto y_of = [&](int u, int t) -> const double* {
     const auto& tv = toks[u];

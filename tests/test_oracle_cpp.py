@@ -128,6 +128,37 @@ def test_quantiser_equals_the_numpy_oracle():
     assert (a[0] == b[0]).all() and (a[1] == b[1]).all()
 
 
+def test_nvfp4_quantiser_equals_the_numpy_oracle():
+    """The two-level NVFP4 activation quantiser, bit for bit: codes, E4M3
+    scale bytes and the per-tensor scale, on rows spanning 10^+-7, zero,
+    negative-zero and underflowing blocks, the hand-worked block of the numpy
+    oracle's pin, a given scale, and a tensor below 2^-100."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((48, 256)) * np.exp(rng.uniform(-16, 16, (48, 1)))).astype(np.float32)
+    x[0, :16] = 0.0
+    x[0, 16:32] = -0.0
+    x[1, :16] *= np.float32(1e-12)
+    worked = np.zeros((1, 64), np.float32)
+    worked[0, 0:3] = [2688.0, 224.0, -672.0]
+    worked[0, 16:25] = [12.0, 3.0, -1.5, 5.0, 7.0, 0.4, -0.6, -0.0, 1.0]
+    for v, s in ((x, None), (worked, None), (x, np.float32(0.125)), (np.full((2, 32), 1e-31, np.float32), None)):
+        a = cpp.nvfp4_quantize_rows(v, s)
+        b = formats.nvfp4_quantize_rows(v, s)
+        assert (a[0] == b[0]).all() and (a[1] == b[1]).all() and a[2] == b[2]
+
+
+def test_nvfp4_layer_equals_the_numpy_oracle():
+    H, I, E, k, T, seed = 256, 128, 16, 4, 12, 1102
+    blobs = {e: synth.expert_blob_nvfp4(seed, 0, e, H, I) for e in range(E + 1)}
+    xb = synth.activations_bf16(seed, 0, T, H)
+    wr = synth.router_weights(seed, 0, E, H)
+    kw = dict(router_w=wr, shared_blob=blobs[E], weights="nvfp4", nvfp4=True)
+    a = cpp.moe_layer(xb, blobs.__getitem__, H, I, E, k, threads=4, **kw)
+    b = layer.moe_layer(xb, blobs.__getitem__, H, I, E, k, **kw)
+    assert (a["ids"] == b["ids"]).all()
+    assert np.allclose(a["out_f64"], b["out_f64"], rtol=1e-12, atol=1e-15)
+
+
 def test_round_bf16_equals_the_numpy_oracle():
     rng = np.random.default_rng(3)
     v = np.concatenate([rng.standard_normal(20000) * np.exp(rng.uniform(-90, 90, 20000)),
