@@ -40,10 +40,11 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 or 4)")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
-    ap.add_argument("--case", default="decode", choices=["decode", "prefill", "miss", "glm", "gemm", "router"],
+    ap.add_argument("--case", default="decode",
+                    choices=["decode", "prefill", "miss", "glm", "gemm", "router", "nvfp4"],
                     help="decode: the 35B-class decode stack (default line); prefill / miss / glm: only that "
-                         "measurement; gemm / router: the prefill GEMMs or router GEMV alone on a small case "
-                         "(the ncu captures' workloads)")
+                         "measurement; nvfp4: the NVFP4 prefill layer alone; gemm / router: the prefill GEMMs or "
+                         "router GEMV alone on a small case (the ncu captures' workloads)")
     ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     ap.add_argument("--layerwise", action="store_true",
                     help="decode with two kernels per layer instead of a persistent stack kernel")
@@ -546,6 +547,7 @@ def measure_prefill(reps=3, layers=3):
                             "fp4_peak_tflops": fp4["tflops"], "fp4_peak_source": "measured (tcgen05 mxf4 probe)",
                             "fp4_nominal_tflops": FP4_DENSE_TFLOPS_NOMINAL}
     res["calibration"] = measure_prefill_calibration(fp4["tflops"])
+    res["nvfp4"] = measure_prefill_nvfp4(fp4["tflops"], pk)
     # (b) pinned host pools, double-buffered prefetch
     hp = host_layer_pools(H2, I2, E2, seed, layers)
     ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, layers, 0, 0, T2), hp, None)
@@ -602,6 +604,57 @@ def available_host_bytes():
         return psutil.virtual_memory().available
     except Exception:
         return os.sysconf("SC_AVPHYS_PAGES") * os.sysconf("SC_PAGE_SIZE")
+
+
+def measure_prefill_nvfp4(fp4_peak, pk, reps=3):
+    """The DSV4-class prefill layer with NVFP4 experts (E4M3 scales per 16,
+    fp32 matrix scales) through FT_ACT_NVFP4: x and h quantised to NVFP4,
+    tcgen05 kind::mxf4nvf4 grouped GEMMs; 4096 tokens through the router
+    GEMV.  GEMM TFLOP/s from the kernel timers against the layer's roofline
+    (its NVFP4 weight bytes at the HBM rate; the tensor peak is the measured
+    kind::mxf4 one, the same nominal rate)."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+    H2, I2, E2, k2, T2, seed = 4096, 2048, 256, 6, 4096, 1006
+    flops = 2.0 * T2 * k2 * 3 * H2 * I2
+    pool = synth.gpu.layer_pool(H2, I2, E2, seed, 0, fmt="nvfp4")
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, 1, 0, 0, T2, weight_format=ft.FT_FMT_NVFP4), None, [pool])
+    x = torch.from_numpy(synth.activations_bf16(seed, 1, T2, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    wr = torch.from_numpy(synth.router_weights(seed, 0, E2, H2)).cuda()
+    out = torch.empty_like(x)
+    flags = ft.FT_ACT_NVFP4 | ft.FT_ROUTE_RENORM
+    for _ in range(2):
+        ft.ft_moe_layer_forward(ctx, 0, x, T2, wr, None, out, flags)
+    torch.cuda.synchronize()
+    ft.ft_kernel_timing_enable(ctx, True)
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, x, T2, wr, None, out, flags)
+    kt = ft.ft_kernel_timing_read(ctx)
+    ft.ft_kernel_timing_enable(ctx, False)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        ft.ft_moe_layer_forward(ctx, 0, x, T2, wr, None, out, flags)
+    b.record()
+    b.synchronize()
+    ft.ft_sync_status(ctx)
+    ft.ft_destroy(ctx)
+    del pool
+    torch.cuda.empty_cache()
+    gemm_ms = (kt["gemm_gate_up"][0] + kt["gemm_down"][0]) / reps
+    tflops = flops / (gemm_ms * 1e-3) / 1e12
+    wbytes = E2 * ft.ft_blob_layout_format(H2, I2, ft.FT_FMT_NVFP4)["used"]
+    return {"workload": "DSV4-class prefill layer with NVFP4 experts: hidden 4096, 256 experts top-6, "
+                        "intermediate 2048, 4096 tokens",
+            "gemm_ms": gemm_ms, "gemm_tflops": tflops, "gate_up_ms": kt["gemm_gate_up"][0] / reps,
+            "down_ms": kt["gemm_down"][0] / reps, "layer_ms_resident": a.elapsed_time(b) / reps,
+            "kernels_ms": {k: v[0] / reps for k, v in kt.items() if v[1]},
+            "gemm_weight_gbs": wbytes / (gemm_ms * 1e-3) / 1e9,
+            "gemm_roofline": {**prefill_roofline(flops, wbytes, pk["hbm"], tflops, fp4_peak),
+                              "hbm_peak_gbs": pk["hbm"], "hbm_peak_source": pk["src"]}}
 
 
 def measure_prefill_calibration(fp4_peak, T=65536, reps=2):
@@ -959,7 +1012,8 @@ def main():
         if rank == 0:
             r = {"prefill": lambda: measure_prefill(reps=max(args.steps, 1)), "miss": measure_misses,
                  "glm": measure_glm, "gemm": lambda: measure_gemm_small(reps=max(args.steps, 1)),
-                 "router": lambda: measure_router(reps=max(args.steps, 1))}[args.case]()
+                 "router": lambda: measure_router(reps=max(args.steps, 1)),
+                 "nvfp4": lambda: measure_prefill_nvfp4(measure_fp4_peak()["tflops"], peaks())}[args.case]()
             print(json.dumps({"case": args.case, **r}))
         return
     if args.impl == "reference":

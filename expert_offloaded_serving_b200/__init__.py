@@ -25,10 +25,11 @@ FT_ACT_MXFP4 = 2
 FT_STACK_LAYERWISE = 4
 FT_STACK_COUNTERS = 8
 FT_CACHE_SERIAL = 16
+FT_ACT_NVFP4 = 32
 FT_EV_HIT, FT_EV_MISS, FT_EV_EVICT, FT_EV_MOVE, FT_EV_PREFETCH = range(5)
 
 EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft_destroy", "ft_sync_status",
-           "ft_router_logits", "ft_moe_route", "ft_moe_permute", "ft_quantize_mxfp4", "ft_moe_layer_forward",
+           "ft_router_logits", "ft_moe_route", "ft_moe_permute", "ft_quantize_mxfp4", "ft_quantize_nvfp4", "ft_moe_layer_forward",
            "ft_expert_cache_lookup", "ft_expert_cache_insert", "ft_expert_cache_resize", "ft_cache_trace",
            "ft_cache_stats_get", "ft_prefetch_layer", "ft_debug_dequant", "ft_kernel_timing_enable",
            "ft_kernel_timing_read", "ft_moe_layer_forward_noalloc", "ft_moe_stack_forward", "ft_last_routing",
@@ -37,7 +38,7 @@ EXPORTS = ("ft_blob_stride", "ft_blob_layout", "ft_last_error", "ft_create", "ft
            "ft_cache_prefetch", "ft_debug_stack_timeline")
 FT_NOALLOC_SCRATCH_BYTES = 8 << 20
 KERNELS = ("router_logits", "topk", "permute", "gate_up", "down_combine", "quant_x", "gemm_gate_up", "gemm_down",
-           "combine", "dec_stack")
+           "combine", "dec_stack", "quant_h")
 
 
 class FtError(RuntimeError):
@@ -93,6 +94,7 @@ def lib() -> C.CDLL:
         "ft_moe_route": (ST, [P, P, I64, I32, I32, U32, P, P, P]),
         "ft_moe_permute": (ST, [P, P, I64, I32, I32, P, P, P, P]),
         "ft_quantize_mxfp4": (ST, [P, P, I64, I32, P, P, P]),
+        "ft_quantize_nvfp4": (ST, [P, P, I64, I32, P, P, P, P]),
         "ft_moe_layer_forward": (ST, [P, I32, P, I64, P, P, P, U32, P]),
         "ft_expert_cache_lookup": (ST, [P, I32, I32, C.POINTER(I32)]),
         "ft_expert_cache_insert": (ST, [P, I32, I32, C.POINTER(I32), C.POINTER(I64), P]),
@@ -243,6 +245,11 @@ def ft_moe_permute(ctx, ids, T, k, E, offs, perm, inv, stream=None) -> None:
 
 def ft_quantize_mxfp4(ctx, x, R, K, codes, scales, stream=None) -> None:
     _check(lib().ft_quantize_mxfp4(ctx, _ptr(x, 4), R, K, _ptr(codes, 1), _ptr(scales, 1), _stream(stream)))
+
+
+def ft_quantize_nvfp4(ctx, x, R, K, codes, scales, tensor_scale, stream=None) -> None:
+    _check(lib().ft_quantize_nvfp4(ctx, _ptr(x, 4), R, K, _ptr(codes, 1), _ptr(scales, 1), _ptr(tensor_scale, 4),
+                                   _stream(stream)))
 
 
 def ft_moe_layer_forward(ctx, layer, x, T, router_w, logits_override, out, flags, stream=None) -> None:

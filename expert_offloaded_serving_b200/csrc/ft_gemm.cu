@@ -51,7 +51,9 @@ constexpr int kEpiWarps = kWarps - kEpiWarp0;
 constexpr int kStagesGU = 4;     // gate/up: 2 weight tiles + 1 token tile per stage (51 KB)
 constexpr int kStagesDn = 6;     // down: 1 + 1 (34 KB)
 constexpr int kTileBytes = kGemmBM * kGemmBK / 2;   // 16 KB of e2m1 codes
-constexpr int kSfBytes = 1024;                      // two 512-byte scale atoms
+// Scale atoms (512 bytes: 128 rows x 4 blocks) per operand and stage of
+// kGemmBK elements: 2 for MXFP4 (blocks of 32), 4 for NVFP4 (blocks of 16).
+__host__ __device__ constexpr int atoms_per_stage(int fmt) { return fmt == kFmtNv ? 4 : 2; }
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 2 * kGemmBN;               // accumulator columns: gate + up, or two down buffers
 
@@ -98,13 +100,15 @@ __device__ __forceinline__ int segment_of(const GemmArgs& a, int row0) {
 // the kernel.  MODE 0: gate/up (two weight matrices, SwiGLU, MXFP4 h);
 // MODE 1: down (one weight matrix, fp32 y).
 // ---------------------------------------------------------------------------
-template <int MODE>
+template <int MODE, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ GemmArgs a,
                                                       const __grid_constant__ GemmMaps maps) {
   constexpr int S = MODE == 0 ? kStagesGU : kStagesDn;
   constexpr int NA = MODE == 0 ? 2 : 1;
   constexpr int NB = MODE == 0 ? 1 : 2;   // accumulator buffers
-  constexpr int SFC = 8 * (NA + 1);       // scale columns per stage
+  constexpr int APS = atoms_per_stage(FMT);
+  constexpr int kSfBytes = APS * 512;     // scale bytes per operand and stage
+  constexpr int SFC = 4 * APS * (NA + 1); // scale columns per stage (4 a tcgen05.cp atom)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tileA = smem;                              // [S][NA] 16 KB, 1024-aligned
@@ -125,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
   const int n_tiles = n_mt * n_jt;
   if ((int)blockIdx.x >= n_tiles) return;  // the whole CTA, before any barrier or allocation
   const int KT = a.K / kGemmBK;
-  const int atoms_k = a.K / 128;
+  const int atoms_k = a.K * APS / kGemmBK;  // scale atoms along K
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; s++) {
@@ -174,11 +178,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
 #pragma unroll
           for (int q = 0; q < NA; q++) {
             tma_3d(tileA + (s * NA + q) * kTileBytes, &maps.a[q], kt * (kGemmBK / 2), mt * kGemmBM, e, &full[s]);
-            bulk_g2s(sfA + (s * NA + q) * kSfBytes, blob + a.sfa_off[q] + ((int64_t)mt * atoms_k + 2 * kt) * 512,
+            bulk_g2s(sfA + (s * NA + q) * kSfBytes, blob + a.sfa_off[q] + ((int64_t)mt * atoms_k + APS * kt) * 512,
                      kSfBytes, &full[s]);
           }
           tma_2d(tileB + s * kTileBytes, &maps.b, kt * (kGemmBK / 2), row0, &full[s]);
-          bulk_g2s(sfB + s * kSfBytes, a.sfb + ((int64_t)jt * atoms_k + 2 * kt) * 512, kSfBytes, &full[s]);
+          bulk_g2s(sfB + s * kSfBytes, a.sfb + ((int64_t)jt * atoms_k + APS * kt) * 512, kSfBytes, &full[s]);
           issued++;
         }
         if (!ok) break;
@@ -217,21 +221,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
 #pragma unroll
           for (int q = 0; q < NA; q++)
 #pragma unroll
-            for (int at = 0; at < 2; at++)
-              utccp_32x128(sfs + q * 8 + 4 * at, desc_sf(sfA + (s * NA + q) * kSfBytes + at * 512));
+            for (int at = 0; at < APS; at++)
+              utccp_32x128(sfs + q * 4 * APS + 4 * at, desc_sf(sfA + (s * NA + q) * kSfBytes + at * 512));
 #pragma unroll
-          for (int at = 0; at < 2; at++) utccp_32x128(sfs + 8 * NA + 4 * at, desc_sf(sfB + s * kSfBytes + at * 512));
+          for (int at = 0; at < APS; at++)
+            utccp_32x128(sfs + 4 * APS * NA + 4 * at, desc_sf(sfB + s * kSfBytes + at * 512));
           const uint64_t bd = desc_sw128(tileB + s * kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 64; kk++) {
-            const uint32_t byte = 2u * (kk & 1), col = 4u * (kk >> 1);
-            const uint32_t idesc = idesc_mxf4(byte, byte, kGemmBM, kGemmBN);
+            // MXFP4: an atom covers two MMAs of K = 64, the scale id picks
+            // bytes 0-1 or 2-3 of each row's word; NVFP4: one atom an MMA
+            const uint32_t byte = FMT == kFmtNv ? 0u : 2u * (kk & 1);
+            const uint32_t col = FMT == kFmtNv ? 4u * kk : 4u * (kk >> 1);
 #pragma unroll
             for (int q = 0; q < NA; q++) {
               const uint64_t ad = desc_sw128(tileA + (s * NA + q) * kTileBytes) + (uint64_t)(kk * 2);  // +32 B of K
-              mma_mxf4(d0 + (uint32_t)(q * kGemmBN), ad, bd + (uint64_t)(kk * 2), idesc,
-                       (sfs + q * 8 + col) | (byte << 30), (sfs + 8 * NA + col) | (byte << 30),
-                       (kt | kk) != 0 ? 1u : 0u);
+              const uint32_t sa = (sfs + q * 4 * APS + col) | (byte << 30), sb = (sfs + 4 * APS * NA + col) | (byte << 30);
+              if (FMT == kFmtNv)
+                mma_nvf4(d0 + (uint32_t)(q * kGemmBN), ad, bd + (uint64_t)(kk * 2), idesc_nvf4(kGemmBM, kGemmBN), sa,
+                         sb, (kt | kk) != 0 ? 1u : 0u);
+              else
+                mma_mxf4(d0 + (uint32_t)(q * kGemmBN), ad, bd + (uint64_t)(kk * 2),
+                         idesc_mxf4(byte, byte, kGemmBM, kGemmBN), sa, sb, (kt | kk) != 0 ? 1u : 0u);
             }
           }
           umma_commit(&empty[s]);
@@ -275,6 +286,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
         if (lane == 0) mbar_arrive(&acc_empty[b]);
         const int I = a.M;
         const int irow = mt * kGemmBM + quad * 32 + lane;
+        if (FMT == kFmtNv) {
+          // NVFP4: g and u scaled by matrix scale x activation scale, h kept
+          // in fp32 for the quantiser that follows (which needs the largest
+          // |h| of the layer first); column q is padded row row0 + 32 cg + q
+          const int e = segment_of(a, row0);
+          const float* ts = reinterpret_cast<const float*>(a.pool + (int64_t)e * a.blob_stride + a.ts_off);
+          const float sx = nv_tensor_scale(*a.amax_in).s;
+          const float cgt = __fmul_rn(ts[0], sx), cut = __fmul_rn(ts[1], sx);
+          float* h_col = a.hf + (size_t)(row0 + 32 * cg) * I + irow;
+          uint32_t m = 0;
+#pragma unroll
+          for (int q = 0; q < 32; q++) {
+            const float g = __fmul_rn(__uint_as_float(q < 16 ? g0[q & 15] : g1[q & 15]), cgt);
+            const float u = __fmul_rn(__uint_as_float(q < 16 ? u0[q & 15] : u1[q & 15]), cut);
+            const float hv = silu(g) * u;
+            h_col[(size_t)q * I] = hv;
+            m = max(m, __float_as_uint(hv) & 0x7fffffffu);
+          }
+          amax_fold(m, a.amax_out);
+          continue;
+        }
         const int atoms_i = I / 128;
         // column q is padded row p = row0 + 32 cg + q: its codes at p * I/2 +
         // irow/2, the scale of its block 4 mt + quad at atom (jt, mt), byte
@@ -322,10 +354,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
         const int valid = shared ? a.T : a.offs[e + 1] - a.offs[e];
         const int base_pos = shared ? a.T * a.k + (e - a.E) * a.T : a.offs[e];
         const int r0 = row0 - a.pad_offs[e] + 32 * cg;
+        // NVFP4: the product of Wd's matrix scale and h's per-tensor scale
+        float f = 1.f;
+        if (FMT == kFmtNv)
+          f = __fmul_rn(reinterpret_cast<const float*>(a.pool + (int64_t)e * a.blob_stride + a.ts_off)[2],
+                        nv_tensor_scale(*a.amax_in).s);
 #pragma unroll
         for (int q = 0; q < 32; q++) {
           const int r = r0 + q;
-          if (r < valid) a.y[(size_t)(base_pos + r) * H + hrow] = __uint_as_float(q < 16 ? v0[q & 15] : v1[q & 15]);
+          const float v = __uint_as_float(q < 16 ? v0[q & 15] : v1[q & 15]);
+          if (r < valid) a.y[(size_t)(base_pos + r) * H + hrow] = FMT == kFmtNv ? __fmul_rn(v, f) : v;
         }
       }
     }
@@ -340,9 +378,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
 
 }  // namespace
 
-size_t gemm_smem_bytes(int mode) {
+size_t gemm_smem_bytes(int mode, int fmt) {
   const int S = mode == 0 ? kStagesGU : kStagesDn, NA = mode == 0 ? 2 : 1, NB = mode == 0 ? 1 : 2;
-  return 1024 + (size_t)S * (NA + 1) * (kTileBytes + kSfBytes) + (2 * S + 2 * NB + 1) * 8 + 16;
+  const int sf_bytes = atoms_per_stage(fmt) * 512;
+  return 1024 + (size_t)S * (NA + 1) * (kTileBytes + sf_bytes) + (2 * S + 2 * NB + 1) * 8 + 16;
+}
+
+template <int MODE, int FMT>
+static cudaError_t launch_one(const GemmArgs& a, const GemmMaps& maps, dim3 grid, cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes(MODE, FMT);
+  cudaError_t e = cudaFuncSetAttribute(k_gemm<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_gemm<MODE, FMT><<<grid, kThreads, smem, s>>>(a, maps);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, const GemmMaps& maps, cudaStream_t s) {
@@ -354,18 +402,9 @@ cudaError_t launch_gemm(const GemmArgs& a, const GemmMaps& maps, cudaStream_t s)
     return e;
   const int tiles = (a.M / kGemmBM) * a.n_tiles_max;
   const dim3 grid(tiles < nsm ? tiles : nsm);
-  if (a.mode == 0) {
-    if ((e = cudaFuncSetAttribute(k_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(0))) !=
-        cudaSuccess)
-      return e;
-    k_gemm<0><<<grid, kThreads, gemm_smem_bytes(0), s>>>(a, maps);
-  } else {
-    if ((e = cudaFuncSetAttribute(k_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(1))) !=
-        cudaSuccess)
-      return e;
-    k_gemm<1><<<grid, kThreads, gemm_smem_bytes(1), s>>>(a, maps);
-  }
-  return cudaGetLastError();
+  if (a.fmt == kFmtNv)
+    return a.mode == 0 ? launch_one<0, kFmtNv>(a, maps, grid, s) : launch_one<1, kFmtNv>(a, maps, grid, s);
+  return a.mode == 0 ? launch_one<0, kFmtMx>(a, maps, grid, s) : launch_one<1, kFmtMx>(a, maps, grid, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,4 +1,5 @@
-// Prefill grouped GEMM on tcgen05 block-scaled FP4 MMA (kind::mxf4).
+// Prefill grouped GEMM on tcgen05 block-scaled FP4 MMA (kind::mxf4 for MXFP4,
+// kind::mxf4nvf4 for NVFP4).
 #pragma once
 
 #include <cuda.h>
@@ -30,6 +31,15 @@ struct GemmArgs {
   const uint8_t* pool;       // blob 0 of the layer pool
   const uint8_t* sfb;        // activation scales, atoms over padded rows
   int mode;                  // 0: gate/up -> SwiGLU -> MXFP4 h;  1: down -> fp32 y
+  int fmt;                   // kFmtMx: UE8M0 per 32, kind::mxf4;  kFmtNv: E4M3 per 16, kind::mxf4nvf4
+  // NVFP4: each blob's fp32 matrix scales (Wg, Wu, Wd) at ts_off; the
+  // activation operand's per-tensor scale from its largest magnitude
+  // *amax_in; gate/up writes h in fp32 to hf ([rows][M]) and folds its
+  // largest magnitude into *amax_out instead of quantising h
+  int64_t ts_off;
+  const uint32_t* amax_in;
+  uint32_t* amax_out;
+  float* hf;
   // gate/up epilogue
   uint8_t* hq;               // [rows][M/2] codes
   uint8_t* hq_sf;            // atoms over [rows][M/32]
@@ -48,7 +58,7 @@ ft_status encode_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner_byte
                          uint64_t row_pitch, uint64_t depth_pitch);
 ft_status encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_pitch);
 
-size_t gemm_smem_bytes(int mode);
+size_t gemm_smem_bytes(int mode, int fmt);
 cudaError_t launch_gemm(const GemmArgs& a, const GemmMaps& maps, cudaStream_t s);
 
 }  // namespace ft

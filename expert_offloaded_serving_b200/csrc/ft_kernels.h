@@ -39,5 +39,12 @@ bool gemv_shape_ok(int H, int I);
 cudaError_t launch_gate_up(const GemvParams& p, cudaStream_t s);
 cudaError_t launch_down_combine(const GemvParams& p, cudaStream_t s);
 cudaError_t launch_quantize_rows(const float* x, int64_t R, int K, uint8_t* codes, uint8_t* scales, cudaStream_t s);
+// Largest |x| over n values (bf16 or fp32), folded into *amax (fp32 bits);
+// the caller zeroes *amax first.
+cudaError_t launch_amax(const void* x, int64_t n, bool bf16, uint32_t* amax, cudaStream_t s);
+// NVFP4 rows: zeroes *amax, takes the largest |x|, quantises; the per-tensor
+// scale goes to *scale_out (device) unless NULL.
+cudaError_t launch_quantize_rows_nv(const float* x, int64_t R, int K, uint32_t* amax, uint8_t* codes,
+                                    uint8_t* scales, float* scale_out, cudaStream_t s);
 
 }  // namespace ft

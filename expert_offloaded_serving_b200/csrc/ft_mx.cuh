@@ -44,4 +44,76 @@ __device__ __forceinline__ uint32_t mx_quant_block(const float4* v, uint4& q) {
   return (uint32_t)e;
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 (two-level) quantisation: a per-tensor fp32 scale s = amax / 2688 and
+// g = 1 / (6 s); per 16 values an E4M3 block scale e = E4M3(amax_block * g)
+// (nearest even, saturating at 448), dq = value(e) * s, r = 1 / dq and codes
+// e2m1(v * r).  Every step is one fp32 operation rounded to nearest even.  A
+// tensor whose largest magnitude is below 2^-100 quantises to zero (s = 0),
+// which keeps g, r and the products finite; a block with dq == 0 has codes 0.
+// ---------------------------------------------------------------------------
+constexpr float kNvMinAmax = 7.8886090522101181e-31f;  // 2^-100
+
+struct NvScale {
+  float s;  // per-tensor scale
+  float g;  // 1 / (6 s)
+};
+
+__device__ __forceinline__ NvScale nv_tensor_scale(uint32_t amax_bits) {
+  const float amax = __uint_as_float(amax_bits);
+  NvScale t{0.f, 0.f};
+  if (amax >= kNvMinAmax) {
+    t.s = __fdiv_rn(amax, 2688.0f);
+    t.g = __frcp_rn(__fmul_rn(t.s, 6.0f));
+  }
+  return t;
+}
+
+// E4M3 byte of v >= 0: nearest, ties to even, saturating at 448.
+__device__ __forceinline__ uint32_t cvt_e4m3(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(v));
+  return r & 0xffu;
+}
+
+// Value of a non-negative finite E4M3 byte (exponent bias 7, 3 fraction
+// bits; exponent 0 is m * 2^-9).
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+}
+
+// Quantise 16 values: returns the E4M3 scale byte and the 8 bytes of codes
+// (element 2i in the low nibble of byte i).
+__device__ __forceinline__ uint32_t nv_quant_block16(const float (&v)[16], NvScale t, uint2& q) {
+  q = make_uint2(0u, 0u);
+  if (t.s == 0.f) return 0u;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t e = cvt_e4m3(__fmul_rn(amax, t.g));
+  const float dq = __fmul_rn(e4m3_value(e), t.s);
+  if (dq > 0.f) {
+    const float r = __frcp_rn(dq);
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int j = 0; j < 4; j++)
+        acc |= cvt_e2m1x2(__fmul_rn(v[8 * h + 2 * j], r), __fmul_rn(v[8 * h + 2 * j + 1], r)) << (8 * j);
+      w[h] = acc;
+    }
+    q = make_uint2(w[0], w[1]);
+  }
+  return e;
+}
+
+// Largest magnitude of a thread's values, folded into *out (fp32 bits of a
+// non-negative value order like the values): warp maximum, one atomic.
+__device__ __forceinline__ void amax_fold(uint32_t m, uint32_t* out) {
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(out, m);
+}
+
 }  // namespace ft

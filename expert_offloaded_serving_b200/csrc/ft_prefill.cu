@@ -65,6 +65,77 @@ __global__ void __launch_bounds__(256) k_quant_x(const uint16_t* __restrict__ x,
   }
 }
 
+// NVFP4 variant of k_quant_x: per 16 values, with the per-tensor scale of x
+// from *amax (all T tokens).
+__global__ void __launch_bounds__(256) k_quant_x_nv(const uint16_t* __restrict__ x, int T, int H, int E, int k,
+                                                    int n_seg, const int32_t* __restrict__ pad_offs,
+                                                    const int32_t* __restrict__ offs, const int32_t* __restrict__ perm,
+                                                    int rows_bound, const uint32_t* __restrict__ amax,
+                                                    uint8_t* __restrict__ xq, uint8_t* __restrict__ xq_sf) {
+  const int lane = threadIdx.x & 31;
+  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (p >= rows_bound || p >= pad_offs[n_seg]) return;
+  const NvScale ts = nv_tensor_scale(*amax);
+  const int e = segment_of(pad_offs, n_seg, p);
+  const int r = p - pad_offs[e];
+  const bool shared = e >= E;
+  const int count = shared ? T : offs[e + 1] - offs[e];
+  const int token = r < count ? (shared ? r : perm[offs[e] + r] / k) : -1;
+  const int atoms_k = H / 64;
+  for (int b = lane; b < H / 32; b += 32) {
+    uint2 q0 = make_uint2(0u, 0u), q1 = q0;
+    uint32_t e0 = 0, e1 = 0;
+    if (token >= 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)token * H + b * 32);
+      float v[2][16];
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const uint4 w = __ldg(src + i);
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          v[i >> 1][8 * (i & 1) + 2 * j] = bf16_bits_to_f32(u[j] & 0xffff);
+          v[i >> 1][8 * (i & 1) + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+        }
+      }
+      e0 = nv_quant_block16(v[0], ts, q0);
+      e1 = nv_quant_block16(v[1], ts, q1);
+    }
+    *reinterpret_cast<uint4*>(xq + (size_t)p * (H / 2) + b * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+    *reinterpret_cast<uint16_t*>(xq_sf + sf_word(p, b >> 1, atoms_k) + ((2 * b) & 3)) = (uint16_t)(e0 | (e1 << 8));
+  }
+}
+
+// NVFP4 h: the gate/up GEMM left h in fp32 ([rows][I], padded rows) and its
+// largest magnitude in *amax; quantise every padded row with that per-tensor
+// scale (padding rows are zeros and give zero codes and scales).
+__global__ void __launch_bounds__(256) k_quant_h_nv(const float* __restrict__ hf, int I, int n_seg,
+                                                    const int32_t* __restrict__ pad_offs, int rows_bound,
+                                                    const uint32_t* __restrict__ amax, uint8_t* __restrict__ hq,
+                                                    uint8_t* __restrict__ hq_sf) {
+  const int lane = threadIdx.x & 31;
+  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (p >= rows_bound || p >= pad_offs[n_seg]) return;
+  const NvScale ts = nv_tensor_scale(*amax);
+  const int atoms_k = I / 64;
+  for (int b = lane; b < I / 32; b += 32) {
+    const float4* src = reinterpret_cast<const float4*>(hf + (size_t)p * I + b * 32);
+    float v[2][16];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float4 f = src[i];
+      v[i >> 2][4 * (i & 3)] = f.x;
+      v[i >> 2][4 * (i & 3) + 1] = f.y;
+      v[i >> 2][4 * (i & 3) + 2] = f.z;
+      v[i >> 2][4 * (i & 3) + 3] = f.w;
+    }
+    uint2 q0, q1;
+    const uint32_t e0 = nv_quant_block16(v[0], ts, q0), e1 = nv_quant_block16(v[1], ts, q1);
+    *reinterpret_cast<uint4*>(hq + (size_t)p * (I / 2) + b * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+    *reinterpret_cast<uint16_t*>(hq_sf + sf_word(p, b >> 1, atoms_k) + ((2 * b) & 3)) = (uint16_t)(e0 | (e1 << 8));
+  }
+}
+
 // out[t][n] = bf16( sum_j w[t][j] * y[inv[t*k+j]][n]  +  sum_s y[T*k + s*T + t][n] )
 __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y, const float* __restrict__ w,
                                                  const int32_t* __restrict__ inv, int T, int H, int k, int n_shared,
@@ -95,11 +166,15 @@ ft_status ensure_prefill_scratch(PrefillScratch& s, const ft_model_desc& d, int 
   s.I = d.inter;
   s.max_pairs = T * k + S * T;
   s.max_rows = prefill_rows_bound(max_tokens, d.n_experts, d.top_k, d.n_shared);
+  s.fmt = d.weight_format == FT_FMT_NVFP4 ? kFmtNv : kFmtMx;
+  const int blk = s.fmt == kFmtNv ? 16 : 32;  // elements per block scale
   if (cudaMalloc(&s.xq, (size_t)s.max_rows * s.H / 2) != cudaSuccess ||
-      cudaMalloc(&s.xq_sf, (size_t)s.max_rows * s.H / 32) != cudaSuccess ||
+      cudaMalloc(&s.xq_sf, (size_t)s.max_rows * s.H / blk) != cudaSuccess ||
       cudaMalloc(&s.hq, (size_t)s.max_rows * s.I / 2) != cudaSuccess ||
-      cudaMalloc(&s.hq_sf, (size_t)s.max_rows * s.I / 32) != cudaSuccess ||
-      cudaMalloc(&s.y, (size_t)s.max_pairs * s.H * sizeof(float)) != cudaSuccess) {
+      cudaMalloc(&s.hq_sf, (size_t)s.max_rows * s.I / blk) != cudaSuccess ||
+      cudaMalloc(&s.y, (size_t)s.max_pairs * s.H * sizeof(float)) != cudaSuccess ||
+      (s.fmt == kFmtNv && (cudaMalloc(&s.hf, (size_t)s.max_rows * s.I * sizeof(float)) != cudaSuccess ||
+                           cudaMalloc(&s.amax, 2 * sizeof(uint32_t)) != cudaSuccess))) {
     free_prefill_scratch(s);
     return FT_ERR_CUDA;
   }
@@ -117,6 +192,8 @@ void free_prefill_scratch(PrefillScratch& s) {
   cudaFree(s.hq);
   cudaFree(s.hq_sf);
   cudaFree(s.y);
+  cudaFree(s.hf);
+  cudaFree(s.amax);
   s = PrefillScratch{};
 }
 
@@ -128,8 +205,26 @@ cudaError_t launch_shared_segments(int32_t* pad_offs, int E, int T, int n_shared
 
 cudaError_t launch_quant_x(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
   const int64_t rows = prefill_rows_bound(a.T, a.E, a.k, a.n_shared);
+  if (s.fmt == kFmtNv) {
+    // the per-tensor scale of x: largest |x| over all T tokens
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(s.amax, 0, 2 * sizeof(uint32_t), st)) != cudaSuccess ||
+        (e = launch_amax(a.x, (int64_t)a.T * a.H, true, s.amax, st)) != cudaSuccess)
+      return e;
+    k_quant_x_nv<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a.x, a.T, a.H, a.E, a.k, a.E + a.n_shared, a.pad_offs,
+                                                            a.offs, a.perm, (int)rows, s.amax, s.xq, s.xq_sf);
+    return cudaGetLastError();
+  }
   k_quant_x<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a.x, a.T, a.H, a.E, a.k, a.E + a.n_shared, a.pad_offs, a.offs,
                                                        a.perm, (int)rows, s.xq, s.xq_sf);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_h(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
+  if (s.fmt != kFmtNv) return cudaSuccess;  // MXFP4: the gate/up epilogue wrote hq itself
+  const int64_t rows = prefill_rows_bound(a.T, a.E, a.k, a.n_shared);
+  k_quant_h_nv<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s.hf, a.I, a.E + a.n_shared, a.pad_offs, (int)rows,
+                                                          s.amax + 1, s.hq, s.hq_sf);
   return cudaGetLastError();
 }
 
@@ -150,6 +245,13 @@ static GemmArgs gemm_args(const PrefillScratch& s, const PrefillArgs& a, int mod
   g.pool = a.pool;
   g.sfb = mode == 0 ? s.xq_sf : s.hq_sf;
   g.mode = mode;
+  g.fmt = s.fmt;
+  if (s.fmt == kFmtNv) {
+    g.ts_off = a.lay.ts;
+    g.amax_in = s.amax + (mode == 0 ? 0 : 1);  // x for gate/up, h for down
+    g.amax_out = s.amax + 1;
+    g.hf = s.hf;
+  }
   g.hq = s.hq;
   g.hq_sf = s.hq_sf;
   g.y = s.y;

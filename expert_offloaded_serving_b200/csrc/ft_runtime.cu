@@ -177,6 +177,7 @@ struct ft_ctx {
   int* d_sync = nullptr;       // persistent stack kernel counters [L][sync_stride]
   int sync_stride = 0;
   int* d_flag = nullptr;       // a device flag nothing sets (failure injection)
+  uint32_t* d_qamax = nullptr; // ft_quantize_nvfp4: largest |x| (fp32 bits)
   uint64_t* d_tagged = nullptr;    // persistent kernels, T <= 2: tagged h, then tagged x
   uint64_t* d_h_tagged = nullptr;  // [T*k + S*T][I] words
   uint64_t* d_x_tagged = nullptr;  // [T][H/2] words (dataflow kernel)
@@ -409,7 +410,7 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
 
   const int T = desc->max_tokens;
   ft_status st;
-  if ((st = dev_alloc(&c->d_status, 1)) || (st = dev_alloc(&c->d_flag, 1)) ||
+  if ((st = dev_alloc(&c->d_status, 1)) || (st = dev_alloc(&c->d_flag, 1)) || (st = dev_alloc(&c->d_qamax, 1)) ||
       (st = dev_alloc(&c->d_logits, (size_t)T * E)) ||
       (st = dev_alloc(&c->d_ids, (size_t)T * k)) || (st = dev_alloc(&c->d_w, (size_t)T * k)) ||
       (st = dev_alloc(&c->d_offs, E + 1)) || (st = dev_alloc(&c->d_perm, (size_t)T * k)) ||
@@ -537,6 +538,7 @@ extern "C" ft_status ft_destroy(ft_ctx* c) {
   free_prefill_scratch(c->pf);
   cudaFree(c->d_status);
   cudaFree(c->d_flag);
+  cudaFree(c->d_qamax);
   cudaFree(c->d_logits);
   cudaFree(c->d_ids);
   cudaFree(c->d_w);
@@ -653,6 +655,15 @@ extern "C" ft_status ft_quantize_mxfp4(ft_ctx* c, const float* x, int64_t R, int
   if (!c || (!x && R > 0) || !codes || !scales) return fail(FT_ERR_INVALID, "NULL argument");
   if (R < 0 || K <= 0 || K % 128) return fail(FT_ERR_INVALID, "K=%d not a positive multiple of 128", K);
   CUDA_TRY(launch_quantize_rows(x, R, K, codes, scales, (cudaStream_t)stream));
+  return FT_OK;
+}
+
+extern "C" ft_status ft_quantize_nvfp4(ft_ctx* c, const float* x, int64_t R, int32_t K, uint8_t* codes,
+                                       uint8_t* scales, float* tensor_scale, void* stream) {
+  if (!c || (!x && R > 0) || !codes || !scales || !tensor_scale) return fail(FT_ERR_INVALID, "NULL argument");
+  if (R < 0 || K <= 0 || K % 128) return fail(FT_ERR_INVALID, "K=%d not a positive multiple of 128", K);
+  CUDA_TRY(launch_quantize_rows_nv(x, R, K, c->d_qamax, codes, scales, tensor_scale, (cudaStream_t)stream));
+  c->last_stream = (cudaStream_t)stream;
   return FT_OK;
 }
 
@@ -1252,14 +1263,19 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   if (T < 0 || T > c->max_tokens) return fail(FT_ERR_INVALID, "T=%lld outside [0, max_tokens=%d]", (long long)T, c->max_tokens);
   if (!logits_override && !router_w) return fail(FT_ERR_INVALID, "need router_w or logits_override");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
-  const bool mx = (flags & FT_ACT_MXFP4) != 0;
-  if (mx && (c->d.hidden % 256 || c->d.inter % 256))
-    return fail(FT_ERR_INVALID, "the MXFP4 prefill path needs hidden and inter to be multiples of 256");
-  if (mx && c->d.weight_format != FT_FMT_MXFP4)
-    return fail(FT_ERR_INVALID, "the prefill path (FT_ACT_MXFP4) takes MXFP4 weights only");
-  if (!mx && T > c->decode_max_t)
+  // prefill path: FT_ACT_MXFP4 (MXFP4 weights) or FT_ACT_NVFP4 (NVFP4 weights)
+  const bool nv = (flags & FT_ACT_NVFP4) != 0;
+  const bool pf = nv || (flags & FT_ACT_MXFP4) != 0;
+  if (nv && (flags & FT_ACT_MXFP4)) return fail(FT_ERR_INVALID, "FT_ACT_MXFP4 and FT_ACT_NVFP4 exclude each other");
+  if (pf && (c->d.hidden % 256 || c->d.inter % 256))
+    return fail(FT_ERR_INVALID, "the prefill path needs hidden and inter to be multiples of 256");
+  if (pf && !nv && c->d.weight_format != FT_FMT_MXFP4)
+    return fail(FT_ERR_INVALID, "FT_ACT_MXFP4 (prefill) takes MXFP4 weights only");
+  if (nv && c->d.weight_format != FT_FMT_NVFP4)
+    return fail(FT_ERR_INVALID, "FT_ACT_NVFP4 (prefill) takes NVFP4 weights only");
+  if (!pf && T > c->decode_max_t)
     return fail(FT_ERR_INVALID, "decode GEMV path takes T <= %d (use FT_ACT_MXFP4 for prefill)", c->decode_max_t);
-  if (!mx && !decode_supported(c->d.hidden, c->d.inter, c->d.weight_format))
+  if (!pf && !decode_supported(c->d.hidden, c->d.inter, c->d.weight_format))
     return fail(FT_ERR_INVALID, "decode GEMV path takes hidden and inter up to 16384 (use FT_ACT_MXFP4)");
   if (T == 0) return FT_OK;
   cudaStream_t s = (cudaStream_t)stream;
@@ -1275,14 +1291,14 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     logits = c->d_logits;
   }
   Route* rec = c->d_routes + layer;
-  if (mx) {
+  if (pf) {
     KTimer kt(c, FT_K_TOPK, s);
     CUDA_TRY(launch_topk(logits, Ti, E, k, (flags & FT_ROUTE_RENORM) ? 1 : 0, c->d_ids, c->d_w, c->d_status, s));
   } else {
     KTimer kt(c, FT_K_TOPK, s);
     CUDA_TRY(launch_route(route_args(c, logits, Ti, 1, flags, rec), s));
   }
-  if (mx) {
+  if (pf) {
     KTimer kt(c, FT_K_PERMUTE, s);
     CUDA_TRY(launch_permute(c->d_ids, Ti * k, E, c->d_offs, c->d_perm, c->d_inv, c->d_active, c->d_nact,
                             c->d_pad_offs, c->d_status, s));
@@ -1301,7 +1317,7 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   if (c->resident[layer]) {
     eptr = c->d_eptr_res + (size_t)layer * c->n_blobs;
     pool = c->resident[layer];
-  } else if (mx) {
+  } else if (pf) {
     if (c->stage_layer[layer & 1] != layer)
       return fail(FT_ERR_NOT_FOUND, "prefill of layer %d: not resident and not prefetched", layer);
     stage_buf = layer & 1;
@@ -1362,7 +1378,7 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   }
 
   // 5: experts and combine
-  if (!mx && !miss_units.empty()) {
+  if (!pf && !miss_units.empty()) {
     // cache path with misses: the resident experts (hits and the shared
     // experts) run at once, while the misses' copies are in flight; each
     // missed expert runs after its own copy ([no] experts fetched over PCIe;
@@ -1407,7 +1423,7 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     // the waits above hold the events' current records: they can be reused
     for (cudaEvent_t e : c->miss_events) c->spare_miss_events.push_back(e);
     c->miss_events.clear();
-  } else if (!mx) {
+  } else if (!pf) {
     for (cudaEvent_t e : c->miss_events) c->spare_miss_events.push_back(e);
     c->miss_events.clear();
     DecodeArgs a = decode_args(c, (const uint16_t*)x, rec, Ti, eptr, (uint16_t*)out);
@@ -1449,6 +1465,10 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
     {
       KTimer kt(c, FT_K_GEMM_GATE_UP, s);
       CUDA_TRY(launch_prefill_gemm(c->pf, a, 0, s));
+    }
+    if (nv) {
+      KTimer kt(c, FT_K_QUANT_H, s);
+      CUDA_TRY(launch_quant_h(c->pf, a, s));
     }
     {
       KTimer kt(c, FT_K_GEMM_DOWN, s);
@@ -1529,7 +1549,8 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   if (T < 0 || T > c->decode_max_t) return fail(FT_ERR_INVALID, "T=%lld outside [0, %d]", (long long)T, c->decode_max_t);
   if (!decode_supported(c->d.hidden, c->d.inter, c->d.weight_format))
     return fail(FT_ERR_INVALID, "decode kernels take hidden and inter up to 16384");
-  if (flags & FT_ACT_MXFP4) return fail(FT_ERR_INVALID, "the stacked forward is the decode path (FT_ACT_BF16)");
+  if (flags & (FT_ACT_MXFP4 | FT_ACT_NVFP4))
+    return fail(FT_ERR_INVALID, "the stacked forward is the decode path (FT_ACT_BF16)");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
   for (int l = first_layer; l < first_layer + n_layers; l++)
     if (!c->resident[l]) return fail(FT_ERR_STATE, "layer %d is not resident", l);

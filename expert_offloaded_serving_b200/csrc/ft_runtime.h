@@ -36,10 +36,13 @@ struct PrefillScratch {
   int64_t max_pairs = 0;    // rows of y
   int H = 0, I = 0;
   uint8_t* xq = nullptr;    // [max_rows][H/2]
-  uint8_t* xq_sf = nullptr; // atoms over [max_rows][H/32]
+  uint8_t* xq_sf = nullptr; // atoms over [max_rows][H/32] (NVFP4: H/16)
   uint8_t* hq = nullptr;    // [max_rows][I/2]
-  uint8_t* hq_sf = nullptr; // atoms over [max_rows][I/32]
+  uint8_t* hq_sf = nullptr; // atoms over [max_rows][I/32] (NVFP4: I/16)
   float* y = nullptr;       // [max_pairs][H]
+  int fmt = 0;              // kFmtMx or kFmtNv (the context's weight format)
+  float* hf = nullptr;      // NVFP4: h in fp32 [max_rows][I] before its quantisation
+  uint32_t* amax = nullptr; // NVFP4: largest |x| and |h| (fp32 bits)
   CUtensorMap map_xq;       // TMA maps of xq and hq (token side of the GEMMs)
   CUtensorMap map_hq;
 };
@@ -52,7 +55,10 @@ ft_status ensure_prefill_scratch(PrefillScratch& s, const ft_model_desc& d, int 
 void free_prefill_scratch(PrefillScratch& s);
 cudaError_t launch_shared_segments(int32_t* pad_offs, int E, int T, int n_shared, cudaStream_t st);
 cudaError_t launch_quant_x(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
-// mode 0: gate/up GEMM + SwiGLU + MXFP4 h;  mode 1: down GEMM -> y
+// NVFP4: quantise the fp32 h the gate/up GEMM left (no-op for MXFP4)
+cudaError_t launch_quant_h(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
+// mode 0: gate/up GEMM + SwiGLU + MXFP4 h (NVFP4: fp32 h and its largest
+// magnitude);  mode 1: down GEMM -> y
 cudaError_t launch_prefill_gemm(const PrefillScratch& s, const PrefillArgs& a, int mode, cudaStream_t st);
 cudaError_t launch_prefill_combine(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st);
 

@@ -87,8 +87,8 @@ typedef struct {
  *          128-row x 4-block atoms; then the fp32 scales of Wg, Wu, Wd and 4
  *          zero bytes.  A weight is code value x block scale x matrix scale.
  *   BF16   Wg [I][H], Wu [I][H], Wd [H][I] as little-endian bf16.
- * The decode paths (FT_ACT_BF16) take every format; the prefill path
- * (FT_ACT_MXFP4) takes MXFP4 weights only. */
+ * The decode paths (FT_ACT_BF16) take every format; the prefill path takes
+ * MXFP4 weights with FT_ACT_MXFP4 and NVFP4 weights with FT_ACT_NVFP4. */
 #define FT_FMT_MXFP4 0
 #define FT_FMT_NVFP4 1
 #define FT_FMT_BF16  2
@@ -100,6 +100,8 @@ typedef struct {
 #define FT_STACK_LAYERWISE 4u /* ft_moe_stack_forward: two kernels per layer, not a persistent kernel */
 #define FT_STACK_COUNTERS  8u /* ft_moe_stack_forward: the counter-synchronised persistent kernel, not the dataflow one */
 #define FT_CACHE_SERIAL   16u /* cache path: every miss copy lands before any expert runs (for comparison) */
+#define FT_ACT_NVFP4      32u /* prefill with NVFP4 weights: x and h quantised to NVFP4, grouped GEMM on
+                                 tcgen05 kind::mxf4nvf4 (see ft_quantize_nvfp4 for the quantiser) */
 
 /* cache trace events */
 #define FT_EV_HIT   0
@@ -219,6 +221,23 @@ FT_API ft_status ft_moe_permute(ft_ctx* ctx, const int32_t* ids, int64_t T, int3
 FT_API ft_status ft_quantize_mxfp4(ft_ctx* ctx, const float* x, int64_t R, int32_t K,
                             uint8_t* codes, uint8_t* scales, void* stream);
 
+/* NVFP4 quantisation of rows (the prefill activations of NVFP4 experts;
+ * [no] "Hvor raskt kjører modellene?" names the NVFP4 build, the scaling is
+ * this library's reading): x dev fp32 [R][K] (finite) -> codes dev uint8
+ * [R][K/2] (two e2m1 per byte, element 2i low), scales dev uint8 (E4M3, one
+ * per 16 elements) laid out in 128x4 atoms over [pad128(R)][K/16] (the NVFP4
+ * blob scale layout), and *tensor_scale (dev fp32) the per-tensor scale s.
+ * Every step is one fp32 operation rounded to nearest even:
+ *   s = amax / 2688 (amax the largest |x|; s = 0 and every byte 0 when amax is
+ *   below 2^-100), g = 1 / (6 s); per block e = E4M3(amax_block * g) (nearest
+ *   even, saturating at 448), dq = value(e) * s, r = 1 / dq, codes
+ *   e2m1(v * r) (nearest even, saturating at 6, sign kept); dq == 0 gives
+ *   codes 0.  A value dequantises to code x value(e) x s.  Uses the
+ *   context's one reduction word: calls on one context must not overlap.
+ *   K % 128 == 0. */
+FT_API ft_status ft_quantize_nvfp4(ft_ctx* ctx, const float* x, int64_t R, int32_t K, uint8_t* codes,
+                                   uint8_t* scales, float* tensor_scale, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* layer forward                                                           */
 /* ---------------------------------------------------------------------- */
@@ -233,7 +252,10 @@ FT_API ft_status ft_quantize_mxfp4(ft_ctx* ctx, const float* x, int64_t R, int32
  *   router_w dev fp32 [E][H], used when logits_override is NULL.
  *   logits_override dev fp32 [T][E] or NULL.
  *   flags: FT_ACT_BF16 (decode GEMV; T <= 16 and <= max_tokens) or
- *   FT_ACT_MXFP4 (prefill grouped GEMM; any T <= max_tokens), | FT_ROUTE_RENORM.
+ *   FT_ACT_MXFP4 / FT_ACT_NVFP4 (prefill grouped GEMM on MXFP4 / NVFP4
+ *   weights; any T <= max_tokens), | FT_ROUTE_RENORM.  NVFP4 prefill
+ *   quantises x with one per-tensor scale over the T tokens and h with one
+ *   over every h row of the layer (routed pairs and the shared expert).
  * Weights come from, in this order: the layer's resident device pool; the
  * prefill staging buffer if ft_prefetch_layer(layer) was issued (the compute
  * stream waits for that copy, [fa] double-buffered prefill); otherwise the
@@ -442,7 +464,8 @@ FT_API ft_status ft_fp4_mma_probe(int64_t iters, float* sink, int32_t* status, i
 #define FT_K_GEMM_DOWN     7   /* prefill grouped GEMM, down */
 #define FT_K_COMBINE       8   /* prefill combine */
 #define FT_K_DEC_STACK     9   /* persistent decode kernel over a stack of layers */
-#define FT_K_COUNT         10
+#define FT_K_QUANT_H       10  /* NVFP4 prefill: quantiser of h (after the gate/up GEMM) */
+#define FT_K_COUNT         11
 
 /* Turn per-kernel CUDA-event timing on (1) or off (0).  While on, every
  * kernel launch of the forward path is bracketed by events on its stream (and

@@ -349,6 +349,63 @@ def nvfp4_matrix_scales_rotated():
     _nvfp4(ts_order=("wu", "wd", "wg"))
 
 
+def _nvfp4_act(block=16, tensor_scale=True, ties_up=False):
+    """The NVFP4 activation quantiser with one slip."""
+    def q(v, s=None):
+        v32 = np.asarray(v, dtype=np.float32)
+        R, K = v32.shape
+        if s is None:
+            s = formats.nvfp4_global_scale(np.abs(v32).max() if v32.size else 0.0)
+        s = np.float32(s) if tensor_scale else np.float32(1.0 if np.float32(s) != 0 else 0.0)
+        blocks = v32.reshape(R, K // block, block)
+        if s == 0:
+            return np.zeros((R, K), np.uint8), np.zeros((R, K // 16), np.uint8), s
+        with np.errstate(all="ignore"):
+            g = np.float32(np.float32(1.0) / np.float32(s * np.float32(6.0)))
+            b = (np.abs(blocks).max(axis=-1) * g).astype(np.float32)
+            e = formats.e4m3_round_vec(b)
+            if ties_up:  # ties to the larger byte
+                pos = formats.E4M3_TABLE[:0x7F]
+                hi = np.clip(np.searchsorted(pos, b, side="left"), 0, 0x7E)
+                tie = (hi > 0) & (np.abs(pos[hi] - b) == np.abs(b - pos[np.clip(hi - 1, 0, 0x7E)]))
+                e = np.where(tie & (b < 448), hi, e).astype(np.uint8)
+            dq = (formats.E4M3_TABLE[e].astype(np.float32) * s).astype(np.float32)
+            r = (np.float32(1.0) / np.where(dq > 0, dq, np.float32(1.0))).astype(np.float32)
+            qv = (blocks * r[..., None]).astype(np.float32)
+        mag = fp4.round_to_grid_vec(np.abs(qv).astype(np.float64))
+        codes = np.where((dq > 0)[..., None], mag | np.where(np.signbit(qv), 8, 0), 0).astype(np.uint8).reshape(R, K)
+        e = np.repeat(e, 16 // block, axis=1) if block < 16 else np.repeat(e, block // 16, axis=1)
+        return codes, e.astype(np.uint8), s
+    formats.nvfp4_quantize_rows = q
+
+
+def nvfp4_act_blocks_of_32():
+    _nvfp4_act(block=32)
+
+
+def nvfp4_act_tensor_scale_dropped():
+    _nvfp4_act(tensor_scale=False)
+
+
+def nvfp4_act_scale_ties_up():
+    _nvfp4_act(ties_up=True)
+
+
+def nvfp4_act_h_scale_per_expert():
+    def f(x, groups, hidden, inter):
+        cx, bx, sx = formats.nvfp4_quantize_rows(x)
+        xq = formats.nvfp4_dequant_rows(cx, bx, sx)
+        ys = []
+        for blob, rows in groups:
+            wg = formats.weight_matrix(blob, "wg", hidden, inter, "nvfp4")
+            wu = formats.weight_matrix(blob, "wu", hidden, inter, "nvfp4")
+            wd = formats.weight_matrix(blob, "wd", hidden, inter, "nvfp4")
+            h = layer.silu(xq[rows] @ wg.T) * (xq[rows] @ wu.T)
+            ys.append(formats.nvfp4_dequant_rows(*formats.nvfp4_quantize_rows(h)) @ wd.T)   # own scale per expert
+        return ys
+    layer._nvfp4_expert_outputs = f
+
+
 def _bf16_matrix(big_endian=False, transposed=False):
     def f(blob, which, hidden, inter):
         off = formats.bf16_layout(hidden, inter)
@@ -470,6 +527,7 @@ MUTANTS = {f.__name__: f for f in (
     silu_sign, gate_up_swapped, mxfp4_x_not_quantised, mxfp4_h_not_quantised, shared_expert_dropped,
     e4m3_bias, e4m3_subnormal_as_normal, nvfp4_blocks_of_32, nvfp4_matrix_scale_dropped,
     nvfp4_matrix_scales_rotated, bf16_big_endian, bf16_matrix_transposed,
+    nvfp4_act_blocks_of_32, nvfp4_act_tensor_scale_dropped, nvfp4_act_scale_ties_up, nvfp4_act_h_scale_per_expert,
     lru_evicts_most_recent, lru_may_evict_a_key_of_the_step, lru_takes_highest_free_slot, lru_hit_does_not_touch,
     lru_lookup_does_not_touch,
     resize_evicts_most_recent, resize_moves_descending, resize_moves_to_highest_free)}

@@ -12,7 +12,8 @@ import _oracle_mutants
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join("tests", f) for f in ("test_oracle_fp4.py", "test_oracle_routing.py", "test_oracle_layer.py",
-                                           "test_oracle_lru.py", "test_oracle_formats.py")]
+                                           "test_oracle_lru.py", "test_oracle_formats.py",
+                                           "test_oracle_nvfp4_act.py")]
 
 
 def run_pins(mutant):

@@ -60,6 +60,23 @@ def test_quantiser_worked_block():
     assert list(deq[0, 16:24]) == [12.0, 3.0, -2.0, 4.0, 8.0, 0.0, -1.0, 0.0]
 
 
+def test_quantiser_block_scale_ties():
+    """Ties of the block scale itself: amax = 1792 gives s = fp32(1792/2688)
+    = fp32(2/3) and 6 s rounds to exactly 4, so g = 1/4.  A block with
+    largest magnitude 4.25 gives b = 1.0625, halfway between E4M3's 1.0 (0x38)
+    and 1.125 (0x39): the even byte 0x38.  One with 4.75 gives b = 1.1875,
+    halfway between 1.125 (0x39) and 1.25 (0x3a): 0x3a.  In the first block
+    dq = s and r = 1/dq = 1.5: 4.25 -> 6.375 saturates to 6 (code 7), -1.0
+    -> -1.5 (code 8|3)."""
+    x = np.zeros((1, 48), np.float32)
+    x[0, 0] = 1792.0
+    x[0, 16], x[0, 17], x[0, 32] = 4.25, -1.0, 4.75
+    codes, scales, s = formats.nvfp4_quantize_rows(x)
+    assert s == np.float32(2.0 / 3.0) and np.float32(s * np.float32(6.0)) == 4.0
+    assert list(scales[0]) == [0x7E, 0x38, 0x3A]
+    assert list(codes[0, 16:18]) == [7, 8 | 3]
+
+
 def test_quantiser_zero_tensor_and_scale_of_the_largest_block():
     c, b, s = formats.nvfp4_quantize_rows(np.zeros((3, 32), np.float32))
     assert s == 0 and not c.any() and not b.any()
@@ -123,3 +140,28 @@ def test_nvfp4_layer_scale_spans_the_whole_batch():
     ea = layer.moe_layer(xb, blobs.__getitem__, H, I, E, K, **kw)["out_f64"]
     eb = layer.moe_layer(big, blobs.__getitem__, H, I, E, K, **kw)["out_f64"]
     assert np.array_equal(ea[:-1], eb[:-1])
+
+
+def _with_gate_scale(blob, H, I, factor):
+    """A copy of an NVFP4 blob with Wg's matrix scale multiplied by factor."""
+    b = np.array(blob, dtype=np.uint8, copy=True)
+    off = formats.nvfp4_layout(H, I)["tensor_scales"]
+    ts = b[off: off + 12].view("<f4")
+    ts[0] = np.float32(ts[0] * factor)
+    return b
+
+
+def test_nvfp4_h_scale_spans_every_expert():
+    """h's per-tensor scale comes from every expert's h: next to an expert
+    whose h is smaller, expert A's outputs are those it has alone; next to
+    one whose h is larger (its Wg scaled up), they change."""
+    H, I, T, seed = 256, 128, 8, 79
+    a = synth.expert_blob_nvfp4(seed, 0, 0, H, I)
+    other = synth.expert_blob_nvfp4(seed, 0, 1, H, I)
+    x = synth.bf16_bits_to_f32(synth.activations_bf16(seed, 1, T, H)).astype(np.float64)
+    rows = np.arange(T)
+    alone = layer._nvfp4_expert_outputs(x, [(a, rows)], H, I)[0]
+    small = layer._nvfp4_expert_outputs(x, [(a, rows), (_with_gate_scale(other, H, I, 1 / 64), rows)], H, I)[0]
+    big = layer._nvfp4_expert_outputs(x, [(a, rows), (_with_gate_scale(other, H, I, 64.0), rows)], H, I)[0]
+    assert np.array_equal(alone, small)
+    assert not np.array_equal(alone, big)
