@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--layerwise", action="store_true",
                     help="decode with two kernels per layer instead of a persistent stack kernel")
     ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4", "bf16"],
-                    help="expert weight format of the decode stack")
+                    help="expert weight format of the decode stack (and of --case gemm)")
     ap.add_argument("--counters", action="store_true",
                     help="decode with the counter-synchronised persistent kernel instead of the dataflow kernel")
     return ap.parse_args()
@@ -697,24 +697,29 @@ def measure_prefill_calibration(fp4_peak, T=65536, reps=2):
             "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps}
 
 
-def measure_gemm_small(reps=2, T=16384, E2=64):
+def measure_gemm_small(reps=2, T=16384, E2=64, fmt="mxfp4"):
     """The prefill GEMMs at the calibration case's 1,536 tokens per expert on
     a small pool: the DSV4-class expert shape (hidden 4096, intermediate
     2048, top-6) with 64 experts and 16,384 tokens (0.8 GB of experts), one
-    warm forward and `reps` timed ones through the MXFP4-activation path.
-    The workload of the GEMMs' ncu capture (a few GB on the device)."""
+    warm forward and `reps` timed ones through the MXFP4-activation path
+    (fmt "nvfp4": NVFP4 experts through the NVFP4-activation path).  The
+    workload of the GEMMs' ncu captures (a few GB on the device)."""
     import numpy as np
     import torch
     import expert_offloaded_serving_b200 as ft
     import synth
     import synth.gpu
     H2, I2, k2, seed = 4096, 2048, 6, 1005
-    pool = synth.gpu.layer_pool(H2, I2, E2, seed, 0)
-    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, 1, 0, 0, T), None, [pool])
+    if fmt not in ("mxfp4", "nvfp4"):
+        raise SystemExit("--case gemm takes --format mxfp4 or nvfp4 (the prefill path has no BF16 experts)")
+    nv = fmt == "nvfp4"
+    pool = synth.gpu.layer_pool(H2, I2, E2, seed, 0, fmt=fmt)
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, 1, 0, 0, T,
+                                    weight_format=ft.FT_FMT_NVFP4 if nv else ft.FT_FMT_MXFP4), None, [pool])
     x = torch.from_numpy(synth.activations_bf16(seed, 1, T, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
     lg = torch.from_numpy(synth.logits_for_sets(seed, 3, synth.near_uniform_sets(seed, 0, T, E2, k2), E2)).cuda()
     out = torch.empty_like(x)
-    flags = ft.FT_ACT_MXFP4 | ft.FT_ROUTE_RENORM
+    flags = (ft.FT_ACT_NVFP4 if nv else ft.FT_ACT_MXFP4) | ft.FT_ROUTE_RENORM
     ft.ft_moe_layer_forward(ctx, 0, x, T, None, lg, out, flags)
     torch.cuda.synchronize()
     ft.ft_kernel_timing_enable(ctx, True)
@@ -726,7 +731,8 @@ def measure_gemm_small(reps=2, T=16384, E2=64):
     ft.ft_destroy(ctx)
     gemm_ms = (kt["gemm_gate_up"][0] + kt["gemm_down"][0]) / reps
     flops = 2.0 * T * k2 * 3 * H2 * I2
-    return {"workload": f"DSV4-shape prefill GEMMs, {E2} experts, {T} tokens top-{k2} ({T * k2 // E2} per expert)",
+    return {"workload": f"DSV4-shape prefill GEMMs, {E2} {fmt.upper()} experts, {T} tokens top-{k2} "
+                        f"({T * k2 // E2} per expert)",
             "gemm_ms": gemm_ms, "gemm_tflops": flops / (gemm_ms * 1e-3) / 1e12,
             "gate_up_ms": kt["gemm_gate_up"][0] / reps, "down_ms": kt["gemm_down"][0] / reps}
 
@@ -1011,7 +1017,7 @@ def main():
     if args.case != "decode":
         if rank == 0:
             r = {"prefill": lambda: measure_prefill(reps=max(args.steps, 1)), "miss": measure_misses,
-                 "glm": measure_glm, "gemm": lambda: measure_gemm_small(reps=max(args.steps, 1)),
+                 "glm": measure_glm, "gemm": lambda: measure_gemm_small(reps=max(args.steps, 1), fmt=args.format),
                  "router": lambda: measure_router(reps=max(args.steps, 1)),
                  "nvfp4": lambda: measure_prefill_nvfp4(measure_fp4_peak()["tflops"], peaks())}[args.case]()
             print(json.dumps({"case": args.case, **r}))
