@@ -295,14 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
           const float sx = nv_tensor_scale(*a.amax_in).s;
           const float cgt = __fmul_rn(ts[0], sx), cut = __fmul_rn(ts[1], sx);
           float* h_col = a.hf + (size_t)(row0 + 32 * cg) * I + irow;
+          // the segment's padding rows hold no token: their h is not stored
+          // (the quantiser writes them as zeros)
+          const int valid = (e >= a.E ? a.T : a.offs[e + 1] - a.offs[e]) - (row0 - a.pad_offs[e] + 32 * cg);
           uint32_t m = 0;
 #pragma unroll
           for (int q = 0; q < 32; q++) {
             const float g = __fmul_rn(__uint_as_float(q < 16 ? g0[q & 15] : g1[q & 15]), cgt);
             const float u = __fmul_rn(__uint_as_float(q < 16 ? u0[q & 15] : u1[q & 15]), cut);
             const float hv = silu(g) * u;
-            h_col[(size_t)q * I] = hv;
-            m = max(m, __float_as_uint(hv) & 0x7fffffffu);
+            if (q < valid) {
+              h_col[(size_t)q * I] = hv;
+              m = max(m, __float_as_uint(hv) & 0x7fffffffu);
+            }
           }
           amax_fold(m, a.amax_out);
           continue;

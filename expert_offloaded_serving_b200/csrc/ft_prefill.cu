@@ -109,8 +109,9 @@ __global__ void __launch_bounds__(256) k_quant_x_nv(const uint16_t* __restrict__
 // NVFP4 h: the gate/up GEMM left h in fp32 ([rows][I], padded rows) and its
 // largest magnitude in *amax; quantise every padded row with that per-tensor
 // scale (padding rows are zeros and give zero codes and scales).
-__global__ void __launch_bounds__(256) k_quant_h_nv(const float* __restrict__ hf, int I, int n_seg,
-                                                    const int32_t* __restrict__ pad_offs, int rows_bound,
+__global__ void __launch_bounds__(256) k_quant_h_nv(const float* __restrict__ hf, int I, int T, int E, int n_seg,
+                                                    const int32_t* __restrict__ pad_offs,
+                                                    const int32_t* __restrict__ offs, int rows_bound,
                                                     const uint32_t* __restrict__ amax, uint8_t* __restrict__ hq,
                                                     uint8_t* __restrict__ hq_sf) {
   const int lane = threadIdx.x & 31;
@@ -118,12 +119,15 @@ __global__ void __launch_bounds__(256) k_quant_h_nv(const float* __restrict__ hf
   if (p >= rows_bound || p >= pad_offs[n_seg]) return;
   const NvScale ts = nv_tensor_scale(*amax);
   const int atoms_k = I / 64;
+  const int e = segment_of(pad_offs, n_seg, p);
+  // a padding row of the segment: its h (never stored) is zero
+  const bool pad = p - pad_offs[e] >= (e >= E ? T : offs[e + 1] - offs[e]);
   for (int b = lane; b < I / 32; b += 32) {
     const float4* src = reinterpret_cast<const float4*>(hf + (size_t)p * I + b * 32);
     float v[2][16];
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-      const float4 f = src[i];
+      const float4 f = pad ? make_float4(0.f, 0.f, 0.f, 0.f) : src[i];
       v[i >> 2][4 * (i & 3)] = f.x;
       v[i >> 2][4 * (i & 3) + 1] = f.y;
       v[i >> 2][4 * (i & 3) + 2] = f.z;
@@ -223,8 +227,8 @@ cudaError_t launch_quant_x(const PrefillScratch& s, const PrefillArgs& a, cudaSt
 cudaError_t launch_quant_h(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
   if (s.fmt != kFmtNv) return cudaSuccess;  // MXFP4: the gate/up epilogue wrote hq itself
   const int64_t rows = prefill_rows_bound(a.T, a.E, a.k, a.n_shared);
-  k_quant_h_nv<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s.hf, a.I, a.E + a.n_shared, a.pad_offs, (int)rows,
-                                                          s.amax + 1, s.hq, s.hq_sf);
+  k_quant_h_nv<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s.hf, a.I, a.T, a.E, a.E + a.n_shared, a.pad_offs, a.offs,
+                                                          (int)rows, s.amax + 1, s.hq, s.hq_sf);
   return cudaGetLastError();
 }
 
