@@ -981,12 +981,19 @@ def measure_decode_batch(args, T, pk):
     return out
 
 
-def decode_kernel_name(T, layerwise=False, counters=False):
+def decode_kernel_name(T, layerwise=False, counters=False, fmt="mxfp4"):
+    """The kernels ft_moe_stack_forward runs for this batch: the dataflow
+    kernel when its geometry takes the stack, else the counter-synchronised
+    kernel (MXFP4 only), else two kernels per layer."""
+    import expert_offloaded_serving_b200 as ft
     if layerwise:
         return "two per layer"
-    if counters or T > 2:
+    code = {"mxfp4": ft.FT_FMT_MXFP4, "nvfp4": ft.FT_FMT_NVFP4, "bf16": ft.FT_FMT_BF16}[fmt]
+    if not counters and ft.ft_flow_geometry(H, I, T, K_TOP, S_SHARED, E, L, code)["ok"]:
+        return "persistent stack kernel, dataflow (tagged hand-overs)"
+    if code == ft.FT_FMT_MXFP4:
         return "persistent stack kernel, counter-synchronised"
-    return "persistent stack kernel, dataflow (tagged hand-overs)"
+    return "two per layer"
 
 
 FORMAT_NAMES = {"mxfp4": "MXFP4 (e2m1 + UE8M0/32)", "nvfp4": "NVFP4 (e2m1 + E4M3/16 + fp32 per matrix)",
@@ -994,7 +1001,7 @@ FORMAT_NAMES = {"mxfp4": "MXFP4 (e2m1 + UE8M0/32)", "nvfp4": "NVFP4 (e2m1 + E4M3
 
 
 def workload_config(T, layerwise=False, counters=False, fmt="mxfp4"):
-    return {"decode_kernels": decode_kernel_name(T, layerwise, counters),
+    return {"decode_kernels": decode_kernel_name(T, layerwise, counters, fmt),
             "workload": f"35B-A3B-class MoE decode stack: hidden {H}, {E} routed experts top-{K_TOP} + {S_SHARED} shared, "
                         f"intermediate {I}, {L} layers, {FORMAT_NAMES[fmt]} weights resident in HBM, "
                         f"batch {T}, Zipf(1.1) routing traces with 0.6 adjacent-token reuse",
