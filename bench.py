@@ -248,8 +248,7 @@ def run_ours(args, world, rank):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             final = one_pass(x0)
-    # the routing kernel, then the persistent kernel or two kernels per layer
-    launches_per_step = 1 + (2 * L if args.layerwise else 1)
+    launches_per_step = stack_launches(T, args.layerwise, getattr(args, "counters", False), args.format)
 
     def step(p):
         logits_buf.copy_(logits_all[p % TRACE_LEN], non_blocking=True)
@@ -297,6 +296,7 @@ def run_ours(args, world, rank):
     gu_launch_bytes = float(np.mean([(uniq[p] + S_SHARED).mean() for p in pos])) * gu_bytes
     dn_launch_bytes = float(np.mean([(uniq[p] + S_SHARED).mean() for p in pos])) * d_bytes
     res["kernels"] = {k: {"ms_total": v[0], "launches": v[1], "us_avg": 1e3 * v[0] / v[1]} for k, v in kt.items() if v[1]}
+    res["kernel_steps"] = nk
     res["gate_up_bytes"] = gu_launch_bytes
     res["down_bytes"] = dn_launch_bytes
     res["stack_bytes"] = float(np.mean(bytes_pos[pos]))  # every layer's routed + shared blobs
@@ -976,22 +976,44 @@ def measure_decode_batch(args, T, pk):
            "clocks": res["clocks"]}
     st = res["kernels"].get("dec_stack")
     if st:
-        gbs = res["stack_bytes"] / (st["us_avg"] * 1e-6) / 1e9
-        out.update(kernel_us=st["us_avg"], kernel_gbs=gbs, kernel_frac=gbs / pk["hbm"])
+        # persistent-kernel time per step (a step runs one launch per wave)
+        us = 1e3 * st["ms_total"] / res["kernel_steps"]
+        gbs = res["stack_bytes"] / (us * 1e-6) / 1e9
+        out.update(kernel_us=us, kernel_gbs=gbs, kernel_frac=gbs / pk["hbm"])
     return out
 
 
-def decode_kernel_name(T, layerwise=False, counters=False, fmt="mxfp4"):
-    """The kernels ft_moe_stack_forward runs for this batch: the dataflow
-    kernel when its geometry takes the stack, else the counter-synchronised
-    kernel (MXFP4 only), else two kernels per layer."""
+def _stack_path(T, layerwise=False, counters=False, fmt="mxfp4"):
+    """The path ft_moe_stack_forward takes for a batch of T: ("flow", waves)
+    when the dataflow kernel's geometry takes the stack (one launch for up to
+    two tokens, waves of two for three or four), ("counters", 1) for the
+    counter-synchronised kernel (MXFP4 only), else ("layerwise", 0)."""
     import expert_offloaded_serving_b200 as ft
     if layerwise:
-        return "two per layer"
+        return "layerwise", 0
     code = {"mxfp4": ft.FT_FMT_MXFP4, "nvfp4": ft.FT_FMT_NVFP4, "bf16": ft.FT_FMT_BF16}[fmt]
-    if not counters and ft.ft_flow_geometry(H, I, T, K_TOP, S_SHARED, E, L, code)["ok"]:
-        return "persistent stack kernel, dataflow (tagged hand-overs)"
+    wave = T if T <= 2 else 2
+    if not counters and T <= 4 and ft.ft_flow_geometry(H, I, wave, K_TOP, S_SHARED, E, L, code)["ok"]:
+        return "flow", (T + wave - 1) // wave
     if code == ft.FT_FMT_MXFP4:
+        return "counters", 1
+    return "layerwise", 0
+
+
+def stack_launches(T, layerwise=False, counters=False, fmt="mxfp4"):
+    """Kernel launches of one stacked pass: a routing kernel and a persistent
+    kernel per wave, or the routing kernel and two kernels per layer."""
+    path, waves = _stack_path(T, layerwise, counters, fmt)
+    return 1 + 2 * L if path == "layerwise" else 2 * waves
+
+
+def decode_kernel_name(T, layerwise=False, counters=False, fmt="mxfp4"):
+    """The kernels ft_moe_stack_forward runs for this batch."""
+    path, waves = _stack_path(T, layerwise, counters, fmt)
+    if path == "flow":
+        return "persistent stack kernel, dataflow (tagged hand-overs)" + (
+            f", {waves} waves of two tokens" if waves > 1 else "")
+    if path == "counters":
         return "persistent stack kernel, counter-synchronised"
     return "two per layer"
 

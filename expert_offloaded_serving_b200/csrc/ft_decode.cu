@@ -754,7 +754,8 @@ template <int PER>
 __global__ void __launch_bounds__(kThreads) k_route(RouteArgs a) {
   __shared__ Route r;
   const int l = blockIdx.x;
-  route_in_cta<PER>(a.logits + (size_t)l * a.T * a.E, a.T, a.E, a.k, a.renorm, r, a.status);
+  route_in_cta<PER>(a.logits + (size_t)l * (a.layer_stride ? a.layer_stride : (int64_t)a.T * a.E), a.T, a.E, a.k,
+                    a.renorm, r, a.status);
   const int4* src = reinterpret_cast<const int4*>(&r);
   int4* dst = reinterpret_cast<int4*>(a.rec + l);
   for (int i = threadIdx.x; i < (int)(sizeof(Route) / 16); i += kThreads) dst[i] = src[i];

@@ -30,7 +30,8 @@ struct alignas(16) Route {
 };
 
 struct RouteArgs {
-  const float* logits;  // fp32 [n_layers][T][E]
+  const float* logits;  // fp32 [n_layers][T][E], layers layer_stride floats apart
+  int64_t layer_stride; // 0: T * E
   int T, E, k, renorm, n_layers;
   Route* rec;           // [n_layers]
   int32_t* ids_out;     // [T*k] of the last layer, or NULL

@@ -1560,13 +1560,64 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   const int H = c->d.hidden, I = c->d.inter;
   const bool layerwise = (flags & FT_STACK_LAYERWISE) != 0;
   // one or two tokens: the dataflow kernel (tagged h and x, down tiles over
-  // every unit); else, or with FT_STACK_COUNTERS, the counter-synchronised
-  // persistent kernel; else two kernels per layer
-  const FlowGeom fg = flow_geometry(H, I, Ti, c->d.top_k, c->d.n_shared, c->d.n_experts, n_layers, c->d.weight_format);
-  const bool flow = !layerwise && !(flags & FT_STACK_COUNTERS) && c->d_tagged != nullptr && fg.ok;
+  // every unit); three or four tokens: the dataflow kernel in waves of two
+  // (the tokens of a MoE layer do not interact, and each wave computes its
+  // tokens' bits as the per-layer path does); else, or with
+  // FT_STACK_COUNTERS, the counter-synchronised persistent kernel; else two
+  // kernels per layer
+  const int wave = Ti <= 2 ? Ti : 2;
+  const FlowGeom fg = flow_geometry(H, I, wave, c->d.top_k, c->d.n_shared, c->d.n_experts, n_layers,
+                                    c->d.weight_format);
+  const bool flow = !layerwise && !(flags & FT_STACK_COUNTERS) && c->d_tagged != nullptr && fg.ok && Ti <= 4;
   // the counter-synchronised kernel computes MXFP4 weights only
   const bool persistent = !layerwise && !flow && c->d_sync != nullptr && c->d.weight_format == FT_FMT_MXFP4 &&
                           stack_supported(H, I, n_layers);
+  if (flow) {
+    int dev = 0, nsm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int E = c->d.n_experts, k = c->d.top_k;
+    for (int t0 = 0; t0 < Ti; t0 += wave) {
+      const int Tw = std::min(wave, Ti - t0);
+      const FlowGeom fw = Tw == wave ? fg : flow_geometry(H, I, Tw, k, c->d.n_shared, E, n_layers, c->d.weight_format);
+      // the wave's routing records, from its rows of every layer's logits
+      {
+        KTimer kt(c, FT_K_TOPK, s);
+        RouteArgs ra = route_args(c, logits + (size_t)t0 * E, Tw, n_layers, flags, c->d_routes + first_layer);
+        ra.layer_stride = (int64_t)Ti * E;
+        ra.ids_out = c->d_ids + (size_t)t0 * k;
+        ra.w_out = c->d_w + (size_t)t0 * k;
+        ra.epoch = c->d_epoch;
+        ra.tagged = c->d_tagged;
+        ra.tagged_words = c->tagged_words;
+        CUDA_TRY(launch_route(ra, s));
+      }
+      FlowArgs a{};
+      a.x0 = (const uint16_t*)x + (size_t)t0 * H;
+      a.out = (uint16_t*)out + (size_t)t0 * H;
+      a.rec = c->d_routes + first_layer;
+      a.eptr = c->d_eptr_res + (size_t)first_layer * c->n_blobs;
+      a.n_layers = n_layers;
+      a.n_blobs = c->n_blobs;
+      a.T = Tw;
+      a.H = H;
+      a.I = I;
+      a.E = E;
+      a.k = k;
+      a.n_shared = c->d.n_shared;
+      a.lay = c->lay;
+      a.h_tagged = c->d_h_tagged;
+      a.x_tagged = c->d_x_tagged;
+      a.epoch = c->d_epoch;
+      a.rows_cap = fw.rows_cap;
+      a.status = c->d_status;
+      a.timeline = c->timeline && c->timeline_words >= (int64_t)n_layers * nsm * 8 ? c->timeline : nullptr;
+      KTimer kt(c, FT_K_DEC_STACK, s);
+      CUDA_TRY(launch_dec_flow(a, s));
+    }
+    c->last_stream = s;
+    return FT_OK;
+  }
   // all layers' routing records in one launch (their logits are inputs); it
   // also zeroes the counter-synchronised kernel's counters of those layers
   {
@@ -1576,41 +1627,7 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
       ra.sync = c->d_sync;
       ra.sync_stride = c->sync_stride;
     }
-    if (flow) {
-      ra.epoch = c->d_epoch;
-      ra.tagged = c->d_tagged;
-      ra.tagged_words = c->tagged_words;
-    }
     CUDA_TRY(launch_route(ra, s));
-  }
-  if (flow) {
-    FlowArgs a{};
-    a.x0 = (const uint16_t*)x;
-    a.out = (uint16_t*)out;
-    a.rec = c->d_routes + first_layer;
-    a.eptr = c->d_eptr_res + (size_t)first_layer * c->n_blobs;
-    a.n_layers = n_layers;
-    a.n_blobs = c->n_blobs;
-    a.T = Ti;
-    a.H = H;
-    a.I = I;
-    a.E = c->d.n_experts;
-    a.k = c->d.top_k;
-    a.n_shared = c->d.n_shared;
-    a.lay = c->lay;
-    a.h_tagged = c->d_h_tagged;
-    a.x_tagged = c->d_x_tagged;
-    a.epoch = c->d_epoch;
-    a.rows_cap = fg.rows_cap;
-    a.status = c->d_status;
-    int dev = 0, nsm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    a.timeline = c->timeline && c->timeline_words >= (int64_t)n_layers * nsm * 8 ? c->timeline : nullptr;
-    KTimer kt(c, FT_K_DEC_STACK, s);
-    CUDA_TRY(launch_dec_flow(a, s));
-    c->last_stream = s;
-    return FT_OK;
   }
   if (persistent) {
     StackArgs a{};

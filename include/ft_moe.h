@@ -278,16 +278,22 @@ FT_API ft_status ft_moe_layer_forward(ft_ctx* ctx, int32_t layer, const void* x,
  *   (router logits of each layer, all ready before the call).
  * Each layer computes what the ft_moe_layer_forward decode path computes, bit
  * for bit.  Because every layer's routing input is known up front, one
- * kernel routes all layers first.  Then, by default, one persistent
- * cooperative kernel runs every layer: each CTA takes its gate/up tile and its
- * down tile of a layer in turn, streams its next tiles' weights while it waits
- * for the layer's other CTAs, and layers hand over through counters in global
- * memory (waits bounded at 2 s; a timeout sets FT_ERR_TIMEOUT's status bit).
- * With FT_STACK_LAYERWISE, or for shapes whose two tiles do not fit one CTA's
- * shared memory, each layer runs as a gate/up and a down kernel instead, the
- * next layer's launched as programmatic dependents of the previous layer's.
+ * kernel routes all layers first; then one persistent cooperative kernel runs
+ * every layer (waits bounded at 2 s; a timeout sets FT_ERR_TIMEOUT's status
+ * bit):
+ *   - up to two tokens (when ft_flow_geometry takes the shape): the dataflow
+ *     kernel, whose hand-overs between CTAs are tagged words;
+ *   - three or four tokens: the same kernel in waves of two tokens (a routing
+ *     launch and a dataflow launch per wave; the tokens of a layer do not
+ *     interact, so the bits are the same);
+ *   - otherwise, or with FT_STACK_COUNTERS: the counter-synchronised kernel
+ *     (MXFP4 weights), in which each CTA takes its gate/up and down tiles of
+ *     a layer in turn and layers hand over through counters.
+ * With FT_STACK_LAYERWISE, or where no persistent kernel takes the shape and
+ * format, each layer runs as a gate/up and a down kernel instead.
  * Intermediate activations live in context scratch; calls on different
- * streams must not overlap.  flags: FT_ROUTE_RENORM | FT_STACK_LAYERWISE.
+ * streams must not overlap.
+ * flags: FT_ROUTE_RENORM | FT_STACK_LAYERWISE | FT_STACK_COUNTERS.
  * Errors: FT_ERR_INVALID, FT_ERR_STATE (a layer is not resident), FT_ERR_CUDA. */
 FT_API ft_status ft_moe_stack_forward(ft_ctx* ctx, int32_t first_layer, int32_t n_layers, const void* x, int64_t T,
                                       const float* logits, void* out, uint32_t flags, void* stream);
@@ -381,7 +387,8 @@ FT_API ft_status ft_debug_dequant(ft_ctx* ctx, const void* blob, int32_t mat, fl
 FT_API ft_status ft_decode_geometry(int32_t hidden, int32_t inter, int32_t n_layers, int64_t out[24]);
 
 /* Geometry of the dataflow decode kernel that ft_moe_stack_forward runs for
- * one or two tokens (host only, no device needed): out[0] = 1 if it takes
+ * one or two tokens, and in waves of two for three or four (host only, no
+ * device needed; T is the tokens of one launch): out[0] = 1 if it takes
  * this shape, batch T, stack depth and weight format (else the
  * counter-synchronised or the per-layer kernels run), out[1] = rows of a down tile over all units,
  * out[2] = shared memory of a CTA in bytes.  FT_ERR_INVALID on a bad shape. */

@@ -116,3 +116,18 @@ def test_clock_sampler_without_nvml_says_so():
     with s:
         pass
     assert s.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+
+
+def test_stack_launch_counts_follow_the_runtime_paths(monkeypatch):
+    """Launches of one stacked pass, as bench.py counts them for its
+    gpu_launches claim: the routing kernel and one dataflow launch for up to
+    two tokens, both per wave of two for three or four, the routing kernel
+    and the counter kernel with FT_STACK_COUNTERS, and the routing kernel plus
+    two kernels per layer layerwise (the 35B-class 40-layer stack)."""
+    import bench
+    monkeypatch.setattr(bench, "L", 40)
+    assert [bench.stack_launches(T) for T in (1, 2, 3, 4)] == [2, 2, 4, 4]
+    assert bench.stack_launches(4, counters=True) == 2
+    assert bench.stack_launches(1, layerwise=True) == 81
+    assert "waves of two" in bench.decode_kernel_name(4) and "waves" not in bench.decode_kernel_name(2)
+    assert "counter" in bench.decode_kernel_name(8)

@@ -20,7 +20,7 @@ def fake_decode(args, world, rank):
                 launches=2 * args.steps, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 40},
                 kernels={"dec_stack": {"ms_total": us * args.steps / 1e3, "launches": args.steps, "us_avg": us},
                          "route": {"ms_total": 0.0109 * args.steps, "launches": args.steps, "us_avg": 10.9}},
-                gate_up_bytes=0.0, down_bytes=0.0, stack_bytes=STACK_BYTES,
+                kernel_steps=args.steps, gate_up_bytes=0.0, down_bytes=0.0, stack_bytes=STACK_BYTES,
                 e2e={"value": 2927.0, "unit": "tok/s", "h2d_bytes_per_step": 45056, "d2h_bytes_per_step": 4096})
 
 
