@@ -38,13 +38,14 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 or 4)")
+    ap.add_argument("--tokens", type=int, default=1, help="decode batch (1 to 16; the extras use 1 and 4)")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--case", default="decode",
-                    choices=["decode", "prefill", "miss", "glm", "gemm", "router", "nvfp4"],
+                    choices=["decode", "prefill", "miss", "glm", "gemm", "router", "nvfp4", "dsv4"],
                     help="decode: the 35B-class decode stack (default line); prefill / miss / glm: only that "
-                         "measurement; nvfp4: the NVFP4 prefill layer alone; gemm / router: the prefill GEMMs or "
-                         "router GEMV alone on a small case (the ncu captures' workloads)")
+                         "measurement; nvfp4: the NVFP4 prefill layer alone; dsv4: the DSV4-class decode stack "
+                         "alone; gemm / router: the prefill GEMMs or router GEMV alone on a small case (the ncu "
+                         "captures' workloads)")
     ap.add_argument("--layers", type=int, default=40, help="layers of the decode stack (40 = the full stack)")
     ap.add_argument("--layerwise", action="store_true",
                     help="decode with two kernels per layer instead of a persistent stack kernel")
@@ -962,6 +963,76 @@ def measure_glm(tokens=256, layers=8, prefill_tokens=2048, reps=3):
     return {"decode": dec, "prefill": pre}
 
 
+def measure_decode_dsv4(pk, n_layers=8, n_pos=64, reps=200):
+    """The decode stack at another shape, through the dataflow kernel's build
+    for any shape: DSV4-class layers (hidden 4096, 256 experts top-6,
+    intermediate 2048, no shared expert), `n_layers` of them resident in HBM
+    (27 GB at 8), batch 1, Zipf(1.1) / 0.6-reuse traces of `n_pos` positions.
+    Time per token from events around `reps` stacked passes (not replayed as
+    a graph); the persistent kernel's time from the kernel timers of a second
+    run; HBM fraction of the distinct experts' blob bytes per token."""
+    import numpy as np
+    import torch
+    import expert_offloaded_serving_b200 as ft
+    import synth
+    import synth.gpu
+    H2, I2, E2, k2, seed = 4096, 2048, 256, 6, 1007
+    pools = [synth.gpu.layer_pool(H2, I2, E2, seed, layer) for layer in range(n_layers)]
+    ctx = ft.ft_create(ft.make_desc(H2, I2, E2, k2, n_layers, 0, 0, 1), None, pools)
+    try:
+        sets = np.stack([synth.zipf_trace(seed, layer, n_pos, E2, k2, 1.1, 0.6) for layer in range(n_layers)],
+                        axis=1)                                                   # [P][L][k]
+        lg = np.stack([np.stack([synth.logits_for_sets(seed, p * 1000 + layer, sets[p, layer][None], E2)
+                                 for layer in range(n_layers)]) for p in range(n_pos)])   # [P][L][1][E]
+        lgd = torch.from_numpy(lg).cuda()
+        x = torch.from_numpy(synth.activations_bf16(seed, 1, 1, H2).view(np.int16).copy()).cuda().view(torch.bfloat16)
+        out = torch.empty_like(x)
+        used = ft.ft_blob_layout(H2, I2)["used"]
+        step_bytes = np.array([sum(len(np.unique(sets[p, layer])) for layer in range(n_layers)) * used
+                               for p in range(n_pos)], np.float64)
+        flags = ft.FT_ROUTE_RENORM
+
+        def run(n):
+            for s in range(n):
+                ft.ft_moe_stack_forward(ctx, 0, n_layers, x, 1, lgd[s % n_pos], out, flags)
+        run(3)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            a.record()
+            run(reps)
+            b.record()
+            b.synchronize()
+        ms = a.elapsed_time(b) / reps
+        ft.ft_kernel_timing_enable(ctx, True)
+        run(reps)
+        kt = ft.ft_kernel_timing_read(ctx)
+        ft.ft_kernel_timing_enable(ctx, False)
+        ft.ft_sync_status(ctx)
+    finally:
+        ft.ft_destroy(ctx)
+    del pools
+    torch.cuda.empty_cache()
+    kernel_us = 1e3 * kt["dec_stack"][0] / reps
+    mean_bytes = float(step_bytes[np.arange(reps) % n_pos].mean())
+    gbs = mean_bytes / (kernel_us * 1e-6) / 1e9
+    return {"workload": f"DSV4-class decode stack: hidden {H2}, {E2} experts top-{k2}, intermediate {I2}, "
+                        f"{n_layers} layers resident in HBM, batch 1, Zipf(1.1) routing traces with 0.6 "
+                        f"adjacent-token reuse",
+            "decode_kernels": decode_kernel_name_shape(H2, I2, E2, k2, 0, n_layers, 1),
+            "ms_per_token_over_these_layers": ms, "us_per_layer": 1e3 * ms / n_layers,
+            "kernel_us": kernel_us, "algorithmic_bytes_per_token": mean_bytes, "kernel_gbs": gbs,
+            "kernel_frac": gbs / pk["hbm"], "clocks": clk.summary()}
+
+
+def decode_kernel_name_shape(H2, I2, E2, k2, S2, L2, T):
+    """The stacked-decode kernel for another shape (MXFP4, no flags)."""
+    import expert_offloaded_serving_b200 as ft
+    if ft.ft_flow_geometry(H2, I2, min(T, 2), k2, S2, E2, L2, ft.FT_FMT_MXFP4)["ok"] and T <= 4:
+        return "persistent stack kernel, dataflow (tagged hand-overs), the build for any shape"
+    return "persistent stack kernel, counter-synchronised"
+
+
 def measure_decode_batch(args, T, pk):
     """The same 35B-class decode stack at batch T (the workload's other batch
     size): tokens/s, ms per step, end-to-end tokens/s and the persistent
@@ -1048,7 +1119,8 @@ def main():
             r = {"prefill": lambda: measure_prefill(reps=max(args.steps, 1)), "miss": measure_misses,
                  "glm": measure_glm, "gemm": lambda: measure_gemm_small(reps=max(args.steps, 1), fmt=args.format),
                  "router": lambda: measure_router(reps=max(args.steps, 1)),
-                 "nvfp4": lambda: measure_prefill_nvfp4(measure_fp4_peak()["tflops"], peaks())}[args.case]()
+                 "nvfp4": lambda: measure_prefill_nvfp4(measure_fp4_peak()["tflops"], peaks()),
+                 "dsv4": lambda: measure_decode_dsv4(peaks())}[args.case]()
             print(json.dumps({"case": args.case, **r}))
         return
     if args.impl == "reference":
@@ -1117,6 +1189,10 @@ def main():
                     line["decode_formats"] = measure_decode_formats(args, pk)
                 except Exception as ex:
                     line["decode_formats"] = {"error": repr(ex)}
+                try:
+                    line["decode_dsv4"] = measure_decode_dsv4(pk)
+                except Exception as ex:
+                    line["decode_dsv4"] = {"error": repr(ex)}
         try:
             line["glm"] = measure_glm()
         except Exception as ex:

@@ -31,6 +31,7 @@ def line(monkeypatch, capsys):
     monkeypatch.setattr(bench, "measure_prefill", lambda: {"workload": "prefill"})
     monkeypatch.setattr(bench, "measure_misses", lambda: {"workload": "miss"})
     monkeypatch.setattr(bench, "measure_glm", lambda: {"decode": {}, "prefill": {}})
+    monkeypatch.setattr(bench, "measure_decode_dsv4", lambda pk: {"workload": "dsv4"})
     monkeypatch.setattr(bench, "oracle_tok_s", lambda T, threads: (0.22 if threads > 1 else 0.05, 12))
     monkeypatch.setattr(bench, "host_cores", lambda: 16)
     monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "10", "--warmup", "3"])

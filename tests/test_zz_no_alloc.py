@@ -13,6 +13,7 @@ import torch
 import expert_offloaded_serving_b200 as ft
 import synth
 import synth.gpu
+from oracle import layer as olayer
 
 from _gpu import Ctx, assert_close, bf16_bits, bits_to_f64, x_dev
 
@@ -29,8 +30,13 @@ def inputs(tag, T):
 
 
 def test_noalloc_matches_context_forward_on_two_calls_in_a_row():
+    """Against the context forward and against the oracle on the same
+    inputs (decode mode), for two calls that reuse the static scratch."""
     pool = synth.gpu.layer_pool(H, I, E + S, SEED, 0)
-    wr = torch.from_numpy(synth.router_weights(SEED, 0, E, H)).cuda()
+    wr_host = synth.router_weights(SEED, 0, E, H)
+    wr = torch.from_numpy(wr_host).cuda()
+    stride = synth.blob_stride(H, I)
+    host = pool.cpu().numpy()
     with Ctx(ft.make_desc(H, I, E, K, 1, S, 0, 16), None, [pool]) as c:
         cases = [(1, 4, False), (2, 3, True)]   # (tag, T, use the router GEMV)
         for tag, T, use_router in cases:
@@ -45,6 +51,11 @@ def test_noalloc_matches_context_forward_on_two_calls_in_a_row():
             torch.cuda.synchronize()
             assert int(status.item()) == 0
             assert_close(bf16_bits(got), bits_to_f64(bf16_bits(want)))
+            r = olayer.moe_layer(bf16_bits(x), lambda e: host[e * stride:(e + 1) * stride], H, I, E, K,
+                                 logits=None if use_router else lg.cpu().numpy(),
+                                 router_w=wr_host if use_router else None,
+                                 shared_blob=host[E * stride:(E + 1) * stride])
+            assert_close(bf16_bits(got), r["out_f64"])
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
