@@ -245,6 +245,32 @@ def expert_blob_wide(seed: int, layer: int, expert: int, hidden: int, inter: int
     return blob
 
 
+def expert_blob_nvfp4_wide(seed: int, layer: int, expert: int, hidden: int, inter: int,
+                           wide=("wg", "wu", "wd"), tensor_scales=(2.0 ** -8, 2.0 ** -8, 2.0 ** -8)) -> np.ndarray:
+    """An NVFP4 blob whose matrices named in ``wide`` get codes uniform over
+    all 16 and E4M3 block-scale bytes uniform over 0x00 .. 0x7e (zero, the
+    seven subnormals and every normal value up to 448); the other matrices
+    keep the usual bytes.  The matrix scales are ``tensor_scales`` (Wg, Wu,
+    Wd).  Byte draws from the wide stream (REGION_WIDE)."""
+    r = nvfp4_blob_regions(hidden, inter)
+    blob = expert_blob_nvfp4(seed, layer, expert, hidden, inter)
+    code_rng = {"wg": (r["wg"], r["wu"]), "wu": (r["wu"], r["wd"]), "wd": (r["wd"], r["codes_end"])}
+    sc_rng = {"wg": (r["wg_sf"], r["wu_sf"]), "wu": (r["wu_sf"], r["wd_sf"]), "wd": (r["wd_sf"], r["tensor_scales"])}
+    n_draw = 0
+    for name in wide:
+        for a, b in (code_rng[name], sc_rng[name]):
+            n = b - a
+            w = words(seed, blob_stream(layer, expert, REGION_WIDE), n_draw, (n + 3) // 4)
+            n_draw += (n + 3) // 4
+            f = np.stack([(w >> np.uint64(16 * q)) & np.uint64(0xFFFF) for q in range(4)], axis=1).reshape(-1)[:n]
+            if (a, b) == code_rng[name]:
+                blob[a:b] = (f & np.uint64(0xFF)).astype(np.uint8)     # two uniform 4-bit codes
+            else:
+                blob[a:b] = (f % np.uint64(0x7F)).astype(np.uint8)     # E4M3 bytes 0x00 .. 0x7e
+    blob[r["tensor_scales"]: r["tensor_scales"] + 12] = np.asarray(tensor_scales, dtype="<f4").view(np.uint8)
+    return blob
+
+
 # ---------------------------------------------------------------------------
 # activations, router weights, traces, logits
 # ---------------------------------------------------------------------------
