@@ -61,3 +61,20 @@ def test_nvfp4_blob_regions_and_bytes():
     ts = a[r["tensor_scales"]:r["tensor_scales"] + 12].view("<f4")
     assert list(ts) == list(np.float32(synth.NVFP4_TENSOR_SCALES))
     assert (a[r["tensor_scales"] + 12:] == 0).all()
+
+
+def test_wide_nvfp4_blob_covers_every_e4m3_byte():
+    """The wide NVFP4 blob: each wide matrix's scale bytes take every value
+    0x00 .. 0x7e and nothing above (no NaN byte 0x7f); all 16 codes occur;
+    the matrix scales are the ones asked for; the draws are deterministic."""
+    import numpy as np
+    import synth
+    H, I = 256, 128
+    b = synth.expert_blob_nvfp4_wide(9, 1, 2, H, I, tensor_scales=(0.5, 0.25, 0.125))
+    r = synth.nvfp4_blob_regions(H, I)
+    for a, z in ((r["wg_sf"], r["wu_sf"]), (r["wu_sf"], r["wd_sf"]), (r["wd_sf"], r["tensor_scales"])):
+        assert set(np.unique(b[a:z])) == set(range(0x7F))
+    codes = b[:r["codes_end"]]
+    assert set(np.unique(np.concatenate([codes & 15, codes >> 4]))) == set(range(16))
+    assert list(b[r["tensor_scales"]:r["tensor_scales"] + 12].view("<f4")) == [0.5, 0.25, 0.125]
+    assert (b == synth.expert_blob_nvfp4_wide(9, 1, 2, H, I, tensor_scales=(0.5, 0.25, 0.125))).all()
