@@ -245,6 +245,22 @@ def expert_blob_wide(seed: int, layer: int, expert: int, hidden: int, inter: int
     return blob
 
 
+def expert_blob_bf16_wide(seed: int, layer: int, expert: int, hidden: int, inter: int) -> np.ndarray:
+    """A BF16 blob of uniform 16-bit patterns over every finite bf16 value
+    (both signs, zeros, subnormals, every exponent up to 254; exponent 255,
+    infinity and NaN, is moved to 254).  Byte draws from the wide stream."""
+    r = bf16_blob_regions(hidden, inter)
+    n = r["used"] // 2
+    w = words(seed, blob_stream(layer, expert, REGION_WIDE), 0, (n + 3) // 4)
+    f = np.stack([(w >> np.uint64(16 * q)) & np.uint64(0xFFFF) for q in range(4)], axis=1).reshape(-1)[:n]
+    f = f.astype(np.uint16)
+    inf_nan = (f & 0x7F80) == 0x7F80
+    f[inf_nan] = f[inf_nan] & np.uint16(0xFF7F)          # exponent 255 -> 254
+    blob = np.zeros(r["stride"], dtype=np.uint8)
+    blob[: r["used"]] = f.astype("<u2").view(np.uint8)
+    return blob
+
+
 def expert_blob_nvfp4_wide(seed: int, layer: int, expert: int, hidden: int, inter: int,
                            wide=("wg", "wu", "wd"), tensor_scales=(2.0 ** -8, 2.0 ** -8, 2.0 ** -8)) -> np.ndarray:
     """An NVFP4 blob whose matrices named in ``wide`` get codes uniform over

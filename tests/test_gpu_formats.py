@@ -145,3 +145,18 @@ def test_prefill_refuses_other_formats(fmt):
             ft.ft_moe_layer_forward(c.h, 0, x, 64, None, torch.zeros((64, E), device="cuda"), torch.empty_like(x),
                                     ft.FT_ACT_MXFP4 | ft.FT_ROUTE_RENORM)
         assert e.value.status == ft.FT_ERR_INVALID and "MXFP4 weights only" in str(e.value)
+
+
+def test_wide_bf16_dequant_bit_exact():
+    """Every finite bf16 bit pattern class (zeros, subnormals, each exponent up
+    to 254, both signs) through the decode tile's BF16 staging and its exact
+    widening to fp32, against the oracle, bit for bit."""
+    H, I = 2048, 512
+    blob = synth.expert_blob_bf16_wide(6301, 0, 1, H, I)
+    d = torch.from_numpy(blob).cuda()
+    with Ctx(ft.make_desc(H, I, 16, 2, weight_format=ft.FT_FMT_BF16)) as c:
+        for mat, name, shape in ((0, "wg", (I, H)), (1, "wu", (I, H)), (2, "wd", (H, I))):
+            out = torch.empty(shape, dtype=torch.float32, device="cuda")
+            ft.ft_debug_dequant(c.h, d, mat, out)
+            want = formats.weight_matrix(blob, name, H, I, "bf16").astype(np.float32)
+            assert (out.cpu().numpy().view(np.uint32) == want.view(np.uint32)).all(), name

@@ -78,3 +78,17 @@ def test_wide_nvfp4_blob_covers_every_e4m3_byte():
     assert set(np.unique(np.concatenate([codes & 15, codes >> 4]))) == set(range(16))
     assert list(b[r["tensor_scales"]:r["tensor_scales"] + 12].view("<f4")) == [0.5, 0.25, 0.125]
     assert (b == synth.expert_blob_nvfp4_wide(9, 1, 2, H, I, tensor_scales=(0.5, 0.25, 0.125))).all()
+
+
+def test_wide_bf16_blob_covers_every_finite_exponent():
+    """The wide BF16 blob: every biased exponent 0 .. 254 (zeros and
+    subnormals included) in both signs, no infinity or NaN; deterministic."""
+    import numpy as np
+    import synth
+    H, I = 256, 128
+    b = synth.expert_blob_bf16_wide(9, 1, 2, H, I)
+    v = b[:6 * H * I].view("<u2")
+    e = (v >> 7) & 0xFF
+    assert set(np.unique(e)) == set(range(255))
+    assert 0.45 < ((v >> 15) & 1).mean() < 0.55
+    assert (b == synth.expert_blob_bf16_wide(9, 1, 2, H, I)).all()
