@@ -82,6 +82,11 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
 
 // Byte offset of the 4-byte scale word holding blocks 4a..4a+3 of `row` in a
 // scale region with `atoms_k` atoms along K (atom = 128 rows x 4 blocks).
+// Device buffers the kernels read or write with vector accesses start on a
+// 16-byte boundary (every cudaMalloc'd or torch-allocated buffer does); the
+// entry points refuse others before any launch.
+__host__ __device__ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
 __host__ __device__ __forceinline__ int64_t sf_word(int row, int a, int atoms_k) {
   return ((int64_t)(row >> 7) * atoms_k + a) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
 }

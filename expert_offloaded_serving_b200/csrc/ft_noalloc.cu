@@ -85,6 +85,9 @@ extern "C" ft_status ft_moe_layer_forward_noalloc(int32_t hidden, int32_t inter,
   if (flags & FT_ACT_MXFP4) return bad("only the decode (bf16-activation) path has a no-alloc form");
   if (!logits_override && !router_w) return bad("need router_w or logits_override");
   if (x == out) return bad("out must not alias x");
+  if (!ft::aligned16(layer_pool) || !ft::aligned16(x) || !ft::aligned16(out) || !ft::aligned16(router_w) ||
+      !ft::aligned16(logits_override))
+    return bad("layer_pool, x, out, router_w and logits must start on a 16-byte boundary");
   if (T == 0) return FT_OK;
   const int Ti = (int)T;
 

@@ -141,20 +141,35 @@ __global__ void __launch_bounds__(256) k_quant_h_nv(const float* __restrict__ hf
 }
 
 // out[t][n] = bf16( sum_j w[t][j] * y[inv[t*k+j]][n]  +  sum_s y[T*k + s*T + t][n] )
+// A thread takes four consecutive n (16-byte loads of y, one 8-byte store);
+// each element's sum is taken in the order above.
 __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y, const float* __restrict__ w,
                                                  const int32_t* __restrict__ inv, int T, int H, int k, int n_shared,
                                                  uint16_t* __restrict__ out) {
+  const int H4 = H / 4;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (int64_t)T * H) return;
-  const int t = (int)(i / H), n = (int)(i % H);
-  float acc = 0.f;
+  if (i >= (int64_t)T * H4) return;
+  const int t = (int)(i / H4), n = 4 * (int)(i % H4);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j = 0; j < k; j++) {
     const int f = t * k + j;
-    acc = fmaf(w[f], y[(size_t)inv[f] * H + n], acc);
+    const float wf = w[f];
+    const float4 v = *reinterpret_cast<const float4*>(y + (size_t)inv[f] * H + n);
+    acc.x = fmaf(wf, v.x, acc.x);
+    acc.y = fmaf(wf, v.y, acc.y);
+    acc.z = fmaf(wf, v.z, acc.z);
+    acc.w = fmaf(wf, v.w, acc.w);
   }
-  for (int s = 0; s < n_shared; s++) acc += y[(size_t)(T * k + s * T + t) * H + n];
-  __nv_bfloat16 b = __float2bfloat16_rn(acc);
-  out[i] = *reinterpret_cast<uint16_t*>(&b);
+  for (int s = 0; s < n_shared; s++) {
+    const float4 v = *reinterpret_cast<const float4*>(y + (size_t)(T * k + s * T + t) * H + n);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+  *reinterpret_cast<uint2*>(out + (size_t)t * H + n) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
 }
 
 }  // namespace
@@ -282,7 +297,7 @@ cudaError_t launch_prefill_gemm(const PrefillScratch& s, const PrefillArgs& a, i
 }
 
 cudaError_t launch_prefill_combine(const PrefillScratch& s, const PrefillArgs& a, cudaStream_t st) {
-  const int64_t n = (int64_t)a.T * a.H;
+  const int64_t n = (int64_t)a.T * (a.H / 4);  // H % 128 == 0: whole groups of four
   k_combine<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(s.y, a.w, a.inv, a.T, a.H, a.k, a.n_shared, a.out);
   return cudaGetLastError();
 }

@@ -372,6 +372,10 @@ extern "C" ft_status ft_create(const ft_model_desc* desc, const void* const* hos
   FT_TRY(check_desc(desc));
   if (!out) return fail(FT_ERR_INVALID, "out is NULL");
   *out = nullptr;
+  if (resident_layers)
+    for (int l = 0; l < desc->n_layers; l++)
+      if (!aligned16(resident_layers[l]))
+        return fail(FT_ERR_INVALID, "resident pool of layer %d must start on a 16-byte boundary", l);
   ft_ctx* c = new ft_ctx();
   c->d = *desc;
   const int H = desc->hidden, I = desc->inter, E = desc->n_experts, k = desc->top_k, L = desc->n_layers;
@@ -625,6 +629,8 @@ extern "C" ft_status ft_router_logits(ft_ctx* c, const void* x, int64_t T, int32
                                       float* logits, void* stream) {
   if (!c || (!x && T > 0) || !wr || !logits) return fail(FT_ERR_INVALID, "NULL argument");
   if (T < 0 || H <= 0 || H % 128 || E <= 0) return fail(FT_ERR_INVALID, "bad shape T=%lld H=%d E=%d", (long long)T, H, E);
+  if (!aligned16(x) || !aligned16(wr) || !aligned16(logits))
+    return fail(FT_ERR_INVALID, "x, wr and logits must start on a 16-byte boundary");
   CUDA_TRY(launch_router_logits((const uint16_t*)x, wr, (int)T, H, E, logits, (cudaStream_t)stream));
   return FT_OK;
 }
@@ -654,6 +660,7 @@ extern "C" ft_status ft_quantize_mxfp4(ft_ctx* c, const float* x, int64_t R, int
                                        uint8_t* scales, void* stream) {
   if (!c || (!x && R > 0) || !codes || !scales) return fail(FT_ERR_INVALID, "NULL argument");
   if (R < 0 || K <= 0 || K % 128) return fail(FT_ERR_INVALID, "K=%d not a positive multiple of 128", K);
+  if (!aligned16(x) || !aligned16(codes)) return fail(FT_ERR_INVALID, "x and codes must start on a 16-byte boundary");
   CUDA_TRY(launch_quantize_rows(x, R, K, codes, scales, (cudaStream_t)stream));
   return FT_OK;
 }
@@ -662,6 +669,7 @@ extern "C" ft_status ft_quantize_nvfp4(ft_ctx* c, const float* x, int64_t R, int
                                        uint8_t* scales, float* tensor_scale, void* stream) {
   if (!c || (!x && R > 0) || !codes || !scales || !tensor_scale) return fail(FT_ERR_INVALID, "NULL argument");
   if (R < 0 || K <= 0 || K % 128) return fail(FT_ERR_INVALID, "K=%d not a positive multiple of 128", K);
+  if (!aligned16(x) || !aligned16(codes)) return fail(FT_ERR_INVALID, "x and codes must start on a 16-byte boundary");
   CUDA_TRY(launch_quantize_rows_nv(x, R, K, c->d_qamax, codes, scales, tensor_scale, (cudaStream_t)stream));
   c->last_stream = (cudaStream_t)stream;
   return FT_OK;
@@ -1263,6 +1271,8 @@ extern "C" ft_status ft_moe_layer_forward(ft_ctx* c, int32_t layer, const void* 
   if (T < 0 || T > c->max_tokens) return fail(FT_ERR_INVALID, "T=%lld outside [0, max_tokens=%d]", (long long)T, c->max_tokens);
   if (!logits_override && !router_w) return fail(FT_ERR_INVALID, "need router_w or logits_override");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
+  if (!aligned16(x) || !aligned16(out) || !aligned16(router_w) || !aligned16(logits_override))
+    return fail(FT_ERR_INVALID, "x, out, router_w and logits must start on a 16-byte boundary");
   // prefill path: FT_ACT_MXFP4 (MXFP4 weights) or FT_ACT_NVFP4 (NVFP4 weights)
   const bool nv = (flags & FT_ACT_NVFP4) != 0;
   const bool pf = nv || (flags & FT_ACT_MXFP4) != 0;
@@ -1552,6 +1562,8 @@ extern "C" ft_status ft_moe_stack_forward(ft_ctx* c, int32_t first_layer, int32_
   if (flags & (FT_ACT_MXFP4 | FT_ACT_NVFP4))
     return fail(FT_ERR_INVALID, "the stacked forward is the decode path (FT_ACT_BF16)");
   if (x == out) return fail(FT_ERR_INVALID, "out must not alias x");
+  if (!aligned16(x) || !aligned16(out) || !aligned16(logits))
+    return fail(FT_ERR_INVALID, "x, out and logits must start on a 16-byte boundary");
   for (int l = first_layer; l < first_layer + n_layers; l++)
     if (!c->resident[l]) return fail(FT_ERR_STATE, "layer %d is not resident", l);
   if (T == 0) return FT_OK;

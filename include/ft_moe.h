@@ -154,6 +154,11 @@ FT_API const char* ft_last_error(void);
 /* context                                                                 */
 /* ---------------------------------------------------------------------- */
 
+/* Alignment: every device buffer passed to the calls below (pools, x, out,
+ * router weights, logits, codes) starts on a 16-byte boundary, as every
+ * cudaMalloc'd or torch-allocated buffer does; a call given another refuses it
+ * with FT_ERR_INVALID before any launch. */
+
 /* Create a context on the current CUDA device.
  *   host_layers     host [L] pointers (or NULL): layer l's pool of
  *                   (E + n_shared) blobs at ft_blob_stride() each, in host

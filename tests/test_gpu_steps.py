@@ -153,3 +153,28 @@ def test_gpu_quantiser_bit_exact(ctx, R, K):
     r = np.arange(R)[:, None]
     b = np.arange(K // 32)[None, :]
     assert (sc[fp4.scale_index(r, b, K // 32)] == want_sc).all()
+
+
+def test_misaligned_buffers_are_refused():
+    """A buffer that does not start on a 16-byte boundary (here a view two
+    bytes into an allocation) is refused on the host with FT_ERR_INVALID
+    before any launch: the forward, the stacked forward, the router logits,
+    and a resident pool at context creation."""
+    H, I, E, k, T = 256, 128, 16, 2, 4
+    big = torch.zeros(T * H + 16, dtype=torch.bfloat16, device="cuda")
+    xm = big[1:1 + T * H].view(T, H)                          # 2 bytes past the allocation's start
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    lg = torch.zeros((T, E), dtype=torch.float32, device="cuda")
+    pool = synth.gpu.layer_pool(H, I, E, 77, 0)
+    with Ctx(ft.make_desc(H, I, E, k, 1, 0, 0, 16), None, [pool]) as c:
+        calls = [lambda: ft.ft_moe_layer_forward(c.h, 0, xm, T, None, lg, out, ft.FT_ROUTE_RENORM),
+                 lambda: ft.ft_moe_stack_forward(c.h, 0, 1, xm, T, lg, out, ft.FT_ROUTE_RENORM),
+                 lambda: ft.ft_router_logits(c.h, xm, T, H, torch.zeros((E, H), device="cuda"), E, lg)]
+        for call in calls:
+            with pytest.raises(ft.FtError) as e:
+                call()
+            assert e.value.status == ft.FT_ERR_INVALID and "16-byte" in str(e.value)
+        ft.ft_sync_status(c.h)
+    with pytest.raises(ft.FtError) as e:
+        ft.ft_create(ft.make_desc(H, I, E, k, 1, 0, 0, 16), None, [pool[8:]])
+    assert e.value.status == ft.FT_ERR_INVALID and "16-byte" in str(e.value)

@@ -152,3 +152,13 @@ def test_binding_holds_borrowed_pools_until_destroy(monkeypatch):
     ft.ft_destroy(h)
     gc.collect()
     assert wh() is None and wr() is None
+
+
+@pytest.mark.parametrize("kw", [dict(layer_pool=POOL + 8), dict(x=X + 2), dict(out=OUT + 4), dict(logits_override=LG + 8),
+                                dict(router_w=WR + 4, logits_override=None)])
+def test_noalloc_refuses_misaligned_buffers(kw):
+    """Buffers the kernels access with vector loads and stores must start on a
+    16-byte boundary; others are refused before any launch."""
+    with pytest.raises(ft.FtError) as e:
+        noalloc(**kw)
+    assert e.value.status == ft.FT_ERR_INVALID and "16-byte" in str(e.value)
