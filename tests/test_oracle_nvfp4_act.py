@@ -165,3 +165,33 @@ def test_nvfp4_h_scale_spans_every_expert():
     big = layer._nvfp4_expert_outputs(x, [(a, rows), (_with_gate_scale(other, H, I, 64.0), rows)], H, I)[0]
     assert np.array_equal(alone, small)
     assert not np.array_equal(alone, big)
+
+
+def test_quantiser_invariants_on_generated_tensors():
+    """Invariants that hold for any finite fp32 tensor, on tensors generated
+    to mix magnitudes (subnormal fp32 to 2^99, zeros, signed zeros): every
+    scale byte is a finite non-negative E4M3 value; a block whose largest
+    magnitude is the tensor's takes 448 (0x7e) up to one E4M3 step; codes of
+    a block with a zero scale are +0; no value dequantises to more than 6
+    block units; signs are kept (a dequantised value is never of the other
+    sign)."""
+    from hypothesis import given, settings, strategies as st
+
+    vals = st.one_of(st.floats(width=32, allow_nan=False, allow_infinity=False, min_value=-2.0 ** 99, max_value=2.0 ** 99),
+                     st.sampled_from([0.0, -0.0, 1e-40, -1e-40, 2688.0, 6.0, 0.25]))
+
+    @settings(max_examples=200, deadline=None, derandomize=True)
+    @given(st.lists(vals, min_size=32, max_size=32))
+    def check(row):
+        x = np.asarray(row, np.float32).reshape(1, 32)
+        c, b, s = formats.nvfp4_quantize_rows(x)
+        assert (b <= 0x7E).all()
+        d = formats.nvfp4_dequant_rows(c, b, s)
+        sv = np.repeat(formats.E4M3_TABLE[b] * float(s), 16, axis=1)
+        assert (np.abs(d) <= 6 * sv + 0).all()
+        assert not ((d > 0) & (x < 0)).any() and not ((d < 0) & (x > 0)).any()
+        assert (c[np.repeat(b == 0, 16, axis=1)] == 0).all()
+        if s > 0:
+            top = int(np.argmax(np.abs(x))) // 16
+            assert formats.E4M3_TABLE[b[0, top]] >= 416.0   # 448 or the E4M3 value below it
+    check()
