@@ -362,3 +362,22 @@ def test_nvfp4_quantiser_equals_the_numpy_oracle_on_generated_tensors():
         b = formats.nvfp4_quantize_rows(x)
         assert (a[0] == b[0]).all() and (a[1] == b[1]).all() and a[2] == b[2]
     check()
+
+
+def test_mxfp4_quantiser_equals_the_numpy_oracle_on_generated_rows():
+    """The C++ and numpy MXFP4 quantisers agree (codes and UE8M0 bytes) on
+    generated rows mixing every fp64 magnitude from subnormal to 1e300, zeros,
+    signed zeros and the e2m1 grid's midpoints."""
+    from hypothesis import given, settings, strategies as st
+
+    vals = st.one_of(st.floats(allow_nan=False, allow_infinity=False, min_value=-1e300, max_value=1e300),
+                     st.sampled_from([0.0, -0.0, 5e-324, 0.25, 0.75, 2.5, 5.0, 6.0, -3.5]))
+
+    @settings(max_examples=200, deadline=None, derandomize=True)
+    @given(st.lists(vals, min_size=64, max_size=64))
+    def check(row):
+        x = np.asarray(row, np.float64).reshape(2, 32)
+        a = cpp.quantize_rows(x)
+        b = fp4.quantize_rows(x)
+        assert (a[0] == b[0]).all() and (a[1] == b[1]).all()
+    check()
